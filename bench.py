@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Benchmark of the CPR Gated DeltaNet layer (one JSON line on rank 0).
+
+Metric: CPR-GDN tokens/s per layer on the rollout-prefill shape (5 x 2048
+tokens packed, H=16, d_k=d_v=128, chunk 64, bf16 q/k/v, fp32 beta/g/state),
+with the decode shape (256 sequences x 1 token, prefixes uniform in
+[1, 2047], 512 consecutive steps) reported in the same line under "decode".
+One step = one gdn_cpr_forward over the whole batch (chunk table, boundary
+prep, boundary walk, intra-chunk fill).  Inputs are resident in HBM; L2 is
+flushed (a 256 MiB write) before every timed step, outside the step's
+events.  Per-kernel times come from CUDA events the library records on the
+launching stream between its kernels.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own batch
+(weak scaling, no collective on the data path); the reported time is the
+max over ranks.  --impl reference times the fp64 CPU oracle on the host.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CPR-GDN tokens/s per layer (prefill 5x2048, decode 256x1); % HBM roofline"
+H, D, C = 16, 128, 64
+PREFILL_LENS = [2048] * 5
+FLUSH_BYTES = 256 << 20
+PAGES_H100 = {"prefill_ms": 1.412, "decode_ms": 0.0846, "trainer_fwd_bwd_ms": 7.386}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", 0.0)),
+                "sm_max_mhz": float(p.get("sm_max_mhz", 1965.0)), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------
+# Algorithmic work (stated per unit)
+# ----------------------------------------------------------------------------
+
+def fill_flops(T, H_, d):
+    """Intra-chunk fill: per token and head 7 d^2 FP32 flops (p: d^2 FMA; update:
+    d^2 MUL + d^2 FMA; o: d^2 FMA; an FMA counts 2)."""
+    return 7.0 * d * d * T * H_
+
+
+def walk_flops(n_full_chunk_heads, d, c=C):
+    """Boundary walk per full chunk and head: U = U~ - W S^T (c x d x d MACs) and
+    S' = g S + Ud^T K (d x c x d MACs): 4 c d^2 flops."""
+    return 4.0 * c * d * d * n_full_chunk_heads
+
+
+def prep_flops(n_full_chunk_heads, d, c=C):
+    """Boundary prep per full chunk and head: K K^T, W, U~ (3 c^2 d MACs)."""
+    return 6.0 * c * c * d * n_full_chunk_heads
+
+
+def prefill_bytes(lens, H_, d, in_bytes=2, out_bytes=2):
+    """Minimal HBM bytes of a forward: read q,k,v,beta,g, write o and the two final
+    states.  Two-pass bytes add the boundary states written by pass 1 and read by
+    pass 2 and pass 1's re-read of k,v,beta,g."""
+    T = sum(lens)
+    n = len(lens)
+    io = T * H_ * (3 * d * in_bytes + 8 + d * out_bytes)
+    finals = 2 * n * H_ * d * d * 4
+    chunks = sum((L + C - 1) // C for L in lens)
+    full = sum(L // C for L in lens)
+    two_pass = io + finals + 2 * chunks * H_ * d * d * 4 + full * C * H_ * (2 * d * in_bytes + 8)
+    return io + finals, two_pass
+
+
+def decode_step_bytes(n_rows, n_resync_units, H_, d, in_bytes=2, out_bytes=2):
+    """Per token and head: read the running state and write it back (2 x 4 d^2),
+    read q,k,v,beta,g, write o, append the token to the chunk buffer, read and
+    write pos.  A unit that resyncs also reads the boundary state (4 d^2) and the
+    C-token buffer; its running-state write is replaced by the boundary write."""
+    per = 2 * 4 * d * d + 3 * d * in_bytes + 8 + d * out_bytes + 2 * d * in_bytes + 8 + 8
+    extra = 4 * d * d + C * (2 * d * in_bytes + 8)
+    return n_rows * H_ * per + n_resync_units * extra
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"gdn_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------
+# Distributed plumbing
+# ----------------------------------------------------------------------------
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# Our arm
+# ----------------------------------------------------------------------------
+
+def bench_prefill(gdn, W, dev, rank, steps, warmup, flush):
+    b = W.prefill(device=dev, seed=rank)
+    T = b.total_tokens
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    srun = torch.empty((len(b.lengths), H, D, D), dtype=torch.float32, device=dev)
+    sbnd = torch.empty_like(srun)
+    ws = torch.zeros(gdn.forward_workspace_bytes(len(b.lengths), T, H, D, D), dtype=torch.uint8,
+                     device=dev)
+
+    def make_events():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        for e in evs:
+            e.record()
+        return evs
+
+    def step(evs):
+        gdn.forward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, o=o, s_run_final=srun,
+                    s_bnd_final=sbnd, workspace=ws, kernel_events=evs)
+
+    warm_evs = make_events()
+    for _ in range(warmup):
+        flush.zero_()
+        step(warm_evs)
+    torch.cuda.synchronize()
+    if gdn.check_error(ws) != 0:
+        raise RuntimeError("device error word set during warm-up")
+    evs = [make_events() for _ in range(steps)]
+    torch.cuda.synchronize()
+    return b, (o, srun, sbnd, ws), step, evs
+
+
+def bench_e2e(gdn, b, dev, steps, warmup):
+    """Host buffers in, host output back: H2D of the step's inputs from pinned
+    memory, the forward, D2H of o, all on one stream inside the events."""
+    host = [t.cpu().pin_memory() for t in (b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens)]
+    devb = [torch.empty_like(t, device=dev) for t in host]
+    T = b.total_tokens
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    o_host = torch.empty((T, H, D), dtype=torch.bfloat16).pin_memory()
+    ws = torch.zeros(gdn.forward_workspace_bytes(len(b.lengths), T, H, D, D), dtype=torch.uint8,
+                     device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = o_host.numel() * o_host.element_size()
+
+    def one():
+        for dst, src in zip(devb, host):
+            dst.copy_(src, non_blocking=True)
+        gdn.forward(*devb, o=o, workspace=ws, want_states=False)
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return ms, h2d, d2h
+
+
+def bench_decode(gdn, W, dev, rank, steps, warmup, slots=256):
+    prefix = W.decode_prefix_lengths(slots)
+    pre = W.make_batch(prefix, H, D, D, seed=100 + rank, device=dev)
+    _, srun, sbnd, ws = gdn.forward(pre.q, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens)
+    st = gdn.DecodeState(slots, H, D, D, device=dev)
+    gdn.decode_state_from_prefill(st, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens, srun, sbnd)
+    del pre, srun, sbnd, ws
+    n_tok = warmup + steps
+    toks = W.decode_tokens(n_tok, slots, H, D, D, seed=200 + rank, device=dev)
+    o = torch.empty((slots, H, D), dtype=torch.bfloat16, device=dev)
+    for s in range(warmup):
+        gdn.decode_step(st, toks[0][s], toks[1][s], toks[2][s], toks[3][s], toks[4][s], o=o)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        s = warmup + i
+        ev[i][0].record()
+        gdn.decode_step(st, toks[0][s], toks[1][s], toks[2][s], toks[3][s], toks[4][s], o=o)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    if gdn.check_error(st.error) != 0:
+        raise RuntimeError("device error word set during decode")
+    times = [a.elapsed_time(b_) for a, b_ in ev]
+    # which units resynced at each timed step: pos before the step == C - 1
+    resync = [sum(1 for P in prefix if (P + warmup + i) % C == C - 1) for i in range(steps)]
+    nbytes = sum(decode_step_bytes(slots, r * H, H, D) for r in resync)
+    return sum(times), nbytes, resync
+
+
+def run_decode_part(gdn, W, dev, rank, world, args, peaks):
+    slots = args.decode_slots
+    dec_ms_total, dec_bytes, resync = bench_decode(gdn, W, dev, rank, args.decode_steps,
+                                                   min(16, args.decode_steps), slots)
+    dec_ms_total = max_over_ranks(dec_ms_total, world)
+    dec_ms = dec_ms_total / args.decode_steps
+    dec_gbs = dec_bytes / (dec_ms_total / 1e3) / 1e9
+    return {"workload": f"{slots} sequences x 1 token per step, prefixes uniform in "
+                        f"[1, 2047], H={H}, d={D}, C={C}, bf16 in/out, fp32 state",
+            "steps": args.decode_steps, "ms_per_step": round(dec_ms, 5),
+            "tokens_per_s": round(world * slots / (dec_ms / 1e3), 1),
+            "resync_units_per_step": round(float(np.mean(resync)) * H, 2),
+            "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(dec_gbs / peaks["hbm_gbs"], 4), "traffic": None},
+            "pages_h100_ms": PAGES_H100["decode_ms"]}
+
+
+def cpu_baseline_sample(W, seconds=10.0):
+    """The fp64 oracle as it stands, all host cores, on whole sequences of the
+    prefill batch until about `seconds` of CPU work has been done."""
+    import oracle
+    b = W.prefill(device="cpu", seed=0)
+    cu = b.cu_seqlens.tolist()
+    done, passes, t0 = 0, 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds and passes < 64:
+        for n in range(len(b.lengths)):
+            sl = slice(cu[n], cu[n + 1])
+            oracle.forward(b.q[sl], b.k[sl], b.v[sl], b.beta[sl], b.g[sl],
+                           np.array([0, cu[n + 1] - cu[n]], np.int32))
+            done += cu[n + 1] - cu[n]
+        passes += 1
+    el = time.perf_counter() - t0
+    return {"value": round(done / el, 1), "unit": "tokens/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"{passes} pass(es) over the whole 5x2048 prefill batch, {H} heads "
+                      f"({done} tokens), fp64 token loop, {el:.1f} s"}
+
+
+def run_ours(args):
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from rl_train_numerics_b200 import _abi as gdn
+    from rl_train_numerics_b200 import workloads as W
+
+    peaks = load_peaks()
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    b, bufs, step, evs = bench_prefill(gdn, W, dev, rank, args.steps, args.warmup, flush)
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    # keep the sampler running on the same work for at least ~1.5 s
+    t_soak = time.perf_counter()
+    while wall + (time.perf_counter() - t_soak) < 1.5:
+        flush.zero_()
+        step(evs[0])
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if gdn.check_error(bufs[3]) != 0:
+        raise RuntimeError("device error word set in the timed region")
+
+    names = ["chunk_table", "boundary_prep", "boundary_walk", "intra_chunk_fill"]
+    per_k = np.zeros(4)
+    total = 0.0
+    for e in evs:
+        for j in range(4):
+            per_k[j] += e[j].elapsed_time(e[j + 1])
+        total += e[0].elapsed_time(e[4])
+    ms_step = max_over_ranks(total / args.steps, world)
+    per_k /= args.steps
+    T = b.total_tokens
+    value = world * T / (ms_step / 1e3)
+
+    lens = b.lengths
+    full = sum(L // C for L in lens) * H
+    work = {
+        "intra_chunk_fill": ("alu", fill_flops(T, H, D)),
+        "boundary_walk": ("alu", walk_flops(full, D)),
+        "boundary_prep": ("alu", prep_flops(full, D)),
+    }
+    dom = max(range(4), key=lambda j: per_k[j])
+    dom_name = names[dom]
+    bound, flops = work.get(dom_name, ("alu", 0.0))
+    fp32_peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12  # TFLOP/s, FMA = 2
+    achieved = flops / (per_k[dom] / 1e3) / 1e12
+    roofline = {"kernel": dom_name, "bound": bound, "achieved": round(achieved, 2),
+                "peak": round(fp32_peak, 2), "unit": "TFLOP/s",
+                "frac": round(achieved / fp32_peak, 4), "traffic": None,
+                "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x sm_max_mhz (nominal)"}
+    minimal, two_pass = prefill_bytes(lens, H, D)
+    hbm = {"minimal_bytes": minimal, "two_pass_bytes": two_pass,
+           "frac_minimal": round(minimal / (ms_step / 1e3) / (peaks["hbm_gbs"] * 1e9), 4),
+           "frac_two_pass": round(two_pass / (ms_step / 1e3) / (peaks["hbm_gbs"] * 1e9), 4),
+           "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]}
+
+    e2e = None
+    if args.only == "all":
+        e2e_ms, h2d, d2h = bench_e2e(gdn, b, dev, args.steps, args.warmup)
+        e2e_ms = max_over_ranks(e2e_ms, world)
+        e2e = {"value": round(world * T / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    decode = None
+    if args.only in ("all", "decode"):
+        decode = run_decode_part(gdn, W, dev, rank, world, args, peaks)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": round(value / (10240 / (PAGES_H100["prefill_ms"] / 1e3)), 3),
+        "vs_baseline_note": "pages' H100 CPR prefill, 1.412 ms per 5x2048 tokens "
+                            "(layer shape unstated): context, other hardware",
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "rollout prefill: 5 sequences x 2048 tokens packed, H=16, "
+                               "d_k=d_v=128, C=64, bf16 q/k/v/o, fp32 beta/g/state",
+                   "global_batch": world * T, "seq_len": 2048, "parallelism": f"dp{world}",
+                   "l2": "flushed (256 MiB write) before every timed step"},
+        "roofline": roofline,
+        "kernels_ms": {n: round(float(t), 5) for n, t in zip(names, per_k)},
+        "hbm_roofline": hbm,
+        "e2e": e2e,
+        "decode": decode,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+        "wall_s_timed_region": round(wall, 4),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_sample(W)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# Reference arm: the fp64 oracle on the host cores
+# ----------------------------------------------------------------------------
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from rl_train_numerics_b200 import workloads as W
+    b = W.prefill(device="cpu", seed=0)
+    cu = b.cu_seqlens.tolist()
+    heads = 4  # each step: one 2048-token sequence x 4 heads (a bounded sample)
+
+    def one(i):
+        n = i % len(b.lengths)
+        sl = slice(cu[n], cu[n + 1])
+        hs = slice((i * heads) % H, (i * heads) % H + heads)
+        oracle.forward(b.q[sl, hs], b.k[sl, hs], b.v[sl, hs], b.beta[sl, hs], b.g[sl, hs],
+                       np.array([0, cu[n + 1] - cu[n]], np.int32))
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(i)
+    el = time.perf_counter() - t0
+    tokens = args.steps * 2048 * heads / H  # whole-layer tokens (all H heads) equivalent
+    value = tokens / el
+    sample = (f"each step: one 2048-token sequence x {heads} of {H} heads of the 5x2048 "
+              "prefill batch (fp64 token loop); tokens counted as token-heads / 16")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "rollout prefill: 5 sequences x 2048 tokens packed, H=16, "
+                                   "d_k=d_v=128, C=64, bf16 q/k/v, fp32 beta/g",
+                       "global_batch": 10240, "seq_len": 2048, "parallelism": "host"},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
+                             "cores": oracle.max_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--decode-steps", type=int, default=512)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                   help="profiling aid: run only part of the benchmark")
+    p.add_argument("--decode-slots", type=int, default=256)
+    args = p.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

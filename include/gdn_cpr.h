@@ -1,0 +1,222 @@
+/*
+ * gdn_cpr.h -- C ABI of the CPR Gated DeltaNet library (libgdn_cpr.so).
+ *
+ * The layer: "NovaSky's IsoExec Fixes the Hidden Math Bug Corrupting AI
+ * Training Runs", section "Solving the linear-attention headache".  Gated
+ * DeltaNet is evaluated by CPR (chunkwise-parallel recurrent): the
+ * recurrence stays the primary algorithm, a first pass computes the state at
+ * chunk boundaries, a second pass fills in the outputs inside every chunk in
+ * parallel, and decode runs the recurrence but re-synchronises its state
+ * every chunk-size tokens, so that training, prefill and decode share one
+ * rounding schedule.  The recurrence (one state per sequence and head):
+ *
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = scale * S_t q_t,        alpha_t = exp(g_t)
+ *
+ * S is d_v x d_k, stored row-major (row = value channel, contiguous over the
+ * key channel), fp32.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every data pointer is caller-owned DEVICE memory on the current device.
+ *   The library allocates no device memory; scratch space is the caller's
+ *   `workspace`.  Pointers must be 16-byte aligned.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  All calls are asynchronous on it and never synchronise the
+ *   host, except gdn_check_error.
+ * - Argument errors are detected on the host before anything is launched
+ *   and returned synchronously (GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED,
+ *   GDN_ERR_WORKSPACE).  A failed launch returns GDN_ERR_CUDA.  Bad device
+ *   data (for example a decreasing cu_seqlens) cannot be seen on the host:
+ *   the kernels skip the affected work, set a device error word and
+ *   gdn_check_error reports GDN_ERR_DEVICE_DATA.  Nothing traps or hangs.
+ * - Supported shapes: d_k == d_v in {64, 128}, chunk size C == 64, H >= 1.
+ *   Input dtype bf16 or fp32 for q/k/v (beta, g and states are always fp32);
+ *   output dtype bf16 (= round-to-nearest-even of the fp32 result) or fp32.
+ * - g must be finite (alpha = 0 is expressed as a large negative g such as
+ *   -1e4, whose exp underflows to zero).
+ * - Determinism: no float atomics; every (sequence, head) result depends only
+ *   on that sequence's inputs, so outputs are bitwise independent of batch
+ *   composition, order and padding and identical across runs.  Forward and
+ *   decode (with chunk resync) produce bitwise identical outputs.
+ */
+#ifndef GDN_CPR_H
+#define GDN_CPR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_CPR_ABI_VERSION 1
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = -1, /* null pointer, negative size, misaligned pointer, ... */
+  GDN_ERR_UNSUPPORTED = -2, /* valid but not implemented: head dims, chunk size, dtype */
+  GDN_ERR_WORKSPACE = -3,   /* workspace missing or smaller than the query says */
+  GDN_ERR_CUDA = -4,        /* a CUDA launch or runtime call failed */
+  GDN_ERR_DEVICE_DATA = -5, /* device-side validation failed (see gdn_check_error) */
+  GDN_ERR_TIMEOUT = -6      /* reserved: a bounded device-side wait gave up */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
+
+/* Bits of the device error word. */
+#define GDN_DEVERR_CU_SEQLENS 1 /* cu_seqlens not 0-based, not nondecreasing or wrong total */
+#define GDN_DEVERR_POS 2        /* a decode position outside [0, C) */
+
+/* ABI version of the loaded library (GDN_CPR_ABI_VERSION it was built with). */
+int gdn_cpr_abi_version(void);
+
+/* Static string for a gdn_status value. */
+const char* gdn_status_string(int status);
+
+/*
+ * Bytes of device workspace gdn_cpr_forward needs for this problem size.
+ * Returns 0 for arguments gdn_cpr_forward would reject.
+ */
+size_t gdn_cpr_forward_workspace_bytes(int n_seqs, int64_t total_tokens, int H, int dk, int dv,
+                                       int C);
+
+/*
+ * gdn_cpr_forward -- CPR forward over packed variable-length sequences.
+ *
+ * Defines: the section "Solving the linear-attention headache" (first pass:
+ * state at chunk boundaries; second pass: outputs within each chunk).
+ * Chunks start at each sequence's first token and never cross a sequence
+ * boundary.  Pass 1 walks the full chunks of each sequence with the chunk
+ * boundary function (the same one gdn_chunk_boundary and the decode resync
+ * use).  Pass 2 runs the exact per-token recurrence inside every chunk, all
+ * chunks in parallel, from that chunk's boundary state.
+ *
+ * q, k        [total_tokens, H, dk]  in_dtype
+ * v           [total_tokens, H, dv]  in_dtype
+ * beta, g     [total_tokens, H]      fp32; alpha = exp(g)
+ * cu_seqlens  [n_seqs + 1] int32, device; cu_seqlens[0] = 0, nondecreasing,
+ *             cu_seqlens[n_seqs] = total_tokens (checked on the device)
+ * h0          [n_seqs, H, dv, dk] fp32 initial states, or NULL for zeros
+ * o           [total_tokens, H, dv] out_dtype (written for every token)
+ * s_run_final [n_seqs, H, dv, dk] fp32 or NULL: the state decode continues
+ *             from.  For a length that is a multiple of C it equals
+ *             s_bnd_final; otherwise it is the recurrent state after the
+ *             trailing partial chunk.
+ * s_bnd_final [n_seqs, H, dv, dk] fp32 or NULL: the boundary state after the
+ *             last full chunk (h0 for sequences shorter than C).
+ * workspace   device scratch of at least gdn_cpr_forward_workspace_bytes;
+ *             its first 4 bytes are the device error word.
+ * n_seqs may be 0 and sequences may be empty.
+ */
+int gdn_cpr_forward(const void* q, const void* k, const void* v, int in_dtype, const float* beta,
+                    const float* g, const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
+                    int H, int dk, int dv, int C, float scale, const float* h0, void* o,
+                    int out_dtype, float* s_run_final, float* s_bnd_final, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * gdn_cpr_forward_ex -- gdn_cpr_forward that also records caller-created
+ * CUDA events on `stream` around its kernels, for per-kernel timing:
+ * kernel_events[0] before the chunk table, [1] before the boundary prep,
+ * [2] before the boundary walk, [3] before the intra-chunk fill and [4] after
+ * it (an array of 5 cudaEvent_t passed as void*, or NULL for none).  The
+ * computation and its bits are exactly those of gdn_cpr_forward.
+ */
+int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype,
+                       const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
+                       int64_t total_tokens, int H, int dk, int dv, int C, float scale,
+                       const float* h0, void* o, int out_dtype, float* s_run_final,
+                       float* s_bnd_final, void* workspace, size_t workspace_bytes,
+                       void* const* kernel_events, void* stream);
+
+/*
+ * Decode state: caller-owned device arrays for n_slots sequences.
+ *   s_run    [n_slots, H, dv, dk] fp32  running state (not read when pos == 0)
+ *   s_bnd    [n_slots, H, dv, dk] fp32  boundary state at the start of the
+ *                                       current chunk
+ *   buf_k    [n_slots, H, C, dk]  in_dtype  keys of the current chunk so far
+ *   buf_v    [n_slots, H, C, dv]  in_dtype  values of the current chunk so far
+ *   buf_beta [n_slots, H, C] fp32, buf_g [n_slots, H, C] fp32
+ *   pos      [n_slots, H] int32  tokens already in the current chunk, 0..C-1
+ *                                (equal over heads; kept per head so that no
+ *                                two thread blocks share a counter)
+ *   error    [1] int32  device error word (GDN_DEVERR_* bits)
+ */
+typedef struct {
+  float* s_run;
+  float* s_bnd;
+  void* buf_k;
+  void* buf_v;
+  float* buf_beta;
+  float* buf_g;
+  int32_t* pos;
+  int32_t* error;
+  int n_slots;
+} gdn_decode_state;
+
+/*
+ * gdn_cpr_decode_state_from_prefill -- hand a prefill over to decode.
+ * For sequence n (slot slot_idx[n], or n when slot_idx is NULL):
+ * pos = L_n mod C, the buffer receives the last pos tokens' k, v, beta, g
+ * (bit copies), s_run <- s_run_final[n], s_bnd <- s_bnd_final[n].
+ * Inputs are the packed tensors, cu_seqlens and total_tokens passed to
+ * gdn_cpr_forward and the final states it produced.  A slot outside
+ * [0, n_slots) or a cu_seqlens entry outside [0, total_tokens] skips that
+ * sequence and sets a GDN_DEVERR_* bit in st.error.
+ */
+int gdn_cpr_decode_state_from_prefill(const void* k, const void* v, int in_dtype,
+                                      const float* beta, const float* g,
+                                      const int32_t* cu_seqlens, int n_seqs,
+                                      int64_t total_tokens, int H, int dk, int dv, int C,
+                                      const float* s_run_final, const float* s_bnd_final,
+                                      const int32_t* slot_idx, gdn_decode_state st,
+                                      void* stream);
+
+/*
+ * gdn_cpr_decode_step -- one batched decode step with chunk resync.
+ *
+ * Defines: the section "Solving the linear-attention headache" (decode runs
+ * the recurrent form and re-synchronises the hidden state every chunk-size
+ * tokens, so its rounding schedule matches prefill and training).
+ * For each row b (slot s = slot_idx[b], or b when slot_idx is NULL) and head:
+ * one recurrence step from the running state (the boundary state when
+ * pos == 0) gives o[b]; the token is appended to the chunk buffer; when the
+ * buffer becomes full the boundary state is advanced over the C buffered
+ * tokens with the chunk boundary function and becomes the running state,
+ * and pos returns to 0.
+ * q, k [B, H, dk], v [B, H, dv] in_dtype; beta, g [B, H] fp32;
+ * o [B, H, dv] out_dtype.  Rows must name distinct slots.
+ * Launch shapes depend only on (B, H, dk, C), so the call can be captured
+ * in a CUDA graph.
+ */
+int gdn_cpr_decode_step(const void* q, const void* k, const void* v, int in_dtype,
+                        const float* beta, const float* g, const int32_t* slot_idx, int B, int H,
+                        int dk, int dv, int C, float scale, gdn_decode_state st, void* o,
+                        int out_dtype, void* stream);
+
+/*
+ * gdn_chunk_boundary -- the chunk boundary function on its own.
+ * s_end[b,h] = state after applying the C tokens of chunk b, head h to
+ * s_start[b,h], evaluated by the boundary schedule that gdn_cpr_forward's
+ * first pass and the decode resync use (bitwise the same values).
+ * s_start, s_end [B, H, dv, dk] fp32 (s_end == s_start allowed);
+ * k [B, H, C, dk], v [B, H, C, dv] in_dtype; beta, g [B, H, C] fp32.
+ */
+int gdn_chunk_boundary(const float* s_start, const void* k, const void* v, int in_dtype,
+                       const float* beta, const float* g, int B, int H, int dk, int dv, int C,
+                       float* s_end, void* stream);
+
+/*
+ * gdn_check_error -- synchronise `stream`, read the device error word at
+ * `error_word` (the forward workspace, or a decode state's `error`), clear
+ * it, and return GDN_OK or GDN_ERR_DEVICE_DATA.  If bits_out is not NULL it
+ * receives the GDN_DEVERR_* bits that were set.
+ */
+int gdn_check_error(void* error_word, int32_t* bits_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_CPR_H */

@@ -1,0 +1,248 @@
+"""Thin Python binding of libgdn_cpr.so (the C ABI in include/gdn_cpr.h).
+
+Argument marshalling only: torch provides device memory and the current CUDA
+stream; every step of the layer runs in the library's CUDA kernels.  There is
+no CPU or PyTorch fallback: if the shared library is missing, importing this
+module raises, and every call checks that its tensors live on a CUDA device.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn_cpr.so")
+
+GDN_OK = 0
+GDN_ERR_INVALID_ARG = -1
+GDN_ERR_UNSUPPORTED = -2
+GDN_ERR_WORKSPACE = -3
+GDN_ERR_CUDA = -4
+GDN_ERR_DEVICE_DATA = -5
+GDN_ERR_TIMEOUT = -6
+GDN_BF16 = 0
+GDN_F32 = 1
+GDN_DEVERR_CU_SEQLENS = 1
+GDN_DEVERR_POS = 2
+CHUNK = 64
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+class DecodeStateStruct(ctypes.Structure):
+    _fields_ = [("s_run", ctypes.c_void_p), ("s_bnd", ctypes.c_void_p),
+                ("buf_k", ctypes.c_void_p), ("buf_v", ctypes.c_void_p),
+                ("buf_beta", ctypes.c_void_p), ("buf_g", ctypes.c_void_p),
+                ("pos", ctypes.c_void_p), ("error", ctypes.c_void_p),
+                ("n_slots", ctypes.c_int)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run __graft_entry__.build() or "
+                          "python -m rl_train_numerics_b200.build_lib")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                             ctypes.c_size_t)
+    sigs = {
+        "gdn_cpr_abi_version": (i32, []),
+        "gdn_status_string": (ctypes.c_char_p, [i32]),
+        "gdn_cpr_forward_workspace_bytes": (sz, [i32, i64, i32, i32, i32, i32]),
+        "gdn_cpr_forward": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32, f32,
+                                  vp, vp, i32, vp, vp, vp, sz, vp]),
+        "gdn_cpr_forward_ex": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                     f32, vp, vp, i32, vp, vp, vp, sz, vp, vp]),
+        "gdn_cpr_decode_state_from_prefill": (i32, [vp, vp, i32, vp, vp, vp, i32, i64, i32, i32,
+                                                    i32, i32, vp, vp, vp, DecodeStateStruct, vp]),
+        "gdn_cpr_decode_step": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32,
+                                      DecodeStateStruct, vp, i32, vp]),
+        "gdn_chunk_boundary": (i32, [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
+        "gdn_check_error": (i32, [vp, vp, vp]),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.gdn_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != GDN_OK:
+        raise GdnError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("gdn_cpr: tensors must be on a CUDA device (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError("gdn_cpr: tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise ValueError(f"gdn_cpr: unsupported dtype {t.dtype}")
+
+
+def _out_code(in_code: int, out_dtype, o) -> int:
+    """Output dtype code: from `o` when given (must agree with out_dtype), else
+    out_dtype, else the input dtype."""
+    if o is not None:
+        code = _dtype_code(o)
+        if out_dtype is not None and _dtype_code(torch.empty(0, dtype=out_dtype)) != code:
+            raise ValueError("gdn_cpr: out_dtype disagrees with the dtype of o")
+        return code
+    if out_dtype is None:
+        return in_code
+    return _dtype_code(torch.empty(0, dtype=out_dtype))
+
+
+def _torch_dtype(code: int):
+    return torch.bfloat16 if code == GDN_BF16 else torch.float32
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def forward_workspace_bytes(n_seqs: int, total_tokens: int, H: int, dk: int, dv: int,
+                            C: int = CHUNK) -> int:
+    return int(lib.gdn_cpr_forward_workspace_bytes(n_seqs, total_tokens, H, dk, dv, C))
+
+
+def forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=None,
+            C: int = CHUNK, scale: float = 1.0, out_dtype=None, o=None, s_run_final=None,
+            s_bnd_final=None, want_states: bool = True, workspace=None, stream=None,
+            kernel_events=None):
+    """gdn_cpr_forward (gdn_cpr_forward_ex when ``kernel_events``, a list of 5
+    recorded torch.cuda.Event objects, is given).
+    Returns (o, s_run_final, s_bnd_final, workspace)."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = (cu_seqlens.numel() - 1) if n_seqs is None else int(n_seqs)
+    in_code = _dtype_code(q)
+    out_code = _out_code(in_code, out_dtype, o)
+    dev = q.device
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=_torch_dtype(out_code), device=dev)
+    if want_states:
+        if s_run_final is None:
+            s_run_final = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+        if s_bnd_final is None:
+            s_bnd_final = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    need = forward_workspace_bytes(N, T, H, dk, dv, C)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    ev = None
+    if kernel_events is not None:
+        if len(kernel_events) != 5 or any(e.cuda_event == 0 for e in kernel_events):
+            raise ValueError("kernel_events: 5 torch.cuda.Event objects, each recorded once")
+        ev = (ctypes.c_void_p * 5)(*[e.cuda_event for e in kernel_events])
+    st = lib.gdn_cpr_forward_ex(_ptr(q), _ptr(k), _ptr(v), in_code, _ptr(beta), _ptr(g),
+                                _ptr(cu_seqlens), N, T, H, dk, dv, C, float(scale), _ptr(h0),
+                                _ptr(o), out_code, _ptr(s_run_final), _ptr(s_bnd_final),
+                                _ptr(workspace), workspace.numel(), ev, _stream(stream))
+    _check(st, "gdn_cpr_forward")
+    return o, s_run_final, s_bnd_final, workspace
+
+
+def check_error(error_word: torch.Tensor, stream=None) -> int:
+    """gdn_check_error: synchronises, returns the device error bits (and clears them)."""
+    bits = ctypes.c_int32(0)
+    st = lib.gdn_check_error(_ptr(error_word), ctypes.byref(bits), _stream(stream))
+    if st not in (GDN_OK, GDN_ERR_DEVICE_DATA):
+        _check(st, "gdn_check_error")
+    return int(bits.value)
+
+
+class DecodeState:
+    """Caller-owned decode state (device tensors) for n_slots sequences."""
+
+    def __init__(self, n_slots: int, H: int, dk: int, dv: int, in_dtype=torch.bfloat16,
+                 C: int = CHUNK, device="cuda"):
+        self.n_slots, self.H, self.dk, self.dv, self.C = n_slots, H, dk, dv, C
+        self.in_dtype = in_dtype
+        f32 = torch.float32
+        self.s_run = torch.zeros((n_slots, H, dv, dk), dtype=f32, device=device)
+        self.s_bnd = torch.zeros((n_slots, H, dv, dk), dtype=f32, device=device)
+        self.buf_k = torch.zeros((n_slots, H, C, dk), dtype=in_dtype, device=device)
+        self.buf_v = torch.zeros((n_slots, H, C, dv), dtype=in_dtype, device=device)
+        self.buf_beta = torch.zeros((n_slots, H, C), dtype=f32, device=device)
+        self.buf_g = torch.zeros((n_slots, H, C), dtype=f32, device=device)
+        self.pos = torch.zeros((n_slots, H), dtype=torch.int32, device=device)
+        self.error = torch.zeros((1,), dtype=torch.int32, device=device)
+
+    def struct(self) -> DecodeStateStruct:
+        return DecodeStateStruct(self.s_run.data_ptr(), self.s_bnd.data_ptr(),
+                                 self.buf_k.data_ptr(), self.buf_v.data_ptr(),
+                                 self.buf_beta.data_ptr(), self.buf_g.data_ptr(),
+                                 self.pos.data_ptr(), self.error.data_ptr(), self.n_slots)
+
+    def tensors(self):
+        return (self.s_run, self.s_bnd, self.buf_k, self.buf_v, self.buf_beta, self.buf_g,
+                self.pos)
+
+    def clone(self) -> "DecodeState":
+        c = DecodeState.__new__(DecodeState)
+        c.__dict__.update({k: (v.clone() if isinstance(v, torch.Tensor) else v)
+                           for k, v in self.__dict__.items()})
+        return c
+
+
+def decode_state_from_prefill(state: DecodeState, k, v, beta, g, cu_seqlens, s_run_final,
+                              s_bnd_final, *, slot_idx=None, stream=None):
+    N = cu_seqlens.numel() - 1
+    T, H, dk = k.shape
+    st = lib.gdn_cpr_decode_state_from_prefill(
+        _ptr(k), _ptr(v), _dtype_code(k), _ptr(beta), _ptr(g), _ptr(cu_seqlens), N, T, H, dk,
+        v.shape[2], state.C, _ptr(s_run_final), _ptr(s_bnd_final), _ptr(slot_idx),
+        state.struct(), _stream(stream))
+    _check(st, "gdn_cpr_decode_state_from_prefill")
+
+
+def decode_step(state: DecodeState, q, k, v, beta, g, *, slot_idx=None, scale: float = 1.0,
+                out_dtype=None, o=None, stream=None):
+    """gdn_cpr_decode_step for B rows: q,k [B,H,dk], v [B,H,dv], beta,g [B,H]."""
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    in_code = _dtype_code(q)
+    out_code = _out_code(in_code, out_dtype, o)
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=_torch_dtype(out_code), device=q.device)
+    st = lib.gdn_cpr_decode_step(_ptr(q), _ptr(k), _ptr(v), in_code, _ptr(beta), _ptr(g),
+                                 _ptr(slot_idx), B, H, dk, dv, state.C, float(scale),
+                                 state.struct(), _ptr(o), out_code, _stream(stream))
+    _check(st, "gdn_cpr_decode_step")
+    return o
+
+
+def chunk_boundary(s_start, k, v, beta, g, *, s_end=None, stream=None):
+    """gdn_chunk_boundary: k [B,H,C,dk], v [B,H,C,dv], beta,g [B,H,C]; s [B,H,dv,dk]."""
+    B, H, C, dk = k.shape
+    dv = v.shape[3]
+    if s_end is None:
+        s_end = torch.empty_like(s_start)
+    st = lib.gdn_chunk_boundary(_ptr(s_start), _ptr(k), _ptr(v), _dtype_code(k), _ptr(beta),
+                                _ptr(g), B, H, dk, dv, C, _ptr(s_end), _stream(stream))
+    _check(st, "gdn_chunk_boundary")
+    return s_end

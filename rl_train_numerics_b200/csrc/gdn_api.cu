@@ -1,0 +1,244 @@
+// gdn_api.cu -- extern "C" entry points of libgdn_cpr.so (declared in
+// include/gdn_cpr.h).  Host-side argument validation happens here, before any
+// CUDA call, so that argument errors are reported synchronously and without
+// touching the device; the kernels are in gdn_kernels.cu.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/gdn_cpr.h"
+#include "gdn_layout.h"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool valid_dtype(int d) { return d == GDN_BF16 || d == GDN_F32; }
+
+// Shape check shared by every entry point: returns GDN_OK, INVALID_ARG or UNSUPPORTED.
+int check_shape(int H, int dk, int dv, int C, int in_dtype) {
+  if (H <= 0 || dk <= 0 || dv <= 0 || C <= 0) return GDN_ERR_INVALID_ARG;
+  if (!valid_dtype(in_dtype)) return GDN_ERR_INVALID_ARG;
+  if (dk != dv || (dk != 64 && dk != 128) || C != 64) return GDN_ERR_UNSUPPORTED;
+  if (H > 65535) return GDN_ERR_UNSUPPORTED;  // grid.y
+  return GDN_OK;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int gdn_cpr_abi_version(void) { return GDN_CPR_ABI_VERSION; }
+
+const char* gdn_status_string(int status) {
+  switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: unsupported shape or dtype";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing or too small";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA launch or runtime error";
+    case GDN_ERR_DEVICE_DATA: return "GDN_ERR_DEVICE_DATA: device-side validation failed";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: bounded device wait gave up";
+    default: return "unknown gdn_status";
+  }
+}
+
+size_t gdn_cpr_forward_workspace_bytes(int n_seqs, int64_t total_tokens, int H, int dk, int dv,
+                                       int C) {
+  if (n_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return 0;
+  if (check_shape(H, dk, dv, C, GDN_BF16) != GDN_OK) return 0;
+  return gdn::fwd_layout(n_seqs, total_tokens, H, dk, dv, C).total;
+}
+
+int gdn_cpr_forward(const void* q, const void* k, const void* v, int in_dtype, const float* beta,
+                    const float* g, const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
+                    int H, int dk, int dv, int C, float scale, const float* h0, void* o,
+                    int out_dtype, float* s_run_final, float* s_bnd_final, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  return gdn_cpr_forward_ex(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs, total_tokens, H, dk,
+                            dv, C, scale, h0, o, out_dtype, s_run_final, s_bnd_final, workspace,
+                            workspace_bytes, nullptr, stream);
+}
+
+int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype,
+                       const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
+                       int64_t total_tokens, int H, int dk, int dv, int C, float scale,
+                       const float* h0, void* o, int out_dtype, float* s_run_final,
+                       float* s_bnd_final, void* workspace, size_t workspace_bytes,
+                       void* const* kernel_events, void* stream) {
+  if (n_seqs < 0 || total_tokens < 0 || !valid_dtype(out_dtype) || !isfinite(scale))
+    return GDN_ERR_INVALID_ARG;
+  int rc = check_shape(H, dk, dv, C, in_dtype);
+  if (rc != GDN_OK) return rc;
+  if (total_tokens > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+  if (n_seqs == 0) return total_tokens == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+  if (!cu_seqlens || !aligned4(cu_seqlens)) return GDN_ERR_INVALID_ARG;
+  if (total_tokens > 0) {
+    if (!q || !k || !v || !beta || !g || !o) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return GDN_ERR_INVALID_ARG;
+    if (!aligned4(beta) || !aligned4(g)) return GDN_ERR_INVALID_ARG;
+  }
+  if ((h0 && !aligned16(h0)) || (s_run_final && !aligned16(s_run_final)) ||
+      (s_bnd_final && !aligned16(s_bnd_final)))
+    return GDN_ERR_INVALID_ARG;
+  const gdn::FwdLayout lay = gdn::fwd_layout(n_seqs, total_tokens, H, dk, dv, C);
+  if (!workspace || workspace_bytes < lay.total) return GDN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDN_ERR_INVALID_ARG;
+  gdn::FwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.in_bf16 = in_dtype == GDN_BF16;
+  a.beta = beta;
+  a.g = g;
+  a.cu_seqlens = cu_seqlens;
+  a.n_seqs = n_seqs;
+  a.T = total_tokens;
+  a.H = H;
+  a.D = dk;
+  a.scale = scale;
+  a.h0 = h0;
+  a.o = o;
+  a.out_bf16 = out_dtype == GDN_BF16;
+  a.s_run_final = s_run_final;
+  a.s_bnd_final = s_bnd_final;
+  a.ws = static_cast<char*>(workspace);
+  a.lay = lay;
+  a.events = kernel_events;
+  return from_cuda(gdn::launch_forward(a, static_cast<cudaStream_t>(stream)));
+}
+
+static int check_state(const gdn_decode_state& st) {
+  if (st.n_slots <= 0 || !st.s_run || !st.s_bnd || !st.buf_k || !st.buf_v || !st.buf_beta ||
+      !st.buf_g || !st.pos || !st.error)
+    return GDN_ERR_INVALID_ARG;
+  if (!aligned16(st.s_run) || !aligned16(st.s_bnd) || !aligned16(st.buf_k) ||
+      !aligned16(st.buf_v) || !aligned4(st.buf_beta) || !aligned4(st.buf_g) ||
+      !aligned4(st.pos) || !aligned4(st.error))
+    return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+int gdn_cpr_decode_state_from_prefill(const void* k, const void* v, int in_dtype,
+                                      const float* beta, const float* g,
+                                      const int32_t* cu_seqlens, int n_seqs,
+                                      int64_t total_tokens, int H, int dk, int dv, int C,
+                                      const float* s_run_final, const float* s_bnd_final,
+                                      const int32_t* slot_idx, gdn_decode_state st,
+                                      void* stream) {
+  if (n_seqs < 0 || total_tokens < 0) return GDN_ERR_INVALID_ARG;
+  int rc = check_shape(H, dk, dv, C, in_dtype);
+  if (rc != GDN_OK) return rc;
+  if (total_tokens > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+  if (n_seqs == 0) return GDN_OK;
+  if ((rc = check_state(st)) != GDN_OK) return rc;
+  if (!cu_seqlens || !s_run_final || !s_bnd_final) return GDN_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (!k || !v || !beta || !g)) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(s_run_final) || !aligned16(s_bnd_final)) return GDN_ERR_INVALID_ARG;
+  if (!slot_idx && n_seqs > st.n_slots) return GDN_ERR_INVALID_ARG;
+  gdn::HandoffArgs a{};
+  a.k = k;
+  a.v = v;
+  a.in_bf16 = in_dtype == GDN_BF16;
+  a.beta = beta;
+  a.g = g;
+  a.cu_seqlens = cu_seqlens;
+  a.n_seqs = n_seqs;
+  a.T = total_tokens;
+  a.H = H;
+  a.D = dk;
+  a.s_run_final = s_run_final;
+  a.s_bnd_final = s_bnd_final;
+  a.slot_idx = slot_idx;
+  a.s_run = st.s_run;
+  a.s_bnd = st.s_bnd;
+  a.buf_k = st.buf_k;
+  a.buf_v = st.buf_v;
+  a.buf_beta = st.buf_beta;
+  a.buf_g = st.buf_g;
+  a.pos = st.pos;
+  a.error = st.error;
+  a.n_slots = st.n_slots;
+  return from_cuda(gdn::launch_handoff(a, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_cpr_decode_step(const void* q, const void* k, const void* v, int in_dtype,
+                        const float* beta, const float* g, const int32_t* slot_idx, int B, int H,
+                        int dk, int dv, int C, float scale, gdn_decode_state st, void* o,
+                        int out_dtype, void* stream) {
+  if (B < 0 || !valid_dtype(out_dtype) || !isfinite(scale)) return GDN_ERR_INVALID_ARG;
+  int rc = check_shape(H, dk, dv, C, in_dtype);
+  if (rc != GDN_OK) return rc;
+  if (B == 0) return GDN_OK;
+  if ((rc = check_state(st)) != GDN_OK) return rc;
+  if (!q || !k || !v || !beta || !g || !o) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(beta) ||
+      !aligned4(g))
+    return GDN_ERR_INVALID_ARG;
+  if (!slot_idx && B > st.n_slots) return GDN_ERR_INVALID_ARG;
+  gdn::DecArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.in_bf16 = in_dtype == GDN_BF16;
+  a.beta = beta;
+  a.g = g;
+  a.slot_idx = slot_idx;
+  a.B = B;
+  a.H = H;
+  a.D = dk;
+  a.scale = scale;
+  a.s_run = st.s_run;
+  a.s_bnd = st.s_bnd;
+  a.buf_k = st.buf_k;
+  a.buf_v = st.buf_v;
+  a.buf_beta = st.buf_beta;
+  a.buf_g = st.buf_g;
+  a.pos = st.pos;
+  a.error = st.error;
+  a.n_slots = st.n_slots;
+  a.o = o;
+  a.out_bf16 = out_dtype == GDN_BF16;
+  return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_chunk_boundary(const float* s_start, const void* k, const void* v, int in_dtype,
+                       const float* beta, const float* g, int B, int H, int dk, int dv, int C,
+                       float* s_end, void* stream) {
+  if (B < 0) return GDN_ERR_INVALID_ARG;
+  int rc = check_shape(H, dk, dv, C, in_dtype);
+  if (rc != GDN_OK) return rc;
+  if (B == 0) return GDN_OK;
+  if (!s_start || !k || !v || !beta || !g || !s_end) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(s_start) || !aligned16(s_end) || !aligned16(k) || !aligned16(v) ||
+      !aligned4(beta) || !aligned4(g))
+    return GDN_ERR_INVALID_ARG;
+  gdn::BndArgs a{};
+  a.s_start = s_start;
+  a.k = k;
+  a.v = v;
+  a.in_bf16 = in_dtype == GDN_BF16;
+  a.beta = beta;
+  a.g = g;
+  a.B = B;
+  a.H = H;
+  a.D = dk;
+  a.s_end = s_end;
+  return from_cuda(gdn::launch_chunk_boundary(a, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_check_error(void* error_word, int32_t* bits_out, void* stream) {
+  if (!error_word || !aligned4(error_word)) return GDN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t bits = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GDN_ERR_CUDA;
+  if (cudaMemcpy(&bits, error_word, sizeof(bits), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (bits != 0 && cudaMemset(error_word, 0, sizeof(int32_t)) != cudaSuccess) return GDN_ERR_CUDA;
+  if (bits_out) *bits_out = bits;
+  return bits ? GDN_ERR_DEVICE_DATA : GDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,555 @@
+// gdn_kernels.cu -- CUDA kernels of the CPR Gated DeltaNet layer (sm_100a).
+//
+// Forward ("NovaSky's IsoExec Fixes the Hidden Math Bug Corrupting AI
+// Training Runs", section "Solving the linear-attention headache": a first
+// pass computes the recurrent state at chunk boundaries, then the outputs
+// within each chunk are filled in):
+//   k_chunk_table   one block: validates cu_seqlens, numbers the chunks
+//   k_prep          one block per (chunk, head): boundary prep of full chunks
+//   k_walk          one block per (sequence, head): serial walk over chunks
+//   k_fill          one block per (chunk, head): per-token recurrence from the
+//                   chunk's boundary state, all chunks in parallel
+// Decode (same section: the recurrent form re-synchronised every chunk):
+//   k_dec_step      one block per (row, head): one recurrence step
+//   k_bnd           one block per (row, head): resync of units whose chunk
+//                   buffer just filled; also gdn_chunk_boundary
+//   k_handoff       prefill -> decode state
+#include "gdn_boundary.cuh"
+#include "gdn_layout.h"
+
+namespace gdn {
+
+// ----------------------------------------------------------------------------
+// Chunk table
+// ----------------------------------------------------------------------------
+constexpr int kTableThreads = 1024;
+
+__global__ void __launch_bounds__(kTableThreads)
+    k_chunk_table(const int32_t* __restrict__ cu, int N, int64_t T, int32_t* hdr,
+                  int32_t* chunk_off, int32_t* chunk_seq, int64_t max_chunks) {
+  __shared__ long long part[kTableThreads];
+  __shared__ int bad;
+  const int tid = threadIdx.x;
+  if (tid == 0) bad = (cu[0] != 0 || (int64_t)cu[N] != T) ? 1 : 0;
+  __syncthreads();
+  const int64_t per = ((int64_t)N + kTableThreads - 1) / kTableThreads;
+  const int64_t n0 = min((int64_t)N, (int64_t)tid * per);
+  const int64_t n1 = min((int64_t)N, n0 + per);
+  long long local = 0;
+  int mybad = 0;
+  for (int64_t n = n0; n < n1; n++) {
+    const int64_t L = (int64_t)cu[n + 1] - (int64_t)cu[n];
+    if (L < 0) mybad = 1;
+    else local += (L + kChunk - 1) / kChunk;
+  }
+  if (mybad) atomicOr(&bad, 1);
+  part[tid] = local;
+  __syncthreads();
+  if (tid == 0) {
+    long long run = 0;
+    for (int i = 0; i < kTableThreads; i++) {
+      const long long x = part[i];
+      part[i] = run;
+      run += x;
+    }
+    if (run > max_chunks) bad = 1;
+    hdr[1] = bad ? 0 : (int32_t)run;
+    if (!bad) chunk_off[N] = (int32_t)run;
+  }
+  __syncthreads();
+  if (bad) {
+    if (tid == 0) {
+      atomicOr(&hdr[0], kErrCuSeqlens);
+      hdr[2] = 0;
+    }
+    return;
+  }
+  long long off = part[tid];
+  for (int64_t n = n0; n < n1; n++) {
+    const int64_t L = (int64_t)cu[n + 1] - (int64_t)cu[n];
+    const long long nc = (L + kChunk - 1) / kChunk;
+    chunk_off[n] = (int32_t)off;
+    for (long long i = 0; i < nc; i++) chunk_seq[off + i] = (int32_t)n;
+    off += nc;
+  }
+  if (tid == 0) hdr[2] = 1;
+}
+
+// ----------------------------------------------------------------------------
+// Pass 1a: boundary prep of every full chunk (independent of the state)
+// ----------------------------------------------------------------------------
+template <int D, class IN>
+__global__ void __launch_bounds__(kBndThreads)
+    k_prep(const IN* __restrict__ k, const IN* __restrict__ v, const float* __restrict__ beta,
+           const float* __restrict__ g, const int32_t* __restrict__ cu, int H,
+           const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+           const int32_t* __restrict__ chunk_seq, float* __restrict__ Wg,
+           float* __restrict__ Utg, float* __restrict__ dvecg, float* __restrict__ gammag) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  BndSmem<D>& sm = *reinterpret_cast<BndSmem<D>*>(smem_raw);
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (hdr[2] != 1 || c >= hdr[1]) return;
+  const int n = chunk_seq[c];
+  const int ci = c - chunk_off[n];
+  const int64_t L = (int64_t)cu[n + 1] - cu[n];
+  if ((int64_t)(ci + 1) * kChunk > L) return;  // trailing partial chunk: no boundary
+  const int64_t t0 = (int64_t)cu[n] + (int64_t)ci * kChunk;
+  const size_t tok = (size_t)t0 * H + h;
+  stage_chunk_kv<D, IN>(sm.K, sm.V, sm.beta, sm.g, k + tok * D, v + tok * D, (size_t)H * D,
+                        beta + tok, g + tok, (size_t)H);
+  __syncthreads();
+  bnd_prep<D>(sm);
+  const size_t unit = (size_t)c * H + h;
+  float* W = Wg + unit * kChunk * D;
+  float* Ut = Utg + unit * kChunk * D;
+  for (int e = threadIdx.x; e < kChunk * D / 4; e += kBndThreads) {
+    reinterpret_cast<float4*>(W)[e] = reinterpret_cast<const float4*>(&sm.W[0][0])[e];
+    reinterpret_cast<float4*>(Ut)[e] = reinterpret_cast<const float4*>(&sm.Ut[0][0])[e];
+  }
+  for (int i = threadIdx.x; i < kChunk; i += kBndThreads) dvecg[unit * kChunk + i] = sm.dvec[i];
+  if (threadIdx.x == 0) gammag[unit] = sm.gammaC;
+}
+
+// ----------------------------------------------------------------------------
+// Pass 1b: serial walk over the full chunks of one (sequence, head)
+// ----------------------------------------------------------------------------
+template <int D, class IN>
+__global__ void __launch_bounds__(kBndThreads)
+    k_walk(const IN* __restrict__ k, const int32_t* __restrict__ cu, int H,
+           const float* __restrict__ h0, const int32_t* __restrict__ hdr,
+           const int32_t* __restrict__ chunk_off, const float* __restrict__ Wg,
+           const float* __restrict__ Utg, const float* __restrict__ dvecg,
+           const float* __restrict__ gammag, float* __restrict__ bstate,
+           float* __restrict__ s_run_final, float* __restrict__ s_bnd_final) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  WalkSmem<D>& sm = *reinterpret_cast<WalkSmem<D>*>(smem_raw);
+  const int n = blockIdx.x, h = blockIdx.y;
+  if (hdr[2] != 1) return;
+  const int64_t L = (int64_t)cu[n + 1] - cu[n];
+  const int64_t nf = L / kChunk, nc = (L + kChunk - 1) / kChunk;
+  const int64_t base = chunk_off[n];
+  const int r = threadIdx.x;
+  const bool active = r < D;
+  const size_t DD = (size_t)D * D;
+  float s[D];
+  if (active) {
+    if (h0) row_load<D>(s, h0 + ((size_t)n * H + h) * DD + (size_t)r * D);
+    else row_zero<D>(s);
+    if (nc > 0) row_store<D>(s, bstate + ((size_t)base * H + h) * DD + (size_t)r * D);
+  }
+  constexpr int G4 = D / 4;
+  for (int64_t c = 0; c < nf; c++) {
+    const size_t unit = (size_t)(base + c) * H + h;
+    const int64_t t0 = (int64_t)cu[n] + c * kChunk;
+    __syncthreads();
+    for (int e = threadIdx.x; e < kChunk * G4; e += kBndThreads) {
+      reinterpret_cast<float4*>(&sm.W[0][0])[e] =
+          reinterpret_cast<const float4*>(Wg + unit * kChunk * D)[e];
+      reinterpret_cast<float4*>(&sm.Ut[0][0])[e] =
+          reinterpret_cast<const float4*>(Utg + unit * kChunk * D)[e];
+      const int i = e / G4, cc = (e % G4) * 4;
+      *reinterpret_cast<float4*>(&sm.K[i][cc]) = ld4(k + ((size_t)(t0 + i) * H + h) * D + cc);
+    }
+    for (int i = threadIdx.x; i < kChunk; i += kBndThreads) sm.dvec[i] = dvecg[unit * kChunk + i];
+    if (threadIdx.x == 0) sm.gammaC = gammag[unit];
+    __syncthreads();
+    if (active) {
+      bnd_walk_row<D>(s, r, &sm.W[0][0], &sm.Ut[0][0], &sm.K[0][0], &sm.Ud[0][0], sm.dvec,
+                      sm.gammaC);
+      if (c + 1 < nc) row_store<D>(s, bstate + (unit + H) * DD + (size_t)r * D);
+    }
+  }
+  if (active) {
+    const size_t so = ((size_t)n * H + h) * DD + (size_t)r * D;
+    if (s_bnd_final) row_store<D>(s, s_bnd_final + so);
+    if (s_run_final && (L % kChunk) == 0) row_store<D>(s, s_run_final + so);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Pass 2: per-token recurrence inside every chunk, from its boundary state
+// ----------------------------------------------------------------------------
+template <int D>
+struct FillSmem {
+  float k[kChunk + 1][D];  // row kChunk stays zero (the "next key" of the last token)
+  float q[kChunk][D];
+  float v[kChunk][D];
+  float a[kChunk];
+  float b[kChunk];
+};
+
+template <int RT>
+__device__ __forceinline__ float pick(const float (&x)[RT], int l) {
+  float val = x[0];
+#pragma unroll
+  for (int i = 1; i < RT; i++)
+    if (l == i) val = x[i];
+  return val;
+}
+
+template <int D, class IN, class OUT>
+__global__ void __launch_bounds__(128, 2)
+    k_fill(const IN* __restrict__ q, const IN* __restrict__ k, const IN* __restrict__ v,
+           const float* __restrict__ beta, const float* __restrict__ g,
+           const int32_t* __restrict__ cu, int H, float scale, const int32_t* __restrict__ hdr,
+           const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
+           const float* __restrict__ bstate, OUT* __restrict__ o,
+           float* __restrict__ s_run_final) {
+  constexpr int RT = D / 32, M4 = D / 16, G4 = D / 4;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  FillSmem<D>& sm = *reinterpret_cast<FillSmem<D>*>(smem_raw);
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (hdr[2] != 1 || c >= hdr[1]) return;
+  const int n = chunk_seq[c];
+  const int ci = c - chunk_off[n];
+  const int64_t L = (int64_t)cu[n + 1] - cu[n];
+  const int64_t t0 = (int64_t)cu[n] + (int64_t)ci * kChunk;
+  const int len = (int)min((int64_t)kChunk, L - (int64_t)ci * kChunk);
+  const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * RT;
+
+  for (int e = tid; e < (kChunk + 1) * G4; e += 128) {
+    const int i = e / G4, cc = (e % G4) * 4;
+    float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), qq = kk, vv = kk;
+    if (i < len) {
+      const size_t off = ((size_t)(t0 + i) * H + h) * D + cc;
+      kk = ld4(k + off);
+      qq = ld4(q + off);
+      vv = ld4(v + off);
+    }
+    *reinterpret_cast<float4*>(&sm.k[i][cc]) = kk;
+    if (i < kChunk) {
+      *reinterpret_cast<float4*>(&sm.q[i][cc]) = qq;
+      *reinterpret_cast<float4*>(&sm.v[i][cc]) = vv;
+    }
+  }
+  for (int i = tid; i < kChunk; i += 128) {
+    float a = 0.f, b = 0.f;
+    if (i < len) {
+      const size_t tok = (size_t)(t0 + i) * H + h;
+      a = step_decay(g[tok]);
+      b = beta[tok];
+    }
+    sm.a[i] = a;
+    sm.b[i] = b;
+  }
+  Slice<RT, M4> S;
+  slice_load<RT, M4>(S, bstate + ((size_t)c * H + h) * D * D, D, r0, l);
+  __syncthreads();
+
+  float p[RT];
+  slice_dot<RT, M4>(S, [&](int m) { return ld4(&sm.k[0][group_col(l, m)]); }, p);
+#pragma unroll
+  for (int i = 0; i < RT; i++) p[i] = quad_sum(p[i]);
+
+  for (int t = 0; t < len; t++) {
+    const float a = sm.a[t], b = sm.b[t];
+    float u[RT], oacc[RT], pacc[RT];
+#pragma unroll
+    for (int i = 0; i < RT; i++) u[i] = step_u(a, b, p[i], sm.v[t][r0 + i]);
+    slice_update<true, RT, M4>(
+        S, a, u, [&](int m) { return ld4(&sm.k[t][group_col(l, m)]); },
+        [&](int m) { return ld4(&sm.q[t][group_col(l, m)]); },
+        [&](int m) { return ld4(&sm.k[t + 1][group_col(l, m)]); }, oacc, pacc);
+    float ov[RT];
+#pragma unroll
+    for (int i = 0; i < RT; i++) {
+      ov[i] = __fmul_rn(scale, quad_sum(oacc[i]));
+      p[i] = quad_sum(pacc[i]);
+    }
+    if (l < RT) st1(o + ((size_t)(t0 + t) * H + h) * D + r0 + l, pick<RT>(ov, l));
+  }
+  const int64_t nc = (L + kChunk - 1) / kChunk;
+  if (s_run_final && ci == nc - 1 && (L % kChunk) != 0)
+    slice_store<RT, M4>(S, s_run_final + ((size_t)n * H + h) * D * D, D, r0, l);
+}
+
+// ----------------------------------------------------------------------------
+// Decode step
+// ----------------------------------------------------------------------------
+template <int D, class IN, class OUT>
+__global__ void __launch_bounds__(128)
+    k_dec_step(const IN* __restrict__ q, const IN* __restrict__ k, const IN* __restrict__ v,
+               const float* __restrict__ beta, const float* __restrict__ g,
+               const int32_t* __restrict__ slot_idx, int H, float scale, float* s_run,
+               const float* s_bnd, IN* buf_k, IN* buf_v, float* buf_beta, float* buf_g,
+               int32_t* pos, int32_t* error, int n_slots, OUT* __restrict__ o) {
+  constexpr int RT = D / 32, M4 = D / 16;
+  __shared__ int sh_pos, sh_slot;
+  const int b = blockIdx.x, h = blockIdx.y;
+  const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * RT;
+  if (tid == 0) {
+    const int slot = slot_idx ? slot_idx[b] : b;
+    int p0 = -1;
+    if (slot >= 0 && slot < n_slots) p0 = pos[(size_t)slot * H + h];
+    if (p0 < 0 || p0 >= kChunk) {
+      atomicOr(error, kErrPos);
+      p0 = -1;
+    }
+    sh_pos = p0;
+    sh_slot = slot;
+  }
+  __syncthreads();
+  const int p0 = sh_pos;
+  if (p0 < 0) return;
+  const size_t unit = (size_t)sh_slot * H + h;
+  const size_t DD = (size_t)D * D;
+  const size_t tok = (size_t)b * H + h;
+  Slice<RT, M4> S;
+  slice_load<RT, M4>(S, (p0 == 0 ? s_bnd : s_run) + unit * DD, D, r0, l);
+  const IN* kp = k + tok * D;
+  const IN* qp = q + tok * D;
+  const float a = step_decay(g[tok]);
+  const float bt = beta[tok];
+  float p[RT], u[RT], oacc[RT], pacc[RT];
+  slice_dot<RT, M4>(S, [&](int m) { return ld4(kp + group_col(l, m)); }, p);
+#pragma unroll
+  for (int i = 0; i < RT; i++) {
+    p[i] = quad_sum(p[i]);
+    u[i] = step_u(a, bt, p[i], ld1(v + tok * D + r0 + i));
+  }
+  slice_update<false, RT, M4>(
+      S, a, u, [&](int m) { return ld4(kp + group_col(l, m)); },
+      [&](int m) { return ld4(qp + group_col(l, m)); },
+      [&](int m) { return make_float4(0.f, 0.f, 0.f, 0.f); }, oacc, pacc);
+  float ov[RT];
+#pragma unroll
+  for (int i = 0; i < RT; i++) ov[i] = __fmul_rn(scale, quad_sum(oacc[i]));
+  if (l < RT) st1(o + tok * D + r0 + l, pick<RT>(ov, l));
+  if (p0 + 1 < kChunk) slice_store<RT, M4>(S, s_run + unit * DD, D, r0, l);
+  // append the token to the chunk buffer (bit copies)
+  const size_t brow = (unit * kChunk + p0) * D;
+  for (int e = tid; e < D; e += 128) {
+    buf_k[brow + e] = k[tok * D + e];
+    buf_v[brow + e] = v[tok * D + e];
+  }
+  if (tid == 0) {
+    buf_beta[unit * kChunk + p0] = bt;
+    buf_g[unit * kChunk + p0] = g[tok];
+    pos[unit] = p0 + 1;  // kChunk here means "resync pending" until k_bnd runs
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Chunk boundary over a buffer: decode resync (RESYNC) or gdn_chunk_boundary
+// ----------------------------------------------------------------------------
+template <int D, class IN, bool RESYNC>
+__global__ void __launch_bounds__(kBndThreads)
+    k_bnd(const float* s_start, const IN* __restrict__ kb, const IN* __restrict__ vb,
+          const float* __restrict__ bb, const float* __restrict__ gb,
+          const int32_t* __restrict__ slot_idx, int H, int32_t* pos, int n_slots,
+          float* s_end) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  BndSmem<D>& sm = *reinterpret_cast<BndSmem<D>*>(smem_raw);
+  __shared__ int sh_go;
+  const int b = blockIdx.x, h = blockIdx.y;
+  size_t unit = (size_t)b * H + h;
+  if (RESYNC) {
+    if (threadIdx.x == 0) {
+      const int slot = slot_idx ? slot_idx[b] : b;
+      int go = 0;
+      if (slot >= 0 && slot < n_slots) go = (pos[(size_t)slot * H + h] == kChunk);
+      sh_go = go ? 1 + slot : 0;
+    }
+    __syncthreads();
+    if (sh_go == 0) return;
+    unit = (size_t)(sh_go - 1) * H + h;
+  }
+  const size_t DD = (size_t)D * D;
+  stage_chunk_kv<D, IN>(sm.K, sm.V, sm.beta, sm.g, kb + unit * kChunk * D, vb + unit * kChunk * D,
+                        (size_t)D, bb + unit * kChunk, gb + unit * kChunk, 1);
+  __syncthreads();
+  bnd_prep<D>(sm);
+  const int r = threadIdx.x;
+  if (r < D) {
+    float s[D];
+    row_load<D>(s, s_start + unit * DD + (size_t)r * D);
+    bnd_walk_row<D>(s, r, &sm.W[0][0], &sm.Ut[0][0], &sm.K[0][0], &sm.u.Ud[0][0], sm.dvec,
+                    sm.gammaC);
+    row_store<D>(s, s_end + unit * DD + (size_t)r * D);
+  }
+  if (RESYNC && threadIdx.x == 0) pos[unit] = 0;
+}
+
+// ----------------------------------------------------------------------------
+// Prefill -> decode handoff
+// ----------------------------------------------------------------------------
+template <int D, class IN>
+__global__ void __launch_bounds__(128)
+    k_handoff(const IN* __restrict__ k, const IN* __restrict__ v, const float* __restrict__ beta,
+              const float* __restrict__ g, const int32_t* __restrict__ cu, int64_t T, int H,
+              const float* __restrict__ s_run_final, const float* __restrict__ s_bnd_final,
+              const int32_t* __restrict__ slot_idx, float* s_run, float* s_bnd, IN* buf_k,
+              IN* buf_v, float* buf_beta, float* buf_g, int32_t* pos, int32_t* error,
+              int n_slots) {
+  const int n = blockIdx.x, h = blockIdx.y;
+  const int slot = slot_idx ? slot_idx[n] : n;
+  const int64_t c0 = cu[n], c1 = cu[n + 1];
+  if (slot < 0 || slot >= n_slots || c0 < 0 || c1 < c0 || c1 > T) {
+    if (threadIdx.x == 0) atomicOr(error, slot < 0 || slot >= n_slots ? kErrPos : kErrCuSeqlens);
+    return;
+  }
+  const int rem = (int)((c1 - c0) % kChunk);
+  const size_t unit = (size_t)slot * H + h, src = (size_t)n * H + h;
+  const size_t DD = (size_t)D * D;
+  for (size_t e = threadIdx.x; e < DD / 4; e += 128) {
+    reinterpret_cast<float4*>(s_run + unit * DD)[e] =
+        reinterpret_cast<const float4*>(s_run_final + src * DD)[e];
+    reinterpret_cast<float4*>(s_bnd + unit * DD)[e] =
+        reinterpret_cast<const float4*>(s_bnd_final + src * DD)[e];
+  }
+  for (int e = threadIdx.x; e < rem * D; e += 128) {
+    const int i = e / D, c = e % D;
+    const size_t t = (size_t)(c1 - rem + i);
+    buf_k[(unit * kChunk + i) * D + c] = k[(t * H + h) * D + c];
+    buf_v[(unit * kChunk + i) * D + c] = v[(t * H + h) * D + c];
+  }
+  for (int i = threadIdx.x; i < rem; i += 128) {
+    const size_t t = (size_t)(c1 - rem + i);
+    buf_beta[unit * kChunk + i] = beta[t * H + h];
+    buf_g[unit * kChunk + i] = g[t * H + h];
+  }
+  if (threadIdx.x == 0) pos[unit] = rem;
+}
+
+// ----------------------------------------------------------------------------
+// Host launchers
+// ----------------------------------------------------------------------------
+template <class KernelT>
+static cudaError_t set_smem(KernelT kern, size_t bytes) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+#define GDN_TRY(expr)                    \
+  do {                                   \
+    cudaError_t e_ = (expr);             \
+    if (e_ != cudaSuccess) return e_;    \
+  } while (0)
+
+template <int D, class IN, class OUT>
+static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
+  const FwdLayout& L = a.lay;
+  char* ws = a.ws;
+  int32_t* hdr = reinterpret_cast<int32_t*>(ws + L.hdr);
+  int32_t* chunk_off = reinterpret_cast<int32_t*>(ws + L.chunk_off);
+  int32_t* chunk_seq = reinterpret_cast<int32_t*>(ws + L.chunk_seq);
+  float* bstate = reinterpret_cast<float*>(ws + L.bstate);
+  float* Wg = reinterpret_cast<float*>(ws + L.W);
+  float* Utg = reinterpret_cast<float*>(ws + L.Ut);
+  float* dvecg = reinterpret_cast<float*>(ws + L.dvec);
+  float* gammag = reinterpret_cast<float*>(ws + L.gamma);
+  const IN* q = static_cast<const IN*>(a.q);
+  const IN* k = static_cast<const IN*>(a.k);
+  const IN* v = static_cast<const IN*>(a.v);
+
+  auto mark = [&](int i) -> cudaError_t {
+    return a.events ? cudaEventRecord(static_cast<cudaEvent_t>(a.events[i]), st) : cudaSuccess;
+  };
+  GDN_TRY(mark(0));
+  k_chunk_table<<<1, kTableThreads, 0, st>>>(a.cu_seqlens, a.n_seqs, a.T, hdr, chunk_off,
+                                             chunk_seq, L.max_chunks);
+  GDN_TRY(cudaGetLastError());
+  const dim3 gchunks((unsigned)L.max_chunks, (unsigned)a.H);
+  GDN_TRY(mark(1));
+  {
+    auto kern = k_prep<D, IN>;
+    const size_t sm = sizeof(BndSmem<D>);
+    GDN_TRY(set_smem(kern, sm));
+    kern<<<gchunks, kBndThreads, sm, st>>>(k, v, a.beta, a.g, a.cu_seqlens, a.H, hdr, chunk_off,
+                                           chunk_seq, Wg, Utg, dvecg, gammag);
+    GDN_TRY(cudaGetLastError());
+  }
+  GDN_TRY(mark(2));
+  {
+    auto kern = k_walk<D, IN>;
+    const size_t sm = sizeof(WalkSmem<D>);
+    GDN_TRY(set_smem(kern, sm));
+    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), kBndThreads, sm, st>>>(
+        k, a.cu_seqlens, a.H, a.h0, hdr, chunk_off, Wg, Utg, dvecg, gammag, bstate,
+        a.s_run_final, a.s_bnd_final);
+    GDN_TRY(cudaGetLastError());
+  }
+  GDN_TRY(mark(3));
+  {
+    auto kern = k_fill<D, IN, OUT>;
+    const size_t sm = sizeof(FillSmem<D>);
+    GDN_TRY(set_smem(kern, sm));
+    kern<<<gchunks, 128, sm, st>>>(q, k, v, a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
+                                   chunk_off, chunk_seq, bstate, static_cast<OUT*>(a.o),
+                                   a.s_run_final);
+    GDN_TRY(cudaGetLastError());
+  }
+  return mark(4);
+}
+
+template <int D, class IN, class OUT>
+static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
+  const dim3 grid((unsigned)a.B, (unsigned)a.H);
+  k_dec_step<D, IN, OUT><<<grid, 128, 0, st>>>(
+      static_cast<const IN*>(a.q), static_cast<const IN*>(a.k), static_cast<const IN*>(a.v),
+      a.beta, a.g, a.slot_idx, a.H, a.scale, a.s_run, a.s_bnd, static_cast<IN*>(a.buf_k),
+      static_cast<IN*>(a.buf_v), a.buf_beta, a.buf_g, a.pos, a.error, a.n_slots,
+      static_cast<OUT*>(a.o));
+  GDN_TRY(cudaGetLastError());
+  auto kern = k_bnd<D, IN, true>;
+  const size_t sm = sizeof(BndSmem<D>);
+  GDN_TRY(set_smem(kern, sm));
+  kern<<<grid, kBndThreads, sm, st>>>(a.s_bnd, static_cast<const IN*>(a.buf_k),
+                                      static_cast<const IN*>(a.buf_v), a.buf_beta, a.buf_g,
+                                      a.slot_idx, a.H, a.pos, a.n_slots, a.s_bnd);
+  return cudaGetLastError();
+}
+
+template <int D, class IN>
+static cudaError_t handoff_impl(const HandoffArgs& a, cudaStream_t st) {
+  k_handoff<D, IN><<<dim3((unsigned)a.n_seqs, (unsigned)a.H), 128, 0, st>>>(
+      static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, a.cu_seqlens, a.T,
+      a.H, a.s_run_final, a.s_bnd_final, a.slot_idx, a.s_run, a.s_bnd,
+      static_cast<IN*>(a.buf_k), static_cast<IN*>(a.buf_v), a.buf_beta, a.buf_g, a.pos,
+      a.error, a.n_slots);
+  return cudaGetLastError();
+}
+
+template <int D, class IN>
+static cudaError_t boundary_impl(const BndArgs& a, cudaStream_t st) {
+  auto kern = k_bnd<D, IN, false>;
+  const size_t sm = sizeof(BndSmem<D>);
+  GDN_TRY(set_smem(kern, sm));
+  kern<<<dim3((unsigned)a.B, (unsigned)a.H), kBndThreads, sm, st>>>(
+      a.s_start, static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, nullptr,
+      a.H, nullptr, 0, a.s_end);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_forward(const FwdArgs& a, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  if (a.D == 64) {
+    if (a.in_bf16) return a.out_bf16 ? forward_impl<64, bf, bf>(a, st) : forward_impl<64, bf, float>(a, st);
+    return a.out_bf16 ? forward_impl<64, float, bf>(a, st) : forward_impl<64, float, float>(a, st);
+  }
+  if (a.in_bf16) return a.out_bf16 ? forward_impl<128, bf, bf>(a, st) : forward_impl<128, bf, float>(a, st);
+  return a.out_bf16 ? forward_impl<128, float, bf>(a, st) : forward_impl<128, float, float>(a, st);
+}
+
+cudaError_t launch_decode_step(const DecArgs& a, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  if (a.D == 64) {
+    if (a.in_bf16) return a.out_bf16 ? decode_impl<64, bf, bf>(a, st) : decode_impl<64, bf, float>(a, st);
+    return a.out_bf16 ? decode_impl<64, float, bf>(a, st) : decode_impl<64, float, float>(a, st);
+  }
+  if (a.in_bf16) return a.out_bf16 ? decode_impl<128, bf, bf>(a, st) : decode_impl<128, bf, float>(a, st);
+  return a.out_bf16 ? decode_impl<128, float, bf>(a, st) : decode_impl<128, float, float>(a, st);
+}
+
+cudaError_t launch_handoff(const HandoffArgs& a, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  if (a.D == 64) return a.in_bf16 ? handoff_impl<64, bf>(a, st) : handoff_impl<64, float>(a, st);
+  return a.in_bf16 ? handoff_impl<128, bf>(a, st) : handoff_impl<128, float>(a, st);
+}
+
+cudaError_t launch_chunk_boundary(const BndArgs& a, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  if (a.D == 64) return a.in_bf16 ? boundary_impl<64, bf>(a, st) : boundary_impl<64, float>(a, st);
+  return a.in_bf16 ? boundary_impl<128, bf>(a, st) : boundary_impl<128, float>(a, st);
+}
+
+}  // namespace gdn

@@ -1,0 +1,140 @@
+// gdn_layout.h -- host-side layout of the forward workspace and the launch
+// interface between the C ABI (gdn_api.cu) and the kernels (gdn_kernels.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// Workspace of gdn_cpr_forward.  Offsets are 256-byte aligned.
+//   hdr        int32[64]: [0] device error word, [1] number of chunks,
+//                         [2] 1 when this call's chunk table is valid
+//   chunk_off  int32[N+1]   first global chunk index of each sequence
+//   chunk_seq  int32[MC]    sequence of each global chunk
+//   bstate     f32[MC,H,dv,dk]  state at the start of every chunk
+//   W          f32[MC,H,C,dk]   boundary prep, full chunks only
+//   Ut         f32[MC,H,C,dv]
+//   dvec       f32[MC,H,C]
+//   gamma      f32[MC,H]
+// MC = floor(T/C) + N + 1 bounds the number of chunks for any valid
+// cu_seqlens (each sequence adds at most one partial chunk).
+struct FwdLayout {
+  int64_t max_chunks;
+  size_t hdr, chunk_off, chunk_seq, bstate, W, Ut, dvec, gamma, total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline FwdLayout fwd_layout(int n_seqs, int64_t T, int H, int dk, int dv, int C) {
+  FwdLayout L{};
+  L.max_chunks = T / C + n_seqs + 1;
+  const size_t mc = (size_t)L.max_chunks;
+  size_t off = 0;
+  L.hdr = off;
+  off += align256(64 * sizeof(int32_t));
+  L.chunk_off = off;
+  off += align256((size_t)(n_seqs + 1) * sizeof(int32_t));
+  L.chunk_seq = off;
+  off += align256(mc * sizeof(int32_t));
+  L.bstate = off;
+  off += align256(mc * H * dv * dk * sizeof(float));
+  L.W = off;
+  off += align256(mc * H * C * dk * sizeof(float));
+  L.Ut = off;
+  off += align256(mc * H * C * dv * sizeof(float));
+  L.dvec = off;
+  off += align256(mc * H * C * sizeof(float));
+  L.gamma = off;
+  off += align256(mc * H * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+struct FwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int in_bf16;
+  const float* beta;
+  const float* g;
+  const int32_t* cu_seqlens;
+  int n_seqs;
+  int64_t T;
+  int H, D;
+  float scale;
+  const float* h0;
+  void* o;
+  int out_bf16;
+  float* s_run_final;
+  float* s_bnd_final;
+  char* ws;
+  FwdLayout lay;
+  void* const* events;  // 5 cudaEvent_t recorded around the kernels, or null
+};
+
+struct DecArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int in_bf16;
+  const float* beta;
+  const float* g;
+  const int32_t* slot_idx;
+  int B, H, D;
+  float scale;
+  float* s_run;
+  float* s_bnd;
+  void* buf_k;
+  void* buf_v;
+  float* buf_beta;
+  float* buf_g;
+  int32_t* pos;
+  int32_t* error;
+  int n_slots;
+  void* o;
+  int out_bf16;
+};
+
+struct HandoffArgs {
+  const void* k;
+  const void* v;
+  int in_bf16;
+  const float* beta;
+  const float* g;
+  const int32_t* cu_seqlens;
+  int n_seqs;
+  int64_t T;
+  int H, D;
+  const float* s_run_final;
+  const float* s_bnd_final;
+  const int32_t* slot_idx;
+  float* s_run;
+  float* s_bnd;
+  void* buf_k;
+  void* buf_v;
+  float* buf_beta;
+  float* buf_g;
+  int32_t* pos;
+  int32_t* error;
+  int n_slots;
+};
+
+struct BndArgs {
+  const float* s_start;
+  const void* k;
+  const void* v;
+  int in_bf16;
+  const float* beta;
+  const float* g;
+  int B, H, D;
+  float* s_end;
+};
+
+cudaError_t launch_forward(const FwdArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_step(const DecArgs& a, cudaStream_t stream);
+cudaError_t launch_handoff(const HandoffArgs& a, cudaStream_t stream);
+cudaError_t launch_chunk_boundary(const BndArgs& a, cudaStream_t stream);
+
+}  // namespace gdn
