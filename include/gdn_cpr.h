@@ -31,8 +31,9 @@
  *   the kernels skip the affected work, set a device error word and
  *   gdn_check_error reports GDN_ERR_DEVICE_DATA.  Nothing traps or hangs.
  * - Supported shapes: d_k == d_v in {64, 128}, chunk size C == 64, H >= 1.
- *   Input dtype bf16 or fp32 for q/k/v (beta, g and states are always fp32);
- *   output dtype bf16 (= round-to-nearest-even of the fp32 result) or fp32.
+ *   q/k/v in bf16 (d = 64 or 128) or fp32 (d = 64); beta, g and states are
+ *   always fp32; output dtype bf16 (= round-to-nearest-even of the fp32
+ *   result) or fp32.
  * - g must be finite (alpha = 0 is expressed as a large negative g such as
  *   -1e4, whose exp underflows to zero).
  * - Determinism: no float atomics; every (sequence, head) result depends only
@@ -79,7 +80,7 @@ const char* gdn_status_string(int status);
  * Returns 0 for arguments gdn_cpr_forward would reject.
  */
 size_t gdn_cpr_forward_workspace_bytes(int n_seqs, int64_t total_tokens, int H, int dk, int dv,
-                                       int C);
+                                       int C, int in_dtype);
 
 /*
  * gdn_cpr_forward -- CPR forward over packed variable-length sequences.

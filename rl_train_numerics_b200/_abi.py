@@ -54,7 +54,7 @@ def _load() -> ctypes.CDLL:
     sigs = {
         "gdn_cpr_abi_version": (i32, []),
         "gdn_status_string": (ctypes.c_char_p, [i32]),
-        "gdn_cpr_forward_workspace_bytes": (sz, [i32, i64, i32, i32, i32, i32]),
+        "gdn_cpr_forward_workspace_bytes": (sz, [i32, i64, i32, i32, i32, i32, i32]),
         "gdn_cpr_forward": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32, f32,
                                   vp, vp, i32, vp, vp, vp, sz, vp]),
         "gdn_cpr_forward_ex": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32,
@@ -126,8 +126,9 @@ def _stream(stream=None):
 
 
 def forward_workspace_bytes(n_seqs: int, total_tokens: int, H: int, dk: int, dv: int,
-                            C: int = CHUNK) -> int:
-    return int(lib.gdn_cpr_forward_workspace_bytes(n_seqs, total_tokens, H, dk, dv, C))
+                            C: int = CHUNK, in_dtype=torch.bfloat16) -> int:
+    code = GDN_BF16 if in_dtype == torch.bfloat16 else GDN_F32
+    return int(lib.gdn_cpr_forward_workspace_bytes(n_seqs, total_tokens, H, dk, dv, C, code))
 
 
 def forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=None,
@@ -150,7 +151,7 @@ def forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=No
             s_run_final = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
         if s_bnd_final is None:
             s_bnd_final = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
-    need = forward_workspace_bytes(N, T, H, dk, dv, C)
+    need = forward_workspace_bytes(N, T, H, dk, dv, C, q.dtype)
     if workspace is None:
         workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
     ev = None

@@ -20,6 +20,7 @@ int check_shape(int H, int dk, int dv, int C, int in_dtype) {
   if (H <= 0 || dk <= 0 || dv <= 0 || C <= 0) return GDN_ERR_INVALID_ARG;
   if (!valid_dtype(in_dtype)) return GDN_ERR_INVALID_ARG;
   if (dk != dv || (dk != 64 && dk != 128) || C != 64) return GDN_ERR_UNSUPPORTED;
+  if (in_dtype == GDN_F32 && dk != 64) return GDN_ERR_UNSUPPORTED;  // fp32 inputs: d = 64
   if (H > 65535) return GDN_ERR_UNSUPPORTED;  // grid.y
   return GDN_OK;
 }
@@ -46,10 +47,10 @@ const char* gdn_status_string(int status) {
 }
 
 size_t gdn_cpr_forward_workspace_bytes(int n_seqs, int64_t total_tokens, int H, int dk, int dv,
-                                       int C) {
+                                       int C, int in_dtype) {
   if (n_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return 0;
-  if (check_shape(H, dk, dv, C, GDN_BF16) != GDN_OK) return 0;
-  return gdn::fwd_layout(n_seqs, total_tokens, H, dk, dv, C).total;
+  if (check_shape(H, dk, dv, C, in_dtype) != GDN_OK) return 0;
+  return gdn::fwd_layout(n_seqs, total_tokens, H, dk, dv, C, in_dtype == GDN_BF16).total;
 }
 
 int gdn_cpr_forward(const void* q, const void* k, const void* v, int in_dtype, const float* beta,
@@ -83,7 +84,8 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
   if ((h0 && !aligned16(h0)) || (s_run_final && !aligned16(s_run_final)) ||
       (s_bnd_final && !aligned16(s_bnd_final)))
     return GDN_ERR_INVALID_ARG;
-  const gdn::FwdLayout lay = gdn::fwd_layout(n_seqs, total_tokens, H, dk, dv, C);
+  const gdn::FwdLayout lay =
+      gdn::fwd_layout(n_seqs, total_tokens, H, dk, dv, C, in_dtype == GDN_BF16);
   if (!workspace || workspace_bytes < lay.total) return GDN_ERR_WORKSPACE;
   if (!aligned16(workspace)) return GDN_ERR_INVALID_ARG;
   gdn::FwdArgs a{};

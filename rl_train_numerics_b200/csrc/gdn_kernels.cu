@@ -83,10 +83,9 @@ __global__ void __launch_bounds__(kBndThreads)
     k_prep(const IN* __restrict__ k, const IN* __restrict__ v, const float* __restrict__ beta,
            const float* __restrict__ g, const int32_t* __restrict__ cu, int H,
            const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
-           const int32_t* __restrict__ chunk_seq, float* __restrict__ Wg,
-           float* __restrict__ Utg, float* __restrict__ dvecg, float* __restrict__ gammag) {
+           const int32_t* __restrict__ chunk_seq, char* __restrict__ packs) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  BndSmem<D>& sm = *reinterpret_cast<BndSmem<D>*>(smem_raw);
+  PrepSmem<D, IN>& sm = *reinterpret_cast<PrepSmem<D, IN>*>(smem_raw);
   const int c = blockIdx.x, h = blockIdx.y;
   if (hdr[2] != 1 || c >= hdr[1]) return;
   const int n = chunk_seq[c];
@@ -95,75 +94,60 @@ __global__ void __launch_bounds__(kBndThreads)
   if ((int64_t)(ci + 1) * kChunk > L) return;  // trailing partial chunk: no boundary
   const int64_t t0 = (int64_t)cu[n] + (int64_t)ci * kChunk;
   const size_t tok = (size_t)t0 * H + h;
-  stage_chunk_kv<D, IN>(sm.K, sm.V, sm.beta, sm.g, k + tok * D, v + tok * D, (size_t)H * D,
-                        beta + tok, g + tok, (size_t)H);
+  prep_stage<D, IN>(sm, k + tok * D, v + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H);
   __syncthreads();
-  bnd_prep<D>(sm);
-  const size_t unit = (size_t)c * H + h;
-  float* W = Wg + unit * kChunk * D;
-  float* Ut = Utg + unit * kChunk * D;
-  for (int e = threadIdx.x; e < kChunk * D / 4; e += kBndThreads) {
-    reinterpret_cast<float4*>(W)[e] = reinterpret_cast<const float4*>(&sm.W[0][0])[e];
-    reinterpret_cast<float4*>(Ut)[e] = reinterpret_cast<const float4*>(&sm.Ut[0][0])[e];
-  }
-  for (int i = threadIdx.x; i < kChunk; i += kBndThreads) dvecg[unit * kChunk + i] = sm.dvec[i];
-  if (threadIdx.x == 0) gammag[unit] = sm.gammaC;
+  bnd_prep<D, IN>(sm, packs + ((size_t)c * H + h) * Pack<D, IN>::kBytes);
 }
 
 // ----------------------------------------------------------------------------
-// Pass 1b: serial walk over the full chunks of one (sequence, head)
+// Pass 1b: serial walk over the full chunks of one (sequence, head, row block)
 // ----------------------------------------------------------------------------
+constexpr int kWalkWarps = 4;  // 64 state rows per block
+
 template <int D, class IN>
-__global__ void __launch_bounds__(kBndThreads)
-    k_walk(const IN* __restrict__ k, const int32_t* __restrict__ cu, int H,
-           const float* __restrict__ h0, const int32_t* __restrict__ hdr,
-           const int32_t* __restrict__ chunk_off, const float* __restrict__ Wg,
-           const float* __restrict__ Utg, const float* __restrict__ dvecg,
-           const float* __restrict__ gammag, float* __restrict__ bstate,
+__device__ __forceinline__ void pack_fetch(char* dst, const char* src) {
+  constexpr int N16 = (int)(Pack<D, IN>::kBytes / 16);
+  for (int e = threadIdx.x; e < N16; e += 32 * kWalkWarps) cp_async16(dst + 16 * e, src + 16 * e);
+  cp_async_commit();
+}
+
+template <int D, class IN>
+__global__ void __launch_bounds__(32 * kWalkWarps, 1)
+    k_walk(const int32_t* __restrict__ cu, int H, const float* __restrict__ h0,
+           const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+           const char* __restrict__ packs, float* __restrict__ bstate,
            float* __restrict__ s_run_final, float* __restrict__ s_bnd_final) {
+  using PK = Pack<D, IN>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  WalkSmem<D>& sm = *reinterpret_cast<WalkSmem<D>*>(smem_raw);
+  char* const buf0 = reinterpret_cast<char*>(smem_raw);  // double buffer: buf0 + (c & 1) * kBytes
   const int n = blockIdx.x, h = blockIdx.y;
   if (hdr[2] != 1) return;
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
   const int64_t nf = L / kChunk, nc = (L + kChunk - 1) / kChunk;
   const int64_t base = chunk_off[n];
-  const int r = threadIdx.x;
-  const bool active = r < D;
+  const int r0 = blockIdx.z * 16 * kWalkWarps + 16 * (threadIdx.x >> 5);
   const size_t DD = (size_t)D * D;
-  float s[D];
-  if (active) {
-    if (h0) row_load<D>(s, h0 + ((size_t)n * H + h) * DD + (size_t)r * D);
-    else row_zero<D>(s);
-    if (nc > 0) row_store<D>(s, bstate + ((size_t)base * H + h) * DD + (size_t)r * D);
-  }
-  constexpr int G4 = D / 4;
+  float sacc[D / 8][4];
+  if (h0) sacc_load<D>(sacc, h0 + ((size_t)n * H + h) * DD, r0);
+  else sacc_zero<D>(sacc);
+  if (nc > 0) sacc_store<D>(sacc, bstate + ((size_t)base * H + h) * DD, r0);
+  if (nf > 0) pack_fetch<D, IN>(buf0, packs + ((size_t)base * H + h) * PK::kBytes);
   for (int64_t c = 0; c < nf; c++) {
     const size_t unit = (size_t)(base + c) * H + h;
-    const int64_t t0 = (int64_t)cu[n] + c * kChunk;
-    __syncthreads();
-    for (int e = threadIdx.x; e < kChunk * G4; e += kBndThreads) {
-      reinterpret_cast<float4*>(&sm.W[0][0])[e] =
-          reinterpret_cast<const float4*>(Wg + unit * kChunk * D)[e];
-      reinterpret_cast<float4*>(&sm.Ut[0][0])[e] =
-          reinterpret_cast<const float4*>(Utg + unit * kChunk * D)[e];
-      const int i = e / G4, cc = (e % G4) * 4;
-      *reinterpret_cast<float4*>(&sm.K[i][cc]) = ld4(k + ((size_t)(t0 + i) * H + h) * D + cc);
+    if (c + 1 < nf) {
+      pack_fetch<D, IN>(buf0 + ((c + 1) & 1) * PK::kBytes, packs + (unit + H) * PK::kBytes);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    for (int i = threadIdx.x; i < kChunk; i += kBndThreads) sm.dvec[i] = dvecg[unit * kChunk + i];
-    if (threadIdx.x == 0) sm.gammaC = gammag[unit];
     __syncthreads();
-    if (active) {
-      bnd_walk_row<D>(s, r, &sm.W[0][0], &sm.Ut[0][0], &sm.K[0][0], &sm.Ud[0][0], sm.dvec,
-                      sm.gammaC);
-      if (c + 1 < nc) row_store<D>(s, bstate + (unit + H) * DD + (size_t)r * D);
-    }
+    bnd_walk_warp<D, IN>(sacc, buf0 + (c & 1) * PK::kBytes, r0);
+    if (c + 1 < nc) sacc_store<D>(sacc, bstate + (unit + H) * DD, r0);
+    __syncthreads();  // buffer c&1 is refilled by the prefetch of chunk c+2
   }
-  if (active) {
-    const size_t so = ((size_t)n * H + h) * DD + (size_t)r * D;
-    if (s_bnd_final) row_store<D>(s, s_bnd_final + so);
-    if (s_run_final && (L % kChunk) == 0) row_store<D>(s, s_run_final + so);
-  }
+  const size_t so = ((size_t)n * H + h) * DD;
+  if (s_bnd_final) sacc_store<D>(sacc, s_bnd_final + so, r0);
+  if (s_run_final && (L % kChunk) == 0) sacc_store<D>(sacc, s_run_final + so, r0);
 }
 
 // ----------------------------------------------------------------------------
@@ -332,6 +316,12 @@ __global__ void __launch_bounds__(128)
 // ----------------------------------------------------------------------------
 // Chunk boundary over a buffer: decode resync (RESYNC) or gdn_chunk_boundary
 // ----------------------------------------------------------------------------
+template <int D, class IN>
+struct BndSmem {
+  PrepSmem<D, IN> prep;
+  alignas(16) char pack[Pack<D, IN>::kBytes];
+};
+
 template <int D, class IN, bool RESYNC>
 __global__ void __launch_bounds__(kBndThreads)
     k_bnd(const float* s_start, const IN* __restrict__ kb, const IN* __restrict__ vb,
@@ -339,7 +329,7 @@ __global__ void __launch_bounds__(kBndThreads)
           const int32_t* __restrict__ slot_idx, int H, int32_t* pos, int n_slots,
           float* s_end) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  BndSmem<D>& sm = *reinterpret_cast<BndSmem<D>*>(smem_raw);
+  BndSmem<D, IN>& sm = *reinterpret_cast<BndSmem<D, IN>*>(smem_raw);
   __shared__ int sh_go;
   const int b = blockIdx.x, h = blockIdx.y;
   size_t unit = (size_t)b * H + h;
@@ -355,17 +345,19 @@ __global__ void __launch_bounds__(kBndThreads)
     unit = (size_t)(sh_go - 1) * H + h;
   }
   const size_t DD = (size_t)D * D;
-  stage_chunk_kv<D, IN>(sm.K, sm.V, sm.beta, sm.g, kb + unit * kChunk * D, vb + unit * kChunk * D,
-                        (size_t)D, bb + unit * kChunk, gb + unit * kChunk, 1);
+  prep_stage<D, IN>(sm.prep, kb + unit * kChunk * D, vb + unit * kChunk * D, (size_t)D,
+                    bb + unit * kChunk, gb + unit * kChunk, 1);
   __syncthreads();
-  bnd_prep<D>(sm);
-  const int r = threadIdx.x;
-  if (r < D) {
-    float s[D];
-    row_load<D>(s, s_start + unit * DD + (size_t)r * D);
-    bnd_walk_row<D>(s, r, &sm.W[0][0], &sm.Ut[0][0], &sm.K[0][0], &sm.u.Ud[0][0], sm.dvec,
-                    sm.gammaC);
-    row_store<D>(s, s_end + unit * DD + (size_t)r * D);
+  bnd_prep<D, IN>(sm.prep, sm.pack);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+#pragma unroll 1
+  for (int rt = 0; rt < D / 64; rt++) {
+    const int r0 = 16 * warp + 64 * rt;
+    float sacc[D / 8][4];
+    sacc_load<D>(sacc, s_start + unit * DD, r0);
+    bnd_walk_warp<D, IN>(sacc, sm.pack, r0);
+    sacc_store<D>(sacc, s_end + unit * DD, r0);
   }
   if (RESYNC && threadIdx.x == 0) pos[unit] = 0;
 }
@@ -427,20 +419,17 @@ static cudaError_t set_smem(KernelT kern, size_t bytes) {
 
 template <int D, class IN, class OUT>
 static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
+  static_assert(Pack<D, IN>::kBytes == pack_bytes(D, sizeof(IN) == 2), "pack layout mismatch");
   const FwdLayout& L = a.lay;
   char* ws = a.ws;
   int32_t* hdr = reinterpret_cast<int32_t*>(ws + L.hdr);
   int32_t* chunk_off = reinterpret_cast<int32_t*>(ws + L.chunk_off);
   int32_t* chunk_seq = reinterpret_cast<int32_t*>(ws + L.chunk_seq);
   float* bstate = reinterpret_cast<float*>(ws + L.bstate);
-  float* Wg = reinterpret_cast<float*>(ws + L.W);
-  float* Utg = reinterpret_cast<float*>(ws + L.Ut);
-  float* dvecg = reinterpret_cast<float*>(ws + L.dvec);
-  float* gammag = reinterpret_cast<float*>(ws + L.gamma);
+  char* packs = ws + L.pack;
   const IN* q = static_cast<const IN*>(a.q);
   const IN* k = static_cast<const IN*>(a.k);
   const IN* v = static_cast<const IN*>(a.v);
-
   auto mark = [&](int i) -> cudaError_t {
     return a.events ? cudaEventRecord(static_cast<cudaEvent_t>(a.events[i]), st) : cudaSuccess;
   };
@@ -452,20 +441,20 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   GDN_TRY(mark(1));
   {
     auto kern = k_prep<D, IN>;
-    const size_t sm = sizeof(BndSmem<D>);
+    const size_t sm = sizeof(PrepSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
     kern<<<gchunks, kBndThreads, sm, st>>>(k, v, a.beta, a.g, a.cu_seqlens, a.H, hdr, chunk_off,
-                                           chunk_seq, Wg, Utg, dvecg, gammag);
+                                           chunk_seq, packs);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(2));
   {
     auto kern = k_walk<D, IN>;
-    const size_t sm = sizeof(WalkSmem<D>);
+    const size_t sm = 2 * Pack<D, IN>::kBytes;
     GDN_TRY(set_smem(kern, sm));
-    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), kBndThreads, sm, st>>>(
-        k, a.cu_seqlens, a.H, a.h0, hdr, chunk_off, Wg, Utg, dvecg, gammag, bstate,
-        a.s_run_final, a.s_bnd_final);
+    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H, D / (16 * kWalkWarps)), 32 * kWalkWarps, sm,
+           st>>>(a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final,
+                 a.s_bnd_final);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(3));
@@ -491,7 +480,7 @@ static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
       static_cast<OUT*>(a.o));
   GDN_TRY(cudaGetLastError());
   auto kern = k_bnd<D, IN, true>;
-  const size_t sm = sizeof(BndSmem<D>);
+  const size_t sm = sizeof(BndSmem<D, IN>);
   GDN_TRY(set_smem(kern, sm));
   kern<<<grid, kBndThreads, sm, st>>>(a.s_bnd, static_cast<const IN*>(a.buf_k),
                                       static_cast<const IN*>(a.buf_v), a.buf_beta, a.buf_g,
@@ -512,7 +501,7 @@ static cudaError_t handoff_impl(const HandoffArgs& a, cudaStream_t st) {
 template <int D, class IN>
 static cudaError_t boundary_impl(const BndArgs& a, cudaStream_t st) {
   auto kern = k_bnd<D, IN, false>;
-  const size_t sm = sizeof(BndSmem<D>);
+  const size_t sm = sizeof(BndSmem<D, IN>);
   GDN_TRY(set_smem(kern, sm));
   kern<<<dim3((unsigned)a.B, (unsigned)a.H), kBndThreads, sm, st>>>(
       a.s_start, static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, nullptr,
@@ -526,8 +515,8 @@ cudaError_t launch_forward(const FwdArgs& a, cudaStream_t st) {
     if (a.in_bf16) return a.out_bf16 ? forward_impl<64, bf, bf>(a, st) : forward_impl<64, bf, float>(a, st);
     return a.out_bf16 ? forward_impl<64, float, bf>(a, st) : forward_impl<64, float, float>(a, st);
   }
-  if (a.in_bf16) return a.out_bf16 ? forward_impl<128, bf, bf>(a, st) : forward_impl<128, bf, float>(a, st);
-  return a.out_bf16 ? forward_impl<128, float, bf>(a, st) : forward_impl<128, float, float>(a, st);
+  if (!a.in_bf16) return cudaErrorNotSupported;  // fp32 inputs: d = 64 only
+  return a.out_bf16 ? forward_impl<128, bf, bf>(a, st) : forward_impl<128, bf, float>(a, st);
 }
 
 cudaError_t launch_decode_step(const DecArgs& a, cudaStream_t st) {
@@ -536,20 +525,22 @@ cudaError_t launch_decode_step(const DecArgs& a, cudaStream_t st) {
     if (a.in_bf16) return a.out_bf16 ? decode_impl<64, bf, bf>(a, st) : decode_impl<64, bf, float>(a, st);
     return a.out_bf16 ? decode_impl<64, float, bf>(a, st) : decode_impl<64, float, float>(a, st);
   }
-  if (a.in_bf16) return a.out_bf16 ? decode_impl<128, bf, bf>(a, st) : decode_impl<128, bf, float>(a, st);
-  return a.out_bf16 ? decode_impl<128, float, bf>(a, st) : decode_impl<128, float, float>(a, st);
+  if (!a.in_bf16) return cudaErrorNotSupported;  // fp32 inputs: d = 64 only
+  return a.out_bf16 ? decode_impl<128, bf, bf>(a, st) : decode_impl<128, bf, float>(a, st);
 }
 
 cudaError_t launch_handoff(const HandoffArgs& a, cudaStream_t st) {
   using bf = __nv_bfloat16;
   if (a.D == 64) return a.in_bf16 ? handoff_impl<64, bf>(a, st) : handoff_impl<64, float>(a, st);
-  return a.in_bf16 ? handoff_impl<128, bf>(a, st) : handoff_impl<128, float>(a, st);
+  if (!a.in_bf16) return cudaErrorNotSupported;  // fp32 inputs: d = 64 only
+  return handoff_impl<128, bf>(a, st);
 }
 
 cudaError_t launch_chunk_boundary(const BndArgs& a, cudaStream_t st) {
   using bf = __nv_bfloat16;
   if (a.D == 64) return a.in_bf16 ? boundary_impl<64, bf>(a, st) : boundary_impl<64, float>(a, st);
-  return a.in_bf16 ? boundary_impl<128, bf>(a, st) : boundary_impl<128, float>(a, st);
+  if (!a.in_bf16) return cudaErrorNotSupported;  // fp32 inputs: d = 64 only
+  return boundary_impl<128, bf>(a, st);
 }
 
 }  // namespace gdn

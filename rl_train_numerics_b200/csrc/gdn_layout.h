@@ -8,28 +8,35 @@
 
 namespace gdn {
 
+// Bytes of one walk pack (mirrors Pack<D, IN>::kBytes in gdn_boundary.cuh;
+// a static_assert there keeps the two equal).
+constexpr size_t pack_bytes(int D, bool in_bf16) {
+  const size_t NW = in_bf16 ? 2 : 3, NK = in_bf16 ? 1 : 3, C = 64;
+  const size_t b = (NW + NK) * C * (size_t)(D + 8) * 2 + (size_t)D * (C + 8) * 4 + C * 4 + 16;
+  return (b + 127) / 128 * 128;
+}
+
 // Workspace of gdn_cpr_forward.  Offsets are 256-byte aligned.
 //   hdr        int32[64]: [0] device error word, [1] number of chunks,
 //                         [2] 1 when this call's chunk table is valid
 //   chunk_off  int32[N+1]   first global chunk index of each sequence
 //   chunk_seq  int32[MC]    sequence of each global chunk
 //   bstate     f32[MC,H,dv,dk]  state at the start of every chunk
-//   W          f32[MC,H,C,dk]   boundary prep, full chunks only
-//   Ut         f32[MC,H,C,dv]
-//   dvec       f32[MC,H,C]
-//   gamma      f32[MC,H]
+//   pack       [MC,H] walk packs (boundary prep of full chunks)
 // MC = floor(T/C) + N + 1 bounds the number of chunks for any valid
 // cu_seqlens (each sequence adds at most one partial chunk).
 struct FwdLayout {
   int64_t max_chunks;
-  size_t hdr, chunk_off, chunk_seq, bstate, W, Ut, dvec, gamma, total;
+  size_t pack_bytes;
+  size_t hdr, chunk_off, chunk_seq, bstate, pack, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline FwdLayout fwd_layout(int n_seqs, int64_t T, int H, int dk, int dv, int C) {
+inline FwdLayout fwd_layout(int n_seqs, int64_t T, int H, int dk, int dv, int C, bool in_bf16) {
   FwdLayout L{};
   L.max_chunks = T / C + n_seqs + 1;
+  L.pack_bytes = pack_bytes(dk, in_bf16);
   const size_t mc = (size_t)L.max_chunks;
   size_t off = 0;
   L.hdr = off;
@@ -40,14 +47,8 @@ inline FwdLayout fwd_layout(int n_seqs, int64_t T, int H, int dk, int dv, int C)
   off += align256(mc * sizeof(int32_t));
   L.bstate = off;
   off += align256(mc * H * dv * dk * sizeof(float));
-  L.W = off;
-  off += align256(mc * H * C * dk * sizeof(float));
-  L.Ut = off;
-  off += align256(mc * H * C * dv * sizeof(float));
-  L.dvec = off;
-  off += align256(mc * H * C * sizeof(float));
-  L.gamma = off;
-  off += align256(mc * H * sizeof(float));
+  L.pack = off;
+  off += align256(mc * H * L.pack_bytes);
   L.total = off;
   return L;
 }

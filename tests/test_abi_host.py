@@ -52,11 +52,14 @@ def test_abi_version_and_status_strings():
 
 
 def test_workspace_query():
+    import torch
     ws = gdn.forward_workspace_bytes
     assert ws(5, 10240, 16, 128, 128) > 0
     assert ws(5, 20480, 16, 128, 128) > ws(5, 10240, 16, 128, 128)
     # chunk states dominate: at least (T/C + N) * H * d * d * 4 bytes
     assert ws(5, 10240, 16, 128, 128) >= (10240 // 64 + 5) * 16 * 128 * 128 * 4
+    assert ws(1, 100, 2, 64, 64, 64, torch.float32) > ws(1, 100, 2, 64, 64)  # 3-term splits
+    assert ws(1, 100, 2, 128, 128, 64, torch.float32) == 0  # fp32 inputs: d = 64 only
     assert ws(1, 100, 2, 96, 96) == 0          # unsupported head dim
     assert ws(1, 100, 2, 64, 64, 32) == 0      # unsupported chunk size
     assert ws(-1, 100, 2, 64, 64) == 0
@@ -83,6 +86,7 @@ def fwd(**over):
     (dict(dk=96, dv=96), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dk=64, dv=128), gdn.GDN_ERR_UNSUPPORTED),
     (dict(C=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(in_dtype=gdn.GDN_F32, dk=128, dv=128), gdn.GDN_ERR_UNSUPPORTED),
     (dict(T=1 << 31), gdn.GDN_ERR_UNSUPPORTED),
     (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
     (dict(cu=None), gdn.GDN_ERR_INVALID_ARG),
