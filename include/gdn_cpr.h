@@ -132,6 +132,37 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
                        void* const* kernel_events, void* stream);
 
 /*
+ * gdn_cpr_forward_noalloc -- gdn_cpr_forward for callers that cannot
+ * allocate device memory.  (No counterpart on the pages: it exists for
+ * callers of this library, such as a host runtime that owns the device memory
+ * pool, a plugin host without a device allocator, or code that must not
+ * allocate on its hot path.)
+ *
+ * Same arguments and results as gdn_cpr_forward, without the workspace: the
+ * scratch space is a GDN_NOALLOC_SCRATCH_BYTES array compiled into the
+ * library, one per GPU, kept from its first use on that device until the
+ * process exits.  No cudaMalloc, cudaFree or other allocating call is made.
+ * - Size limit: a problem whose gdn_cpr_forward_workspace_bytes exceeds
+ *   GDN_NOALLOC_SCRATCH_BYTES is rejected with GDN_ERR_WORKSPACE before any
+ *   device work.
+ * - The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ * - Every call shares the array, so calls that can overlap on the GPU race;
+ *   order them (one stream, or events).  Each call clears the array's error
+ *   word before its kernels run.
+ * - error_word: optional caller-owned device int32; when not NULL it
+ *   receives the call's device error bits (GDN_DEVERR_*), readable with
+ *   gdn_check_error(error_word, ...).
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int gdn_cpr_forward_noalloc(const void* q, const void* k, const void* v, int in_dtype,
+                            const float* beta, const float* g, const int32_t* cu_seqlens,
+                            int n_seqs, int64_t total_tokens, int H, int dk, int dv, int C,
+                            float scale, const float* h0, void* o, int out_dtype,
+                            float* s_run_final, float* s_bnd_final, int32_t* error_word,
+                            void* stream);
+
+/*
  * Decode state: caller-owned device arrays for n_slots sequences.
  *   s_run    [n_slots, H, dv, dk] fp32  running state (not read when pos == 0)
  *   s_bnd    [n_slots, H, dv, dk] fp32  boundary state at the start of the

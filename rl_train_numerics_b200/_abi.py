@@ -59,6 +59,8 @@ def _load() -> ctypes.CDLL:
                                   vp, vp, i32, vp, vp, vp, sz, vp]),
         "gdn_cpr_forward_ex": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32,
                                      f32, vp, vp, i32, vp, vp, vp, sz, vp, vp]),
+        "gdn_cpr_forward_noalloc": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32,
+                                          i32, f32, vp, vp, i32, vp, vp, vp, vp]),
         "gdn_cpr_decode_state_from_prefill": (i32, [vp, vp, i32, vp, vp, vp, i32, i64, i32, i32,
                                                     i32, i32, vp, vp, vp, DecodeStateStruct, vp]),
         "gdn_cpr_decode_step": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32,

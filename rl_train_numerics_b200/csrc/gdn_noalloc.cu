@@ -1,0 +1,89 @@
+// gdn_noalloc.cu -- gdn_cpr_forward_noalloc: the CPR forward for callers that
+// cannot allocate device memory.
+//
+// Some callers of this library cannot call cudaMalloc: for example a host
+// runtime that owns the device memory pool and does not lend it out, a plugin
+// host that gives a C library no allocator, or code that must not allocate on
+// its hot path.  This entry point runs exactly gdn_cpr_forward, with its
+// scratch space taken from a fixed-size array compiled into the library
+// instead of a caller-provided workspace.  It calls no cudaMalloc, cudaFree or
+// other allocating routine.
+//
+// The array holds GDN_NOALLOC_SCRATCH_BYTES (32 MiB).  Every GPU on which the
+// library's device code for this file is loaded keeps that much memory until
+// the process exits (with CUDA's default lazy module loading, from the first
+// call of this entry point on that device).  In host code the array's name is
+// only a host-side stand-in, not a device address, so the device address is
+// looked up once per device with cudaGetSymbolAddress (with that device
+// current) and cached; that set-up happens in the first call on each device,
+// which should therefore come before any stream capture.
+//
+// Every call shares the one array per device and leaves its contents behind
+// for the next call.  The forward writes every part of the scratch it reads
+// before reading it, except the device error word, which this entry point
+// clears at the start of each call.  Calls whose work can overlap on the GPU
+// (for instance on two streams without an ordering between them) race on the
+// array: callers must order them.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/gdn_cpr.h"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up once).
+int scratch_on_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return GDN_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" int gdn_cpr_forward_noalloc(const void* q, const void* k, const void* v, int in_dtype,
+                                       const float* beta, const float* g,
+                                       const int32_t* cu_seqlens, int n_seqs,
+                                       int64_t total_tokens, int H, int dk, int dv, int C,
+                                       float scale, const float* h0, void* o, int out_dtype,
+                                       float* s_run_final, float* s_bnd_final,
+                                       int32_t* error_word, void* stream) {
+  const size_t need = gdn_cpr_forward_workspace_bytes(n_seqs, total_tokens, H, dk, dv, C,
+                                                      in_dtype);
+  if (need == 0 || n_seqs == 0) {
+    // Rejected shapes, or an empty batch: the regular entry point reports the
+    // exact status (or returns GDN_OK for an empty batch) without device work.
+    return gdn_cpr_forward_ex(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs, total_tokens, H,
+                              dk, dv, C, scale, h0, o, out_dtype, s_run_final, s_bnd_final,
+                              nullptr, 0, nullptr, stream);
+  }
+  if (need > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;  // beyond the fixed scratch
+  void* scratch = nullptr;
+  int rc = scratch_on_current_device(&scratch);
+  if (rc != GDN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, sizeof(int32_t), st) != cudaSuccess) return GDN_ERR_CUDA;
+  rc = gdn_cpr_forward_ex(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs, total_tokens, H, dk,
+                          dv, C, scale, h0, o, out_dtype, s_run_final, s_bnd_final, scratch,
+                          GDN_NOALLOC_SCRATCH_BYTES, nullptr, stream);
+  if (rc != GDN_OK || error_word == nullptr) return rc;
+  if (cudaMemcpyAsync(error_word, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
+      cudaSuccess)
+    return GDN_ERR_CUDA;
+  return GDN_OK;
+}
