@@ -38,7 +38,8 @@
 //   T        right-looking substitution: T_ij accumulates -A_im T_mj over
 //            m = j .. i-1 (one fma each)
 //   W, U~    (T_im * (beta_m expf(G_m))) and (T_im * beta_m), split, then
-//            k16 steps m ascending up to the diagonal block
+//            k16 steps m ascending up to the diagonal block (U~ is formed
+//            transposed, as V^T Tv^T)
 //   U        Ud_i = exp(G_C - G_i) * (U~_ir - (S0 W^T)_ri)
 //   S_C      accumulator starts at exp(G_C) * S0, then k16 steps over i
 #pragma once
@@ -97,17 +98,17 @@ struct Pack {
   }
 };
 
-// Shared memory of the prep.
+// Shared memory of the prep.  A is stored packed (strictly lower triangle,
+// row-major: element (i, j), j < i, at i(i-1)/2 + j).
 template <int D, class IN>
 struct PrepSmem {
   static constexpr int NW = Splits<IN>::W, NK = Splits<IN>::K;
-  static constexpr int LDB = D + 8, LDA = kChunk + 4, LDT = kChunk + 8;
+  static constexpr int LDB = D + 8, LDT = kChunk + 8;
   __nv_bfloat16 K[NK][kChunk][LDB];
   __nv_bfloat16 V[NK][kChunk][LDB];
-  float A[kChunk][LDA];
-  float T[kChunk][LDA];
   __nv_bfloat16 Tb[NW][kChunk][LDT];
   __nv_bfloat16 Tv[NW][kChunk][LDT];
+  float A[kChunk * (kChunk - 1) / 2];
   double G[kChunk];
   float beta[kChunk];
   float g[kChunk];
@@ -116,27 +117,42 @@ struct PrepSmem {
   float gammaC;
 };
 
+__device__ __forceinline__ constexpr int tri(int i, int j) { return i * (i - 1) / 2 + j; }
+
 // Stage one chunk's k, v (rows at stride `ld` elements), beta, g (stride ldbg)
-// into the prep's shared memory, splitting k and v into bf16 terms.
+// into the prep's shared memory.  bf16 inputs are copied as is (cp.async);
+// fp32 inputs are split into three bf16 terms.  Ends with the copies landed
+// and a block barrier.
 template <int D, class IN>
 __device__ __forceinline__ void prep_stage(PrepSmem<D, IN>& sm, const IN* k, const IN* v,
                                            size_t ld, const float* bsrc, const float* gsrc,
                                            size_t ldbg) {
-  constexpr int NK = Splits<IN>::K, G4 = D / 4;
-  for (int e = threadIdx.x; e < kChunk * G4; e += kBndThreads) {
-    const int i = e / G4, c = (e % G4) * 4;
-    const float4 kk = ld4(k + i * ld + c);
-    const float4 vv = ld4(v + i * ld + c);
-    const float kx[4] = {kk.x, kk.y, kk.z, kk.w}, vx[4] = {vv.x, vv.y, vv.z, vv.w};
+  constexpr int NK = Splits<IN>::K;
+  if constexpr (NK == 1) {
+    constexpr int P = D / 8;  // 16-byte pieces per row
+    for (int e = threadIdx.x; e < 2 * kChunk * P; e += kBndThreads) {
+      const int r = (e / P) % kChunk, c = (e % P) * 8;
+      if (e < kChunk * P) cp_async16(&sm.K[0][r][c], k + (size_t)r * ld + c);
+      else cp_async16(&sm.V[0][r][c], v + (size_t)r * ld + c);
+    }
+    cp_async_commit();
+  } else {
+    constexpr int G4 = D / 4;
+    for (int e = threadIdx.x; e < kChunk * G4; e += kBndThreads) {
+      const int i = e / G4, c = (e % G4) * 4;
+      const float4 kk = ld4(k + i * ld + c);
+      const float4 vv = ld4(v + i * ld + c);
+      const float kx[4] = {kk.x, kk.y, kk.z, kk.w}, vx[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
-    for (int q = 0; q < 4; q++) {
-      __nv_bfloat16 ks[NK], vs[NK];
-      split_bf16<NK>(kx[q], ks);
-      split_bf16<NK>(vx[q], vs);
+      for (int q = 0; q < 4; q++) {
+        __nv_bfloat16 ks[NK], vs[NK];
+        split_bf16<NK>(kx[q], ks);
+        split_bf16<NK>(vx[q], vs);
 #pragma unroll
-      for (int t = 0; t < NK; t++) {
-        sm.K[t][i][c + q] = ks[t];
-        sm.V[t][i][c + q] = vs[t];
+        for (int t = 0; t < NK; t++) {
+          sm.K[t][i][c + q] = ks[t];
+          sm.V[t][i][c + q] = vs[t];
+        }
       }
     }
   }
@@ -144,6 +160,8 @@ __device__ __forceinline__ void prep_stage(PrepSmem<D, IN>& sm, const IN* k, con
     sm.beta[i] = bsrc[i * ldbg];
     sm.g[i] = gsrc[i * ldbg];
   }
+  if constexpr (NK == 1) cp_async_wait<0>();
+  __syncthreads();
 }
 
 // ldmatrix address of the A fragment (x4) of rows r0.., columns c0.. in a
@@ -152,6 +170,12 @@ __device__ __forceinline__ const __nv_bfloat16* afrag_addr(const __nv_bfloat16* 
                                                            int r0, int c0) {
   const int lane = threadIdx.x & 31, mi = lane >> 3;
   return base + (size_t)(r0 + (mi & 1) * 8 + (lane & 7)) * ld + c0 + (mi >> 1) * 8;
+}
+// A fragment (x4.trans) of A[r][c] = M[c][r] (M row-major, rows = the k index).
+__device__ __forceinline__ const __nv_bfloat16* afrag_t_addr(const __nv_bfloat16* base, int ld,
+                                                             int r0, int c0) {
+  const int lane = threadIdx.x & 31, mi = lane >> 3;
+  return base + (size_t)(c0 + (mi >> 1) * 8 + (lane & 7)) * ld + r0 + (mi & 1) * 8;
 }
 // B fragments (x4 = two n8 tiles) of B[k][n] = M[n][k] (M row-major, rows = n).
 __device__ __forceinline__ const __nv_bfloat16* bfrag_nk_addr(const __nv_bfloat16* base, int ld,
@@ -166,8 +190,9 @@ __device__ __forceinline__ const __nv_bfloat16* bfrag_kn_addr(const __nv_bfloat1
   return base + (size_t)(k0 + (mi & 1) * 8 + (lane & 7)) * ld + n0 + (mi >> 1) * 8;
 }
 
-// Prep of one chunk: sm.K, sm.V, sm.beta, sm.g staged -> the walk pack at
-// `pack` (global or shared; generic addressing).  All kBndThreads threads.
+// Prep of one chunk: sm.K, sm.V, sm.beta, sm.g staged (prep_stage) -> the
+// walk pack at `pack` (global or shared; generic addressing).  All
+// kBndThreads threads.
 template <int D, class IN>
 __device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
   using PK = Pack<D, IN>;
@@ -175,33 +200,13 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
   constexpr int LDB = PrepSmem<D, IN>::LDB, LDT = PrepSmem<D, IN>::LDT;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
 
-  if (tid == 0) {
-    double acc = 0.0;
-    for (int i = 0; i < kChunk; i++) {
-      acc += (double)sm.g[i];
-      sm.G[i] = acc;
-    }
-  }
-  __syncthreads();
-  for (int i = tid; i < kChunk; i += kBndThreads) {
-    sm.bg[i] = __fmul_rn(sm.beta[i], expf(__double2float_rn(sm.G[i])));
-    sm.dvec[i] = expf(__double2float_rn(sm.G[kChunk - 1] - sm.G[i]));
-  }
-  if (tid == 0) sm.gammaC = expf(__double2float_rn(sm.G[kChunk - 1]));
-  for (int e = tid; e < kChunk * kChunk; e += kBndThreads) {
-    const int i = e / kChunk, j = e % kChunk;
-    sm.T[i][j] = (i == j) ? 1.f : 0.f;
-    sm.A[i][j] = 0.f;
-  }
-  __syncthreads();
-
   // P = K K^T on the tensor cores; warp w owns rows 16w..16w+15 (m-tile w)
-  // and the n8 tiles that reach below the diagonal.
+  // and the n8 tiles that reach below the diagonal.  Warp 0, which has the
+  // fewest tiles, then accumulates G.
+  float acc[8][4];
   {
     using PP = SplitPairs<NK, NK>;
     const int m0 = 16 * warp;
-    const int ntiles = 2 * warp + 2;  // columns 0 .. 16w+15
-    float acc[8][4];
 #pragma unroll
     for (int n = 0; n < 8; n++)
 #pragma unroll
@@ -213,7 +218,7 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
       for (int t = 0; t < NK; t++) ldsm_x4(a[t], afrag_addr(&sm.K[t][0][0], LDB, m0, 16 * ks));
 #pragma unroll
       for (int np = 0; np < 4; np++) {
-        if (2 * np < ntiles) {
+        if (np <= warp) {
           uint32_t b[NK][4];
 #pragma unroll
           for (int t = 0; t < NK; t++)
@@ -226,88 +231,98 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
         }
       }
     }
+  }
+  if (tid == 0) {
+    double s = 0.0;
+    for (int i = 0; i < kChunk; i++) {
+      s += (double)sm.g[i];
+      sm.G[i] = s;
+    }
+  }
+  __syncthreads();
+  {
+    const int m0 = 16 * warp;
 #pragma unroll
     for (int n = 0; n < 8; n++) {
-      if (n < ntiles) {
+      if (n < 2 * warp + 2) {
 #pragma unroll
         for (int e = 0; e < 4; e++) {
           const int i = m0 + gq + (e >> 1) * 8, j = 8 * n + 2 * tq + (e & 1);
           if (j < i) {
             const float decay = expf(__double2float_rn(sm.G[i] - sm.G[j]));
-            sm.A[i][j] = __fmul_rn(__fmul_rn(sm.beta[i], decay), acc[n][e]);
+            sm.A[tri(i, j)] = __fmul_rn(__fmul_rn(sm.beta[i], decay), acc[n][e]);
           }
         }
       }
     }
   }
+  for (int i = tid; i < kChunk; i += kBndThreads) {
+    sm.bg[i] = __fmul_rn(sm.beta[i], expf(__double2float_rn(sm.G[i])));
+    sm.dvec[i] = expf(__double2float_rn(sm.G[kChunk - 1] - sm.G[i]));
+  }
+  if (tid == 0) sm.gammaC = expf(__double2float_rn(sm.G[kChunk - 1]));
   __syncthreads();
 
-  // T = (I + A)^{-1}, right-looking: step m finalises row m.
-  for (int m = 0; m < kChunk - 1; m++) {
-    const int ni = kChunk - 1 - m, nj = m + 1;
-    for (int e = tid; e < ni * nj; e += kBndThreads) {
-      const int i = m + 1 + e / nj, j = e % nj;
-      sm.T[i][j] = __fmaf_rn(-sm.A[i][m], sm.T[m][j], sm.T[i][j]);
-    }
-    __syncthreads();
-  }
-
-  // Tb = T diag(beta*gamma), Tv = T diag(beta), split into bf16 terms.
-  for (int e = tid; e < kChunk * kChunk; e += kBndThreads) {
-    const int i = e / kChunk, m = e % kChunk;
-    const float t = sm.T[i][m];
-    __nv_bfloat16 sb[NW], sv[NW];
-    split_bf16<NW>(__fmul_rn(t, sm.bg[m]), sb);
-    split_bf16<NW>(__fmul_rn(t, sm.beta[m]), sv);
+  // T = (I + A)^{-1}, column j held in registers by thread j: right-looking
+  // over m, so T_ij accumulates -A_im T_mj in ascending m.  Steps m < j only
+  // add signed zeros to zeros (T_mj = 0 there), leaving the bits unchanged.
+  // Then Tb = T diag(beta*gamma), Tv = T diag(beta), split into bf16 terms.
+  if (tid < kChunk) {
+    const int j = tid;
+    float t[kChunk];
 #pragma unroll
-    for (int q = 0; q < NW; q++) {
-      sm.Tb[q][i][m] = sb[q];
-      sm.Tv[q][i][m] = sv[q];
+    for (int i = 0; i < kChunk; i++) t[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int m = 0; m < kChunk - 1; m++) {
+      const float tm = t[m];
+#pragma unroll
+      for (int i = m + 1; i < kChunk; i++) t[i] = __fmaf_rn(-sm.A[tri(i, m)], tm, t[i]);
+    }
+    const float bgj = sm.bg[j], bj = sm.beta[j];
+#pragma unroll
+    for (int i = 0; i < kChunk; i++) {
+      __nv_bfloat16 sb[NW], sv[NW];
+      split_bf16<NW>(__fmul_rn(t[i], bgj), sb);
+      split_bf16<NW>(__fmul_rn(t[i], bj), sv);
+#pragma unroll
+      for (int q = 0; q < NW; q++) {
+        sm.Tb[q][i][j] = sb[q];
+        sm.Tv[q][i][j] = sv[q];
+      }
     }
   }
   __syncthreads();
 
-  // W = Tb K and U~ = Tv V; warp w owns columns [D/4 * w, D/4 * (w+1)).
+  // W = Tb K (rows i; warp w owns columns [D/4 w, D/4 (w+1))), and
+  // U~^T = V^T Tv^T (rows c; warp w owns rows [D/4 w, D/4 (w+1))).
   {
-    using PP = SplitPairs<NW, NK>;
-    constexpr int NT = D / 32;  // n8 tiles per warp: D/4 columns
+    using PW = SplitPairs<NW, NK>;
+    constexpr int NT = D / 32;  // n8 tiles of W per warp (D/4 columns)
     const int c0 = (D / 4) * warp;
-    __nv_bfloat16* Wp[NW];
-#pragma unroll
-    for (int q = 0; q < NW; q++) Wp[q] = PK::W(pack, q);
-    float* Up = PK::U(pack);
 #pragma unroll 1
     for (int mt = 0; mt < 4; mt++) {
-      float w[NT][4], u[NT][4];
+      float w[NT][4];
 #pragma unroll
       for (int n = 0; n < NT; n++)
 #pragma unroll
-        for (int e = 0; e < 4; e++) w[n][e] = u[n][e] = 0.f;
+        for (int e = 0; e < 4; e++) w[n][e] = 0.f;
       for (int ks = 0; ks <= mt; ks++) {
-        uint32_t ab[NW][4], av[NW][4];
+        uint32_t ab[NW][4];
 #pragma unroll
-        for (int q = 0; q < NW; q++) {
-          ldsm_x4(ab[q], afrag_addr(&sm.Tb[q][0][0], LDT, 16 * mt, 16 * ks));
-          ldsm_x4(av[q], afrag_addr(&sm.Tv[q][0][0], LDT, 16 * mt, 16 * ks));
-        }
+        for (int q = 0; q < NW; q++) ldsm_x4(ab[q], afrag_addr(&sm.Tb[q][0][0], LDT, 16 * mt, 16 * ks));
 #pragma unroll
         for (int np = 0; np < NT / 2; np++) {
-          uint32_t bk[NK][4], bv[NK][4];
+          uint32_t bk[NK][4];
 #pragma unroll
-          for (int t = 0; t < NK; t++) {
+          for (int t = 0; t < NK; t++)
             ldsm_x4_t(bk[t], bfrag_kn_addr(&sm.K[t][0][0], LDB, 16 * ks, c0 + 16 * np));
-            ldsm_x4_t(bv[t], bfrag_kn_addr(&sm.V[t][0][0], LDB, 16 * ks, c0 + 16 * np));
-          }
 #pragma unroll
-          for (int p = 0; p < PP::kCount; p++) {
-            mma16816(w[2 * np], ab[PP::a(p)], bk[PP::b(p)][0], bk[PP::b(p)][1]);
-            mma16816(w[2 * np + 1], ab[PP::a(p)], bk[PP::b(p)][2], bk[PP::b(p)][3]);
-            mma16816(u[2 * np], av[PP::a(p)], bv[PP::b(p)][0], bv[PP::b(p)][1]);
-            mma16816(u[2 * np + 1], av[PP::a(p)], bv[PP::b(p)][2], bv[PP::b(p)][3]);
+          for (int p = 0; p < PW::kCount; p++) {
+            mma16816(w[2 * np], ab[PW::a(p)], bk[PW::b(p)][0], bk[PW::b(p)][1]);
+            mma16816(w[2 * np + 1], ab[PW::a(p)], bk[PW::b(p)][2], bk[PW::b(p)][3]);
           }
         }
       }
-      // W -> bf16 terms (row i, column c); U~ -> U~^T (row c, column i), fp32.
 #pragma unroll
       for (int n = 0; n < NT; n++) {
 #pragma unroll
@@ -318,11 +333,47 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
           split_bf16<NW>(w[n][2 * hf + 1], s1);
 #pragma unroll
           for (int q = 0; q < NW; q++)
-            *reinterpret_cast<uint32_t*>(Wp[q] + (size_t)i * PK::LDB + c) = pack_bf16(s0[q], s1[q]);
-          Up[(size_t)c * PK::LDU + i] = u[n][2 * hf];
-          Up[(size_t)(c + 1) * PK::LDU + i] = u[n][2 * hf + 1];
+            *reinterpret_cast<uint32_t*>(PK::W(pack, q) + (size_t)i * PK::LDB + c) =
+                pack_bf16(s0[q], s1[q]);
         }
       }
+    }
+    using PU = SplitPairs<NK, NW>;
+    float* Up = PK::U(pack);
+#pragma unroll 1
+    for (int mt = 0; mt < D / 64; mt++) {
+      const int r0 = c0 + 16 * mt;  // rows c of U~^T
+      float u[8][4];
+#pragma unroll
+      for (int n = 0; n < 8; n++)
+#pragma unroll
+        for (int e = 0; e < 4; e++) u[n][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < 4; ks++) {
+        uint32_t av[NK][4];
+#pragma unroll
+        for (int t = 0; t < NK; t++) ldsm_x4_t(av[t], afrag_t_addr(&sm.V[t][0][0], LDB, r0, 16 * ks));
+#pragma unroll
+        for (int np = 0; np < 4; np++) {
+          if (np >= ks) {  // Tv^T is zero above the diagonal block (m > i)
+            uint32_t bt[NW][4];
+#pragma unroll
+            for (int q = 0; q < NW; q++)
+              ldsm_x4(bt[q], bfrag_nk_addr(&sm.Tv[q][0][0], LDT, 16 * np, 16 * ks));
+#pragma unroll
+            for (int p = 0; p < PU::kCount; p++) {
+              mma16816(u[2 * np], av[PU::a(p)], bt[PU::b(p)][0], bt[PU::b(p)][1]);
+              mma16816(u[2 * np + 1], av[PU::a(p)], bt[PU::b(p)][2], bt[PU::b(p)][3]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int n = 0; n < 8; n++)
+#pragma unroll
+        for (int hf = 0; hf < 2; hf++)
+          *reinterpret_cast<float2*>(Up + (size_t)(r0 + gq + 8 * hf) * PK::LDU + 8 * n + 2 * tq) =
+              make_float2(u[n][2 * hf], u[n][2 * hf + 1]);
     }
   }
   // Keys (bf16 terms), decay vector and chunk decay into the pack.

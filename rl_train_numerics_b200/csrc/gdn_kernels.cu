@@ -6,9 +6,9 @@
 // within each chunk are filled in):
 //   k_chunk_table   one block: validates cu_seqlens, numbers the chunks
 //   k_prep          one block per (chunk, head): boundary prep of full chunks
-//   k_walk          one block per (sequence, head): serial walk over chunks
-//   k_fill          one block per (chunk, head): per-token recurrence from the
-//                   chunk's boundary state, all chunks in parallel
+//   k_walk          one block per (sequence, head): serial walk
+//   k_fill          persistent blocks over (chunk, head) items: per-token
+//                   recurrence from each chunk's boundary state
 // Decode (same section: the recurrent form re-synchronised every chunk):
 //   k_dec_step      one block per (row, head): one recurrence step
 //   k_bnd           one block per (row, head): resync of units whose chunk
@@ -18,6 +18,12 @@
 #include "gdn_layout.h"
 
 namespace gdn {
+
+// Workspace header words (int32).
+constexpr int kHdrError = 0;     // device error word (GDN_DEVERR_* bits)
+constexpr int kHdrChunks = 1;    // number of chunks of this call
+constexpr int kHdrValid = 2;     // 1 when this call's chunk table is valid
+constexpr int kHdrFillNext = 3;  // work counter of k_fill
 
 // ----------------------------------------------------------------------------
 // Chunk table
@@ -53,14 +59,15 @@ __global__ void __launch_bounds__(kTableThreads)
       run += x;
     }
     if (run > max_chunks) bad = 1;
-    hdr[1] = bad ? 0 : (int32_t)run;
+    hdr[kHdrChunks] = bad ? 0 : (int32_t)run;
+    hdr[kHdrFillNext] = 0;
     if (!bad) chunk_off[N] = (int32_t)run;
   }
   __syncthreads();
   if (bad) {
     if (tid == 0) {
-      atomicOr(&hdr[0], kErrCuSeqlens);
-      hdr[2] = 0;
+      atomicOr(&hdr[kHdrError], kErrCuSeqlens);
+      hdr[kHdrValid] = 0;
     }
     return;
   }
@@ -72,7 +79,7 @@ __global__ void __launch_bounds__(kTableThreads)
     for (long long i = 0; i < nc; i++) chunk_seq[off + i] = (int32_t)n;
     off += nc;
   }
-  if (tid == 0) hdr[2] = 1;
+  if (tid == 0) hdr[kHdrValid] = 1;
 }
 
 // ----------------------------------------------------------------------------
@@ -87,7 +94,7 @@ __global__ void __launch_bounds__(kBndThreads)
   extern __shared__ __align__(16) unsigned char smem_raw[];
   PrepSmem<D, IN>& sm = *reinterpret_cast<PrepSmem<D, IN>*>(smem_raw);
   const int c = blockIdx.x, h = blockIdx.y;
-  if (hdr[2] != 1 || c >= hdr[1]) return;
+  if (hdr[kHdrValid] != 1 || c >= hdr[kHdrChunks]) return;
   const int n = chunk_seq[c];
   const int ci = c - chunk_off[n];
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
@@ -95,24 +102,25 @@ __global__ void __launch_bounds__(kBndThreads)
   const int64_t t0 = (int64_t)cu[n] + (int64_t)ci * kChunk;
   const size_t tok = (size_t)t0 * H + h;
   prep_stage<D, IN>(sm, k + tok * D, v + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H);
-  __syncthreads();
   bnd_prep<D, IN>(sm, packs + ((size_t)c * H + h) * Pack<D, IN>::kBytes);
 }
 
 // ----------------------------------------------------------------------------
 // Pass 1b: serial walk over the full chunks of one (sequence, head, row block)
 // ----------------------------------------------------------------------------
-constexpr int kWalkWarps = 4;  // 64 state rows per block
+// One block per (sequence, head): D/16 warps, 16 state rows each.
+template <int D>
+constexpr int walk_threads() { return 32 * (D / 16); }
 
 template <int D, class IN>
 __device__ __forceinline__ void pack_fetch(char* dst, const char* src) {
   constexpr int N16 = (int)(Pack<D, IN>::kBytes / 16);
-  for (int e = threadIdx.x; e < N16; e += 32 * kWalkWarps) cp_async16(dst + 16 * e, src + 16 * e);
+  for (int e = threadIdx.x; e < N16; e += walk_threads<D>()) cp_async16(dst + 16 * e, src + 16 * e);
   cp_async_commit();
 }
 
 template <int D, class IN>
-__global__ void __launch_bounds__(32 * kWalkWarps, 1)
+__global__ void __launch_bounds__(walk_threads<D>(), 1)
     k_walk(const int32_t* __restrict__ cu, int H, const float* __restrict__ h0,
            const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
            const char* __restrict__ packs, float* __restrict__ bstate,
@@ -121,11 +129,11 @@ __global__ void __launch_bounds__(32 * kWalkWarps, 1)
   extern __shared__ __align__(16) unsigned char smem_raw[];
   char* const buf0 = reinterpret_cast<char*>(smem_raw);  // double buffer: buf0 + (c & 1) * kBytes
   const int n = blockIdx.x, h = blockIdx.y;
-  if (hdr[2] != 1) return;
+  if (hdr[kHdrValid] != 1) return;
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
   const int64_t nf = L / kChunk, nc = (L + kChunk - 1) / kChunk;
   const int64_t base = chunk_off[n];
-  const int r0 = blockIdx.z * 16 * kWalkWarps + 16 * (threadIdx.x >> 5);
+  const int r0 = 16 * (threadIdx.x >> 5);
   const size_t DD = (size_t)D * D;
   float sacc[D / 8][4];
   if (h0) sacc_load<D>(sacc, h0 + ((size_t)n * H + h) * DD, r0);
@@ -151,16 +159,31 @@ __global__ void __launch_bounds__(32 * kWalkWarps, 1)
 }
 
 // ----------------------------------------------------------------------------
-// Pass 2: per-token recurrence inside every chunk, from its boundary state
+// Pass 2: per-token recurrence inside every chunk, from its boundary state.
+// Persistent blocks take (chunk, head) items from a work counter; the next
+// item's q/k/v/beta/g are staged into shared memory (input dtype, cp.async)
+// while the current item runs, and its boundary state is prefetched to L2.
+// Which block runs an item does not change the item's bits.
 // ----------------------------------------------------------------------------
-template <int D>
-struct FillSmem {
-  float k[kChunk + 1][D];  // row kChunk stays zero (the "next key" of the last token)
-  float q[kChunk][D];
-  float v[kChunk][D];
-  float a[kChunk];
+constexpr int kFillThreads = 128;
+
+template <int D, class IN>
+struct FillStage {
+  IN k[kChunk + 1][D];  // row kChunk stays zero: the "next key" of the last token
+  IN q[kChunk][D];
+  IN v[kChunk][D];
+  float a[kChunk];  // log-decay g as staged, then exp(g)
   float b[kChunk];
 };
+
+__device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),
+               "l"(gmem), "r"(valid ? 16 : 0));
+}
+__device__ __forceinline__ void cp_async4_zfill(void* smem, const void* gmem, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(smem)),
+               "l"(gmem), "r"(valid ? 4 : 0));
+}
 
 template <int RT>
 __device__ __forceinline__ float pick(const float (&x)[RT], int l) {
@@ -171,80 +194,145 @@ __device__ __forceinline__ float pick(const float (&x)[RT], int l) {
   return val;
 }
 
+struct FillItem {
+  int c, h, n, ci, len;
+  int64_t t0, L;
+};
+
+__device__ __forceinline__ FillItem fill_item(int item, int H, const int32_t* cu,
+                                              const int32_t* chunk_off,
+                                              const int32_t* chunk_seq) {
+  FillItem it;
+  it.c = item / H;
+  it.h = item - it.c * H;
+  it.n = chunk_seq[it.c];
+  it.ci = it.c - chunk_off[it.n];
+  it.L = (int64_t)cu[it.n + 1] - cu[it.n];
+  it.t0 = (int64_t)cu[it.n] + (int64_t)it.ci * kChunk;
+  it.len = (int)min((int64_t)kChunk, it.L - (int64_t)it.ci * kChunk);
+  return it;
+}
+
+// Issue the cp.async copies of one item's inputs into a stage (rows past the
+// item's length are zero-filled without reading memory) as one commit group.
+template <int D, class IN>
+__device__ __forceinline__ void fill_stage_issue(FillStage<D, IN>& st, const FillItem& it,
+                                                 const IN* q, const IN* k, const IN* v,
+                                                 const float* beta, const float* g, int H) {
+  constexpr int P = (int)(D * sizeof(IN) / 16);  // 16-byte pieces per row
+  constexpr int E = (int)(16 / sizeof(IN));      // elements per piece
+  const size_t ld = (size_t)H * D;
+  const size_t tb = (size_t)it.t0 * H + it.h;
+  const IN* kb = k + tb * D;
+  const IN* qb = q + tb * D;
+  const IN* vb = v + tb * D;
+  for (int e = threadIdx.x; e < (3 * kChunk + 1) * P; e += kFillThreads) {
+    const int row = e / P, pc = (e % P) * E;
+    if (row <= kChunk) {
+      const bool ok = row < it.len;
+      cp_async16_zfill(&st.k[row][pc], kb + (size_t)(ok ? row : 0) * ld + pc, ok);
+    } else if (row <= 2 * kChunk) {
+      const int r = row - kChunk - 1;
+      const bool ok = r < it.len;
+      cp_async16_zfill(&st.q[r][pc], qb + (size_t)(ok ? r : 0) * ld + pc, ok);
+    } else {
+      const int r = row - 2 * kChunk - 1;
+      const bool ok = r < it.len;
+      cp_async16_zfill(&st.v[r][pc], vb + (size_t)(ok ? r : 0) * ld + pc, ok);
+    }
+  }
+  for (int i = threadIdx.x; i < 2 * kChunk; i += kFillThreads) {
+    const int r = i & (kChunk - 1);
+    const bool ok = r < it.len;
+    const float* src = (i < kChunk ? g : beta) + tb + (size_t)(ok ? r : 0) * H;
+    cp_async4_zfill(i < kChunk ? &st.a[r] : &st.b[r], src, ok);
+  }
+  cp_async_commit();
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes));
+}
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
 template <int D, class IN, class OUT>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(kFillThreads, 2)
     k_fill(const IN* __restrict__ q, const IN* __restrict__ k, const IN* __restrict__ v,
            const float* __restrict__ beta, const float* __restrict__ g,
-           const int32_t* __restrict__ cu, int H, float scale, const int32_t* __restrict__ hdr,
+           const int32_t* __restrict__ cu, int H, float scale, int32_t* __restrict__ hdr,
            const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
            const float* __restrict__ bstate, OUT* __restrict__ o,
            float* __restrict__ s_run_final) {
-  constexpr int RT = D / 32, M4 = D / 16, G4 = D / 4;
+  constexpr int RT = D / 32, M4 = D / 16;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  FillSmem<D>& sm = *reinterpret_cast<FillSmem<D>*>(smem_raw);
-  const int c = blockIdx.x, h = blockIdx.y;
-  if (hdr[2] != 1 || c >= hdr[1]) return;
-  const int n = chunk_seq[c];
-  const int ci = c - chunk_off[n];
-  const int64_t L = (int64_t)cu[n + 1] - cu[n];
-  const int64_t t0 = (int64_t)cu[n] + (int64_t)ci * kChunk;
-  const int len = (int)min((int64_t)kChunk, L - (int64_t)ci * kChunk);
+  FillStage<D, IN>* stages = reinterpret_cast<FillStage<D, IN>*>(smem_raw);
+  __shared__ int sh_item;
+  if (hdr[kHdrValid] != 1) return;
+  const int n_items = hdr[kHdrChunks] * H;
   const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * RT;
+  const size_t DD = (size_t)D * D;
 
-  for (int e = tid; e < (kChunk + 1) * G4; e += 128) {
-    const int i = e / G4, cc = (e % G4) * 4;
-    float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), qq = kk, vv = kk;
-    if (i < len) {
-      const size_t off = ((size_t)(t0 + i) * H + h) * D + cc;
-      kk = ld4(k + off);
-      qq = ld4(q + off);
-      vv = ld4(v + off);
-    }
-    *reinterpret_cast<float4*>(&sm.k[i][cc]) = kk;
-    if (i < kChunk) {
-      *reinterpret_cast<float4*>(&sm.q[i][cc]) = qq;
-      *reinterpret_cast<float4*>(&sm.v[i][cc]) = vv;
-    }
-  }
-  for (int i = tid; i < kChunk; i += 128) {
-    float a = 0.f, b = 0.f;
-    if (i < len) {
-      const size_t tok = (size_t)(t0 + i) * H + h;
-      a = step_decay(g[tok]);
-      b = beta[tok];
-    }
-    sm.a[i] = a;
-    sm.b[i] = b;
-  }
-  Slice<RT, M4> S;
-  slice_load<RT, M4>(S, bstate + ((size_t)c * H + h) * D * D, D, r0, l);
+  if (tid == 0) sh_item = atomicAdd(&hdr[kHdrFillNext], 1);
   __syncthreads();
-
-  float p[RT];
-  slice_dot<RT, M4>(S, [&](int m) { return ld4(&sm.k[0][group_col(l, m)]); }, p);
-#pragma unroll
-  for (int i = 0; i < RT; i++) p[i] = quad_sum(p[i]);
-
-  for (int t = 0; t < len; t++) {
-    const float a = sm.a[t], b = sm.b[t];
-    float u[RT], oacc[RT], pacc[RT];
-#pragma unroll
-    for (int i = 0; i < RT; i++) u[i] = step_u(a, b, p[i], sm.v[t][r0 + i]);
-    slice_update<true, RT, M4>(
-        S, a, u, [&](int m) { return ld4(&sm.k[t][group_col(l, m)]); },
-        [&](int m) { return ld4(&sm.q[t][group_col(l, m)]); },
-        [&](int m) { return ld4(&sm.k[t + 1][group_col(l, m)]); }, oacc, pacc);
-    float ov[RT];
-#pragma unroll
-    for (int i = 0; i < RT; i++) {
-      ov[i] = __fmul_rn(scale, quad_sum(oacc[i]));
-      p[i] = quad_sum(pacc[i]);
-    }
-    if (l < RT) st1(o + ((size_t)(t0 + t) * H + h) * D + r0 + l, pick<RT>(ov, l));
+  int item = sh_item;
+  int bi = 0;
+  FillItem cur{};
+  if (item < n_items) {
+    cur = fill_item(item, H, cu, chunk_off, chunk_seq);
+    fill_stage_issue<D, IN>(stages[0], cur, q, k, v, beta, g, H);
   }
-  const int64_t nc = (L + kChunk - 1) / kChunk;
-  if (s_run_final && ci == nc - 1 && (L % kChunk) != 0)
-    slice_store<RT, M4>(S, s_run_final + ((size_t)n * H + h) * D * D, D, r0, l);
+  while (item < n_items) {
+    __syncthreads();  // every thread is done with stage bi^1 and has read sh_item
+    if (tid == 0) sh_item = atomicAdd(&hdr[kHdrFillNext], 1);
+    __syncthreads();
+    const int next = sh_item;
+    FillItem nxt{};
+    if (next < n_items) {
+      nxt = fill_item(next, H, cu, chunk_off, chunk_seq);
+      fill_stage_issue<D, IN>(stages[bi ^ 1], nxt, q, k, v, beta, g, H);
+      if (tid == 0) prefetch_l2(bstate + ((size_t)nxt.c * H + nxt.h) * DD, (uint32_t)(DD * 4));
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    FillStage<D, IN>& st = stages[bi];
+    for (int i = tid; i < cur.len; i += kFillThreads) st.a[i] = step_decay(st.a[i]);
+    Slice<RT, M4> S;
+    slice_load<RT, M4>(S, bstate + ((size_t)cur.c * H + cur.h) * DD, D, r0, l);
+    __syncthreads();
+
+    float p[RT];
+    slice_dot<RT, M4>(S, [&](int m) { return sld4(&st.k[0][group_col(l, m)]); }, p);
+#pragma unroll
+    for (int i = 0; i < RT; i++) p[i] = quad_sum(p[i]);
+    OUT* ob = o + ((size_t)cur.t0 * H + cur.h) * D + r0 + l;
+    for (int t = 0; t < cur.len; t++) {
+      const float a = st.a[t], b = st.b[t];
+      float u[RT], oacc[RT], pacc[RT];
+#pragma unroll
+      for (int i = 0; i < RT; i++) u[i] = step_u(a, b, p[i], to_f(st.v[t][r0 + i]));
+      slice_update<true, RT, M4>(
+          S, a, u, [&](int m) { return sld4(&st.k[t][group_col(l, m)]); },
+          [&](int m) { return sld4(&st.q[t][group_col(l, m)]); },
+          [&](int m) { return sld4(&st.k[t + 1][group_col(l, m)]); }, oacc, pacc);
+      float ov[RT];
+#pragma unroll
+      for (int i = 0; i < RT; i++) {
+        ov[i] = __fmul_rn(scale, quad_sum(oacc[i]));
+        p[i] = quad_sum(pacc[i]);
+      }
+      if (l < RT) st1(ob + (size_t)t * H * D, pick<RT>(ov, l));
+    }
+    const int64_t nc = (cur.L + kChunk - 1) / kChunk;
+    if (s_run_final && cur.ci == nc - 1 && (cur.L % kChunk) != 0)
+      slice_store<RT, M4>(S, s_run_final + ((size_t)cur.n * H + cur.h) * DD, D, r0, l);
+    item = next;
+    cur = nxt;
+    bi ^= 1;
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -347,7 +435,6 @@ __global__ void __launch_bounds__(kBndThreads)
   const size_t DD = (size_t)D * D;
   prep_stage<D, IN>(sm.prep, kb + unit * kChunk * D, vb + unit * kChunk * D, (size_t)D,
                     bb + unit * kChunk, gb + unit * kChunk, 1);
-  __syncthreads();
   bnd_prep<D, IN>(sm.prep, sm.pack);
   __syncthreads();
   const int warp = threadIdx.x >> 5;
@@ -411,11 +498,22 @@ static cudaError_t set_smem(KernelT kern, size_t bytes) {
   return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-#define GDN_TRY(expr)                    \
-  do {                                   \
-    cudaError_t e_ = (expr);             \
-    if (e_ != cudaSuccess) return e_;    \
+#define GDN_TRY(expr)                 \
+  do {                                \
+    cudaError_t e_ = (expr);          \
+    if (e_ != cudaSuccess) return e_; \
   } while (0)
+
+// Persistent grid size of a kernel: resident blocks per SM x SMs.
+template <class KernelT>
+static cudaError_t persistent_grid(KernelT kern, int threads, size_t smem, int* grid) {
+  int dev = 0, sms = 0, per_sm = 0;
+  GDN_TRY(cudaGetDevice(&dev));
+  GDN_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  GDN_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem));
+  *grid = (per_sm > 0 ? per_sm : 1) * sms;
+  return cudaSuccess;
+}
 
 template <int D, class IN, class OUT>
 static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
@@ -452,19 +550,22 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     auto kern = k_walk<D, IN>;
     const size_t sm = 2 * Pack<D, IN>::kBytes;
     GDN_TRY(set_smem(kern, sm));
-    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H, D / (16 * kWalkWarps)), 32 * kWalkWarps, sm,
-           st>>>(a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final,
-                 a.s_bnd_final);
+    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), walk_threads<D>(), sm, st>>>(
+        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final, a.s_bnd_final);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(3));
   {
     auto kern = k_fill<D, IN, OUT>;
-    const size_t sm = sizeof(FillSmem<D>);
+    const size_t sm = 2 * sizeof(FillStage<D, IN>);
     GDN_TRY(set_smem(kern, sm));
-    kern<<<gchunks, 128, sm, st>>>(q, k, v, a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
-                                   chunk_off, chunk_seq, bstate, static_cast<OUT*>(a.o),
-                                   a.s_run_final);
+    int grid = 0;
+    GDN_TRY(persistent_grid(kern, kFillThreads, sm, &grid));
+    const int64_t items = L.max_chunks * a.H;
+    if ((int64_t)grid > items) grid = (int)items;
+    kern<<<grid, kFillThreads, sm, st>>>(q, k, v, a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
+                                         chunk_off, chunk_seq, bstate, static_cast<OUT*>(a.o),
+                                         a.s_run_final);
     GDN_TRY(cudaGetLastError());
   }
   return mark(4);
@@ -509,38 +610,38 @@ static cudaError_t boundary_impl(const BndArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+using bf16 = __nv_bfloat16;
+
 cudaError_t launch_forward(const FwdArgs& a, cudaStream_t st) {
-  using bf = __nv_bfloat16;
   if (a.D == 64) {
-    if (a.in_bf16) return a.out_bf16 ? forward_impl<64, bf, bf>(a, st) : forward_impl<64, bf, float>(a, st);
-    return a.out_bf16 ? forward_impl<64, float, bf>(a, st) : forward_impl<64, float, float>(a, st);
+    if (a.in_bf16)
+      return a.out_bf16 ? forward_impl<64, bf16, bf16>(a, st) : forward_impl<64, bf16, float>(a, st);
+    return a.out_bf16 ? forward_impl<64, float, bf16>(a, st) : forward_impl<64, float, float>(a, st);
   }
   if (!a.in_bf16) return cudaErrorNotSupported;  // fp32 inputs: d = 64 only
-  return a.out_bf16 ? forward_impl<128, bf, bf>(a, st) : forward_impl<128, bf, float>(a, st);
+  return a.out_bf16 ? forward_impl<128, bf16, bf16>(a, st) : forward_impl<128, bf16, float>(a, st);
 }
 
 cudaError_t launch_decode_step(const DecArgs& a, cudaStream_t st) {
-  using bf = __nv_bfloat16;
   if (a.D == 64) {
-    if (a.in_bf16) return a.out_bf16 ? decode_impl<64, bf, bf>(a, st) : decode_impl<64, bf, float>(a, st);
-    return a.out_bf16 ? decode_impl<64, float, bf>(a, st) : decode_impl<64, float, float>(a, st);
+    if (a.in_bf16)
+      return a.out_bf16 ? decode_impl<64, bf16, bf16>(a, st) : decode_impl<64, bf16, float>(a, st);
+    return a.out_bf16 ? decode_impl<64, float, bf16>(a, st) : decode_impl<64, float, float>(a, st);
   }
   if (!a.in_bf16) return cudaErrorNotSupported;  // fp32 inputs: d = 64 only
-  return a.out_bf16 ? decode_impl<128, bf, bf>(a, st) : decode_impl<128, bf, float>(a, st);
+  return a.out_bf16 ? decode_impl<128, bf16, bf16>(a, st) : decode_impl<128, bf16, float>(a, st);
 }
 
 cudaError_t launch_handoff(const HandoffArgs& a, cudaStream_t st) {
-  using bf = __nv_bfloat16;
-  if (a.D == 64) return a.in_bf16 ? handoff_impl<64, bf>(a, st) : handoff_impl<64, float>(a, st);
+  if (a.D == 64) return a.in_bf16 ? handoff_impl<64, bf16>(a, st) : handoff_impl<64, float>(a, st);
   if (!a.in_bf16) return cudaErrorNotSupported;  // fp32 inputs: d = 64 only
-  return handoff_impl<128, bf>(a, st);
+  return handoff_impl<128, bf16>(a, st);
 }
 
 cudaError_t launch_chunk_boundary(const BndArgs& a, cudaStream_t st) {
-  using bf = __nv_bfloat16;
-  if (a.D == 64) return a.in_bf16 ? boundary_impl<64, bf>(a, st) : boundary_impl<64, float>(a, st);
+  if (a.D == 64) return a.in_bf16 ? boundary_impl<64, bf16>(a, st) : boundary_impl<64, float>(a, st);
   if (!a.in_bf16) return cudaErrorNotSupported;  // fp32 inputs: d = 64 only
-  return boundary_impl<128, bf>(a, st);
+  return boundary_impl<128, bf16>(a, st);
 }
 
 }  // namespace gdn
