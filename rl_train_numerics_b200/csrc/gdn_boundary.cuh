@@ -12,24 +12,24 @@
 //   G_i   = g_1 + ... + g_i                 (cumulative log-decay, in double)
 //   A_ij  = beta_i exp(G_i - G_j) (k_i . k_j)       j < i
 //   T     = (I + A)^{-1}                    unit lower triangular
-//   W     = T diag(beta_m exp(G_m)) K       C x d_k
-//   U~    = T diag(beta_m) V                C x d_v
-//   U     = U~ - W S0^T                     C x d_v
+//   Tb    = T diag(beta_m exp(G_m)),  Tv = T diag(beta_m)
+//   U     = Tv V - Tb (K S0^T)              C x d_v
 //   S_C   = exp(G_C) S0 + U^T diag(exp(G_C - G_i)) K
 //
-// "Prep" (everything but the last two lines) depends only on the chunk's
-// tokens and runs for all chunks in parallel; the "walk" (last two lines) is
-// the serial step from one boundary state to the next.  The forward's first
-// pass and the decode resync call exactly these device functions, so boundary
-// states are bitwise identical wherever they are computed.
+// "Prep" (G, A, T, Tb, Tv) depends only on the chunk's tokens and runs for all
+// chunks in parallel; the "walk" (last two lines) is the serial step from one
+// boundary state to the next.  The forward's first pass and the decode resync
+// call exactly these device functions, so boundary states are bitwise
+// identical wherever they are computed.
 //
 // Contractions run on the tensor cores (mma.sync m16n8k16, bf16 operands,
 // fp32 accumulation).  Operands that are not exactly bf16 (the fp32 state,
-// T, the intermediate U, and fp32 inputs) are split exactly into bf16 terms
-// (gdn_mma.cuh); the products of all term pairs down to the finer split's
-// precision are accumulated in a fixed order, which keeps the boundary at
-// about fp32 accuracy: two terms (16 significant bits) for bf16 inputs, whose
-// K and V are exact in bf16, and three terms (24 bits) for fp32 inputs.
+// Tb, Tv, the intermediate K S0^T and U, and fp32 inputs) are split exactly
+// into bf16 terms (gdn_mma.cuh); the products of all term pairs down to the
+// finer split's precision are accumulated in a fixed order.  That keeps the
+// boundary at about fp32 accuracy: two terms (16 significant bits) for bf16
+// inputs, whose K and V are exact in bf16, and three terms (24 bits) for fp32
+// inputs.
 //
 // Fixed evaluation order (part of the rounding schedule):
 //   G        double, ascending i
@@ -37,10 +37,11 @@
 //   A_ij     (beta_i * expf((float)(G_i - G_j))) * P_ij
 //   T        right-looking substitution: T_ij accumulates -A_im T_mj over
 //            m = j .. i-1 (one fma each)
-//   W, U~    (T_im * (beta_m expf(G_m))) and (T_im * beta_m), split, then
-//            k16 steps m ascending up to the diagonal block (U~ is formed
-//            transposed, as V^T Tv^T)
-//   U        Ud_i = exp(G_C - G_i) * (U~_ir - (S0 W^T)_ri)
+//   Tb, Tv   T_im * (beta_m expf(G_m)) and T_im * beta_m, then split
+//   Y        (S0 K^T): k16 steps over the key channel ascending
+//   U^T      one accumulator: per k16 step over m (ascending, up to the
+//            diagonal block), first + V^T Tv^T then - Y Tb^T
+//   Ud       exp(G_C - G_i) * U^T
 //   S_C      accumulator starts at exp(G_C) * S0, then k16 steps over i
 #pragma once
 
@@ -56,8 +57,8 @@ template <class IN>
 struct Splits;
 template <>
 struct Splits<__nv_bfloat16> {
-  static constexpr int S = 2;  // state and U (walk A operands)
-  static constexpr int W = 2;  // T-derived operands and W
+  static constexpr int S = 2;  // state, K S0^T, U (walk A operands)
+  static constexpr int W = 2;  // Tb, Tv
   static constexpr int K = 1;  // keys and values
 };
 template <>
@@ -69,99 +70,76 @@ struct Splits<float> {
 
 constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// The walk pack: everything the walk needs from one (chunk, head), in the
-// padded shared-memory layout (bank-conflict-free ldmatrix rows).
+// What the walk needs from the prep of one (chunk, head): the walk pack.  It
+// is copied as raw bytes (global <-> shared), so its layout is the shared
+// memory layout: bf16 planes with padded rows (bank-conflict-free ldmatrix).
 template <int D, class IN>
-struct Pack {
-  static constexpr int NW = Splits<IN>::W, NK = Splits<IN>::K;
-  static constexpr int LDB = D + 8;       // bf16 row stride of W and K planes
-  static constexpr int LDU = kChunk + 8;  // fp32 row stride of U~^T
-  static constexpr size_t kW = 0;                                        // NW x [C][LDB] bf16
-  static constexpr size_t kK = kW + (size_t)NW * kChunk * LDB * 2;       // NK x [C][LDB] bf16
-  static constexpr size_t kU = kK + (size_t)NK * kChunk * LDB * 2;       // [D][LDU] fp32
-  static constexpr size_t kDvec = kU + (size_t)D * LDU * 4;              // [C] fp32
-  static constexpr size_t kGamma = kDvec + (size_t)kChunk * 4;           // fp32
-  static constexpr size_t kBytes = round_up(kGamma + 16, 128);
-
-  static __device__ __forceinline__ __nv_bfloat16* W(char* p, int t) {
-    return reinterpret_cast<__nv_bfloat16*>(p + kW) + (size_t)t * kChunk * LDB;
-  }
-  static __device__ __forceinline__ __nv_bfloat16* K(char* p, int t) {
-    return reinterpret_cast<__nv_bfloat16*>(p + kK) + (size_t)t * kChunk * LDB;
-  }
-  static __device__ __forceinline__ float* U(char* p) { return reinterpret_cast<float*>(p + kU); }
-  static __device__ __forceinline__ float* dvec(char* p) {
-    return reinterpret_cast<float*>(p + kDvec);
-  }
-  static __device__ __forceinline__ float* gamma(char* p) {
-    return reinterpret_cast<float*>(p + kGamma);
-  }
+struct PackHead {
+  static constexpr int NW = Splits<IN>::W;
+  static constexpr int LDT = kChunk + 8;
+  __nv_bfloat16 Tb[NW][kChunk][LDT];
+  __nv_bfloat16 Tv[NW][kChunk][LDT];
+  float dvec[kChunk];
+  float gamma[4];  // [0] = exp(G_C)
 };
 
-// Shared memory of the prep.  A is stored packed (strictly lower triangle,
-// row-major: element (i, j), j < i, at i(i-1)/2 + j).
+// Keys and values of one chunk as bf16 term planes (padded rows).
+template <int D, class IN>
+struct KVPlanes {
+  static constexpr int NK = Splits<IN>::K;
+  static constexpr int LDB = D + 8;
+  __nv_bfloat16 K[NK][kChunk][LDB];
+  __nv_bfloat16 V[NK][kChunk][LDB];
+};
+
+template <int D, class IN>
+constexpr size_t pack_size() {
+  return round_up(sizeof(PackHead<D, IN>), 128);
+}
+
+// Shared memory of the prep.  AT holds A transposed with padded columns:
+// AT[m][i] = A_im for i > m (zero elsewhere), so a column of A is contiguous.
 template <int D, class IN>
 struct PrepSmem {
   static constexpr int NW = Splits<IN>::W, NK = Splits<IN>::K;
-  static constexpr int LDB = D + 8, LDT = kChunk + 8;
+  static constexpr int LDB = D + 8;
+  PackHead<D, IN> head;
   __nv_bfloat16 K[NK][kChunk][LDB];
-  __nv_bfloat16 V[NK][kChunk][LDB];
-  __nv_bfloat16 Tb[NW][kChunk][LDT];
-  __nv_bfloat16 Tv[NW][kChunk][LDT];
-  float A[kChunk * (kChunk - 1) / 2];
+  float AT[kChunk][kChunk];
   double G[kChunk];
   float beta[kChunk];
   float g[kChunk];
   float bg[kChunk];
-  float dvec[kChunk];
-  float gammaC;
 };
 
-__device__ __forceinline__ constexpr int tri(int i, int j) { return i * (i - 1) / 2 + j; }
-
-// Stage one chunk's k, v (rows at stride `ld` elements), beta, g (stride ldbg)
-// into the prep's shared memory.  bf16 inputs are copied as is (cp.async);
-// fp32 inputs are split into three bf16 terms.  Ends with the copies landed
-// and a block barrier.
+// Stage the rows of a [C][D] block (row stride ld elements) into bf16 term
+// planes: bf16 inputs are copied with cp.async (the caller commits and waits),
+// fp32 inputs are split into three bf16 terms with plain loads and stores.
 template <int D, class IN>
-__device__ __forceinline__ void prep_stage(PrepSmem<D, IN>& sm, const IN* k, const IN* v,
-                                           size_t ld, const float* bsrc, const float* gsrc,
-                                           size_t ldbg) {
+__device__ __forceinline__ void stage_planes(__nv_bfloat16 (*dst)[kChunk][D + 8], const IN* src,
+                                             size_t ld, int nthreads) {
   constexpr int NK = Splits<IN>::K;
   if constexpr (NK == 1) {
     constexpr int P = D / 8;  // 16-byte pieces per row
-    for (int e = threadIdx.x; e < 2 * kChunk * P; e += kBndThreads) {
-      const int r = (e / P) % kChunk, c = (e % P) * 8;
-      if (e < kChunk * P) cp_async16(&sm.K[0][r][c], k + (size_t)r * ld + c);
-      else cp_async16(&sm.V[0][r][c], v + (size_t)r * ld + c);
+    for (int e = threadIdx.x; e < kChunk * P; e += nthreads) {
+      const int r = e / P, c = (e % P) * 8;
+      cp_async16(&dst[0][r][c], src + (size_t)r * ld + c);
     }
-    cp_async_commit();
   } else {
     constexpr int G4 = D / 4;
-    for (int e = threadIdx.x; e < kChunk * G4; e += kBndThreads) {
-      const int i = e / G4, c = (e % G4) * 4;
-      const float4 kk = ld4(k + i * ld + c);
-      const float4 vv = ld4(v + i * ld + c);
-      const float kx[4] = {kk.x, kk.y, kk.z, kk.w}, vx[4] = {vv.x, vv.y, vv.z, vv.w};
+    for (int e = threadIdx.x; e < kChunk * G4; e += nthreads) {
+      const int r = e / G4, c = (e % G4) * 4;
+      const float4 x4 = ld4(src + (size_t)r * ld + c);
+      const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
       for (int q = 0; q < 4; q++) {
-        __nv_bfloat16 ks[NK], vs[NK];
-        split_bf16<NK>(kx[q], ks);
-        split_bf16<NK>(vx[q], vs);
+        __nv_bfloat16 s[NK];
+        split_bf16<NK>(xs[q], s);
 #pragma unroll
-        for (int t = 0; t < NK; t++) {
-          sm.K[t][i][c + q] = ks[t];
-          sm.V[t][i][c + q] = vs[t];
-        }
+        for (int t = 0; t < NK; t++) dst[t][r][c + q] = s[t];
       }
     }
   }
-  for (int i = threadIdx.x; i < kChunk; i += kBndThreads) {
-    sm.beta[i] = bsrc[i * ldbg];
-    sm.g[i] = gsrc[i * ldbg];
-  }
-  if constexpr (NK == 1) cp_async_wait<0>();
-  __syncthreads();
 }
 
 // ldmatrix address of the A fragment (x4) of rows r0.., columns c0.. in a
@@ -190,19 +168,31 @@ __device__ __forceinline__ const __nv_bfloat16* bfrag_kn_addr(const __nv_bfloat1
   return base + (size_t)(k0 + (mi & 1) * 8 + (lane & 7)) * ld + n0 + (mi >> 1) * 8;
 }
 
-// Prep of one chunk: sm.K, sm.V, sm.beta, sm.g staged (prep_stage) -> the
-// walk pack at `pack` (global or shared; generic addressing).  All
-// kBndThreads threads.
+// Stage one chunk for the prep: keys (rows at stride ld), beta and g
+// (stride ldbg).  Ends with the data landed and a block barrier.
 template <int D, class IN>
-__device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
-  using PK = Pack<D, IN>;
+__device__ __forceinline__ void prep_stage(PrepSmem<D, IN>& sm, const IN* k, size_t ld,
+                                           const float* bsrc, const float* gsrc, size_t ldbg) {
+  stage_planes<D, IN>(sm.K, k, ld, kBndThreads);
+  cp_async_commit();
+  for (int i = threadIdx.x; i < kChunk; i += kBndThreads) {
+    sm.beta[i] = bsrc[i * ldbg];
+    sm.g[i] = gsrc[i * ldbg];
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+}
+
+// Prep of one chunk: sm.K, sm.beta, sm.g staged -> sm.head (Tb, Tv, dvec,
+// gamma).  All kBndThreads threads; ends with a block barrier.
+template <int D, class IN>
+__device__ void bnd_prep(PrepSmem<D, IN>& sm) {
   constexpr int NW = Splits<IN>::W, NK = Splits<IN>::K;
-  constexpr int LDB = PrepSmem<D, IN>::LDB, LDT = PrepSmem<D, IN>::LDT;
+  constexpr int LDB = PrepSmem<D, IN>::LDB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
 
   // P = K K^T on the tensor cores; warp w owns rows 16w..16w+15 (m-tile w)
-  // and the n8 tiles that reach below the diagonal.  Warp 0, which has the
-  // fewest tiles, then accumulates G.
+  // and the n8 tiles that reach below the diagonal.
   float acc[8][4];
   {
     using PP = SplitPairs<NK, NK>;
@@ -239,6 +229,8 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
       sm.G[i] = s;
     }
   }
+  for (int e = tid; e < kChunk * kChunk / 4; e += kBndThreads)
+    reinterpret_cast<float4*>(&sm.AT[0][0])[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
   {
     const int m0 = 16 * warp;
@@ -250,7 +242,7 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
           const int i = m0 + gq + (e >> 1) * 8, j = 8 * n + 2 * tq + (e & 1);
           if (j < i) {
             const float decay = expf(__double2float_rn(sm.G[i] - sm.G[j]));
-            sm.A[tri(i, j)] = __fmul_rn(__fmul_rn(sm.beta[i], decay), acc[n][e]);
+            sm.AT[j][i] = __fmul_rn(__fmul_rn(sm.beta[i], decay), acc[n][e]);
           }
         }
       }
@@ -258,9 +250,12 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
   }
   for (int i = tid; i < kChunk; i += kBndThreads) {
     sm.bg[i] = __fmul_rn(sm.beta[i], expf(__double2float_rn(sm.G[i])));
-    sm.dvec[i] = expf(__double2float_rn(sm.G[kChunk - 1] - sm.G[i]));
+    sm.head.dvec[i] = expf(__double2float_rn(sm.G[kChunk - 1] - sm.G[i]));
   }
-  if (tid == 0) sm.gammaC = expf(__double2float_rn(sm.G[kChunk - 1]));
+  if (tid == 0) {
+    sm.head.gamma[0] = expf(__double2float_rn(sm.G[kChunk - 1]));
+    sm.head.gamma[1] = sm.head.gamma[2] = sm.head.gamma[3] = 0.f;
+  }
   __syncthreads();
 
   // T = (I + A)^{-1}, column j held in registers by thread j: right-looking
@@ -275,8 +270,15 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
 #pragma unroll
     for (int m = 0; m < kChunk - 1; m++) {
       const float tm = t[m];
+      const float* col = &sm.AT[m][0];
 #pragma unroll
-      for (int i = m + 1; i < kChunk; i++) t[i] = __fmaf_rn(-sm.A[tri(i, m)], tm, t[i]);
+      for (int i4 = (m + 1) & ~3; i4 < kChunk; i4 += 4) {
+        const float4 a4 = *reinterpret_cast<const float4*>(col + i4);
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int q = 0; q < 4; q++)
+          if (i4 + q > m) t[i4 + q] = __fmaf_rn(-av[q], tm, t[i4 + q]);
+      }
     }
     const float bgj = sm.bg[j], bj = sm.beta[j];
 #pragma unroll
@@ -286,104 +288,12 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, char* pack) {
       split_bf16<NW>(__fmul_rn(t[i], bj), sv);
 #pragma unroll
       for (int q = 0; q < NW; q++) {
-        sm.Tb[q][i][j] = sb[q];
-        sm.Tv[q][i][j] = sv[q];
+        sm.head.Tb[q][i][j] = sb[q];
+        sm.head.Tv[q][i][j] = sv[q];
       }
     }
   }
   __syncthreads();
-
-  // W = Tb K (rows i; warp w owns columns [D/4 w, D/4 (w+1))), and
-  // U~^T = V^T Tv^T (rows c; warp w owns rows [D/4 w, D/4 (w+1))).
-  {
-    using PW = SplitPairs<NW, NK>;
-    constexpr int NT = D / 32;  // n8 tiles of W per warp (D/4 columns)
-    const int c0 = (D / 4) * warp;
-#pragma unroll 1
-    for (int mt = 0; mt < 4; mt++) {
-      float w[NT][4];
-#pragma unroll
-      for (int n = 0; n < NT; n++)
-#pragma unroll
-        for (int e = 0; e < 4; e++) w[n][e] = 0.f;
-      for (int ks = 0; ks <= mt; ks++) {
-        uint32_t ab[NW][4];
-#pragma unroll
-        for (int q = 0; q < NW; q++) ldsm_x4(ab[q], afrag_addr(&sm.Tb[q][0][0], LDT, 16 * mt, 16 * ks));
-#pragma unroll
-        for (int np = 0; np < NT / 2; np++) {
-          uint32_t bk[NK][4];
-#pragma unroll
-          for (int t = 0; t < NK; t++)
-            ldsm_x4_t(bk[t], bfrag_kn_addr(&sm.K[t][0][0], LDB, 16 * ks, c0 + 16 * np));
-#pragma unroll
-          for (int p = 0; p < PW::kCount; p++) {
-            mma16816(w[2 * np], ab[PW::a(p)], bk[PW::b(p)][0], bk[PW::b(p)][1]);
-            mma16816(w[2 * np + 1], ab[PW::a(p)], bk[PW::b(p)][2], bk[PW::b(p)][3]);
-          }
-        }
-      }
-#pragma unroll
-      for (int n = 0; n < NT; n++) {
-#pragma unroll
-        for (int hf = 0; hf < 2; hf++) {
-          const int i = 16 * mt + gq + 8 * hf, c = c0 + 8 * n + 2 * tq;
-          __nv_bfloat16 s0[NW], s1[NW];
-          split_bf16<NW>(w[n][2 * hf], s0);
-          split_bf16<NW>(w[n][2 * hf + 1], s1);
-#pragma unroll
-          for (int q = 0; q < NW; q++)
-            *reinterpret_cast<uint32_t*>(PK::W(pack, q) + (size_t)i * PK::LDB + c) =
-                pack_bf16(s0[q], s1[q]);
-        }
-      }
-    }
-    using PU = SplitPairs<NK, NW>;
-    float* Up = PK::U(pack);
-#pragma unroll 1
-    for (int mt = 0; mt < D / 64; mt++) {
-      const int r0 = c0 + 16 * mt;  // rows c of U~^T
-      float u[8][4];
-#pragma unroll
-      for (int n = 0; n < 8; n++)
-#pragma unroll
-        for (int e = 0; e < 4; e++) u[n][e] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < 4; ks++) {
-        uint32_t av[NK][4];
-#pragma unroll
-        for (int t = 0; t < NK; t++) ldsm_x4_t(av[t], afrag_t_addr(&sm.V[t][0][0], LDB, r0, 16 * ks));
-#pragma unroll
-        for (int np = 0; np < 4; np++) {
-          if (np >= ks) {  // Tv^T is zero above the diagonal block (m > i)
-            uint32_t bt[NW][4];
-#pragma unroll
-            for (int q = 0; q < NW; q++)
-              ldsm_x4(bt[q], bfrag_nk_addr(&sm.Tv[q][0][0], LDT, 16 * np, 16 * ks));
-#pragma unroll
-            for (int p = 0; p < PU::kCount; p++) {
-              mma16816(u[2 * np], av[PU::a(p)], bt[PU::b(p)][0], bt[PU::b(p)][1]);
-              mma16816(u[2 * np + 1], av[PU::a(p)], bt[PU::b(p)][2], bt[PU::b(p)][3]);
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int n = 0; n < 8; n++)
-#pragma unroll
-        for (int hf = 0; hf < 2; hf++)
-          *reinterpret_cast<float2*>(Up + (size_t)(r0 + gq + 8 * hf) * PK::LDU + 8 * n + 2 * tq) =
-              make_float2(u[n][2 * hf], u[n][2 * hf + 1]);
-    }
-  }
-  // Keys (bf16 terms), decay vector and chunk decay into the pack.
-  for (int e = tid; e < NK * kChunk * (D / 8); e += kBndThreads) {
-    const int t = e / (kChunk * (D / 8)), r = (e / (D / 8)) % kChunk, c = (e % (D / 8)) * 8;
-    *reinterpret_cast<uint4*>(PK::K(pack, t) + (size_t)r * PK::LDB + c) =
-        *reinterpret_cast<const uint4*>(&sm.K[t][r][c]);
-  }
-  for (int i = tid; i < kChunk; i += kBndThreads) PK::dvec(pack)[i] = sm.dvec[i];
-  if (tid == 0) *PK::gamma(pack) = sm.gammaC;
 }
 
 // ----------------------------------------------------------------------------
@@ -404,15 +314,25 @@ __device__ __forceinline__ void sacc_load(float (&sacc)[D / 8][4], const float* 
     }
 }
 
+// Store 16 rows; lanes t and t^1 swap halves so that every lane writes one
+// 16-byte run of one row.
 template <int D>
 __device__ __forceinline__ void sacc_store(const float (&sacc)[D / 8][4], float* S, int r0) {
-  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3, odd = tq & 1;
 #pragma unroll
-  for (int n = 0; n < D / 8; n++)
-#pragma unroll
-    for (int hf = 0; hf < 2; hf++)
-      *reinterpret_cast<float2*>(S + (size_t)(r0 + gq + 8 * hf) * D + 8 * n + 2 * tq) =
-          make_float2(sacc[n][2 * hf], sacc[n][2 * hf + 1]);
+  for (int n = 0; n < D / 8; n++) {
+    // even t keeps row g and receives its partner's row-g pair; odd t keeps
+    // row g+8 and receives its partner's row-(g+8) pair.
+    const float s0 = odd ? sacc[n][0] : sacc[n][2];
+    const float s1 = odd ? sacc[n][1] : sacc[n][3];
+    const float r0v = __shfl_xor_sync(kFull, s0, 1);
+    const float r1v = __shfl_xor_sync(kFull, s1, 1);
+    float4 out;
+    if (!odd) out = make_float4(sacc[n][0], sacc[n][1], r0v, r1v);
+    else out = make_float4(r0v, r1v, sacc[n][2], sacc[n][3]);
+    const int row = r0 + gq + 8 * odd, col = 8 * n + 2 * (tq & 2);
+    *reinterpret_cast<float4*>(S + (size_t)row * D + col) = out;
+  }
 }
 
 template <int D>
@@ -424,54 +344,93 @@ __device__ __forceinline__ void sacc_zero(float (&sacc)[D / 8][4]) {
 }
 
 // One boundary step for the warp's 16 rows (r0 = first row within the head):
-// sacc <- exp(G_C) sacc + Ud^T K with Ud = dvec * (U~ - W sacc^T).  `pack` is
-// in shared memory.
+//   Y  = S K^T                      (16 x C)
+//   Z  = (V^T Tv^T) - Y Tb^T        (= U^T for these rows)
+//   S <- exp(G_C) S + (dvec * Z) K
+// hd (Tb, Tv, dvec, gamma) and the K, V planes are in shared memory.
 template <int D, class IN>
-__device__ __forceinline__ void bnd_walk_warp(float (&sacc)[D / 8][4], char* pack, int r0) {
-  using PK = Pack<D, IN>;
+__device__ __forceinline__ void bnd_walk_warp(float (&sacc)[D / 8][4], const PackHead<D, IN>& hd,
+                                              const __nv_bfloat16* Kp, const __nv_bfloat16* Vp,
+                                              int r0) {
   constexpr int NS = Splits<IN>::S, NW = Splits<IN>::W, NK = Splits<IN>::K;
-  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
-  // X = S W^T  (16 x C)
-  float x[kChunk / 8][4];
+  constexpr int LDB = D + 8, LDT = kChunk + 8;
+  constexpr size_t PL = (size_t)kChunk * LDB;  // elements per K/V plane
+  const int lane = threadIdx.x & 31, tq = lane & 3;
+  // Y = S K^T
+  float y[kChunk / 8][4];
 #pragma unroll
   for (int n = 0; n < kChunk / 8; n++)
 #pragma unroll
-    for (int e = 0; e < 4; e++) x[n][e] = 0.f;
+    for (int e = 0; e < 4; e++) y[n][e] = 0.f;
   {
-    using PP = SplitPairs<NS, NW>;
+    using PP = SplitPairs<NS, NK>;
 #pragma unroll
     for (int ks = 0; ks < D / 16; ks++) {
       uint32_t a[NS][4];
       acc_to_afrag<NS>(sacc[2 * ks], sacc[2 * ks + 1], a);
 #pragma unroll
       for (int np = 0; np < kChunk / 16; np++) {
-        uint32_t b[NW][4];
+        uint32_t b[NK][4];
 #pragma unroll
-        for (int q = 0; q < NW; q++)
-          ldsm_x4(b[q], bfrag_nk_addr(PK::W(pack, q), PK::LDB, 16 * np, 16 * ks));
+        for (int q = 0; q < NK; q++) ldsm_x4(b[q], bfrag_nk_addr(Kp + q * PL, LDB, 16 * np, 16 * ks));
 #pragma unroll
         for (int p = 0; p < PP::kCount; p++) {
-          mma16816(x[2 * np], a[PP::a(p)], b[PP::b(p)][0], b[PP::b(p)][1]);
-          mma16816(x[2 * np + 1], a[PP::a(p)], b[PP::b(p)][2], b[PP::b(p)][3]);
+          mma16816(y[2 * np], a[PP::a(p)], b[PP::b(p)][0], b[PP::b(p)][1]);
+          mma16816(y[2 * np + 1], a[PP::a(p)], b[PP::b(p)][2], b[PP::b(p)][3]);
         }
       }
     }
   }
-  // Ud = dvec * (U~^T - X)
-  {
-    const float* U = PK::U(pack);
-    const float* dv = PK::dvec(pack);
+  // Z = V^T Tv^T - Y Tb^T  (Tb, Tv vanish above the diagonal block)
+  float z[kChunk / 8][4];
 #pragma unroll
-    for (int n = 0; n < kChunk / 8; n++)
+  for (int n = 0; n < kChunk / 8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) z[n][e] = 0.f;
+  {
+    using PV = SplitPairs<NK, NW>;
+    using PY = SplitPairs<NS, NW>;
+#pragma unroll
+    for (int ks = 0; ks < kChunk / 16; ks++) {
+      uint32_t av[NK][4], ay[NS][4];
+#pragma unroll
+      for (int q = 0; q < NK; q++) ldsm_x4_t(av[q], afrag_t_addr(Vp + q * PL, LDB, r0, 16 * ks));
+      float ny0[4], ny1[4];
 #pragma unroll
       for (int e = 0; e < 4; e++) {
-        const int r = r0 + gq + 8 * (e >> 1), i = 8 * n + 2 * tq + (e & 1);
-        x[n][e] = __fmul_rn(dv[i], __fsub_rn(U[(size_t)r * PK::LDU + i], x[n][e]));
+        ny0[e] = -y[2 * ks][e];
+        ny1[e] = -y[2 * ks + 1][e];
       }
+      acc_to_afrag<NS>(ny0, ny1, ay);
+#pragma unroll
+      for (int np = ks; np < kChunk / 16; np++) {
+        uint32_t bv[NW][4], bb[NW][4];
+#pragma unroll
+        for (int q = 0; q < NW; q++) {
+          ldsm_x4(bv[q], bfrag_nk_addr(&hd.Tv[q][0][0], LDT, 16 * np, 16 * ks));
+          ldsm_x4(bb[q], bfrag_nk_addr(&hd.Tb[q][0][0], LDT, 16 * np, 16 * ks));
+        }
+#pragma unroll
+        for (int p = 0; p < PV::kCount; p++) {
+          mma16816(z[2 * np], av[PV::a(p)], bv[PV::b(p)][0], bv[PV::b(p)][1]);
+          mma16816(z[2 * np + 1], av[PV::a(p)], bv[PV::b(p)][2], bv[PV::b(p)][3]);
+        }
+#pragma unroll
+        for (int p = 0; p < PY::kCount; p++) {
+          mma16816(z[2 * np], ay[PY::a(p)], bb[PY::b(p)][0], bb[PY::b(p)][1]);
+          mma16816(z[2 * np + 1], ay[PY::a(p)], bb[PY::b(p)][2], bb[PY::b(p)][3]);
+        }
+      }
+    }
   }
-  // S' = gamma S + Ud^T K  (16 x D)
+  // Ud = dvec * Z
+#pragma unroll
+  for (int n = 0; n < kChunk / 8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) z[n][e] = __fmul_rn(hd.dvec[8 * n + 2 * tq + (e & 1)], z[n][e]);
+  // S' = gamma S + Ud^T K
   {
-    const float gam = *PK::gamma(pack);
+    const float gam = hd.gamma[0];
 #pragma unroll
     for (int n = 0; n < D / 8; n++)
 #pragma unroll
@@ -480,13 +439,12 @@ __device__ __forceinline__ void bnd_walk_warp(float (&sacc)[D / 8][4], char* pac
 #pragma unroll
     for (int ks = 0; ks < kChunk / 16; ks++) {
       uint32_t a[NS][4];
-      acc_to_afrag<NS>(x[2 * ks], x[2 * ks + 1], a);
+      acc_to_afrag<NS>(z[2 * ks], z[2 * ks + 1], a);
 #pragma unroll
       for (int np = 0; np < D / 16; np++) {
         uint32_t b[NK][4];
 #pragma unroll
-        for (int q = 0; q < NK; q++)
-          ldsm_x4_t(b[q], bfrag_kn_addr(PK::K(pack, q), PK::LDB, 16 * ks, 16 * np));
+        for (int q = 0; q < NK; q++) ldsm_x4_t(b[q], bfrag_kn_addr(Kp + q * PL, LDB, 16 * ks, 16 * np));
 #pragma unroll
         for (int p = 0; p < PP::kCount; p++) {
           mma16816(sacc[2 * np], a[PP::a(p)], b[PP::b(p)][0], b[PP::b(p)][1]);

@@ -86,11 +86,18 @@ __global__ void __launch_bounds__(kTableThreads)
 // Pass 1a: boundary prep of every full chunk (independent of the state)
 // ----------------------------------------------------------------------------
 template <int D, class IN>
+__device__ __forceinline__ void copy16(char* dst, const char* src, size_t bytes, int nthreads) {
+  for (size_t e = threadIdx.x; e < bytes / 16; e += nthreads)
+    reinterpret_cast<uint4*>(dst)[e] = reinterpret_cast<const uint4*>(src)[e];
+}
+
+template <int D, class IN>
 __global__ void __launch_bounds__(kBndThreads)
-    k_prep(const IN* __restrict__ k, const IN* __restrict__ v, const float* __restrict__ beta,
-           const float* __restrict__ g, const int32_t* __restrict__ cu, int H,
-           const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
-           const int32_t* __restrict__ chunk_seq, char* __restrict__ packs) {
+    k_prep(const IN* __restrict__ k, const float* __restrict__ beta, const float* __restrict__ g,
+           const int32_t* __restrict__ cu, int H, const int32_t* __restrict__ hdr,
+           const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
+           char* __restrict__ packs) {
+  static_assert(sizeof(PackHead<D, IN>) % 16 == 0, "pack copies are 16-byte pieces");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   PrepSmem<D, IN>& sm = *reinterpret_cast<PrepSmem<D, IN>*>(smem_raw);
   const int c = blockIdx.x, h = blockIdx.y;
@@ -101,8 +108,10 @@ __global__ void __launch_bounds__(kBndThreads)
   if ((int64_t)(ci + 1) * kChunk > L) return;  // trailing partial chunk: no boundary
   const int64_t t0 = (int64_t)cu[n] + (int64_t)ci * kChunk;
   const size_t tok = (size_t)t0 * H + h;
-  prep_stage<D, IN>(sm, k + tok * D, v + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H);
-  bnd_prep<D, IN>(sm, packs + ((size_t)c * H + h) * Pack<D, IN>::kBytes);
+  prep_stage<D, IN>(sm, k + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H);
+  bnd_prep<D, IN>(sm);
+  copy16<D, IN>(packs + ((size_t)c * H + h) * pack_size<D, IN>(),
+                reinterpret_cast<const char*>(&sm.head), sizeof(PackHead<D, IN>), kBndThreads);
 }
 
 // ----------------------------------------------------------------------------
@@ -113,43 +122,60 @@ template <int D>
 constexpr int walk_threads() { return 32 * (D / 16); }
 
 template <int D, class IN>
-__device__ __forceinline__ void pack_fetch(char* dst, const char* src) {
-  constexpr int N16 = (int)(Pack<D, IN>::kBytes / 16);
-  for (int e = threadIdx.x; e < N16; e += walk_threads<D>()) cp_async16(dst + 16 * e, src + 16 * e);
+struct WalkBuf {
+  PackHead<D, IN> head;
+  KVPlanes<D, IN> kv;
+};
+
+// Issue the loads of chunk c's walk inputs into a buffer: the pack (cp.async)
+// and the chunk's keys and values from the packed inputs; one commit group.
+template <int D, class IN>
+__device__ __forceinline__ void walk_fetch(WalkBuf<D, IN>& buf, const char* pack, const IN* k,
+                                           const IN* v, size_t ld) {
+  constexpr int N16 = (int)(sizeof(PackHead<D, IN>) / 16);
+  char* dst = reinterpret_cast<char*>(&buf.head);
+  for (int e = threadIdx.x; e < N16; e += walk_threads<D>()) cp_async16(dst + 16 * e, pack + 16 * e);
+  stage_planes<D, IN>(buf.kv.K, k, ld, walk_threads<D>());
+  stage_planes<D, IN>(buf.kv.V, v, ld, walk_threads<D>());
   cp_async_commit();
 }
 
 template <int D, class IN>
 __global__ void __launch_bounds__(walk_threads<D>(), 1)
-    k_walk(const int32_t* __restrict__ cu, int H, const float* __restrict__ h0,
-           const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
-           const char* __restrict__ packs, float* __restrict__ bstate,
-           float* __restrict__ s_run_final, float* __restrict__ s_bnd_final) {
-  using PK = Pack<D, IN>;
+    k_walk(const IN* __restrict__ k, const IN* __restrict__ v, const int32_t* __restrict__ cu,
+           int H, const float* __restrict__ h0, const int32_t* __restrict__ hdr,
+           const int32_t* __restrict__ chunk_off, const char* __restrict__ packs,
+           float* __restrict__ bstate, float* __restrict__ s_run_final,
+           float* __restrict__ s_bnd_final) {
+  constexpr size_t PB = pack_size<D, IN>();
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  char* const buf0 = reinterpret_cast<char*>(smem_raw);  // double buffer: buf0 + (c & 1) * kBytes
+  WalkBuf<D, IN>* bufs = reinterpret_cast<WalkBuf<D, IN>*>(smem_raw);  // double buffer
   const int n = blockIdx.x, h = blockIdx.y;
   if (hdr[kHdrValid] != 1) return;
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
   const int64_t nf = L / kChunk, nc = (L + kChunk - 1) / kChunk;
   const int64_t base = chunk_off[n];
   const int r0 = 16 * (threadIdx.x >> 5);
-  const size_t DD = (size_t)D * D;
+  const size_t DD = (size_t)D * D, ld = (size_t)H * D;
+  const size_t tok0 = (size_t)cu[n] * H + h;  // first token of the sequence, this head
   float sacc[D / 8][4];
   if (h0) sacc_load<D>(sacc, h0 + ((size_t)n * H + h) * DD, r0);
   else sacc_zero<D>(sacc);
   if (nc > 0) sacc_store<D>(sacc, bstate + ((size_t)base * H + h) * DD, r0);
-  if (nf > 0) pack_fetch<D, IN>(buf0, packs + ((size_t)base * H + h) * PK::kBytes);
+  if (nf > 0)
+    walk_fetch<D, IN>(bufs[0], packs + ((size_t)base * H + h) * PB, k + tok0 * D, v + tok0 * D, ld);
   for (int64_t c = 0; c < nf; c++) {
     const size_t unit = (size_t)(base + c) * H + h;
     if (c + 1 < nf) {
-      pack_fetch<D, IN>(buf0 + ((c + 1) & 1) * PK::kBytes, packs + (unit + H) * PK::kBytes);
+      const size_t tk = tok0 + (size_t)(c + 1) * kChunk * H;
+      walk_fetch<D, IN>(bufs[(c + 1) & 1], packs + (unit + H) * PB, k + tk * D, v + tk * D, ld);
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
     __syncthreads();
-    bnd_walk_warp<D, IN>(sacc, buf0 + (c & 1) * PK::kBytes, r0);
+    const WalkBuf<D, IN>& b = bufs[c & 1];
+    bnd_walk_warp<D, IN>(sacc, b.head, &b.kv.K[0][0][0], &b.kv.V[0][0][0], r0);
     if (c + 1 < nc) sacc_store<D>(sacc, bstate + (unit + H) * DD, r0);
     __syncthreads();  // buffer c&1 is refilled by the prefetch of chunk c+2
   }
@@ -407,7 +433,7 @@ __global__ void __launch_bounds__(128)
 template <int D, class IN>
 struct BndSmem {
   PrepSmem<D, IN> prep;
-  alignas(16) char pack[Pack<D, IN>::kBytes];
+  __nv_bfloat16 V[Splits<IN>::K][kChunk][D + 8];
 };
 
 template <int D, class IN, bool RESYNC>
@@ -433,17 +459,17 @@ __global__ void __launch_bounds__(kBndThreads)
     unit = (size_t)(sh_go - 1) * H + h;
   }
   const size_t DD = (size_t)D * D;
-  prep_stage<D, IN>(sm.prep, kb + unit * kChunk * D, vb + unit * kChunk * D, (size_t)D,
-                    bb + unit * kChunk, gb + unit * kChunk, 1);
-  bnd_prep<D, IN>(sm.prep, sm.pack);
-  __syncthreads();
+  stage_planes<D, IN>(sm.V, vb + unit * kChunk * D, (size_t)D, kBndThreads);
+  prep_stage<D, IN>(sm.prep, kb + unit * kChunk * D, (size_t)D, bb + unit * kChunk,
+                    gb + unit * kChunk, 1);
+  bnd_prep<D, IN>(sm.prep);
   const int warp = threadIdx.x >> 5;
 #pragma unroll 1
   for (int rt = 0; rt < D / 64; rt++) {
     const int r0 = 16 * warp + 64 * rt;
     float sacc[D / 8][4];
     sacc_load<D>(sacc, s_start + unit * DD, r0);
-    bnd_walk_warp<D, IN>(sacc, sm.pack, r0);
+    bnd_walk_warp<D, IN>(sacc, sm.prep.head, &sm.prep.K[0][0][0], &sm.V[0][0][0], r0);
     sacc_store<D>(sacc, s_end + unit * DD, r0);
   }
   if (RESYNC && threadIdx.x == 0) pos[unit] = 0;
@@ -517,7 +543,7 @@ static cudaError_t persistent_grid(KernelT kern, int threads, size_t smem, int* 
 
 template <int D, class IN, class OUT>
 static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
-  static_assert(Pack<D, IN>::kBytes == pack_bytes(D, sizeof(IN) == 2), "pack layout mismatch");
+  static_assert(pack_size<D, IN>() == pack_bytes(D, sizeof(IN) == 2), "pack layout mismatch");
   const FwdLayout& L = a.lay;
   char* ws = a.ws;
   int32_t* hdr = reinterpret_cast<int32_t*>(ws + L.hdr);
@@ -541,17 +567,18 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     auto kern = k_prep<D, IN>;
     const size_t sm = sizeof(PrepSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
-    kern<<<gchunks, kBndThreads, sm, st>>>(k, v, a.beta, a.g, a.cu_seqlens, a.H, hdr, chunk_off,
+    kern<<<gchunks, kBndThreads, sm, st>>>(k, a.beta, a.g, a.cu_seqlens, a.H, hdr, chunk_off,
                                            chunk_seq, packs);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(2));
   {
     auto kern = k_walk<D, IN>;
-    const size_t sm = 2 * Pack<D, IN>::kBytes;
+    const size_t sm = 2 * sizeof(WalkBuf<D, IN>);
     GDN_TRY(set_smem(kern, sm));
     kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), walk_threads<D>(), sm, st>>>(
-        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final, a.s_bnd_final);
+        k, v, a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final,
+        a.s_bnd_final);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(3));
