@@ -255,10 +255,14 @@ def bench_e2e(gdn, b, dev, steps, warmup):
 def bench_decode(gdn, W, dev, rank, steps, warmup, slots=256):
     prefix = W.decode_prefix_lengths(slots)
     pre = W.make_batch(prefix, H, D, D, seed=100 + rank, device=dev)
-    _, srun, sbnd, ws = gdn.forward(pre.q, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens)
+    sscale = torch.empty((slots, H), device=dev)
+    _, srun, sbnd, ws = gdn.forward(pre.q, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens,
+                                    s_run_scale=sscale)
     st = gdn.DecodeState(slots, H, D, D, device=dev)
-    gdn.decode_state_from_prefill(st, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens, srun, sbnd)
+    gdn.decode_state_from_prefill(st, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens, srun, sbnd,
+                                  s_run_scale=sscale)
     del pre, srun, sbnd, ws
+    torch.cuda.empty_cache()  # keep only the decode state resident
     n_tok = warmup + steps
     toks = W.decode_tokens(n_tok, slots, H, D, D, seed=200 + rank, device=dev)
     o = torch.empty((slots, H, D), dtype=torch.bfloat16, device=dev)

@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define GDN_CPR_ABI_VERSION 1
+#define GDN_CPR_ABI_VERSION 2
 
 typedef enum {
   GDN_OK = 0,
@@ -100,10 +100,17 @@ size_t gdn_cpr_forward_workspace_bytes(int n_seqs, int64_t total_tokens, int H, 
  *             cu_seqlens[n_seqs] = total_tokens (checked on the device)
  * h0          [n_seqs, H, dv, dk] fp32 initial states, or NULL for zeros
  * o           [total_tokens, H, dv] out_dtype (written for every token)
- * s_run_final [n_seqs, H, dv, dk] fp32 or NULL: the state decode continues
- *             from.  For a length that is a multiple of C it equals
- *             s_bnd_final; otherwise it is the recurrent state after the
- *             trailing partial chunk.
+ * s_run_final [n_seqs, H, dv, dk] fp32 or NULL: the running state after
+ *             the last token.  For a length that is a multiple of C it
+ *             equals s_bnd_final; otherwise it is the recurrent state after
+ *             the trailing partial chunk.  Inside a chunk the kernels keep
+ *             that state as scale x mantissa (one fp32 scale per sequence
+ *             and head).  With s_run_scale == NULL, s_run_final receives the
+ *             state itself (scale x mantissa, rounded once).  With
+ *             s_run_scale != NULL ([n_seqs, H] fp32), s_run_final receives
+ *             the mantissa and s_run_scale the scale: the exact pair that
+ *             gdn_cpr_decode_state_from_prefill needs for decode to continue
+ *             bit for bit.
  * s_bnd_final [n_seqs, H, dv, dk] fp32 or NULL: the boundary state after the
  *             last full chunk (h0 for sequences shorter than C).
  * workspace   device scratch of at least gdn_cpr_forward_workspace_bytes;
@@ -113,8 +120,8 @@ size_t gdn_cpr_forward_workspace_bytes(int n_seqs, int64_t total_tokens, int H, 
 int gdn_cpr_forward(const void* q, const void* k, const void* v, int in_dtype, const float* beta,
                     const float* g, const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
                     int H, int dk, int dv, int C, float scale, const float* h0, void* o,
-                    int out_dtype, float* s_run_final, float* s_bnd_final, void* workspace,
-                    size_t workspace_bytes, void* stream);
+                    int out_dtype, float* s_run_final, float* s_run_scale, float* s_bnd_final,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * gdn_cpr_forward_ex -- gdn_cpr_forward that also records caller-created
@@ -128,8 +135,8 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
                        const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
                        int64_t total_tokens, int H, int dk, int dv, int C, float scale,
                        const float* h0, void* o, int out_dtype, float* s_run_final,
-                       float* s_bnd_final, void* workspace, size_t workspace_bytes,
-                       void* const* kernel_events, void* stream);
+                       float* s_run_scale, float* s_bnd_final, void* workspace,
+                       size_t workspace_bytes, void* const* kernel_events, void* stream);
 
 /*
  * gdn_cpr_forward_noalloc -- gdn_cpr_forward for callers that cannot
@@ -159,12 +166,15 @@ int gdn_cpr_forward_noalloc(const void* q, const void* k, const void* v, int in_
                             const float* beta, const float* g, const int32_t* cu_seqlens,
                             int n_seqs, int64_t total_tokens, int H, int dk, int dv, int C,
                             float scale, const float* h0, void* o, int out_dtype,
-                            float* s_run_final, float* s_bnd_final, int32_t* error_word,
-                            void* stream);
+                            float* s_run_final, float* s_run_scale, float* s_bnd_final,
+                            int32_t* error_word, void* stream);
 
 /*
  * Decode state: caller-owned device arrays for n_slots sequences.
- *   s_run    [n_slots, H, dv, dk] fp32  running state (not read when pos == 0)
+ *   s_run    [n_slots, H, dv, dk] fp32  mantissa of the running state
+ *   s_scale  [n_slots, H] fp32          its scale: running state =
+ *                                       s_scale x s_run (neither is read
+ *                                       when pos == 0)
  *   s_bnd    [n_slots, H, dv, dk] fp32  boundary state at the start of the
  *                                       current chunk
  *   buf_k    [n_slots, H, C, dk]  in_dtype  keys of the current chunk so far
@@ -177,6 +187,7 @@ int gdn_cpr_forward_noalloc(const void* q, const void* k, const void* v, int in_
  */
 typedef struct {
   float* s_run;
+  float* s_scale;
   float* s_bnd;
   void* buf_k;
   void* buf_v;
@@ -191,7 +202,10 @@ typedef struct {
  * gdn_cpr_decode_state_from_prefill -- hand a prefill over to decode.
  * For sequence n (slot slot_idx[n], or n when slot_idx is NULL):
  * pos = L_n mod C, the buffer receives the last pos tokens' k, v, beta, g
- * (bit copies), s_run <- s_run_final[n], s_bnd <- s_bnd_final[n].
+ * (bit copies), s_run <- s_run_final[n], s_scale <- s_run_scale[n] (1 when
+ * s_run_scale is NULL), s_bnd <- s_bnd_final[n].  Decode continues bit for
+ * bit from a forward only when given the forward's (s_run_final,
+ * s_run_scale) pair.
  * Inputs are the packed tensors, cu_seqlens and total_tokens passed to
  * gdn_cpr_forward and the final states it produced.  A slot outside
  * [0, n_slots) or a cu_seqlens entry outside [0, total_tokens] skips that
@@ -201,9 +215,9 @@ int gdn_cpr_decode_state_from_prefill(const void* k, const void* v, int in_dtype
                                       const float* beta, const float* g,
                                       const int32_t* cu_seqlens, int n_seqs,
                                       int64_t total_tokens, int H, int dk, int dv, int C,
-                                      const float* s_run_final, const float* s_bnd_final,
-                                      const int32_t* slot_idx, gdn_decode_state st,
-                                      void* stream);
+                                      const float* s_run_final, const float* s_run_scale,
+                                      const float* s_bnd_final, const int32_t* slot_idx,
+                                      gdn_decode_state st, void* stream);
 
 /*
  * gdn_cpr_decode_step -- one batched decode step with chunk resync.

@@ -37,7 +37,8 @@ class GdnError(RuntimeError):
 
 
 class DecodeStateStruct(ctypes.Structure):
-    _fields_ = [("s_run", ctypes.c_void_p), ("s_bnd", ctypes.c_void_p),
+    _fields_ = [("s_run", ctypes.c_void_p), ("s_scale", ctypes.c_void_p),
+                ("s_bnd", ctypes.c_void_p),
                 ("buf_k", ctypes.c_void_p), ("buf_v", ctypes.c_void_p),
                 ("buf_beta", ctypes.c_void_p), ("buf_g", ctypes.c_void_p),
                 ("pos", ctypes.c_void_p), ("error", ctypes.c_void_p),
@@ -56,13 +57,14 @@ def _load() -> ctypes.CDLL:
         "gdn_status_string": (ctypes.c_char_p, [i32]),
         "gdn_cpr_forward_workspace_bytes": (sz, [i32, i64, i32, i32, i32, i32, i32]),
         "gdn_cpr_forward": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32, f32,
-                                  vp, vp, i32, vp, vp, vp, sz, vp]),
+                                  vp, vp, i32, vp, vp, vp, vp, sz, vp]),
         "gdn_cpr_forward_ex": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32,
-                                     f32, vp, vp, i32, vp, vp, vp, sz, vp, vp]),
+                                     f32, vp, vp, i32, vp, vp, vp, vp, sz, vp, vp]),
         "gdn_cpr_forward_noalloc": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32,
-                                          i32, f32, vp, vp, i32, vp, vp, vp, vp]),
+                                          i32, f32, vp, vp, i32, vp, vp, vp, vp, vp]),
         "gdn_cpr_decode_state_from_prefill": (i32, [vp, vp, i32, vp, vp, vp, i32, i64, i32, i32,
-                                                    i32, i32, vp, vp, vp, DecodeStateStruct, vp]),
+                                                    i32, i32, vp, vp, vp, vp,
+                                                    DecodeStateStruct, vp]),
         "gdn_cpr_decode_step": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32,
                                       DecodeStateStruct, vp, i32, vp]),
         "gdn_chunk_boundary": (i32, [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
@@ -135,11 +137,14 @@ def forward_workspace_bytes(n_seqs: int, total_tokens: int, H: int, dk: int, dv:
 
 def forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=None,
             C: int = CHUNK, scale: float = 1.0, out_dtype=None, o=None, s_run_final=None,
-            s_bnd_final=None, want_states: bool = True, workspace=None, stream=None,
-            kernel_events=None):
+            s_bnd_final=None, s_run_scale=None, want_states: bool = True, workspace=None,
+            stream=None, kernel_events=None):
     """gdn_cpr_forward (gdn_cpr_forward_ex when ``kernel_events``, a list of 5
     recorded torch.cuda.Event objects, is given).
-    Returns (o, s_run_final, s_bnd_final, workspace)."""
+    Returns (o, s_run_final, s_bnd_final, workspace).  s_run_final is the
+    running state itself, unless an ``s_run_scale`` tensor [N, H] fp32 is
+    passed: then s_run_final holds the mantissa and s_run_scale the scale (the
+    pair decode needs to continue bit for bit)."""
     T, H, dk = q.shape
     dv = v.shape[2]
     N = (cu_seqlens.numel() - 1) if n_seqs is None else int(n_seqs)
@@ -163,8 +168,9 @@ def forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=No
         ev = (ctypes.c_void_p * 5)(*[e.cuda_event for e in kernel_events])
     st = lib.gdn_cpr_forward_ex(_ptr(q), _ptr(k), _ptr(v), in_code, _ptr(beta), _ptr(g),
                                 _ptr(cu_seqlens), N, T, H, dk, dv, C, float(scale), _ptr(h0),
-                                _ptr(o), out_code, _ptr(s_run_final), _ptr(s_bnd_final),
-                                _ptr(workspace), workspace.numel(), ev, _stream(stream))
+                                _ptr(o), out_code, _ptr(s_run_final), _ptr(s_run_scale),
+                                _ptr(s_bnd_final), _ptr(workspace), workspace.numel(), ev,
+                                _stream(stream))
     _check(st, "gdn_cpr_forward")
     return o, s_run_final, s_bnd_final, workspace
 
@@ -187,6 +193,7 @@ class DecodeState:
         self.in_dtype = in_dtype
         f32 = torch.float32
         self.s_run = torch.zeros((n_slots, H, dv, dk), dtype=f32, device=device)
+        self.s_scale = torch.ones((n_slots, H), dtype=f32, device=device)
         self.s_bnd = torch.zeros((n_slots, H, dv, dk), dtype=f32, device=device)
         self.buf_k = torch.zeros((n_slots, H, C, dk), dtype=in_dtype, device=device)
         self.buf_v = torch.zeros((n_slots, H, C, dv), dtype=in_dtype, device=device)
@@ -196,14 +203,15 @@ class DecodeState:
         self.error = torch.zeros((1,), dtype=torch.int32, device=device)
 
     def struct(self) -> DecodeStateStruct:
-        return DecodeStateStruct(self.s_run.data_ptr(), self.s_bnd.data_ptr(),
+        return DecodeStateStruct(self.s_run.data_ptr(), self.s_scale.data_ptr(),
+                                 self.s_bnd.data_ptr(),
                                  self.buf_k.data_ptr(), self.buf_v.data_ptr(),
                                  self.buf_beta.data_ptr(), self.buf_g.data_ptr(),
                                  self.pos.data_ptr(), self.error.data_ptr(), self.n_slots)
 
     def tensors(self):
-        return (self.s_run, self.s_bnd, self.buf_k, self.buf_v, self.buf_beta, self.buf_g,
-                self.pos)
+        return (self.s_run, self.s_scale, self.s_bnd, self.buf_k, self.buf_v, self.buf_beta,
+                self.buf_g, self.pos)
 
     def clone(self) -> "DecodeState":
         c = DecodeState.__new__(DecodeState)
@@ -213,13 +221,13 @@ class DecodeState:
 
 
 def decode_state_from_prefill(state: DecodeState, k, v, beta, g, cu_seqlens, s_run_final,
-                              s_bnd_final, *, slot_idx=None, stream=None):
+                              s_bnd_final, *, s_run_scale=None, slot_idx=None, stream=None):
     N = cu_seqlens.numel() - 1
     T, H, dk = k.shape
     st = lib.gdn_cpr_decode_state_from_prefill(
         _ptr(k), _ptr(v), _dtype_code(k), _ptr(beta), _ptr(g), _ptr(cu_seqlens), N, T, H, dk,
-        v.shape[2], state.C, _ptr(s_run_final), _ptr(s_bnd_final), _ptr(slot_idx),
-        state.struct(), _stream(stream))
+        v.shape[2], state.C, _ptr(s_run_final), _ptr(s_run_scale), _ptr(s_bnd_final),
+        _ptr(slot_idx), state.struct(), _stream(stream))
     _check(st, "gdn_cpr_decode_state_from_prefill")
 
 

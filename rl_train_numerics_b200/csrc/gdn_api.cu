@@ -56,19 +56,19 @@ size_t gdn_cpr_forward_workspace_bytes(int n_seqs, int64_t total_tokens, int H, 
 int gdn_cpr_forward(const void* q, const void* k, const void* v, int in_dtype, const float* beta,
                     const float* g, const int32_t* cu_seqlens, int n_seqs, int64_t total_tokens,
                     int H, int dk, int dv, int C, float scale, const float* h0, void* o,
-                    int out_dtype, float* s_run_final, float* s_bnd_final, void* workspace,
-                    size_t workspace_bytes, void* stream) {
+                    int out_dtype, float* s_run_final, float* s_run_scale, float* s_bnd_final,
+                    void* workspace, size_t workspace_bytes, void* stream) {
   return gdn_cpr_forward_ex(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs, total_tokens, H, dk,
-                            dv, C, scale, h0, o, out_dtype, s_run_final, s_bnd_final, workspace,
-                            workspace_bytes, nullptr, stream);
+                            dv, C, scale, h0, o, out_dtype, s_run_final, s_run_scale, s_bnd_final,
+                            workspace, workspace_bytes, nullptr, stream);
 }
 
 int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype,
                        const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
                        int64_t total_tokens, int H, int dk, int dv, int C, float scale,
                        const float* h0, void* o, int out_dtype, float* s_run_final,
-                       float* s_bnd_final, void* workspace, size_t workspace_bytes,
-                       void* const* kernel_events, void* stream) {
+                       float* s_run_scale, float* s_bnd_final, void* workspace,
+                       size_t workspace_bytes, void* const* kernel_events, void* stream) {
   if (n_seqs < 0 || total_tokens < 0 || !valid_dtype(out_dtype) || !isfinite(scale))
     return GDN_ERR_INVALID_ARG;
   int rc = check_shape(H, dk, dv, C, in_dtype);
@@ -82,8 +82,9 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
     if (!aligned4(beta) || !aligned4(g)) return GDN_ERR_INVALID_ARG;
   }
   if ((h0 && !aligned16(h0)) || (s_run_final && !aligned16(s_run_final)) ||
-      (s_bnd_final && !aligned16(s_bnd_final)))
+      (s_bnd_final && !aligned16(s_bnd_final)) || (s_run_scale && !aligned4(s_run_scale)))
     return GDN_ERR_INVALID_ARG;
+  if (s_run_scale && !s_run_final) return GDN_ERR_INVALID_ARG;
   const gdn::FwdLayout lay =
       gdn::fwd_layout(n_seqs, total_tokens, H, dk, dv, C, in_dtype == GDN_BF16);
   if (!workspace || workspace_bytes < lay.total) return GDN_ERR_WORKSPACE;
@@ -105,6 +106,7 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
   a.o = o;
   a.out_bf16 = out_dtype == GDN_BF16;
   a.s_run_final = s_run_final;
+  a.s_run_scale = s_run_scale;
   a.s_bnd_final = s_bnd_final;
   a.ws = static_cast<char*>(workspace);
   a.lay = lay;
@@ -113,12 +115,12 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
 }
 
 static int check_state(const gdn_decode_state& st) {
-  if (st.n_slots <= 0 || !st.s_run || !st.s_bnd || !st.buf_k || !st.buf_v || !st.buf_beta ||
-      !st.buf_g || !st.pos || !st.error)
+  if (st.n_slots <= 0 || !st.s_run || !st.s_scale || !st.s_bnd || !st.buf_k || !st.buf_v ||
+      !st.buf_beta || !st.buf_g || !st.pos || !st.error)
     return GDN_ERR_INVALID_ARG;
   if (!aligned16(st.s_run) || !aligned16(st.s_bnd) || !aligned16(st.buf_k) ||
       !aligned16(st.buf_v) || !aligned4(st.buf_beta) || !aligned4(st.buf_g) ||
-      !aligned4(st.pos) || !aligned4(st.error))
+      !aligned4(st.pos) || !aligned4(st.error) || !aligned4(st.s_scale))
     return GDN_ERR_INVALID_ARG;
   return GDN_OK;
 }
@@ -127,9 +129,9 @@ int gdn_cpr_decode_state_from_prefill(const void* k, const void* v, int in_dtype
                                       const float* beta, const float* g,
                                       const int32_t* cu_seqlens, int n_seqs,
                                       int64_t total_tokens, int H, int dk, int dv, int C,
-                                      const float* s_run_final, const float* s_bnd_final,
-                                      const int32_t* slot_idx, gdn_decode_state st,
-                                      void* stream) {
+                                      const float* s_run_final, const float* s_run_scale,
+                                      const float* s_bnd_final, const int32_t* slot_idx,
+                                      gdn_decode_state st, void* stream) {
   if (n_seqs < 0 || total_tokens < 0) return GDN_ERR_INVALID_ARG;
   int rc = check_shape(H, dk, dv, C, in_dtype);
   if (rc != GDN_OK) return rc;
@@ -139,6 +141,7 @@ int gdn_cpr_decode_state_from_prefill(const void* k, const void* v, int in_dtype
   if (!cu_seqlens || !s_run_final || !s_bnd_final) return GDN_ERR_INVALID_ARG;
   if (total_tokens > 0 && (!k || !v || !beta || !g)) return GDN_ERR_INVALID_ARG;
   if (!aligned16(s_run_final) || !aligned16(s_bnd_final)) return GDN_ERR_INVALID_ARG;
+  if (s_run_scale && !aligned4(s_run_scale)) return GDN_ERR_INVALID_ARG;
   if (!slot_idx && n_seqs > st.n_slots) return GDN_ERR_INVALID_ARG;
   gdn::HandoffArgs a{};
   a.k = k;
@@ -152,9 +155,11 @@ int gdn_cpr_decode_state_from_prefill(const void* k, const void* v, int in_dtype
   a.H = H;
   a.D = dk;
   a.s_run_final = s_run_final;
+  a.s_run_scale = s_run_scale;
   a.s_bnd_final = s_bnd_final;
   a.slot_idx = slot_idx;
   a.s_run = st.s_run;
+  a.s_scale = st.s_scale;
   a.s_bnd = st.s_bnd;
   a.buf_k = st.buf_k;
   a.buf_v = st.buf_v;
@@ -193,6 +198,7 @@ int gdn_cpr_decode_step(const void* q, const void* k, const void* v, int in_dtyp
   a.D = dk;
   a.scale = scale;
   a.s_run = st.s_run;
+  a.s_scale = st.s_scale;
   a.s_bnd = st.s_bnd;
   a.buf_k = st.buf_k;
   a.buf_v = st.buf_v;

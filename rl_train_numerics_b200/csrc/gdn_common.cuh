@@ -5,15 +5,27 @@
 // section "Solving the linear-attention headache" of "NovaSky's IsoExec Fixes
 // the Hidden Math Bug Corrupting AI Training Runs" asks that prefill,
 // training and decode share one rounding schedule; here that schedule is
-// fixed instruction by instruction:
+// fixed instruction by instruction.
 //
-//   a   = expf(g_t)
-//   p_r = sum_j S[r][j] k_j              per-row dot (order below)
+// Scaled running state.  Inside a chunk the state is kept as S = c * M: a
+// per-(sequence, head) scale c and a d_v x d_k mantissa M.  At a chunk
+// boundary M is the boundary state and c = 1.  One token (a = expf(g)):
+//
+//   p_r = c * dot(M_r, k)                 (dot order below)
 //   u_r = beta * fma(-a, p_r, v_r)
-//   S[r][j] <- fma(a, S[r][j], u_r * k_j)
-//   o_r = scale * sum_j S[r][j] q_j      same dot order
+//   c'  = a * c
+//   if c' >= 2^-64:   M_r[j] <- fma(u_r * (1/c'), k_j, M_r[j]),  c <- c'
+//   else (renormalise, also when a underflows to 0):
+//                     M_r[j] <- fma(c', M_r[j], u_r * k_j),      c <- 1
+//   o_r = scale * (c * dot(M_r, q))
 //
-// Row-dot order.  Rows of S evolve independently.  A row of d_k values is
+// which is S_t = a S_{t-1} + u k^T, o_t = scale * S_t q_t with
+// u = beta (v - a S_{t-1} k) -- the recurrence
+// S_t = a S_{t-1} (I - beta k k^T) + beta v k^T -- with one fused
+// multiply-add per state element for the update instead of a multiply and an
+// add.  1/c' is the correctly rounded reciprocal.
+//
+// Row-dot order.  Rows of M evolve independently.  A row of d_k values is
 // split over the 4 lanes of a quad; lane l holds the column groups l, l+4,
 // l+8, ... (columns 4(l+4m) .. 4(l+4m)+3).  Each lane keeps two partial sums
 // (a packed fp32 pair): columns 4c and 4c+2 of each group go to the first,
@@ -62,6 +74,17 @@ __device__ __forceinline__ float ld1(const __nv_bfloat16* p) { return __bfloat16
 __device__ __forceinline__ void st1(float* p, float x) { *p = x; }
 __device__ __forceinline__ void st1(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
+// Four consecutive elements of a shared-memory row as fp32 (bf16 widening is
+// a bit shift, exact).
+__device__ __forceinline__ float4 sld4(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ float4 sld4(const __nv_bfloat16* p) {
+  const uint2 r = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u),
+                     __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
+}
+
 // ----------------------------------------------------------------------------
 // The pinned step arithmetic
 // ----------------------------------------------------------------------------
@@ -77,9 +100,10 @@ __device__ __forceinline__ float step_u(float a, float beta, float p, float v) {
   return __fmul_rn(beta, __fmaf_rn(-a, p, v));
 }
 
-__device__ __forceinline__ float step_s(float a, float s, float u, float k) {
-  return __fmaf_rn(a, s, __fmul_rn(u, k));
-}
+// Smallest scale kept without renormalising: 2^-64.
+__device__ __forceinline__ bool scale_ok(float c) { return c >= 5.42101086242752217e-20f; }
+
+__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
 
 // State slice of one thread: RT rows x M4 groups of 4 columns, each group held
 // as two float2 (columns 4c, 4c+1 and 4c+2, 4c+3).
@@ -87,8 +111,6 @@ template <int RT, int M4>
 struct Slice {
   float2 s[RT][M4][2];
 };
-
-__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
 
 // out[i] = lane-partial dot of row i with x (x fetched per group m as a
 // float4).  Columns 4c and 4c+2 of every group accumulate into the .x half,
@@ -113,18 +135,20 @@ __device__ __forceinline__ void slice_dot(const Slice<RT, M4>& S, Fetch fx, floa
   for (int i = 0; i < RT; i++) out[i] = __fadd_rn(acc[i].x, acc[i].y);
 }
 
-// Update every element with s <- fma(a, s, u*k), and in the same sweep
-// accumulate the lane-partial dots with q (the output) and, when NEXT, with
-// the next token's key (the next step's p), in the slice_dot order, so the
-// fused dots carry the same bits as separate slice_dot sweeps.
-template <bool NEXT, int RT, int M4, class FK, class FQ, class FN>
-__device__ __forceinline__ void slice_update(Slice<RT, M4>& S, float a, const float (&u)[RT],
+// Update every mantissa element and, in the same sweep, accumulate the
+// lane-partial dots with q (the output) and, when NEXT, with the next
+// token's key (the next step's dot), in the slice_dot order, so the fused
+// dots carry the same bits as separate slice_dot sweeps.
+//   RENORM = false:  M <- fma(w_r, k_j, M)          (w = u / c')
+//   RENORM = true:   M <- fma(c', M, u_r * k_j)     (w holds u, cn = c')
+template <bool NEXT, bool RENORM, int RT, int M4, class FK, class FQ, class FN>
+__device__ __forceinline__ void slice_update(Slice<RT, M4>& S, float cn, const float (&w)[RT],
                                              FK fk, FQ fq, FN fn, float (&oout)[RT],
                                              float (&pout)[RT]) {
   float2 oacc[RT], pacc[RT];
 #pragma unroll
   for (int i = 0; i < RT; i++) oacc[i] = pacc[i] = f2(0.f, 0.f);
-  const float2 aa = f2(a, a);
+  const float2 cc = f2(cn, cn);
 #pragma unroll
   for (int m = 0; m < M4; m++) {
     const float4 k4 = fk(m);
@@ -136,9 +160,15 @@ __device__ __forceinline__ void slice_update(Slice<RT, M4>& S, float a, const fl
     const float2 n01 = f2(n4.x, n4.y), n23 = f2(n4.z, n4.w);
 #pragma unroll
     for (int i = 0; i < RT; i++) {
-      const float2 uu = f2(u[i], u[i]);
-      const float2 s01 = __ffma2_rn(aa, S.s[i][m][0], __fmul2_rn(uu, k01));
-      const float2 s23 = __ffma2_rn(aa, S.s[i][m][1], __fmul2_rn(uu, k23));
+      const float2 ww = f2(w[i], w[i]);
+      float2 s01, s23;
+      if (RENORM) {
+        s01 = __ffma2_rn(cc, S.s[i][m][0], __fmul2_rn(ww, k01));
+        s23 = __ffma2_rn(cc, S.s[i][m][1], __fmul2_rn(ww, k23));
+      } else {
+        s01 = __ffma2_rn(ww, k01, S.s[i][m][0]);
+        s23 = __ffma2_rn(ww, k23, S.s[i][m][1]);
+      }
       S.s[i][m][0] = s01;
       S.s[i][m][1] = s23;
       oacc[i] = __ffma2_rn(s01, q01, oacc[i]);
@@ -153,6 +183,37 @@ __device__ __forceinline__ void slice_update(Slice<RT, M4>& S, float a, const fl
   for (int i = 0; i < RT; i++) {
     oout[i] = __fadd_rn(oacc[i].x, oacc[i].y);
     pout[i] = __fadd_rn(pacc[i].x, pacc[i].y);
+  }
+}
+
+// One token on a slice: given the quad-reduced dot pd = dot(M_r, k) of each
+// row and the scale c, apply the step (with NEXT, also return the next
+// token's dot in pd), write o (before `scale`) to ov and update c.
+template <bool NEXT, int RT, int M4, class FK, class FQ, class FN, class FV>
+__device__ __forceinline__ void slice_token(Slice<RT, M4>& S, float& c, float a, float beta,
+                                            FV fv, FK fk, FQ fq, FN fn, float (&pd)[RT],
+                                            float (&ov)[RT]) {
+  float u[RT], oacc[RT], pacc[RT];
+#pragma unroll
+  for (int i = 0; i < RT; i++) u[i] = step_u(a, beta, __fmul_rn(c, pd[i]), fv(i));
+  const float cn = __fmul_rn(a, c);
+  float cnew;
+  if (scale_ok(cn)) {
+    const float d = __frcp_rn(cn);
+    float w[RT];
+#pragma unroll
+    for (int i = 0; i < RT; i++) w[i] = __fmul_rn(u[i], d);
+    slice_update<NEXT, false, RT, M4>(S, cn, w, fk, fq, fn, oacc, pacc);
+    cnew = cn;
+  } else {
+    slice_update<NEXT, true, RT, M4>(S, cn, u, fk, fq, fn, oacc, pacc);
+    cnew = 1.f;
+  }
+  c = cnew;
+#pragma unroll
+  for (int i = 0; i < RT; i++) {
+    ov[i] = __fmul_rn(cnew, quad_sum(oacc[i]));
+    if (NEXT) pd[i] = quad_sum(pacc[i]);
   }
 }
 
@@ -185,15 +246,19 @@ __device__ __forceinline__ void slice_store(const Slice<RT, M4>& S, float* rows,
     }
 }
 
-// Four consecutive elements of a shared-memory row as fp32 (bf16 widening is
-// a bit shift, exact).
-__device__ __forceinline__ float4 sld4(const float* p) {
-  return *reinterpret_cast<const float4*>(p);
-}
-__device__ __forceinline__ float4 sld4(const __nv_bfloat16* p) {
-  const uint2 r = *reinterpret_cast<const uint2*>(p);
-  return make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u),
-                     __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
+// Store c * M (the state itself) instead of the mantissa.
+template <int RT, int M4>
+__device__ __forceinline__ void slice_store_scaled(const Slice<RT, M4>& S, float c, float* rows,
+                                                   int ld, int r0, int l) {
+  const float2 cc = f2(c, c);
+#pragma unroll
+  for (int i = 0; i < RT; i++)
+#pragma unroll
+    for (int m = 0; m < M4; m++) {
+      const float2 a = __fmul2_rn(cc, S.s[i][m][0]), b = __fmul2_rn(cc, S.s[i][m][1]);
+      *reinterpret_cast<float4*>(rows + (size_t)(r0 + i) * ld + group_col(l, m)) =
+          make_float4(a.x, a.y, b.x, b.y);
+    }
 }
 
 }  // namespace gdn

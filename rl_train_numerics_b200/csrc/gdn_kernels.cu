@@ -10,9 +10,9 @@
 //   k_fill          persistent blocks over (chunk, head) items: per-token
 //                   recurrence from each chunk's boundary state
 // Decode (same section: the recurrent form re-synchronised every chunk):
-//   k_dec_step      one block per (row, head): one recurrence step
-//   k_bnd           one block per (row, head): resync of units whose chunk
-//                   buffer just filled; also gdn_chunk_boundary
+//   k_dec_step      one block per (row, head): one recurrence step, then the
+//                   chunk boundary when the step filled the chunk buffer
+//   k_bnd           one block per (row, head): gdn_chunk_boundary
 //   k_handoff       prefill -> decode state
 #include "gdn_boundary.cuh"
 #include "gdn_layout.h"
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(walk_threads<D>(), 1)
            int H, const float* __restrict__ h0, const int32_t* __restrict__ hdr,
            const int32_t* __restrict__ chunk_off, const char* __restrict__ packs,
            float* __restrict__ bstate, float* __restrict__ s_run_final,
-           float* __restrict__ s_bnd_final) {
+           float* __restrict__ s_run_scale, float* __restrict__ s_bnd_final) {
   constexpr size_t PB = pack_size<D, IN>();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   WalkBuf<D, IN>* bufs = reinterpret_cast<WalkBuf<D, IN>*>(smem_raw);  // double buffer
@@ -181,35 +181,30 @@ __global__ void __launch_bounds__(walk_threads<D>(), 1)
   }
   const size_t so = ((size_t)n * H + h) * DD;
   if (s_bnd_final) sacc_store<D>(sacc, s_bnd_final + so, r0);
-  if (s_run_final && (L % kChunk) == 0) sacc_store<D>(sacc, s_run_final + so, r0);
+  if (s_run_final && (L % kChunk) == 0) {
+    sacc_store<D>(sacc, s_run_final + so, r0);
+    if (s_run_scale && threadIdx.x == 0) s_run_scale[(size_t)n * H + h] = 1.f;
+  }
 }
 
 // ----------------------------------------------------------------------------
 // Pass 2: per-token recurrence inside every chunk, from its boundary state.
-// Persistent blocks take (chunk, head) items from a work counter; the next
-// item's q/k/v/beta/g are staged into shared memory (input dtype, cp.async)
-// while the current item runs, and its boundary state is prefetched to L2.
+// Persistent blocks (three per SM) take (chunk, head) items from a work
+// counter.  An item's keys are widened to fp32 in shared memory (they are
+// read twice per token); queries and values stay in the input dtype.  While
+// an item runs, the next item's state and inputs are prefetched into L2.
 // Which block runs an item does not change the item's bits.
 // ----------------------------------------------------------------------------
 constexpr int kFillThreads = 128;
 
 template <int D, class IN>
-struct FillStage {
-  IN k[kChunk + 1][D];  // row kChunk stays zero: the "next key" of the last token
+struct FillSmem {
+  float k[kChunk + 1][D];  // row kChunk stays zero: the "next key" of the last token
   IN q[kChunk][D];
   IN v[kChunk][D];
-  float a[kChunk];  // log-decay g as staged, then exp(g)
-  float b[kChunk];
+  float a[kChunk];  // exp(g)
+  float b[kChunk];  // beta
 };
-
-__device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),
-               "l"(gmem), "r"(valid ? 16 : 0));
-}
-__device__ __forceinline__ void cp_async4_zfill(void* smem, const void* gmem, bool valid) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(smem)),
-               "l"(gmem), "r"(valid ? 4 : 0));
-}
 
 template <int RT>
 __device__ __forceinline__ float pick(const float (&x)[RT], int l) {
@@ -239,43 +234,6 @@ __device__ __forceinline__ FillItem fill_item(int item, int H, const int32_t* cu
   return it;
 }
 
-// Issue the cp.async copies of one item's inputs into a stage (rows past the
-// item's length are zero-filled without reading memory) as one commit group.
-template <int D, class IN>
-__device__ __forceinline__ void fill_stage_issue(FillStage<D, IN>& st, const FillItem& it,
-                                                 const IN* q, const IN* k, const IN* v,
-                                                 const float* beta, const float* g, int H) {
-  constexpr int P = (int)(D * sizeof(IN) / 16);  // 16-byte pieces per row
-  constexpr int E = (int)(16 / sizeof(IN));      // elements per piece
-  const size_t ld = (size_t)H * D;
-  const size_t tb = (size_t)it.t0 * H + it.h;
-  const IN* kb = k + tb * D;
-  const IN* qb = q + tb * D;
-  const IN* vb = v + tb * D;
-  for (int e = threadIdx.x; e < (3 * kChunk + 1) * P; e += kFillThreads) {
-    const int row = e / P, pc = (e % P) * E;
-    if (row <= kChunk) {
-      const bool ok = row < it.len;
-      cp_async16_zfill(&st.k[row][pc], kb + (size_t)(ok ? row : 0) * ld + pc, ok);
-    } else if (row <= 2 * kChunk) {
-      const int r = row - kChunk - 1;
-      const bool ok = r < it.len;
-      cp_async16_zfill(&st.q[r][pc], qb + (size_t)(ok ? r : 0) * ld + pc, ok);
-    } else {
-      const int r = row - 2 * kChunk - 1;
-      const bool ok = r < it.len;
-      cp_async16_zfill(&st.v[r][pc], vb + (size_t)(ok ? r : 0) * ld + pc, ok);
-    }
-  }
-  for (int i = threadIdx.x; i < 2 * kChunk; i += kFillThreads) {
-    const int r = i & (kChunk - 1);
-    const bool ok = r < it.len;
-    const float* src = (i < kChunk ? g : beta) + tb + (size_t)(ok ? r : 0) * H;
-    cp_async4_zfill(i < kChunk ? &st.a[r] : &st.b[r], src, ok);
-  }
-  cp_async_commit();
-}
-
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes));
 }
@@ -283,17 +241,67 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
+// Load one item's inputs into shared memory (rows past its length are zero).
+template <int D, class IN>
+__device__ __forceinline__ void fill_load(FillSmem<D, IN>& sm, const FillItem& it, const IN* q,
+                                          const IN* k, const IN* v, const float* beta,
+                                          const float* g, int H) {
+  constexpr int G4 = D / 4;                        // float4 groups of a key row
+  constexpr int P = (int)(D * sizeof(IN) / 16);    // 16-byte pieces of a q/v row
+  constexpr int E = (int)(16 / sizeof(IN));
+  const size_t ld = (size_t)H * D;
+  const size_t tb = (size_t)it.t0 * H + it.h;
+  for (int e = threadIdx.x; e < (kChunk + 1) * G4; e += kFillThreads) {
+    const int r = e / G4, c = (e % G4) * 4;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < it.len) x = ld4(k + (tb + (size_t)r * H) * D + c);
+    *reinterpret_cast<float4*>(&sm.k[r][c]) = x;
+  }
+  for (int e = threadIdx.x; e < 2 * kChunk * P; e += kFillThreads) {
+    const int rr = e / P, pc = (e % P) * E, r = rr % kChunk;
+    IN* dst = rr < kChunk ? &sm.q[r][pc] : &sm.v[r][pc];
+    const IN* src = (rr < kChunk ? q : v) + (tb + (size_t)r * H) * D + pc;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (r < it.len) x = *reinterpret_cast<const uint4*>(src);
+    *reinterpret_cast<uint4*>(dst) = x;
+  }
+  for (int i = threadIdx.x; i < kChunk; i += kFillThreads) {
+    float a = 0.f, b = 0.f;
+    if (i < it.len) {
+      a = step_decay(g[tb + (size_t)i * H]);
+      b = beta[tb + (size_t)i * H];
+    }
+    sm.a[i] = a;
+    sm.b[i] = b;
+  }
+}
+
+// Ask L2 for an item's boundary state and input rows.
+template <int D, class IN>
+__device__ __forceinline__ void fill_prefetch(const FillItem& it, const float* bstate,
+                                              const IN* q, const IN* k, const IN* v, int H) {
+  const int tid = threadIdx.x;
+  const size_t tb = (size_t)it.t0 * H + it.h;
+  if (tid == 0)
+    prefetch_l2(bstate + ((size_t)it.c * H + it.h) * D * D, (uint32_t)(D * D * sizeof(float)));
+  if (tid < 3 * kChunk) {
+    const int r = tid % kChunk;
+    const IN* src = (tid < kChunk ? k : tid < 2 * kChunk ? q : v) + (tb + (size_t)r * H) * D;
+    if (r < it.len) prefetch_l2(src, (uint32_t)(D * sizeof(IN)));
+  }
+}
+
 template <int D, class IN, class OUT>
-__global__ void __launch_bounds__(kFillThreads, 2)
+__global__ void __launch_bounds__(kFillThreads, 3)
     k_fill(const IN* __restrict__ q, const IN* __restrict__ k, const IN* __restrict__ v,
            const float* __restrict__ beta, const float* __restrict__ g,
            const int32_t* __restrict__ cu, int H, float scale, int32_t* __restrict__ hdr,
            const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
            const float* __restrict__ bstate, OUT* __restrict__ o,
-           float* __restrict__ s_run_final) {
+           float* __restrict__ s_run_final, float* __restrict__ s_run_scale) {
   constexpr int RT = D / 32, M4 = D / 16;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  FillStage<D, IN>* stages = reinterpret_cast<FillStage<D, IN>*>(smem_raw);
+  FillSmem<D, IN>& sm = *reinterpret_cast<FillSmem<D, IN>*>(smem_raw);
   __shared__ int sh_item;
   if (hdr[kHdrValid] != 1) return;
   const int n_items = hdr[kHdrChunks] * H;
@@ -303,75 +311,107 @@ __global__ void __launch_bounds__(kFillThreads, 2)
   if (tid == 0) sh_item = atomicAdd(&hdr[kHdrFillNext], 1);
   __syncthreads();
   int item = sh_item;
-  int bi = 0;
-  FillItem cur{};
-  if (item < n_items) {
-    cur = fill_item(item, H, cu, chunk_off, chunk_seq);
-    fill_stage_issue<D, IN>(stages[0], cur, q, k, v, beta, g, H);
-  }
   while (item < n_items) {
-    __syncthreads();  // every thread is done with stage bi^1 and has read sh_item
+    const FillItem cur = fill_item(item, H, cu, chunk_off, chunk_seq);
+    fill_load<D, IN>(sm, cur, q, k, v, beta, g, H);
+    Slice<RT, M4> S;
+    slice_load<RT, M4>(S, bstate + ((size_t)cur.c * H + cur.h) * DD, D, r0, l);
     if (tid == 0) sh_item = atomicAdd(&hdr[kHdrFillNext], 1);
     __syncthreads();
     const int next = sh_item;
-    FillItem nxt{};
-    if (next < n_items) {
-      nxt = fill_item(next, H, cu, chunk_off, chunk_seq);
-      fill_stage_issue<D, IN>(stages[bi ^ 1], nxt, q, k, v, beta, g, H);
-      if (tid == 0) prefetch_l2(bstate + ((size_t)nxt.c * H + nxt.h) * DD, (uint32_t)(DD * 4));
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    FillStage<D, IN>& st = stages[bi];
-    for (int i = tid; i < cur.len; i += kFillThreads) st.a[i] = step_decay(st.a[i]);
-    Slice<RT, M4> S;
-    slice_load<RT, M4>(S, bstate + ((size_t)cur.c * H + cur.h) * DD, D, r0, l);
-    __syncthreads();
+    if (next < n_items)
+      fill_prefetch<D, IN>(fill_item(next, H, cu, chunk_off, chunk_seq), bstate, q, k, v, H);
 
     float p[RT];
-    slice_dot<RT, M4>(S, [&](int m) { return sld4(&st.k[0][group_col(l, m)]); }, p);
+    slice_dot<RT, M4>(S, [&](int m) { return sld4(&sm.k[0][group_col(l, m)]); }, p);
 #pragma unroll
     for (int i = 0; i < RT; i++) p[i] = quad_sum(p[i]);
+    float c = 1.f;  // scale of the running state: 1 at the chunk boundary
     OUT* ob = o + ((size_t)cur.t0 * H + cur.h) * D + r0 + l;
     for (int t = 0; t < cur.len; t++) {
-      const float a = st.a[t], b = st.b[t];
-      float u[RT], oacc[RT], pacc[RT];
-#pragma unroll
-      for (int i = 0; i < RT; i++) u[i] = step_u(a, b, p[i], to_f(st.v[t][r0 + i]));
-      slice_update<true, RT, M4>(
-          S, a, u, [&](int m) { return sld4(&st.k[t][group_col(l, m)]); },
-          [&](int m) { return sld4(&st.q[t][group_col(l, m)]); },
-          [&](int m) { return sld4(&st.k[t + 1][group_col(l, m)]); }, oacc, pacc);
       float ov[RT];
+      slice_token<true, RT, M4>(
+          S, c, sm.a[t], sm.b[t], [&](int i) { return to_f(sm.v[t][r0 + i]); },
+          [&](int m) { return sld4(&sm.k[t][group_col(l, m)]); },
+          [&](int m) { return sld4(&sm.q[t][group_col(l, m)]); },
+          [&](int m) { return sld4(&sm.k[t + 1][group_col(l, m)]); }, p, ov);
 #pragma unroll
-      for (int i = 0; i < RT; i++) {
-        ov[i] = __fmul_rn(scale, quad_sum(oacc[i]));
-        p[i] = quad_sum(pacc[i]);
-      }
+      for (int i = 0; i < RT; i++) ov[i] = __fmul_rn(scale, ov[i]);
       if (l < RT) st1(ob + (size_t)t * H * D, pick<RT>(ov, l));
     }
     const int64_t nc = (cur.L + kChunk - 1) / kChunk;
-    if (s_run_final && cur.ci == nc - 1 && (cur.L % kChunk) != 0)
-      slice_store<RT, M4>(S, s_run_final + ((size_t)cur.n * H + cur.h) * DD, D, r0, l);
+    if (s_run_final && cur.ci == nc - 1 && (cur.L % kChunk) != 0) {
+      float* dst = s_run_final + ((size_t)cur.n * H + cur.h) * DD;
+      if (s_run_scale) {
+        slice_store<RT, M4>(S, dst, D, r0, l);
+        if (tid == 0) s_run_scale[(size_t)cur.n * H + cur.h] = c;
+      } else {
+        slice_store_scaled<RT, M4>(S, c, dst, D, r0, l);
+      }
+    }
     item = next;
-    cur = nxt;
-    bi ^= 1;
+    __syncthreads();  // shared memory is reloaded for the next item
   }
 }
 
 // ----------------------------------------------------------------------------
-// Decode step
+// Chunk boundary over a buffer: decode resync (RESYNC) or gdn_chunk_boundary
 // ----------------------------------------------------------------------------
+template <int D, class IN>
+struct BndSmem {
+  PrepSmem<D, IN> prep;
+  __nv_bfloat16 V[Splits<IN>::K][kChunk][D + 8];
+};
+
+// One chunk boundary for `unit` (prep + walk of all D rows), in place allowed.
+template <int D, class IN>
+__device__ __forceinline__ void bnd_unit(BndSmem<D, IN>& sm, const float* s_start, const IN* kb,
+                                         const IN* vb, const float* bb, const float* gb,
+                                         size_t unit, float* s_end) {
+  const size_t DD = (size_t)D * D;
+  stage_planes<D, IN>(sm.V, vb + unit * kChunk * D, (size_t)D, kBndThreads);
+  prep_stage<D, IN>(sm.prep, kb + unit * kChunk * D, (size_t)D, bb + unit * kChunk,
+                    gb + unit * kChunk, 1);
+  bnd_prep<D, IN>(sm.prep);
+  const int warp = threadIdx.x >> 5;
+#pragma unroll 1
+  for (int rt = 0; rt < D / 64; rt++) {
+    const int r0 = 16 * warp + 64 * rt;
+    float sacc[D / 8][4];
+    sacc_load<D>(sacc, s_start + unit * DD, r0);
+    bnd_walk_warp<D, IN>(sacc, sm.prep.head, &sm.prep.K[0][0][0], &sm.V[0][0][0], r0);
+    sacc_store<D>(sacc, s_end + unit * DD, r0);
+  }
+  __syncthreads();  // shared memory is reused by the next unit
+}
+
+// gdn_chunk_boundary: one block per (row, head).
+template <int D, class IN>
+__global__ void __launch_bounds__(kBndThreads)
+    k_bnd(const float* s_start, const IN* __restrict__ kb, const IN* __restrict__ vb,
+          const float* __restrict__ bb, const float* __restrict__ gb, int H, float* s_end) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  BndSmem<D, IN>& sm = *reinterpret_cast<BndSmem<D, IN>*>(smem_raw);
+  bnd_unit<D, IN>(sm, s_start, kb, vb, bb, gb, (size_t)blockIdx.x * H + blockIdx.y, s_end);
+}
+
+// ----------------------------------------------------------------------------
+// Decode step: one block per (row, head) unit.  The block that appends the
+// last token of a chunk then runs the chunk boundary for its unit (the
+// resync), while the other units' blocks are still stepping.
+// ----------------------------------------------------------------------------
+constexpr int kDecThreads = 128;  // four state rows per thread
+
 template <int D, class IN, class OUT>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kDecThreads)
     k_dec_step(const IN* __restrict__ q, const IN* __restrict__ k, const IN* __restrict__ v,
                const float* __restrict__ beta, const float* __restrict__ g,
                const int32_t* __restrict__ slot_idx, int H, float scale, float* s_run,
-               const float* s_bnd, IN* buf_k, IN* buf_v, float* buf_beta, float* buf_g,
-               int32_t* pos, int32_t* error, int n_slots, OUT* __restrict__ o) {
+               float* s_scale, float* s_bnd, IN* buf_k, IN* buf_v, float* buf_beta,
+               float* buf_g, int32_t* pos, int32_t* error, int n_slots, OUT* __restrict__ o) {
+  static_assert(kDecThreads == kBndThreads, "the resync runs in the step's block");
   constexpr int RT = D / 32, M4 = D / 16;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int sh_pos, sh_slot;
   const int b = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * RT;
@@ -398,81 +438,42 @@ __global__ void __launch_bounds__(128)
   const IN* qp = q + tok * D;
   const float a = step_decay(g[tok]);
   const float bt = beta[tok];
-  float p[RT], u[RT], oacc[RT], pacc[RT];
-  slice_dot<RT, M4>(S, [&](int m) { return ld4(kp + group_col(l, m)); }, p);
+  float c = (p0 == 0) ? 1.f : s_scale[unit];
+  float p[RT], ov[RT];
+  auto kf = [&](int m) { return ld4(kp + group_col(l, m)); };
+  slice_dot<RT, M4>(S, kf, p);
 #pragma unroll
-  for (int i = 0; i < RT; i++) {
-    p[i] = quad_sum(p[i]);
-    u[i] = step_u(a, bt, p[i], ld1(v + tok * D + r0 + i));
-  }
-  slice_update<false, RT, M4>(
-      S, a, u, [&](int m) { return ld4(kp + group_col(l, m)); },
+  for (int i = 0; i < RT; i++) p[i] = quad_sum(p[i]);
+  slice_token<false, RT, M4>(
+      S, c, a, bt, [&](int i) { return ld1(v + tok * D + r0 + i); }, kf,
       [&](int m) { return ld4(qp + group_col(l, m)); },
-      [&](int m) { return make_float4(0.f, 0.f, 0.f, 0.f); }, oacc, pacc);
-  float ov[RT];
+      [&](int m) { return make_float4(0.f, 0.f, 0.f, 0.f); }, p, ov);
 #pragma unroll
-  for (int i = 0; i < RT; i++) ov[i] = __fmul_rn(scale, quad_sum(oacc[i]));
+  for (int i = 0; i < RT; i++) ov[i] = __fmul_rn(scale, ov[i]);
   if (l < RT) st1(o + tok * D + r0 + l, pick<RT>(ov, l));
-  if (p0 + 1 < kChunk) slice_store<RT, M4>(S, s_run + unit * DD, D, r0, l);
+  if (p0 + 1 < kChunk) {
+    slice_store<RT, M4>(S, s_run + unit * DD, D, r0, l);
+    if (tid == 0) s_scale[unit] = c;
+  }
   // append the token to the chunk buffer (bit copies)
   const size_t brow = (unit * kChunk + p0) * D;
-  for (int e = tid; e < D; e += 128) {
+  for (int e = tid; e < D; e += kDecThreads) {
     buf_k[brow + e] = k[tok * D + e];
     buf_v[brow + e] = v[tok * D + e];
   }
   if (tid == 0) {
     buf_beta[unit * kChunk + p0] = bt;
     buf_g[unit * kChunk + p0] = g[tok];
-    pos[unit] = p0 + 1;  // kChunk here means "resync pending" until k_bnd runs
+    if (p0 + 1 < kChunk) pos[unit] = p0 + 1;
   }
-}
-
-// ----------------------------------------------------------------------------
-// Chunk boundary over a buffer: decode resync (RESYNC) or gdn_chunk_boundary
-// ----------------------------------------------------------------------------
-template <int D, class IN>
-struct BndSmem {
-  PrepSmem<D, IN> prep;
-  __nv_bfloat16 V[Splits<IN>::K][kChunk][D + 8];
-};
-
-template <int D, class IN, bool RESYNC>
-__global__ void __launch_bounds__(kBndThreads)
-    k_bnd(const float* s_start, const IN* __restrict__ kb, const IN* __restrict__ vb,
-          const float* __restrict__ bb, const float* __restrict__ gb,
-          const int32_t* __restrict__ slot_idx, int H, int32_t* pos, int n_slots,
-          float* s_end) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  BndSmem<D, IN>& sm = *reinterpret_cast<BndSmem<D, IN>*>(smem_raw);
-  __shared__ int sh_go;
-  const int b = blockIdx.x, h = blockIdx.y;
-  size_t unit = (size_t)b * H + h;
-  if (RESYNC) {
-    if (threadIdx.x == 0) {
-      const int slot = slot_idx ? slot_idx[b] : b;
-      int go = 0;
-      if (slot >= 0 && slot < n_slots) go = (pos[(size_t)slot * H + h] == kChunk);
-      sh_go = go ? 1 + slot : 0;
-    }
-    __syncthreads();
-    if (sh_go == 0) return;
-    unit = (size_t)(sh_go - 1) * H + h;
+  if (p0 + 1 == kChunk) {
+    // The buffer is full: advance the boundary state over its C tokens.  The
+    // running state of the next step is the new boundary state (pos = 0).
+    __syncthreads();  // the appended token is visible to the whole block
+    BndSmem<D, IN>& sm = *reinterpret_cast<BndSmem<D, IN>*>(smem_raw);
+    bnd_unit<D, IN>(sm, s_bnd, buf_k, buf_v, buf_beta, buf_g, unit, s_bnd);
+    if (tid == 0) pos[unit] = 0;
   }
-  const size_t DD = (size_t)D * D;
-  stage_planes<D, IN>(sm.V, vb + unit * kChunk * D, (size_t)D, kBndThreads);
-  prep_stage<D, IN>(sm.prep, kb + unit * kChunk * D, (size_t)D, bb + unit * kChunk,
-                    gb + unit * kChunk, 1);
-  bnd_prep<D, IN>(sm.prep);
-  const int warp = threadIdx.x >> 5;
-#pragma unroll 1
-  for (int rt = 0; rt < D / 64; rt++) {
-    const int r0 = 16 * warp + 64 * rt;
-    float sacc[D / 8][4];
-    sacc_load<D>(sacc, s_start + unit * DD, r0);
-    bnd_walk_warp<D, IN>(sacc, sm.prep.head, &sm.prep.K[0][0][0], &sm.V[0][0][0], r0);
-    sacc_store<D>(sacc, s_end + unit * DD, r0);
-  }
-  if (RESYNC && threadIdx.x == 0) pos[unit] = 0;
 }
 
 // ----------------------------------------------------------------------------
@@ -482,8 +483,9 @@ template <int D, class IN>
 __global__ void __launch_bounds__(128)
     k_handoff(const IN* __restrict__ k, const IN* __restrict__ v, const float* __restrict__ beta,
               const float* __restrict__ g, const int32_t* __restrict__ cu, int64_t T, int H,
-              const float* __restrict__ s_run_final, const float* __restrict__ s_bnd_final,
-              const int32_t* __restrict__ slot_idx, float* s_run, float* s_bnd, IN* buf_k,
+              const float* __restrict__ s_run_final, const float* __restrict__ s_run_scale,
+              const float* __restrict__ s_bnd_final, const int32_t* __restrict__ slot_idx,
+              float* s_run, float* s_scale, float* s_bnd, IN* buf_k,
               IN* buf_v, float* buf_beta, float* buf_g, int32_t* pos, int32_t* error,
               int n_slots) {
   const int n = blockIdx.x, h = blockIdx.y;
@@ -513,7 +515,10 @@ __global__ void __launch_bounds__(128)
     buf_beta[unit * kChunk + i] = beta[t * H + h];
     buf_g[unit * kChunk + i] = g[t * H + h];
   }
-  if (threadIdx.x == 0) pos[unit] = rem;
+  if (threadIdx.x == 0) {
+    pos[unit] = rem;
+    s_scale[unit] = s_run_scale ? s_run_scale[src] : 1.f;
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -578,13 +583,13 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     GDN_TRY(set_smem(kern, sm));
     kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), walk_threads<D>(), sm, st>>>(
         k, v, a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final,
-        a.s_bnd_final);
+        a.s_run_scale, a.s_bnd_final);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(3));
   {
     auto kern = k_fill<D, IN, OUT>;
-    const size_t sm = 2 * sizeof(FillStage<D, IN>);
+    const size_t sm = sizeof(FillSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
     int grid = 0;
     GDN_TRY(persistent_grid(kern, kFillThreads, sm, &grid));
@@ -592,7 +597,7 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     if ((int64_t)grid > items) grid = (int)items;
     kern<<<grid, kFillThreads, sm, st>>>(q, k, v, a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
                                          chunk_off, chunk_seq, bstate, static_cast<OUT*>(a.o),
-                                         a.s_run_final);
+                                         a.s_run_final, a.s_run_scale);
     GDN_TRY(cudaGetLastError());
   }
   return mark(4);
@@ -600,19 +605,14 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
 
 template <int D, class IN, class OUT>
 static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
-  const dim3 grid((unsigned)a.B, (unsigned)a.H);
-  k_dec_step<D, IN, OUT><<<grid, 128, 0, st>>>(
-      static_cast<const IN*>(a.q), static_cast<const IN*>(a.k), static_cast<const IN*>(a.v),
-      a.beta, a.g, a.slot_idx, a.H, a.scale, a.s_run, a.s_bnd, static_cast<IN*>(a.buf_k),
-      static_cast<IN*>(a.buf_v), a.buf_beta, a.buf_g, a.pos, a.error, a.n_slots,
-      static_cast<OUT*>(a.o));
-  GDN_TRY(cudaGetLastError());
-  auto kern = k_bnd<D, IN, true>;
+  auto kern = k_dec_step<D, IN, OUT>;
   const size_t sm = sizeof(BndSmem<D, IN>);
   GDN_TRY(set_smem(kern, sm));
-  kern<<<grid, kBndThreads, sm, st>>>(a.s_bnd, static_cast<const IN*>(a.buf_k),
-                                      static_cast<const IN*>(a.buf_v), a.buf_beta, a.buf_g,
-                                      a.slot_idx, a.H, a.pos, a.n_slots, a.s_bnd);
+  kern<<<dim3((unsigned)a.B, (unsigned)a.H), kDecThreads, sm, st>>>(
+      static_cast<const IN*>(a.q), static_cast<const IN*>(a.k), static_cast<const IN*>(a.v),
+      a.beta, a.g, a.slot_idx, a.H, a.scale, a.s_run, a.s_scale, a.s_bnd,
+      static_cast<IN*>(a.buf_k), static_cast<IN*>(a.buf_v), a.buf_beta, a.buf_g, a.pos, a.error,
+      a.n_slots, static_cast<OUT*>(a.o));
   return cudaGetLastError();
 }
 
@@ -620,7 +620,7 @@ template <int D, class IN>
 static cudaError_t handoff_impl(const HandoffArgs& a, cudaStream_t st) {
   k_handoff<D, IN><<<dim3((unsigned)a.n_seqs, (unsigned)a.H), 128, 0, st>>>(
       static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, a.cu_seqlens, a.T,
-      a.H, a.s_run_final, a.s_bnd_final, a.slot_idx, a.s_run, a.s_bnd,
+      a.H, a.s_run_final, a.s_run_scale, a.s_bnd_final, a.slot_idx, a.s_run, a.s_scale, a.s_bnd,
       static_cast<IN*>(a.buf_k), static_cast<IN*>(a.buf_v), a.buf_beta, a.buf_g, a.pos,
       a.error, a.n_slots);
   return cudaGetLastError();
@@ -628,12 +628,12 @@ static cudaError_t handoff_impl(const HandoffArgs& a, cudaStream_t st) {
 
 template <int D, class IN>
 static cudaError_t boundary_impl(const BndArgs& a, cudaStream_t st) {
-  auto kern = k_bnd<D, IN, false>;
+  auto kern = k_bnd<D, IN>;
   const size_t sm = sizeof(BndSmem<D, IN>);
   GDN_TRY(set_smem(kern, sm));
   kern<<<dim3((unsigned)a.B, (unsigned)a.H), kBndThreads, sm, st>>>(
-      a.s_start, static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, nullptr,
-      a.H, nullptr, 0, a.s_end);
+      a.s_start, static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, a.H,
+      a.s_end);
   return cudaGetLastError();
 }
 

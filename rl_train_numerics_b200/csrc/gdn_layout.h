@@ -71,6 +71,7 @@ struct FwdArgs {
   void* o;
   int out_bf16;
   float* s_run_final;
+  float* s_run_scale;
   float* s_bnd_final;
   char* ws;
   FwdLayout lay;
@@ -88,6 +89,7 @@ struct DecArgs {
   int B, H, D;
   float scale;
   float* s_run;
+  float* s_scale;
   float* s_bnd;
   void* buf_k;
   void* buf_v;
@@ -111,9 +113,11 @@ struct HandoffArgs {
   int64_t T;
   int H, D;
   const float* s_run_final;
+  const float* s_run_scale;
   const float* s_bnd_final;
   const int32_t* slot_idx;
   float* s_run;
+  float* s_scale;
   float* s_bnd;
   void* buf_k;
   void* buf_v;

@@ -61,16 +61,17 @@ extern "C" int gdn_cpr_forward_noalloc(const void* q, const void* k, const void*
                                        const int32_t* cu_seqlens, int n_seqs,
                                        int64_t total_tokens, int H, int dk, int dv, int C,
                                        float scale, const float* h0, void* o, int out_dtype,
-                                       float* s_run_final, float* s_bnd_final,
-                                       int32_t* error_word, void* stream) {
+                                       float* s_run_final, float* s_run_scale,
+                                       float* s_bnd_final, int32_t* error_word,
+                                       void* stream) {
   const size_t need = gdn_cpr_forward_workspace_bytes(n_seqs, total_tokens, H, dk, dv, C,
                                                       in_dtype);
   if (need == 0 || n_seqs == 0) {
     // Rejected shapes, or an empty batch: the regular entry point reports the
     // exact status (or returns GDN_OK for an empty batch) without device work.
     return gdn_cpr_forward_ex(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs, total_tokens, H,
-                              dk, dv, C, scale, h0, o, out_dtype, s_run_final, s_bnd_final,
-                              nullptr, 0, nullptr, stream);
+                              dk, dv, C, scale, h0, o, out_dtype, s_run_final, s_run_scale,
+                              s_bnd_final, nullptr, 0, nullptr, stream);
   }
   if (need > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;  // beyond the fixed scratch
   void* scratch = nullptr;
@@ -79,8 +80,8 @@ extern "C" int gdn_cpr_forward_noalloc(const void* q, const void* k, const void*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(scratch, 0, sizeof(int32_t), st) != cudaSuccess) return GDN_ERR_CUDA;
   rc = gdn_cpr_forward_ex(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs, total_tokens, H, dk,
-                          dv, C, scale, h0, o, out_dtype, s_run_final, s_bnd_final, scratch,
-                          GDN_NOALLOC_SCRATCH_BYTES, nullptr, stream);
+                          dv, C, scale, h0, o, out_dtype, s_run_final, s_run_scale, s_bnd_final,
+                          scratch, GDN_NOALLOC_SCRATCH_BYTES, nullptr, stream);
   if (rc != GDN_OK || error_word == nullptr) return rc;
   if (cudaMemcpyAsync(error_word, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
       cudaSuccess)

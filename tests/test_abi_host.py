@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert gdn.lib.gdn_cpr_abi_version() == 1
+    assert gdn.lib.gdn_cpr_abi_version() == 2
     for code in range(-6, 1):
         assert gdn.status_string(code).startswith("GDN_")
     assert "unknown" in gdn.status_string(42)
@@ -68,12 +68,13 @@ def test_workspace_query():
 def fwd(**over):
     a = dict(q=FAKE, k=FAKE, v=FAKE, in_dtype=gdn.GDN_BF16, beta=FAKE, g=FAKE, cu=FAKE, N=2,
              T=128, H=2, dk=64, dv=64, C=64, scale=1.0, h0=None, o=FAKE,
-             out_dtype=gdn.GDN_BF16, srun=None, sbnd=None, ws=FAKE, wsb=1 << 40, stream=None)
+             out_dtype=gdn.GDN_BF16, srun=None, sscale=None, sbnd=None, ws=FAKE, wsb=1 << 40,
+             stream=None)
     a.update(over)
     return gdn.lib.gdn_cpr_forward(a["q"], a["k"], a["v"], a["in_dtype"], a["beta"], a["g"],
                                    a["cu"], a["N"], a["T"], a["H"], a["dk"], a["dv"], a["C"],
                                    a["scale"], a["h0"], a["o"], a["out_dtype"], a["srun"],
-                                   a["sbnd"], a["ws"], a["wsb"], a["stream"])
+                                   a["sscale"], a["sbnd"], a["ws"], a["wsb"], a["stream"])
 
 
 @pytest.mark.parametrize("over,expect", [
@@ -95,6 +96,8 @@ def fwd(**over):
     (dict(o=MIS), gdn.GDN_ERR_INVALID_ARG),
     (dict(h0=MIS), gdn.GDN_ERR_INVALID_ARG),
     (dict(srun=MIS), gdn.GDN_ERR_INVALID_ARG),
+    (dict(sscale=FAKE), gdn.GDN_ERR_INVALID_ARG),            # scale without a state buffer
+    (dict(srun=FAKE, sscale=MIS + 2), gdn.GDN_ERR_INVALID_ARG),
     (dict(ws=None), gdn.GDN_ERR_WORKSPACE),
     (dict(wsb=1024), gdn.GDN_ERR_WORKSPACE),
     (dict(N=0, T=5), gdn.GDN_ERR_INVALID_ARG),
@@ -109,11 +112,11 @@ def test_forward_empty_batch_is_a_no_op():
 
 
 def _state(**over):
-    f = dict(s_run=FAKE, s_bnd=FAKE, buf_k=FAKE, buf_v=FAKE, buf_beta=FAKE, buf_g=FAKE,
-             pos=FAKE, error=FAKE, n_slots=4)
+    f = dict(s_run=FAKE, s_scale=FAKE, s_bnd=FAKE, buf_k=FAKE, buf_v=FAKE, buf_beta=FAKE,
+             buf_g=FAKE, pos=FAKE, error=FAKE, n_slots=4)
     f.update(over)
-    return gdn.DecodeStateStruct(f["s_run"], f["s_bnd"], f["buf_k"], f["buf_v"], f["buf_beta"],
-                                 f["buf_g"], f["pos"], f["error"], f["n_slots"])
+    return gdn.DecodeStateStruct(f["s_run"], f["s_scale"], f["s_bnd"], f["buf_k"], f["buf_v"],
+                                 f["buf_beta"], f["buf_g"], f["pos"], f["error"], f["n_slots"])
 
 
 def dec(st=None, **over):
@@ -134,6 +137,7 @@ def dec(st=None, **over):
     (dict(o=MIS), {}, gdn.GDN_ERR_INVALID_ARG),
     ({}, dict(s_run=None), gdn.GDN_ERR_INVALID_ARG),
     ({}, dict(pos=None), gdn.GDN_ERR_INVALID_ARG),
+    ({}, dict(s_scale=None), gdn.GDN_ERR_INVALID_ARG),
     ({}, dict(error=None), gdn.GDN_ERR_INVALID_ARG),
     ({}, dict(s_bnd=MIS), gdn.GDN_ERR_INVALID_ARG),
     ({}, dict(n_slots=0), gdn.GDN_ERR_INVALID_ARG),
@@ -158,10 +162,10 @@ def test_boundary_and_handoff_reject_on_host():
     assert L.gdn_chunk_boundary(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 0, 2, 64, 64, 64, FAKE,
                                 None) == gdn.GDN_OK
     assert L.gdn_cpr_decode_state_from_prefill(
-        FAKE, FAKE, 0, FAKE, FAKE, FAKE, 8, 100, 2, 64, 64, 64, FAKE, FAKE, None,
+        FAKE, FAKE, 0, FAKE, FAKE, FAKE, 8, 100, 2, 64, 64, 64, FAKE, None, FAKE, None,
         _state(n_slots=4), None) == gdn.GDN_ERR_INVALID_ARG  # 8 sequences, 4 slots
     assert L.gdn_cpr_decode_state_from_prefill(
-        FAKE, FAKE, 0, FAKE, FAKE, FAKE, 2, 100, 2, 64, 64, 64, None, FAKE, None,
+        FAKE, FAKE, 0, FAKE, FAKE, FAKE, 2, 100, 2, 64, 64, 64, None, None, FAKE, None,
         _state(), None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_check_error(None, None, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_check_error(MIS + 1, None, None) == gdn.GDN_ERR_INVALID_ARG

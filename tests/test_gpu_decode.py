@@ -45,12 +45,20 @@ def decode_tokens_of(full: W.Batch, prefix_lens, step):
             full.beta[idx].contiguous(), full.g[idx].contiguous())
 
 
+def prefill_pair(gdn, pre, out_dtype=torch.float32):
+    """Forward returning the exact running-state pair (mantissa, scale)."""
+    scale = torch.empty((len(pre.lengths), pre.q.shape[1]), device=pre.q.device)
+    o, srun, sbnd = forward(gdn, pre, out_dtype=out_dtype, s_run_scale=scale)
+    return o, srun, scale, sbnd
+
+
 def run_prefill_then_decode(gdn, full, prefix_lens, n_steps, out_dtype=torch.float32):
     H, d = full.q.shape[1], full.q.shape[2]
     pre = split_batch(full, prefix_lens)
-    o_pre, srun, sbnd = forward(gdn, pre, out_dtype=out_dtype)
+    o_pre, srun, sscale, sbnd = prefill_pair(gdn, pre, out_dtype=out_dtype)
     st = gdn.DecodeState(len(prefix_lens), H, d, d, in_dtype=full.q.dtype)
-    gdn.decode_state_from_prefill(st, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens, srun, sbnd)
+    gdn.decode_state_from_prefill(st, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens, srun, sbnd,
+                                  s_run_scale=sscale)
     outs = []
     for s in range(n_steps):
         q, k, v, beta, g = decode_tokens_of(full, prefix_lens, s)
@@ -142,12 +150,12 @@ def test_decode_slot_order_invariance(gdn):
     full = W.make_batch([L + 70 for L in lens], 2, 128, 128, seed=24).to("cuda")
     _, o_ref, _ = run_prefill_then_decode(gdn, full, lens, 70)
     pre = split_batch(full, lens)
-    _, srun, sbnd = forward(gdn, pre, out_dtype=torch.float32)
+    _, srun, sscale, sbnd = prefill_pair(gdn, pre)
     perm = [3, 0, 4, 2, 1]
     st = gdn.DecodeState(5, 2, 128, 128)
     slot_of_seq = torch.tensor(perm, dtype=torch.int32, device="cuda")
     gdn.decode_state_from_prefill(st, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens, srun, sbnd,
-                                  slot_idx=slot_of_seq)
+                                  s_run_scale=sscale, slot_idx=slot_of_seq)
     rev = list(reversed(range(5)))  # present the rows in reverse sequence order
     rows = torch.tensor([perm[n] for n in rev], dtype=torch.int32, device="cuda")
     for s in range(70):
@@ -163,9 +171,10 @@ def test_decode_state_save_restore(gdn):
     lens = [40, 100]
     full = W.make_batch([L + 80 for L in lens], 2, 64, 64, seed=25).to("cuda")
     pre = split_batch(full, lens)
-    _, srun, sbnd = forward(gdn, pre, out_dtype=torch.float32)
+    _, srun, sscale, sbnd = prefill_pair(gdn, pre)
     st = gdn.DecodeState(2, 2, 64, 64)
-    gdn.decode_state_from_prefill(st, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens, srun, sbnd)
+    gdn.decode_state_from_prefill(st, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens, srun, sbnd,
+                                  s_run_scale=sscale)
     for s in range(30):
         gdn.decode_step(st, *decode_tokens_of(full, lens, s))
     saved = [t.cpu() for t in st.tensors()]

@@ -164,3 +164,30 @@ def test_chunk_boundary_matches_forward_bits(gdn, d, dtype):
     S2 = S.cuda().clone()
     gdn.chunk_boundary(S2, kc, vc, bc, gc, s_end=S2)
     assert torch.equal(S2, out)
+
+
+def test_running_state_pair(gdn):
+    """With s_run_scale the forward returns (mantissa, scale); scale x mantissa,
+    rounded once, is bit for bit the state returned without it."""
+    lens = [100, 64, 1, 190]
+    b = W.make_batch(lens, 4, 128, 128, seed=18).to("cuda")
+    _, s_state, _ = run(gdn, b)
+    scale = torch.full((4, 4), float("nan"), device="cuda")
+    _, s_mant, _ = run(gdn, b, s_run_scale=scale)
+    assert torch.isfinite(scale).all()
+    assert torch.equal(scale[1], torch.ones(4, device="cuda"))  # chunk-aligned end
+    assert torch.equal(scale[:, :, None, None] * s_mant, s_state)
+
+
+def test_hard_reset_tokens(gdn):
+    """g = -1e4 makes exp(g) exactly 0 (a reset) at scattered tokens; long decays
+    (g = -8 runs) force the scaled state to renormalise many times."""
+    lens = [200, 64, 77]
+    b = W.make_batch(lens, 2, 128, 128, seed=19)
+    gen = torch.Generator().manual_seed(20)
+    pick = torch.rand(b.g.shape, generator=gen)
+    g = torch.where(pick < 0.03, torch.full_like(b.g, -1e4), b.g)
+    g = torch.where((pick >= 0.03) & (pick < 0.3), torch.full_like(b.g, -8.0), g)
+    b = W.Batch(b.q, b.k, b.v, b.beta, g.contiguous(), b.cu_seqlens, b.lengths)
+    o, srun, sbnd = run(gdn, b.to("cuda"), out_dtype=torch.float32)
+    check_units(gdn, b, o, srun, sbnd, [(n, h) for n in range(3) for h in range(2)])

@@ -27,9 +27,9 @@ def stress():
     return W.stress()
 
 
-def forward(gdn, b):
+def forward(gdn, b, **kw):
     o, srun, sbnd, ws = gdn.forward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens,
-                                    out_dtype=torch.float32)
+                                    out_dtype=torch.float32, **kw)
     assert gdn.check_error(ws) == 0
     return o, srun, sbnd
 
@@ -92,11 +92,13 @@ def test_decode_batch_invariance(gdn, stress):
     H = b.q.shape[1]
     steps = 128
     toks = W.decode_tokens(steps, n, H, 128, 128, seed=33, g_mode="stress", device="cuda")
-    _, srun, sbnd = forward(gdn, b)
+    sscale = torch.empty((n, H), device="cuda")
+    _, srun, sbnd = forward(gdn, b, s_run_scale=sscale)
 
     def decode(order):
         st = gdn.DecodeState(n, H, 128, 128)
-        gdn.decode_state_from_prefill(st, b.k, b.v, b.beta, b.g, b.cu_seqlens, srun, sbnd)
+        gdn.decode_state_from_prefill(st, b.k, b.v, b.beta, b.g, b.cu_seqlens, srun, sbnd,
+                                      s_run_scale=sscale)
         slots = torch.tensor(order, dtype=torch.int32, device="cuda")
         r = torch.tensor(order, device="cuda")
         outs = []

@@ -40,7 +40,7 @@ def call_noalloc(gdn, b, o, srun, sbnd, err):
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     return gdn.lib.gdn_cpr_forward_noalloc(
         p(b.q), p(b.k), p(b.v), in_code, p(b.beta), p(b.g), p(b.cu_seqlens), len(b.lengths), T,
-        H, d, d, 64, 1.0, None, p(o), out_code, p(srun), p(sbnd), p(err), stream)
+        H, d, d, 64, 1.0, None, p(o), out_code, p(srun), None, p(sbnd), p(err), stream)
 
 
 def regular(gdn, b):
