@@ -40,6 +40,26 @@ FLUSH_BYTES = 256 << 20
 PAGES_H100 = {"prefill_ms": 1.412, "decode_ms": 0.0846, "trainer_fwd_bwd_ms": 7.386}
 
 
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when
+    the kernel sources have changed since that capture."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            rec = json.load(f)
+        csrc = os.path.join(ROOT, "rl_train_numerics_b200", "csrc")
+        h = hashlib.sha256()
+        for name in sorted(os.listdir(csrc)):
+            if name.endswith((".cu", ".cuh", ".h")):
+                with open(os.path.join(csrc, name), "rb") as f:
+                    h.update(f.read())
+        if h.hexdigest() != rec.get("kernel_sources_sha256"):
+            return None
+        return rec.get("traffic_bytes", {}).get(kernel)
+    except (OSError, ValueError):
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -58,9 +78,9 @@ def load_peaks():
 # ----------------------------------------------------------------------------
 
 def fill_flops(T, H_, d):
-    """Intra-chunk fill: per token and head 7 d^2 FP32 flops (p: d^2 FMA; update:
-    d^2 MUL + d^2 FMA; o: d^2 FMA; an FMA counts 2)."""
-    return 7.0 * d * d * T * H_
+    """Intra-chunk fill: per token and head 3 d^2 fused multiply-adds = 6 d^2 flops
+    (the dot with k, the rank-one update of the scaled state, the dot with q)."""
+    return 6.0 * d * d * T * H_
 
 
 def walk_flops(n_full_chunk_heads, d, c=C):
@@ -177,12 +197,19 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank number over all ranks (device tensor for NCCL, host for gloo)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, max_ms: float, world: int) -> float:
+    """Whole-job throughput: units all ranks processed / the slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1e3)
 
 
 # ----------------------------------------------------------------------------
@@ -366,7 +393,7 @@ def run_ours(args):
     ms_step = max_over_ranks(total / args.steps, world)
     per_k /= args.steps
     T = b.total_tokens
-    value = world * T / (ms_step / 1e3)
+    value = weak_scaling_value(T, ms_step, world)
 
     lens = b.lengths
     full = sum(L // C for L in lens) * H
@@ -382,7 +409,7 @@ def run_ours(args):
     achieved = flops / (per_k[dom] / 1e3) / 1e12
     roofline = {"kernel": dom_name, "bound": bound, "achieved": round(achieved, 2),
                 "peak": round(fp32_peak, 2), "unit": "TFLOP/s",
-                "frac": round(achieved / fp32_peak, 4), "traffic": None,
+                "frac": round(achieved / fp32_peak, 4), "traffic": ncu_traffic(dom_name),
                 "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x sm_max_mhz (nominal)"}
     minimal, two_pass = prefill_bytes(lens, H, D)
     hbm = {"minimal_bytes": minimal, "two_pass_bytes": two_pass,
