@@ -68,6 +68,7 @@ typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
 /* Bits of the device error word. */
 #define GDN_DEVERR_CU_SEQLENS 1 /* cu_seqlens not 0-based, not nondecreasing or wrong total */
 #define GDN_DEVERR_POS 2        /* a decode position outside [0, C) */
+#define GDN_DEVERR_TIMEOUT 4    /* a bounded tensor-core completion wait gave up */
 
 /* ABI version of the loaded library (GDN_CPR_ABI_VERSION it was built with). */
 int gdn_cpr_abi_version(void);

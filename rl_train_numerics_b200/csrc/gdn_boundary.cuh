@@ -47,6 +47,9 @@
 
 #include "gdn_common.cuh"
 #include "gdn_mma.cuh"
+#include "gdn_umma.cuh"
+
+#include <type_traits>
 
 namespace gdn {
 
@@ -72,58 +75,72 @@ constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // What the walk needs from the prep of one (chunk, head): the walk pack.  It
 // is copied as raw bytes (global <-> shared), so its layout is the shared
-// memory layout: bf16 planes with padded rows (bank-conflict-free ldmatrix).
+// memory layout.  Tb and Tv are stored transposed, in the core-matrix layout
+// of gdn_umma.cuh with 64 rows: TbT[q][core_off<64>(j, i)] is split term q of
+// Tb_ij (zero above the diagonal, j > i).
 template <int D, class IN>
 struct PackHead {
   static constexpr int NW = Splits<IN>::W;
-  static constexpr int LDT = kChunk + 8;
-  __nv_bfloat16 Tb[NW][kChunk][LDT];
-  __nv_bfloat16 Tv[NW][kChunk][LDT];
+  __nv_bfloat16 TbT[NW][kChunk * kChunk];
+  __nv_bfloat16 TvT[NW][kChunk * kChunk];
   float dvec[kChunk];
   float gamma[4];  // [0] = exp(G_C)
 };
 
-// Keys and values of one chunk as bf16 term planes (padded rows).
+// Keys and values of one chunk as bf16 term planes, core-matrix layout with
+// 64 rows (token i) and D columns (channel): plane[core_off<64>(i, c)].
 template <int D, class IN>
 struct KVPlanes {
   static constexpr int NK = Splits<IN>::K;
-  static constexpr int LDB = D + 8;
-  __nv_bfloat16 K[NK][kChunk][LDB];
-  __nv_bfloat16 V[NK][kChunk][LDB];
+  __nv_bfloat16 K[NK][kChunk * D];
+  __nv_bfloat16 V[NK][kChunk * D];
+};
+
+// The walk's input for one (chunk, head), written by the prep and read back
+// with one bulk copy: the pack head and the chunk's key and value planes.
+template <int D, class IN>
+struct WalkPack {
+  PackHead<D, IN> head;
+  KVPlanes<D, IN> kv;
 };
 
 template <int D, class IN>
 constexpr size_t pack_size() {
-  return round_up(sizeof(PackHead<D, IN>), 128);
+  return round_up(sizeof(WalkPack<D, IN>), 128);
 }
 
-// Shared memory of the prep.  AT holds A transposed with padded columns:
-// AT[m][i] = A_im for i > m (zero elsewhere), so a column of A is contiguous.
+// Shared memory of the prep, apart from its scratch matrix AT (PrepAT), which
+// callers place where it can share space with later work.
 template <int D, class IN>
 struct PrepSmem {
   static constexpr int NW = Splits<IN>::W, NK = Splits<IN>::K;
-  static constexpr int LDB = D + 8;
   PackHead<D, IN> head;
-  __nv_bfloat16 K[NK][kChunk][LDB];
-  float AT[kChunk][kChunk];
+  __nv_bfloat16 K[NK][kChunk * D];
   double G[kChunk];
   float beta[kChunk];
   float g[kChunk];
   float bg[kChunk];
 };
+// AT[m][i] = A_im for i > m (zero elsewhere): a column of A is contiguous.
+using PrepAT = float[kChunk][kChunk];
 
-// Stage the rows of a [C][D] block (row stride ld elements) into bf16 term
-// planes: bf16 inputs are copied with cp.async (the caller commits and waits),
-// fp32 inputs are split into three bf16 terms with plain loads and stores.
+// The rows of a [C][D] block (row stride ld elements) as bf16 term planes
+// (core-matrix layout) written with plain loads and stores: bf16 inputs are
+// copied, fp32 inputs split into three bf16 terms.  A warp takes 8 rows x 4
+// column groups of bf16 input: 64 contiguous bytes of each row, 128
+// contiguous destination bytes per quarter warp.
 template <int D, class IN>
-__device__ __forceinline__ void stage_planes(__nv_bfloat16 (*dst)[kChunk][D + 8], const IN* src,
-                                             size_t ld, int nthreads) {
+__device__ __forceinline__ void copy_planes(__nv_bfloat16 (*dst)[kChunk * D], const IN* src,
+                                            size_t ld, int nthreads) {
   constexpr int NK = Splits<IN>::K;
   if constexpr (NK == 1) {
     constexpr int P = D / 8;  // 16-byte pieces per row
+    static_assert(P % 4 == 0, "column groups come in fours");
     for (int e = threadIdx.x; e < kChunk * P; e += nthreads) {
-      const int r = e / P, c = (e % P) * 8;
-      cp_async16(&dst[0][r][c], src + (size_t)r * ld + c);
+      const int w = e >> 5, l = e & 31;
+      const int cg = (w % (P / 4)) * 4 + (l >> 3), r = (w / (P / 4)) * 8 + (l & 7);
+      *reinterpret_cast<uint4*>(&dst[0][core_off<kChunk>(r, 8 * cg)]) =
+          *reinterpret_cast<const uint4*>(src + (size_t)r * ld + 8 * cg);
     }
   } else {
     constexpr int G4 = D / 4;
@@ -136,36 +153,103 @@ __device__ __forceinline__ void stage_planes(__nv_bfloat16 (*dst)[kChunk][D + 8]
         __nv_bfloat16 s[NK];
         split_bf16<NK>(xs[q], s);
 #pragma unroll
-        for (int t = 0; t < NK; t++) dst[t][r][c + q] = s[t];
+        for (int t = 0; t < NK; t++) dst[t][core_off<kChunk>(r, c + q)] = s[t];
       }
     }
   }
 }
 
-// ldmatrix address of the A fragment (x4) of rows r0.., columns c0.. in a
-// row-major bf16 matrix with row stride ld.
-__device__ __forceinline__ const __nv_bfloat16* afrag_addr(const __nv_bfloat16* base, int ld,
-                                                           int r0, int c0) {
-  const int lane = threadIdx.x & 31, mi = lane >> 3;
-  return base + (size_t)(r0 + (mi & 1) * 8 + (lane & 7)) * ld + c0 + (mi >> 1) * 8;
+// One thread's share (NT threads) of a [C][D] block held in registers: loaded
+// early, written out as bf16 term planes (core-matrix layout) later, so the
+// load latency hides behind other work.  Same piece mapping as copy_planes.
+template <int D, class IN, int NT>
+struct PlaneRows {
+  static constexpr bool kBf16 = Splits<IN>::K == 1;
+  static constexpr int kPerRow = kBf16 ? D / 8 : D / 4;  // 16-byte pieces of a row
+  static constexpr int kPieces = kChunk * kPerRow / NT;
+  static_assert(kChunk * kPerRow % NT == 0, "whole pieces per thread");
+  uint4 x[kPieces];
+  __device__ __forceinline__ static void where(int e, int& r, int& c) {
+    if constexpr (kBf16) {
+      const int w = e >> 5, l = e & 31;
+      c = 8 * ((w % (kPerRow / 4)) * 4 + (l >> 3));
+      r = (w / (kPerRow / 4)) * 8 + (l & 7);
+    } else {
+      r = e / kPerRow;
+      c = (e % kPerRow) * 4;
+    }
+  }
+  __device__ __forceinline__ void load(const IN* src, size_t ld) {
+#pragma unroll
+    for (int j = 0; j < kPieces; j++) {
+      int r, c;
+      where((int)threadIdx.x + j * NT, r, c);
+      x[j] = *reinterpret_cast<const uint4*>(src + (size_t)r * ld + c);
+    }
+  }
+  __device__ __forceinline__ void store(__nv_bfloat16 (*dst)[kChunk * D]) const {
+#pragma unroll
+    for (int j = 0; j < kPieces; j++) {
+      int r, c;
+      where((int)threadIdx.x + j * NT, r, c);
+      if constexpr (kBf16) {
+        *reinterpret_cast<uint4*>(&dst[0][core_off<kChunk>(r, c)]) = x[j];
+      } else {
+        const float xs[4] = {__uint_as_float(x[j].x), __uint_as_float(x[j].y),
+                             __uint_as_float(x[j].z), __uint_as_float(x[j].w)};
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          __nv_bfloat16 t3[Splits<IN>::K];
+          split_bf16<Splits<IN>::K>(xs[q], t3);
+#pragma unroll
+          for (int tt = 0; tt < Splits<IN>::K; tt++) dst[tt][core_off<kChunk>(r, c + q)] = t3[tt];
+        }
+      }
+    }
+  }
+};
+
+// The same into shared memory; bf16 inputs go with cp.async (the caller
+// commits and waits).
+template <int D, class IN>
+__device__ __forceinline__ void stage_planes(__nv_bfloat16 (*dst)[kChunk * D], const IN* src,
+                                             size_t ld, int nthreads) {
+  if constexpr (Splits<IN>::K == 1) {
+    constexpr int P = D / 8;
+    for (int e = threadIdx.x; e < kChunk * P; e += nthreads) {
+      const int w = e >> 5, l = e & 31;
+      const int cg = (w % (P / 4)) * 4 + (l >> 3), r = (w / (P / 4)) * 8 + (l & 7);
+      cp_async16(&dst[0][core_off<kChunk>(r, 8 * cg)], src + (size_t)r * ld + 8 * cg);
+    }
+  } else {
+    copy_planes<D, IN>(dst, src, ld, nthreads);
+  }
 }
-// A fragment (x4.trans) of A[r][c] = M[c][r] (M row-major, rows = the k index).
-__device__ __forceinline__ const __nv_bfloat16* afrag_t_addr(const __nv_bfloat16* base, int ld,
-                                                             int r0, int c0) {
+
+// ldmatrix row addresses (x4) in 64-row core-layout tiles.  A fragment of
+// rows r0.., columns c0.. of the tile:
+__device__ __forceinline__ const __nv_bfloat16* afrag_addr(const __nv_bfloat16* base, int r0,
+                                                           int c0) {
   const int lane = threadIdx.x & 31, mi = lane >> 3;
-  return base + (size_t)(c0 + (mi >> 1) * 8 + (lane & 7)) * ld + r0 + (mi & 1) * 8;
+  return base + core_off<kChunk>(r0 + (mi & 1) * 8 + (lane & 7), c0 + (mi >> 1) * 8);
 }
-// B fragments (x4 = two n8 tiles) of B[k][n] = M[n][k] (M row-major, rows = n).
-__device__ __forceinline__ const __nv_bfloat16* bfrag_nk_addr(const __nv_bfloat16* base, int ld,
-                                                              int n0, int k0) {
+// A fragment (x4.trans) of A[r][c] = M[c][r] (the tile's rows are the k index).
+__device__ __forceinline__ const __nv_bfloat16* afrag_t_addr(const __nv_bfloat16* base, int r0,
+                                                             int c0) {
   const int lane = threadIdx.x & 31, mi = lane >> 3;
-  return base + (size_t)(n0 + (mi >> 1) * 8 + (lane & 7)) * ld + k0 + (mi & 1) * 8;
+  return base + core_off<kChunk>(c0 + (mi >> 1) * 8 + (lane & 7), r0 + (mi & 1) * 8);
 }
-// B fragments (x4.trans = two n8 tiles) of B[k][n] = M[k][n] (M row-major, rows = k).
-__device__ __forceinline__ const __nv_bfloat16* bfrag_kn_addr(const __nv_bfloat16* base, int ld,
-                                                              int k0, int n0) {
+// B fragments (x4 = two n8 tiles) of B[k][n] = M[n][k] (the tile's rows are n).
+__device__ __forceinline__ const __nv_bfloat16* bfrag_nk_addr(const __nv_bfloat16* base, int n0,
+                                                              int k0) {
   const int lane = threadIdx.x & 31, mi = lane >> 3;
-  return base + (size_t)(k0 + (mi & 1) * 8 + (lane & 7)) * ld + n0 + (mi >> 1) * 8;
+  return base + core_off<kChunk>(n0 + (mi >> 1) * 8 + (lane & 7), k0 + (mi & 1) * 8);
+}
+// B fragments (x4.trans = two n8 tiles) of B[k][n] = M[k][n] (the tile's rows are k).
+__device__ __forceinline__ const __nv_bfloat16* bfrag_kn_addr(const __nv_bfloat16* base, int k0,
+                                                              int n0) {
+  const int lane = threadIdx.x & 31, mi = lane >> 3;
+  return base + core_off<kChunk>(k0 + (mi & 1) * 8 + (lane & 7), n0 + (mi >> 1) * 8);
 }
 
 // Stage one chunk for the prep: keys (rows at stride ld), beta and g
@@ -186,9 +270,8 @@ __device__ __forceinline__ void prep_stage(PrepSmem<D, IN>& sm, const IN* k, siz
 // Prep of one chunk: sm.K, sm.beta, sm.g staged -> sm.head (Tb, Tv, dvec,
 // gamma).  All kBndThreads threads; ends with a block barrier.
 template <int D, class IN>
-__device__ void bnd_prep(PrepSmem<D, IN>& sm) {
+__device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT) {
   constexpr int NW = Splits<IN>::W, NK = Splits<IN>::K;
-  constexpr int LDB = PrepSmem<D, IN>::LDB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
 
   // P = K K^T on the tensor cores; warp w owns rows 16w..16w+15 (m-tile w)
@@ -205,14 +288,14 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm) {
     for (int ks = 0; ks < D / 16; ks++) {
       uint32_t a[NK][4];
 #pragma unroll
-      for (int t = 0; t < NK; t++) ldsm_x4(a[t], afrag_addr(&sm.K[t][0][0], LDB, m0, 16 * ks));
+      for (int t = 0; t < NK; t++) ldsm_x4(a[t], afrag_addr(sm.K[t], m0, 16 * ks));
 #pragma unroll
       for (int np = 0; np < 4; np++) {
         if (np <= warp) {
           uint32_t b[NK][4];
 #pragma unroll
           for (int t = 0; t < NK; t++)
-            ldsm_x4(b[t], bfrag_nk_addr(&sm.K[t][0][0], LDB, 16 * np, 16 * ks));
+            ldsm_x4(b[t], bfrag_nk_addr(sm.K[t], 16 * np, 16 * ks));
 #pragma unroll
           for (int p = 0; p < PP::kCount; p++) {
             mma16816(acc[2 * np], a[PP::a(p)], b[PP::b(p)][0], b[PP::b(p)][1]);
@@ -230,7 +313,7 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm) {
     }
   }
   for (int e = tid; e < kChunk * kChunk / 4; e += kBndThreads)
-    reinterpret_cast<float4*>(&sm.AT[0][0])[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4*>(&AT[0][0])[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
   {
     const int m0 = 16 * warp;
@@ -242,7 +325,7 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm) {
           const int i = m0 + gq + (e >> 1) * 8, j = 8 * n + 2 * tq + (e & 1);
           if (j < i) {
             const float decay = expf(__double2float_rn(sm.G[i] - sm.G[j]));
-            sm.AT[j][i] = __fmul_rn(__fmul_rn(sm.beta[i], decay), acc[n][e]);
+            AT[j][i] = __fmul_rn(__fmul_rn(sm.beta[i], decay), acc[n][e]);
           }
         }
       }
@@ -261,7 +344,8 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm) {
   // T = (I + A)^{-1}, column j held in registers by thread j: right-looking
   // over m, so T_ij accumulates -A_im T_mj in ascending m.  Steps m < j only
   // add signed zeros to zeros (T_mj = 0 there), leaving the bits unchanged.
-  // Then Tb = T diag(beta*gamma), Tv = T diag(beta), split into bf16 terms.
+  // Then Tb = T diag(beta*gamma), Tv = T diag(beta), split into bf16 terms;
+  // thread j's column is row j of the transposed tiles: 16-byte stores.
   if (tid < kChunk) {
     const int j = tid;
     float t[kChunk];
@@ -270,7 +354,7 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm) {
 #pragma unroll
     for (int m = 0; m < kChunk - 1; m++) {
       const float tm = t[m];
-      const float* col = &sm.AT[m][0];
+      const float* col = &AT[m][0];
 #pragma unroll
       for (int i4 = (m + 1) & ~3; i4 < kChunk; i4 += 4) {
         const float4 a4 = *reinterpret_cast<const float4*>(col + i4);
@@ -282,14 +366,21 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm) {
     }
     const float bgj = sm.bg[j], bj = sm.beta[j];
 #pragma unroll
-    for (int i = 0; i < kChunk; i++) {
-      __nv_bfloat16 sb[NW], sv[NW];
-      split_bf16<NW>(__fmul_rn(t[i], bgj), sb);
-      split_bf16<NW>(__fmul_rn(t[i], bj), sv);
+    for (int i8 = 0; i8 < kChunk; i8 += 8) {
+      __nv_bfloat16 sb[8][NW], sv[8][NW];
+#pragma unroll
+      for (int e = 0; e < 8; e++) {
+        split_bf16<NW>(__fmul_rn(t[i8 + e], bgj), sb[e]);
+        split_bf16<NW>(__fmul_rn(t[i8 + e], bj), sv[e]);
+      }
 #pragma unroll
       for (int q = 0; q < NW; q++) {
-        sm.head.Tb[q][i][j] = sb[q];
-        sm.head.Tv[q][i][j] = sv[q];
+        const uint4 pb = make_uint4(pack_bf16(sb[0][q], sb[1][q]), pack_bf16(sb[2][q], sb[3][q]),
+                                    pack_bf16(sb[4][q], sb[5][q]), pack_bf16(sb[6][q], sb[7][q]));
+        const uint4 pv = make_uint4(pack_bf16(sv[0][q], sv[1][q]), pack_bf16(sv[2][q], sv[3][q]),
+                                    pack_bf16(sv[4][q], sv[5][q]), pack_bf16(sv[6][q], sv[7][q]));
+        *reinterpret_cast<uint4*>(&sm.head.TbT[q][core_off<kChunk>(j, i8)]) = pb;
+        *reinterpret_cast<uint4*>(&sm.head.TvT[q][core_off<kChunk>(j, i8)]) = pv;
       }
     }
   }
@@ -335,6 +426,24 @@ __device__ __forceinline__ void sacc_store(const float (&sacc)[D / 8][4], float*
   }
 }
 
+// sacc_store into the permuted boundary-state layout of the forward workspace.
+template <int D>
+__device__ __forceinline__ void sacc_store_bst(const float (&sacc)[D / 8][4], float* S, int r0) {
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3, odd = tq & 1;
+#pragma unroll
+  for (int n = 0; n < D / 8; n++) {
+    const float s0 = odd ? sacc[n][0] : sacc[n][2];
+    const float s1 = odd ? sacc[n][1] : sacc[n][3];
+    const float r0v = __shfl_xor_sync(kFull, s0, 1);
+    const float r1v = __shfl_xor_sync(kFull, s1, 1);
+    float4 out;
+    if (!odd) out = make_float4(sacc[n][0], sacc[n][1], r0v, r1v);
+    else out = make_float4(r0v, r1v, sacc[n][2], sacc[n][3]);
+    const int row = r0 + gq + 8 * odd, col = 8 * n + 2 * (tq & 2);
+    *reinterpret_cast<float4*>(S + (size_t)row * D + bst_col(row, col)) = out;
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void sacc_zero(float (&sacc)[D / 8][4]) {
 #pragma unroll
@@ -353,8 +462,7 @@ __device__ __forceinline__ void bnd_walk_warp(float (&sacc)[D / 8][4], const Pac
                                               const __nv_bfloat16* Kp, const __nv_bfloat16* Vp,
                                               int r0) {
   constexpr int NS = Splits<IN>::S, NW = Splits<IN>::W, NK = Splits<IN>::K;
-  constexpr int LDB = D + 8, LDT = kChunk + 8;
-  constexpr size_t PL = (size_t)kChunk * LDB;  // elements per K/V plane
+  constexpr size_t PL = (size_t)kChunk * D;  // elements per K/V plane
   const int lane = threadIdx.x & 31, tq = lane & 3;
   // Y = S K^T
   float y[kChunk / 8][4];
@@ -372,7 +480,7 @@ __device__ __forceinline__ void bnd_walk_warp(float (&sacc)[D / 8][4], const Pac
       for (int np = 0; np < kChunk / 16; np++) {
         uint32_t b[NK][4];
 #pragma unroll
-        for (int q = 0; q < NK; q++) ldsm_x4(b[q], bfrag_nk_addr(Kp + q * PL, LDB, 16 * np, 16 * ks));
+        for (int q = 0; q < NK; q++) ldsm_x4(b[q], bfrag_nk_addr(Kp + q * PL, 16 * np, 16 * ks));
 #pragma unroll
         for (int p = 0; p < PP::kCount; p++) {
           mma16816(y[2 * np], a[PP::a(p)], b[PP::b(p)][0], b[PP::b(p)][1]);
@@ -394,7 +502,7 @@ __device__ __forceinline__ void bnd_walk_warp(float (&sacc)[D / 8][4], const Pac
     for (int ks = 0; ks < kChunk / 16; ks++) {
       uint32_t av[NK][4], ay[NS][4];
 #pragma unroll
-      for (int q = 0; q < NK; q++) ldsm_x4_t(av[q], afrag_t_addr(Vp + q * PL, LDB, r0, 16 * ks));
+      for (int q = 0; q < NK; q++) ldsm_x4_t(av[q], afrag_t_addr(Vp + q * PL, r0, 16 * ks));
       float ny0[4], ny1[4];
 #pragma unroll
       for (int e = 0; e < 4; e++) {
@@ -407,8 +515,8 @@ __device__ __forceinline__ void bnd_walk_warp(float (&sacc)[D / 8][4], const Pac
         uint32_t bv[NW][4], bb[NW][4];
 #pragma unroll
         for (int q = 0; q < NW; q++) {
-          ldsm_x4(bv[q], bfrag_nk_addr(&hd.Tv[q][0][0], LDT, 16 * np, 16 * ks));
-          ldsm_x4(bb[q], bfrag_nk_addr(&hd.Tb[q][0][0], LDT, 16 * np, 16 * ks));
+          ldsm_x4_t(bv[q], bfrag_kn_addr(hd.TvT[q], 16 * ks, 16 * np));
+          ldsm_x4_t(bb[q], bfrag_kn_addr(hd.TbT[q], 16 * ks, 16 * np));
         }
 #pragma unroll
         for (int p = 0; p < PV::kCount; p++) {
@@ -444,7 +552,7 @@ __device__ __forceinline__ void bnd_walk_warp(float (&sacc)[D / 8][4], const Pac
       for (int np = 0; np < D / 16; np++) {
         uint32_t b[NK][4];
 #pragma unroll
-        for (int q = 0; q < NK; q++) ldsm_x4_t(b[q], bfrag_kn_addr(Kp + q * PL, LDB, 16 * ks, 16 * np));
+        for (int q = 0; q < NK; q++) ldsm_x4_t(b[q], bfrag_kn_addr(Kp + q * PL, 16 * ks, 16 * np));
 #pragma unroll
         for (int p = 0; p < PP::kCount; p++) {
           mma16816(sacc[2 * np], a[PP::a(p)], b[PP::b(p)][0], b[PP::b(p)][1]);
@@ -453,6 +561,263 @@ __device__ __forceinline__ void bnd_walk_warp(float (&sacc)[D / 8][4], const Pac
       }
     }
   }
+}
+
+// ----------------------------------------------------------------------------
+// Walk step on the fifth-generation tensor cores (tcgen05), for
+// d_k = d_v = 128 with bf16 inputs.  128 * NCS threads: warp w works on the
+// state rows of its tensor-memory lane quadrant, 32 (w % 4) .. 32 (w % 4) + 31,
+// and on column slice w / 4 of NCS; each thread holds its row's slice of S in
+// registers.  Warp 0 issues every product (M = 128) into tensor memory and
+// one mbarrier signals their completion.  Tensor-memory columns (fp32
+// accumulators; bf16 terms packed two per column):
+//   [  0,128)  S terms (hi [0,64), lo [64,128)), the A operand of Y; then P
+//   [128,192)  Y; then the -Y terms, then the Ud terms (hi [128,160), lo [160,192))
+//   [192,256)  Z
+// Products:
+//   Y = S K^T              A: S terms          B: K (K-major)
+//   Z = V^T Tv^T - Y Tb^T  A: V (MN-major), then the -Y terms
+//                          B: TvT, TbT (MN-major); k16 step ks only reaches
+//                          the columns >= 16 ks (Tb, Tv are lower triangular)
+//   P = Ud K               A: Ud terms         B: K (MN-major)
+//   S <- fma(exp(G_C), S, P)   per element
+// Fixed evaluation order (the rounding schedule of this path):
+//   Y   k16 steps over the key channel ascending; per step S hi, then S lo
+//   Z   first V^T Tv^T (k16 steps ascending; Tv hi, then lo), then -Y Tb^T
+//       (k16 steps ascending; pairs (hi,hi), (hi,lo), (lo,hi))
+//   Ud  dvec_i * Z, split into two bf16 terms
+//   P   k16 steps over i ascending; per step Ud hi, then Ud lo
+// Which thread does an element's elementwise work does not change its bits,
+// so every NCS gives the same results.  Every wait is bounded; a step that
+// gives up returns false on all threads.
+// ----------------------------------------------------------------------------
+constexpr int kTcRows = 128;
+constexpr uint32_t kTmSA = 0, kTmP = 0, kTmY = 128, kTmYA = 128, kTmZ = 192;
+constexpr uint32_t kTmemCols = 256;
+constexpr int kTcWaitPolls = 1 << 22;
+
+template <int D, class IN>
+constexpr bool use_tc() {
+  return D == 128 && std::is_same<IN, __nv_bfloat16>::value;
+}
+
+struct TcCtx {
+  uint32_t tmem;   // first of the kTmemCols allocated columns
+  uint32_t mbar;   // completion mbarrier (shared address)
+  uint32_t phase;  // parity of the phase waited for next
+};
+
+// Allocate tensor memory (warp 0) and initialise the mbarrier; all threads.
+__device__ __forceinline__ void tc_setup(TcCtx& cx, uint64_t* mbar, uint32_t* tmem_slot) {
+  if (threadIdx.x < 32) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(mbar), 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cx.tmem = *tmem_slot;
+  cx.mbar = smem_u32(mbar);
+  cx.phase = 0;
+}
+
+// Wait (bounded) for the products committed last.  After a timeout the phase
+// is not advanced, so tc_drain waits for the same completion.
+__device__ __forceinline__ bool tc_wait(TcCtx& cx) {
+  const bool ok = mbar_wait(cx.mbar, cx.phase, kTcWaitPolls);
+  if (ok) cx.phase ^= 1;
+  tc_fence_after();
+  return ok;
+}
+
+// After a failed step: wait once more (bounded) for the products in flight.
+__device__ __forceinline__ void tc_drain(TcCtx& cx) { (void)tc_wait(cx); }
+
+// Release tensor memory (warp 0) once every thread's tensor-memory accesses
+// are done; all threads.
+__device__ __forceinline__ void tc_teardown(const TcCtx& cx) {
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x < 32) tmem_dealloc(cx.tmem, kTmemCols);
+  if (threadIdx.x == 0) mbar_inval(cx.mbar);
+}
+
+// Two-term bf16 split of (x0, x1), packed as bf16 pairs (x0 in the low half).
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const __nv_bfloat162 l =
+      __floats2bfloat162_rn(__fsub_rn(x0, __low2float(h)), __fsub_rn(x1, __high2float(h)));
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// N consecutive tensor-memory columns of this thread's lane, loaded and waited.
+template <int N>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, float (&x)[N]) {
+  static_assert(N == 16 || N == 32, "16 or 32 columns");
+  if constexpr (N == 16) tmem_ld16(taddr, x);
+  else tmem_ld32(taddr, x);
+  tmem_wait_ld(x);
+}
+template <int N>
+__device__ __forceinline__ void tmem_store(uint32_t taddr, const uint32_t (&r)[N]) {
+  static_assert(N == 8 || N == 16 || N == 32, "8, 16 or 32 columns");
+  if constexpr (N == 8) tmem_st8(taddr, r);
+  else if constexpr (N == 16) tmem_st16(taddr, r);
+  else tmem_st32(taddr, r);
+}
+
+// Writes n = 2 NP values as two bf16 term blocks (hi at taddr, lo at
+// taddr + lo_off), optionally negated.
+template <int NP, bool NEG>
+__device__ __forceinline__ void store_terms(uint32_t taddr, uint32_t lo_off, const float* x) {
+  uint32_t hi[NP], lo[NP];
+#pragma unroll
+  for (int j = 0; j < NP; j++) split2(NEG ? -x[2 * j] : x[2 * j], NEG ? -x[2 * j + 1] : x[2 * j + 1], hi[j], lo[j]);
+  tmem_store<NP>(taddr, hi);
+  tmem_store<NP>(taddr + lo_off, lo);
+}
+
+// Warp-0 hooks of a step: after_first() runs right after the first round of
+// products is committed, after_last() after the last.
+struct TcNoHooks {
+  __device__ void after_first() const {}
+  __device__ void after_last() const {}
+};
+
+// One boundary step S <- S_C for the block's 128 rows (see above).  Kp, Vp:
+// the chunk's key and value planes; hd: its pack.
+template <int NCS, class Hooks>
+__device__ __forceinline__ bool tc_walk_step(float (&s)[128 / NCS],
+                                             const PackHead<128, __nv_bfloat16>& hd,
+                                             const __nv_bfloat16* Kp, const __nv_bfloat16* Vp,
+                                             TcCtx& cx, const Hooks& hooks) {
+  constexpr int D = 128, SC = D / NCS, YC = kChunk / NCS, YP = YC < 32 ? YC : 32;
+  static_assert(SC % 32 == 0, "state slices are whole 32-column pieces");
+  constexpr uint32_t TPLANE = kChunk * kChunk * 2;
+  constexpr uint32_t IY = idesc_bf16(kTcRows, kChunk, false, false);
+  constexpr uint32_t IP = idesc_bf16(kTcRows, D, false, true);
+  const int t = threadIdx.x, w = t >> 5, cs = w >> 2;
+  const uint32_t tl = cx.tmem + ((uint32_t)(32 * (w & 3)) << 16);  // this warp's lanes
+  const uint32_t kb = smem_u32(Kp), vb = smem_u32(Vp);
+  const uint32_t tbb = smem_u32(hd.TbT[0]), tvb = smem_u32(hd.TvT[0]);
+  bool ok = true;
+
+  // S terms -> tensor memory; Y = S K^T and V^T Tv^T into Z
+  tc_fence_after();
+#pragma unroll
+  for (int pc = 0; pc < SC / 32; pc++)
+    store_terms<16, false>(tl + kTmSA + (cs * SC + 32 * pc) / 2, 64, &s[32 * pc]);
+  tmem_wait_st();
+  tc_fence_before();
+  __syncthreads();
+  if (w == 0) {
+    tc_fence_after();
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ks++)
+#pragma unroll
+      for (int a = 0; a < 2; a++)
+        umma_bf16_ts(cx.tmem + kTmY, cx.tmem + kTmSA + 64 * a + 8 * ks,
+                     desc_kmajor<kChunk>(kb + ks * 2 * kChunk * 16), IY, (ks > 0 || a > 0));
+#pragma unroll
+    for (int ks = 0; ks < kChunk / 16; ks++)
+#pragma unroll
+      for (int q = 0; q < 2; q++)
+        umma_bf16(cx.tmem + kTmZ + 16 * ks, desc_mnmajor<kChunk>(vb + ks * 256),
+                  desc_mnmajor<kChunk>(tvb + q * TPLANE + ks * 256 + ks * 2 * kChunk * 16),
+                  idesc_bf16(kTcRows, kChunk - 16 * ks, true, true), (ks > 0 || q > 0));
+    umma_commit(cx.mbar);
+    hooks.after_first();
+  }
+  ok = tc_wait(cx);
+
+  // -Y terms over Y's columns (once every thread has its slice of Y); Z -= Y Tb^T
+  {
+    float y[YC];
+#pragma unroll
+    for (int pc = 0; pc < YC / YP; pc++)
+      tmem_load<YP>(tl + kTmY + cs * YC + YP * pc, *reinterpret_cast<float(*)[YP]>(&y[YP * pc]));
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+#pragma unroll
+    for (int pc = 0; pc < YC / YP; pc++)
+      store_terms<YP / 2, true>(tl + kTmYA + (cs * YC + YP * pc) / 2, 32, &y[YP * pc]);
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  if (__syncthreads_or(!ok)) return false;
+  if (w == 0) {
+    tc_fence_after();
+    using PY = SplitPairs<2, 2>;
+#pragma unroll
+    for (int ks = 0; ks < kChunk / 16; ks++)
+#pragma unroll
+      for (int p = 0; p < PY::kCount; p++)
+        umma_bf16_ts(cx.tmem + kTmZ + 16 * ks, cx.tmem + kTmYA + 32 * PY::a(p) + 8 * ks,
+                     desc_mnmajor<kChunk>(tbb + PY::b(p) * TPLANE + ks * 256 + ks * 2 * kChunk * 16),
+                     idesc_bf16(kTcRows, kChunk - 16 * ks, false, true), 1u);
+    umma_commit(cx.mbar);
+  }
+  ok = tc_wait(cx);
+
+  // Ud = dvec * Z -> terms; P = Ud K
+#pragma unroll
+  for (int pc = 0; pc < YC / YP; pc++) {
+    float z[YP];
+    tmem_load<YP>(tl + kTmZ + cs * YC + YP * pc, z);
+#pragma unroll
+    for (int i = 0; i < YP; i++) z[i] = __fmul_rn(hd.dvec[cs * YC + YP * pc + i], z[i]);
+    store_terms<YP / 2, false>(tl + kTmYA + (cs * YC + YP * pc) / 2, 32, z);
+  }
+  tmem_wait_st();
+  tc_fence_before();
+  if (__syncthreads_or(!ok)) return false;
+  if (w == 0) {
+    tc_fence_after();
+#pragma unroll
+    for (int ks = 0; ks < kChunk / 16; ks++)
+#pragma unroll
+      for (int a = 0; a < 2; a++)
+        umma_bf16_ts(cx.tmem + kTmP, cx.tmem + kTmYA + 32 * a + 8 * ks,
+                     desc_mnmajor<kChunk>(kb + ks * 256), IP, (ks > 0 || a > 0));
+    umma_commit(cx.mbar);
+    hooks.after_last();
+  }
+  ok = tc_wait(cx);
+
+  // S <- exp(G_C) S + P
+  const float gam = hd.gamma[0];
+#pragma unroll
+  for (int pc = 0; pc < SC / 32; pc++) {
+    float p[32];
+    tmem_load<32>(tl + kTmP + cs * SC + 32 * pc, p);
+#pragma unroll
+    for (int i = 0; i < 32; i++) s[32 * pc + i] = __fmaf_rn(gam, s[32 * pc + i], p[i]);
+  }
+  tc_fence_before();
+  return !__syncthreads_or(!ok);
+}
+
+// A state row of D fp32 values (16-byte pieces).
+template <int D>
+__device__ __forceinline__ void row_load(float (&s)[D], const float* src) {
+#pragma unroll
+  for (int c = 0; c < D; c += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(src + c);
+    s[c] = x.x;
+    s[c + 1] = x.y;
+    s[c + 2] = x.z;
+    s[c + 3] = x.w;
+  }
+}
+template <int D>
+__device__ __forceinline__ void row_store(const float (&s)[D], float* dst) {
+#pragma unroll
+  for (int c = 0; c < D; c += 4)
+    *reinterpret_cast<float4*>(dst + c) = make_float4(s[c], s[c + 1], s[c + 2], s[c + 3]);
 }
 
 }  // namespace gdn

@@ -54,6 +54,7 @@ constexpr unsigned kFull = 0xffffffffu;
 
 constexpr int kErrCuSeqlens = 1;  // GDN_DEVERR_CU_SEQLENS
 constexpr int kErrPos = 2;        // GDN_DEVERR_POS
+constexpr int kErrTimeout = 4;    // GDN_DEVERR_TIMEOUT
 
 // ----------------------------------------------------------------------------
 // Loads / stores with conversion to fp32
@@ -228,6 +229,30 @@ __device__ __forceinline__ void slice_load(Slice<RT, M4>& S, const float* rows, 
 #pragma unroll
     for (int m = 0; m < M4; m++) {
       const float4 x = ld4(rows + (size_t)(r0 + i) * ld + group_col(l, m));
+      S.s[i][m][0] = f2(x.x, x.y);
+      S.s[i][m][1] = f2(x.z, x.w);
+    }
+}
+
+// Boundary-state rows in the forward workspace keep their 16-byte pieces
+// permuted inside every 128-byte line: piece g of row r is stored at piece
+// (g & ~7) | ((g ^ r) & 7), so that rows written one per thread through
+// shared memory hit distinct banks.  Column c (a multiple of 4) of row r:
+__device__ __forceinline__ int bst_col(int r, int c) {
+  const int g = c >> 2;
+  return ((g & ~7) | ((g ^ r) & 7)) << 2;
+}
+
+// slice_load from the permuted boundary-state layout.
+template <int RT, int M4>
+__device__ __forceinline__ void slice_load_bst(Slice<RT, M4>& S, const float* rows, int ld,
+                                               int r0, int l) {
+#pragma unroll
+  for (int i = 0; i < RT; i++)
+#pragma unroll
+    for (int m = 0; m < M4; m++) {
+      const int r = r0 + i;
+      const float4 x = ld4(rows + (size_t)r * ld + bst_col(r, group_col(l, m)));
       S.s[i][m][0] = f2(x.x, x.y);
       S.s[i][m][1] = f2(x.z, x.w);
     }

@@ -6,7 +6,9 @@
 // within each chunk are filled in):
 //   k_chunk_table   one block: validates cu_seqlens, numbers the chunks
 //   k_prep          one block per (chunk, head): boundary prep of full chunks
-//   k_walk          one block per (sequence, head): serial walk
+//   k_walk          one block per (sequence, head): serial walk (mma.sync,
+//                   d = 64)
+//   k_walk_tc       the same on tcgen05 / tensor memory (d = 128, bf16)
 //   k_fill          persistent blocks over (chunk, head) items: per-token
 //                   recurrence from each chunk's boundary state
 // Decode (same section: the recurrent form re-synchronised every chunk):
@@ -86,20 +88,28 @@ __global__ void __launch_bounds__(kTableThreads)
 // Pass 1a: boundary prep of every full chunk (independent of the state)
 // ----------------------------------------------------------------------------
 template <int D, class IN>
-__device__ __forceinline__ void copy16(char* dst, const char* src, size_t bytes, int nthreads) {
-  for (size_t e = threadIdx.x; e < bytes / 16; e += nthreads)
-    reinterpret_cast<uint4*>(dst)[e] = reinterpret_cast<const uint4*>(src)[e];
-}
+struct PrepKernelSmem {
+  PrepSmem<D, IN> prep;
+  PrepAT AT;
+};
 
 template <int D, class IN>
 __global__ void __launch_bounds__(kBndThreads)
-    k_prep(const IN* __restrict__ k, const float* __restrict__ beta, const float* __restrict__ g,
+    k_prep(const IN* __restrict__ k, const IN* __restrict__ v, const float* __restrict__ beta,
+           const float* __restrict__ g,
            const int32_t* __restrict__ cu, int H, const int32_t* __restrict__ hdr,
            const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
            char* __restrict__ packs) {
-  static_assert(sizeof(PackHead<D, IN>) % 16 == 0, "pack copies are 16-byte pieces");
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  PrepSmem<D, IN>& sm = *reinterpret_cast<PrepSmem<D, IN>*>(smem_raw);
+  static_assert(sizeof(PackHead<D, IN>) % 16 == 0 && sizeof(KVPlanes<D, IN>) % 16 == 0,
+                "pack copies are 16-byte pieces");
+  using PS = PrepSmem<D, IN>;
+  using WP = WalkPack<D, IN>;
+  static_assert(offsetof(PS, K) == sizeof(PackHead<D, IN>) &&
+                    offsetof(WP, kv) == sizeof(PackHead<D, IN>),
+                "head and key planes are contiguous in both layouts");
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  PrepKernelSmem<D, IN>& ks = *reinterpret_cast<PrepKernelSmem<D, IN>*>(smem_raw);
+  PrepSmem<D, IN>& sm = ks.prep;
   const int c = blockIdx.x, h = blockIdx.y;
   if (hdr[kHdrValid] != 1 || c >= hdr[kHdrChunks]) return;
   const int n = chunk_seq[c];
@@ -108,10 +118,22 @@ __global__ void __launch_bounds__(kBndThreads)
   if ((int64_t)(ci + 1) * kChunk > L) return;  // trailing partial chunk: no boundary
   const int64_t t0 = (int64_t)cu[n] + (int64_t)ci * kChunk;
   const size_t tok = (size_t)t0 * H + h;
+  PlaneRows<D, IN, kBndThreads> vrows;  // the chunk's values, in flight during the prep
+  vrows.load(v + tok * D, (size_t)H * D);
   prep_stage<D, IN>(sm, k + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H);
-  bnd_prep<D, IN>(sm);
-  copy16<D, IN>(packs + ((size_t)c * H + h) * pack_size<D, IN>(),
-                reinterpret_cast<const char*>(&sm.head), sizeof(PackHead<D, IN>), kBndThreads);
+  bnd_prep<D, IN>(sm, ks.AT);
+  // Pack: head and key planes are contiguous in shared memory, in the pack's
+  // layout (one bulk store); the value planes go from registers.
+  WalkPack<D, IN>& pk =
+      *reinterpret_cast<WalkPack<D, IN>*>(packs + ((size_t)c * H + h) * pack_size<D, IN>());
+  fence_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bulk_store(&pk.head, smem_u32(&sm.head), (uint32_t)(sizeof(PackHead<D, IN>) + sizeof(sm.K)));
+    bulk_commit();
+  }
+  vrows.store(pk.kv.V);
+  if (threadIdx.x == 0) bulk_wait();
 }
 
 // ----------------------------------------------------------------------------
@@ -121,70 +143,232 @@ __global__ void __launch_bounds__(kBndThreads)
 template <int D>
 constexpr int walk_threads() { return 32 * (D / 16); }
 
+// Pack arrival: thread 0 issues one bulk copy per chunk into a buffer whose
+// mbarrier counts the bytes; every thread waits (bounded) on that barrier.
+// Buffer b's j-th use completes phase j, so chunk c waits for parity
+// (c >> 1) & 1 on buffer c & 1.
 template <int D, class IN>
-struct WalkBuf {
-  PackHead<D, IN> head;
-  KVPlanes<D, IN> kv;
-};
-
-// Issue the loads of chunk c's walk inputs into a buffer: the pack (cp.async)
-// and the chunk's keys and values from the packed inputs; one commit group.
-template <int D, class IN>
-__device__ __forceinline__ void walk_fetch(WalkBuf<D, IN>& buf, const char* pack, const IN* k,
-                                           const IN* v, size_t ld) {
-  constexpr int N16 = (int)(sizeof(PackHead<D, IN>) / 16);
-  char* dst = reinterpret_cast<char*>(&buf.head);
-  for (int e = threadIdx.x; e < N16; e += walk_threads<D>()) cp_async16(dst + 16 * e, pack + 16 * e);
-  stage_planes<D, IN>(buf.kv.K, k, ld, walk_threads<D>());
-  stage_planes<D, IN>(buf.kv.V, v, ld, walk_threads<D>());
-  cp_async_commit();
+__device__ __forceinline__ void pack_fetch(WalkPack<D, IN>& dst, const char* src, uint64_t* bar) {
+  const uint32_t mb = smem_u32(bar);
+  mbar_expect_tx(mb, (uint32_t)sizeof(WalkPack<D, IN>));
+  bulk_load(smem_u32(&dst), src, (uint32_t)sizeof(WalkPack<D, IN>), mb);
+}
+__device__ __forceinline__ bool pack_wait(uint64_t* bars, int64_t c) {
+  return mbar_wait(smem_u32(&bars[c & 1]), (uint32_t)((c >> 1) & 1), kTcWaitPolls);
+}
+// After a failed wait: wait (bounded) for every pack copy still in flight,
+// chunks c .. issued - 1.
+__device__ __forceinline__ void pack_drain(uint64_t* bars, int64_t c, int64_t issued) {
+  for (int64_t j = c; j < issued; j++) (void)pack_wait(bars, j);
+}
+__device__ __forceinline__ void pack_bars_init(uint64_t* bars) {
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars[0]), 1);
+    mbar_init(smem_u32(&bars[1]), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
 }
 
 template <int D, class IN>
+struct WalkSmem {
+  WalkPack<D, IN> buf[2];
+  uint64_t ld_bar[2];
+};
+
+template <int D, class IN>
 __global__ void __launch_bounds__(walk_threads<D>(), 1)
-    k_walk(const IN* __restrict__ k, const IN* __restrict__ v, const int32_t* __restrict__ cu,
-           int H, const float* __restrict__ h0, const int32_t* __restrict__ hdr,
-           const int32_t* __restrict__ chunk_off, const char* __restrict__ packs,
-           float* __restrict__ bstate, float* __restrict__ s_run_final,
-           float* __restrict__ s_run_scale, float* __restrict__ s_bnd_final) {
+    k_walk(const int32_t* __restrict__ cu, int H, const float* __restrict__ h0,
+           int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+           const char* __restrict__ packs, float* __restrict__ bstate,
+           float* __restrict__ s_run_final, float* __restrict__ s_run_scale,
+           float* __restrict__ s_bnd_final) {
   constexpr size_t PB = pack_size<D, IN>();
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  WalkBuf<D, IN>* bufs = reinterpret_cast<WalkBuf<D, IN>*>(smem_raw);  // double buffer
-  const int n = blockIdx.x, h = blockIdx.y;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  WalkSmem<D, IN>& sm = *reinterpret_cast<WalkSmem<D, IN>*>(smem_raw);
+  const int n = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
   if (hdr[kHdrValid] != 1) return;
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
   const int64_t nf = L / kChunk, nc = (L + kChunk - 1) / kChunk;
   const int64_t base = chunk_off[n];
-  const int r0 = 16 * (threadIdx.x >> 5);
-  const size_t DD = (size_t)D * D, ld = (size_t)H * D;
-  const size_t tok0 = (size_t)cu[n] * H + h;  // first token of the sequence, this head
+  const int r0 = 16 * (t >> 5);
+  const size_t DD = (size_t)D * D;
+  auto pack = [&](int64_t c) { return packs + ((size_t)(base + c) * H + h) * PB; };
+  pack_bars_init(sm.ld_bar);
   float sacc[D / 8][4];
   if (h0) sacc_load<D>(sacc, h0 + ((size_t)n * H + h) * DD, r0);
   else sacc_zero<D>(sacc);
-  if (nc > 0) sacc_store<D>(sacc, bstate + ((size_t)base * H + h) * DD, r0);
-  if (nf > 0)
-    walk_fetch<D, IN>(bufs[0], packs + ((size_t)base * H + h) * PB, k + tok0 * D, v + tok0 * D, ld);
+  if (nc > 0) sacc_store_bst<D>(sacc, bstate + ((size_t)base * H + h) * DD, r0);
+  if (t == 0 && nf > 0) pack_fetch<D, IN>(sm.buf[0], pack(0), &sm.ld_bar[0]);
+  int64_t issued = nf > 0 ? 1 : 0;
+  bool ok = true;
   for (int64_t c = 0; c < nf; c++) {
     const size_t unit = (size_t)(base + c) * H + h;
-    if (c + 1 < nf) {
-      const size_t tk = tok0 + (size_t)(c + 1) * kChunk * H;
-      walk_fetch<D, IN>(bufs[(c + 1) & 1], packs + (unit + H) * PB, k + tk * D, v + tk * D, ld);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+    if (c + 1 < nf) {  // one chunk ahead into shared memory, two into L2
+      if (t == 0) pack_fetch<D, IN>(sm.buf[(c + 1) & 1], pack(c + 1), &sm.ld_bar[(c + 1) & 1]);
+      issued = c + 2;
     }
-    __syncthreads();
-    const WalkBuf<D, IN>& b = bufs[c & 1];
-    bnd_walk_warp<D, IN>(sacc, b.head, &b.kv.K[0][0][0], &b.kv.V[0][0][0], r0);
-    if (c + 1 < nc) sacc_store<D>(sacc, bstate + (unit + H) * DD, r0);
-    __syncthreads();  // buffer c&1 is refilled by the prefetch of chunk c+2
+    if (c + 2 < nf && t == 0) prefetch_l2(pack(c + 2), (uint32_t)sizeof(WalkPack<D, IN>));
+    if (__syncthreads_or(!pack_wait(sm.ld_bar, c))) {
+      ok = false;
+      pack_drain(sm.ld_bar, c, issued);
+      break;
+    }
+    const WalkPack<D, IN>& b = sm.buf[c & 1];
+    bnd_walk_warp<D, IN>(sacc, b.head, b.kv.K[0], b.kv.V[0], r0);
+    if (c + 1 < nc) sacc_store_bst<D>(sacc, bstate + (unit + H) * DD, r0);
+    __syncthreads();  // buffer c & 1 is refilled with chunk c + 2
+  }
+  if (!ok) {
+    if (t == 0) atomicOr(&hdr[kHdrError], kErrTimeout);
+    return;
   }
   const size_t so = ((size_t)n * H + h) * DD;
   if (s_bnd_final) sacc_store<D>(sacc, s_bnd_final + so, r0);
   if (s_run_final && (L % kChunk) == 0) {
     sacc_store<D>(sacc, s_run_final + so, r0);
-    if (s_run_scale && threadIdx.x == 0) s_run_scale[(size_t)n * H + h] = 1.f;
+    if (s_run_scale && t == 0) s_run_scale[(size_t)n * H + h] = 1.f;
   }
+}
+
+// The walk on tcgen05 (d = 128, bf16): one block of 512 threads per
+// (sequence, head); warp w holds columns 32 (w / 4) .. + 31 of the rows of its
+// tensor-memory lane quadrant.  Chunk c + 1's pack is copied in (one bulk
+// copy) and chunk c + 2's prefetched into L2 while chunk c's products run.
+// Each boundary state goes to the workspace through a shared-memory staging
+// copy (permuted rows, conflict-free) and one bulk asynchronous store, issued
+// with the chunk's first products.
+constexpr int kWalkSlices = 4;
+constexpr int kWalkThreads = kTcRows * kWalkSlices;
+
+template <int D, class IN>
+struct WalkTcSmem {
+  WalkPack<D, IN> buf[2];
+  alignas(128) float stage[kTcRows * D];
+  uint64_t ld_bar[2];
+  uint64_t mbar;
+  uint32_t tmem;
+};
+
+// Warp-0 hooks of the walk step (lane 0 acts): store the staged boundary
+// state with the first products, and wait until the store has read the
+// staging buffer after the last ones (the step's final barrier follows).
+struct WalkStoreHooks {
+  float* dst;
+  uint32_t stage;
+  __device__ void after_first() const {
+    if (dst && (threadIdx.x & 31) == 0) {
+      bulk_store(dst, stage, (uint32_t)(kTcRows * 128 * sizeof(float)));
+      bulk_commit();
+    }
+  }
+  __device__ void after_last() const {
+    if (dst && (threadIdx.x & 31) == 0) bulk_wait_read();
+  }
+};
+
+template <int D, class IN>
+__global__ void __launch_bounds__(kWalkThreads, 1)
+    k_walk_tc(const int32_t* __restrict__ cu, int H, const float* __restrict__ h0,
+              int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+              const char* __restrict__ packs, float* __restrict__ bstate,
+              float* __restrict__ s_run_final, float* __restrict__ s_run_scale,
+              float* __restrict__ s_bnd_final) {
+  static_assert(use_tc<D, IN>(), "tcgen05 walk: d = 128, bf16 inputs");
+  constexpr int SC = D / kWalkSlices;
+  constexpr size_t PB = pack_size<D, IN>();
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  WalkTcSmem<D, IN>& sm = *reinterpret_cast<WalkTcSmem<D, IN>*>(smem_raw);
+  const int n = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
+  if (hdr[kHdrValid] != 1) return;
+  const int w = t >> 5, row = 32 * (w & 3) + (t & 31), col0 = SC * (w >> 2);
+  const int64_t L = (int64_t)cu[n + 1] - cu[n];
+  const int64_t nf = L / kChunk, nc = (L + kChunk - 1) / kChunk;
+  const int64_t base = chunk_off[n];
+  const size_t DD = (size_t)D * D;
+  auto pack = [&](int64_t c) { return packs + ((size_t)(base + c) * H + h) * PB; };
+  pack_bars_init(sm.ld_bar);
+  TcCtx cx;
+  tc_setup(cx, &sm.mbar, &sm.tmem);
+  if (t == 0 && nf > 0) pack_fetch<D, IN>(sm.buf[0], pack(0), &sm.ld_bar[0]);
+  int64_t issued = nf > 0 ? 1 : 0;
+  float s[SC];
+  if (h0) {
+    const float* src = h0 + ((size_t)n * H + h) * DD + (size_t)row * D + col0;
+#pragma unroll
+    for (int c = 0; c < SC; c += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(src + c);
+      s[c] = x.x;
+      s[c + 1] = x.y;
+      s[c + 2] = x.z;
+      s[c + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < SC; i++) s[i] = 0.f;
+  }
+  // Stage this thread's slice of the state (permuted rows); the previous bulk
+  // store has finished reading the buffer (warp 0 waited, barriers since).
+  auto stage_state = [&]() {
+    float* dst = sm.stage + (size_t)row * D;
+#pragma unroll
+    for (int c = 0; c < SC; c += 4)
+      *reinterpret_cast<float4*>(dst + bst_col(row, col0 + c)) =
+          make_float4(s[c], s[c + 1], s[c + 2], s[c + 3]);
+    fence_async_smem();
+  };
+  bool ok = true;
+  for (int64_t c = 0; c < nf; c++) {
+    const size_t unit = (size_t)(base + c) * H + h;
+    if (c + 1 < nf) {  // one chunk ahead into shared memory, two into L2
+      if (t == 0) pack_fetch<D, IN>(sm.buf[(c + 1) & 1], pack(c + 1), &sm.ld_bar[(c + 1) & 1]);
+      issued = c + 2;
+    }
+    if (c + 2 < nf && t == 0) prefetch_l2(pack(c + 2), (uint32_t)sizeof(WalkPack<D, IN>));
+    stage_state();  // boundary state of chunk c
+    if (!pack_wait(sm.ld_bar, c)) {
+      ok = false;  // made uniform by the step's first barrier
+    }
+    const WalkPack<D, IN>& b = sm.buf[c & 1];
+    // The step's first barrier publishes the staged state; it ends with a
+    // barrier after its last product, so buffer c & 1 is free for chunk c + 2.
+    const WalkStoreHooks hooks{ok ? bstate + unit * DD : nullptr, smem_u32(sm.stage)};
+    if (__syncthreads_or(!ok)) {
+      ok = false;
+      pack_drain(sm.ld_bar, c, issued);
+      break;
+    }
+    ok = tc_walk_step<kWalkSlices>(s, b.head, b.kv.K[0], b.kv.V[0], cx, hooks);
+    if (!ok) {
+      pack_drain(sm.ld_bar, c + 1, issued);
+      break;
+    }
+  }
+  if (!ok) {
+    tc_drain(cx);
+    if (t == 0) atomicOr(&hdr[kHdrError], kErrTimeout);
+  } else {
+    if (nc > nf) {  // the trailing partial chunk starts from the last boundary
+      stage_state();
+      __syncthreads();
+      if (t == 0) {
+        bulk_store(bstate + ((size_t)(base + nf) * H + h) * DD, smem_u32(sm.stage),
+                   (uint32_t)(DD * sizeof(float)));
+        bulk_commit();
+      }
+    }
+    const size_t so = ((size_t)n * H + h) * DD + (size_t)row * D + col0;
+#pragma unroll
+    for (int c = 0; c < SC; c += 4) {
+      const float4 x = make_float4(s[c], s[c + 1], s[c + 2], s[c + 3]);
+      if (s_bnd_final) *reinterpret_cast<float4*>(s_bnd_final + so + c) = x;
+      if (s_run_final && (L % kChunk) == 0) *reinterpret_cast<float4*>(s_run_final + so + c) = x;
+    }
+    if (s_run_final && s_run_scale && (L % kChunk) == 0 && t == 0)
+      s_run_scale[(size_t)n * H + h] = 1.f;
+  }
+  if (t == 0) bulk_wait();  // every bulk store complete before the block exits
+  tc_teardown(cx);
 }
 
 // ----------------------------------------------------------------------------
@@ -234,10 +418,6 @@ __device__ __forceinline__ FillItem fill_item(int item, int H, const int32_t* cu
   return it;
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes));
-}
-
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
@@ -249,7 +429,6 @@ __device__ __forceinline__ void fill_load(FillSmem<D, IN>& sm, const FillItem& i
   constexpr int G4 = D / 4;                        // float4 groups of a key row
   constexpr int P = (int)(D * sizeof(IN) / 16);    // 16-byte pieces of a q/v row
   constexpr int E = (int)(16 / sizeof(IN));
-  const size_t ld = (size_t)H * D;
   const size_t tb = (size_t)it.t0 * H + it.h;
   for (int e = threadIdx.x; e < (kChunk + 1) * G4; e += kFillThreads) {
     const int r = e / G4, c = (e % G4) * 4;
@@ -300,7 +479,7 @@ __global__ void __launch_bounds__(kFillThreads, 3)
            const float* __restrict__ bstate, OUT* __restrict__ o,
            float* __restrict__ s_run_final, float* __restrict__ s_run_scale) {
   constexpr int RT = D / 32, M4 = D / 16;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   FillSmem<D, IN>& sm = *reinterpret_cast<FillSmem<D, IN>*>(smem_raw);
   __shared__ int sh_item;
   if (hdr[kHdrValid] != 1) return;
@@ -315,7 +494,7 @@ __global__ void __launch_bounds__(kFillThreads, 3)
     const FillItem cur = fill_item(item, H, cu, chunk_off, chunk_seq);
     fill_load<D, IN>(sm, cur, q, k, v, beta, g, H);
     Slice<RT, M4> S;
-    slice_load<RT, M4>(S, bstate + ((size_t)cur.c * H + cur.h) * DD, D, r0, l);
+    slice_load_bst<RT, M4>(S, bstate + ((size_t)cur.c * H + cur.h) * DD, D, r0, l);
     if (tid == 0) sh_item = atomicAdd(&hdr[kHdrFillNext], 1);
     __syncthreads();
     const int next = sh_item;
@@ -360,29 +539,65 @@ __global__ void __launch_bounds__(kFillThreads, 3)
 template <int D, class IN>
 struct BndSmem {
   PrepSmem<D, IN> prep;
-  __nv_bfloat16 V[Splits<IN>::K][kChunk][D + 8];
+  PrepAT AT;
+  alignas(16) __nv_bfloat16 V[Splits<IN>::K][kChunk * D];
 };
 
-// One chunk boundary for `unit` (prep + walk of all D rows), in place allowed.
+// The tcgen05 form keeps the walk's operands in tensor memory.
 template <int D, class IN>
-__device__ __forceinline__ void bnd_unit(BndSmem<D, IN>& sm, const float* s_start, const IN* kb,
-                                         const IN* vb, const float* bb, const float* gb,
-                                         size_t unit, float* s_end) {
+struct BndTcSmem {
+  PrepSmem<D, IN> prep;
+  PrepAT AT;
+  alignas(16) __nv_bfloat16 V[Splits<IN>::K][kChunk * D];
+  uint64_t mbar;
+  uint32_t tmem;
+};
+
+template <int D, class IN>
+using BndUnitSmem = typename std::conditional<use_tc<D, IN>(), BndTcSmem<D, IN>, BndSmem<D, IN>>::type;
+
+// One chunk boundary for `unit` (prep + walk of all D rows), in place allowed.
+// Returns false if a tensor-core wait gave up (the unit's s_end is then NaN).
+template <int D, class IN>
+__device__ __forceinline__ bool bnd_unit(BndUnitSmem<D, IN>& sm, const float* s_start,
+                                         const IN* kb, const IN* vb, const float* bb,
+                                         const float* gb, size_t unit, float* s_end) {
   const size_t DD = (size_t)D * D;
   stage_planes<D, IN>(sm.V, vb + unit * kChunk * D, (size_t)D, kBndThreads);
   prep_stage<D, IN>(sm.prep, kb + unit * kChunk * D, (size_t)D, bb + unit * kChunk,
                     gb + unit * kChunk, 1);
-  bnd_prep<D, IN>(sm.prep);
-  const int warp = threadIdx.x >> 5;
+  if constexpr (use_tc<D, IN>()) {
+    static_assert(kBndThreads == kTcRows, "one state row per thread");
+    bnd_prep<D, IN>(sm.prep, sm.AT);
+    TcCtx cx;
+    tc_setup(cx, &sm.mbar, &sm.tmem);
+    const size_t row = unit * DD + (size_t)threadIdx.x * D;
+    float s[D];
+    row_load<D>(s, s_start + row);
+    const bool ok = tc_walk_step<1>(s, sm.prep.head, sm.prep.K[0], sm.V[0], cx, TcNoHooks{});
+    if (!ok) {
+      tc_drain(cx);
+#pragma unroll
+      for (int i = 0; i < D; i++) s[i] = __int_as_float(0x7fc00000);
+    }
+    row_store<D>(s, s_end + row);
+    tc_teardown(cx);
+    __syncthreads();  // shared memory is reused by the next unit
+    return ok;
+  } else {
+    bnd_prep<D, IN>(sm.prep, sm.AT);
+    const int warp = threadIdx.x >> 5;
 #pragma unroll 1
-  for (int rt = 0; rt < D / 64; rt++) {
-    const int r0 = 16 * warp + 64 * rt;
-    float sacc[D / 8][4];
-    sacc_load<D>(sacc, s_start + unit * DD, r0);
-    bnd_walk_warp<D, IN>(sacc, sm.prep.head, &sm.prep.K[0][0][0], &sm.V[0][0][0], r0);
-    sacc_store<D>(sacc, s_end + unit * DD, r0);
+    for (int rt = 0; rt < D / 64; rt++) {
+      const int r0 = 16 * warp + 64 * rt;
+      float sacc[D / 8][4];
+      sacc_load<D>(sacc, s_start + unit * DD, r0);
+      bnd_walk_warp<D, IN>(sacc, sm.prep.head, sm.prep.K[0], sm.V[0], r0);
+      sacc_store<D>(sacc, s_end + unit * DD, r0);
+    }
+    __syncthreads();  // shared memory is reused by the next unit
+    return true;
   }
-  __syncthreads();  // shared memory is reused by the next unit
 }
 
 // gdn_chunk_boundary: one block per (row, head).
@@ -390,8 +605,8 @@ template <int D, class IN>
 __global__ void __launch_bounds__(kBndThreads)
     k_bnd(const float* s_start, const IN* __restrict__ kb, const IN* __restrict__ vb,
           const float* __restrict__ bb, const float* __restrict__ gb, int H, float* s_end) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  BndSmem<D, IN>& sm = *reinterpret_cast<BndSmem<D, IN>*>(smem_raw);
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  BndUnitSmem<D, IN>& sm = *reinterpret_cast<BndUnitSmem<D, IN>*>(smem_raw);
   bnd_unit<D, IN>(sm, s_start, kb, vb, bb, gb, (size_t)blockIdx.x * H + blockIdx.y, s_end);
 }
 
@@ -411,7 +626,7 @@ __global__ void __launch_bounds__(kDecThreads)
                float* buf_g, int32_t* pos, int32_t* error, int n_slots, OUT* __restrict__ o) {
   static_assert(kDecThreads == kBndThreads, "the resync runs in the step's block");
   constexpr int RT = D / 32, M4 = D / 16;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ int sh_pos, sh_slot;
   const int b = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * RT;
@@ -470,8 +685,9 @@ __global__ void __launch_bounds__(kDecThreads)
     // The buffer is full: advance the boundary state over its C tokens.  The
     // running state of the next step is the new boundary state (pos = 0).
     __syncthreads();  // the appended token is visible to the whole block
-    BndSmem<D, IN>& sm = *reinterpret_cast<BndSmem<D, IN>*>(smem_raw);
-    bnd_unit<D, IN>(sm, s_bnd, buf_k, buf_v, buf_beta, buf_g, unit, s_bnd);
+    BndUnitSmem<D, IN>& sm = *reinterpret_cast<BndUnitSmem<D, IN>*>(smem_raw);
+    if (!bnd_unit<D, IN>(sm, s_bnd, buf_k, buf_v, buf_beta, buf_g, unit, s_bnd) && tid == 0)
+      atomicOr(error, kErrTimeout);
     if (tid == 0) pos[unit] = 0;
   }
 }
@@ -570,20 +786,28 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   GDN_TRY(mark(1));
   {
     auto kern = k_prep<D, IN>;
-    const size_t sm = sizeof(PrepSmem<D, IN>);
+    const size_t sm = sizeof(PrepKernelSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
-    kern<<<gchunks, kBndThreads, sm, st>>>(k, a.beta, a.g, a.cu_seqlens, a.H, hdr, chunk_off,
+    kern<<<gchunks, kBndThreads, sm, st>>>(k, v, a.beta, a.g, a.cu_seqlens, a.H, hdr, chunk_off,
                                            chunk_seq, packs);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(2));
-  {
+  if constexpr (use_tc<D, IN>()) {
+    auto kern = k_walk_tc<D, IN>;
+    const size_t sm = sizeof(WalkTcSmem<D, IN>);
+    GDN_TRY(set_smem(kern, sm));
+    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), kWalkThreads, sm, st>>>(
+        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final, a.s_run_scale,
+        a.s_bnd_final);
+    GDN_TRY(cudaGetLastError());
+  } else {
     auto kern = k_walk<D, IN>;
-    const size_t sm = 2 * sizeof(WalkBuf<D, IN>);
+    const size_t sm = sizeof(WalkSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
     kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), walk_threads<D>(), sm, st>>>(
-        k, v, a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final,
-        a.s_run_scale, a.s_bnd_final);
+        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final, a.s_run_scale,
+        a.s_bnd_final);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(3));
@@ -606,7 +830,7 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
 template <int D, class IN, class OUT>
 static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
   auto kern = k_dec_step<D, IN, OUT>;
-  const size_t sm = sizeof(BndSmem<D, IN>);
+  const size_t sm = sizeof(BndUnitSmem<D, IN>);
   GDN_TRY(set_smem(kern, sm));
   kern<<<dim3((unsigned)a.B, (unsigned)a.H), kDecThreads, sm, st>>>(
       static_cast<const IN*>(a.q), static_cast<const IN*>(a.k), static_cast<const IN*>(a.v),
@@ -629,7 +853,7 @@ static cudaError_t handoff_impl(const HandoffArgs& a, cudaStream_t st) {
 template <int D, class IN>
 static cudaError_t boundary_impl(const BndArgs& a, cudaStream_t st) {
   auto kern = k_bnd<D, IN>;
-  const size_t sm = sizeof(BndSmem<D, IN>);
+  const size_t sm = sizeof(BndUnitSmem<D, IN>);
   GDN_TRY(set_smem(kern, sm));
   kern<<<dim3((unsigned)a.B, (unsigned)a.H), kBndThreads, sm, st>>>(
       a.s_start, static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, a.H,

@@ -9,12 +9,12 @@
 namespace gdn {
 
 // Bytes of one walk pack (mirrors pack_size<D, IN>() in gdn_boundary.cuh; a
-// static_assert there keeps the two equal): Tb and Tv as bf16 term planes
-// [C][C+8], the decay vector [C] and 4 floats.
+// static_assert there keeps the two equal): Tb and Tv as bf16 term planes of
+// C x C, the decay vector [C] and 4 floats, then the chunk's keys and values
+// as bf16 term planes of C x D.
 constexpr size_t pack_bytes(int D, bool in_bf16) {
-  (void)D;
-  const size_t NW = in_bf16 ? 2 : 3, C = 64;
-  const size_t b = 2 * NW * C * (C + 8) * 2 + C * 4 + 16;
+  const size_t NW = in_bf16 ? 2 : 3, NK = in_bf16 ? 1 : 3, C = 64;
+  const size_t b = 2 * NW * C * C * 2 + C * 4 + 16 + 2 * NK * C * (size_t)D * 2;
   return (b + 127) / 128 * 128;
 }
 
