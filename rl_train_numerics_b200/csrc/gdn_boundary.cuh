@@ -35,8 +35,8 @@
 //   G        double, ascending i
 //   P=KK^T   k16 steps ascending; split pairs in SplitPairs order
 //   A_ij     (beta_i * expf((float)(G_i - G_j))) * P_ij
-//   T        right-looking substitution: T_ij accumulates -A_im T_mj over
-//            m = j .. i-1 (one fma each)
+//   T        blocked forward substitution over 16 x 16 blocks (bnd_prep
+//            states the order of every sum)
 //   Tb, Tv   T_im * (beta_m expf(G_m)) and T_im * beta_m, then split
 //   Y        (S0 K^T): k16 steps over the key channel ascending
 //   U^T      one accumulator: per k16 step over m (ascending, up to the
@@ -341,29 +341,106 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT) {
   }
   __syncthreads();
 
-  // T = (I + A)^{-1}, column j held in registers by thread j: right-looking
-  // over m, so T_ij accumulates -A_im T_mj in ascending m.  Steps m < j only
-  // add signed zeros to zeros (T_mj = 0 there), leaving the bits unchanged.
-  // Then Tb = T diag(beta*gamma), Tv = T diag(beta), split into bf16 terms;
-  // thread j's column is row j of the transposed tiles: 16-byte stores.
+  // T = (I + A)^{-1} (unit lower triangular) by blocked forward substitution
+  // over 16 x 16 blocks, kept in AT's free lower triangle: AT[i][j] = T_ij for
+  // i >= j (A stays above the diagonal, AT[m][i] = A_im for i > m).
+  //  1. diagonal blocks D_b = (I + A_bb)^{-1}, column j of block b held by
+  //     one thread: right-looking, T_ij accumulates -A_im T_mj in ascending m;
+  //  2. for s = 1, 2, 3 and every block (b, c) with b - c = s:
+  //     X = sum over k = c .. b-1 (ascending) of A_bk T_kc, one fma chain per
+  //     element in ascending inner index; then T_bc = -(D_b X), accumulated
+  //     from X_ij with D_b[i][k] X_kj in ascending k < i.
+  {
+    constexpr int NB = 16;
+    if (tid < kChunk) {
+      const int b0 = (tid / NB) * NB, j = tid % NB;
+      float t[NB];
+#pragma unroll
+      for (int i = 0; i < NB; i++) t[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+      for (int m = 0; m < NB - 1; m++) {
+        const float tm = t[m];
+        const float* col = &AT[b0 + m][b0];
+#pragma unroll
+        for (int i4 = (m + 1) & ~3; i4 < NB; i4 += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(col + i4);
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+          for (int q = 0; q < 4; q++)
+            if (i4 + q > m) t[i4 + q] = __fmaf_rn(-av[q], tm, t[i4 + q]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < NB; i++)
+        if (i >= j) AT[b0 + i][b0 + j] = t[i];
+    }
+    __syncthreads();
+    // Stages: thread (block, row i, 8 columns j0..j0+7), 8 accumulators.
+    float* X = reinterpret_cast<float*>(sm.head.TbT[0]);  // scratch until the splits below
+#pragma unroll
+    for (int st = 1; st < kChunk / NB; st++) {
+      const int nblk = kChunk / NB - st;
+      const int blk = tid / (2 * NB), i = (tid % (2 * NB)) / 2, j0 = (tid % 2) * 8;
+      const int c0 = blk * NB, b0 = c0 + st * NB;
+      float* Xr = X + blk * NB * NB;
+      if (blk < nblk) {
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; e++) acc[e] = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < st; kb++) {
+          const int k0 = c0 + kb * NB;
+#pragma unroll
+          for (int q = 0; q < NB; q++) {
+            const float a = AT[k0 + q][b0 + i];  // A_{b0+i, k0+q}
+            const float4 u0 = *reinterpret_cast<const float4*>(&AT[k0 + q][c0 + j0]);
+            const float4 u1 = *reinterpret_cast<const float4*>(&AT[k0 + q][c0 + j0 + 4]);
+            float tv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+            for (int e = 0; e < 8; e++) {
+              if (kb == 0 && q < j0 + e) tv[e] = 0.f;  // above T's diagonal (A lives there)
+              acc[e] = __fmaf_rn(a, tv[e], acc[e]);
+            }
+          }
+        }
+        *reinterpret_cast<float4*>(Xr + i * NB + j0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(Xr + i * NB + j0 + 4) =
+            make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
+      __syncthreads();
+      if (blk < nblk) {
+        float acc[8];
+        const float4 x0 = *reinterpret_cast<const float4*>(Xr + i * NB + j0);
+        const float4 x1 = *reinterpret_cast<const float4*>(Xr + i * NB + j0 + 4);
+        acc[0] = x0.x, acc[1] = x0.y, acc[2] = x0.z, acc[3] = x0.w;
+        acc[4] = x1.x, acc[5] = x1.y, acc[6] = x1.z, acc[7] = x1.w;
+#pragma unroll
+        for (int k = 0; k < NB - 1; k++) {
+          if (k < i) {
+            const float d = AT[b0 + i][b0 + k];  // D_b[i][k]
+            const float4 y0 = *reinterpret_cast<const float4*>(Xr + k * NB + j0);
+            const float4 y1 = *reinterpret_cast<const float4*>(Xr + k * NB + j0 + 4);
+            const float yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+            for (int e = 0; e < 8; e++) acc[e] = __fmaf_rn(d, yv[e], acc[e]);
+          }
+        }
+        *reinterpret_cast<float4*>(&AT[b0 + i][c0 + j0]) =
+            make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+        *reinterpret_cast<float4*>(&AT[b0 + i][c0 + j0 + 4]) =
+            make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
+      }
+      __syncthreads();
+    }
+  }
+
+  // Tb = T diag(beta*gamma), Tv = T diag(beta), split into bf16 terms; thread
+  // j's column of T is row j of the transposed tiles: 16-byte stores.
   if (tid < kChunk) {
     const int j = tid;
     float t[kChunk];
 #pragma unroll
-    for (int i = 0; i < kChunk; i++) t[i] = (i == j) ? 1.f : 0.f;
-#pragma unroll
-    for (int m = 0; m < kChunk - 1; m++) {
-      const float tm = t[m];
-      const float* col = &AT[m][0];
-#pragma unroll
-      for (int i4 = (m + 1) & ~3; i4 < kChunk; i4 += 4) {
-        const float4 a4 = *reinterpret_cast<const float4*>(col + i4);
-        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-        for (int q = 0; q < 4; q++)
-          if (i4 + q > m) t[i4 + q] = __fmaf_rn(-av[q], tm, t[i4 + q]);
-      }
-    }
+    for (int i = 0; i < kChunk; i++) t[i] = (i >= j) ? AT[i][j] : 0.f;
     const float bgj = sm.bg[j], bj = sm.beta[j];
 #pragma unroll
     for (int i8 = 0; i8 < kChunk; i8 += 8) {
@@ -680,17 +757,30 @@ __device__ __forceinline__ void store_terms(uint32_t taddr, uint32_t lo_off, con
   tmem_store<NP>(taddr + lo_off, lo);
 }
 
-// Warp-0 hooks of a step: after_first() runs right after the first round of
-// products is committed, after_last() after the last.
+// Hooks of a step, for work that overlaps it:
+//   inputs_ready()  all threads, before the first barrier: false gives up
+//   after_first()   warp 0, once the first round of products is committed
+//   during_first(s) all threads, while the first round runs (s: the state
+//                   the step starts from)
+//   after_second()  warp 0, once the second round is committed
+//   after_last()    warp 0, once the last round is committed (the step's
+//                   final barrier follows)
 struct TcNoHooks {
+  __device__ bool inputs_ready() const { return true; }
   __device__ void after_first() const {}
+  __device__ void during_first(const float*) const {}
+  __device__ void after_second() const {}
   __device__ void after_last() const {}
 };
 
+// Outcome of a step: done, gave up before issuing any product, or gave up
+// after (products may still be in flight: tc_drain).
+enum TcStep { kStepDone = 0, kStepNoInputs = 1, kStepFailed = 2 };
+
 // One boundary step S <- S_C for the block's 128 rows (see above).  Kp, Vp:
-// the chunk's key and value planes; hd: its pack.
+// the chunk's key and value planes; hd: its pack.  Returns a TcStep.
 template <int NCS, class Hooks>
-__device__ __forceinline__ bool tc_walk_step(float (&s)[128 / NCS],
+__device__ __forceinline__ int tc_walk_step(float (&s)[128 / NCS],
                                              const PackHead<128, __nv_bfloat16>& hd,
                                              const __nv_bfloat16* Kp, const __nv_bfloat16* Vp,
                                              TcCtx& cx, const Hooks& hooks) {
@@ -711,8 +801,9 @@ __device__ __forceinline__ bool tc_walk_step(float (&s)[128 / NCS],
   for (int pc = 0; pc < SC / 32; pc++)
     store_terms<16, false>(tl + kTmSA + (cs * SC + 32 * pc) / 2, 64, &s[32 * pc]);
   tmem_wait_st();
+  const bool in_ok = hooks.inputs_ready();
   tc_fence_before();
-  __syncthreads();
+  if (__syncthreads_or(!in_ok)) return kStepNoInputs;
   if (w == 0) {
     tc_fence_after();
 #pragma unroll
@@ -731,6 +822,7 @@ __device__ __forceinline__ bool tc_walk_step(float (&s)[128 / NCS],
     umma_commit(cx.mbar);
     hooks.after_first();
   }
+  hooks.during_first(s);
   ok = tc_wait(cx);
 
   // -Y terms over Y's columns (once every thread has its slice of Y); Z -= Y Tb^T
@@ -748,7 +840,7 @@ __device__ __forceinline__ bool tc_walk_step(float (&s)[128 / NCS],
     tmem_wait_st();
   }
   tc_fence_before();
-  if (__syncthreads_or(!ok)) return false;
+  if (__syncthreads_or(!ok)) return kStepFailed;
   if (w == 0) {
     tc_fence_after();
     using PY = SplitPairs<2, 2>;
@@ -760,6 +852,7 @@ __device__ __forceinline__ bool tc_walk_step(float (&s)[128 / NCS],
                      desc_mnmajor<kChunk>(tbb + PY::b(p) * TPLANE + ks * 256 + ks * 2 * kChunk * 16),
                      idesc_bf16(kTcRows, kChunk - 16 * ks, false, true), 1u);
     umma_commit(cx.mbar);
+    hooks.after_second();
   }
   ok = tc_wait(cx);
 
@@ -774,7 +867,7 @@ __device__ __forceinline__ bool tc_walk_step(float (&s)[128 / NCS],
   }
   tmem_wait_st();
   tc_fence_before();
-  if (__syncthreads_or(!ok)) return false;
+  if (__syncthreads_or(!ok)) return kStepFailed;
   if (w == 0) {
     tc_fence_after();
 #pragma unroll
@@ -798,7 +891,7 @@ __device__ __forceinline__ bool tc_walk_step(float (&s)[128 / NCS],
     for (int i = 0; i < 32; i++) s[32 * pc + i] = __fmaf_rn(gam, s[32 * pc + i], p[i]);
   }
   tc_fence_before();
-  return !__syncthreads_or(!ok);
+  return __syncthreads_or(!ok) ? kStepFailed : kStepDone;
 }
 
 // A state row of D fp32 values (16-byte pieces).

@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kBndThreads)
     bulk_commit();
   }
   vrows.store(pk.kv.V);
-  if (threadIdx.x == 0) bulk_wait();
+  if (threadIdx.x == 0) bulk_wait_read();  // shared memory must outlive the copy's reads
 }
 
 // ----------------------------------------------------------------------------
@@ -250,21 +250,49 @@ struct WalkTcSmem {
   uint32_t tmem;
 };
 
-// Warp-0 hooks of the walk step (lane 0 acts): store the staged boundary
-// state with the first products, and wait until the store has read the
-// staging buffer after the last ones (the step's final barrier follows).
-struct WalkStoreHooks {
-  float* dst;
-  uint32_t stage;
+// Stage a thread's slice of the state (permuted rows) for a bulk store.
+template <int D, int SC>
+__device__ __forceinline__ void stage_slice(float* stage, const float* s, int row, int col0) {
+  float* dst = stage + (size_t)row * D;
+#pragma unroll
+  for (int c = 0; c < SC; c += 4)
+    *reinterpret_cast<float4*>(dst + bst_col(row, col0 + c)) =
+        make_float4(s[c], s[c + 1], s[c + 2], s[c + 3]);
+  fence_async_smem();
+}
+
+// The walk's work around the step of chunk c (warp-0 parts by lane 0):
+// before the first barrier, wait until the previous chunk's state store has
+// read the staging buffer (thread 0) and for this chunk's pack; issue chunk
+// c + 1's pack copy and chunk c + 2's L2 prefetch with the first products;
+// stage the boundary state while they run and store it with the second
+// round.
+template <int D, class IN>
+struct WalkHooks {
+  WalkTcSmem<D, IN>* sm;
+  int64_t c;
+  const char* next;  // pack of chunk c + 1, or null
+  const char* ahead; // pack of chunk c + 2, or null
+  float* dst;        // boundary state of chunk c in the workspace
+  int row, col0;
+  __device__ bool inputs_ready() const {
+    if (threadIdx.x == 0) bulk_wait_read();
+    return pack_wait(sm->ld_bar, c);
+  }
   __device__ void after_first() const {
-    if (dst && (threadIdx.x & 31) == 0) {
-      bulk_store(dst, stage, (uint32_t)(kTcRows * 128 * sizeof(float)));
-      bulk_commit();
-    }
+    if ((threadIdx.x & 31) != 0) return;
+    if (next) pack_fetch<D, IN>(sm->buf[(c + 1) & 1], next, &sm->ld_bar[(c + 1) & 1]);
+    if (ahead) prefetch_l2(ahead, (uint32_t)sizeof(WalkPack<D, IN>));
   }
-  __device__ void after_last() const {
-    if (dst && (threadIdx.x & 31) == 0) bulk_wait_read();
+  __device__ void during_first(const float* s) const {
+    stage_slice<D, D / kWalkSlices>(sm->stage, s, row, col0);
   }
+  __device__ void after_second() const {
+    if ((threadIdx.x & 31) != 0) return;
+    bulk_store(dst, smem_u32(sm->stage), (uint32_t)(kTcRows * D * sizeof(float)));
+    bulk_commit();
+  }
+  __device__ void after_last() const {}
 };
 
 template <int D, class IN>
@@ -291,7 +319,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
   TcCtx cx;
   tc_setup(cx, &sm.mbar, &sm.tmem);
   if (t == 0 && nf > 0) pack_fetch<D, IN>(sm.buf[0], pack(0), &sm.ld_bar[0]);
-  int64_t issued = nf > 0 ? 1 : 0;
+  if (t == 0 && nf > 1) prefetch_l2(pack(1), (uint32_t)sizeof(WalkPack<D, IN>));
   float s[SC];
   if (h0) {
     const float* src = h0 + ((size_t)n * H + h) * DD + (size_t)row * D + col0;
@@ -307,49 +335,29 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
 #pragma unroll
     for (int i = 0; i < SC; i++) s[i] = 0.f;
   }
-  // Stage this thread's slice of the state (permuted rows); the previous bulk
-  // store has finished reading the buffer (warp 0 waited, barriers since).
-  auto stage_state = [&]() {
-    float* dst = sm.stage + (size_t)row * D;
-#pragma unroll
-    for (int c = 0; c < SC; c += 4)
-      *reinterpret_cast<float4*>(dst + bst_col(row, col0 + c)) =
-          make_float4(s[c], s[c + 1], s[c + 2], s[c + 3]);
-    fence_async_smem();
-  };
-  bool ok = true;
-  for (int64_t c = 0; c < nf; c++) {
+  int status = kStepDone;
+  int64_t c = 0;
+  for (; c < nf; c++) {
     const size_t unit = (size_t)(base + c) * H + h;
-    if (c + 1 < nf) {  // one chunk ahead into shared memory, two into L2
-      if (t == 0) pack_fetch<D, IN>(sm.buf[(c + 1) & 1], pack(c + 1), &sm.ld_bar[(c + 1) & 1]);
-      issued = c + 2;
-    }
-    if (c + 2 < nf && t == 0) prefetch_l2(pack(c + 2), (uint32_t)sizeof(WalkPack<D, IN>));
-    stage_state();  // boundary state of chunk c
-    if (!pack_wait(sm.ld_bar, c)) {
-      ok = false;  // made uniform by the step's first barrier
-    }
+    const WalkHooks<D, IN> hooks{&sm, c, c + 1 < nf ? pack(c + 1) : nullptr,
+                                 c + 2 < nf ? pack(c + 2) : nullptr, bstate + unit * DD, row,
+                                 col0};
     const WalkPack<D, IN>& b = sm.buf[c & 1];
-    // The step's first barrier publishes the staged state; it ends with a
-    // barrier after its last product, so buffer c & 1 is free for chunk c + 2.
-    const WalkStoreHooks hooks{ok ? bstate + unit * DD : nullptr, smem_u32(sm.stage)};
-    if (__syncthreads_or(!ok)) {
-      ok = false;
-      pack_drain(sm.ld_bar, c, issued);
-      break;
-    }
-    ok = tc_walk_step<kWalkSlices>(s, b.head, b.kv.K[0], b.kv.V[0], cx, hooks);
-    if (!ok) {
-      pack_drain(sm.ld_bar, c + 1, issued);
-      break;
-    }
+    status = tc_walk_step<kWalkSlices>(s, b.head, b.kv.K[0], b.kv.V[0], cx, hooks);
+    if (status != kStepDone) break;
   }
-  if (!ok) {
-    tc_drain(cx);
+  if (status != kStepDone) {
+    // Pack copies possibly in flight: chunks c .. issued - 1 (the step issues
+    // chunk c + 1's copy once it is past its first barrier).
+    const int64_t issued = status == kStepNoInputs ? c + 1 : (c + 2 < nf ? c + 2 : nf);
+    pack_drain(sm.ld_bar, c, issued);
+    if (status == kStepFailed) tc_drain(cx);
     if (t == 0) atomicOr(&hdr[kHdrError], kErrTimeout);
   } else {
     if (nc > nf) {  // the trailing partial chunk starts from the last boundary
-      stage_state();
+      if (t == 0) bulk_wait_read();
+      __syncthreads();
+      stage_slice<D, SC>(sm.stage, s, row, col0);
       __syncthreads();
       if (t == 0) {
         bulk_store(bstate + ((size_t)(base + nf) * H + h) * DD, smem_u32(sm.stage),
@@ -359,10 +367,10 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     }
     const size_t so = ((size_t)n * H + h) * DD + (size_t)row * D + col0;
 #pragma unroll
-    for (int c = 0; c < SC; c += 4) {
-      const float4 x = make_float4(s[c], s[c + 1], s[c + 2], s[c + 3]);
-      if (s_bnd_final) *reinterpret_cast<float4*>(s_bnd_final + so + c) = x;
-      if (s_run_final && (L % kChunk) == 0) *reinterpret_cast<float4*>(s_run_final + so + c) = x;
+    for (int i = 0; i < SC; i += 4) {
+      const float4 x = make_float4(s[i], s[i + 1], s[i + 2], s[i + 3]);
+      if (s_bnd_final) *reinterpret_cast<float4*>(s_bnd_final + so + i) = x;
+      if (s_run_final && (L % kChunk) == 0) *reinterpret_cast<float4*>(s_run_final + so + i) = x;
     }
     if (s_run_final && s_run_scale && (L % kChunk) == 0 && t == 0)
       s_run_scale[(size_t)n * H + h] = 1.f;
@@ -574,7 +582,8 @@ __device__ __forceinline__ bool bnd_unit(BndUnitSmem<D, IN>& sm, const float* s_
     const size_t row = unit * DD + (size_t)threadIdx.x * D;
     float s[D];
     row_load<D>(s, s_start + row);
-    const bool ok = tc_walk_step<1>(s, sm.prep.head, sm.prep.K[0], sm.V[0], cx, TcNoHooks{});
+    const bool ok =
+        tc_walk_step<1>(s, sm.prep.head, sm.prep.K[0], sm.V[0], cx, TcNoHooks{}) == kStepDone;
     if (!ok) {
       tc_drain(cx);
 #pragma unroll
