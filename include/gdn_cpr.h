@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define GDN_CPR_ABI_VERSION 2
+#define GDN_CPR_ABI_VERSION 3
 
 typedef enum {
   GDN_OK = 0,
@@ -185,6 +185,10 @@ int gdn_cpr_forward_noalloc(const void* q, const void* k, const void* v, int in_
  *                                (equal over heads; kept per head so that no
  *                                two thread blocks share a counter)
  *   error    [1] int32  device error word (GDN_DEVERR_* bits)
+ *   resync   [4 + n_slots * H] int32  work list of the chunk resync inside
+ *                                gdn_cpr_decode_step (scratch: all zero
+ *                                before the first step; every step leaves
+ *                                it zero again)
  */
 typedef struct {
   float* s_run;
@@ -196,6 +200,7 @@ typedef struct {
   float* buf_g;
   int32_t* pos;
   int32_t* error;
+  int32_t* resync;
   int n_slots;
 } gdn_decode_state;
 
@@ -234,8 +239,10 @@ int gdn_cpr_decode_state_from_prefill(const void* k, const void* v, int in_dtype
  * and pos returns to 0.
  * q, k [B, H, dk], v [B, H, dv] in_dtype; beta, g [B, H] fp32;
  * o [B, H, dv] out_dtype.  Rows must name distinct slots.
- * Launch shapes depend only on (B, H, dk, C), so the call can be captured
- * in a CUDA graph.
+ * Two kernels run: the step (which lists the (slot, head) units whose buffer
+ * became full in st.resync) and the chunk boundary of the listed units.
+ * Launch shapes depend only on (B, H, dk, C) and the device, so the call can
+ * be captured in a CUDA graph.
  */
 int gdn_cpr_decode_step(const void* q, const void* k, const void* v, int in_dtype,
                         const float* beta, const float* g, const int32_t* slot_idx, int B, int H,

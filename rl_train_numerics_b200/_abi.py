@@ -42,7 +42,7 @@ class DecodeStateStruct(ctypes.Structure):
                 ("buf_k", ctypes.c_void_p), ("buf_v", ctypes.c_void_p),
                 ("buf_beta", ctypes.c_void_p), ("buf_g", ctypes.c_void_p),
                 ("pos", ctypes.c_void_p), ("error", ctypes.c_void_p),
-                ("n_slots", ctypes.c_int)]
+                ("resync", ctypes.c_void_p), ("n_slots", ctypes.c_int)]
 
 
 def _load() -> ctypes.CDLL:
@@ -201,13 +201,16 @@ class DecodeState:
         self.buf_g = torch.zeros((n_slots, H, C), dtype=f32, device=device)
         self.pos = torch.zeros((n_slots, H), dtype=torch.int32, device=device)
         self.error = torch.zeros((1,), dtype=torch.int32, device=device)
+        # work list of the resync inside decode_step (scratch, zero between steps)
+        self.resync = torch.zeros((4 + n_slots * H,), dtype=torch.int32, device=device)
 
     def struct(self) -> DecodeStateStruct:
         return DecodeStateStruct(self.s_run.data_ptr(), self.s_scale.data_ptr(),
                                  self.s_bnd.data_ptr(),
                                  self.buf_k.data_ptr(), self.buf_v.data_ptr(),
                                  self.buf_beta.data_ptr(), self.buf_g.data_ptr(),
-                                 self.pos.data_ptr(), self.error.data_ptr(), self.n_slots)
+                                 self.pos.data_ptr(), self.error.data_ptr(),
+                                 self.resync.data_ptr(), self.n_slots)
 
     def tensors(self):
         return (self.s_run, self.s_scale, self.s_bnd, self.buf_k, self.buf_v, self.buf_beta,

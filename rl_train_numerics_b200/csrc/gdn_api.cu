@@ -116,11 +116,11 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
 
 static int check_state(const gdn_decode_state& st) {
   if (st.n_slots <= 0 || !st.s_run || !st.s_scale || !st.s_bnd || !st.buf_k || !st.buf_v ||
-      !st.buf_beta || !st.buf_g || !st.pos || !st.error)
+      !st.buf_beta || !st.buf_g || !st.pos || !st.error || !st.resync)
     return GDN_ERR_INVALID_ARG;
   if (!aligned16(st.s_run) || !aligned16(st.s_bnd) || !aligned16(st.buf_k) ||
       !aligned16(st.buf_v) || !aligned4(st.buf_beta) || !aligned4(st.buf_g) ||
-      !aligned4(st.pos) || !aligned4(st.error) || !aligned4(st.s_scale))
+      !aligned4(st.pos) || !aligned4(st.error) || !aligned4(st.s_scale) || !aligned4(st.resync))
     return GDN_ERR_INVALID_ARG;
   return GDN_OK;
 }
@@ -206,6 +206,7 @@ int gdn_cpr_decode_step(const void* q, const void* k, const void* v, int in_dtyp
   a.buf_g = st.buf_g;
   a.pos = st.pos;
   a.error = st.error;
+  a.resync = st.resync;
   a.n_slots = st.n_slots;
   a.o = o;
   a.out_bf16 = out_dtype == GDN_BF16;

@@ -257,7 +257,7 @@ __device__ __forceinline__ const __nv_bfloat16* bfrag_kn_addr(const __nv_bfloat1
 template <int D, class IN>
 __device__ __forceinline__ void prep_stage(PrepSmem<D, IN>& sm, const IN* k, size_t ld,
                                            const float* bsrc, const float* gsrc, size_t ldbg) {
-  stage_planes<D, IN>(sm.K, k, ld, kBndThreads);
+  stage_planes<D, IN>(sm.K, k, ld, (int)blockDim.x);
   cp_async_commit();
   for (int i = threadIdx.x; i < kChunk; i += kBndThreads) {
     sm.beta[i] = bsrc[i * ldbg];
@@ -268,7 +268,8 @@ __device__ __forceinline__ void prep_stage(PrepSmem<D, IN>& sm, const IN* k, siz
 }
 
 // Prep of one chunk: sm.K, sm.beta, sm.g staged -> sm.head (Tb, Tv, dvec,
-// gamma).  All kBndThreads threads; ends with a block barrier.
+// gamma), with AT as scratch.  The first kBndThreads threads do the work;
+// every thread of the block takes the barriers.  Ends with a block barrier.
 template <int D, class IN>
 __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT) {
   constexpr int NW = Splits<IN>::W, NK = Splits<IN>::K;
@@ -277,7 +278,7 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT) {
   // P = K K^T on the tensor cores; warp w owns rows 16w..16w+15 (m-tile w)
   // and the n8 tiles that reach below the diagonal.
   float acc[8][4];
-  {
+  if (warp < kBndThreads / 32) {
     using PP = SplitPairs<NK, NK>;
     const int m0 = 16 * warp;
 #pragma unroll
@@ -312,10 +313,11 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT) {
       sm.G[i] = s;
     }
   }
-  for (int e = tid; e < kChunk * kChunk / 4; e += kBndThreads)
-    reinterpret_cast<float4*>(&AT[0][0])[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (tid < kBndThreads)
+    for (int e = tid; e < kChunk * kChunk / 4; e += kBndThreads)
+      reinterpret_cast<float4*>(&AT[0][0])[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
-  {
+  if (warp < kBndThreads / 32) {
     const int m0 = 16 * warp;
 #pragma unroll
     for (int n = 0; n < 8; n++) {

@@ -12,8 +12,9 @@
 //   k_fill          persistent blocks over (chunk, head) items: per-token
 //                   recurrence from each chunk's boundary state
 // Decode (same section: the recurrent form re-synchronised every chunk):
-//   k_dec_step      one block per (row, head): one recurrence step, then the
-//                   chunk boundary when the step filled the chunk buffer
+//   k_dec_step      one block per (row, head): one recurrence step; units
+//                   whose chunk buffer became full go on a work list
+//   k_resync        persistent blocks: the chunk boundary of listed units
 //   k_bnd           one block per (row, head): gdn_chunk_boundary
 //   k_handoff       prefill -> decode state
 #include "gdn_boundary.cuh"
@@ -564,35 +565,54 @@ struct BndTcSmem {
 template <int D, class IN>
 using BndUnitSmem = typename std::conditional<use_tc<D, IN>(), BndTcSmem<D, IN>, BndSmem<D, IN>>::type;
 
-// One chunk boundary for `unit` (prep + walk of all D rows), in place allowed.
-// Returns false if a tensor-core wait gave up (the unit's s_end is then NaN).
+// Threads of a block that runs whole chunk boundaries: the tcgen05 walk uses
+// four column slices (512 threads), the mma.sync walk 128 threads.
+template <int D, class IN>
+constexpr int unit_threads() {
+  return use_tc<D, IN>() ? kTcRows * kWalkSlices : kBndThreads;
+}
+
+// One chunk boundary for `unit` (prep + walk of all D rows), in place allowed,
+// by a block of unit_threads<D, IN>() threads.  Returns false if a
+// tensor-core wait gave up (the unit's s_end is then NaN).
 template <int D, class IN>
 __device__ __forceinline__ bool bnd_unit(BndUnitSmem<D, IN>& sm, const float* s_start,
                                          const IN* kb, const IN* vb, const float* bb,
                                          const float* gb, size_t unit, float* s_end) {
+  constexpr int NT = unit_threads<D, IN>();
   const size_t DD = (size_t)D * D;
-  stage_planes<D, IN>(sm.V, vb + unit * kChunk * D, (size_t)D, kBndThreads);
+  stage_planes<D, IN>(sm.V, vb + unit * kChunk * D, (size_t)D, NT);
   prep_stage<D, IN>(sm.prep, kb + unit * kChunk * D, (size_t)D, bb + unit * kChunk,
                     gb + unit * kChunk, 1);
   if constexpr (use_tc<D, IN>()) {
-    static_assert(kBndThreads == kTcRows, "one state row per thread");
+    constexpr int SC = D / kWalkSlices;
     bnd_prep<D, IN>(sm.prep, sm.AT);
     TcCtx cx;
     tc_setup(cx, &sm.mbar, &sm.tmem);
-    const size_t row = unit * DD + (size_t)threadIdx.x * D;
-    float s[D];
-    row_load<D>(s, s_start + row);
-    const bool ok =
-        tc_walk_step<1>(s, sm.prep.head, sm.prep.K[0], sm.V[0], cx, TcNoHooks{}) == kStepDone;
-    if (!ok) {
-      tc_drain(cx);
+    const int w = threadIdx.x >> 5, row = 32 * (w & 3) + (threadIdx.x & 31);
+    const size_t off = unit * DD + (size_t)row * D + SC * (w >> 2);
+    float s[SC];
 #pragma unroll
-      for (int i = 0; i < D; i++) s[i] = __int_as_float(0x7fc00000);
+    for (int c = 0; c < SC; c += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(s_start + off + c);
+      s[c] = x.x;
+      s[c + 1] = x.y;
+      s[c + 2] = x.z;
+      s[c + 3] = x.w;
     }
-    row_store<D>(s, s_end + row);
+    const int st =
+        tc_walk_step<kWalkSlices>(s, sm.prep.head, sm.prep.K[0], sm.V[0], cx, TcNoHooks{});
+    if (st != kStepDone) {
+      if (st == kStepFailed) tc_drain(cx);
+#pragma unroll
+      for (int i = 0; i < SC; i++) s[i] = __int_as_float(0x7fc00000);
+    }
+#pragma unroll
+    for (int c = 0; c < SC; c += 4)
+      *reinterpret_cast<float4*>(s_end + off + c) = make_float4(s[c], s[c + 1], s[c + 2], s[c + 3]);
     tc_teardown(cx);
     __syncthreads();  // shared memory is reused by the next unit
-    return ok;
+    return st == kStepDone;
   } else {
     bnd_prep<D, IN>(sm.prep, sm.AT);
     const int warp = threadIdx.x >> 5;
@@ -611,7 +631,7 @@ __device__ __forceinline__ bool bnd_unit(BndUnitSmem<D, IN>& sm, const float* s_
 
 // gdn_chunk_boundary: one block per (row, head).
 template <int D, class IN>
-__global__ void __launch_bounds__(kBndThreads)
+__global__ void __launch_bounds__(unit_threads<D, IN>())
     k_bnd(const float* s_start, const IN* __restrict__ kb, const IN* __restrict__ vb,
           const float* __restrict__ bb, const float* __restrict__ gb, int H, float* s_end) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -626,16 +646,21 @@ __global__ void __launch_bounds__(kBndThreads)
 // ----------------------------------------------------------------------------
 constexpr int kDecThreads = 128;  // four state rows per thread
 
+// Words of a decode state's resync work list.
+constexpr int kResyncCount = 0;  // units listed by this step
+constexpr int kResyncNext = 1;   // work counter of k_resync
+constexpr int kResyncDone = 2;   // k_resync blocks finished
+constexpr int kResyncList = 4;   // the units
+
 template <int D, class IN, class OUT>
 __global__ void __launch_bounds__(kDecThreads)
     k_dec_step(const IN* __restrict__ q, const IN* __restrict__ k, const IN* __restrict__ v,
                const float* __restrict__ beta, const float* __restrict__ g,
                const int32_t* __restrict__ slot_idx, int H, float scale, float* s_run,
                float* s_scale, float* s_bnd, IN* buf_k, IN* buf_v, float* buf_beta,
-               float* buf_g, int32_t* pos, int32_t* error, int n_slots, OUT* __restrict__ o) {
-  static_assert(kDecThreads == kBndThreads, "the resync runs in the step's block");
+               float* buf_g, int32_t* pos, int32_t* error, int32_t* resync, int n_slots,
+               OUT* __restrict__ o) {
   constexpr int RT = D / 32, M4 = D / 16;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ int sh_pos, sh_slot;
   const int b = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * RT;
@@ -690,14 +715,42 @@ __global__ void __launch_bounds__(kDecThreads)
     buf_g[unit * kChunk + p0] = g[tok];
     if (p0 + 1 < kChunk) pos[unit] = p0 + 1;
   }
-  if (p0 + 1 == kChunk) {
-    // The buffer is full: advance the boundary state over its C tokens.  The
-    // running state of the next step is the new boundary state (pos = 0).
-    __syncthreads();  // the appended token is visible to the whole block
-    BndUnitSmem<D, IN>& sm = *reinterpret_cast<BndUnitSmem<D, IN>*>(smem_raw);
-    if (!bnd_unit<D, IN>(sm, s_bnd, buf_k, buf_v, buf_beta, buf_g, unit, s_bnd) && tid == 0)
+  if (p0 + 1 == kChunk && tid == 0) {
+    // The buffer is full: k_resync advances the boundary state over its C
+    // tokens, and that becomes the running state of the next step (pos = 0).
+    const int j = atomicAdd(&resync[kResyncCount], 1);
+    if (j < n_slots * H) resync[kResyncList + j] = (int32_t)unit;
+    else atomicOr(error, kErrPos);  // rows naming the same slot twice
+    pos[unit] = 0;
+  }
+}
+
+// The chunk boundary of every unit that k_dec_step listed, in place on s_bnd.
+// Persistent blocks take list entries from a counter; the last block to
+// finish empties the list for the next step.
+template <int D, class IN>
+__global__ void __launch_bounds__(unit_threads<D, IN>())
+    k_resync(int H, float* s_bnd, const IN* buf_k, const IN* buf_v, const float* buf_beta,
+             const float* buf_g, int32_t* resync, int n_slots, int32_t* error) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  BndUnitSmem<D, IN>& sm = *reinterpret_cast<BndUnitSmem<D, IN>*>(smem_raw);
+  __shared__ int sh_j;
+  const int count = min(resync[kResyncCount], n_slots * H);
+  for (;;) {
+    if (threadIdx.x == 0) sh_j = atomicAdd(&resync[kResyncNext], 1);
+    __syncthreads();
+    const int j = sh_j;
+    __syncthreads();  // every thread has j before thread 0 takes the next one
+    if (j >= count) break;
+    const size_t unit = (size_t)resync[kResyncList + j];
+    if (!bnd_unit<D, IN>(sm, s_bnd, buf_k, buf_v, buf_beta, buf_g, unit, s_bnd) &&
+        threadIdx.x == 0)
       atomicOr(error, kErrTimeout);
-    if (tid == 0) pos[unit] = 0;
+  }
+  if (threadIdx.x == 0 && atomicAdd(&resync[kResyncDone], 1) == (int)gridDim.x - 1) {
+    resync[kResyncCount] = 0;  // every block has read the count and left the loop
+    resync[kResyncNext] = 0;
+    resync[kResyncDone] = 0;
   }
 }
 
@@ -838,14 +891,20 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
 
 template <int D, class IN, class OUT>
 static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
-  auto kern = k_dec_step<D, IN, OUT>;
-  const size_t sm = sizeof(BndUnitSmem<D, IN>);
-  GDN_TRY(set_smem(kern, sm));
-  kern<<<dim3((unsigned)a.B, (unsigned)a.H), kDecThreads, sm, st>>>(
+  k_dec_step<D, IN, OUT><<<dim3((unsigned)a.B, (unsigned)a.H), kDecThreads, 0, st>>>(
       static_cast<const IN*>(a.q), static_cast<const IN*>(a.k), static_cast<const IN*>(a.v),
       a.beta, a.g, a.slot_idx, a.H, a.scale, a.s_run, a.s_scale, a.s_bnd,
       static_cast<IN*>(a.buf_k), static_cast<IN*>(a.buf_v), a.buf_beta, a.buf_g, a.pos, a.error,
-      a.n_slots, static_cast<OUT*>(a.o));
+      a.resync, a.n_slots, static_cast<OUT*>(a.o));
+  GDN_TRY(cudaGetLastError());
+  auto kern = k_resync<D, IN>;
+  const size_t sm = sizeof(BndUnitSmem<D, IN>);
+  GDN_TRY(set_smem(kern, sm));
+  int grid = 0;
+  GDN_TRY(persistent_grid(kern, unit_threads<D, IN>(), sm, &grid));
+  kern<<<grid, unit_threads<D, IN>(), sm, st>>>(
+      a.H, a.s_bnd, static_cast<const IN*>(a.buf_k), static_cast<const IN*>(a.buf_v), a.buf_beta,
+      a.buf_g, a.resync, a.n_slots, a.error);
   return cudaGetLastError();
 }
 
@@ -864,7 +923,7 @@ static cudaError_t boundary_impl(const BndArgs& a, cudaStream_t st) {
   auto kern = k_bnd<D, IN>;
   const size_t sm = sizeof(BndUnitSmem<D, IN>);
   GDN_TRY(set_smem(kern, sm));
-  kern<<<dim3((unsigned)a.B, (unsigned)a.H), kBndThreads, sm, st>>>(
+  kern<<<dim3((unsigned)a.B, (unsigned)a.H), unit_threads<D, IN>(), sm, st>>>(
       a.s_start, static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, a.H,
       a.s_end);
   return cudaGetLastError();

@@ -97,6 +97,7 @@ struct DecArgs {
   float* buf_g;
   int32_t* pos;
   int32_t* error;
+  int32_t* resync;
   int n_slots;
   void* o;
   int out_bf16;

@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert gdn.lib.gdn_cpr_abi_version() == 2
+    assert gdn.lib.gdn_cpr_abi_version() == 3
     for code in range(-6, 1):
         assert gdn.status_string(code).startswith("GDN_")
     assert "unknown" in gdn.status_string(42)
@@ -113,10 +113,11 @@ def test_forward_empty_batch_is_a_no_op():
 
 def _state(**over):
     f = dict(s_run=FAKE, s_scale=FAKE, s_bnd=FAKE, buf_k=FAKE, buf_v=FAKE, buf_beta=FAKE,
-             buf_g=FAKE, pos=FAKE, error=FAKE, n_slots=4)
+             buf_g=FAKE, pos=FAKE, error=FAKE, resync=FAKE, n_slots=4)
     f.update(over)
     return gdn.DecodeStateStruct(f["s_run"], f["s_scale"], f["s_bnd"], f["buf_k"], f["buf_v"],
-                                 f["buf_beta"], f["buf_g"], f["pos"], f["error"], f["n_slots"])
+                                 f["buf_beta"], f["buf_g"], f["pos"], f["error"], f["resync"],
+                                 f["n_slots"])
 
 
 def dec(st=None, **over):
@@ -139,6 +140,7 @@ def dec(st=None, **over):
     ({}, dict(pos=None), gdn.GDN_ERR_INVALID_ARG),
     ({}, dict(s_scale=None), gdn.GDN_ERR_INVALID_ARG),
     ({}, dict(error=None), gdn.GDN_ERR_INVALID_ARG),
+    ({}, dict(resync=None), gdn.GDN_ERR_INVALID_ARG),
     ({}, dict(s_bnd=MIS), gdn.GDN_ERR_INVALID_ARG),
     ({}, dict(n_slots=0), gdn.GDN_ERR_INVALID_ARG),
     (dict(B=5), {}, gdn.GDN_ERR_INVALID_ARG),   # more rows than slots without slot_idx
