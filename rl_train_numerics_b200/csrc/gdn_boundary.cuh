@@ -32,7 +32,7 @@
 // inputs.
 //
 // Fixed evaluation order (part of the rounding schedule):
-//   G        double, ascending i
+//   G        double: pair sums, then a Kogge-Stone scan (bnd_prep)
 //   P=KK^T   k16 steps ascending; split pairs in SplitPairs order
 //   A_ij     (beta_i * expf((float)(G_i - G_j))) * P_ij
 //   T        blocked forward substitution over 16 x 16 blocks (bnd_prep
@@ -270,8 +270,14 @@ __device__ __forceinline__ void prep_stage(PrepSmem<D, IN>& sm, const IN* k, siz
 // Prep of one chunk: sm.K, sm.beta, sm.g staged -> sm.head (Tb, Tv, dvec,
 // gamma), with AT as scratch.  The first kBndThreads threads do the work;
 // every thread of the block takes the barriers.  Ends with a block barrier.
-template <int D, class IN>
-__device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT) {
+struct PrepNoHook {
+  __device__ void operator()() const {}
+};
+
+// after_p(): all threads, once P = K K^T is in registers and before AT is
+// first written (a caller whose AT shares memory with K saves K there).
+template <int D, class IN, class AfterP = PrepNoHook>
+__device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT, const AfterP& after_p = AfterP{}) {
   constexpr int NW = Splits<IN>::W, NK = Splits<IN>::K;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
 
@@ -306,13 +312,22 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT) {
       }
     }
   }
-  if (tid == 0) {
-    double s = 0.0;
-    for (int i = 0; i < kChunk; i++) {
-      s += (double)sm.g[i];
-      sm.G[i] = s;
+  // G = cumulative sum of g in double: warp 0, lane l sums g_2l + g_2l+1,
+  // then an inclusive Kogge-Stone scan over the 32 pair sums (offsets 1, 2,
+  // 4, 8, 16); G_2l+1 = scan_l, G_2l = scan_(l-1) + g_2l (scan_(-1) = 0).
+  if (warp == 0) {
+    const double g0 = (double)sm.g[2 * lane], g1 = (double)sm.g[2 * lane + 1];
+    double x = g0 + g1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const double y = __shfl_up_sync(kFull, x, off);
+      if (lane >= off) x += y;
     }
+    const double e = __shfl_up_sync(kFull, x, 1);
+    sm.G[2 * lane + 1] = x;
+    sm.G[2 * lane] = lane > 0 ? e + g0 : g0;
   }
+  after_p();
   if (tid < kBndThreads)
     for (int e = tid; e < kChunk * kChunk / 4; e += kBndThreads)
       reinterpret_cast<float4*>(&AT[0][0])[e] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -377,6 +392,16 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT) {
         if (i >= j) AT[b0 + i][b0 + j] = t[i];
     }
     __syncthreads();
+    // A_bb is no longer needed: its place above the diagonal takes D_b
+    // transposed, AT[b0 + k][b0 + i] = D_b[i][k] for i > k, so that the
+    // products below read D_b by rows of AT.
+    if (tid < kChunk) {
+      const int b0 = (tid / NB) * NB, j = tid % NB;
+#pragma unroll
+      for (int i = 0; i < NB; i++)
+        if (i > j) AT[b0 + j][b0 + i] = AT[b0 + i][b0 + j];
+    }
+    __syncthreads();
     // Stages: thread (block, row i, 8 columns j0..j0+7), 8 accumulators.
     float* X = reinterpret_cast<float*>(sm.head.TbT[0]);  // scratch until the splits below
 #pragma unroll
@@ -419,7 +444,7 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT) {
 #pragma unroll
         for (int k = 0; k < NB - 1; k++) {
           if (k < i) {
-            const float d = AT[b0 + i][b0 + k];  // D_b[i][k]
+            const float d = AT[b0 + k][b0 + i];  // D_b[i][k]
             const float4 y0 = *reinterpret_cast<const float4*>(Xr + k * NB + j0);
             const float4 y1 = *reinterpret_cast<const float4*>(Xr + k * NB + j0 + 4);
             const float yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
@@ -440,17 +465,15 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT) {
   // j's column of T is row j of the transposed tiles: 16-byte stores.
   if (tid < kChunk) {
     const int j = tid;
-    float t[kChunk];
-#pragma unroll
-    for (int i = 0; i < kChunk; i++) t[i] = (i >= j) ? AT[i][j] : 0.f;
     const float bgj = sm.bg[j], bj = sm.beta[j];
 #pragma unroll
     for (int i8 = 0; i8 < kChunk; i8 += 8) {
       __nv_bfloat16 sb[8][NW], sv[8][NW];
 #pragma unroll
       for (int e = 0; e < 8; e++) {
-        split_bf16<NW>(__fmul_rn(t[i8 + e], bgj), sb[e]);
-        split_bf16<NW>(__fmul_rn(t[i8 + e], bj), sv[e]);
+        const float tij = (i8 + e >= j) ? AT[i8 + e][j] : 0.f;
+        split_bf16<NW>(__fmul_rn(tij, bgj), sb[e]);
+        split_bf16<NW>(__fmul_rn(tij, bj), sv[e]);
       }
 #pragma unroll
       for (int q = 0; q < NW; q++) {

@@ -88,14 +88,26 @@ __global__ void __launch_bounds__(kTableThreads)
 // ----------------------------------------------------------------------------
 // Pass 1a: boundary prep of every full chunk (independent of the state)
 // ----------------------------------------------------------------------------
+// The prep kernel's AT shares memory with the key planes where they are big
+// enough: the keys go to the pack once P = K K^T is formed.
 template <int D, class IN>
+constexpr bool prep_at_on_keys() {
+  return Splits<IN>::K * kChunk * D * 2 >= (int)sizeof(PrepAT);
+}
+template <int D, class IN, bool ON_KEYS = prep_at_on_keys<D, IN>()>
 struct PrepKernelSmem {
   PrepSmem<D, IN> prep;
   PrepAT AT;
+  __device__ PrepAT& at() { return AT; }
+};
+template <int D, class IN>
+struct PrepKernelSmem<D, IN, true> {
+  PrepSmem<D, IN> prep;
+  __device__ PrepAT& at() { return *reinterpret_cast<PrepAT*>(prep.K); }
 };
 
 template <int D, class IN>
-__global__ void __launch_bounds__(kBndThreads)
+__global__ void __launch_bounds__(kBndThreads, prep_at_on_keys<D, IN>() ? 4 : 3)
     k_prep(const IN* __restrict__ k, const IN* __restrict__ v, const float* __restrict__ beta,
            const float* __restrict__ g,
            const int32_t* __restrict__ cu, int H, const int32_t* __restrict__ hdr,
@@ -122,15 +134,32 @@ __global__ void __launch_bounds__(kBndThreads)
   PlaneRows<D, IN, kBndThreads> vrows;  // the chunk's values, in flight during the prep
   vrows.load(v + tok * D, (size_t)H * D);
   prep_stage<D, IN>(sm, k + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H);
-  bnd_prep<D, IN>(sm, ks.AT);
-  // Pack: head and key planes are contiguous in shared memory, in the pack's
-  // layout (one bulk store); the value planes go from registers.
   WalkPack<D, IN>& pk =
       *reinterpret_cast<WalkPack<D, IN>*>(packs + ((size_t)c * H + h) * pack_size<D, IN>());
+  if constexpr (prep_at_on_keys<D, IN>()) {
+    // Keys to the pack (bulk store) before AT overwrites them.
+    bnd_prep<D, IN>(sm, ks.at(), [&]() {
+      fence_async_smem();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        bulk_store(pk.kv.K, smem_u32(sm.K), (uint32_t)sizeof(sm.K));
+        bulk_commit();
+        bulk_wait_read();
+      }
+      __syncthreads();
+    });
+  } else {
+    bnd_prep<D, IN>(sm, ks.at());
+  }
+  // The head (and the keys, unless they are stored already) in one bulk
+  // store: in shared memory they are contiguous, in the pack's layout.  The
+  // value planes go from registers.
+  constexpr uint32_t kOut =
+      (uint32_t)(sizeof(PackHead<D, IN>) + (prep_at_on_keys<D, IN>() ? 0 : sizeof(sm.K)));
   fence_async_smem();
   __syncthreads();
   if (threadIdx.x == 0) {
-    bulk_store(&pk.head, smem_u32(&sm.head), (uint32_t)(sizeof(PackHead<D, IN>) + sizeof(sm.K)));
+    bulk_store(&pk.head, smem_u32(&sm.head), kOut);
     bulk_commit();
   }
   vrows.store(pk.kv.V);
