@@ -327,7 +327,8 @@ def run_decode_part(gdn, W, dev, rank, world, args, peaks):
             "resync_units_per_step": round(float(np.mean(resync)) * H, 2),
             "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(dec_gbs / peaks["hbm_gbs"], 4), "traffic": None},
+                         "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
+                         "traffic": ncu_traffic("decode_step")},
             "pages_h100_ms": PAGES_H100["decode_ms"]}
 
 
