@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define GDN_CPR_ABI_VERSION 3
+#define GDN_CPR_ABI_VERSION 4
 
 typedef enum {
   GDN_OK = 0,
@@ -60,7 +60,8 @@ typedef enum {
   GDN_ERR_WORKSPACE = -3,   /* workspace missing or smaller than the query says */
   GDN_ERR_CUDA = -4,        /* a CUDA launch or runtime call failed */
   GDN_ERR_DEVICE_DATA = -5, /* device-side validation failed (see gdn_check_error) */
-  GDN_ERR_TIMEOUT = -6      /* reserved: a bounded device-side wait gave up */
+  GDN_ERR_TIMEOUT = -6,     /* reserved: a bounded device-side wait gave up */
+  GDN_ERR_CONTRACT = -7     /* a peer's numerical-policy digest differs from this library's */
 } gdn_status;
 
 typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
@@ -268,6 +269,48 @@ int gdn_chunk_boundary(const float* s_start, const void* k, const void* v, int i
  * receives the GDN_DEVERR_* bits that were set.
  */
 int gdn_check_error(void* error_word, int32_t* bits_out, void* stream);
+
+/*
+ * Contract digests of the CPR region (host only, no device work).
+ *
+ * Defines: "NovaSky's IsoExec Fixes the Hidden Math Bug Corrupting AI
+ * Training Runs", section "The execution contract": a contract pins every
+ * choice that can move bits and carries three SHA-256 identity digests
+ * (semantic equivalence, numerical policy, deployment settings that do not
+ * affect bits); engines whose numerical policies differ refuse to run
+ * together.  Each digest is the SHA-256 (FIPS 180-4) of a canonical text
+ * descriptor of this library's region for one (in_dtype, out_dtype, dk, dv,
+ * C): what it computes (semantic); every choice that fixes its bits, i.e.
+ * dtypes, shapes, the step and boundary schedules and their versions, the
+ * operand splits, the MMA shapes and the compile flags (numerical policy);
+ * and settings that do not change bits such as the ABI version and the SM
+ * count of the current device (deployment).
+ * Status: GDN_ERR_INVALID_ARG for an unknown kind or a NULL output,
+ * GDN_ERR_UNSUPPORTED for a shape or dtype the library does not run.
+ */
+typedef enum {
+  GDN_DIGEST_SEMANTIC = 0,
+  GDN_DIGEST_POLICY = 1,
+  GDN_DIGEST_DEPLOYMENT = 2
+} gdn_digest_kind;
+
+/* The descriptor text (NUL-terminated) into buf[buf_bytes]; *len_out = its
+ * length without the NUL.  buf == NULL only queries the length;
+ * GDN_ERR_INVALID_ARG when buf is too small. */
+int gdn_cpr_contract_descriptor(int kind, int in_dtype, int out_dtype, int dk, int dv, int C,
+                                char* buf, size_t buf_bytes, size_t* len_out);
+
+/* out32[32] = SHA-256 of that descriptor. */
+int gdn_cpr_contract_digest(int kind, int in_dtype, int out_dtype, int dk, int dv, int C,
+                            uint8_t* out32);
+
+/* Refuse to mix: GDN_OK when peer_policy32[32] equals this library's
+ * numerical-policy digest for the shape, GDN_ERR_CONTRACT when it differs. */
+int gdn_cpr_contract_check(const uint8_t* peer_policy32, int in_dtype, int out_dtype, int dk,
+                           int dv, int C);
+
+/* out32[32] = SHA-256 of data[n] (the hash the digests use). */
+int gdn_sha256(const void* data, size_t n, uint8_t* out32);
 
 #ifdef __cplusplus
 }

@@ -23,10 +23,15 @@ GDN_ERR_WORKSPACE = -3
 GDN_ERR_CUDA = -4
 GDN_ERR_DEVICE_DATA = -5
 GDN_ERR_TIMEOUT = -6
+GDN_ERR_CONTRACT = -7
+GDN_DIGEST_SEMANTIC = 0
+GDN_DIGEST_POLICY = 1
+GDN_DIGEST_DEPLOYMENT = 2
 GDN_BF16 = 0
 GDN_F32 = 1
 GDN_DEVERR_CU_SEQLENS = 1
 GDN_DEVERR_POS = 2
+GDN_DEVERR_TIMEOUT = 4
 CHUNK = 64
 
 
@@ -69,6 +74,11 @@ def _load() -> ctypes.CDLL:
                                       DecodeStateStruct, vp, i32, vp]),
         "gdn_chunk_boundary": (i32, [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
         "gdn_check_error": (i32, [vp, vp, vp]),
+        "gdn_cpr_contract_descriptor": (i32, [i32, i32, i32, i32, i32, i32, ctypes.c_char_p, sz,
+                                              ctypes.POINTER(ctypes.c_size_t)]),
+        "gdn_cpr_contract_digest": (i32, [i32, i32, i32, i32, i32, i32, ctypes.c_char_p]),
+        "gdn_cpr_contract_check": (i32, [ctypes.c_char_p, i32, i32, i32, i32, i32]),
+        "gdn_sha256": (i32, [ctypes.c_char_p, sz, ctypes.c_char_p]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -260,3 +270,44 @@ def chunk_boundary(s_start, k, v, beta, g, *, s_end=None, stream=None):
                                 _ptr(g), B, H, dk, dv, C, _ptr(s_end), _stream(stream))
     _check(st, "gdn_chunk_boundary")
     return s_end
+
+
+def _dt(dtype) -> int:
+    return GDN_BF16 if dtype == torch.bfloat16 else GDN_F32 if dtype == torch.float32 else -1
+
+
+def contract_descriptor(kind: int, in_dtype=torch.bfloat16, out_dtype=torch.bfloat16, dk: int = 128,
+                        dv: int = 128, C: int = CHUNK) -> str:
+    """gdn_cpr_contract_descriptor: the canonical text a digest hashes."""
+    n = ctypes.c_size_t(0)
+    args = (kind, _dt(in_dtype), _dt(out_dtype), dk, dv, C)
+    _check(lib.gdn_cpr_contract_descriptor(*args, None, 0, ctypes.byref(n)),
+           "gdn_cpr_contract_descriptor")
+    buf = ctypes.create_string_buffer(n.value + 1)
+    _check(lib.gdn_cpr_contract_descriptor(*args, buf, n.value + 1, ctypes.byref(n)),
+           "gdn_cpr_contract_descriptor")
+    return buf.value.decode()
+
+
+def contract_digest(kind: int, in_dtype=torch.bfloat16, out_dtype=torch.bfloat16, dk: int = 128,
+                    dv: int = 128, C: int = CHUNK) -> bytes:
+    """gdn_cpr_contract_digest: 32-byte SHA-256 identity digest."""
+    out = ctypes.create_string_buffer(32)
+    _check(lib.gdn_cpr_contract_digest(kind, _dt(in_dtype), _dt(out_dtype), dk, dv, C, out),
+           "gdn_cpr_contract_digest")
+    return out.raw
+
+
+def contract_check(peer_policy: bytes, in_dtype=torch.bfloat16, out_dtype=torch.bfloat16,
+                   dk: int = 128, dv: int = 128, C: int = CHUNK) -> int:
+    """gdn_cpr_contract_check: GDN_OK, or GDN_ERR_CONTRACT when the policies differ."""
+    if len(peer_policy) != 32:
+        raise ValueError("a digest is 32 bytes")
+    return lib.gdn_cpr_contract_check(peer_policy, _dt(in_dtype), _dt(out_dtype), dk, dv, C)
+
+
+def sha256(data: bytes) -> bytes:
+    """gdn_sha256 of a byte string."""
+    out = ctypes.create_string_buffer(32)
+    _check(lib.gdn_sha256(data, len(data), out), "gdn_sha256")
+    return out.raw

@@ -42,6 +42,7 @@ const char* gdn_status_string(int status) {
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA launch or runtime error";
     case GDN_ERR_DEVICE_DATA: return "GDN_ERR_DEVICE_DATA: device-side validation failed";
     case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: bounded device wait gave up";
+    case GDN_ERR_CONTRACT: return "GDN_ERR_CONTRACT: numerical policies differ";
     default: return "unknown gdn_status";
   }
 }
