@@ -40,20 +40,27 @@ FLUSH_BYTES = 256 << 20
 PAGES_H100 = {"prefill_ms": 1.412, "decode_ms": 0.0846, "trainer_fwd_bwd_ms": 7.386}
 
 
+def kernel_sources_sha256() -> str:
+    """SHA-256 over the files that define the kernels (gdn_kernels.cu and the
+    device headers; the host-only entry points are left out)."""
+    import hashlib
+    csrc = os.path.join(ROOT, "rl_train_numerics_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name == "gdn_kernels.cu" or name.endswith((".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
 def ncu_traffic(kernel: str):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when
     the kernel sources have changed since that capture."""
-    import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
             rec = json.load(f)
-        csrc = os.path.join(ROOT, "rl_train_numerics_b200", "csrc")
-        h = hashlib.sha256()
-        for name in sorted(os.listdir(csrc)):
-            if name.endswith((".cu", ".cuh", ".h")):
-                with open(os.path.join(csrc, name), "rb") as f:
-                    h.update(f.read())
-        if h.hexdigest() != rec.get("kernel_sources_sha256"):
+        digest = kernel_sources_sha256()
+        if digest != rec.get("kernel_sources_sha256"):
             return None
         return rec.get("traffic_bytes", {}).get(kernel)
     except (OSError, ValueError):
