@@ -312,6 +312,17 @@ int gdn_cpr_contract_check(const uint8_t* peer_policy32, int in_dtype, int out_d
 /* out32[32] = SHA-256 of data[n] (the hash the digests use). */
 int gdn_sha256(const void* data, size_t n, uint8_t* out32);
 
+/*
+ * gdn_selftest_bounded_wait -- exercise the give-up path of the boundary
+ * walk's bounded waits (this library's own safeguard; the pages have no
+ * counterpart).  One block allocates tensor memory as the walk does, waits
+ * `polls` polls (1 .. 2^22) on a completion barrier that nothing arrives at,
+ * sets GDN_DEVERR_TIMEOUT in *error_word (device int32), frees the tensor
+ * memory and returns; the context stays usable.  Asynchronous on `stream`;
+ * read the bit with gdn_check_error.
+ */
+int gdn_selftest_bounded_wait(int polls, int32_t* error_word, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

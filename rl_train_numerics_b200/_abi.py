@@ -79,6 +79,7 @@ def _load() -> ctypes.CDLL:
         "gdn_cpr_contract_digest": (i32, [i32, i32, i32, i32, i32, i32, ctypes.c_char_p]),
         "gdn_cpr_contract_check": (i32, [ctypes.c_char_p, i32, i32, i32, i32, i32]),
         "gdn_sha256": (i32, [ctypes.c_char_p, sz, ctypes.c_char_p]),
+        "gdn_selftest_bounded_wait": (i32, [i32, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)

@@ -179,3 +179,10 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         gdn.forward(x, x, x, torch.zeros(4, 2), torch.zeros(4, 2),
                     torch.tensor([0, 4], dtype=torch.int32))
+
+
+def test_selftest_rejects_on_host():
+    L = gdn.lib
+    assert L.gdn_selftest_bounded_wait(0, FAKE, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_selftest_bounded_wait((1 << 22) + 1, FAKE, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_selftest_bounded_wait(10, None, None) == gdn.GDN_ERR_INVALID_ARG
