@@ -25,6 +25,9 @@ Functions
 ---------
 forward / forward_alpha   the token loop, in C (``gdn_oracle.c``), OpenMP
                           over (sequence, head) units.
+backward                  its reverse mode (the gradient of a loss through the
+                          token loop), in C, fp64, with the states recomputed
+                          from checkpoints every 64 tokens.
 explicit_product_state    the closed product form of the recurrence with the
                           per-token transition matrices written out, in
                           float64 (numpy matmul) or exact rationals
@@ -77,6 +80,11 @@ def _load():
             fn.restype = ctypes.c_int
             fn.argtypes = [dp, dp, dp, dp, dp, ip, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                            ctypes.c_int, ctypes.c_double, dp, dp, dp, ctypes.c_int]
+        fb = lib.gdn_oracle_backward
+        fb.restype = ctypes.c_int
+        fb.argtypes = [dp, dp, dp, dp, dp, ip, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                       ctypes.c_int, ctypes.c_double, dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                       ctypes.c_int]
         lib.gdn_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -136,6 +144,38 @@ def forward_alpha(q, k, v, beta, alpha, cu_seqlens, h0=None, scale: float = 1.0,
                   threads: Optional[int] = None):
     """Same recurrence with the decay alpha_t given directly (alpha = 0 allowed)."""
     return _run("gdn_oracle_forward_alpha", q, k, v, beta, alpha, cu_seqlens, h0, scale, threads)
+
+
+def backward(q, k, v, beta, g, cu_seqlens, do, h0=None, ds_final=None, scale: float = 1.0,
+             threads: Optional[int] = None):
+    """Reverse mode of the token loop (fp64): the gradient of a loss L given
+    do = dL/do [T,H,dv] and ds_final = dL/dS_final [N,H,dv,dk] (None = 0).
+    Returns dict(dq, dk [T,H,dk], dv [T,H,dv], dbeta, dg [T,H], dh0 [N,H,dv,dk])."""
+    q, k, v, beta, g, do = (_f64(a) for a in (q, k, v, beta, g, do))
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    n = cu.shape[0] - 1
+    assert k.shape == (T, H, dk) and v.shape == (T, H, dv) and do.shape == (T, H, dv)
+    assert beta.shape == (T, H) and g.shape == (T, H)
+    assert n >= 0 and int(cu[0]) == 0 and int(cu[-1]) == T
+    h0a = None if h0 is None else _f64(h0)
+    dsf = None if ds_final is None else _f64(ds_final)
+    out = {"dq": np.zeros((T, H, dk)), "dk": np.zeros((T, H, dk)), "dv": np.zeros((T, H, dv)),
+           "dbeta": np.zeros((T, H)), "dg": np.zeros((T, H)), "dh0": np.zeros((n, H, dv, dk))}
+    dp = ctypes.POINTER(ctypes.c_double)
+
+    def ptr(a):
+        return None if a is None else a.ctypes.data_as(dp)
+
+    rc = _load().gdn_oracle_backward(
+        ptr(q), ptr(k), ptr(v), ptr(beta), ptr(g),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n, H, dk, dv, float(scale),
+        ptr(h0a), ptr(do), ptr(dsf), ptr(out["dq"]), ptr(out["dk"]), ptr(out["dv"]),
+        ptr(out["dbeta"]), ptr(out["dg"]), ptr(out["dh0"]), int(threads or 0))
+    if rc != 0:
+        raise ValueError(f"gdn_oracle_backward failed with status {rc}")
+    return out
 
 
 # ---------------------------------------------------------------------------

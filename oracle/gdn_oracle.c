@@ -145,3 +145,168 @@ int gdn_oracle_max_threads(void) {
   return 1;
 #endif
 }
+
+/*
+ * Reverse mode of the same recurrence (the gradient of a loss through the
+ * token loop above, plain definition, fp64).  Given dO = dL/do_t and dS_end =
+ * dL/dS_final, it returns dL/dq, dL/dk, dL/dv, dL/dbeta, dL/dg and dL/dh0.
+ * Per token, with p = S_{t-1} k_t, a = exp(g_t), b = beta_t and
+ * S_t = a (S_{t-1} - b p k^T) + b v k^T, o_t = scale S_t q_t, walking t
+ * downwards with dS = dL/dS_t:
+ *   dS   += scale do_t q_t^T           dq_t  = scale S_t^T do_t
+ *   w     = dS k_t                     da    = <dS, S_{t-1}> - b w.p
+ *   dbeta = w.(v_t - a p)              dv_t  = b w
+ *   dk_t  = dS^T (b (v_t - a p)) + S_{t-1}^T dp,   dp = -a b w
+ *   dg_t  = a da                       dS_{t-1} = a dS + dp k_t^T
+ * and finally dh0 = dS.  States are kept at every ORACLE_CKPT-th token and the
+ * ones in between recomputed by the forward loop (the same operations in the
+ * same order, so the same values).
+ */
+#define ORACLE_CKPT 64
+
+static void fwd_token(double* S, double* p, const double* kt, const double* vt, double a,
+                      double b, int dk, int dv) {
+  for (int r = 0; r < dv; r++) {
+    double acc = 0.0;
+    for (int j = 0; j < dk; j++) acc += S[(size_t)r * dk + j] * kt[j];
+    p[r] = acc;
+  }
+  for (int r = 0; r < dv; r++)
+    for (int j = 0; j < dk; j++) {
+      double s = S[(size_t)r * dk + j];
+      S[(size_t)r * dk + j] = a * (s - b * p[r] * kt[j]) + b * vt[r] * kt[j];
+    }
+}
+
+static void bwd_unit(const double* q, const double* k, const double* v, const double* beta,
+                     const double* g, int64_t t0, int64_t t1, int H, int h, int dk, int dv,
+                     double scale, const double* s0, const double* dO, const double* dS_end,
+                     double* dq, double* dkk, double* dvv, double* dbeta, double* dg,
+                     double* dh0, double* ck, double* st, double* dS, double* p, double* w) {
+  const size_t DD = (size_t)dv * dk;
+  const int64_t L = t1 - t0;
+  const int64_t nck = (L + ORACLE_CKPT - 1) / ORACLE_CKPT;
+  /* checkpoints: state before token t0 + c * ORACLE_CKPT */
+  if (s0) memcpy(ck, s0, sizeof(double) * DD);
+  else memset(ck, 0, sizeof(double) * DD);
+  for (int64_t c = 1; c < nck; c++) {
+    memcpy(ck + (size_t)c * DD, ck + (size_t)(c - 1) * DD, sizeof(double) * DD);
+    for (int64_t t = t0 + (c - 1) * ORACLE_CKPT; t < t0 + c * ORACLE_CKPT; t++) {
+      const size_t u = (size_t)t * H + h;
+      fwd_token(ck + (size_t)c * DD, p, k + u * dk, v + u * dv, exp(g[u]), beta[u], dk, dv);
+    }
+  }
+  if (dS_end) memcpy(dS, dS_end, sizeof(double) * DD);
+  else memset(dS, 0, sizeof(double) * DD);
+  for (int64_t c = nck - 1; c >= 0; c--) {
+    const int64_t a0 = t0 + c * ORACLE_CKPT;
+    const int64_t a1 = (a0 + ORACLE_CKPT < t1) ? a0 + ORACLE_CKPT : t1;
+    /* st[i] = state before token a0 + i, i = 0 .. a1 - a0 (last = after a1 - 1) */
+    memcpy(st, ck + (size_t)c * DD, sizeof(double) * DD);
+    for (int64_t t = a0; t < a1; t++) {
+      const size_t u = (size_t)t * H + h;
+      double* nx = st + (size_t)(t - a0 + 1) * DD;
+      memcpy(nx, st + (size_t)(t - a0) * DD, sizeof(double) * DD);
+      fwd_token(nx, p, k + u * dk, v + u * dv, exp(g[u]), beta[u], dk, dv);
+    }
+    for (int64_t t = a1 - 1; t >= a0; t--) {
+      const size_t u = (size_t)t * H + h;
+      const double* Sp = st + (size_t)(t - a0) * DD;      /* S_{t-1} */
+      const double* Sc = st + (size_t)(t - a0 + 1) * DD;  /* S_t */
+      const double *kt = k + u * dk, *vt = v + u * dv, *qt = q + u * dk, *dot = dO + u * dv;
+      const double a = exp(g[u]), b = beta[u];
+      for (int r = 0; r < dv; r++)
+        for (int j = 0; j < dk; j++) dS[(size_t)r * dk + j] += scale * dot[r] * qt[j];
+      for (int j = 0; j < dk; j++) {
+        double acc = 0.0;
+        for (int r = 0; r < dv; r++) acc += Sc[(size_t)r * dk + j] * dot[r];
+        dq[u * dk + j] = scale * acc;
+      }
+      for (int r = 0; r < dv; r++) {
+        double acc = 0.0, pr = 0.0;
+        for (int j = 0; j < dk; j++) {
+          acc += dS[(size_t)r * dk + j] * kt[j];
+          pr += Sp[(size_t)r * dk + j] * kt[j];
+        }
+        w[r] = acc;
+        p[r] = pr;
+      }
+      double da = 0.0, db = 0.0;
+      for (size_t e = 0; e < DD; e++) da += dS[e] * Sp[e];
+      for (int r = 0; r < dv; r++) {
+        da -= b * w[r] * p[r];
+        db += w[r] * (vt[r] - a * p[r]);
+        dvv[u * dv + r] = b * w[r];
+      }
+      for (int j = 0; j < dk; j++) {
+        double acc = 0.0;
+        for (int r = 0; r < dv; r++) {
+          const double dpr = -a * b * w[r];
+          acc += dS[(size_t)r * dk + j] * (b * (vt[r] - a * p[r])) + Sp[(size_t)r * dk + j] * dpr;
+        }
+        dkk[u * dk + j] = acc;
+      }
+      dbeta[u] = db;
+      dg[u] = a * da;
+      for (int r = 0; r < dv; r++) {
+        const double dpr = -a * b * w[r];
+        for (int j = 0; j < dk; j++)
+          dS[(size_t)r * dk + j] = a * dS[(size_t)r * dk + j] + dpr * kt[j];
+      }
+    }
+  }
+  if (dh0) memcpy(dh0, dS, sizeof(double) * DD);
+}
+
+int gdn_oracle_backward(const double* q, const double* k, const double* v, const double* beta,
+                        const double* g, const int32_t* cu_seqlens, int n_seqs, int H, int dk,
+                        int dv, double scale, const double* h0, const double* dO,
+                        const double* dS_end, double* dq, double* dkk, double* dvv,
+                        double* dbeta, double* dg, double* dh0, int n_threads) {
+  if (!q || !k || !v || !beta || !g || !cu_seqlens || !dO || !dq || !dkk || !dvv || !dbeta ||
+      !dg)
+    return ORACLE_BAD_ARG;
+  if (n_seqs < 0 || H <= 0 || dk <= 0 || dv <= 0 || cu_seqlens[0] != 0) return ORACLE_BAD_ARG;
+  int64_t maxlen = 0;
+  for (int n = 0; n < n_seqs; n++) {
+    if (cu_seqlens[n + 1] < cu_seqlens[n]) return ORACLE_BAD_ARG;
+    if (cu_seqlens[n + 1] - cu_seqlens[n] > maxlen) maxlen = cu_seqlens[n + 1] - cu_seqlens[n];
+  }
+  const size_t DD = (size_t)dv * dk;
+  const int64_t nck = (maxlen + ORACLE_CKPT - 1) / ORACLE_CKPT + 1;
+  const int64_t units = (int64_t)n_seqs * H;
+  int failed = 0;
+#ifdef _OPENMP
+  if (n_threads <= 0) n_threads = omp_get_max_threads();
+#pragma omp parallel num_threads(n_threads)
+#endif
+  {
+    double* ck = (double*)malloc(sizeof(double) * DD * (size_t)nck);
+    double* st = (double*)malloc(sizeof(double) * DD * (ORACLE_CKPT + 1));
+    double* dS = (double*)malloc(sizeof(double) * DD);
+    double* p = (double*)malloc(sizeof(double) * (size_t)dv);
+    double* w = (double*)malloc(sizeof(double) * (size_t)dv);
+    if (!ck || !st || !dS || !p || !w) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+      failed = 1;
+    } else {
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+      for (int64_t u = 0; u < units; u++) {
+        const int n = (int)(u / H), h = (int)(u % H);
+        bwd_unit(q, k, v, beta, g, cu_seqlens[n], cu_seqlens[n + 1], H, h, dk, dv, scale,
+                 h0 ? h0 + (size_t)u * DD : NULL, dO, dS_end ? dS_end + (size_t)u * DD : NULL,
+                 dq, dkk, dvv, dbeta, dg, dh0 ? dh0 + (size_t)u * DD : NULL, ck, st, dS, p, w);
+      }
+    }
+    free(ck);
+    free(st);
+    free(dS);
+    free(p);
+    free(w);
+  }
+  return failed ? ORACLE_NO_MEMORY : ORACLE_OK;
+}
