@@ -270,6 +270,90 @@ __device__ __forceinline__ void prep_stage(PrepSmem<D, IN>& sm, const IN* k, siz
 // Prep of one chunk: sm.K, sm.beta, sm.g staged -> sm.head (Tb, Tv, dvec,
 // gamma), with AT as scratch.  The first kBndThreads threads do the work;
 // every thread of the block takes the barriers.  Ends with a block barrier.
+// CPT consecutive floats of a row of AT (16-byte loads where CPT allows).
+template <int CPT>
+__device__ __forceinline__ void at_row(float (&x)[CPT], const float* src) {
+  if constexpr (CPT % 4 == 0) {
+#pragma unroll
+    for (int e = 0; e < CPT; e += 4) {
+      const float4 u = *reinterpret_cast<const float4*>(src + e);
+      x[e] = u.x, x[e + 1] = u.y, x[e + 2] = u.z, x[e + 3] = u.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < CPT; e += 2) {
+      const float2 u = *reinterpret_cast<const float2*>(src + e);
+      x[e] = u.x, x[e + 1] = u.y;
+    }
+  }
+}
+template <int CPT>
+__device__ __forceinline__ void at_row_store(float* dst, const float2 (&x)[CPT / 2], float sgn) {
+#pragma unroll
+  for (int e = 0; e < CPT / 2; e++)
+    *reinterpret_cast<float2*>(dst + 2 * e) = f2(sgn * x[e].x, sgn * x[e].y);
+}
+
+// Stage ST of the blocked inverse (see bnd_prep): the blocks (b, c) of T with
+// b - c = ST, thread (block, row i, columns j0 .. j0 + CPT - 1).  X = the sum
+// over k = c .. b-1 of A_bk T_kc (one fma chain per element, ascending inner
+// index), then T_bc = -(D_b X) (from X_ij, D_b[i][k] X_kj in ascending k < i).
+// Packed pairs of fmas: each element's arithmetic is the scalar fma chain.
+template <int ST, int CPT>
+__device__ __forceinline__ void t_stage(PrepAT& AT, float* X, int tid) {
+  constexpr int NB = 16, NBLK = kChunk / NB - ST, TPB = NB * NB / CPT;
+  const int blk = tid / TPB, rem = tid % TPB;
+  const int i = rem / (NB / CPT), j0 = (rem % (NB / CPT)) * CPT;
+  const int c0 = blk * NB, b0 = c0 + ST * NB;
+  float* Xr = X + blk * NB * NB;
+  const bool active = blk < NBLK;
+  if (active) {
+    float2 acc[CPT / 2];
+#pragma unroll
+    for (int e = 0; e < CPT / 2; e++) acc[e] = f2(0.f, 0.f);
+#pragma unroll
+    for (int kb = 0; kb < ST; kb++) {
+      const int k0 = c0 + kb * NB;
+#pragma unroll
+      for (int q = 0; q < NB; q++) {
+        const float a = AT[k0 + q][b0 + i];  // A_{b0+i, k0+q}
+        float tv[CPT];
+        at_row<CPT>(tv, &AT[k0 + q][c0 + j0]);
+        if (kb == 0) {
+#pragma unroll
+          for (int e = 0; e < CPT; e++)
+            if (q < j0 + e) tv[e] = 0.f;  // above T's diagonal (A lives there)
+        }
+#pragma unroll
+        for (int e = 0; e < CPT / 2; e++) acc[e] = __ffma2_rn(f2(a, a), f2(tv[2 * e], tv[2 * e + 1]), acc[e]);
+      }
+    }
+    at_row_store<CPT>(Xr + i * NB + j0, acc, 1.f);
+  }
+  __syncthreads();
+  if (active) {
+    float2 acc[CPT / 2];
+    {
+      float x[CPT];
+      at_row<CPT>(x, Xr + i * NB + j0);
+#pragma unroll
+      for (int e = 0; e < CPT / 2; e++) acc[e] = f2(x[2 * e], x[2 * e + 1]);
+    }
+#pragma unroll
+    for (int k = 0; k < NB - 1; k++) {
+      if (k < i) {
+        const float d = AT[b0 + k][b0 + i];  // D_b[i][k]
+        float y[CPT];
+        at_row<CPT>(y, Xr + k * NB + j0);
+#pragma unroll
+        for (int e = 0; e < CPT / 2; e++) acc[e] = __ffma2_rn(f2(d, d), f2(y[2 * e], y[2 * e + 1]), acc[e]);
+      }
+    }
+    at_row_store<CPT>(&AT[b0 + i][c0 + j0], acc, -1.f);
+  }
+  __syncthreads();
+}
+
 struct PrepNoHook {
   __device__ void operator()() const {}
 };
@@ -402,72 +486,22 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT, const AfterP& after_p 
         if (i > j) AT[b0 + j][b0 + i] = AT[b0 + i][b0 + j];
     }
     __syncthreads();
-    // Stages: thread (block, row i, 8 columns j0..j0+7), 8 accumulators.
+    // Stages s = 1, 2, 3: thread (block, row i, CPT columns), CPT = 8, 4, 2
+    // so that every stage but the first keeps all 128 threads busy.
     float* X = reinterpret_cast<float*>(sm.head.TbT[0]);  // scratch until the splits below
-#pragma unroll
-    for (int st = 1; st < kChunk / NB; st++) {
-      const int nblk = kChunk / NB - st;
-      const int blk = tid / (2 * NB), i = (tid % (2 * NB)) / 2, j0 = (tid % 2) * 8;
-      const int c0 = blk * NB, b0 = c0 + st * NB;
-      float* Xr = X + blk * NB * NB;
-      if (blk < nblk) {
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; e++) acc[e] = 0.f;
-#pragma unroll
-        for (int kb = 0; kb < st; kb++) {
-          const int k0 = c0 + kb * NB;
-#pragma unroll
-          for (int q = 0; q < NB; q++) {
-            const float a = AT[k0 + q][b0 + i];  // A_{b0+i, k0+q}
-            const float4 u0 = *reinterpret_cast<const float4*>(&AT[k0 + q][c0 + j0]);
-            const float4 u1 = *reinterpret_cast<const float4*>(&AT[k0 + q][c0 + j0 + 4]);
-            float tv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-            for (int e = 0; e < 8; e++) {
-              if (kb == 0 && q < j0 + e) tv[e] = 0.f;  // above T's diagonal (A lives there)
-              acc[e] = __fmaf_rn(a, tv[e], acc[e]);
-            }
-          }
-        }
-        *reinterpret_cast<float4*>(Xr + i * NB + j0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4*>(Xr + i * NB + j0 + 4) =
-            make_float4(acc[4], acc[5], acc[6], acc[7]);
-      }
-      __syncthreads();
-      if (blk < nblk) {
-        float acc[8];
-        const float4 x0 = *reinterpret_cast<const float4*>(Xr + i * NB + j0);
-        const float4 x1 = *reinterpret_cast<const float4*>(Xr + i * NB + j0 + 4);
-        acc[0] = x0.x, acc[1] = x0.y, acc[2] = x0.z, acc[3] = x0.w;
-        acc[4] = x1.x, acc[5] = x1.y, acc[6] = x1.z, acc[7] = x1.w;
-#pragma unroll
-        for (int k = 0; k < NB - 1; k++) {
-          if (k < i) {
-            const float d = AT[b0 + k][b0 + i];  // D_b[i][k]
-            const float4 y0 = *reinterpret_cast<const float4*>(Xr + k * NB + j0);
-            const float4 y1 = *reinterpret_cast<const float4*>(Xr + k * NB + j0 + 4);
-            const float yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-#pragma unroll
-            for (int e = 0; e < 8; e++) acc[e] = __fmaf_rn(d, yv[e], acc[e]);
-          }
-        }
-        *reinterpret_cast<float4*>(&AT[b0 + i][c0 + j0]) =
-            make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-        *reinterpret_cast<float4*>(&AT[b0 + i][c0 + j0 + 4]) =
-            make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
-      }
-      __syncthreads();
-    }
+    t_stage<1, 8>(AT, X, tid);
+    t_stage<2, 4>(AT, X, tid);
+    t_stage<3, 2>(AT, X, tid);
   }
 
   // Tb = T diag(beta*gamma), Tv = T diag(beta), split into bf16 terms; thread
-  // j's column of T is row j of the transposed tiles: 16-byte stores.
-  if (tid < kChunk) {
-    const int j = tid;
+  // (j, half) takes rows 32 half .. 32 half + 31 of column j of T, which is
+  // row j of the transposed tiles: 16-byte stores.
+  if (tid < 2 * kChunk) {
+    const int j = tid % kChunk, i0 = (tid / kChunk) * (kChunk / 2);
     const float bgj = sm.bg[j], bj = sm.beta[j];
 #pragma unroll
-    for (int i8 = 0; i8 < kChunk; i8 += 8) {
+    for (int i8 = i0; i8 < i0 + kChunk / 2; i8 += 8) {
       __nv_bfloat16 sb[8][NW], sv[8][NW];
 #pragma unroll
       for (int e = 0; e < 8; e++) {
