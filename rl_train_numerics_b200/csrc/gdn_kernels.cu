@@ -36,7 +36,7 @@ constexpr int kTableThreads = 1024;
 __global__ void __launch_bounds__(kTableThreads)
     k_chunk_table(const int32_t* __restrict__ cu, int N, int64_t T, int32_t* hdr,
                   int32_t* chunk_off, int32_t* chunk_seq, int64_t max_chunks) {
-  __shared__ long long part[kTableThreads];
+  __shared__ long long part[64 + kTableThreads];
   __shared__ int bad;
   const int tid = threadIdx.x;
   if (tid == 0) bad = (cu[0] != 0 || (int64_t)cu[N] != T) ? 1 : 0;
@@ -52,15 +52,30 @@ __global__ void __launch_bounds__(kTableThreads)
     else local += (L + kChunk - 1) / kChunk;
   }
   if (mybad) atomicOr(&bad, 1);
-  part[tid] = local;
+  // Exclusive prefix sum of the per-thread chunk counts: inclusive scans
+  // inside each warp, then over the warp totals.
+  const int lane = tid & 31, warp = tid >> 5;
+  long long x = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const long long y = __shfl_up_sync(kFull, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) part[warp] = x;
   __syncthreads();
-  if (tid == 0) {
-    long long run = 0;
-    for (int i = 0; i < kTableThreads; i++) {
-      const long long x = part[i];
-      part[i] = run;
-      run += x;
+  if (warp == 0) {
+    long long wsum = part[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long y = __shfl_up_sync(kFull, wsum, off);
+      if (lane >= off) wsum += y;
     }
+    part[32 + lane] = wsum;  // inclusive over warps 0 .. lane
+  }
+  __syncthreads();
+  const long long run = part[32 + 31];
+  part[64 + tid] = x - local + (warp > 0 ? part[32 + warp - 1] : 0);  // exclusive, this thread
+  if (tid == 0) {
     if (run > max_chunks) bad = 1;
     hdr[kHdrChunks] = bad ? 0 : (int32_t)run;
     hdr[kHdrFillNext] = 0;
@@ -74,7 +89,7 @@ __global__ void __launch_bounds__(kTableThreads)
     }
     return;
   }
-  long long off = part[tid];
+  long long off = part[64 + tid];
   for (int64_t n = n0; n < n1; n++) {
     const int64_t L = (int64_t)cu[n + 1] - (int64_t)cu[n];
     const long long nc = (L + kChunk - 1) / kChunk;
