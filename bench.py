@@ -255,35 +255,82 @@ def bench_prefill(gdn, W, dev, rank, steps, warmup, flush):
 
 
 def bench_e2e(gdn, b, dev, steps, warmup):
-    """Host buffers in, host output back: H2D of the step's inputs from pinned
-    memory, the forward, D2H of o, all on one stream inside the events."""
+    """Host buffers in, host output back, through the public forward: every step
+    copies its inputs from pinned host memory (H2D), runs the forward and copies
+    o back (D2H), all inside the timed region.  Measured two ways:
+      serial     one stream: H2D, forward, D2H back to back;
+      pipelined  a streaming caller: H2D on one copy stream, forwards on a
+                 compute stream, D2H on another copy stream, double-buffered
+                 device inputs and outputs, so step i+1's H2D and step i-1's D2H
+                 overlap step i's forward (events order every reuse of a buffer).
+    Returns (serial ms, pipelined ms, h2d bytes, d2h bytes) per step."""
     host = [t.cpu().pin_memory() for t in (b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens)]
-    devb = [torch.empty_like(t, device=dev) for t in host]
+    devb = [[torch.empty_like(t, device=dev) for t in host] for _ in range(2)]
     T = b.total_tokens
-    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
-    o_host = torch.empty((T, H, D), dtype=torch.bfloat16).pin_memory()
+    o = [torch.empty((T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    o_host = [torch.empty((T, H, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     ws = torch.zeros(gdn.forward_workspace_bytes(len(b.lengths), T, H, D, D), dtype=torch.uint8,
                      device=dev)
     h2d = sum(t.numel() * t.element_size() for t in host)
-    d2h = o_host.numel() * o_host.element_size()
+    d2h = o_host[0].numel() * o_host[0].element_size()
 
-    def one():
-        for dst, src in zip(devb, host):
+    def serial_step():
+        for dst, src in zip(devb[0], host):
             dst.copy_(src, non_blocking=True)
-        gdn.forward(*devb, o=o, workspace=ws, want_states=False)
-        o_host.copy_(o, non_blocking=True)
+        gdn.forward(*devb[0], o=o[0], workspace=ws, want_states=False)
+        o_host[0].copy_(o[0], non_blocking=True)
 
     for _ in range(warmup):
-        one()
+        serial_step()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(steps):
-        one()
+        serial_step()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    return ms, h2d, d2h
+    serial_ms = e0.elapsed_time(e1) / steps
+
+    s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def pipelined(n):
+        done_run, done_out = {}, {}
+        for i in range(n):
+            slot = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(done_run[i - 2])  # the forward of step i-2 read this slot
+                for dst, src in zip(devb[slot], host):
+                    dst.copy_(src, non_blocking=True)
+                got = torch.cuda.Event()
+                got.record(s_in)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(got)
+                if i >= 2:
+                    s_run.wait_event(done_out[i - 2])  # o of step i-2 has left the device
+                gdn.forward(*devb[slot], o=o[slot], workspace=ws, want_states=False)
+                done_run[i] = torch.cuda.Event()
+                done_run[i].record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done_run[i])
+                o_host[slot].copy_(o[slot], non_blocking=True)
+                done_out[i] = torch.cuda.Event()
+                done_out[i].record(s_out)
+        return done_out[n - 1]
+
+    pipelined(max(warmup, 2))
+    torch.cuda.synchronize()
+    p0 = torch.cuda.Event(enable_timing=True)
+    p0.record(s_in)
+    s_run.wait_event(p0)
+    s_out.wait_event(p0)
+    last = pipelined(steps)
+    p1 = torch.cuda.Event(enable_timing=True)
+    s_out.wait_event(last)
+    p1.record(s_out)
+    torch.cuda.synchronize()
+    pipe_ms = p0.elapsed_time(p1) / steps
+    return serial_ms, pipe_ms, h2d, d2h
 
 
 def bench_decode(gdn, W, dev, rank, steps, warmup, slots=256):
@@ -427,10 +474,17 @@ def run_ours(args):
 
     e2e = None
     if args.only == "all":
-        e2e_ms, h2d, d2h = bench_e2e(gdn, b, dev, args.steps, args.warmup)
-        e2e_ms = max_over_ranks(e2e_ms, world)
-        e2e = {"value": round(world * T / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        serial_ms, pipe_ms, h2d, d2h = bench_e2e(gdn, b, dev, args.steps, args.warmup)
+        serial_ms = max_over_ranks(serial_ms, world)
+        pipe_ms = max_over_ranks(pipe_ms, world)
+        e2e = {"value": round(world * T / (pipe_ms / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(pipe_ms, 4),
+               "mode": "pipelined: H2D, forward and D2H on three streams, double-buffered, "
+                       "every step's copies inside the timed region",
+               "serial": {"value": round(world * T / (serial_ms / 1e3), 1),
+                          "ms_per_step": round(serial_ms, 4),
+                          "mode": "one stream: H2D, forward, D2H back to back"}}
     decode = None
     if args.only in ("all", "decode"):
         decode = run_decode_part(gdn, W, dev, rank, world, args, peaks)
