@@ -386,6 +386,54 @@ def run_decode_part(gdn, W, dev, rank, world, args, peaks):
             "pages_h100_ms": PAGES_H100["decode_ms"]}
 
 
+def run_train_part(gdn, W, dev, rank, world, args, flush):
+    """Trainer step: the forward (o and final states) and the backward (every
+    gradient, from a fixed synthetic dL/do) over the 10240-token trainer batch,
+    L2 flushed before every step outside its events."""
+    b = W.trainer(device=dev, seed=rank)
+    T, N = b.total_tokens, len(b.lengths)
+    gen = torch.Generator(device=dev).manual_seed(1000 + rank)
+    d_o = torch.randn((T, H, D), generator=gen, device=dev).to(torch.bfloat16)
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    srun = torch.empty((N, H, D, D), dtype=torch.float32, device=dev)
+    fws = torch.zeros(gdn.forward_workspace_bytes(N, T, H, D, D), dtype=torch.uint8, device=dev)
+    grads, bws = gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o)
+
+    def step(e0, e1, e2):
+        e0.record()
+        gdn.forward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, o=o, s_run_final=srun,
+                    workspace=fws)
+        e1.record()
+        gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o, grads=grads, workspace=bws)
+        e2.record()
+
+    steps, warmup = args.steps, args.warmup
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for _ in range(warmup):
+        flush.zero_()
+        step(*evs[0])
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        step(*evs[i])
+    torch.cuda.synchronize()
+    barrier(world)
+    if gdn.check_error(fws) != 0 or gdn.check_error(bws) != 0:
+        raise RuntimeError("device error word set in the trainer step")
+    fwd = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ms = max_over_ranks(fwd + bwd, world)
+    return {"workload": f"trainer: {T} tokens as {N} documents (lengths {b.lengths}), H={H}, "
+                        f"d_k=d_v={D}, C={C}, bf16 q/k/v/do, fp32 beta/g/state/gradients",
+            "steps": steps, "ms_per_step": round(ms, 5), "fwd_ms": round(fwd, 5),
+            "bwd_ms": round(bwd, 5), "tokens_per_s": round(world * T / (ms / 1e3), 1),
+            "gpu_launches_per_step": 4 + 6,
+            "l2": "flushed (256 MiB write) before every timed step",
+            "pages_h100_ms": PAGES_H100["trainer_fwd_bwd_ms"]}
+
+
 def cpu_baseline_sample(W, seconds=10.0):
     """The fp64 oracle as it stands, all host cores, on whole sequences of the
     prefill batch until about `seconds` of CPU work has been done."""
@@ -488,6 +536,9 @@ def run_ours(args):
     decode = None
     if args.only in ("all", "decode"):
         decode = run_decode_part(gdn, W, dev, rank, world, args, peaks)
+    train = None
+    if args.only in ("all", "train"):
+        train = run_train_part(gdn, W, dev, rank, world, args, flush)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -506,6 +557,7 @@ def run_ours(args):
         "hbm_roofline": hbm,
         "e2e": e2e,
         "decode": decode,
+        "train_step": train,
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
         "wall_s_timed_region": round(wall, 4),
@@ -573,7 +625,7 @@ def main():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--decode-steps", type=int, default=512)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+    p.add_argument("--only", choices=["all", "prefill", "decode", "train"], default="all",
                    help="profiling aid: run only part of the benchmark")
     p.add_argument("--decode-slots", type=int, default=256)
     args = p.parse_args()

@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define GDN_CPR_ABI_VERSION 4
+#define GDN_CPR_ABI_VERSION 5
 
 typedef enum {
   GDN_OK = 0,
@@ -261,6 +261,53 @@ int gdn_cpr_decode_step(const void* q, const void* k, const void* v, int in_dtyp
 int gdn_chunk_boundary(const float* s_start, const void* k, const void* v, int in_dtype,
                        const float* beta, const float* g, int B, int H, int dk, int dv, int C,
                        float* s_end, void* stream);
+
+/*
+ * Bytes of device workspace gdn_cpr_backward needs for this problem size.
+ * Returns 0 for arguments gdn_cpr_backward would reject.
+ */
+size_t gdn_cpr_backward_workspace_bytes(int n_seqs, int64_t total_tokens, int H, int dk, int dv,
+                                        int C, int in_dtype);
+
+/*
+ * gdn_cpr_backward -- reverse mode of gdn_cpr_forward: the gradients of a
+ * loss L(o, S_final) with respect to q, k, v, beta, g and h0, given dL/do and
+ * dL/dS_final.  S_final is the state after each sequence's last token.
+ *
+ * Defines: the trainer's forward plus backward of the section "Solving the
+ * linear-attention headache" (its timing table has a row for it); the pages
+ * give no formulas, so the gradients are those of the recurrence
+ * S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ * o_t = scale S_t q_t, alpha_t = exp(g_t).
+ * Schedule: the forward's first pass runs again (boundary states); an
+ * adjoint recurrence runs over each sequence, last token first (row-parallel,
+ * like the state); each chunk's states are recomputed from its boundary state
+ * with the forward's per-token step; each chunk's dq and dk come from
+ * products of C x C and C x d matrices.  Every reduction has a fixed order,
+ * so repeated calls return identical bits.
+ *
+ * Inputs:  q, k, v, beta, g, cu_seqlens, n_seqs, total_tokens, H, dk, dv, C,
+ *          scale, h0 exactly as for gdn_cpr_forward.
+ *   d_o       [total_tokens, H, dv] in_dtype: dL/do
+ *   ds_final  [n_seqs, H, dv, dk] fp32 dL/dS_final, or NULL for zeros
+ * Outputs (fp32, written for every token; caller-owned device memory):
+ *   d_q, d_k  [total_tokens, H, dk]
+ *   d_v       [total_tokens, H, dv]
+ *   d_beta, d_g [total_tokens, H]
+ *   d_h0      [n_seqs, H, dv, dk] dL/dh0 (whether or not h0 is NULL), or
+ *             NULL to skip it
+ * workspace: device scratch of at least gdn_cpr_backward_workspace_bytes
+ *   bytes, 16-byte aligned.  Its first 4 bytes are the device error word.
+ * Pointers to device arrays of 16-byte rows must be 16-byte aligned.
+ * Status: as gdn_cpr_forward; invalid cu_seqlens set GDN_DEVERR_CU_SEQLENS
+ * in the error word and leave the outputs unwritten.
+ */
+int gdn_cpr_backward(const void* q, const void* k, const void* v, int in_dtype,
+                     const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
+                     int64_t total_tokens, int H, int dk, int dv, int C, float scale,
+                     const float* h0, const void* d_o, const float* ds_final, float* d_q,
+                     float* d_k, float* d_v, float* d_beta, float* d_g, float* d_h0,
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * gdn_check_error -- synchronise `stream`, read the device error word at

@@ -73,6 +73,9 @@ def _load() -> ctypes.CDLL:
         "gdn_cpr_decode_step": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32,
                                       DecodeStateStruct, vp, i32, vp]),
         "gdn_chunk_boundary": (i32, [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
+        "gdn_cpr_backward_workspace_bytes": (sz, [i32, i64, i32, i32, i32, i32, i32]),
+        "gdn_cpr_backward": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                   f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gdn_check_error": (i32, [vp, vp, vp]),
         "gdn_cpr_contract_descriptor": (i32, [i32, i32, i32, i32, i32, i32, ctypes.c_char_p, sz,
                                               ctypes.POINTER(ctypes.c_size_t)]),
@@ -184,6 +187,44 @@ def forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=No
                                 _stream(stream))
     _check(st, "gdn_cpr_forward")
     return o, s_run_final, s_bnd_final, workspace
+
+
+def backward_workspace_bytes(n_seqs: int, total_tokens: int, H: int, dk: int, dv: int,
+                             C: int = CHUNK, dtype=torch.bfloat16) -> int:
+    code = _dtype_code(torch.empty(0, dtype=dtype))
+    return int(lib.gdn_cpr_backward_workspace_bytes(n_seqs, total_tokens, H, dk, dv, C, code))
+
+
+def backward(q, k, v, beta, g, cu_seqlens, d_o, *, n_seqs: Optional[int] = None, h0=None,
+             ds_final=None, C: int = CHUNK, scale: float = 1.0, want_dh0: bool = True,
+             grads=None, workspace=None, stream=None):
+    """gdn_cpr_backward.  Returns (grads, workspace); grads is a dict of fp32
+    tensors dq, dk, dv [T, H, d], dbeta, dg [T, H] and dh0 [N, H, dv, dk]
+    (None unless want_dh0).  Pass ``grads`` (the same dict) to reuse buffers."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = (cu_seqlens.numel() - 1) if n_seqs is None else int(n_seqs)
+    in_code = _dtype_code(q)
+    if d_o.dtype != q.dtype:
+        raise ValueError("gdn_cpr: d_o must have the dtype of q, k and v")
+    dev = q.device
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = {"dq": torch.empty((T, H, dk), **f32), "dk": torch.empty((T, H, dk), **f32),
+                 "dv": torch.empty((T, H, dv), **f32), "dbeta": torch.empty((T, H), **f32),
+                 "dg": torch.empty((T, H), **f32),
+                 "dh0": torch.empty((N, H, dv, dk), **f32) if want_dh0 else None}
+    need = backward_workspace_bytes(N, T, H, dk, dv, C, q.dtype)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    st = lib.gdn_cpr_backward(_ptr(q), _ptr(k), _ptr(v), in_code, _ptr(beta), _ptr(g),
+                              _ptr(cu_seqlens), N, T, H, dk, dv, C, float(scale), _ptr(h0),
+                              _ptr(d_o), _ptr(ds_final), _ptr(grads["dq"]), _ptr(grads["dk"]),
+                              _ptr(grads["dv"]), _ptr(grads["dbeta"]), _ptr(grads["dg"]),
+                              _ptr(grads.get("dh0")), _ptr(workspace), workspace.numel(),
+                              _stream(stream))
+    _check(st, "gdn_cpr_backward")
+    return grads, workspace
 
 
 def check_error(error_word: torch.Tensor, stream=None) -> int:

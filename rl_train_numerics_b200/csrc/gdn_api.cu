@@ -115,6 +115,68 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
   return from_cuda(gdn::launch_forward(a, static_cast<cudaStream_t>(stream)));
 }
 
+size_t gdn_cpr_backward_workspace_bytes(int n_seqs, int64_t total_tokens, int H, int dk, int dv,
+                                        int C, int in_dtype) {
+  if (n_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return 0;
+  if (check_shape(H, dk, dv, C, in_dtype) != GDN_OK) return 0;
+  return gdn::bwd_layout(n_seqs, total_tokens, H, dk, dv, C, in_dtype == GDN_BF16).total;
+}
+
+int gdn_cpr_backward(const void* q, const void* k, const void* v, int in_dtype,
+                     const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
+                     int64_t total_tokens, int H, int dk, int dv, int C, float scale,
+                     const float* h0, const void* d_o, const float* ds_final, float* d_q,
+                     float* d_k, float* d_v, float* d_beta, float* d_g, float* d_h0,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (n_seqs < 0 || total_tokens < 0 || !isfinite(scale)) return GDN_ERR_INVALID_ARG;
+  int rc = check_shape(H, dk, dv, C, in_dtype);
+  if (rc != GDN_OK) return rc;
+  if (total_tokens > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+  if (n_seqs == 0) return total_tokens == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+  if (!cu_seqlens || !aligned4(cu_seqlens)) return GDN_ERR_INVALID_ARG;
+  if (total_tokens > 0) {
+    if (!q || !k || !v || !beta || !g || !d_o || !d_q || !d_k || !d_v || !d_beta || !d_g)
+      return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_o) || !aligned16(d_q) ||
+        !aligned16(d_k) || !aligned16(d_v))
+      return GDN_ERR_INVALID_ARG;
+    if (!aligned4(beta) || !aligned4(g) || !aligned4(d_beta) || !aligned4(d_g))
+      return GDN_ERR_INVALID_ARG;
+  }
+  if ((h0 && !aligned16(h0)) || (ds_final && !aligned16(ds_final)) || (d_h0 && !aligned16(d_h0)))
+    return GDN_ERR_INVALID_ARG;
+  const gdn::BwdLayout lay =
+      gdn::bwd_layout(n_seqs, total_tokens, H, dk, dv, C, in_dtype == GDN_BF16);
+  if (!workspace || workspace_bytes < lay.total) return GDN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDN_ERR_INVALID_ARG;
+  gdn::BwdArgs a{};
+  a.fwd.q = q;
+  a.fwd.k = k;
+  a.fwd.v = v;
+  a.fwd.in_bf16 = in_dtype == GDN_BF16;
+  a.fwd.beta = beta;
+  a.fwd.g = g;
+  a.fwd.cu_seqlens = cu_seqlens;
+  a.fwd.n_seqs = n_seqs;
+  a.fwd.T = total_tokens;
+  a.fwd.H = H;
+  a.fwd.D = dk;
+  a.fwd.scale = scale;
+  a.fwd.h0 = h0;
+  a.fwd.ws = static_cast<char*>(workspace);
+  a.fwd.lay = lay.fwd;
+  a.d_o = d_o;
+  a.ds_final = ds_final;
+  a.d_q = d_q;
+  a.d_k = d_k;
+  a.d_v = d_v;
+  a.d_beta = d_beta;
+  a.d_g = d_g;
+  a.d_h0 = d_h0;
+  a.lay = lay;
+  return from_cuda(gdn::launch_backward(a, static_cast<cudaStream_t>(stream)));
+}
+
 static int check_state(const gdn_decode_state& st) {
   if (st.n_slots <= 0 || !st.s_run || !st.s_scale || !st.s_bnd || !st.buf_k || !st.buf_v ||
       !st.buf_beta || !st.buf_g || !st.pos || !st.error || !st.resync)

@@ -1,0 +1,658 @@
+// gdn_backward.cu -- reverse mode of the CPR Gated DeltaNet layer (sm_100a).
+//
+// Gradients of a loss L(o, S_final) with respect to q, k, v, beta, g and h0,
+// on the forward's chunk schedule.  "NovaSky's IsoExec Fixes the Hidden Math
+// Bug Corrupting AI Training Runs" times the trainer's forward plus backward
+// (section "Solving the linear-attention headache" and its timing table) but
+// does not spell the backward out; everything below is derived from the
+// recurrence itself.
+//
+// Per (sequence, head); the state S is d_v x d_k, one row per value channel.
+//   F_t = alpha_t (I - beta_t k_t k_t^T)            (symmetric)
+//   S_t = S_{t-1} F_t + beta_t v_t k_t^T = alpha_t S_{t-1} + u_t k_t^T
+//   p_t = S_{t-1} k_t,  u_t = beta_t (v_t - alpha_t p_t),  o_t = scale S_t q_t
+// Adjoints.  Lambda_t = dL/dS_t; mu_t is Lambda_t without the direct term of
+// o_t, i.e. the part that flows on through S_{t+1}:
+//   Lambda_t = mu_t + scale do_t q_t^T,   mu_T = dS_final,
+//   w_t = Lambda_t k_t,   mu_{t-1} = Lambda_t F_t = alpha_t (Lambda_t - beta_t w_t k_t^T),
+//   dh0 = mu_0.
+// Rows of mu evolve independently, like rows of S, and never need S: the
+// adjoint runs the same gated delta rule backwards in time with the input
+// scale do q^T.  Per token:
+//   dv_t    = beta_t w_t
+//   dbeta_t = w_t . (v_t - alpha_t p_t)
+//   dg_t    = <mu_{t-1}, S_{t-1}>_F  (dS_t / dg_t = S_{t-1} F_t), which
+//             telescopes: with Z_t = <mu_t, S_t>_F,
+//             Z_{t-1} = <Lambda_t, S_{t-1} F_t> = Z_t + do_t . o_t - beta_t v_t . w_t
+//   dq_t    = scale S_t^T do_t
+//   dk_t    = -alpha_t beta_t S_{t-1}^T w_t + Lambda_t^T u_t
+// Inside a chunk that starts from S_a (chunk-local t = 0 .. L-1 and
+// G_t = g_0 + ... + g_t), unrolling both recurrences gives
+//   S_t  = e^{G_t} S_a + sum_{s<=t} e^{G_t - G_s} u_s k_s^T
+//   mu_t = e^{G_{L-1} - G_t} mu_e + sum_{r>t} e^{G_r - G_t} (scale do_r q_r^T - beta_r w_r k_r^T)
+// (mu_e: the adjoint at the chunk's end), and substituted into dq and dk the
+// vector gradients of a chunk become products of C x C and C x d matrices:
+//   Y = DO U^T,  A_ts = [s <= t] e^{G_t - G_s} Y_ts
+//   X = W U^T,   B_ts = [s < t] beta_t e^{G_t - G_s} X_ts
+//   DQ = scale (diag(e^G) DO S_a + A K)
+//   DK = scale A^T Q - (B + B^T) K - diag(beta e^G) W S_a + diag(e^{G_{L-1} - G}) U mu_e
+// (the A^T Q term collects both scale q_t (do_t . u_t) and the do part of
+// mu_t^T u_t; B^T collects the w part of mu_t^T u_t).
+//
+// Kernels, in launch order:
+//   forward pass 1   chunk table and boundary states S_a, exactly as the
+//                    forward computes them
+//   k_bwd_scan       one block per (sequence, head, 32 rows): the adjoint
+//                    recurrence over the whole sequence, last token first;
+//                    writes w, dv, the adjoint at every chunk end and dh0
+//   k_bwd_rows       one block per (chunk, head): recomputes the chunk's
+//                    states from S_a with the forward fill's per-token step
+//                    (the states the outputs came from); writes u, dbeta, dg
+//   k_bwd_gemm       one block per (chunk, head): DQ and DK from the
+//                    products above, in fp32 fused multiply-adds
+// Every sum has a fixed order, so repeated runs give identical bits.
+#include "gdn_fill.cuh"
+#include "gdn_layout.h"
+
+namespace gdn {
+
+#define GDN_BWD_TRY(expr)             \
+  do {                                \
+    cudaError_t e_ = (expr);          \
+    if (e_ != cudaSuccess) return e_; \
+  } while (0)
+
+constexpr int kScanRows = 32;                    // state rows per k_bwd_scan block
+constexpr int kScanThreads = kScanRows * kQuad;  // one quad per row
+constexpr int kGemmThreads = 256;
+constexpr int kWarps = kFillThreads / 32;        // warps of a k_bwd_rows block
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) x = __fadd_rn(x, __shfl_xor_sync(kFull, x, off));
+  return x;
+}
+
+// ----------------------------------------------------------------------------
+// Adjoint scan: mu over the whole sequence, last token first
+// ----------------------------------------------------------------------------
+// Tokens arrive in tiles of 32 (two per chunk), double-buffered with cp.async
+// so that the next tile's keys, queries and do rows load while this tile's
+// tokens run.
+constexpr int kScanTile = 32;
+
+template <int D, class IN>
+struct ScanTile {
+  IN k[kScanTile][D];
+  IN q[kScanTile][D];
+  IN dor[kScanTile][kScanRows];  // do of the block's rows
+  float graw[kScanTile];         // g
+  float b[kScanTile];            // beta
+  float a[kScanTile];            // exp(g), by the tile's pre-pass
+  float qk[kScanTile];           // q . k, by the tile's pre-pass
+};
+
+template <int D, class IN>
+struct ScanSmem {
+  ScanTile<D, IN> buf[2];
+};
+
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(smem)), "l"(gmem));
+}
+
+template <int D, class IN>
+__device__ __forceinline__ void scan_issue(ScanTile<D, IN>& tl, const IN* q, const IN* k,
+                                           const IN* d_o, const float* beta, const float* g,
+                                           size_t tb, int H, int rb, int len) {
+  constexpr int P = (int)(D * sizeof(IN) / 16), E = (int)(16 / sizeof(IN));
+  constexpr int PD = (int)(kScanRows * sizeof(IN) / 16);
+  for (int e = threadIdx.x; e < 2 * len * P; e += kScanThreads) {
+    const int row = e / P, pc = (e % P) * E;
+    const bool isk = row < len;
+    const int t = isk ? row : row - len;
+    cp_async16(isk ? &tl.k[t][pc] : &tl.q[t][pc], (isk ? k : q) + (tb + (size_t)t * H) * D + pc);
+  }
+  for (int e = threadIdx.x; e < len * PD; e += kScanThreads) {
+    const int t = e / PD, pc = (e % PD) * E;
+    cp_async16(&tl.dor[t][pc], d_o + (tb + (size_t)t * H) * D + rb + pc);
+  }
+  for (int t = threadIdx.x; t < len; t += kScanThreads) {
+    cp_async4(&tl.graw[t], g + tb + (size_t)t * H);
+    cp_async4(&tl.b[t], beta + tb + (size_t)t * H);
+  }
+  cp_async_commit();
+}
+
+// Lane-partial dot of a state row with a key row: four independent
+// accumulators (groups m = 0, 4, ... into the first, 1, 5, ... into the
+// second, ...), combined pairwise.
+template <int M4, class IN>
+__device__ __forceinline__ float row_dot4(const Slice<1, M4>& x, const IN* krow, int l) {
+  float2 acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+  for (int m = 0; m < M4; m++) {
+    const float4 k4 = sld4(krow + group_col(l, m));
+    acc[m & 3] = __ffma2_rn(x.s[0][m][0], f2(k4.x, k4.y), acc[m & 3]);
+    acc[m & 3] = __ffma2_rn(x.s[0][m][1], f2(k4.z, k4.w), acc[m & 3]);
+  }
+  const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+  const float2 s = __fadd2_rn(s01, s23);
+  return __fadd_rn(s.x, s.y);
+}
+
+template <int D, class IN>
+__global__ void __launch_bounds__(kScanThreads)
+    k_bwd_scan(const IN* __restrict__ q, const IN* __restrict__ k, const float* __restrict__ beta,
+               const float* __restrict__ g, const IN* __restrict__ d_o,
+               const float* __restrict__ ds_final, const int32_t* __restrict__ cu, int H,
+               float scale, const int32_t* __restrict__ hdr,
+               const int32_t* __restrict__ chunk_off, float* __restrict__ mu_end,
+               float* __restrict__ wbuf, float* __restrict__ d_v, float* __restrict__ d_h0) {
+  constexpr int M4 = D / 16;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  ScanSmem<D, IN>& sm = *reinterpret_cast<ScanSmem<D, IN>*>(smem_raw);
+  if (hdr[kHdrValid] != 1) return;
+  const int n = blockIdx.x, h = blockIdx.y, rb = blockIdx.z * kScanRows;
+  const int tid = threadIdx.x, l = tid & 3, rr = tid >> 2, r = rb + rr;
+  const int lane = tid & 31, warp = tid >> 5;
+  const size_t DD = (size_t)D * D;
+  const int64_t L = (int64_t)cu[n + 1] - cu[n];
+  const int nc = (int)((L + kChunk - 1) / kChunk);
+  const int nt = (int)((L + kScanTile - 1) / kScanTile);
+  const int c0 = chunk_off[n];
+  const size_t tseq = (size_t)cu[n] * H + h;
+
+  Slice<1, M4> mu;
+  if (ds_final) {
+    slice_load<1, M4>(mu, ds_final + ((size_t)n * H + h) * DD, D, r, l);
+  } else {
+#pragma unroll
+    for (int m = 0; m < M4; m++) mu.s[0][m][0] = mu.s[0][m][1] = f2(0.f, 0.f);
+  }
+  if (nc > 0) slice_store<1, M4>(mu, mu_end + ((size_t)(c0 + nc - 1) * H + h) * DD, D, r, l);
+
+  auto tile_len = [&](int ti) {
+    return (int)min((int64_t)kScanTile, L - (int64_t)ti * kScanTile);
+  };
+  if (nt > 0)
+    scan_issue<D, IN>(sm.buf[(nt - 1) & 1], q, k, d_o, beta, g,
+                      tseq + (size_t)(nt - 1) * kScanTile * H, H, rb, tile_len(nt - 1));
+  for (int ti = nt - 1; ti >= 0; ti--) {
+    ScanTile<D, IN>& tl = sm.buf[ti & 1];
+    const int len = tile_len(ti);
+    const size_t tb = tseq + (size_t)ti * kScanTile * H;
+    cp_async_wait<0>();
+    __syncthreads();  // the tile is in; the other buffer's tokens are done
+    if (ti > 0)
+      scan_issue<D, IN>(sm.buf[(ti - 1) & 1], q, k, d_o, beta, g,
+                        tseq + (size_t)(ti - 1) * kScanTile * H, H, rb, tile_len(ti - 1));
+    // Pre-pass: exp(g) and q . k (one warp per token, columns over the lanes).
+    if (tid < len) tl.a[tid] = step_decay(tl.graw[tid]);
+    for (int t = warp; t < len; t += kScanThreads / 32) {
+      float x = 0.f;
+#pragma unroll
+      for (int j = 0; j < D / 32; j++) {
+        const int col = lane + 32 * j;
+        x = __fmaf_rn(to_f(tl.q[t][col]), to_f(tl.k[t][col]), x);
+      }
+      x = warp_sum(x);
+      if (lane == 0) tl.qk[t] = x;
+    }
+    __syncthreads();
+    for (int t = len - 1; t >= 0; t--) {
+      const float sdo = __fmul_rn(scale, to_f(tl.dor[t][rr]));
+      const float w = __fmaf_rn(sdo, tl.qk[t], quad_sum(row_dot4<M4>(mu, &tl.k[t][0], l)));
+      const float a = tl.a[t], bw = __fmul_rn(tl.b[t], w);
+      if (l == 0) {
+        const size_t idx = (tb + (size_t)t * H) * D + r;
+        wbuf[idx] = w;
+        d_v[idx] = bw;
+      }
+      const float2 s2 = f2(sdo, sdo), nb = f2(-bw, -bw), aa = f2(a, a);
+#pragma unroll
+      for (int m = 0; m < M4; m++) {
+        const float4 k4 = sld4(&tl.k[t][group_col(l, m)]);
+        const float4 q4 = sld4(&tl.q[t][group_col(l, m)]);
+        float2 x01 = __ffma2_rn(s2, f2(q4.x, q4.y), mu.s[0][m][0]);
+        float2 x23 = __ffma2_rn(s2, f2(q4.z, q4.w), mu.s[0][m][1]);
+        x01 = __ffma2_rn(nb, f2(k4.x, k4.y), x01);
+        x23 = __ffma2_rn(nb, f2(k4.z, k4.w), x23);
+        mu.s[0][m][0] = __fmul2_rn(aa, x01);
+        mu.s[0][m][1] = __fmul2_rn(aa, x23);
+      }
+    }
+    // The tile that starts a chunk (even ti) leaves mu at that chunk's start,
+    // which is the end of the chunk before it.
+    const int ci = ti / 2;
+    if ((ti & 1) == 0 && ci > 0)
+      slice_store<1, M4>(mu, mu_end + ((size_t)(c0 + ci - 1) * H + h) * DD, D, r, l);
+  }
+  if (d_h0) slice_store<1, M4>(mu, d_h0 + ((size_t)n * H + h) * DD, D, r, l);
+}
+
+// ----------------------------------------------------------------------------
+// Per-row recomputation of a chunk: u, dbeta, dg
+// ----------------------------------------------------------------------------
+template <int D, class IN>
+struct RowsSmem {
+  FillSmem<D, IN> f;
+  float part[kWarps][kChunk][2];  // per-warp sums of the dbeta and dg terms
+  float zpart[kWarps];
+};
+
+template <int D, class IN>
+__global__ void __launch_bounds__(kFillThreads, 3)
+    k_bwd_rows(const IN* __restrict__ q, const IN* __restrict__ k, const IN* __restrict__ v,
+               const float* __restrict__ beta, const float* __restrict__ g,
+               const IN* __restrict__ d_o, const int32_t* __restrict__ cu, int H, float scale,
+               const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+               const int32_t* __restrict__ chunk_seq, const float* __restrict__ bstate,
+               const float* __restrict__ mu_end, const float* __restrict__ wbuf,
+               float* __restrict__ ubuf, float* __restrict__ d_beta, float* __restrict__ d_g) {
+  constexpr int RT = D / 32, M4 = D / 16;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  RowsSmem<D, IN>& sm = *reinterpret_cast<RowsSmem<D, IN>*>(smem_raw);
+  if (hdr[kHdrValid] != 1) return;
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (c >= hdr[kHdrChunks]) return;
+  const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * RT;
+  const int lane = tid & 31, warp = tid >> 5;
+  const size_t DD = (size_t)D * D;
+  const FillItem it = fill_item(c * H + h, H, cu, chunk_off, chunk_seq);
+  fill_load<D, IN>(sm.f, it, q, k, v, beta, g, H);
+  Slice<RT, M4> S;
+  slice_load_bst<RT, M4>(S, bstate + ((size_t)c * H + h) * DD, D, r0, l);
+  __syncthreads();
+
+  float p[RT];
+  slice_dot<RT, M4>(S, [&](int m) { return sld4(&sm.f.k[0][group_col(l, m)]); }, p);
+#pragma unroll
+  for (int i = 0; i < RT; i++) p[i] = quad_sum(p[i]);
+  float cs = 1.f;  // scale of the running state (the forward fill's form)
+  const bool mine = l < RT;  // lane l accounts for row r0 + l
+  const int rl = mine ? l : 0;
+  const size_t tb = (size_t)it.t0 * H + h;
+  for (int t = 0; t < it.len; t++) {
+    const float a = sm.f.a[t], b = sm.f.b[t];
+    const float pr = __fmul_rn(cs, pick<RT>(p, rl));  // p_t of row r0 + rl
+    const float vr = to_f(sm.f.v[t][r0 + rl]);
+    const size_t idx = (tb + (size_t)t * H) * D + r0 + rl;
+    const float wr = mine ? wbuf[idx] : 0.f;
+    const float dor = mine ? ld1(d_o + idx) : 0.f;
+    float ov[RT];
+    slice_token<true, RT, M4>(
+        S, cs, a, b, [&](int i) { return to_f(sm.f.v[t][r0 + i]); },
+        [&](int m) { return sld4(&sm.f.k[t][group_col(l, m)]); },
+        [&](int m) { return sld4(&sm.f.q[t][group_col(l, m)]); },
+        [&](int m) { return sld4(&sm.f.k[t + 1][group_col(l, m)]); }, p, ov);
+    float db = 0.f, dgt = 0.f;
+    if (mine) {
+      const float orr = __fmul_rn(scale, pick<RT>(ov, rl));
+      ubuf[idx] = step_u(a, b, pr, vr);
+      db = __fmul_rn(wr, __fmaf_rn(-a, pr, vr));
+      dgt = __fmaf_rn(dor, orr, -__fmul_rn(__fmul_rn(b, vr), wr));
+    }
+    db = warp_sum(db);
+    dgt = warp_sum(dgt);
+    if (lane == 0) {
+      sm.part[warp][t][0] = db;
+      sm.part[warp][t][1] = dgt;
+    }
+  }
+  // Z at the chunk's end: <mu_e, S_e> with S_e = cs * M.
+  const float* me = mu_end + ((size_t)c * H + h) * DD;
+  float z = 0.f;
+#pragma unroll
+  for (int i = 0; i < RT; i++)
+#pragma unroll
+    for (int m = 0; m < M4; m++) {
+      const float4 x = ld4(me + (size_t)(r0 + i) * D + group_col(l, m));
+      z = __fmaf_rn(x.x, S.s[i][m][0].x, z);
+      z = __fmaf_rn(x.y, S.s[i][m][0].y, z);
+      z = __fmaf_rn(x.z, S.s[i][m][1].x, z);
+      z = __fmaf_rn(x.w, S.s[i][m][1].y, z);
+    }
+  z = warp_sum(z);
+  if (lane == 0) sm.zpart[warp] = z;
+  __syncthreads();
+  if (tid == 0) {
+    float zs = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) zs = __fadd_rn(zs, sm.zpart[w]);
+    float Z = __fmul_rn(cs, zs);
+    for (int t = it.len - 1; t >= 0; t--) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; w++) s = __fadd_rn(s, sm.part[w][t][1]);
+      Z = __fadd_rn(Z, s);
+      d_g[tb + (size_t)t * H] = Z;
+    }
+  }
+  for (int t = tid; t < it.len; t += kFillThreads) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) s = __fadd_rn(s, sm.part[w][t][0]);
+    d_beta[tb + (size_t)t * H] = s;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Chunk products: DQ and DK
+// ----------------------------------------------------------------------------
+// One block of 256 threads per (chunk, head).  DO, W and U sit transposed in
+// shared memory ([row i][token t]); A and B + B^T are each kept as one
+// symmetric C x C array (A's lower triangle mirrored into the upper one: the
+// entry at [s][t] is A_ts for s <= t and A_st for s >= t).  S_a and mu_e
+// stream through shared memory in slabs of 16 rows, double-buffered with
+// cp.async.  Each thread owns 4 tokens x D/16 columns of DQ and of DK.
+constexpr int kSlab = 16;
+
+template <int D, class IN>
+struct GemmSmem {
+  float DOt[D][kChunk];
+  float Wt[D][kChunk];
+  float Ut[D][kChunk];
+  IN Q[kChunk][D];
+  IN K[kChunk][D];
+  float As[kChunk][kChunk];
+  float Bs[kChunk][kChunk];
+  float Sa[2][kSlab][D];  // boundary-state rows (unpermuted)
+  float Me[2][kSlab][D];  // adjoint rows at the chunk's end
+  double G[kChunk];       // chunk-local cumulative log decay
+  float bet[kChunk];
+};
+
+// Transpose C x D rows (token-major in HBM, [t][h][i]) into [i][t] fp32.
+template <int D, class T>
+__device__ __forceinline__ void load_transposed(float (*dst)[kChunk], const T* src, size_t tb,
+                                                int H, int len) {
+  for (int e = threadIdx.x; e < kChunk * (D / 4); e += kGemmThreads) {
+    const int t = e % kChunk, i = (e / kChunk) * 4;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < len) x = ld4(src + (tb + (size_t)t * H) * D + i);
+    dst[i][t] = x.x;
+    dst[i + 1][t] = x.y;
+    dst[i + 2][t] = x.z;
+    dst[i + 3][t] = x.w;
+  }
+}
+
+// Slab j (rows 16j .. 16j+15) of S_a (permuted boundary layout) and mu_e.
+template <int D, class IN>
+__device__ __forceinline__ void slab_issue(GemmSmem<D, IN>& sm, int buf, int j, const float* Sa,
+                                           const float* Me) {
+  constexpr int PR = D / 4;  // 16-byte pieces per row
+  for (int e = threadIdx.x; e < 2 * kSlab * PR; e += kGemmThreads) {
+    const int which = e / (kSlab * PR), rem = e % (kSlab * PR);
+    const int rr = rem / PR, c = (rem % PR) * 4, i = j * kSlab + rr;
+    if (which == 0)
+      cp_async16(&sm.Sa[buf][rr][c], Sa + (size_t)i * D + bst_col(i, c));
+    else
+      cp_async16(&sm.Me[buf][rr][c], Me + (size_t)i * D + c);
+  }
+  cp_async_commit();
+}
+
+template <int NC>
+__device__ __forceinline__ void row_ld(const float* p, float (&x)[NC]) {
+#pragma unroll
+  for (int j = 0; j < NC; j += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(p + j);
+    x[j] = v.x;
+    x[j + 1] = v.y;
+    x[j + 2] = v.z;
+    x[j + 3] = v.w;
+  }
+}
+template <int NC>
+__device__ __forceinline__ void row_ld(const __nv_bfloat16* p, float (&x)[NC]) {
+#pragma unroll
+  for (int j = 0; j < NC; j += 4) {
+    const float4 v = sld4(p + j);
+    x[j] = v.x;
+    x[j + 1] = v.y;
+    x[j + 2] = v.z;
+    x[j + 3] = v.w;
+  }
+}
+
+__device__ __forceinline__ void f4a(const float4 v, float (&x)[4]) {
+  x[0] = v.x;
+  x[1] = v.y;
+  x[2] = v.z;
+  x[3] = v.w;
+}
+
+template <int D, class IN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_bwd_gemm(const IN* __restrict__ q, const IN* __restrict__ k,
+               const float* __restrict__ beta, const float* __restrict__ g,
+               const IN* __restrict__ d_o, const int32_t* __restrict__ cu, int H, float scale,
+               const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+               const int32_t* __restrict__ chunk_seq, const float* __restrict__ bstate,
+               const float* __restrict__ mu_end, const float* __restrict__ wbuf,
+               const float* __restrict__ ubuf, float* __restrict__ d_q, float* __restrict__ d_k) {
+  constexpr int NC = D / 16;  // output columns per thread
+  constexpr int P = (int)(D * sizeof(IN) / 16);
+  constexpr int E = (int)(16 / sizeof(IN));
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  GemmSmem<D, IN>& sm = *reinterpret_cast<GemmSmem<D, IN>*>(smem_raw);
+  if (hdr[kHdrValid] != 1) return;
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (c >= hdr[kHdrChunks]) return;
+  const int tid = threadIdx.x;
+  const size_t DD = (size_t)D * D;
+  const FillItem it = fill_item(c * H + h, H, cu, chunk_off, chunk_seq);
+  const int len = it.len;
+  const size_t tb = (size_t)it.t0 * H + h;
+  const float* Sa = bstate + ((size_t)c * H + h) * DD;
+  const float* Me = mu_end + ((size_t)c * H + h) * DD;
+
+  slab_issue<D, IN>(sm, 0, 0, Sa, Me);  // lands while the chunk's rows load
+  load_transposed<D>(sm.DOt, d_o, tb, H, len);
+  load_transposed<D>(sm.Wt, wbuf, tb, H, len);
+  load_transposed<D>(sm.Ut, ubuf, tb, H, len);
+  for (int e = tid; e < 2 * kChunk * P; e += kGemmThreads) {
+    const int row = e / P, pc = (e % P) * E, t = row % kChunk;
+    IN* dst = row < kChunk ? &sm.Q[t][pc] : &sm.K[t][pc];
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (t < len) x = *reinterpret_cast<const uint4*>((row < kChunk ? q : k) +
+                                                      (tb + (size_t)t * H) * D + pc);
+    *reinterpret_cast<uint4*>(dst) = x;
+  }
+  if (tid < kChunk) sm.bet[tid] = tid < len ? beta[tb + (size_t)tid * H] : 0.f;
+  if (tid == 0) {
+    double G = 0.0;
+    for (int t = 0; t < kChunk; t++) {
+      if (t < len) G += (double)g[tb + (size_t)t * H];
+      sm.G[t] = G;
+    }
+  }
+  __syncthreads();
+
+  const int ty = tid >> 4, tx = tid & 15;
+  const int t4 = 4 * ty;
+  // Y = DO U^T and X = W U^T on a 4 x 4 tile, then the masked, decayed A and
+  // B written with their mirror images.
+  {
+    float y[4][4] = {}, x[4][4] = {};
+    const int s4 = 4 * tx;
+#pragma unroll 4
+    for (int i = 0; i < D; i++) {
+      float dv[4], wv[4], uv[4];
+      f4a(*reinterpret_cast<const float4*>(&sm.DOt[i][t4]), dv);
+      f4a(*reinterpret_cast<const float4*>(&sm.Wt[i][t4]), wv);
+      f4a(*reinterpret_cast<const float4*>(&sm.Ut[i][s4]), uv);
+#pragma unroll
+      for (int a = 0; a < 4; a++)
+#pragma unroll
+        for (int b = 0; b < 4; b++) {
+          y[a][b] = __fmaf_rn(dv[a], uv[b], y[a][b]);
+          x[a][b] = __fmaf_rn(wv[a], uv[b], x[a][b]);
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; a++)
+#pragma unroll
+      for (int b = 0; b < 4; b++) {
+        const int t = t4 + a, s = s4 + b;
+        if (s > t) continue;  // written by the owner of (s, t)
+        const float e = expf((float)(sm.G[t] - sm.G[s]));
+        const float av = __fmul_rn(e, y[a][b]);
+        const float bv = s < t ? __fmul_rn(__fmul_rn(sm.bet[t], e), x[a][b]) : 0.f;
+        sm.As[t][s] = av;
+        sm.As[s][t] = av;
+        sm.Bs[t][s] = bv;
+        sm.Bs[s][t] = bv;
+      }
+  }
+
+  // Per-token factors of this thread's four rows.
+  float fq[4], fw[4], fu[4];
+  const double GL = sm.G[len > 0 ? len - 1 : 0];
+#pragma unroll
+  for (int a = 0; a < 4; a++) {
+    const int t = t4 + a;
+    const float eg = expf((float)sm.G[t]);
+    fq[a] = eg;                              // e^{G_t}          (DO S_a)
+    fw[a] = -__fmul_rn(sm.bet[t], eg);       // -beta_t e^{G_t}  (W S_a)
+    fu[a] = expf((float)(GL - sm.G[t]));     // e^{G_{L-1}-G_t}  (U mu_e)
+  }
+  const int c0 = tx * NC;
+  float aq[4][NC] = {}, ak[4][NC] = {};
+  constexpr int NS = D / kSlab;
+  for (int j = 0; j < NS; j++) {
+    cp_async_wait<0>();
+    __syncthreads();  // slab j is in; slab j-1's buffer is free (and, at j = 0, A and B are)
+    if (j + 1 < NS) slab_issue<D, IN>(sm, (j + 1) & 1, j + 1, Sa, Me);
+    const int bi = j & 1;
+#pragma unroll 4
+    for (int rr = 0; rr < kSlab; rr++) {
+      const int i = j * kSlab + rr;
+      float sv[NC], mv[NC], dv[4], wv[4], uv[4];
+      row_ld<NC>(&sm.Sa[bi][rr][c0], sv);
+      row_ld<NC>(&sm.Me[bi][rr][c0], mv);
+      f4a(*reinterpret_cast<const float4*>(&sm.DOt[i][t4]), dv);
+      f4a(*reinterpret_cast<const float4*>(&sm.Wt[i][t4]), wv);
+      f4a(*reinterpret_cast<const float4*>(&sm.Ut[i][t4]), uv);
+#pragma unroll
+      for (int a = 0; a < 4; a++) {
+        const float d1 = __fmul_rn(fq[a], dv[a]), w1 = __fmul_rn(fw[a], wv[a]);
+        const float u1 = __fmul_rn(fu[a], uv[a]);
+#pragma unroll
+        for (int jj = 0; jj < NC; jj++) {
+          aq[a][jj] = __fmaf_rn(d1, sv[jj], aq[a][jj]);
+          ak[a][jj] = __fmaf_rn(w1, sv[jj], ak[a][jj]);
+          ak[a][jj] = __fmaf_rn(u1, mv[jj], ak[a][jj]);
+        }
+      }
+    }
+  }
+  for (int s = 0; s < len; s++) {
+    float kr[NC], qr[NC], av[4], bv[4];
+    row_ld<NC>(&sm.K[s][c0], kr);
+    row_ld<NC>(&sm.Q[s][c0], qr);
+    f4a(*reinterpret_cast<const float4*>(&sm.As[s][t4]), av);
+    f4a(*reinterpret_cast<const float4*>(&sm.Bs[s][t4]), bv);
+#pragma unroll
+    for (int a = 0; a < 4; a++) {
+      const int t = t4 + a;
+      const float ck = s <= t ? av[a] : 0.f;                  // A_ts
+      const float cq = s >= t ? __fmul_rn(scale, av[a]) : 0.f;  // scale A_st
+      const float cb = -bv[a];                                 // -(B + B^T)_ts
+#pragma unroll
+      for (int jj = 0; jj < NC; jj++) {
+        aq[a][jj] = __fmaf_rn(ck, kr[jj], aq[a][jj]);
+        ak[a][jj] = __fmaf_rn(cq, qr[jj], ak[a][jj]);
+        ak[a][jj] = __fmaf_rn(cb, kr[jj], ak[a][jj]);
+      }
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 4; a++) {
+    const int t = t4 + a;
+    if (t >= len) continue;
+    float* oq = d_q + (tb + (size_t)t * H) * D + c0;
+    float* ok = d_k + (tb + (size_t)t * H) * D + c0;
+#pragma unroll
+    for (int jj = 0; jj < NC; jj += 4) {
+      *reinterpret_cast<float4*>(oq + jj) =
+          make_float4(__fmul_rn(scale, aq[a][jj]), __fmul_rn(scale, aq[a][jj + 1]),
+                      __fmul_rn(scale, aq[a][jj + 2]), __fmul_rn(scale, aq[a][jj + 3]));
+      *reinterpret_cast<float4*>(ok + jj) =
+          make_float4(ak[a][jj], ak[a][jj + 1], ak[a][jj + 2], ak[a][jj + 3]);
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Launcher
+// ----------------------------------------------------------------------------
+template <class KernelT>
+static cudaError_t bwd_set_smem(KernelT kern, size_t bytes) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int D, class IN>
+static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
+  FwdArgs f = a.fwd;
+  f.pass1_only = 1;
+  f.o = nullptr;
+  f.s_run_final = f.s_run_scale = f.s_bnd_final = nullptr;
+  f.events = nullptr;
+  f.lay = a.lay.fwd;
+  GDN_BWD_TRY(launch_forward(f, st));
+  const BwdLayout& L = a.lay;
+  char* ws = f.ws;
+  const int32_t* hdr = reinterpret_cast<const int32_t*>(ws + L.fwd.hdr);
+  const int32_t* chunk_off = reinterpret_cast<const int32_t*>(ws + L.fwd.chunk_off);
+  const int32_t* chunk_seq = reinterpret_cast<const int32_t*>(ws + L.fwd.chunk_seq);
+  const float* bstate = reinterpret_cast<const float*>(ws + L.fwd.bstate);
+  float* mu_end = reinterpret_cast<float*>(ws + L.mu_end);
+  float* wbuf = reinterpret_cast<float*>(ws + L.wbuf);
+  float* ubuf = reinterpret_cast<float*>(ws + L.ubuf);
+  const IN* q = static_cast<const IN*>(f.q);
+  const IN* k = static_cast<const IN*>(f.k);
+  const IN* v = static_cast<const IN*>(f.v);
+  const IN* d_o = static_cast<const IN*>(a.d_o);
+  {
+    auto kern = k_bwd_scan<D, IN>;
+    const size_t sm = sizeof(ScanSmem<D, IN>);
+    GDN_BWD_TRY(bwd_set_smem(kern, sm));
+    kern<<<dim3((unsigned)f.n_seqs, (unsigned)f.H, D / kScanRows), kScanThreads, sm, st>>>(
+        q, k, f.beta, f.g, d_o, a.ds_final, f.cu_seqlens, f.H, f.scale, hdr, chunk_off, mu_end,
+        wbuf, a.d_v, a.d_h0);
+    GDN_BWD_TRY(cudaGetLastError());
+  }
+  const dim3 gchunks((unsigned)L.fwd.max_chunks, (unsigned)f.H);
+  {
+    auto kern = k_bwd_rows<D, IN>;
+    const size_t sm = sizeof(RowsSmem<D, IN>);
+    GDN_BWD_TRY(bwd_set_smem(kern, sm));
+    kern<<<gchunks, kFillThreads, sm, st>>>(q, k, v, f.beta, f.g, d_o, f.cu_seqlens, f.H, f.scale,
+                                            hdr, chunk_off, chunk_seq, bstate, mu_end, wbuf, ubuf,
+                                            a.d_beta, a.d_g);
+    GDN_BWD_TRY(cudaGetLastError());
+  }
+  {
+    auto kern = k_bwd_gemm<D, IN>;
+    const size_t sm = sizeof(GemmSmem<D, IN>);
+    GDN_BWD_TRY(bwd_set_smem(kern, sm));
+    kern<<<gchunks, kGemmThreads, sm, st>>>(q, k, f.beta, f.g, d_o, f.cu_seqlens, f.H, f.scale,
+                                            hdr, chunk_off, chunk_seq, bstate, mu_end, wbuf, ubuf,
+                                            a.d_q, a.d_k);
+    GDN_BWD_TRY(cudaGetLastError());
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_backward(const BwdArgs& a, cudaStream_t st) {
+  using bf16 = __nv_bfloat16;
+  if (a.fwd.D == 64) return a.fwd.in_bf16 ? backward_impl<64, bf16>(a, st)
+                                          : backward_impl<64, float>(a, st);
+  if (!a.fwd.in_bf16) return cudaErrorNotSupported;  // fp32 inputs: d = 64 only
+  return backward_impl<128, bf16>(a, st);
+}
+
+}  // namespace gdn

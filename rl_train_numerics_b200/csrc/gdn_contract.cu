@@ -121,6 +121,7 @@ std::string descriptor(int kind, int in_dtype, int out_dtype, int dk, int dv, in
     s += line("output", "o_t=scale*S_t*q_t");
     s += line("state", "fp32[d_v][d_k], row=value channel");
     s += line("chunks", "C tokens from each sequence's token 0; boundary state every C tokens");
+    s += line("gradients", "dL/d(q,k,v,beta,g,h0) of the recurrence given dL/do, dL/dS_final");
     s += line("d_k", num(dk));
     s += line("d_v", num(dv));
     s += line("C", num(C));
@@ -147,6 +148,10 @@ std::string descriptor(int kind, int in_dtype, int out_dtype, int dk, int dv, in
                          : "mma.sync m16n8k16 bf16, state in accumulator registers");
     s += line("splits", in_dtype == GDN_BF16 ? "state/Y/U 2 bf16 terms, Tb/Tv 2, K/V 1"
                                              : "state/Y/U 3 bf16 terms, Tb/Tv 3, K/V 3");
+    s += line("backward",
+              "boundary states by the forward's first pass; adjoint scan per row (4 packed "
+              "accumulators per lane, xor butterfly 1,2); chunk states by the step schedule; "
+              "chunk products Y,X,A,B,DQ,DK in f32 fma, fixed order; dg by a telescoped sum");
     s += line("rounding", "round to nearest even, IEEE denormals, no contraction");
     s += line("compile", "sm_100a -O3 --fmad=false -ftz=false -prec-div=true -prec-sqrt=true");
   } else {

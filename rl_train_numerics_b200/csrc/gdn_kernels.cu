@@ -18,15 +18,10 @@
 //   k_bnd           one block per (row, head): gdn_chunk_boundary
 //   k_handoff       prefill -> decode state
 #include "gdn_boundary.cuh"
+#include "gdn_fill.cuh"
 #include "gdn_layout.h"
 
 namespace gdn {
-
-// Workspace header words (int32).
-constexpr int kHdrError = 0;     // device error word (GDN_DEVERR_* bits)
-constexpr int kHdrChunks = 1;    // number of chunks of this call
-constexpr int kHdrValid = 2;     // 1 when this call's chunk table is valid
-constexpr int kHdrFillNext = 3;  // work counter of k_fill
 
 // ----------------------------------------------------------------------------
 // Chunk table
@@ -432,97 +427,6 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
 // an item runs, the next item's state and inputs are prefetched into L2.
 // Which block runs an item does not change the item's bits.
 // ----------------------------------------------------------------------------
-constexpr int kFillThreads = 128;
-
-template <int D, class IN>
-struct FillSmem {
-  float k[kChunk + 1][D];  // row kChunk stays zero: the "next key" of the last token
-  IN q[kChunk][D];
-  IN v[kChunk][D];
-  float a[kChunk];  // exp(g)
-  float b[kChunk];  // beta
-};
-
-template <int RT>
-__device__ __forceinline__ float pick(const float (&x)[RT], int l) {
-  float val = x[0];
-#pragma unroll
-  for (int i = 1; i < RT; i++)
-    if (l == i) val = x[i];
-  return val;
-}
-
-struct FillItem {
-  int c, h, n, ci, len;
-  int64_t t0, L;
-};
-
-__device__ __forceinline__ FillItem fill_item(int item, int H, const int32_t* cu,
-                                              const int32_t* chunk_off,
-                                              const int32_t* chunk_seq) {
-  FillItem it;
-  it.c = item / H;
-  it.h = item - it.c * H;
-  it.n = chunk_seq[it.c];
-  it.ci = it.c - chunk_off[it.n];
-  it.L = (int64_t)cu[it.n + 1] - cu[it.n];
-  it.t0 = (int64_t)cu[it.n] + (int64_t)it.ci * kChunk;
-  it.len = (int)min((int64_t)kChunk, it.L - (int64_t)it.ci * kChunk);
-  return it;
-}
-
-__device__ __forceinline__ float to_f(float x) { return x; }
-__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
-
-// Load one item's inputs into shared memory (rows past its length are zero).
-template <int D, class IN>
-__device__ __forceinline__ void fill_load(FillSmem<D, IN>& sm, const FillItem& it, const IN* q,
-                                          const IN* k, const IN* v, const float* beta,
-                                          const float* g, int H) {
-  constexpr int G4 = D / 4;                        // float4 groups of a key row
-  constexpr int P = (int)(D * sizeof(IN) / 16);    // 16-byte pieces of a q/v row
-  constexpr int E = (int)(16 / sizeof(IN));
-  const size_t tb = (size_t)it.t0 * H + it.h;
-  for (int e = threadIdx.x; e < (kChunk + 1) * G4; e += kFillThreads) {
-    const int r = e / G4, c = (e % G4) * 4;
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < it.len) x = ld4(k + (tb + (size_t)r * H) * D + c);
-    *reinterpret_cast<float4*>(&sm.k[r][c]) = x;
-  }
-  for (int e = threadIdx.x; e < 2 * kChunk * P; e += kFillThreads) {
-    const int rr = e / P, pc = (e % P) * E, r = rr % kChunk;
-    IN* dst = rr < kChunk ? &sm.q[r][pc] : &sm.v[r][pc];
-    const IN* src = (rr < kChunk ? q : v) + (tb + (size_t)r * H) * D + pc;
-    uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (r < it.len) x = *reinterpret_cast<const uint4*>(src);
-    *reinterpret_cast<uint4*>(dst) = x;
-  }
-  for (int i = threadIdx.x; i < kChunk; i += kFillThreads) {
-    float a = 0.f, b = 0.f;
-    if (i < it.len) {
-      a = step_decay(g[tb + (size_t)i * H]);
-      b = beta[tb + (size_t)i * H];
-    }
-    sm.a[i] = a;
-    sm.b[i] = b;
-  }
-}
-
-// Ask L2 for an item's boundary state and input rows.
-template <int D, class IN>
-__device__ __forceinline__ void fill_prefetch(const FillItem& it, const float* bstate,
-                                              const IN* q, const IN* k, const IN* v, int H) {
-  const int tid = threadIdx.x;
-  const size_t tb = (size_t)it.t0 * H + it.h;
-  if (tid == 0)
-    prefetch_l2(bstate + ((size_t)it.c * H + it.h) * D * D, (uint32_t)(D * D * sizeof(float)));
-  if (tid < 3 * kChunk) {
-    const int r = tid % kChunk;
-    const IN* src = (tid < kChunk ? k : tid < 2 * kChunk ? q : v) + (tb + (size_t)r * H) * D;
-    if (r < it.len) prefetch_l2(src, (uint32_t)(D * sizeof(IN)));
-  }
-}
-
 template <int D, class IN, class OUT>
 __global__ void __launch_bounds__(kFillThreads, 3)
     k_fill(const IN* __restrict__ q, const IN* __restrict__ k, const IN* __restrict__ v,
@@ -917,7 +821,7 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(3));
-  {
+  if (!a.pass1_only) {
     auto kern = k_fill<D, IN, OUT>;
     const size_t sm = sizeof(FillSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));

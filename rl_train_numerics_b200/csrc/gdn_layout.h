@@ -76,6 +76,7 @@ struct FwdArgs {
   char* ws;
   FwdLayout lay;
   void* const* events;  // 5 cudaEvent_t recorded around the kernels, or null
+  int pass1_only;       // 1: chunk table and boundary states only (no fill, o unused)
 };
 
 struct DecArgs {
@@ -140,7 +141,46 @@ struct BndArgs {
   float* s_end;
 };
 
+// Workspace of gdn_cpr_backward: the forward's (its first pass runs again
+// inside the backward) followed by
+//   mu_end  f32[MC,H,dv,dk]  adjoint flowing into the state at the end of
+//                            every chunk (from the tokens after it)
+//   wbuf    f32[T,H,dv]      w_t = Lambda_t k_t, one value per state row
+//   ubuf    f32[T,H,dv]      u_t = beta_t (v_t - alpha_t S_{t-1} k_t) per row
+struct BwdLayout {
+  FwdLayout fwd;
+  size_t mu_end, wbuf, ubuf, total;
+};
+
+inline BwdLayout bwd_layout(int n_seqs, int64_t T, int H, int dk, int dv, int C, bool in_bf16) {
+  BwdLayout L{};
+  L.fwd = fwd_layout(n_seqs, T, H, dk, dv, C, in_bf16);
+  size_t off = L.fwd.total;
+  L.mu_end = off;
+  off += align256((size_t)L.fwd.max_chunks * H * dv * dk * sizeof(float));
+  L.wbuf = off;
+  off += align256((size_t)T * H * dv * sizeof(float));
+  L.ubuf = off;
+  off += align256((size_t)T * H * dv * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+struct BwdArgs {
+  FwdArgs fwd;  // inputs, shapes, scale, h0 and the workspace (first pass only)
+  const void* d_o;
+  const float* ds_final;
+  float* d_q;
+  float* d_k;
+  float* d_v;
+  float* d_beta;
+  float* d_g;
+  float* d_h0;
+  BwdLayout lay;
+};
+
 cudaError_t launch_forward(const FwdArgs& a, cudaStream_t stream);
+cudaError_t launch_backward(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_step(const DecArgs& a, cudaStream_t stream);
 cudaError_t launch_handoff(const HandoffArgs& a, cudaStream_t stream);
 cudaError_t launch_chunk_boundary(const BndArgs& a, cudaStream_t stream);

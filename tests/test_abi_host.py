@@ -34,7 +34,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["gdn_cpr_forward", "gdn_cpr_decode_step", "gdn_chunk_boundary",
               "gdn_cpr_decode_state_from_prefill", "gdn_check_error",
-              "gdn_cpr_forward_workspace_bytes", "gdn_status_string", "gdn_cpr_abi_version"]:
+              "gdn_cpr_forward_workspace_bytes", "gdn_status_string", "gdn_cpr_abi_version",
+              "gdn_cpr_backward", "gdn_cpr_backward_workspace_bytes"]:
         assert n in names
 
 
@@ -45,7 +46,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert gdn.lib.gdn_cpr_abi_version() == 4
+    assert gdn.lib.gdn_cpr_abi_version() == 5
     for code in range(-6, 1):
         assert gdn.status_string(code).startswith("GDN_")
     assert "unknown" in gdn.status_string(42)
@@ -109,6 +110,63 @@ def test_forward_rejects_on_host(over, expect):
 def test_forward_empty_batch_is_a_no_op():
     assert fwd(N=0, T=0, q=None, k=None, v=None, beta=None, g=None, o=None, cu=None,
                ws=None, wsb=0) == gdn.GDN_OK
+
+
+def test_backward_workspace_query():
+    import torch
+    fw, bw = gdn.forward_workspace_bytes, gdn.backward_workspace_bytes
+    # the forward's workspace plus adjoints at chunk ends and two [T, H, d] fp32 rows
+    assert bw(5, 10240, 16, 128, 128) >= fw(5, 10240, 16, 128, 128) + \
+        (10240 // 64 + 5) * 16 * 128 * 128 * 4 + 2 * 10240 * 16 * 128 * 4
+    assert bw(1, 100, 2, 128, 128, 64, torch.float32) == 0
+    assert bw(1, 100, 2, 96, 96) == 0
+    assert bw(-1, 100, 2, 64, 64) == 0
+
+
+def bwd(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, in_dtype=gdn.GDN_BF16, beta=FAKE, g=FAKE, cu=FAKE, N=2,
+             T=128, H=2, dk=64, dv=64, C=64, scale=1.0, h0=None, do=FAKE, dsf=None, dq=FAKE,
+             dk_=FAKE, dv_=FAKE, db=FAKE, dg=FAKE, dh0=None, ws=FAKE, wsb=1 << 40, stream=None)
+    a.update(over)
+    return gdn.lib.gdn_cpr_backward(a["q"], a["k"], a["v"], a["in_dtype"], a["beta"], a["g"],
+                                    a["cu"], a["N"], a["T"], a["H"], a["dk"], a["dv"], a["C"],
+                                    a["scale"], a["h0"], a["do"], a["dsf"], a["dq"], a["dk_"],
+                                    a["dv_"], a["db"], a["dg"], a["dh0"], a["ws"], a["wsb"],
+                                    a["stream"])
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(H=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(in_dtype=7), gdn.GDN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=96, dv=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(in_dtype=gdn.GDN_F32, dk=128, dv=128), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(C=128), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(T=1 << 31), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(do=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dq=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk_=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dv_=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(db=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dg=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(do=MIS), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dq=MIS), gdn.GDN_ERR_INVALID_ARG),
+    (dict(db=MIS + 2), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dsf=MIS), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dh0=MIS), gdn.GDN_ERR_INVALID_ARG),
+    (dict(ws=None), gdn.GDN_ERR_WORKSPACE),
+    (dict(wsb=4096), gdn.GDN_ERR_WORKSPACE),
+    (dict(ws=MIS), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=0, T=3), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_backward_rejects_on_host(over, expect):
+    assert bwd(**over) == expect
+
+
+def test_backward_empty_batch_is_a_no_op():
+    assert bwd(N=0, T=0, q=None, k=None, v=None, beta=None, g=None, do=None, dq=None, dk_=None,
+               dv_=None, db=None, dg=None, cu=None, ws=None, wsb=0) == gdn.GDN_OK
 
 
 def _state(**over):

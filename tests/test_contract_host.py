@@ -56,8 +56,11 @@ def test_policy_separates_what_moves_bits_semantic_does_not():
     assert sem(torch.bfloat16, torch.bfloat16, 64) == sem(torch.float32, torch.float32, 64)
     assert sem(torch.bfloat16, torch.bfloat16, 64) != sem(torch.bfloat16, torch.bfloat16, 128)
     text = gdn.contract_descriptor(gdn.GDN_DIGEST_POLICY, torch.bfloat16, torch.bfloat16, 128, 128)
-    for key in ("step_schedule=", "boundary_schedule=", "walk=tcgen05", "compile=", "splits="):
+    for key in ("step_schedule=", "boundary_schedule=", "walk=tcgen05", "compile=", "splits=",
+                "backward="):
         assert key in text
+    assert "gradients=" in gdn.contract_descriptor(gdn.GDN_DIGEST_SEMANTIC, torch.bfloat16,
+                                                   torch.bfloat16, 128, 128)
     text64 = gdn.contract_descriptor(gdn.GDN_DIGEST_POLICY, torch.bfloat16, torch.bfloat16, 64, 64)
     assert "walk=mma.sync" in text64
 
