@@ -40,14 +40,18 @@ FLUSH_BYTES = 256 << 20
 PAGES_H100 = {"prefill_ms": 1.412, "decode_ms": 0.0846, "trainer_fwd_bwd_ms": 7.386}
 
 
+KERNEL_FILES = ("gdn_kernels.cu", "gdn_backward.cu")
+
+
 def kernel_sources_sha256() -> str:
-    """SHA-256 over the files that define the kernels (gdn_kernels.cu and the
-    device headers; the host-only entry points are left out)."""
+    """SHA-256 over the files that define the kernels (the forward/decode and
+    backward kernel files and the device headers; the host-only entry points
+    are left out)."""
     import hashlib
     csrc = os.path.join(ROOT, "rl_train_numerics_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(csrc)):
-        if name == "gdn_kernels.cu" or name.endswith((".cuh", ".h")):
+        if name in KERNEL_FILES or name.endswith((".cuh", ".h")):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(f.read())
     return h.hexdigest()
@@ -386,7 +390,21 @@ def run_decode_part(gdn, W, dev, rank, world, args, peaks):
             "pages_h100_ms": PAGES_H100["decode_ms"]}
 
 
-def run_train_part(gdn, W, dev, rank, world, args, flush):
+def bwd_gemm_flops(lengths, H, D):
+    """Algorithmic FLOPs of the backward's chunk products: per chunk of length L,
+    Y (lower triangle incl. diagonal) and X (strict) over d, the three L x d x d
+    products (DO S_a, W S_a, U mu_e), A K and A^T Q (triangles incl. diagonal)
+    and (B + B^T) K (off-diagonal), two FLOPs per multiply-add."""
+    mac = 0
+    for Ln in lengths:
+        for c0 in range(0, Ln, C):
+            L = min(C, Ln - c0)
+            tri, stri = L * (L + 1) // 2, L * (L - 1) // 2
+            mac += D * (3 * tri + stri + 2 * stri) + 3 * L * D * D
+    return 2 * mac * H
+
+
+def run_train_part(gdn, W, dev, rank, world, args, flush, peaks):
     """Trainer step: the forward (o and final states) and the backward (every
     gradient, from a fixed synthetic dL/do) over the 10240-token trainer batch,
     L2 flushed before every step outside its events."""
@@ -396,40 +414,60 @@ def run_train_part(gdn, W, dev, rank, world, args, flush):
     d_o = torch.randn((T, H, D), generator=gen, device=dev).to(torch.bfloat16)
     o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
     srun = torch.empty((N, H, D, D), dtype=torch.float32, device=dev)
-    fws = torch.zeros(gdn.forward_workspace_bytes(N, T, H, D, D), dtype=torch.uint8, device=dev)
-    grads, bws = gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o)
+    grads, ws = gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o)
 
-    def step(e0, e1, e2):
-        e0.record()
+    def make_events():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+        for e in evs:
+            e.record()
+        return evs
+
+    # The forward runs on the backward's workspace, and the backward reuses its
+    # first pass (boundary states) instead of running it again.
+    def step(evs):
         gdn.forward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, o=o, s_run_final=srun,
-                    workspace=fws)
-        e1.record()
-        gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o, grads=grads, workspace=bws)
-        e2.record()
+                    workspace=ws, kernel_events=evs[:5])
+        gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o, grads=grads, workspace=ws,
+                     reuse_forward=True, kernel_events=evs[5:])
 
     steps, warmup = args.steps, args.warmup
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    warm = make_events()
     for _ in range(warmup):
         flush.zero_()
-        step(*evs[0])
+        step(warm)
+    evs = [make_events() for _ in range(steps)]
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     for i in range(steps):
         flush.zero_()
-        step(*evs[i])
+        step(evs[i])
     torch.cuda.synchronize()
     barrier(world)
-    if gdn.check_error(fws) != 0 or gdn.check_error(bws) != 0:
+    if gdn.check_error(ws) != 0:
         raise RuntimeError("device error word set in the trainer step")
-    fwd = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    bwd = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    el = lambda a, z: float(np.mean([e[a].elapsed_time(e[z]) for e in evs]))  # noqa: E731
+    fwd, bwd = el(0, 4), el(5, 9)
+    kern = {"fwd_chunk_table": el(0, 1), "fwd_boundary_prep": el(1, 2),
+            "fwd_boundary_walk": el(2, 3), "fwd_intra_chunk_fill": el(3, 4),
+            "bwd_adjoint_scan": el(6, 7), "bwd_chunk_rows": el(7, 8),
+            "bwd_chunk_products": el(8, 9)}
     ms = max_over_ranks(fwd + bwd, world)
+    fp32_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    gflop = bwd_gemm_flops(b.lengths, H, D) / 1e9
+    achieved = gflop / kern["bwd_chunk_products"]  # GFLOP per ms = TFLOP/s
     return {"workload": f"trainer: {T} tokens as {N} documents (lengths {b.lengths}), H={H}, "
                         f"d_k=d_v={D}, C={C}, bf16 q/k/v/do, fp32 beta/g/state/gradients",
             "steps": steps, "ms_per_step": round(ms, 5), "fwd_ms": round(fwd, 5),
             "bwd_ms": round(bwd, 5), "tokens_per_s": round(world * T / (ms / 1e3), 1),
-            "gpu_launches_per_step": 4 + 6,
+            "kernels_ms": {k: round(v, 5) for k, v in kern.items()},
+            "bwd_roofline": {"kernel": "bwd_chunk_products", "bound": "alu",
+                             "achieved": round(achieved, 2), "peak": round(fp32_peak, 2),
+                             "unit": "TFLOP/s", "frac": round(achieved / fp32_peak, 4),
+                             "traffic": ncu_traffic("bwd_chunk_products"),
+                             "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x sm_max_mhz "
+                                            "(nominal)"},
+            "gpu_launches_per_step": 4 + 3,
             "l2": "flushed (256 MiB write) before every timed step",
             "pages_h100_ms": PAGES_H100["trainer_fwd_bwd_ms"]}
 
@@ -462,6 +500,17 @@ def run_ours(args):
     from rl_train_numerics_b200 import _abi as gdn
     from rl_train_numerics_b200 import workloads as W
 
+    if args.only == "bwd-small":
+        # Profiling case for full ncu captures of the backward kernels: two
+        # backward calls on 2 x 1024 tokens, H = 8, d = 128, bf16; no JSON line.
+        b = W.make_batch([1024, 1024], 8, D, D, dtype=torch.bfloat16, seed=3, device=dev)
+        gen = torch.Generator(device=dev).manual_seed(4)
+        d_o = torch.randn((b.total_tokens, 8, D), generator=gen, device=dev).to(torch.bfloat16)
+        grads, ws = gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o)
+        gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o, grads=grads, workspace=ws)
+        if gdn.check_error(ws) != 0:
+            raise RuntimeError("device error word set by the backward")
+        return
     peaks = load_peaks()
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     b, bufs, step, evs = bench_prefill(gdn, W, dev, rank, args.steps, args.warmup, flush)
@@ -538,7 +587,7 @@ def run_ours(args):
         decode = run_decode_part(gdn, W, dev, rank, world, args, peaks)
     train = None
     if args.only in ("all", "train"):
-        train = run_train_part(gdn, W, dev, rank, world, args, flush)
+        train = run_train_part(gdn, W, dev, rank, world, args, flush, peaks)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -625,7 +674,8 @@ def main():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--decode-steps", type=int, default=512)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--only", choices=["all", "prefill", "decode", "train"], default="all",
+    p.add_argument("--only", choices=["all", "prefill", "decode", "train", "bwd-small"],
+                   default="all",
                    help="profiling aid: run only part of the benchmark")
     p.add_argument("--decode-slots", type=int, default=256)
     args = p.parse_args()

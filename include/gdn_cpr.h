@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define GDN_CPR_ABI_VERSION 5
+#define GDN_CPR_ABI_VERSION 6
 
 typedef enum {
   GDN_OK = 0,
@@ -298,16 +298,43 @@ size_t gdn_cpr_backward_workspace_bytes(int n_seqs, int64_t total_tokens, int H,
  *             NULL to skip it
  * workspace: device scratch of at least gdn_cpr_backward_workspace_bytes
  *   bytes, 16-byte aligned.  Its first 4 bytes are the device error word.
+ *   Its first gdn_cpr_forward_workspace_bytes bytes are laid out as the
+ *   forward's workspace, so the same buffer can serve a gdn_cpr_forward call.
+ * flags: 0, or GDN_BWD_REUSE_FORWARD: the workspace was last written by a
+ *   gdn_cpr_forward call with the same q, k, v, beta, g, cu_seqlens, h0,
+ *   shapes and C (a trainer's forward followed by its backward); the first
+ *   pass is then not run again, and the gradients are bit for bit those of a
+ *   call without the flag.  The library cannot check that promise; gradients
+ *   of a different batch's boundary states are wrong, not an error.
  * Pointers to device arrays of 16-byte rows must be 16-byte aligned.
- * Status: as gdn_cpr_forward; invalid cu_seqlens set GDN_DEVERR_CU_SEQLENS
- * in the error word and leave the outputs unwritten.
+ * Status: as gdn_cpr_forward (GDN_ERR_INVALID_ARG also for unknown flags);
+ * invalid cu_seqlens set GDN_DEVERR_CU_SEQLENS in the error word and leave
+ * the outputs unwritten.
  */
+#define GDN_BWD_REUSE_FORWARD 1
 int gdn_cpr_backward(const void* q, const void* k, const void* v, int in_dtype,
                      const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
                      int64_t total_tokens, int H, int dk, int dv, int C, float scale,
                      const float* h0, const void* d_o, const float* ds_final, float* d_q,
                      float* d_k, float* d_v, float* d_beta, float* d_g, float* d_h0,
-                     void* workspace, size_t workspace_bytes, void* stream);
+                     void* workspace, size_t workspace_bytes, int flags, void* stream);
+
+/*
+ * gdn_cpr_backward_ex -- gdn_cpr_backward that also records caller-created
+ * CUDA events on `stream` around its kernels, for per-kernel timing:
+ * kernel_events[0] before the first pass (recorded even when it is reused),
+ * [1] before the adjoint scan, [2] before the per-chunk state recomputation,
+ * [3] before the chunk products and [4] after them (an array of 5
+ * cudaEvent_t passed as void*, or NULL for none).  The computation and its
+ * bits are exactly those of gdn_cpr_backward.
+ */
+int gdn_cpr_backward_ex(const void* q, const void* k, const void* v, int in_dtype,
+                        const float* beta, const float* g, const int32_t* cu_seqlens,
+                        int n_seqs, int64_t total_tokens, int H, int dk, int dv, int C,
+                        float scale, const float* h0, const void* d_o, const float* ds_final,
+                        float* d_q, float* d_k, float* d_v, float* d_beta, float* d_g,
+                        float* d_h0, void* workspace, size_t workspace_bytes, int flags,
+                        void* const* kernel_events, void* stream);
 
 /*
  * gdn_check_error -- synchronise `stream`, read the device error word at

@@ -32,6 +32,7 @@ GDN_F32 = 1
 GDN_DEVERR_CU_SEQLENS = 1
 GDN_DEVERR_POS = 2
 GDN_DEVERR_TIMEOUT = 4
+GDN_BWD_REUSE_FORWARD = 1
 CHUNK = 64
 
 
@@ -75,7 +76,10 @@ def _load() -> ctypes.CDLL:
         "gdn_chunk_boundary": (i32, [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
         "gdn_cpr_backward_workspace_bytes": (sz, [i32, i64, i32, i32, i32, i32, i32]),
         "gdn_cpr_backward": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32,
-                                   f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+                                   f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, vp]),
+        "gdn_cpr_backward_ex": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32,
+                                      i32, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i32,
+                                      vp, vp]),
         "gdn_check_error": (i32, [vp, vp, vp]),
         "gdn_cpr_contract_descriptor": (i32, [i32, i32, i32, i32, i32, i32, ctypes.c_char_p, sz,
                                               ctypes.POINTER(ctypes.c_size_t)]),
@@ -197,10 +201,14 @@ def backward_workspace_bytes(n_seqs: int, total_tokens: int, H: int, dk: int, dv
 
 def backward(q, k, v, beta, g, cu_seqlens, d_o, *, n_seqs: Optional[int] = None, h0=None,
              ds_final=None, C: int = CHUNK, scale: float = 1.0, want_dh0: bool = True,
-             grads=None, workspace=None, stream=None):
+             grads=None, workspace=None, reuse_forward: bool = False, stream=None,
+             kernel_events=None):
     """gdn_cpr_backward.  Returns (grads, workspace); grads is a dict of fp32
     tensors dq, dk, dv [T, H, d], dbeta, dg [T, H] and dh0 [N, H, dv, dk]
-    (None unless want_dh0).  Pass ``grads`` (the same dict) to reuse buffers."""
+    (None unless want_dh0).  Pass ``grads`` (the same dict) to reuse buffers.
+    reuse_forward=True (GDN_BWD_REUSE_FORWARD): ``workspace`` was last used by
+    forward() on this same batch, whose first pass is then reused.
+    kernel_events: 5 recorded torch.cuda.Event objects (gdn_cpr_backward_ex)."""
     T, H, dk = q.shape
     dv = v.shape[2]
     N = (cu_seqlens.numel() - 1) if n_seqs is None else int(n_seqs)
@@ -217,12 +225,18 @@ def backward(q, k, v, beta, g, cu_seqlens, d_o, *, n_seqs: Optional[int] = None,
     need = backward_workspace_bytes(N, T, H, dk, dv, C, q.dtype)
     if workspace is None:
         workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
-    st = lib.gdn_cpr_backward(_ptr(q), _ptr(k), _ptr(v), in_code, _ptr(beta), _ptr(g),
-                              _ptr(cu_seqlens), N, T, H, dk, dv, C, float(scale), _ptr(h0),
-                              _ptr(d_o), _ptr(ds_final), _ptr(grads["dq"]), _ptr(grads["dk"]),
-                              _ptr(grads["dv"]), _ptr(grads["dbeta"]), _ptr(grads["dg"]),
-                              _ptr(grads.get("dh0")), _ptr(workspace), workspace.numel(),
-                              _stream(stream))
+    ev = None
+    if kernel_events is not None:
+        if len(kernel_events) != 5 or any(e.cuda_event == 0 for e in kernel_events):
+            raise ValueError("kernel_events: 5 torch.cuda.Event objects, each recorded once")
+        ev = (ctypes.c_void_p * 5)(*[e.cuda_event for e in kernel_events])
+    st = lib.gdn_cpr_backward_ex(_ptr(q), _ptr(k), _ptr(v), in_code, _ptr(beta), _ptr(g),
+                                 _ptr(cu_seqlens), N, T, H, dk, dv, C, float(scale), _ptr(h0),
+                                 _ptr(d_o), _ptr(ds_final), _ptr(grads["dq"]),
+                                 _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["dbeta"]),
+                                 _ptr(grads["dg"]), _ptr(grads.get("dh0")), _ptr(workspace),
+                                 workspace.numel(), GDN_BWD_REUSE_FORWARD if reuse_forward else 0,
+                                 ev, _stream(stream))
     _check(st, "gdn_cpr_backward")
     return grads, workspace
 

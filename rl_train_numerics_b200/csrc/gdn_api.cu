@@ -127,8 +127,21 @@ int gdn_cpr_backward(const void* q, const void* k, const void* v, int in_dtype,
                      int64_t total_tokens, int H, int dk, int dv, int C, float scale,
                      const float* h0, const void* d_o, const float* ds_final, float* d_q,
                      float* d_k, float* d_v, float* d_beta, float* d_g, float* d_h0,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+                     void* workspace, size_t workspace_bytes, int flags, void* stream) {
+  return gdn_cpr_backward_ex(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs, total_tokens, H, dk,
+                             dv, C, scale, h0, d_o, ds_final, d_q, d_k, d_v, d_beta, d_g, d_h0,
+                             workspace, workspace_bytes, flags, nullptr, stream);
+}
+
+int gdn_cpr_backward_ex(const void* q, const void* k, const void* v, int in_dtype,
+                        const float* beta, const float* g, const int32_t* cu_seqlens,
+                        int n_seqs, int64_t total_tokens, int H, int dk, int dv, int C,
+                        float scale, const float* h0, const void* d_o, const float* ds_final,
+                        float* d_q, float* d_k, float* d_v, float* d_beta, float* d_g,
+                        float* d_h0, void* workspace, size_t workspace_bytes, int flags,
+                        void* const* kernel_events, void* stream) {
   if (n_seqs < 0 || total_tokens < 0 || !isfinite(scale)) return GDN_ERR_INVALID_ARG;
+  if ((flags & ~GDN_BWD_REUSE_FORWARD) != 0) return GDN_ERR_INVALID_ARG;
   int rc = check_shape(H, dk, dv, C, in_dtype);
   if (rc != GDN_OK) return rc;
   if (total_tokens > INT32_MAX) return GDN_ERR_UNSUPPORTED;
@@ -173,7 +186,9 @@ int gdn_cpr_backward(const void* q, const void* k, const void* v, int in_dtype,
   a.d_beta = d_beta;
   a.d_g = d_g;
   a.d_h0 = d_h0;
+  a.reuse_forward = (flags & GDN_BWD_REUSE_FORWARD) ? 1 : 0;
   a.lay = lay;
+  a.events = kernel_events;
   return from_cuda(gdn::launch_backward(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -273,13 +273,21 @@ __global__ void __launch_bounds__(kFillThreads, 3)
   const bool mine = l < RT;  // lane l accounts for row r0 + l
   const int rl = mine ? l : 0;
   const size_t tb = (size_t)it.t0 * H + h;
+  // w and do of row r0 + rl are loaded one token ahead, so that their latency
+  // hides behind a token's work.
+  const size_t idx0 = tb * D + r0 + rl, tstride = (size_t)H * D;
+  float wr_next = (mine && it.len > 0) ? wbuf[idx0] : 0.f;
+  float do_next = (mine && it.len > 0) ? ld1(d_o + idx0) : 0.f;
   for (int t = 0; t < it.len; t++) {
     const float a = sm.f.a[t], b = sm.f.b[t];
     const float pr = __fmul_rn(cs, pick<RT>(p, rl));  // p_t of row r0 + rl
     const float vr = to_f(sm.f.v[t][r0 + rl]);
-    const size_t idx = (tb + (size_t)t * H) * D + r0 + rl;
-    const float wr = mine ? wbuf[idx] : 0.f;
-    const float dor = mine ? ld1(d_o + idx) : 0.f;
+    const size_t idx = idx0 + (size_t)t * tstride;
+    const float wr = wr_next, dor = do_next;
+    if (mine && t + 1 < it.len) {
+      wr_next = wbuf[idx + tstride];
+      do_next = ld1(d_o + idx + tstride);
+    }
     float ov[RT];
     slice_token<true, RT, M4>(
         S, cs, a, b, [&](int i) { return to_f(sm.f.v[t][r0 + i]); },
@@ -363,18 +371,37 @@ struct GemmSmem {
   float bet[kChunk];
 };
 
-// Transpose C x D rows (token-major in HBM, [t][h][i]) into [i][t] fp32.
-template <int D, class T>
-__device__ __forceinline__ void load_transposed(float (*dst)[kChunk], const T* src, size_t tb,
-                                                int H, int len) {
-  for (int e = threadIdx.x; e < kChunk * (D / 4); e += kGemmThreads) {
+// Transpose the chunk's C x D rows of do, w and u (token-major in HBM,
+// [t][h][i]) into [i][t] fp32: every load is issued before the first store.
+template <int D, class IN>
+__device__ __forceinline__ void load_transposed3(GemmSmem<D, IN>& sm, const IN* d_o,
+                                                 const float* wbuf, const float* ubuf, size_t tb,
+                                                 int H, int len) {
+  constexpr int IT = kChunk * (D / 4) / kGemmThreads;
+  float4 x[3][IT];
+#pragma unroll
+  for (int j = 0; j < IT; j++) {
+    const int e = threadIdx.x + j * kGemmThreads;
     const int t = e % kChunk, i = (e / kChunk) * 4;
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (t < len) x = ld4(src + (tb + (size_t)t * H) * D + i);
-    dst[i][t] = x.x;
-    dst[i + 1][t] = x.y;
-    dst[i + 2][t] = x.z;
-    dst[i + 3][t] = x.w;
+    const size_t off = (tb + (size_t)t * H) * D + i;
+    const bool in = t < len;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    x[0][j] = in ? ld4(d_o + off) : z;
+    x[1][j] = in ? ld4(wbuf + off) : z;
+    x[2][j] = in ? ld4(ubuf + off) : z;
+  }
+#pragma unroll
+  for (int j = 0; j < IT; j++) {
+    const int e = threadIdx.x + j * kGemmThreads;
+    const int t = e % kChunk, i = (e / kChunk) * 4;
+    float (*dst[3])[kChunk] = {sm.DOt, sm.Wt, sm.Ut};
+#pragma unroll
+    for (int a = 0; a < 3; a++) {
+      dst[a][i][t] = x[a][j].x;
+      dst[a][i + 1][t] = x[a][j].y;
+      dst[a][i + 2][t] = x[a][j].z;
+      dst[a][i + 3][t] = x[a][j].w;
+    }
   }
 }
 
@@ -394,26 +421,30 @@ __device__ __forceinline__ void slab_issue(GemmSmem<D, IN>& sm, int buf, int j, 
   cp_async_commit();
 }
 
+// The NC columns a thread owns: groups of four at 4 tx + 64 jg, so that the
+// 16 threads of a row read 16 consecutive float4 (no bank conflicts).
+__device__ __forceinline__ int own_col(int tx, int jg) { return 4 * tx + 64 * jg; }
+
 template <int NC>
-__device__ __forceinline__ void row_ld(const float* p, float (&x)[NC]) {
+__device__ __forceinline__ void cols_ld(const float* row, int tx, float (&x)[NC]) {
 #pragma unroll
-  for (int j = 0; j < NC; j += 4) {
-    const float4 v = *reinterpret_cast<const float4*>(p + j);
-    x[j] = v.x;
-    x[j + 1] = v.y;
-    x[j + 2] = v.z;
-    x[j + 3] = v.w;
+  for (int jg = 0; jg < NC / 4; jg++) {
+    const float4 v = *reinterpret_cast<const float4*>(row + own_col(tx, jg));
+    x[4 * jg] = v.x;
+    x[4 * jg + 1] = v.y;
+    x[4 * jg + 2] = v.z;
+    x[4 * jg + 3] = v.w;
   }
 }
 template <int NC>
-__device__ __forceinline__ void row_ld(const __nv_bfloat16* p, float (&x)[NC]) {
+__device__ __forceinline__ void cols_ld(const __nv_bfloat16* row, int tx, float (&x)[NC]) {
 #pragma unroll
-  for (int j = 0; j < NC; j += 4) {
-    const float4 v = sld4(p + j);
-    x[j] = v.x;
-    x[j + 1] = v.y;
-    x[j + 2] = v.z;
-    x[j + 3] = v.w;
+  for (int jg = 0; jg < NC / 4; jg++) {
+    const float4 v = sld4(row + own_col(tx, jg));
+    x[4 * jg] = v.x;
+    x[4 * jg + 1] = v.y;
+    x[4 * jg + 2] = v.z;
+    x[4 * jg + 3] = v.w;
   }
 }
 
@@ -450,16 +481,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const float* Me = mu_end + ((size_t)c * H + h) * DD;
 
   slab_issue<D, IN>(sm, 0, 0, Sa, Me);  // lands while the chunk's rows load
-  load_transposed<D>(sm.DOt, d_o, tb, H, len);
-  load_transposed<D>(sm.Wt, wbuf, tb, H, len);
-  load_transposed<D>(sm.Ut, ubuf, tb, H, len);
-  for (int e = tid; e < 2 * kChunk * P; e += kGemmThreads) {
-    const int row = e / P, pc = (e % P) * E, t = row % kChunk;
-    IN* dst = row < kChunk ? &sm.Q[t][pc] : &sm.K[t][pc];
-    uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (t < len) x = *reinterpret_cast<const uint4*>((row < kChunk ? q : k) +
-                                                      (tb + (size_t)t * H) * D + pc);
-    *reinterpret_cast<uint4*>(dst) = x;
+  {
+    constexpr int QI = 2 * kChunk * P / kGemmThreads;
+    uint4 x[QI];
+#pragma unroll
+    for (int j = 0; j < QI; j++) {
+      const int e = tid + j * kGemmThreads;
+      const int row = e / P, pc = (e % P) * E, t = row % kChunk;
+      x[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (t < len) x[j] = *reinterpret_cast<const uint4*>((row < kChunk ? q : k) +
+                                                           (tb + (size_t)t * H) * D + pc);
+    }
+    load_transposed3<D, IN>(sm, d_o, wbuf, ubuf, tb, H, len);
+#pragma unroll
+    for (int j = 0; j < QI; j++) {
+      const int e = tid + j * kGemmThreads;
+      const int row = e / P, pc = (e % P) * E, t = row % kChunk;
+      *reinterpret_cast<uint4*>(row < kChunk ? &sm.Q[t][pc] : &sm.K[t][pc]) = x[j];
+    }
   }
   if (tid < kChunk) sm.bet[tid] = tid < len ? beta[tb + (size_t)tid * H] : 0.f;
   if (tid == 0) {
@@ -519,7 +558,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fw[a] = -__fmul_rn(sm.bet[t], eg);       // -beta_t e^{G_t}  (W S_a)
     fu[a] = expf((float)(GL - sm.G[t]));     // e^{G_{L-1}-G_t}  (U mu_e)
   }
-  const int c0 = tx * NC;
   float aq[4][NC] = {}, ak[4][NC] = {};
   constexpr int NS = D / kSlab;
   for (int j = 0; j < NS; j++) {
@@ -531,8 +569,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int rr = 0; rr < kSlab; rr++) {
       const int i = j * kSlab + rr;
       float sv[NC], mv[NC], dv[4], wv[4], uv[4];
-      row_ld<NC>(&sm.Sa[bi][rr][c0], sv);
-      row_ld<NC>(&sm.Me[bi][rr][c0], mv);
+      cols_ld<NC>(&sm.Sa[bi][rr][0], tx, sv);
+      cols_ld<NC>(&sm.Me[bi][rr][0], tx, mv);
       f4a(*reinterpret_cast<const float4*>(&sm.DOt[i][t4]), dv);
       f4a(*reinterpret_cast<const float4*>(&sm.Wt[i][t4]), wv);
       f4a(*reinterpret_cast<const float4*>(&sm.Ut[i][t4]), uv);
@@ -551,8 +589,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   for (int s = 0; s < len; s++) {
     float kr[NC], qr[NC], av[4], bv[4];
-    row_ld<NC>(&sm.K[s][c0], kr);
-    row_ld<NC>(&sm.Q[s][c0], qr);
+    cols_ld<NC>(&sm.K[s][0], tx, kr);
+    cols_ld<NC>(&sm.Q[s][0], tx, qr);
     f4a(*reinterpret_cast<const float4*>(&sm.As[s][t4]), av);
     f4a(*reinterpret_cast<const float4*>(&sm.Bs[s][t4]), bv);
 #pragma unroll
@@ -573,14 +611,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   for (int a = 0; a < 4; a++) {
     const int t = t4 + a;
     if (t >= len) continue;
-    float* oq = d_q + (tb + (size_t)t * H) * D + c0;
-    float* ok = d_k + (tb + (size_t)t * H) * D + c0;
+    float* oq = d_q + (tb + (size_t)t * H) * D;
+    float* ok = d_k + (tb + (size_t)t * H) * D;
 #pragma unroll
-    for (int jj = 0; jj < NC; jj += 4) {
-      *reinterpret_cast<float4*>(oq + jj) =
+    for (int jg = 0; jg < NC / 4; jg++) {
+      const int jj = 4 * jg, col = own_col(tx, jg);
+      *reinterpret_cast<float4*>(oq + col) =
           make_float4(__fmul_rn(scale, aq[a][jj]), __fmul_rn(scale, aq[a][jj + 1]),
                       __fmul_rn(scale, aq[a][jj + 2]), __fmul_rn(scale, aq[a][jj + 3]));
-      *reinterpret_cast<float4*>(ok + jj) =
+      *reinterpret_cast<float4*>(ok + col) =
           make_float4(ak[a][jj], ak[a][jj + 1], ak[a][jj + 2], ak[a][jj + 3]);
     }
   }
@@ -602,7 +641,12 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   f.s_run_final = f.s_run_scale = f.s_bnd_final = nullptr;
   f.events = nullptr;
   f.lay = a.lay.fwd;
-  GDN_BWD_TRY(launch_forward(f, st));
+  auto mark = [&](int i) -> cudaError_t {
+    return a.events ? cudaEventRecord(static_cast<cudaEvent_t>(a.events[i]), st) : cudaSuccess;
+  };
+  GDN_BWD_TRY(mark(0));
+  if (!a.reuse_forward) GDN_BWD_TRY(launch_forward(f, st));
+  GDN_BWD_TRY(mark(1));
   const BwdLayout& L = a.lay;
   char* ws = f.ws;
   const int32_t* hdr = reinterpret_cast<const int32_t*>(ws + L.fwd.hdr);
@@ -626,6 +670,7 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
     GDN_BWD_TRY(cudaGetLastError());
   }
   const dim3 gchunks((unsigned)L.fwd.max_chunks, (unsigned)f.H);
+  GDN_BWD_TRY(mark(2));
   {
     auto kern = k_bwd_rows<D, IN>;
     const size_t sm = sizeof(RowsSmem<D, IN>);
@@ -635,6 +680,7 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
                                             a.d_beta, a.d_g);
     GDN_BWD_TRY(cudaGetLastError());
   }
+  GDN_BWD_TRY(mark(3));
   {
     auto kern = k_bwd_gemm<D, IN>;
     const size_t sm = sizeof(GemmSmem<D, IN>);
@@ -644,7 +690,7 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
                                             a.d_q, a.d_k);
     GDN_BWD_TRY(cudaGetLastError());
   }
-  return cudaSuccess;
+  return mark(4);
 }
 
 cudaError_t launch_backward(const BwdArgs& a, cudaStream_t st) {

@@ -176,7 +176,9 @@ struct BwdArgs {
   float* d_beta;
   float* d_g;
   float* d_h0;
+  int reuse_forward;  // 1: the workspace already holds this batch's first pass
   BwdLayout lay;
+  void* const* events;  // 5 cudaEvent_t recorded around the kernels, or null
 };
 
 cudaError_t launch_forward(const FwdArgs& a, cudaStream_t stream);

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert gdn.lib.gdn_cpr_abi_version() == 5
+    assert gdn.lib.gdn_cpr_abi_version() == 6
     for code in range(-6, 1):
         assert gdn.status_string(code).startswith("GDN_")
     assert "unknown" in gdn.status_string(42)
@@ -126,13 +126,14 @@ def test_backward_workspace_query():
 def bwd(**over):
     a = dict(q=FAKE, k=FAKE, v=FAKE, in_dtype=gdn.GDN_BF16, beta=FAKE, g=FAKE, cu=FAKE, N=2,
              T=128, H=2, dk=64, dv=64, C=64, scale=1.0, h0=None, do=FAKE, dsf=None, dq=FAKE,
-             dk_=FAKE, dv_=FAKE, db=FAKE, dg=FAKE, dh0=None, ws=FAKE, wsb=1 << 40, stream=None)
+             dk_=FAKE, dv_=FAKE, db=FAKE, dg=FAKE, dh0=None, ws=FAKE, wsb=1 << 40, flags=0,
+             stream=None)
     a.update(over)
     return gdn.lib.gdn_cpr_backward(a["q"], a["k"], a["v"], a["in_dtype"], a["beta"], a["g"],
                                     a["cu"], a["N"], a["T"], a["H"], a["dk"], a["dv"], a["C"],
                                     a["scale"], a["h0"], a["do"], a["dsf"], a["dq"], a["dk_"],
                                     a["dv_"], a["db"], a["dg"], a["dh0"], a["ws"], a["wsb"],
-                                    a["stream"])
+                                    a["flags"], a["stream"])
 
 
 @pytest.mark.parametrize("over,expect", [
@@ -159,6 +160,8 @@ def bwd(**over):
     (dict(wsb=4096), gdn.GDN_ERR_WORKSPACE),
     (dict(ws=MIS), gdn.GDN_ERR_INVALID_ARG),
     (dict(N=0, T=3), gdn.GDN_ERR_INVALID_ARG),
+    (dict(flags=2), gdn.GDN_ERR_INVALID_ARG),
+    (dict(flags=-1), gdn.GDN_ERR_INVALID_ARG),
 ])
 def test_backward_rejects_on_host(over, expect):
     assert bwd(**over) == expect

@@ -136,6 +136,24 @@ def test_repeat_runs_are_identical(gdn):
             assert torch.equal(first[k], again[k]), k
 
 
+def test_reusing_the_forwards_first_pass_changes_no_bit(gdn):
+    """forward() on the backward's workspace, then backward(reuse_forward=True):
+    the same bits as a backward that runs the first pass itself."""
+    b = W.make_batch([300, 64, 5, 190], 3, 128, 128, seed=32).to("cuda")
+    d_o, dsf = cotangents(b, 3, 128, 33, torch.bfloat16)
+    d_o, dsf = d_o.cuda(), dsf.cuda()
+    h0 = (torch.randn((4, 3, 128, 128), generator=torch.Generator().manual_seed(34)) * 0.2).cuda()
+    ref, _ = gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o, ds_final=dsf, h0=h0)
+    ws = torch.zeros(gdn.backward_workspace_bytes(4, b.total_tokens, 3, 128, 128),
+                     dtype=torch.uint8, device="cuda")
+    gdn.forward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, h0=h0, workspace=ws)
+    got, _ = gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o, ds_final=dsf, h0=h0,
+                          workspace=ws, reuse_forward=True)
+    assert gdn.check_error(ws) == 0
+    for k in NAMES:
+        assert torch.equal(ref[k], got[k]), k
+
+
 def test_bad_cu_seqlens_sets_the_error_word(gdn):
     b = W.make_batch([64, 64], 2, 64, 64, dtype=torch.float32, seed=30).to("cuda")
     bad = torch.tensor([0, 100, 64], dtype=torch.int32, device="cuda")  # decreasing
