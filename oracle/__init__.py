@@ -21,6 +21,9 @@ oracle for every output is the plain recurrence
 
 evaluated token by token in float64 with no chunking (``forward``).
 
+The module ``oracle.pik`` is the oracle of the parallelism-invariant K-leaf
+GEMM (section "Making kernels parallelism-invariant" of the same page).
+
 Functions
 ---------
 forward / forward_alpha   the token loop, in C (``gdn_oracle.c``), OpenMP
