@@ -472,6 +472,56 @@ def run_train_part(gdn, W, dev, rank, world, args, flush, peaks):
             "pages_h100_ms": PAGES_H100["trainer_fwd_bwd_ms"]}
 
 
+PIK_SHAPE = (8192, 8192, 8192, 8)  # M, N, K, leaves
+
+
+def run_pik_part(gdn, dev, rank, world, args, flush, peaks):
+    """Parallelism-invariant K-leaf GEMM: C = A B^T, M = N = K = 8192, 8 leaves,
+    bf16 in, fp32 out, one emulated rank; L2 flushed before every timed call.
+    cuBLAS bf16 (torch.matmul) on the same operands is timed beside it."""
+    M, N, K, L = PIK_SHAPE
+    gen = torch.Generator(device=dev).manual_seed(2000 + rank)
+    A = torch.randn((M, K), generator=gen, device=dev).to(torch.bfloat16)
+    B = torch.randn((N, K), generator=gen, device=dev).to(torch.bfloat16)
+    C = torch.empty((M, N), dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def timed(fn, steps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs]))
+
+    steps = max(3, min(args.steps, 10))
+    ms = timed(lambda: gdn.pik_gemm(A, B, L, 1, C=C, error=err), steps)
+    if gdn.check_error(err) != 0:
+        raise RuntimeError("device error word set by the K-leaf GEMM")
+    ms_cublas = timed(lambda: torch.matmul(A, B.T), steps)
+    ms = max_over_ranks(ms, world)
+    tflops = 2.0 * M * N * K / (ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"workload": f"C = A B^T, M=N=K={M}, {L} leaves of {K // L}, bf16 in, fp32 out, "
+                        "1 emulated rank (the bits are the same for every rank count)",
+            "ms": round(ms, 4), "tflops": round(world * tflops, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                         "traffic": ncu_traffic("pik_gemm"),
+                         "peak_source": f"measured cuBLAS bf16 burst ({peaks['source']})"},
+            "cublas_bf16_ms": round(ms_cublas, 4),
+            "cublas_bf16_tflops": round(2.0 * M * N * K / (ms_cublas / 1e3) / 1e12, 1),
+            "gpu_launches_per_call": 1,
+            "l2": "flushed (256 MiB write) before every timed call"}
+
+
 def cpu_baseline_sample(W, seconds=10.0):
     """The fp64 oracle as it stands, all host cores, on whole sequences of the
     prefill batch until about `seconds` of CPU work has been done."""
@@ -588,6 +638,9 @@ def run_ours(args):
     train = None
     if args.only in ("all", "train"):
         train = run_train_part(gdn, W, dev, rank, world, args, flush, peaks)
+    pikr = None
+    if args.only in ("all", "pik"):
+        pikr = run_pik_part(gdn, dev, rank, world, args, flush, peaks)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -607,6 +660,7 @@ def run_ours(args):
         "e2e": e2e,
         "decode": decode,
         "train_step": train,
+        "pik_gemm": pikr,
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
         "wall_s_timed_region": round(wall, 4),
@@ -674,7 +728,7 @@ def main():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--decode-steps", type=int, default=512)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--only", choices=["all", "prefill", "decode", "train", "bwd-small"],
+    p.add_argument("--only", choices=["all", "prefill", "decode", "train", "pik", "bwd-small"],
                    default="all",
                    help="profiling aid: run only part of the benchmark")
     p.add_argument("--decode-slots", type=int, default=256)

@@ -80,6 +80,8 @@ def _load() -> ctypes.CDLL:
         "gdn_cpr_backward_ex": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32,
                                       i32, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i32,
                                       vp, vp]),
+        "gdn_pik_workspace_bytes": (sz, [i64, i64, i64, i32, i32]),
+        "gdn_pik_gemm": (i32, [vp, vp, vp, i64, i64, i64, i32, i32, vp, sz, vp, vp]),
         "gdn_check_error": (i32, [vp, vp, vp]),
         "gdn_cpr_contract_descriptor": (i32, [i32, i32, i32, i32, i32, i32, ctypes.c_char_p, sz,
                                               ctypes.POINTER(ctypes.c_size_t)]),
@@ -239,6 +241,37 @@ def backward(q, k, v, beta, g, cu_seqlens, d_o, *, n_seqs: Optional[int] = None,
                                  ev, _stream(stream))
     _check(st, "gdn_cpr_backward")
     return grads, workspace
+
+
+def pik_workspace_bytes(M: int, N: int, K: int, n_leaves: int, n_ranks: int = 1) -> int:
+    return int(lib.gdn_pik_workspace_bytes(M, N, K, n_leaves, n_ranks))
+
+
+def pik_gemm(A, B, n_leaves: int, n_ranks: int = 1, *, C=None, workspace=None, error=None,
+             stream=None):
+    """gdn_pik_gemm: C = A B^T (A [M, K], B [N, K] bf16; C [M, N] fp32) with K in
+    n_leaves contiguous leaves combined by the fixed binary tree, computed in the
+    layout of n_ranks emulated ranks.  Returns (C, error word tensor)."""
+    if A.dtype != torch.bfloat16 or B.dtype != torch.bfloat16:
+        raise ValueError("gdn_pik_gemm: A and B must be bf16")
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError("gdn_pik_gemm: A and B must have the same K")
+    dev = A.device
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.float32, device=dev)
+    need = pik_workspace_bytes(M, N, K, n_leaves, n_ranks)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if error is None:
+        error = torch.zeros(1, dtype=torch.int32, device=dev)
+    st = lib.gdn_pik_gemm(_ptr(A) if K else None, _ptr(B) if K else None, _ptr(C), M, N, K,
+                          int(n_leaves), int(n_ranks),
+                          _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                          _ptr(error), _stream(stream))
+    _check(st, "gdn_pik_gemm")
+    return C, error
 
 
 def check_error(error_word: torch.Tensor, stream=None) -> int:

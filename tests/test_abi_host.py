@@ -24,7 +24,9 @@ MIS = 0x10004   # misaligned
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    inc = os.path.join(ROOT, "include")
+    text = "".join(open(os.path.join(inc, f)).read() for f in sorted(os.listdir(inc))
+                   if f.endswith(".h"))
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\s*\*)\s*(gdn_\w+)\s*\(",
                                  text, flags=re.M)))
@@ -35,7 +37,8 @@ def test_header_declares_the_entry_points():
     for n in ["gdn_cpr_forward", "gdn_cpr_decode_step", "gdn_chunk_boundary",
               "gdn_cpr_decode_state_from_prefill", "gdn_check_error",
               "gdn_cpr_forward_workspace_bytes", "gdn_status_string", "gdn_cpr_abi_version",
-              "gdn_cpr_backward", "gdn_cpr_backward_workspace_bytes"]:
+              "gdn_cpr_backward", "gdn_cpr_backward_workspace_bytes", "gdn_pik_gemm",
+              "gdn_pik_workspace_bytes"]:
         assert n in names
 
 
@@ -170,6 +173,44 @@ def test_backward_rejects_on_host(over, expect):
 def test_backward_empty_batch_is_a_no_op():
     assert bwd(N=0, T=0, q=None, k=None, v=None, beta=None, g=None, do=None, dq=None, dk_=None,
                dv_=None, db=None, dg=None, cu=None, ws=None, wsb=0) == gdn.GDN_OK
+
+
+def pik(**over):
+    a = dict(A=FAKE, B=FAKE, C=FAKE, M=256, N=256, K=1024, L=8, R=1, ws=FAKE, wsb=1 << 40,
+             err=FAKE, stream=None)
+    a.update(over)
+    return gdn.lib.gdn_pik_gemm(a["A"], a["B"], a["C"], a["M"], a["N"], a["K"], a["L"], a["R"],
+                                a["ws"], a["wsb"], a["err"], a["stream"])
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(M=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(L=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(L=3), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(L=128, K=128 * 64), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(R=3), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(R=16), gdn.GDN_ERR_UNSUPPORTED),   # more ranks than leaves
+    (dict(N=200), gdn.GDN_ERR_UNSUPPORTED),  # not a multiple of 16
+    (dict(K=1000), gdn.GDN_ERR_UNSUPPORTED),  # not a multiple of 64 L
+    (dict(A=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(err=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(C=MIS), gdn.GDN_ERR_INVALID_ARG),
+    (dict(err=MIS + 2), gdn.GDN_ERR_INVALID_ARG),
+    (dict(R=2, ws=None), gdn.GDN_ERR_WORKSPACE),   # L / R = 4 leaves per rank: two groups
+    (dict(L=16, wsb=16), gdn.GDN_ERR_WORKSPACE),
+])
+def test_pik_rejects_on_host(over, expect):
+    assert pik(**over) == expect
+
+
+def test_pik_workspace_and_empty_shapes():
+    w = gdn.pik_workspace_bytes
+    assert w(256, 256, 1024, 8, 1) == 0           # one group of 8 leaves: no workspace
+    assert w(256, 256, 1024, 16, 1) == 2 * 256 * 256 * 4
+    assert w(256, 256, 1024, 8, 8) == 8 * 256 * 256 * 4
+    assert w(256, 200, 1024, 8, 1) == 0 and w(256, 256, 1024, 3, 1) == 0
+    assert pik(M=0, A=None, B=None, C=None, err=None) == gdn.GDN_OK
+    assert pik(N=0, A=None, B=None, C=None, err=None) == gdn.GDN_OK
 
 
 def _state(**over):
