@@ -16,17 +16,24 @@
 // k; the epilogue reads the G accumulators back and adds them level by level
 // (neighbours 2i, 2i + 1).  A group is a node of the tree, so when L / G > 1
 // the group sums go to a workspace and k_pik_combine applies the levels
-// above them, again neighbours first.  The group size is min(L / R, 8) for R
+// above them, again neighbours first.  The group size is min(L / R, 2) for R
 // emulated ranks, and whatever it is, every addition of the tree happens in
 // the same order on the same operands: the result is the same for every R.
 //
 // Operands: A [M, K] and B [N, K] bf16, both K-major (row-major with K
-// innermost); C [M, N] fp32.  Tiles are staged through shared memory in the
-// no-swizzle core-matrix layout by cp.async (rows past M or N are zero),
-// four stages deep; an mbarrier per stage tells when the MMAs reading it are
-// done.  Waits are bounded: one that gives up sets GDN_DEVERR_TIMEOUT in the
-// error word, waits (bounded) for the MMAs in flight, frees tensor memory and
-// returns.
+// innermost); C [M, N] fp32.  Tiles reach shared memory by TMA in the
+// 128-byte swizzled K-major layout: one 2-D tensor copy per operand and stage
+// (64 K columns = 128 bytes per row, 8-row atoms of 1024 bytes, 16-byte
+// chunks permuted by the row's low three bits), which is also the MMA's
+// operand layout; a k16 step starts 32 bytes further along the row.  Rows
+// past M or N read as zero.  Roles: thread 0 issues the copies
+// of a stage once the MMAs that read it last have committed ("empty"
+// mbarrier), warp 1 issues a stage's four MMAs once its copies have landed
+// ("full" mbarrier, transaction bytes), and all four warps run the epilogue.
+// Four stages.  Waits are bounded: one that gives up sets GDN_DEVERR_TIMEOUT
+// in the error word, waits (bounded) for the copies and MMAs in flight, frees
+// tensor memory and returns.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -48,34 +55,29 @@ template <int BN>
 struct PikSmem {
   __nv_bfloat16 A[kPikStages][128 * kPikKStep];
   __nv_bfloat16 B[kPikStages][BN * kPikKStep];
-  uint64_t mbar[kPikStages];
+  uint64_t full[kPikStages];   // copies of the stage have landed
+  uint64_t empty[kPikStages];  // MMAs reading the stage are done
+  uint64_t done;               // every MMA is done
   uint32_t tmem_slot;
 };
 
-__device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),
-               "l"(gmem), "r"(valid ? 16 : 0));
+// 2-D tiled TMA load of one box into shared memory, completion counted on the
+// mbarrier in transaction bytes.  x (the K coordinate) is a multiple of 8
+// elements, so x * 2 bytes is a multiple of 16.
+__device__ __forceinline__ void tma_load_2d(uint32_t sdst, const CUtensorMap* map, int x, int y,
+                                            uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(sdst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(mbar)
+      : "memory");
 }
 
-// Stage the K step starting at k0: A rows m0 .. m0+127 and B rows n0 ..
-// n0+BN-1, 64 columns each, into the core-matrix layout.  Eight consecutive
-// threads read one row's 128 contiguous bytes.
-template <int BN>
-__device__ __forceinline__ void pik_stage(PikSmem<BN>& sm, int st, const __nv_bfloat16* A,
-                                          const __nv_bfloat16* B, int64_t M, int64_t N,
-                                          int64_t K, int64_t m0, int64_t n0, int64_t k0) {
-  for (int e = threadIdx.x; e < 128 * 8; e += kPikThreads) {
-    const int r = e >> 3, kg = e & 7;
-    const bool ok = m0 + r < M;
-    const __nv_bfloat16* src = ok ? A + (m0 + r) * K + k0 + kg * 8 : A;
-    cp_async16_zfill(&sm.A[st][core_off<128>(r, kg * 8)], src, ok);
-  }
-  for (int e = threadIdx.x; e < BN * 8; e += kPikThreads) {
-    const int r = e >> 3, kg = e & 7;
-    const bool ok = n0 + r < N;
-    const __nv_bfloat16* src = ok ? B + (n0 + r) * K + k0 + kg * 8 : B;
-    cp_async16_zfill(&sm.B[st][core_off<BN>(r, kg * 8)], src, ok);
-  }
+// Descriptor of a K-major operand in the 128-byte swizzled layout: 8-row
+// atoms 1024 bytes apart; the leading offset is unused within one 128-byte
+// row (encoded as 16 bytes); layout type 2 = 128-byte swizzle.
+__device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
+  return smem_desc(saddr, 16, 1024) | ((uint64_t)2 << 61);
 }
 
 template <int G>
@@ -92,14 +94,18 @@ __device__ __forceinline__ void tree16(float (&x)[G][16]) {
 // group); out is C (one group) or the group's slice of the workspace.
 template <int G, int BN>
 __global__ void __launch_bounds__(kPikThreads, 1)
-    k_pik_gemm(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B,
-               int64_t M, int64_t N, int64_t K, int64_t leaf_k, float* __restrict__ out,
-               int32_t* __restrict__ error) {
+    k_pik_gemm(const __grid_constant__ CUtensorMap map_a,
+               const __grid_constant__ CUtensorMap map_b, int64_t M, int64_t N,
+               int64_t leaf_k, float* __restrict__ out, int32_t* __restrict__ error) {
   constexpr int kCols = (G * BN < 32) ? 32 : G * BN;  // a power of two here
+  constexpr uint32_t kStageBytes = (128 + BN) * kPikKStep * 2;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  PikSmem<BN>& sm = *reinterpret_cast<PikSmem<BN>*>(smem_raw);
+  // The swizzled tiles need 1024-byte alignment: round the base up (the
+  // launch requests 1 KB more than the tiles need).
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  PikSmem<BN>& sm = *reinterpret_cast<PikSmem<BN>*>(smem_raw + pad);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t m0 = (int64_t)blockIdx.x * 128, n0 = (int64_t)blockIdx.y * BN;
+  const int m0 = (int)blockIdx.x * 128, n0 = (int)blockIdx.y * BN;
   const int64_t kbase = (int64_t)blockIdx.z * G * leaf_k;
   const int spl = (int)(leaf_k / kPikKStep);  // K steps per leaf
   const int S = G * spl;
@@ -107,7 +113,11 @@ __global__ void __launch_bounds__(kPikThreads, 1)
 
   if (warp == 0) tmem_alloc(smem_u32(&sm.tmem_slot), kCols);
   if (tid == 0) {
-    for (int i = 0; i < kPikStages; i++) mbar_init(smem_u32(&sm.mbar[i]), 1);
+    for (int i = 0; i < kPikStages; i++) {
+      mbar_init(smem_u32(&sm.full[i]), 1);
+      mbar_init(smem_u32(&sm.empty[i]), 1);
+    }
+    mbar_init(smem_u32(&sm.done), 1);
     fence_mbar_init();
   }
   tc_fence_before();
@@ -115,49 +125,51 @@ __global__ void __launch_bounds__(kPikThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_slot;
   constexpr uint32_t idesc = idesc_bf16(128, BN, false, false);
-
-  for (int p = 0; p < kPikStages - 1; p++) {
-    if (p < S) pik_stage<BN>(sm, p, A, B, M, N, K, m0, n0, kbase + (int64_t)p * kPikKStep);
-    cp_async_commit();
-  }
   bool ok = true;
-  for (int s = 0; s < S; s++) {
-    const int st = s % kPikStages;
-    cp_async_wait<kPikStages - 2>();  // this thread's copies of step s are in
-    fence_async_smem();
-    __syncthreads();                  // everyone's are, and visible to the tensor core
-    if (warp == 0) {
+  int issued = 0;  // steps whose copies thread 0 issued
+
+  if (tid == 0) {
+    // Producer: the copies of step s go to stage s % NS once the MMAs of step
+    // s - NS (the stage's previous use) have committed.
+    for (int s = 0; s < S; s++) {
+      const int st = s % kPikStages;
+      if (s >= kPikStages &&
+          !mbar_wait(smem_u32(&sm.empty[st]), (uint32_t)((s / kPikStages - 1) & 1), kPikPolls)) {
+        ok = false;
+        break;
+      }
+      const uint32_t fb = smem_u32(&sm.full[st]);
+      mbar_expect_tx(fb, kStageBytes);
+      const int k0 = (int)(kbase + (int64_t)s * kPikKStep);
+      const uint32_t a0 = smem_u32(sm.A[st]), b0 = smem_u32(sm.B[st]);
+      tma_load_2d(a0, &map_a, k0, m0, fb);
+      tma_load_2d(b0, &map_b, k0, n0, fb);
+      issued = s + 1;
+    }
+  } else if (warp == 1) {
+    // MMA issuer: a stage's four k16 MMAs once its copies have landed.
+    for (int s = 0; s < S; s++) {
+      const int st = s % kPikStages;
+      if (!mbar_wait(smem_u32(&sm.full[st]), (uint32_t)((s / kPikStages) & 1), kPikPolls)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const uint32_t a0 = smem_u32(sm.A[st]), b0 = smem_u32(sm.B[st]);
       const uint32_t d = tmem + (uint32_t)((s / spl) * BN);
 #pragma unroll
       for (int j = 0; j < kPikKStep / 16; j++)
-        umma_bf16(d, desc_kmajor<128>(a0 + j * 2 * 128 * 16), desc_kmajor<BN>(b0 + j * 2 * BN * 16),
-                  idesc, (s % spl != 0 || j > 0) ? 1u : 0u);
-      umma_commit(smem_u32(&sm.mbar[st]));
+        umma_bf16(d, desc_kmajor_sw128(a0 + j * 32), desc_kmajor_sw128(b0 + j * 32), idesc,
+                  (s % spl != 0 || j > 0) ? 1u : 0u);
+      umma_commit(smem_u32(&sm.empty[st]));
     }
-    const int sn = s + kPikStages - 1;  // refill the stage step s - 1 used
-    if (sn < S) {
-      if (s >= 1) {
-        const int sp = s - 1;
-        if (!mbar_wait(smem_u32(&sm.mbar[sp % kPikStages]), (uint32_t)((sp / kPikStages) & 1),
-                       kPikPolls))
-          ok = false;
-      }
-      pik_stage<BN>(sm, sn % kPikStages, A, B, M, N, K, m0, n0,
-                    kbase + (int64_t)sn * kPikKStep);
-    }
-    cp_async_commit();
+    umma_commit(smem_u32(&sm.done));  // every MMA issued so far
   }
-  // Every MMA is done once the last step's commit has arrived.
-  const int sl = S - 1;
-  const uint32_t last_bar = smem_u32(&sm.mbar[sl % kPikStages]);
-  const uint32_t last_par = (uint32_t)((sl / kPikStages) & 1);
-  if (!mbar_wait(last_bar, last_par, kPikPolls)) {
+  // Everyone: wait until every MMA is done (bounded).
+  if (!mbar_wait(smem_u32(&sm.done), 0u, kPikPolls)) {
     ok = false;
-    (void)mbar_wait(last_bar, last_par, kPikPolls);  // bounded drain before freeing
+    (void)mbar_wait(smem_u32(&sm.done), 0u, kPikPolls);  // bounded drain before freeing
   }
-  cp_async_wait<0>();
   tc_fence_after();
   const bool failed = __syncthreads_or(!ok);
   if (!failed) {
@@ -181,13 +193,23 @@ __global__ void __launch_bounds__(kPikThreads, 1)
     }
   } else if (tid == 0) {
     atomicOr(error, kPikErrTimeout);
+    // Copies still in flight land before the block's shared memory is freed:
+    // wait (bounded) for the last phase of every stage that was filled.
+    for (int s = issued - kPikStages < 0 ? 0 : issued - kPikStages; s < issued; s++)
+      (void)mbar_wait(smem_u32(&sm.full[s % kPikStages]), (uint32_t)((s / kPikStages) & 1),
+                      kPikPolls);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, kCols);
-  if (tid == 0)
-    for (int i = 0; i < kPikStages; i++) mbar_inval(smem_u32(&sm.mbar[i]));
+  if (tid == 0) {
+    for (int i = 0; i < kPikStages; i++) {
+      mbar_inval(smem_u32(&sm.full[i]));
+      mbar_inval(smem_u32(&sm.empty[i]));
+    }
+    mbar_inval(smem_u32(&sm.done));
+  }
 }
 
 // The levels above the groups: C = tree over n_groups group sums (a power of
@@ -222,11 +244,15 @@ struct PikPlan {
   size_t ws;          // workspace bytes (group sums when groups > 1)
 };
 
+// Group size: at most two leaves per block, so that every block runs the
+// widest tile (BN = 256) and the deeper levels go to k_pik_combine.  Deeper
+// in-memory trees (four or eight leaves, BN = 128 or 64) ran up to 3x slower at
+// the 8192^3 shape; the grouping never changes the bits.
 PikPlan pik_plan(int64_t M, int64_t N, int L, int R) {
   PikPlan p{};
   const int per_rank = L / R;  // leaves per emulated rank
-  p.G = per_rank < 8 ? per_rank : 8;
-  p.BN = p.G <= 2 ? 256 : 512 / p.G;
+  p.G = per_rank < 2 ? per_rank : 2;
+  p.BN = 256;
   p.groups = L / p.G;
   p.ws = p.groups > 1 ? (size_t)p.groups * (size_t)M * (size_t)N * sizeof(float) : 0;
   return p;
@@ -238,8 +264,44 @@ int validate(int64_t M, int64_t N, int64_t K, int L, int R) {
   if (M < 0 || N < 0 || K < 0 || L < 1 || R < 1) return GDN_ERR_INVALID_ARG;
   if (!pow2(L) || !pow2(R) || L % R != 0 || L > 64) return GDN_ERR_UNSUPPORTED;
   if (N % 16 != 0 || K % ((int64_t)kPikKStep * L) != 0) return GDN_ERR_UNSUPPORTED;
-  if (N / 64 > 65535 || (M + 127) / 128 > 0x7fffffff) return GDN_ERR_UNSUPPORTED;
+  // TMA coordinates are 32-bit: rows and K below 2^31.
+  if (N / 64 > 65535 || M >= 0x7fffffff || N >= 0x7fffffff || K >= 0x7fffffff)
+    return GDN_ERR_UNSUPPORTED;
   return GDN_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Map over a [rows, K] bf16 row-major matrix with a box of 64 K columns
+// (128 bytes) x box_rows rows, written to shared memory 128-byte swizzled.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kPikKStep, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Each block allocates all 512 tensor-memory columns of its SM (or 256 with
@@ -249,18 +311,20 @@ int validate(int64_t M, int64_t N, int64_t K, int L, int R) {
 constexpr size_t kPikMinSmem = 116 * 1024;
 
 template <int G, int BN>
-cudaError_t launch_gemm(const PikPlan& p, const __nv_bfloat16* A, const __nv_bfloat16* B,
-                        int64_t M, int64_t N, int64_t K, int64_t leaf_k, float* out,
-                        int32_t* error, cudaStream_t st) {
+int launch_gemm(const PikPlan& p, const void* A, const void* B, int64_t M, int64_t N, int64_t K,
+                int64_t leaf_k, float* out, int32_t* error, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, M, K, 128) || !make_map(&mb, B, N, K, BN)) return GDN_ERR_CUDA;
   auto kern = k_pik_gemm<G, BN>;
-  const size_t smem = sizeof(PikSmem<BN>) < kPikMinSmem ? kPikMinSmem : sizeof(PikSmem<BN>);
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  const size_t need = sizeof(PikSmem<BN>) + 1024;
+  const size_t smem = need < kPikMinSmem ? kPikMinSmem : need;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return GDN_ERR_CUDA;
   const dim3 grid((unsigned)((M + 127) / 128), (unsigned)((N + BN - 1) / BN),
                   (unsigned)p.groups);
-  kern<<<grid, kPikThreads, smem, st>>>(A, B, M, N, K, leaf_k, out, error);
-  return cudaGetLastError();
+  kern<<<grid, kPikThreads, smem, st>>>(ma, mb, M, N, leaf_k, out, error);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 }  // namespace
@@ -293,18 +357,14 @@ int gdn_pik_gemm(const void* A, const void* B, float* C, int64_t M, int64_t N, i
   if (p.ws > 0 && (!workspace || workspace_bytes < p.ws || !al16(workspace)))
     return GDN_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const auto* a = static_cast<const __nv_bfloat16*>(A);
-  const auto* b = static_cast<const __nv_bfloat16*>(B);
   float* out = p.groups > 1 ? static_cast<float*>(workspace) : C;
   const int64_t leaf_k = K / n_leaves;
-  cudaError_t e;
-  switch (p.G) {
-    case 1: e = gdn::launch_gemm<1, 256>(p, a, b, M, N, K, leaf_k, out, error_word, st); break;
-    case 2: e = gdn::launch_gemm<2, 256>(p, a, b, M, N, K, leaf_k, out, error_word, st); break;
-    case 4: e = gdn::launch_gemm<4, 128>(p, a, b, M, N, K, leaf_k, out, error_word, st); break;
-    default: e = gdn::launch_gemm<8, 64>(p, a, b, M, N, K, leaf_k, out, error_word, st); break;
-  }
-  if (e != cudaSuccess) return GDN_ERR_CUDA;
+  int r;
+  if (p.G == 1)
+    r = gdn::launch_gemm<1, 256>(p, A, B, M, N, K, leaf_k, out, error_word, st);
+  else
+    r = gdn::launch_gemm<2, 256>(p, A, B, M, N, K, leaf_k, out, error_word, st);
+  if (r != GDN_OK) return r;
   if (p.groups > 1) {
     const int64_t MN = M * N, threads = 256, items = MN / 4;
     gdn::k_pik_combine<<<(unsigned)((items + threads - 1) / threads), (unsigned)threads, 0, st>>>(

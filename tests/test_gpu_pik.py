@@ -51,7 +51,8 @@ def test_matches_the_product_within_the_float32_bound(gdn, L):
 
 
 def test_same_bits_for_every_rank_count(gdn):
-    """L = 16 leaves: 1, 2, 4, 8 and 16 emulated ranks (group sizes 8, 8, 4, 2, 1)."""
+    """L = 16 leaves: 1, 2, 4, 8 and 16 emulated ranks (blocks of 2 leaves with 8 group
+    sums combined, down to blocks of 1 leaf with 16)."""
     M, N, K = 256, 320, 16 * 128
     A, B = operands(M, N, K, 50)
     A, B = A.cuda(), B.cuda()
