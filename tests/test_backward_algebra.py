@@ -1,0 +1,100 @@
+"""The algebra of the CUDA backward, checked in float64 against the oracle (CPU).
+
+gdn_cpr_backward does not run the reverse token loop that oracle.backward
+runs.  It splits the gradient into (i) an adjoint recurrence per state row,
+mu_{t-1} = alpha_t (Lambda_t - beta_t w_t k_t^T), (ii) per-chunk recomputed
+states, (iii) dg as a telescoped sum Z_{t-1} = Z_t + do_t.o_t - beta_t v_t.w_t
+and (iv) dq, dk of a chunk as products of C x C and C x d matrices
+(Y = DO U^T, X = W U^T, A, B).  This test writes that schedule out in float64
+numpy and requires it to equal the oracle's reverse mode to 1e-12 on ragged
+batches with chunk sizes that leave partial chunks, so the identities the
+kernels rely on are exact, independently of the GPU.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def _batch(lens, H, d, seed):
+    rng = np.random.default_rng(seed)
+    T = sum(lens)
+    q = rng.normal(size=(T, H, d))
+    k = rng.normal(size=(T, H, d))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.normal(size=(T, H, d))
+    beta = 1.0 / (1.0 + np.exp(-rng.normal(size=(T, H))))
+    g = -np.log1p(np.exp(rng.normal(size=(T, H))))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    h0 = rng.normal(size=(len(lens), H, d, d))
+    do = rng.normal(size=(T, H, d))
+    dsf = rng.normal(size=h0.shape)
+    return q, k, v, beta, g, cu, h0, do, dsf
+
+
+def chunked_backward(q, k, v, beta, g, cu, do, h0, dsf, scale, C):
+    T, H, d = q.shape
+    out = {n: np.zeros_like(x) for n, x in
+           [("dq", q), ("dk", k), ("dv", v), ("dbeta", beta), ("dg", g), ("dh0", h0)]}
+    for n in range(len(cu) - 1):
+        a0, e0 = int(cu[n]), int(cu[n + 1])
+        for h in range(H):
+            # boundary states S_a at every chunk start (the forward's first pass)
+            S, Sb = h0[n, h].copy(), {}
+            for j in range(a0, e0):
+                if (j - a0) % C == 0:
+                    Sb[j] = S.copy()
+                al = np.exp(g[j, h])
+                S = al * S + np.outer(beta[j, h] * (v[j, h] - al * (S @ k[j, h])), k[j, h])
+            # (i) adjoint recurrence, last token first: w per token, mu at chunk ends
+            mu, W, mu_end = dsf[n, h].copy(), np.zeros((e0 - a0, d)), {}
+            for j in range(e0 - 1, a0 - 1, -1):
+                if (j - a0) % C == C - 1 or j == e0 - 1:
+                    mu_end[j + 1] = mu.copy()
+                lam = mu + scale * np.outer(do[j, h], q[j, h])
+                W[j - a0] = lam @ k[j, h]
+                mu = np.exp(g[j, h]) * (lam - beta[j, h] * np.outer(W[j - a0], k[j, h]))
+            out["dh0"][n, h] = mu
+            out["dv"][a0:e0, h] = beta[a0:e0, h, None] * W
+            for a in range(a0, e0, C):
+                e = min(a + C, e0)
+                L = e - a
+                # (ii) the chunk's states recomputed from S_a: p, u, o per token
+                S = Sb[a].copy()
+                P, U, O = np.zeros((L, d)), np.zeros((L, d)), np.zeros((L, d))
+                for j in range(a, e):
+                    al = np.exp(g[j, h])
+                    P[j - a] = S @ k[j, h]
+                    U[j - a] = beta[j, h] * (v[j, h] - al * P[j - a])
+                    S = al * S + np.outer(U[j - a], k[j, h])
+                    O[j - a] = scale * S @ q[j, h]
+                Wc, al, bt = W[a - a0:e - a0], np.exp(g[a:e, h]), beta[a:e, h]
+                out["dbeta"][a:e, h] = np.sum(Wc * (v[a:e, h] - al[:, None] * P), 1)
+                # (iii) dg_t = Z_{t-1}, telescoped from Z at the chunk's end
+                Z = np.sum(mu_end[e] * S)
+                for j in range(e - 1, a - 1, -1):
+                    Z = Z + do[j, h] @ O[j - a] - bt[j - a] * (v[j, h] @ Wc[j - a])
+                    out["dg"][j, h] = Z
+                # (iv) dq, dk from the chunk products
+                G = np.cumsum(g[a:e, h])
+                DO, Q, K = do[a:e, h], q[a:e, h], k[a:e, h]
+                ii = np.arange(L)
+                dec = np.exp(G[:, None] - G[None, :])
+                A = np.where(ii[:, None] >= ii[None, :], dec, 0.0) * (DO @ U.T)
+                B = np.where(ii[:, None] > ii[None, :], dec, 0.0) * (Wc @ U.T) * bt[:, None]
+                out["dq"][a:e, h] = scale * (np.exp(G)[:, None] * (DO @ Sb[a]) + A @ K)
+                out["dk"][a:e, h] = (scale * A.T @ Q - (B + B.T) @ K
+                                     - (bt * np.exp(G))[:, None] * (Wc @ Sb[a])
+                                     + np.exp(G[-1] - G)[:, None] * (U @ mu_end[e]))
+    return out
+
+
+@pytest.mark.parametrize("C", [1, 3, 16, 64])
+def test_chunked_schedule_equals_the_oracles_reverse_mode(C):
+    q, k, v, beta, g, cu, h0, do, dsf = _batch([1, 63, 64, 65, 130, 0, 7], 2, 6, seed=C)
+    scale = 0.6
+    ref = oracle.backward(q, k, v, beta, g, cu, do, h0=h0, ds_final=dsf, scale=scale, threads=1)
+    got = chunked_backward(q, k, v, beta, g, cu, do, h0, dsf, scale, C)
+    for name in ref:
+        err = np.max(np.abs(got[name] - ref[name])) / max(1.0, np.max(np.abs(ref[name])))
+        assert err < 1e-12, (name, C, err)
