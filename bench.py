@@ -85,7 +85,7 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------------------
-# Algorithmic work (stated per unit)
+# Algorithmic work, per unit of each measured kernel
 # ----------------------------------------------------------------------------
 
 def fill_flops(T, H_, d):
