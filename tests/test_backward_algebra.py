@@ -98,3 +98,44 @@ def test_chunked_schedule_equals_the_oracles_reverse_mode(C):
     for name in ref:
         err = np.max(np.abs(got[name] - ref[name])) / max(1.0, np.max(np.abs(ref[name])))
         assert err < 1e-12, (name, C, err)
+
+
+def test_adjoint_chunk_map_is_the_transposed_boundary_map():
+    """The adjoint crosses a chunk as mu_a = mu_e P^T + W_loc, where P is the
+    chunk's state transition (S_end = S_a P with v = 0), W_loc the adjoint the
+    chunk's own outputs produce from mu_e = 0, and P^T has the closed form
+    e^{G_n} I - K^T diag(e^{G_n - G}) T diag(beta e^G) K in the quantities of
+    the forward's boundary computation (T = (I + A)^{-1}).  So a reverse walk
+    over chunk boundaries can run on the forward's boundary data."""
+    rng = np.random.default_rng(5)
+    n, d, scale = 13, 5, 0.7
+    K = rng.normal(size=(n, d))
+    K /= np.linalg.norm(K, axis=1, keepdims=True)
+    Q = rng.normal(size=(n, d))
+    beta = 1.0 / (1.0 + np.exp(-rng.normal(size=n)))
+    g = -np.log1p(np.exp(rng.normal(size=n)))
+    DO = rng.normal(size=(n, d))
+    cb = oracle.chunk_boundary(np.zeros((d, d)), K, np.zeros((n, d)), beta, g)
+    T, G = cb["T"], cb["G"]
+    # P from the token loop: S -> S F_1 ... F_n with F_t = a_t (I - b_t k_t k_t^T)
+    P = np.eye(d)
+    for t in range(n):
+        P = P @ (np.exp(g[t]) * (np.eye(d) - beta[t] * np.outer(K[t], K[t])))
+    S0 = rng.normal(size=(d, d))
+    assert np.allclose(S0 @ P, oracle.chunk_boundary(S0, K, np.zeros((n, d)), beta, g)["S"],
+                       rtol=0, atol=1e-12)
+    Pt = (np.exp(G[-1]) * np.eye(d)
+          - K.T @ (np.exp(G[-1] - G)[:, None] * T * (beta * np.exp(G))[None, :]) @ K)
+    assert np.allclose(Pt, P.T, rtol=0, atol=1e-12)
+
+    def adjoint(mu_e):
+        mu = mu_e.copy()
+        for t in range(n - 1, -1, -1):
+            lam = mu + scale * np.outer(DO[t], Q[t])
+            w = lam @ K[t]
+            mu = np.exp(g[t]) * (lam - beta[t] * np.outer(w, K[t]))
+        return mu
+
+    mu_e = rng.normal(size=(d, d))
+    W_loc = adjoint(np.zeros((d, d)))
+    assert np.allclose(adjoint(mu_e), mu_e @ Pt + W_loc, rtol=0, atol=1e-12)
