@@ -453,13 +453,30 @@ def run_train_part(gdn, W, dev, rank, world, args, flush, peaks):
             "bwd_adjoint_scan": el(6, 7), "bwd_chunk_rows": el(7, 8),
             "bwd_chunk_products": el(8, 9)}
     ms = max_over_ranks(fwd + bwd, world)
+    fwd_max = max_over_ranks(fwd, world)
     fp32_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
     gflop = bwd_gemm_flops(b.lengths, H, D) / 1e9
     achieved = gflop / kern["bwd_chunk_products"]  # GFLOP per ms = TFLOP/s
+    # The trainer forward on its own: the fill's FP32 roofline and the whole
+    # forward's HBM fraction on the minimal and two-pass byte counts.
+    fill_tf = fill_flops(T, H, D) / 1e9 / kern["fwd_intra_chunk_fill"]
+    minimal, two_pass = prefill_bytes(b.lengths, H, D)
+    hbm_bps = peaks["hbm_gbs"] * 1e9
     return {"workload": f"trainer: {T} tokens as {N} documents (lengths {b.lengths}), H={H}, "
                         f"d_k=d_v={D}, C={C}, bf16 q/k/v/do, fp32 beta/g/state/gradients",
             "steps": steps, "ms_per_step": round(ms, 5), "fwd_ms": round(fwd, 5),
             "bwd_ms": round(bwd, 5), "tokens_per_s": round(world * T / (ms / 1e3), 1),
+            "fwd_tokens_per_s": round(world * T / (fwd_max / 1e3), 1),
+            "fwd_roofline": {"kernel": "fwd_intra_chunk_fill", "bound": "alu",
+                             "achieved": round(fill_tf, 2), "peak": round(fp32_peak, 2),
+                             "unit": "TFLOP/s", "frac": round(fill_tf / fp32_peak, 4),
+                             "traffic": ncu_traffic("trainer_intra_chunk_fill"),
+                             "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x sm_max_mhz "
+                                            "(nominal)"},
+            "fwd_hbm_roofline": {"minimal_bytes": minimal, "two_pass_bytes": two_pass,
+                                 "frac_minimal": round(minimal / (fwd_max / 1e3) / hbm_bps, 4),
+                                 "frac_two_pass": round(two_pass / (fwd_max / 1e3) / hbm_bps, 4),
+                                 "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]},
             "kernels_ms": {k: round(v, 5) for k, v in kern.items()},
             "bwd_roofline": {"kernel": "bwd_chunk_products", "bound": "alu",
                              "achieved": round(achieved, 2), "peak": round(fp32_peak, 2),
@@ -524,25 +541,67 @@ def run_pik_part(gdn, dev, rank, world, args, flush, peaks):
             "l2": "flushed (256 MiB write) before every timed call"}
 
 
-def cpu_baseline_sample(W, seconds=10.0):
-    """The fp64 oracle as it stands, all host cores, on whole sequences of the
-    prefill batch until about `seconds` of CPU work has been done."""
+def _oracle_prefill_passes(oracle, b, seconds, threads=None, max_passes=64):
+    """Whole-batch oracle passes over `b` (every sequence and head) until about
+    `seconds` have gone by; returns (tokens, passes, elapsed s)."""
+    done, passes, t0 = 0, 0, time.perf_counter()
+    while passes < max_passes and (passes == 0 or time.perf_counter() - t0 < seconds):
+        oracle.forward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens.numpy(), threads=threads)
+        done += b.total_tokens
+        passes += 1
+    return done, passes, time.perf_counter() - t0
+
+
+def cpu_baseline_sample(W, seconds=8.0):
+    """The fp64 oracle as it stands on the host cores.  The headline figure:
+    all cores, whole passes over the 5x2048 prefill batch (all 80 sequence-head
+    units, the GPU arm's workload).  Beside it: one core on whole sequence-head
+    units of the same batch, the 10240-token trainer forward on all cores, and
+    the 256-row decode step (one token per row and head, the state carried as
+    h0) on all cores."""
     import oracle
     b = W.prefill(device="cpu", seed=0)
+    done, passes, el = _oracle_prefill_passes(oracle, b, seconds)
+    out = {"value": round(done / el, 1), "unit": "tokens/s", "cores": oracle.max_threads(),
+           "kind": "oracle",
+           "sample": f"{passes} pass(es) over the whole 5x2048 prefill batch, {H} heads "
+                     f"({done} tokens), fp64 token loop, {el:.1f} s"}
+    # one core: whole (sequence, head) units, counted as token-heads / H
     cu = b.cu_seqlens.tolist()
-    done, passes, t0 = 0, 0, time.perf_counter()
-    while time.perf_counter() - t0 < seconds and passes < 64:
-        for n in range(len(b.lengths)):
-            sl = slice(cu[n], cu[n + 1])
-            oracle.forward(b.q[sl], b.k[sl], b.v[sl], b.beta[sl], b.g[sl],
-                           np.array([0, cu[n + 1] - cu[n]], np.int32))
-            done += cu[n + 1] - cu[n]
-        passes += 1
-    el = time.perf_counter() - t0
-    return {"value": round(done / el, 1), "unit": "tokens/s", "cores": oracle.max_threads(),
-            "kind": "oracle",
-            "sample": f"{passes} pass(es) over the whole 5x2048 prefill batch, {H} heads "
-                      f"({done} tokens), fp64 token loop, {el:.1f} s"}
+    units, th, t0 = 0, 0, time.perf_counter()
+    while units < 2 * H and (units == 0 or time.perf_counter() - t0 < 3.0):
+        n, h = units % len(b.lengths), (units // len(b.lengths)) % H
+        sl, hs = slice(cu[n], cu[n + 1]), slice(h, h + 1)
+        oracle.forward(b.q[sl, hs], b.k[sl, hs], b.v[sl, hs], b.beta[sl, hs], b.g[sl, hs],
+                       np.array([0, cu[n + 1] - cu[n]], np.int32), threads=1)
+        th += cu[n + 1] - cu[n]
+        units += 1
+    el1 = time.perf_counter() - t0
+    out["one_core"] = {"value": round(th / H / el1, 1), "unit": "tokens/s", "cores": 1,
+                       "sample": f"{units} (sequence, head) units of the prefill batch "
+                                 f"({th} token-heads = {th / H:.0f} tokens), {el1:.1f} s"}
+    # trainer forward, all cores
+    bt = W.trainer(device="cpu", seed=0)
+    done, passes, el = _oracle_prefill_passes(oracle, bt, 3.0, max_passes=8)
+    out["trainer_forward"] = {"value": round(done / el, 1), "unit": "tokens/s",
+                              "cores": oracle.max_threads(),
+                              "sample": f"{passes} pass(es) over the 10240-token trainer batch "
+                                        f"(5 documents, {H} heads), {el:.1f} s"}
+    # decode: 256 rows x 1 token per step, fp64 state carried between steps
+    slots = 256
+    toks = W.decode_tokens(32, slots, H, D, D, seed=2, device="cpu")
+    S = np.zeros((slots, H, D, D))
+    cu1 = np.arange(slots + 1, dtype=np.int32)
+    steps, t0 = 0, time.perf_counter()
+    while steps < 32 and (steps == 0 or time.perf_counter() - t0 < 3.0):
+        _, S = oracle.forward(*(t[steps] for t in toks), cu1, h0=S)
+        steps += 1
+    eld = time.perf_counter() - t0
+    out["decode"] = {"value": round(steps * slots / eld, 1), "unit": "tokens/s",
+                     "cores": oracle.max_threads(),
+                     "sample": f"{steps} decode step(s) of {slots} rows x {H} heads from a "
+                               f"zero state (one fp64 token-loop step per row), {eld:.1f} s"}
+    return out
 
 
 def run_ours(args):
@@ -681,6 +740,9 @@ def run_ours(args):
 # ----------------------------------------------------------------------------
 
 def run_reference(args):
+    """The fp64 oracle as it stands, on the host cores, over the GPU arm's
+    workload: each step is one whole pass over the 5x2048 prefill batch (every
+    sequence and head)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -688,32 +750,26 @@ def run_reference(args):
     import oracle
     from rl_train_numerics_b200 import workloads as W
     b = W.prefill(device="cpu", seed=0)
-    cu = b.cu_seqlens.tolist()
-    heads = 4  # each step: one 2048-token sequence x 4 heads (a bounded sample)
+    cu = b.cu_seqlens.numpy()
 
-    def one(i):
-        n = i % len(b.lengths)
-        sl = slice(cu[n], cu[n + 1])
-        hs = slice((i * heads) % H, (i * heads) % H + heads)
-        oracle.forward(b.q[sl, hs], b.k[sl, hs], b.v[sl, hs], b.beta[sl, hs], b.g[sl, hs],
-                       np.array([0, cu[n + 1] - cu[n]], np.int32))
+    def one():
+        oracle.forward(b.q, b.k, b.v, b.beta, b.g, cu)
 
-    for i in range(args.warmup):
-        one(i)
+    for _ in range(args.warmup):
+        one()
     t0 = time.perf_counter()
-    for i in range(args.steps):
-        one(i)
+    for _ in range(args.steps):
+        one()
     el = time.perf_counter() - t0
-    tokens = args.steps * 2048 * heads / H  # whole-layer tokens (all H heads) equivalent
-    value = tokens / el
-    sample = (f"each step: one 2048-token sequence x {heads} of {H} heads of the 5x2048 "
-              "prefill batch (fp64 token loop); tokens counted as token-heads / 16")
+    value = args.steps * b.total_tokens / el
+    sample = (f"each step: one whole pass over the 5x2048 prefill batch, all {H} heads "
+              f"({b.total_tokens} tokens, fp64 token loop)")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "rollout prefill: 5 sequences x 2048 tokens packed, H=16, "
-                                   "d_k=d_v=128, C=64, bf16 q/k/v, fp32 beta/g",
+                                   "d_k=d_v=128, C=64, bf16 q/k/v/o, fp32 beta/g/state",
                        "global_batch": 10240, "seq_len": 2048, "parallelism": "host"},
             "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
                              "cores": oracle.max_threads(), "kind": "oracle", "sample": sample},

@@ -3,12 +3,14 @@
  *
  * The layer: "NovaSky's IsoExec Fixes the Hidden Math Bug Corrupting AI
  * Training Runs", section "Solving the linear-attention headache".  Gated
- * DeltaNet is evaluated by CPR (chunkwise-parallel recurrent): the
- * recurrence stays the primary algorithm, a first pass computes the state at
- * chunk boundaries, a second pass fills in the outputs inside every chunk in
- * parallel, and decode runs the recurrence but re-synchronises its state
- * every chunk-size tokens, so that training, prefill and decode share one
- * rounding schedule.  The recurrence (one state per sequence and head):
+ * DeltaNet is evaluated by CPR (chunkwise-parallel recurrent).  The token
+ * recurrence is what gets computed; the chunks only organise the work.  A
+ * serial sweep over chunk starts produces the state that enters each chunk;
+ * then every chunk replays the token recurrence from its entry state, all
+ * chunks at once.  Decode steps the same recurrence one token at a time and,
+ * whenever a chunk's worth of tokens has gone by, replaces its state by the
+ * one the chunk-start computation gives.  Training, prefill and decode thus
+ * round identically.  The recurrence (one state per sequence and head):
  *
  *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
  *     o_t = scale * S_t q_t,        alpha_t = exp(g_t)
@@ -159,9 +161,14 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
  * - Every call shares the array, so calls that can overlap on the GPU race;
  *   order them (one stream, or events).  Each call clears the array's error
  *   word before its kernels run.
- * - error_word: optional caller-owned device int32; when not NULL it
- *   receives the call's device error bits (GDN_DEVERR_*), readable with
- *   gdn_check_error(error_word, ...).
+ * - error_word: optional caller-owned device int32 (4-byte aligned); when
+ *   not NULL it receives the call's device error bits (GDN_DEVERR_*),
+ *   readable with gdn_check_error(error_word, ...).  An empty batch sets it to
+ *   zero.  Argument errors are returned before any device work, as for
+ *   gdn_cpr_forward.
+ * - The array's device address is cached per device for the process; after
+ *   cudaDeviceReset (or any other teardown of the device's primary context)
+ *   the cache is stale, so this entry point must not be called again.
  */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 int gdn_cpr_forward_noalloc(const void* q, const void* k, const void* v, int in_dtype,

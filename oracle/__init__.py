@@ -9,12 +9,12 @@ What the layer computes
 -----------------------
 "NovaSky's IsoExec Fixes the Hidden Math Bug Corrupting AI Training Runs",
 section "Solving the linear-attention headache": Gated DeltaNet is evaluated
-by CPR (chunkwise-parallel recurrent).  The recurrence stays the primary
-algorithm; a first pass produces the state at chunk boundaries, a second pass
-fills in the outputs inside every chunk, and decode runs the recurrence while
-re-synchronising its state every chunk-size tokens.  The same section states
-that the chunkwise and recurrent forms are mathematically identical, so the
-oracle for every output is the plain recurrence
+by CPR (chunkwise-parallel recurrent): the token recurrence defines the
+result, a serial sweep gives the state entering each chunk, the chunks then
+replay the recurrence from those states, and decode swaps its running state
+for the chunk-start computation after each chunk's worth of tokens.  The
+section also says that the chunked and the token-by-token forms agree in
+exact arithmetic, so the oracle for every output is the plain recurrence
 
     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
     o_t = scale * S_t q_t,          alpha_t = exp(g_t),

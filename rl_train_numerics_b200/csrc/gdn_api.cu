@@ -64,18 +64,23 @@ int gdn_cpr_forward(const void* q, const void* k, const void* v, int in_dtype, c
                             workspace, workspace_bytes, nullptr, stream);
 }
 
-int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype,
-                       const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
-                       int64_t total_tokens, int H, int dk, int dv, int C, float scale,
-                       const float* h0, void* o, int out_dtype, float* s_run_final,
-                       float* s_run_scale, float* s_bnd_final, void* workspace,
-                       size_t workspace_bytes, void* const* kernel_events, void* stream) {
+}  // extern "C"
+
+// Every host-side check of a forward call except the workspace's: returns
+// GDN_OK, an error status, or kFwdEmpty for a valid empty batch (nothing
+// to launch).
+int gdn::forward_check_args(const void* q, const void* k, const void* v, int in_dtype,
+                            const float* beta, const float* g, const int32_t* cu_seqlens,
+                            int n_seqs, int64_t total_tokens, int H, int dk, int dv, int C,
+                            float scale, const float* h0, const void* o, int out_dtype,
+                            const float* s_run_final, const float* s_run_scale,
+                            const float* s_bnd_final) {
   if (n_seqs < 0 || total_tokens < 0 || !valid_dtype(out_dtype) || !isfinite(scale))
     return GDN_ERR_INVALID_ARG;
   int rc = check_shape(H, dk, dv, C, in_dtype);
   if (rc != GDN_OK) return rc;
   if (total_tokens > INT32_MAX) return GDN_ERR_UNSUPPORTED;
-  if (n_seqs == 0) return total_tokens == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+  if (n_seqs == 0) return total_tokens == 0 ? kFwdEmpty : GDN_ERR_INVALID_ARG;
   if (!cu_seqlens || !aligned4(cu_seqlens)) return GDN_ERR_INVALID_ARG;
   if (total_tokens > 0) {
     if (!q || !k || !v || !beta || !g || !o) return GDN_ERR_INVALID_ARG;
@@ -86,6 +91,22 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
       (s_bnd_final && !aligned16(s_bnd_final)) || (s_run_scale && !aligned4(s_run_scale)))
     return GDN_ERR_INVALID_ARG;
   if (s_run_scale && !s_run_final) return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+extern "C" {
+
+int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype,
+                       const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
+                       int64_t total_tokens, int H, int dk, int dv, int C, float scale,
+                       const float* h0, void* o, int out_dtype, float* s_run_final,
+                       float* s_run_scale, float* s_bnd_final, void* workspace,
+                       size_t workspace_bytes, void* const* kernel_events, void* stream) {
+  const int rc = gdn::forward_check_args(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs,
+                                         total_tokens, H, dk, dv, C, scale, h0, o, out_dtype,
+                                         s_run_final, s_run_scale, s_bnd_final);
+  if (rc == gdn::kFwdEmpty) return GDN_OK;
+  if (rc != GDN_OK) return rc;
   const gdn::FwdLayout lay =
       gdn::fwd_layout(n_seqs, total_tokens, H, dk, dv, C, in_dtype == GDN_BF16);
   if (!workspace || workspace_bytes < lay.total) return GDN_ERR_WORKSPACE;

@@ -2,9 +2,10 @@
 // decode resync), on tensor cores.
 //
 // "NovaSky's IsoExec Fixes the Hidden Math Bug Corrupting AI Training Runs",
-// section "Solving the linear-attention headache": a first pass computes the
-// recurrent state at chunk boundaries; decode re-synchronises its state every
-// chunk-size tokens with the same computation.  The pages do not write the
+// section "Solving the linear-attention headache": CPR's serial sweep yields
+// the state entering every chunk, and decode, after each chunk's worth of
+// tokens, swaps its state for the result of that same computation.  The pages
+// do not write the
 // boundary formula; it is derived here from the recurrence
 // S_i = alpha_i S_{i-1} (I - beta_i k_i k_i^T) + beta_i v_i k_i^T
 // (the UT / WY form of a product of generalised Householder updates):

@@ -182,6 +182,15 @@ struct BwdArgs {
 };
 
 cudaError_t launch_forward(const FwdArgs& a, cudaStream_t stream);
+
+// Host-side argument checks of gdn_cpr_forward (all but the workspace);
+// kFwdEmpty marks a valid call with nothing to launch.
+constexpr int kFwdEmpty = 1;
+int forward_check_args(const void* q, const void* k, const void* v, int in_dtype,
+                       const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
+                       int64_t total_tokens, int H, int dk, int dv, int C, float scale,
+                       const float* h0, const void* o, int out_dtype, const float* s_run_final,
+                       const float* s_run_scale, const float* s_bnd_final);
 cudaError_t launch_backward(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_step(const DecArgs& a, cudaStream_t stream);
 cudaError_t launch_handoff(const HandoffArgs& a, cudaStream_t stream);

@@ -16,7 +16,10 @@
 // only a host-side stand-in, not a device address, so the device address is
 // looked up once per device with cudaGetSymbolAddress (with that device
 // current) and cached; that set-up happens in the first call on each device,
-// which should therefore come before any stream capture.
+// which should therefore come before any stream capture.  The cached address
+// belongs to the device's primary context: after cudaDeviceReset (or anything
+// else that destroys that context) the cache is stale and this entry point
+// must not be called again in the process.
 //
 // Every call shares the one array per device and leaves its contents behind
 // for the next call.  The forward writes every part of the scratch it reads
@@ -29,6 +32,7 @@
 #include <mutex>
 
 #include "../../include/gdn_cpr.h"
+#include "gdn_layout.h"
 
 namespace {
 
@@ -64,20 +68,27 @@ extern "C" int gdn_cpr_forward_noalloc(const void* q, const void* k, const void*
                                        float* s_run_final, float* s_run_scale,
                                        float* s_bnd_final, int32_t* error_word,
                                        void* stream) {
+  // Every argument check comes before any device work.
+  const int chk = gdn::forward_check_args(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs,
+                                          total_tokens, H, dk, dv, C, scale, h0, o, out_dtype,
+                                          s_run_final, s_run_scale, s_bnd_final);
+  if (chk != GDN_OK && chk != gdn::kFwdEmpty) return chk;
+  if (error_word && (reinterpret_cast<uintptr_t>(error_word) & 3u) != 0)
+    return GDN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (chk == gdn::kFwdEmpty) {
+    // An empty batch launches nothing; the caller's error word still reports
+    // this call (no error) rather than keeping an earlier call's bits.
+    if (error_word && cudaMemsetAsync(error_word, 0, sizeof(int32_t), st) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    return GDN_OK;
+  }
   const size_t need = gdn_cpr_forward_workspace_bytes(n_seqs, total_tokens, H, dk, dv, C,
                                                       in_dtype);
-  if (need == 0 || n_seqs == 0) {
-    // Rejected shapes, or an empty batch: the regular entry point reports the
-    // exact status (or returns GDN_OK for an empty batch) without device work.
-    return gdn_cpr_forward_ex(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs, total_tokens, H,
-                              dk, dv, C, scale, h0, o, out_dtype, s_run_final, s_run_scale,
-                              s_bnd_final, nullptr, 0, nullptr, stream);
-  }
-  if (need > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;  // beyond the fixed scratch
+  if (need == 0 || need > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
   void* scratch = nullptr;
   int rc = scratch_on_current_device(&scratch);
   if (rc != GDN_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(scratch, 0, sizeof(int32_t), st) != cudaSuccess) return GDN_ERR_CUDA;
   rc = gdn_cpr_forward_ex(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs, total_tokens, H, dk,
                           dv, C, scale, h0, o, out_dtype, s_run_final, s_run_scale, s_bnd_final,

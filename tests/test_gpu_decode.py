@@ -121,6 +121,58 @@ def test_prefill_plus_decode_equals_trainer_forward(gdn):
             assert rel_err(o_dec[:, n, h], o_ref[P:P + n_steps]) <= 2e-3
 
 
+def effective_running_state(st):
+    """The decode state's running state as a (mantissa, scale) pair: after a
+    resync (pos == 0) it is the boundary state with scale 1."""
+    at_bnd = (st.pos == 0)
+    mant = torch.where(at_bnd[..., None, None], st.s_bnd, st.s_run)
+    scale = torch.where(at_bnd, torch.ones_like(st.s_scale), st.s_scale)
+    return mant, scale
+
+
+def test_trainer_config_prefill_plus_decode_equals_forward(gdn):
+    """The trainer-forward workload at its stated shape: 10240 tokens as 5
+    documents (Dirichlet lengths, seed 3), H=16, d=128, bf16.  Each document is
+    split at a seeded point; its prefix is prefilled and the rest decoded token
+    by token to the document's end (rows leave the decode batch as their
+    documents end).  Prefill outputs followed by decode outputs equal one
+    forward over all 10240 tokens bit for bit, and so do both final states."""
+    full = W.trainer(device="cuda")
+    lens = full.lengths
+    assert sum(lens) == 10240 and len(lens) == 5 and full.q.shape[1:] == (16, 128)
+    gen = torch.Generator().manual_seed(26)
+    prefix = [int(torch.randint(1, L - 2 * C + 1, (1,), generator=gen)) for L in lens]
+    rest = [L - P for L, P in zip(lens, prefix)]
+    assert min(rest) >= 2 * C  # every document crosses at least two resyncs in decode
+
+    fscale = torch.empty((5, 16), device="cuda")
+    o_all, srun_all, sbnd_all = forward(gdn, full, out_dtype=torch.float32, s_run_scale=fscale)
+
+    pre = split_batch(full, prefix)
+    o_pre, srun, sscale, sbnd = prefill_pair(gdn, pre)
+    st = gdn.DecodeState(5, 16, 128, 128)
+    gdn.decode_state_from_prefill(st, pre.k, pre.v, pre.beta, pre.g, pre.cu_seqlens, srun, sbnd,
+                                  s_run_scale=sscale)
+    cu = full.cu_seqlens.tolist()
+    o_cat = torch.full_like(o_all, float("nan"))
+    cp = pre.cu_seqlens.tolist()
+    for n, P in enumerate(prefix):
+        o_cat[cu[n]:cu[n] + P] = o_pre[cp[n]:cp[n + 1]]
+    for s in range(max(rest)):
+        live = [n for n in range(5) if s < rest[n]]
+        rows = torch.tensor([cu[n] + prefix[n] + s for n in live], device="cuda")
+        slots = torch.tensor(live, dtype=torch.int32, device="cuda")
+        o = gdn.decode_step(st, full.q[rows].contiguous(), full.k[rows].contiguous(),
+                            full.v[rows].contiguous(), full.beta[rows].contiguous(),
+                            full.g[rows].contiguous(), slot_idx=slots, out_dtype=torch.float32)
+        o_cat[rows] = o
+    assert gdn.check_error(st.error) == 0
+    assert torch.equal(o_cat, o_all)
+    mant, scale = effective_running_state(st)
+    assert torch.equal(mant, srun_all) and torch.equal(scale, fscale)
+    assert torch.equal(st.s_bnd, sbnd_all)
+
+
 def test_rollout_decode_shape_sampled(gdn):
     """256 slots, prefix lengths uniform in [1, 2047], H=16, d=128, bf16, 512 steps."""
     prefix = W.decode_prefix_lengths(256)

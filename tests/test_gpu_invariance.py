@@ -87,18 +87,31 @@ def test_stress_parity_sampled(gdn, stress):
 
 
 def test_decode_batch_invariance(gdn, stress):
+    """128 decode steps continued from each forward mode's own handoff (whole
+    batch, shuffled batch, one sequence at a time, padded between empty
+    sequences), each with that mode's running-state pair and boundary state:
+    every slot's decode outputs and states are bit-identical across the modes,
+    and also when the whole-batch state is decoded as a reversed subset."""
     b = stress.to("cuda")
     n = len(b.lengths)
     H = b.q.shape[1]
     steps = 128
     toks = W.decode_tokens(steps, n, H, 128, 128, seed=33, g_mode="stress", device="cuda")
-    sscale = torch.empty((n, H), device="cuda")
-    _, srun, sbnd = forward(gdn, b, s_run_scale=sscale)
 
-    def decode(order):
-        st = gdn.DecodeState(n, H, 128, 128)
-        gdn.decode_state_from_prefill(st, b.k, b.v, b.beta, b.g, b.cu_seqlens, srun, sbnd,
-                                      s_run_scale=sscale)
+    def handoff(batch, slots, n_slots):
+        """Forward over `batch`, then its handoff into `n_slots` slots (sequence i
+        of the batch goes to slot slots[i])."""
+        N = len(batch.lengths)
+        sscale = torch.empty((N, H), device="cuda")
+        _, srun, sbnd = forward(gdn, batch, s_run_scale=sscale)
+        st = gdn.DecodeState(n_slots, H, 128, 128)
+        gdn.decode_state_from_prefill(st, batch.k, batch.v, batch.beta, batch.g,
+                                      batch.cu_seqlens, srun, sbnd, s_run_scale=sscale,
+                                      slot_idx=torch.tensor(slots, dtype=torch.int32,
+                                                            device="cuda"))
+        return st
+
+    def decode(st, order):
         slots = torch.tensor(order, dtype=torch.int32, device="cuda")
         r = torch.tensor(order, device="cuda")
         outs = []
@@ -107,11 +120,50 @@ def test_decode_batch_invariance(gdn, stress):
             outs.append(gdn.decode_step(st, q, k, v, beta, g, slot_idx=slots,
                                         out_dtype=torch.float32))
         assert gdn.check_error(st.error) == 0
-        return torch.stack(outs), st
+        return torch.stack(outs)
 
-    o_all, st_all = decode(list(range(n)))
+    every = list(range(n))
+    # whole batch
+    st_whole = handoff(b, every, n)
+    st_sub = st_whole.clone()
+    o_whole = decode(st_whole, every)
+    states = {"whole": st_whole}
+    outs = {}
+    # shuffled batch: sequence i of the shuffled batch is original perm[i]
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(31)).tolist()
+    st = handoff(b.select(perm), perm, n)
+    outs["shuffled"], states["shuffled"] = decode(st, every), st
+    # one sequence at a time, each handed off into its own slot of one state
+    st = gdn.DecodeState(n, H, 128, 128)
+    for i in range(n):
+        bi = b.select([i])
+        sscale = torch.empty((1, H), device="cuda")
+        _, srun, sbnd = forward(gdn, bi, s_run_scale=sscale)
+        gdn.decode_state_from_prefill(st, bi.k, bi.v, bi.beta, bi.g, bi.cu_seqlens, srun, sbnd,
+                                      s_run_scale=sscale,
+                                      slot_idx=torch.tensor([i], dtype=torch.int32,
+                                                            device="cuda"))
+    outs["alone"], states["alone"] = decode(st, every), st
+    # padded: an empty sequence before, between and after the real ones; the
+    # empty ones are handed off into extra slots n .. 2n
+    lens, slots = [], []
+    for i, L in enumerate(b.lengths):
+        lens += [0, L]
+        slots += [n + i, i]
+    lens.append(0)
+    slots.append(2 * n)
+    pad = W.Batch(b.q, b.k, b.v, b.beta, b.g, W.cu_seqlens_of(lens, "cuda"), lens)
+    st = handoff(pad, slots, 2 * n + 1)
+    outs["padded"], states["padded"] = decode(st, every), st
+
+    for mode, o in outs.items():
+        assert torch.equal(o, o_whole), mode
+        for name in ("s_run", "s_scale", "s_bnd", "pos"):
+            a = getattr(states[mode], name)[:n]
+            assert torch.equal(a, getattr(st_whole, name)), (mode, name)
+
     sub = list(reversed(range(0, n, 3)))
-    o_sub, st_sub = decode(sub)
+    o_sub = decode(st_sub, sub)
     for j, i in enumerate(sub):
-        assert torch.equal(o_sub[:, j], o_all[:, i]), i
-        assert torch.equal(st_sub.s_bnd[i], st_all.s_bnd[i])
+        assert torch.equal(o_sub[:, j], o_whole[:, i]), i
+        assert torch.equal(st_sub.s_bnd[i], st_whole.s_bnd[i])

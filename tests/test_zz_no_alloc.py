@@ -4,11 +4,14 @@ Some callers of this library cannot call cudaMalloc (a host runtime that
 owns the device memory pool, a plugin host without a device allocator, code
 that must not allocate on its hot path).  gdn_cpr_forward_noalloc serves them
 from a fixed scratch array compiled into the library.  This test calls it
-through the C ABI twice in a row, on two different problems, and checks each
-result against the regular gdn_cpr_forward (with a caller workspace) within
-the tolerance the other GPU tests use; it also checks that a problem larger
-than the fixed scratch is refused.  This file is collected last so that a
-run stopping at the first failure has already run every other test.
+through the C ABI twice in a row, on two different problems (the larger one
+first, so the second call runs on scratch that still holds the first call's
+data), and checks each result against the regular gdn_cpr_forward (with a
+caller workspace).  Both run the same kernels on the same inputs, so the
+results must agree bit for bit, which is stricter than the oracle tolerance
+of the other GPU tests.  It also checks that a problem larger than the fixed
+scratch is refused.  This file is collected last so that a run stopping at
+the first failure has already run every other test.
 """
 import ctypes
 
@@ -16,7 +19,6 @@ import pytest
 import torch
 
 from rl_train_numerics_b200 import workloads as W
-from tests.gdn_testlib import rel_err, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -53,10 +55,10 @@ def regular(gdn, b):
 def test_noalloc_matches_regular_forward_two_calls_in_a_row(gdn):
     cases = [W.make_batch([300, 64, 17, 0, 129], 4, 128, 128, seed=41),
              W.make_batch([256, 70, 1], 2, 64, 64, dtype=torch.float32, seed=42)]
-    for b in cases:
-        need = gdn.forward_workspace_bytes(len(b.lengths), b.total_tokens, b.q.shape[1],
-                                           b.q.shape[2], b.q.shape[2], in_dtype=b.q.dtype)
-        assert 0 < need <= NOALLOC_LIMIT
+    need = [gdn.forward_workspace_bytes(len(b.lengths), b.total_tokens, b.q.shape[1],
+                                        b.q.shape[2], b.q.shape[2], in_dtype=b.q.dtype)
+            for b in cases]
+    assert 0 < need[1] < need[0] <= NOALLOC_LIMIT  # a smaller problem follows a larger one
     results = []
     for b in [cases[0].to("cuda"), cases[1].to("cuda")]:  # two calls in a row
         T, H, d = b.q.shape
@@ -70,10 +72,9 @@ def test_noalloc_matches_regular_forward_two_calls_in_a_row(gdn):
         results.append((b, o, srun, sbnd))
     for b, o, srun, sbnd in results:
         o_ref, srun_ref, sbnd_ref = regular(gdn, b)
-        tol = tol_for(b.q.dtype)
-        assert rel_err(o, o_ref.double().cpu().numpy()) <= tol
-        assert rel_err(srun, srun_ref.double().cpu().numpy()) <= tol
-        assert rel_err(sbnd, sbnd_ref.double().cpu().numpy()) <= tol
+        assert torch.equal(o, o_ref)
+        assert torch.equal(srun, srun_ref)
+        assert torch.equal(sbnd, sbnd_ref)
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch(gdn):
@@ -85,3 +86,17 @@ def test_noalloc_refuses_problems_beyond_its_scratch(gdn):
     o = torch.zeros((T, H, d), dtype=torch.bfloat16, device="cuda")
     b = W.Batch(x, x, x, bg, bg, cu, [2048] * 5)
     assert call_noalloc(gdn, b, o, None, None, None) == gdn.GDN_ERR_WORKSPACE
+
+
+def test_noalloc_empty_batch_clears_the_error_word(gdn):
+    """An empty batch launches no kernel but still reports this call's status
+    in the caller's error word (zero) instead of an earlier call's bits."""
+    err = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    cu = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = gdn.lib.gdn_cpr_forward_noalloc(None, None, None, gdn.GDN_BF16, None, None, p(cu), 0, 0,
+                                         4, 128, 128, 64, 1.0, None, None, gdn.GDN_BF16, None,
+                                         None, None, p(err), stream)
+    assert rc == gdn.GDN_OK
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
