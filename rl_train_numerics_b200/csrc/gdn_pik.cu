@@ -9,30 +9,41 @@
 // owns the same contiguous block of leaves (a complete subtree), so the bits
 // do not depend on how many ranks share the work.
 //
-// On one GPU the work is cut the same way.  k_pik_gemm<G, BN> computes, for a
-// 128 x BN tile of C, one group of G consecutive leaves: each leaf
-// accumulates in its own G-th of the tile's tensor-memory columns
-// (G x BN <= 512), in 64-wide K steps of four m128 x BN x k16 MMAs, ascending
-// k; the epilogue reads the G accumulators back and adds them level by level
-// (neighbours 2i, 2i + 1).  A group is a node of the tree, so when L / G > 1
-// the group sums go to a workspace and k_pik_combine applies the levels
-// above them, again neighbours first.  The group size is min(L / R, 2) for R
-// emulated ranks, and whatever it is, every addition of the tree happens in
-// the same order on the same operands: the result is the same for every R.
+// On one GPU the work is cut the same way.  A work unit is one 128 x 256 tile
+// of C and one emulated rank's L / R consecutive leaves.  k_pik_gemm is
+// persistent (one block per SM, units taken round-robin in a grouped raster
+// that keeps a band of A rows and the B tiles beside it in L2) and
+// warp-specialised:
+//   warp 0      TMA producer: one 2-D box of A (128 x 64) and of B (256 x 64)
+//               per 64-wide K step into a four-stage ring ("full" mbarriers
+//               with transaction bytes, "empty" mbarriers from the MMAs);
+//   warp 1      MMA issuer: each leaf accumulates in one of two 256-column
+//               tensor-memory buffers (alternating), four m128 n256 k16 MMAs
+//               per K step, ascending k, a fresh accumulator at the leaf's
+//               first step; the leaf's last commit signals the epilogue;
+//   warps 2-9   epilogue: read a finished leaf back (one tile row and half the
+//               columns per thread),
+//               release its buffer, and advance the balanced tree as a binary
+//               counter: the leaf is added to the pending subtree sums of
+//               equal size, left operand first, and the result is either the
+//               unit's sum (stored) or pushed as a pending sum.  Pending sums
+//               live in a per-block slice of the workspace (one 128 KB slot
+//               per tree level, written and read by the same threads).
+// The epilogue of leaf i overlaps the MMAs of leaf i + 1.  With R > 1 ranks
+// the unit sums go to the workspace and k_pik_combine applies the levels
+// above the ranks, again neighbours first.  Whatever R is, every addition of
+// the tree happens in the same order on the same operands.
 //
 // Operands: A [M, K] and B [N, K] bf16, both K-major (row-major with K
 // innermost); C [M, N] fp32.  Tiles reach shared memory by TMA in the
-// 128-byte swizzled K-major layout: one 2-D tensor copy per operand and stage
-// (64 K columns = 128 bytes per row, 8-row atoms of 1024 bytes, 16-byte
-// chunks permuted by the row's low three bits), which is also the MMA's
-// operand layout; a k16 step starts 32 bytes further along the row.  Rows
-// past M or N read as zero.  Roles: thread 0 issues the copies
-// of a stage once the MMAs that read it last have committed ("empty"
-// mbarrier), warp 1 issues a stage's four MMAs once its copies have landed
-// ("full" mbarrier, transaction bytes), and all four warps run the epilogue.
-// Four stages.  Waits are bounded: one that gives up sets GDN_DEVERR_TIMEOUT
-// in the error word, waits (bounded) for the copies and MMAs in flight, frees
-// tensor memory and returns.
+// 128-byte swizzled K-major layout (64 K columns = 128 bytes per row, 8-row
+// atoms of 1024 bytes, 16-byte chunks permuted by the row's low three bits),
+// which is also the MMA's operand layout; a k16 step starts 32 bytes further
+// along the row.  Rows past M or N read as zero.  Waits are bounded: a role
+// that gives up sets GDN_DEVERR_TIMEOUT in the error word and raises a shared
+// abort flag so the other roles stop at their next wait; the block then waits
+// (bounded) for its copies and MMAs in flight, frees tensor memory and
+// returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -45,24 +56,32 @@
 namespace gdn {
 namespace {
 
-constexpr int kPikThreads = 128;   // four warps: tensor-memory lanes 0..127 = tile rows
+constexpr int kPikBM = 128;        // tile rows (tensor-memory lanes)
+constexpr int kPikBN = 256;        // tile columns (one accumulator buffer)
+constexpr int kPikEpiThreads = 256;  // two warps per tensor-memory lane quarter
+constexpr int kPikThreads = 64 + kPikEpiThreads;  // producer warp, MMA warp, 8 epilogue warps
+constexpr int kPikChunksPerThread = kPikBN / 32 / 2;  // 32-column chunks per epilogue thread
 constexpr int kPikStages = 4;
 constexpr int kPikKStep = 64;      // K per stage
+constexpr int kPikBand = 16;       // M tiles per band of the raster
+constexpr int kPikMaxBlocks = 148; // persistent blocks at most (one per SM of a B200)
+constexpr uint32_t kPikStageBytes = (kPikBM + kPikBN) * kPikKStep * 2;
 constexpr int kPikPolls = 1 << 22;
 constexpr int kPikErrTimeout = 4;  // GDN_DEVERR_TIMEOUT
 
-template <int BN>
 struct PikSmem {
-  __nv_bfloat16 A[kPikStages][128 * kPikKStep];
-  __nv_bfloat16 B[kPikStages][BN * kPikKStep];
+  __nv_bfloat16 A[kPikStages][kPikBM * kPikKStep];
+  __nv_bfloat16 B[kPikStages][kPikBN * kPikKStep];
   uint64_t full[kPikStages];   // copies of the stage have landed
   uint64_t empty[kPikStages];  // MMAs reading the stage are done
-  uint64_t done;               // every MMA is done
+  uint64_t acc_full[2];        // a leaf's MMAs into the buffer are done
+  uint64_t acc_empty[2];       // the epilogue has read the buffer
   uint32_t tmem_slot;
+  int abort;                   // a role gave up: the others stop
 };
 
 // 2-D tiled TMA load of one box into shared memory, completion counted on the
-// mbarrier in transaction bytes.  x (the K coordinate) is a multiple of 8
+// mbarrier in transaction bytes.  x (the K coordinate) is a multiple of 64
 // elements, so x * 2 bytes is a multiple of 16.
 __device__ __forceinline__ void tma_load_2d(uint32_t sdst, const CUtensorMap* map, int x, int y,
                                             uint32_t mbar) {
@@ -80,135 +99,248 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return smem_desc(saddr, 16, 1024) | ((uint64_t)2 << 61);
 }
 
-template <int G>
-__device__ __forceinline__ void tree16(float (&x)[G][16]) {
-#pragma unroll
-  for (int w = G; w > 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w / 2; i++)
-#pragma unroll
-      for (int j = 0; j < 16; j++) x[i][j] = __fadd_rn(x[2 * i][j], x[2 * i + 1][j]);
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
 }
 
-// One 128 x BN tile of one group of G leaves.  blockIdx = (M tile, N tile,
-// group); out is C (one group) or the group's slice of the workspace.
-template <int G, int BN>
+// Work unit u of the grouped raster: rank group z, M tile tm, N tile tn.
+// Bands of kPikBand M tiles; inside a band the M tile runs fastest.
+struct PikUnit {
+  int z, tm, tn;
+};
+__device__ __forceinline__ PikUnit pik_unit(int u, int m_tiles, int n_tiles) {
+  const int tiles = m_tiles * n_tiles;
+  PikUnit w;
+  w.z = u / tiles;
+  const int t = u - w.z * tiles;
+  const int per_band = kPikBand * n_tiles;
+  const int band = t / per_band;
+  const int r = t - band * per_band;
+  const int rows = min(kPikBand, m_tiles - band * kPikBand);
+  w.tm = band * kPikBand + r % rows;
+  w.tn = r / rows;
+  return w;
+}
+
+__device__ __forceinline__ int ctz32(uint32_t x) { return __ffs((int)x) - 1; }
+
+// The persistent K-leaf GEMM (see the file comment).  out: C (R = 1) or the
+// R rank sums [R, M, N] in the workspace; stack: kPikMaxBlocks x depth slots of
+// 128 x 256 fp32 pending sums (depth = log2(L / R)).
 __global__ void __launch_bounds__(kPikThreads, 1)
     k_pik_gemm(const __grid_constant__ CUtensorMap map_a,
-               const __grid_constant__ CUtensorMap map_b, int64_t M, int64_t N,
-               int64_t leaf_k, float* __restrict__ out, int32_t* __restrict__ error) {
-  constexpr int kCols = (G * BN < 32) ? 32 : G * BN;  // a power of two here
-  constexpr uint32_t kStageBytes = (128 + BN) * kPikKStep * 2;
+               const __grid_constant__ CUtensorMap map_b, int M, int N, int leaf_k,
+               int leaves, int n_units, float* __restrict__ out, float4* __restrict__ stack,
+               int32_t* __restrict__ error) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // The swizzled tiles need 1024-byte alignment: round the base up (the
-  // launch requests 1 KB more than the tiles need).
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
-  PikSmem<BN>& sm = *reinterpret_cast<PikSmem<BN>*>(smem_raw + pad);
+  PikSmem& sm = *reinterpret_cast<PikSmem*>(smem_raw + pad);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = (int)blockIdx.x * 128, n0 = (int)blockIdx.y * BN;
-  const int64_t kbase = (int64_t)blockIdx.z * G * leaf_k;
-  const int spl = (int)(leaf_k / kPikKStep);  // K steps per leaf
-  const int S = G * spl;
-  out += (int64_t)blockIdx.z * M * N;
+  const int m_tiles = (M + kPikBM - 1) / kPikBM, n_tiles = (N + kPikBN - 1) / kPikBN;
+  const int spl = leaf_k / kPikKStep;  // K steps per leaf
+  const int depth = 31 - __clz(leaves);
 
-  if (warp == 0) tmem_alloc(smem_u32(&sm.tmem_slot), kCols);
+  if (warp == 1) tmem_alloc(smem_u32(&sm.tmem_slot), 2 * kPikBN);
   if (tid == 0) {
     for (int i = 0; i < kPikStages; i++) {
       mbar_init(smem_u32(&sm.full[i]), 1);
       mbar_init(smem_u32(&sm.empty[i]), 1);
     }
-    mbar_init(smem_u32(&sm.done), 1);
+    for (int b = 0; b < 2; b++) {
+      mbar_init(smem_u32(&sm.acc_full[b]), 1);
+      mbar_init(smem_u32(&sm.acc_empty[b]), kPikEpiThreads);
+    }
+    sm.abort = 0;
     fence_mbar_init();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_slot;
-  constexpr uint32_t idesc = idesc_bf16(128, BN, false, false);
+  volatile int* abort_flag = &sm.abort;
   bool ok = true;
-  int issued = 0;  // steps whose copies thread 0 issued
+  int issued = 0;     // K steps whose copies the producer issued
+  int committed = 0;  // K steps whose MMAs were issued (and committed)
 
-  if (tid == 0) {
-    // Producer: the copies of step s go to stage s % NS once the MMAs of step
-    // s - NS (the stage's previous use) have committed.
-    for (int s = 0; s < S; s++) {
-      const int st = s % kPikStages;
-      if (s >= kPikStages &&
-          !mbar_wait(smem_u32(&sm.empty[st]), (uint32_t)((s / kPikStages - 1) & 1), kPikPolls)) {
-        ok = false;
-        break;
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const PikUnit w = pik_unit(u, m_tiles, n_tiles);
+        const int kbase = w.z * leaves * leaf_k;
+        for (int step = 0; step < leaves * spl; step++, s++) {
+          const int st = s % kPikStages;
+          if (s >= kPikStages &&
+              !mbar_wait(smem_u32(&sm.empty[st]), (uint32_t)((s / kPikStages - 1) & 1),
+                         kPikPolls)) {
+            ok = false;
+            break;
+          }
+          if (*abort_flag) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&sm.full[st]);
+          mbar_expect_tx(fb, kPikStageBytes);
+          const int k0 = kbase + step * kPikKStep;
+          tma_load_2d(smem_u32(sm.A[st]), &map_a, k0, w.tm * kPikBM, fb);
+          tma_load_2d(smem_u32(sm.B[st]), &map_b, k0, w.tn * kPikBN, fb);
+          issued = s + 1;
+        }
       }
-      const uint32_t fb = smem_u32(&sm.full[st]);
-      mbar_expect_tx(fb, kStageBytes);
-      const int k0 = (int)(kbase + (int64_t)s * kPikKStep);
-      const uint32_t a0 = smem_u32(sm.A[st]), b0 = smem_u32(sm.B[st]);
-      tma_load_2d(a0, &map_a, k0, m0, fb);
-      tma_load_2d(b0, &map_b, k0, n0, fb);
-      issued = s + 1;
+      if (!ok) *abort_flag = 1;
     }
   } else if (warp == 1) {
-    // MMA issuer: a stage's four k16 MMAs once its copies have landed.
-    for (int s = 0; s < S; s++) {
-      const int st = s % kPikStages;
-      if (!mbar_wait(smem_u32(&sm.full[st]), (uint32_t)((s / kPikStages) & 1), kPikPolls)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t a0 = smem_u32(sm.A[st]), b0 = smem_u32(sm.B[st]);
-      const uint32_t d = tmem + (uint32_t)((s / spl) * BN);
+    constexpr uint32_t idesc = idesc_bf16(kPikBM, kPikBN, false, false);
+    int s = 0, lc = 0;  // K step and leaf counters of this block
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      for (int leaf = 0; leaf < leaves && ok; leaf++, lc++) {
+        const int b = lc & 1, use = lc >> 1;
+        // (every wait's result is made warp-uniform: the MMA wrappers need
+        // the whole warp)
+        if (use > 0 &&
+            !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.acc_empty[b]),
+                                               (uint32_t)((use - 1) & 1), kPikPolls))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(b * kPikBN);
+        for (int ks = 0; ks < spl; ks++, s++) {
+          const int st = s % kPikStages;
+          if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.full[st]),
+                                                 (uint32_t)((s / kPikStages) & 1), kPikPolls) &&
+                                           !*abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sm.A[st]), b0 = smem_u32(sm.B[st]);
 #pragma unroll
-      for (int j = 0; j < kPikKStep / 16; j++)
-        umma_bf16(d, desc_kmajor_sw128(a0 + j * 32), desc_kmajor_sw128(b0 + j * 32), idesc,
-                  (s % spl != 0 || j > 0) ? 1u : 0u);
-      umma_commit(smem_u32(&sm.empty[st]));
+          for (int j = 0; j < kPikKStep / 16; j++)
+            umma_bf16(d, desc_kmajor_sw128(a0 + j * 32), desc_kmajor_sw128(b0 + j * 32), idesc,
+                      (ks > 0 || j > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&sm.empty[st]));
+          committed = s + 1;
+        }
+        if (ok) umma_commit(smem_u32(&sm.acc_full[b]));
+      }
     }
-    umma_commit(smem_u32(&sm.done));  // every MMA issued so far
-  }
-  // Everyone: wait until every MMA is done (bounded).
-  if (!mbar_wait(smem_u32(&sm.done), 0u, kPikPolls)) {
-    ok = false;
-    (void)mbar_wait(smem_u32(&sm.done), 0u, kPikPolls);  // bounded drain before freeing
-  }
-  tc_fence_after();
-  const bool failed = __syncthreads_or(!ok);
-  if (!failed) {
-    const int64_t m = m0 + warp * 32 + lane;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    float* orow = out + m * N + n0;
+    if (!ok && lane == 0) *abort_flag = 1;
+  } else {
+    // Epilogue: tile row r (tensor-memory lane quarter warp % 4) and one half
+    // of the tile's columns per thread (two warps per lane quarter).
+    const int q = warp & 3, r = q * 32 + lane, half = (warp - 2) >> 2;
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    float4* my_stack = stack + (size_t)blockIdx.x * depth * (kPikBM * kPikBN / 4);
+    int lc = 0;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const PikUnit w = pik_unit(u, m_tiles, n_tiles);
+      const int m = w.tm * kPikBM + r, n0 = w.tn * kPikBN;
+      float* orow = out + (size_t)w.z * M * N + (size_t)m * N + n0;
+      for (int leaf = 0; leaf < leaves; leaf++, lc++) {
+        const int b = lc & 1, use = lc >> 1;
+        bool got = mbar_wait(smem_u32(&sm.acc_full[b]), (uint32_t)(use & 1), kPikPolls);
+        got = __all_sync(0xffffffffu, got) && !*abort_flag;
+        if (!got) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int combos = ctz32((uint32_t)(leaf + 1));  // pending sums this leaf closes
+        const bool last = leaf == leaves - 1;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
-      float x[G][16];
+        for (int cc = 0; cc < kPikChunksPerThread; cc++) {
+          const int c = half * kPikChunksPerThread + cc;  // 32-column chunk of the tile
+          float x[32];
+          tmem_ld32(lane_base + (uint32_t)(b * kPikBN + c * 32), x);
+          tmem_wait_ld(x);
+          if (cc == kPikChunksPerThread - 1) {
+            // this thread has read all its columns of the buffer
+            tc_fence_before();
+            mbar_arrive(smem_u32(&sm.acc_empty[b]));
+          }
+          // x = pending(level 0) + x, then pending(level 1) + x, ...: each
+          // pending sum is the left (earlier) subtree.  Two levels' loads are
+          // issued together.
+#pragma unroll 1
+          for (int lev = 0; lev < combos; lev += 2) {
+            const bool two = lev + 1 < combos;
+            const float4* s0 = my_stack + ((size_t)(lev * 8 + c) * 8) * kPikBM + r;
+            const float4* s1 = s0 + (size_t)64 * kPikBM;
+            float4 y0[8], y1[8];
 #pragma unroll
-      for (int i = 0; i < G; i++) tmem_ld16(lane_base + (uint32_t)(i * BN + c), x[i]);
+            for (int f = 0; f < 8; f++) y0[f] = s0[(size_t)f * kPikBM];
+            if (two) {
 #pragma unroll
-      for (int i = 0; i < G; i++) tmem_wait_ld(x[i]);
-      tree16<G>(x);
-      if (m < M && n0 + c < N) {
+              for (int f = 0; f < 8; f++) y1[f] = s1[(size_t)f * kPikBM];
+            }
 #pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(orow + c + j) =
-              make_float4(x[0][j], x[0][j + 1], x[0][j + 2], x[0][j + 3]);
+            for (int f = 0; f < 8; f++) {
+              x[4 * f + 0] = __fadd_rn(y0[f].x, x[4 * f + 0]);
+              x[4 * f + 1] = __fadd_rn(y0[f].y, x[4 * f + 1]);
+              x[4 * f + 2] = __fadd_rn(y0[f].z, x[4 * f + 2]);
+              x[4 * f + 3] = __fadd_rn(y0[f].w, x[4 * f + 3]);
+            }
+            if (two) {
+#pragma unroll
+              for (int f = 0; f < 8; f++) {
+                x[4 * f + 0] = __fadd_rn(y1[f].x, x[4 * f + 0]);
+                x[4 * f + 1] = __fadd_rn(y1[f].y, x[4 * f + 1]);
+                x[4 * f + 2] = __fadd_rn(y1[f].z, x[4 * f + 2]);
+                x[4 * f + 3] = __fadd_rn(y1[f].w, x[4 * f + 3]);
+              }
+            }
+          }
+          if (last) {
+            if (m < M) {
+#pragma unroll
+              for (int f = 0; f < 8; f++)
+                if (n0 + c * 32 + 4 * f < N)
+                  *reinterpret_cast<float4*>(orow + c * 32 + 4 * f) =
+                      make_float4(x[4 * f], x[4 * f + 1], x[4 * f + 2], x[4 * f + 3]);
+            }
+          } else {
+            float4* dst = my_stack + ((size_t)(combos * 8 + c) * 8) * kPikBM + r;
+#pragma unroll
+            for (int f = 0; f < 8; f++)
+              dst[(size_t)f * kPikBM] = make_float4(x[4 * f], x[4 * f + 1], x[4 * f + 2],
+                                                    x[4 * f + 3]);
+          }
+        }
       }
     }
-  } else if (tid == 0) {
+    if (!ok && lane == 0) *abort_flag = 1;
+  }
+
+  const bool failed = __syncthreads_or(!ok) || *abort_flag;
+  if (failed && tid == 0) {
     atomicOr(error, kPikErrTimeout);
     // Copies still in flight land before the block's shared memory is freed:
-    // wait (bounded) for the last phase of every stage that was filled.
+    // wait (bounded) for the last phase of every stage that was filled; then
+    // for the MMAs issued (their last commit).
     for (int s = issued - kPikStages < 0 ? 0 : issued - kPikStages; s < issued; s++)
       (void)mbar_wait(smem_u32(&sm.full[s % kPikStages]), (uint32_t)((s / kPikStages) & 1),
                       kPikPolls);
   }
+  if (failed && warp == 1 && committed > 0) {
+    const int s = committed - 1;
+    (void)mbar_wait(smem_u32(&sm.empty[s % kPikStages]), (uint32_t)((s / kPikStages) & 1),
+                    kPikPolls);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, kCols);
+  if (warp == 1) tmem_dealloc(tmem, 2 * kPikBN);
   if (tid == 0) {
     for (int i = 0; i < kPikStages; i++) {
       mbar_inval(smem_u32(&sm.full[i]));
       mbar_inval(smem_u32(&sm.empty[i]));
     }
-    mbar_inval(smem_u32(&sm.done));
+    for (int b = 0; b < 2; b++) {
+      mbar_inval(smem_u32(&sm.acc_full[b]));
+      mbar_inval(smem_u32(&sm.acc_empty[b]));
+    }
   }
 }
 
@@ -240,21 +372,26 @@ __global__ void __launch_bounds__(256)
 }
 
 struct PikPlan {
-  int G, BN, groups;  // leaves per block, tile width, groups per output tile
-  size_t ws;          // workspace bytes (group sums when groups > 1)
+  int leaves;       // leaves per work unit (one rank's subtree)
+  int units;        // work units: ranks x tiles
+  int blocks;       // persistent blocks
+  int depth;        // tree levels inside a unit = log2(leaves)
+  size_t ws_ranks;  // rank sums [R, M, N] fp32 when R > 1
+  size_t ws_stack;  // pending subtree sums: blocks x depth x 128 x 256 fp32
 };
 
-// Group size: at most two leaves per block, so that every block runs the
-// widest tile (BN = 256) and the deeper levels go to k_pik_combine.  Deeper
-// in-memory trees (four or eight leaves, BN = 128 or 64) ran up to 3x slower at
-// the 8192^3 shape; the grouping never changes the bits.
+// Every unit is one rank's L / R leaves of one 128 x 256 tile; the grouping
+// never changes the bits.
 PikPlan pik_plan(int64_t M, int64_t N, int L, int R) {
   PikPlan p{};
-  const int per_rank = L / R;  // leaves per emulated rank
-  p.G = per_rank < 2 ? per_rank : 2;
-  p.BN = 256;
-  p.groups = L / p.G;
-  p.ws = p.groups > 1 ? (size_t)p.groups * (size_t)M * (size_t)N * sizeof(float) : 0;
+  p.leaves = L / R;
+  const int64_t tiles = ((M + kPikBM - 1) / kPikBM) * ((N + kPikBN - 1) / kPikBN);
+  p.units = (int)(tiles * R);
+  p.blocks = p.units < kPikMaxBlocks ? p.units : kPikMaxBlocks;
+  p.depth = 0;
+  while ((1 << p.depth) < p.leaves) p.depth++;
+  p.ws_ranks = R > 1 ? (size_t)R * (size_t)M * (size_t)N * sizeof(float) : 0;
+  p.ws_stack = (size_t)p.blocks * p.depth * kPikBM * kPikBN * sizeof(float);
   return p;
 }
 
@@ -264,8 +401,9 @@ int validate(int64_t M, int64_t N, int64_t K, int L, int R) {
   if (M < 0 || N < 0 || K < 0 || L < 1 || R < 1) return GDN_ERR_INVALID_ARG;
   if (!pow2(L) || !pow2(R) || L % R != 0 || L > 64) return GDN_ERR_UNSUPPORTED;
   if (N % 16 != 0 || K % ((int64_t)kPikKStep * L) != 0) return GDN_ERR_UNSUPPORTED;
-  // TMA coordinates are 32-bit: rows and K below 2^31.
-  if (N / 64 > 65535 || M >= 0x7fffffff || N >= 0x7fffffff || K >= 0x7fffffff)
+  // TMA coordinates and the unit count are 32-bit.
+  if (M >= 0x7fffffff || N >= 0x7fffffff || K >= 0x7fffffff) return GDN_ERR_UNSUPPORTED;
+  if (((M + kPikBM - 1) / kPikBM) * ((N + kPikBN - 1) / kPikBN) * R >= 0x7fffffff)
     return GDN_ERR_UNSUPPORTED;
   return GDN_OK;
 }
@@ -304,26 +442,20 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int b
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Each block allocates all 512 tensor-memory columns of its SM (or 256 with
-// G = 1, whose 192 KB of shared memory already keeps blocks one per SM), so
-// the shared-memory request is raised to at least 116 KB: a second block on
-// the SM would otherwise sit in tcgen05.alloc until the first one frees.
-constexpr size_t kPikMinSmem = 116 * 1024;
-
-template <int G, int BN>
 int launch_gemm(const PikPlan& p, const void* A, const void* B, int64_t M, int64_t N, int64_t K,
-                int64_t leaf_k, float* out, int32_t* error, cudaStream_t st) {
+                int64_t leaf_k, float* out, float* stack, int32_t* error, cudaStream_t st) {
   CUtensorMap ma, mb;
-  if (!make_map(&ma, A, M, K, 128) || !make_map(&mb, B, N, K, BN)) return GDN_ERR_CUDA;
-  auto kern = k_pik_gemm<G, BN>;
-  const size_t need = sizeof(PikSmem<BN>) + 1024;
-  const size_t smem = need < kPikMinSmem ? kPikMinSmem : need;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
+  if (!make_map(&ma, A, M, K, kPikBM) || !make_map(&mb, B, N, K, kPikBN)) return GDN_ERR_CUDA;
+  // 1 KB more than the tiles need, for the 1024-byte alignment of the swizzled
+  // tiles; about 194 KB keeps one block per SM, which owns all 512
+  // tensor-memory columns.
+  const size_t smem = sizeof(PikSmem) + 1024;
+  if (cudaFuncSetAttribute(k_pik_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
     return GDN_ERR_CUDA;
-  const dim3 grid((unsigned)((M + 127) / 128), (unsigned)((N + BN - 1) / BN),
-                  (unsigned)p.groups);
-  kern<<<grid, kPikThreads, smem, st>>>(ma, mb, M, N, leaf_k, out, error);
+  k_pik_gemm<<<p.blocks, kPikThreads, smem, st>>>(ma, mb, (int)M, (int)N, (int)leaf_k, p.leaves,
+                                                 p.units, out, reinterpret_cast<float4*>(stack),
+                                                 error);
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -334,7 +466,9 @@ extern "C" {
 
 size_t gdn_pik_workspace_bytes(int64_t M, int64_t N, int64_t K, int n_leaves, int n_ranks) {
   if (gdn::validate(M, N, K, n_leaves, n_ranks) != GDN_OK) return 0;
-  return gdn::pik_plan(M, N, n_leaves, n_ranks).ws;
+  if (M == 0 || N == 0 || K == 0) return 0;
+  const gdn::PikPlan p = gdn::pik_plan(M, N, n_leaves, n_ranks);
+  return p.ws_ranks + p.ws_stack;
 }
 
 int gdn_pik_gemm(const void* A, const void* B, float* C, int64_t M, int64_t N, int64_t K,
@@ -354,21 +488,20 @@ int gdn_pik_gemm(const void* A, const void* B, float* C, int64_t M, int64_t N, i
   }
   if (!A || !B || !al16(A) || !al16(B)) return GDN_ERR_INVALID_ARG;
   const gdn::PikPlan p = gdn::pik_plan(M, N, n_leaves, n_ranks);
-  if (p.ws > 0 && (!workspace || workspace_bytes < p.ws || !al16(workspace)))
+  const size_t need = p.ws_ranks + p.ws_stack;
+  if (need > 0 && (!workspace || workspace_bytes < need || !al16(workspace)))
     return GDN_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* out = p.groups > 1 ? static_cast<float*>(workspace) : C;
+  char* ws = static_cast<char*>(workspace);
+  float* out = p.ws_ranks > 0 ? reinterpret_cast<float*>(ws) : C;
+  float* stack = p.ws_stack > 0 ? reinterpret_cast<float*>(ws + p.ws_ranks) : nullptr;
   const int64_t leaf_k = K / n_leaves;
-  int r;
-  if (p.G == 1)
-    r = gdn::launch_gemm<1, 256>(p, A, B, M, N, K, leaf_k, out, error_word, st);
-  else
-    r = gdn::launch_gemm<2, 256>(p, A, B, M, N, K, leaf_k, out, error_word, st);
+  int r = gdn::launch_gemm(p, A, B, M, N, K, leaf_k, out, stack, error_word, st);
   if (r != GDN_OK) return r;
-  if (p.groups > 1) {
+  if (n_ranks > 1) {
     const int64_t MN = M * N, threads = 256, items = MN / 4;
     gdn::k_pik_combine<<<(unsigned)((items + threads - 1) / threads), (unsigned)threads, 0, st>>>(
-        static_cast<const float*>(workspace), p.groups, MN, C);
+        reinterpret_cast<const float*>(ws), n_ranks, MN, C);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
   }
   return GDN_OK;

@@ -1,12 +1,15 @@
-"""Host-side checks of the K-leaf GEMM's grouping (no GPU).
+"""Host-side checks of the K-leaf GEMM's work split (no GPU).
 
-gdn_pik_gemm runs blocks of G = min(L / R, 2) consecutive leaves and, when
-L / G > 1, adds the group sums with a combine kernel that evaluates the tree's
-upper levels as a binary counter.  The grouping is read back through
-gdn_pik_workspace_bytes (one fp32 M x N slice per group); the counter's order
-of additions, transcribed from the combine kernel, must be the balanced tree's
-(oracle.pik.tree_f32) bit for bit for every power-of-two group count, and a
-group of two leaves followed by the counter must be the tree over the leaves.
+gdn_pik_gemm runs one work unit per 128 x 256 tile and emulated rank: the
+rank's L / R leaves, added in the kernel by the balanced tree evaluated as a
+binary counter (pending subtree sums in a per-block workspace slice, one
+128 x 256 fp32 slot per tree level, at most 148 persistent blocks).  With
+R > 1 the rank sums go to the workspace (one fp32 M x N slice per rank) and a
+combine kernel applies the levels above the ranks with the same counter.  The
+split is read back through gdn_pik_workspace_bytes; the counter's order of
+additions, transcribed from the kernels, must be the balanced tree's
+(oracle.pik.tree_f32) bit for bit for every power-of-two count, and rank
+subtrees followed by the counter must be the tree over the leaves.
 """
 import numpy as np
 import pytest
@@ -19,12 +22,14 @@ from rl_train_numerics_b200 import _abi as gdn  # noqa: E402
 
 
 @pytest.mark.parametrize("L", [1, 2, 4, 8, 16, 32, 64])
-def test_group_count_for_every_rank_count(L):
+def test_workspace_for_every_rank_count(L):
     M, N, K = 256, 512, 64 * L
+    tiles = (M // 128) * (N // 256)
     R = 1
     while R <= L:
-        G = min(L // R, 2)
-        want = (L // G) * M * N * 4 if L // G > 1 else 0
+        depth = int(np.log2(L // R))
+        blocks = min(tiles * R, 148)
+        want = (R * M * N * 4 if R > 1 else 0) + blocks * depth * 128 * 256 * 4
         assert gdn.pik_workspace_bytes(M, N, K, L, R) == want, (L, R)
         R *= 2
 
@@ -53,10 +58,11 @@ def test_combine_counter_is_the_balanced_tree(n):
     assert np.array_equal(binary_counter(parts), opik.tree_f32(parts))
 
 
-@pytest.mark.parametrize("L", [2, 4, 8, 16])
-def test_pairs_then_counter_is_the_tree_over_leaves(L):
-    rng = np.random.default_rng(100 + L)
+@pytest.mark.parametrize("L,R", [(2, 2), (4, 2), (8, 4), (16, 2), (16, 8)])
+def test_rank_subtrees_then_counter_is_the_tree_over_leaves(L, R):
+    rng = np.random.default_rng(100 + L + R)
     leaves = [(rng.normal(size=(4, 4)) * 10.0 ** rng.integers(-4, 5)).astype(np.float32)
               for _ in range(L)]
-    pairs = [np.add(leaves[2 * i], leaves[2 * i + 1], dtype=np.float32) for i in range(L // 2)]
-    assert np.array_equal(binary_counter(pairs), opik.tree_f32(leaves))
+    per = L // R
+    ranks = [binary_counter(leaves[r * per:(r + 1) * per]) for r in range(R)]
+    assert np.array_equal(binary_counter(ranks), opik.tree_f32(leaves))
