@@ -40,34 +40,39 @@ FLUSH_BYTES = 256 << 20
 PAGES_H100 = {"prefill_ms": 1.412, "decode_ms": 0.0846, "trainer_fwd_bwd_ms": 7.386}
 
 
-KERNEL_FILES = ("gdn_kernels.cu", "gdn_backward.cu")
+# Source files whose kernels a traffic figure belongs to: a recorded figure is
+# reported only while these files hash to what they were when it was captured.
+TRAFFIC_SOURCES = {
+    "forward": ("gdn_kernels.cu", "gdn_boundary.cuh", "gdn_common.cuh", "gdn_fill.cuh",
+                "gdn_mma.cuh", "gdn_umma.cuh", "gdn_layout.h"),
+    "backward": ("gdn_backward.cu", "gdn_boundary.cuh", "gdn_common.cuh", "gdn_fill.cuh",
+                 "gdn_mma.cuh", "gdn_umma.cuh", "gdn_layout.h"),
+    "pik": ("gdn_pik.cu", "gdn_mma.cuh", "gdn_umma.cuh"),
+}
 
 
-def kernel_sources_sha256() -> str:
-    """SHA-256 over the files that define the kernels (the forward/decode and
-    backward kernel files and the device headers; the host-only entry points
-    are left out)."""
+def sources_sha256(group: str) -> str:
+    """SHA-256 over the kernel source files of one group (in the order listed)."""
     import hashlib
     csrc = os.path.join(ROOT, "rl_train_numerics_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name in KERNEL_FILES or name.endswith((".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in TRAFFIC_SOURCES[group]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()
 
 
 def ncu_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when
-    the kernel sources have changed since that capture."""
+    """DRAM bytes per launch of `kernel` (dram__bytes_read.sum + dram__bytes_write.sum
+    from a single-kernel ncu capture, profiles/ncu_traffic.json), or None when its
+    kernel sources have changed since that capture."""
     try:
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
-            rec = json.load(f)
-        digest = kernel_sources_sha256()
-        if digest != rec.get("kernel_sources_sha256"):
+            rec = json.load(f)["entries"].get(kernel)
+        if rec is None or sources_sha256(rec["group"]) != rec["sources_sha256"]:
             return None
-        return rec.get("traffic_bytes", {}).get(kernel)
-    except (OSError, ValueError):
+        return rec["bytes"]
+    except (OSError, ValueError, KeyError):
         return None
 
 
@@ -489,14 +494,15 @@ def run_train_part(gdn, W, dev, rank, world, args, flush, peaks):
             "pages_h100_ms": PAGES_H100["trainer_fwd_bwd_ms"]}
 
 
-PIK_SHAPE = (8192, 8192, 8192, 8)  # M, N, K, leaves
+PIK_SHAPE = (8192, 8192, 8192, 8)  # M, N, K, leaves (M = N = K = --pik-size)
 
 
 def run_pik_part(gdn, dev, rank, world, args, flush, peaks):
     """Parallelism-invariant K-leaf GEMM: C = A B^T, M = N = K = 8192, 8 leaves,
     bf16 in, fp32 out, one emulated rank; L2 flushed before every timed call.
     cuBLAS bf16 (torch.matmul) on the same operands is timed beside it."""
-    M, N, K, L = PIK_SHAPE
+    M = N = K = args.pik_size
+    L = PIK_SHAPE[3]
     gen = torch.Generator(device=dev).manual_seed(2000 + rank)
     A = torch.randn((M, K), generator=gen, device=dev).to(torch.bfloat16)
     B = torch.randn((N, K), generator=gen, device=dev).to(torch.bfloat16)
@@ -790,6 +796,8 @@ def main():
                    default="all",
                    help="profiling aid: run only part of the benchmark")
     p.add_argument("--decode-slots", type=int, default=256)
+    p.add_argument("--pik-size", type=int, default=PIK_SHAPE[0],
+                   help="M = N = K of the K-leaf GEMM (profiling aid: a smaller case)")
     args = p.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")

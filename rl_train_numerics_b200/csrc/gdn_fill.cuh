@@ -105,4 +105,87 @@ __device__ __forceinline__ void fill_prefetch(const FillItem& it, const float* b
   }
 }
 
+// ----------------------------------------------------------------------------
+// The forward fill at d = 128 (4 state rows per thread): quad reductions
+// without shuffling unused values.
+//
+// Slot i of lane l (of its quad) holds state row r0 + (i ^ sigma(l)) with
+// sigma = (0, 2, 1, 3).  The row's lane partial sum is in the same slot on
+// every lane, and a reduce-scatter over the quad then needs no selects:
+//   step 1 (xor 1): slot 0 += partner's slot 2, slot 1 += partner's slot 3;
+//   step 2 (xor 2): slot 0 += partner's (new) slot 1.
+// Lane l ends with the full sum of row r0 + sigma(l) in slot 0, equal in bits
+// to the butterfly (x0 + x1) + (x2 + x3) of quad_sum: each addition adds the
+// same two values (IEEE addition is commutative).  A value of the owned row
+// reaches every lane's slot i from lane l ^ sigma(i) (all-gather).
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ int quad_sigma(int l) { return ((l & 1) << 1) | (l >> 1); }
+
+__device__ __forceinline__ float quad_rs(const float (&x)[4]) {
+  const float a = __fadd_rn(x[0], __shfl_xor_sync(kFull, x[2], 1));
+  const float b = __fadd_rn(x[1], __shfl_xor_sync(kFull, x[3], 1));
+  return __fadd_rn(a, __shfl_xor_sync(kFull, b, 2));
+}
+
+__device__ __forceinline__ void quad_ag(float own, float (&w)[4]) {
+  w[0] = own;
+  w[1] = __shfl_xor_sync(kFull, own, 2);
+  w[2] = __shfl_xor_sync(kFull, own, 1);
+  w[3] = __shfl_xor_sync(kFull, own, 3);
+}
+
+// State slice with permuted slots: slot i <- row r0 + (i ^ sg), from the
+// permuted boundary-state layout.
+template <int M4>
+__device__ __forceinline__ void slice4_load_bst(Slice<4, M4>& S, const float* rows, int ld,
+                                                int r0, int sg, int l) {
+#pragma unroll
+  for (int i = 0; i < 4; i++)
+#pragma unroll
+    for (int m = 0; m < M4; m++) {
+      const int r = r0 + (i ^ sg);
+      const float4 x = ld4(rows + (size_t)r * ld + bst_col(r, group_col(l, m)));
+      S.s[i][m][0] = f2(x.x, x.y);
+      S.s[i][m][1] = f2(x.z, x.w);
+    }
+}
+
+template <int M4>
+__device__ __forceinline__ void slice4_store(const Slice<4, M4>& S, float* rows, int ld, int r0,
+                                             int sg, int l) {
+#pragma unroll
+  for (int i = 0; i < 4; i++)
+#pragma unroll
+    for (int m = 0; m < M4; m++)
+      *reinterpret_cast<float4*>(rows + (size_t)(r0 + (i ^ sg)) * ld + group_col(l, m)) =
+          make_float4(S.s[i][m][0].x, S.s[i][m][0].y, S.s[i][m][1].x, S.s[i][m][1].y);
+}
+
+template <int M4>
+__device__ __forceinline__ void slice4_store_scaled(const Slice<4, M4>& S, float c, float* rows,
+                                                    int ld, int r0, int sg, int l) {
+  const float2 cc = f2(c, c);
+#pragma unroll
+  for (int i = 0; i < 4; i++)
+#pragma unroll
+    for (int m = 0; m < M4; m++) {
+      const float2 a = __fmul2_rn(cc, S.s[i][m][0]), b = __fmul2_rn(cc, S.s[i][m][1]);
+      *reinterpret_cast<float4*>(rows + (size_t)(r0 + (i ^ sg)) * ld + group_col(l, m)) =
+          make_float4(a.x, a.y, b.x, b.y);
+    }
+}
+
+// Shared memory of one item of the d = 128 fill: keys widened to fp32 (read
+// twice per token), queries and values as bf16, and per token the step's
+// scalars, computed once per item:
+//   t0 = (a = exp(g), beta, c before the token, c after it),
+//   t1 = (c' = a c, 1 / c' (0 when renormalising), renormalise flag, 0).
+struct Fill128Smem {
+  float k[kChunk + 1][128];  // row kChunk stays zero: the "next key" of the last token
+  __nv_bfloat16 q[kChunk][128];
+  __nv_bfloat16 v[kChunk][128];
+  float4 t0[kChunk];
+  float4 t1[kChunk];
+};
+
 }  // namespace gdn

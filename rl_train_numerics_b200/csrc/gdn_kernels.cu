@@ -491,6 +491,157 @@ __global__ void __launch_bounds__(kFillThreads, 3)
 }
 
 // ----------------------------------------------------------------------------
+// Pass 2 at d = 128 with bf16 inputs: the same step, in the same order, with
+// the quad reductions of gdn_fill.cuh (reduce-scatter of the row sums, the
+// row's scalar work on its owning lane, all-gather of the update weight),
+// keys widened to fp32 in shared memory once per item, and the per-token
+// scale sequence (c, c' = a c, 1 / c', renormalise) computed once per item (a
+// left-to-right chain, then the reciprocals in parallel).  Bits are those of
+// k_fill.
+// ----------------------------------------------------------------------------
+template <class OUT>
+__global__ void __launch_bounds__(kFillThreads, 3)
+    k_fill128(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+              const __nv_bfloat16* __restrict__ v, const float* __restrict__ beta,
+              const float* __restrict__ g, const int32_t* __restrict__ cu, int H, float scale,
+              int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+              const int32_t* __restrict__ chunk_seq, const float* __restrict__ bstate,
+              OUT* __restrict__ o, float* __restrict__ s_run_final,
+              float* __restrict__ s_run_scale) {
+  constexpr int D = 128, M4 = D / 16;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  Fill128Smem& sm = *reinterpret_cast<Fill128Smem*>(smem_raw);
+  __shared__ int sh_item;
+  if (hdr[kHdrValid] != 1) return;
+  const int n_items = hdr[kHdrChunks] * H;
+  const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * 4, sg = quad_sigma(l);
+  const int my_row = r0 + sg;
+  const size_t DD = (size_t)D * D;
+
+  for (int c = tid; c < D; c += kFillThreads) sm.k[kChunk][c] = 0.f;
+  if (tid == 0) sh_item = atomicAdd(&hdr[kHdrFillNext], 1);
+  __syncthreads();
+  int item = sh_item;
+  while (item < n_items) {
+    const FillItem cur = fill_item(item, H, cu, chunk_off, chunk_seq);
+    const size_t tb = (size_t)cur.t0 * H + cur.h;
+    // Keys (widened), queries and values of the item (rows past its length
+    // are zero): 2 x 8 float4 groups of each per thread, loads issued in
+    // batches.
+#pragma unroll
+    for (int half = 0; half < 2; half++) {
+      float4 xk[8];
+      uint2 xq[8], xv[8];
+#pragma unroll
+      for (int j = 0; j < 8; j++) {
+        const int e = tid + (half * 8 + j) * kFillThreads, r = e >> 5, c = (e & 31) * 4;
+        xk[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        xq[j] = xv[j] = make_uint2(0u, 0u);
+        if (r < cur.len) {
+          const size_t off = (tb + (size_t)r * H) * D + c;
+          xk[j] = ld4(k + off);
+          xq[j] = *reinterpret_cast<const uint2*>(q + off);
+          xv[j] = *reinterpret_cast<const uint2*>(v + off);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; j++) {
+        const int e = tid + (half * 8 + j) * kFillThreads, r = e >> 5, c = (e & 31) * 4;
+        *reinterpret_cast<float4*>(&sm.k[r][c]) = xk[j];
+        *reinterpret_cast<uint2*>(&sm.q[r][c]) = xq[j];
+        *reinterpret_cast<uint2*>(&sm.v[r][c]) = xv[j];
+      }
+    }
+    // Per-token scalars: a = exp(g) and beta, two tokens per thread of warps
+    // 0-1 in parallel.
+    if (tid < kChunk) {
+      float a = 0.f, b = 0.f;
+      if (tid < cur.len) {
+        a = step_decay(g[tb + (size_t)tid * H]);
+        b = beta[tb + (size_t)tid * H];
+      }
+      sm.t0[tid] = make_float4(a, b, 0.f, 0.f);
+    }
+    {
+      __syncthreads();
+      // The scale sequence: a left-to-right chain that every lane of warp 0
+      // follows (a_t read ahead from shared memory), keeping the values of
+      // its own two tokens; then each lane writes its tokens' entries.
+      if (tid < 32) {
+        float c = 1.f, my_c[2] = {1.f, 1.f}, my_cn[2] = {0.f, 0.f};
+        for (int t = 0; t < cur.len; t++) {
+          const float cn = __fmul_rn(sm.t0[t].x, c);
+          if (t == tid) { my_c[0] = c; my_cn[0] = cn; }
+          if (t == tid + 32) { my_c[1] = c; my_cn[1] = cn; }
+          c = scale_ok(cn) ? cn : 1.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+          const int t = tid + 32 * j;
+          if (t < cur.len) {
+            const bool keep = scale_ok(my_cn[j]);
+            sm.t0[t].z = my_c[j];
+            sm.t0[t].w = keep ? my_cn[j] : 1.f;
+            sm.t1[t] = make_float4(my_cn[j], keep ? __frcp_rn(my_cn[j]) : 0.f,
+                                   keep ? 0.f : 1.f, 0.f);
+          }
+        }
+      }
+    }
+    Slice<4, M4> S;
+    slice4_load_bst<M4>(S, bstate + ((size_t)cur.c * H + cur.h) * DD, D, r0, sg, l);
+    if (tid == 0) sh_item = atomicAdd(&hdr[kHdrFillNext], 1);
+    __syncthreads();
+    const int next = sh_item;
+    if (next < n_items)
+      fill_prefetch<D, __nv_bfloat16>(fill_item(next, H, cu, chunk_off, chunk_seq), bstate, q,
+                                      k, v, H);
+
+    float p_own;
+    {
+      float x[4];
+      slice_dot<4, M4>(S, [&](int m) { return sld4(&sm.k[0][group_col(l, m)]); }, x);
+      p_own = quad_rs(x);
+    }
+    float c = 1.f;  // scale of the running state: 1 at the chunk boundary
+    OUT* ob = o + tb * D + my_row;
+    for (int t = 0; t < cur.len; t++) {
+      const float v_own = to_f(sm.v[t][my_row]);
+      const float4 T0 = sm.t0[t], T1 = sm.t1[t];
+      const float cn = T1.x, d = T1.y, cnew = T0.w;
+      const bool keep = T1.z == 0.f;
+      const float u = step_u(T0.x, T0.y, __fmul_rn(T0.z, p_own), v_own);
+      auto fk = [&](int m) { return sld4(&sm.k[t][group_col(l, m)]); };
+      auto fq = [&](int m) { return sld4(&sm.q[t][group_col(l, m)]); };
+      auto fn = [&](int m) { return sld4(&sm.k[t + 1][group_col(l, m)]); };
+      float w[4], oacc[4], pacc[4];
+      if (keep) {
+        quad_ag(__fmul_rn(u, d), w);
+        slice_update<true, false, 4, M4>(S, cn, w, fk, fq, fn, oacc, pacc);
+      } else {
+        quad_ag(u, w);
+        slice_update<true, true, 4, M4>(S, cn, w, fk, fq, fn, oacc, pacc);
+      }
+      c = cnew;
+      p_own = quad_rs(pacc);
+      st1(ob + (size_t)t * H * D, __fmul_rn(scale, __fmul_rn(cnew, quad_rs(oacc))));
+    }
+    const int64_t nc = (cur.L + kChunk - 1) / kChunk;
+    if (s_run_final && cur.ci == nc - 1 && (cur.L % kChunk) != 0) {
+      float* dst = s_run_final + ((size_t)cur.n * H + cur.h) * DD;
+      if (s_run_scale) {
+        slice4_store<M4>(S, dst, D, r0, sg, l);
+        if (tid == 0) s_run_scale[(size_t)cur.n * H + cur.h] = c;
+      } else {
+        slice4_store_scaled<M4>(S, c, dst, D, r0, sg, l);
+      }
+    }
+    item = next;
+    __syncthreads();  // shared memory is reloaded for the next item
+  }
+}
+
+// ----------------------------------------------------------------------------
 // Chunk boundary over a buffer: decode resync (RESYNC) or gdn_chunk_boundary
 // ----------------------------------------------------------------------------
 template <int D, class IN>
@@ -588,17 +739,22 @@ __global__ void __launch_bounds__(unit_threads<D, IN>())
 }
 
 // ----------------------------------------------------------------------------
-// Decode step: one block per (row, head) unit.  The block that appends the
-// last token of a chunk then runs the chunk boundary for its unit (the
-// resync), while the other units' blocks are still stepping.
+// Decode step.  Two kernels per step on the caller's stream, running side by
+// side: k_resync first lists the units whose chunk buffer this step's token
+// completes (pos == C - 1 before the step), lets the step kernel start
+// (programmatic dependent launch) and advances those units' boundary states
+// over their C buffered tokens, the last one taken from the step's inputs;
+// k_dec_step runs the recurrence step of every unit, one block per (row,
+// head).  They touch disjoint data: k_resync reads pos before the step kernel
+// can start and writes only the listed units' boundary states and last
+// buffer row; k_dec_step reads a listed unit's running state (not its
+// boundary state) and does not write that buffer row.
 // ----------------------------------------------------------------------------
 constexpr int kDecThreads = 128;  // four state rows per thread
 
-// Words of a decode state's resync work list.
-constexpr int kResyncCount = 0;  // units listed by this step
-constexpr int kResyncNext = 1;   // work counter of k_resync
-constexpr int kResyncDone = 2;   // k_resync blocks finished
-constexpr int kResyncList = 4;   // the units
+// The resync list (rows x heads whose unit resyncs this step) lives in the
+// decode state's work array from this word on.
+constexpr int kResyncList = 4;
 
 template <int D, class IN, class OUT>
 __global__ void __launch_bounds__(kDecThreads)
@@ -606,8 +762,7 @@ __global__ void __launch_bounds__(kDecThreads)
                const float* __restrict__ beta, const float* __restrict__ g,
                const int32_t* __restrict__ slot_idx, int H, float scale, float* s_run,
                float* s_scale, float* s_bnd, IN* buf_k, IN* buf_v, float* buf_beta,
-               float* buf_g, int32_t* pos, int32_t* error, int32_t* resync, int n_slots,
-               OUT* __restrict__ o) {
+               float* buf_g, int32_t* pos, int32_t* error, int n_slots, OUT* __restrict__ o) {
   constexpr int RT = D / 32, M4 = D / 16;
   __shared__ int sh_pos, sh_slot;
   const int b = blockIdx.x, h = blockIdx.y;
@@ -652,53 +807,122 @@ __global__ void __launch_bounds__(kDecThreads)
     slice_store<RT, M4>(S, s_run + unit * DD, D, r0, l);
     if (tid == 0) s_scale[unit] = c;
   }
-  // append the token to the chunk buffer (bit copies)
-  const size_t brow = (unit * kChunk + p0) * D;
-  for (int e = tid; e < D; e += kDecThreads) {
-    buf_k[brow + e] = k[tok * D + e];
-    buf_v[brow + e] = v[tok * D + e];
-  }
-  if (tid == 0) {
-    buf_beta[unit * kChunk + p0] = bt;
-    buf_g[unit * kChunk + p0] = g[tok];
-    if (p0 + 1 < kChunk) pos[unit] = p0 + 1;
-  }
-  if (p0 + 1 == kChunk && tid == 0) {
-    // The buffer is full: k_resync advances the boundary state over its C
-    // tokens, and that becomes the running state of the next step (pos = 0).
-    const int j = atomicAdd(&resync[kResyncCount], 1);
-    if (j < n_slots * H) resync[kResyncList + j] = (int32_t)unit;
-    else atomicOr(error, kErrPos);  // rows naming the same slot twice
+  if (p0 + 1 < kChunk) {
+    // append the token to the chunk buffer (bit copies)
+    const size_t brow = (unit * kChunk + p0) * D;
+    for (int e = tid; e < D; e += kDecThreads) {
+      buf_k[brow + e] = k[tok * D + e];
+      buf_v[brow + e] = v[tok * D + e];
+    }
+    if (tid == 0) {
+      buf_beta[unit * kChunk + p0] = bt;
+      buf_g[unit * kChunk + p0] = g[tok];
+      pos[unit] = p0 + 1;
+    }
+  } else if (tid == 0) {
+    // This token completes the chunk: k_resync (running beside this kernel)
+    // appends it and advances the boundary state, which is the running state
+    // of the next step (pos = 0).
     pos[unit] = 0;
   }
 }
 
-// The chunk boundary of every unit that k_dec_step listed, in place on s_bnd.
-// Persistent blocks take list entries from a counter; the last block to
-// finish empties the list for the next step.
+// The resync of one decode step, in place on s_bnd.  Every block scans the
+// step's rows and lists, in row-major (row, head) order, the units at
+// pos == C - 1; list entry r belongs to block r mod gridDim.x.  Once the scan
+// has read pos, the step kernel may start.  Each block then, for each of its
+// entries, appends the step's token as the buffer's last row and runs the
+// chunk boundary on the unit (the same device code as the forward's first
+// pass).
 template <int D, class IN>
 __global__ void __launch_bounds__(unit_threads<D, IN>())
-    k_resync(int H, float* s_bnd, const IN* buf_k, const IN* buf_v, const float* buf_beta,
-             const float* buf_g, int32_t* resync, int n_slots, int32_t* error) {
+    k_resync(const IN* __restrict__ k, const IN* __restrict__ v, const float* __restrict__ beta,
+             const float* __restrict__ g, const int32_t* __restrict__ slot_idx, int B, int H,
+             float* s_bnd, IN* buf_k, IN* buf_v, float* buf_beta, float* buf_g,
+             const int32_t* __restrict__ pos, int32_t* list, int n_slots, int32_t* error) {
+  constexpr int NT = unit_threads<D, IN>(), NW = NT / 32;
+  constexpr int PER = 16;  // (row, head) entries per thread and scan pass
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   BndUnitSmem<D, IN>& sm = *reinterpret_cast<BndUnitSmem<D, IN>*>(smem_raw);
-  __shared__ int sh_j;
-  const int count = min(resync[kResyncCount], n_slots * H);
-  for (;;) {
-    if (threadIdx.x == 0) sh_j = atomicAdd(&resync[kResyncNext], 1);
+  __shared__ int sh_warp[NW];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int total = B * H, cap = n_slots * H;
+  const int passes = (total + NT * PER - 1) / (NT * PER);
+  int listed = 0;  // entries listed so far (the same in every thread)
+  for (int pass = 0; pass < passes; pass++) {
+    // Thread tid owns entries e0 .. e0 + PER - 1 of this pass: every load is
+    // issued before any is used.
+    const int e0 = pass * NT * PER + tid * PER;
+    int slot[PER];
+#pragma unroll
+    for (int j = 0; j < PER; j++) {
+      const int e = e0 + j;
+      slot[j] = -1;
+      if (e < total) slot[j] = slot_idx ? slot_idx[e / H] : e / H;
+    }
+    int pv[PER];
+#pragma unroll
+    for (int j = 0; j < PER; j++) {
+      const int e = e0 + j;
+      pv[j] = -1;
+      if (slot[j] >= 0 && slot[j] < n_slots) pv[j] = pos[(size_t)slot[j] * H + (e % H)];
+    }
+    unsigned flags = 0;
+#pragma unroll
+    for (int j = 0; j < PER; j++) flags |= (pv[j] == kChunk - 1 ? 1u : 0u) << j;
+    if (pass == passes - 1) {
+      // pos has been read (and used) by every thread of this block: the step
+      // kernel may start.
+      __syncthreads();
+      asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
+    // ranks: an exclusive scan of the per-thread counts over the block
+    const int cnt = __popc(flags);
+    int x = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(kFull, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) sh_warp[warp] = x;
     __syncthreads();
-    const int j = sh_j;
-    __syncthreads();  // every thread has j before thread 0 takes the next one
-    if (j >= count) break;
-    const size_t unit = (size_t)resync[kResyncList + j];
-    if (!bnd_unit<D, IN>(sm, s_bnd, buf_k, buf_v, buf_beta, buf_g, unit, s_bnd) &&
-        threadIdx.x == 0)
-      atomicOr(error, kErrTimeout);
+    int before = x - cnt, sum = 0;
+#pragma unroll
+    for (int w = 0; w < NW; w++) {
+      before += w < warp ? sh_warp[w] : 0;
+      sum += sh_warp[w];
+    }
+    int rank = listed + before;
+#pragma unroll
+    for (int j = 0; j < PER; j++) {
+      if ((flags >> j) & 1u) {
+        if (rank < cap && rank % (int)gridDim.x == (int)blockIdx.x)
+          list[kResyncList + rank] = e0 + j;
+        rank++;
+      }
+    }
+    listed += sum;
+    __syncthreads();  // sh_warp is rewritten by the next pass
   }
-  if (threadIdx.x == 0 && atomicAdd(&resync[kResyncDone], 1) == (int)gridDim.x - 1) {
-    resync[kResyncCount] = 0;  // every block has read the count and left the loop
-    resync[kResyncNext] = 0;
-    resync[kResyncDone] = 0;
+  if (listed > cap) listed = cap;
+  for (int r = blockIdx.x; r < listed; r += gridDim.x) {
+    const int e = list[kResyncList + r];
+    const int b = e / H, h = e - b * H;
+    const size_t unit = (size_t)(slot_idx ? slot_idx[b] : b) * H + h;
+    const size_t tok = (size_t)b * H + h;
+    const size_t brow = (unit * kChunk + kChunk - 1) * D;
+    for (int c = tid; c < D; c += NT) {
+      buf_k[brow + c] = k[tok * D + c];
+      buf_v[brow + c] = v[tok * D + c];
+    }
+    if (tid == 0) {
+      buf_beta[unit * kChunk + kChunk - 1] = beta[tok];
+      buf_g[unit * kChunk + kChunk - 1] = g[tok];
+    }
+    __threadfence();
+    __syncthreads();  // the row is in place before the unit's staging reads it
+    if (!bnd_unit<D, IN>(sm, s_bnd, buf_k, buf_v, buf_beta, buf_g, unit, s_bnd) && tid == 0)
+      atomicOr(error, kErrTimeout);
   }
 }
 
@@ -772,6 +996,23 @@ static cudaError_t persistent_grid(KernelT kern, int threads, size_t smem, int* 
   return cudaSuccess;
 }
 
+// The fill kernel of a (d, dtype): k_fill128 at d = 128 with bf16 inputs,
+// k_fill otherwise.  Both take the same arguments and give the same bits.
+template <int D, class IN, class OUT>
+static auto fill_kernel() {
+  if constexpr (D == 128 && sizeof(IN) == 2)
+    return k_fill128<OUT>;
+  else
+    return k_fill<D, IN, OUT>;
+}
+template <int D, class IN>
+static constexpr size_t fill_smem() {
+  if constexpr (D == 128 && sizeof(IN) == 2)
+    return sizeof(Fill128Smem);
+  else
+    return sizeof(FillSmem<D, IN>);
+}
+
 template <int D, class IN, class OUT>
 static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   static_assert(pack_size<D, IN>() == pack_bytes(D, sizeof(IN) == 2), "pack layout mismatch");
@@ -822,8 +1063,8 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   }
   GDN_TRY(mark(3));
   if (!a.pass1_only) {
-    auto kern = k_fill<D, IN, OUT>;
-    const size_t sm = sizeof(FillSmem<D, IN>);
+    auto kern = fill_kernel<D, IN, OUT>();
+    const size_t sm = fill_smem<D, IN>();
     GDN_TRY(set_smem(kern, sm));
     int grid = 0;
     GDN_TRY(persistent_grid(kern, kFillThreads, sm, &grid));
@@ -839,20 +1080,33 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
 
 template <int D, class IN, class OUT>
 static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
-  k_dec_step<D, IN, OUT><<<dim3((unsigned)a.B, (unsigned)a.H), kDecThreads, 0, st>>>(
-      static_cast<const IN*>(a.q), static_cast<const IN*>(a.k), static_cast<const IN*>(a.v),
-      a.beta, a.g, a.slot_idx, a.H, a.scale, a.s_run, a.s_scale, a.s_bnd,
-      static_cast<IN*>(a.buf_k), static_cast<IN*>(a.buf_v), a.buf_beta, a.buf_g, a.pos, a.error,
-      a.resync, a.n_slots, static_cast<OUT*>(a.o));
-  GDN_TRY(cudaGetLastError());
-  auto kern = k_resync<D, IN>;
+  auto rk = k_resync<D, IN>;
   const size_t sm = sizeof(BndUnitSmem<D, IN>);
-  GDN_TRY(set_smem(kern, sm));
+  GDN_TRY(set_smem(rk, sm));
   int grid = 0;
-  GDN_TRY(persistent_grid(kern, unit_threads<D, IN>(), sm, &grid));
-  kern<<<grid, unit_threads<D, IN>(), sm, st>>>(
-      a.H, a.s_bnd, static_cast<const IN*>(a.buf_k), static_cast<const IN*>(a.buf_v), a.buf_beta,
-      a.buf_g, a.resync, a.n_slots, a.error);
+  GDN_TRY(persistent_grid(rk, unit_threads<D, IN>(), sm, &grid));
+  rk<<<grid, unit_threads<D, IN>(), sm, st>>>(
+      static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, a.slot_idx, a.B,
+      a.H, a.s_bnd, static_cast<IN*>(a.buf_k), static_cast<IN*>(a.buf_v), a.buf_beta, a.buf_g,
+      a.pos, a.resync, a.n_slots, a.error);
+  GDN_TRY(cudaGetLastError());
+  // The step kernel may start once every resync block has read pos
+  // (programmatic dependent launch); it consumes nothing k_resync writes.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.B, (unsigned)a.H);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  GDN_TRY(cudaLaunchKernelEx(&cfg, k_dec_step<D, IN, OUT>, static_cast<const IN*>(a.q),
+                             static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta,
+                             a.g, a.slot_idx, a.H, a.scale, a.s_run, a.s_scale, a.s_bnd,
+                             static_cast<IN*>(a.buf_k), static_cast<IN*>(a.buf_v), a.buf_beta,
+                             a.buf_g, a.pos, a.error, a.n_slots, static_cast<OUT*>(a.o)));
   return cudaGetLastError();
 }
 

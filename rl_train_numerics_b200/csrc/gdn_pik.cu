@@ -21,17 +21,21 @@
 //               tensor-memory buffers (alternating), four m128 n256 k16 MMAs
 //               per K step, ascending k, a fresh accumulator at the leaf's
 //               first step; the leaf's last commit signals the epilogue;
-//   warps 2-9   epilogue: read a finished leaf back (one tile row and half the
-//               columns per thread),
-//               release its buffer, and advance the balanced tree as a binary
-//               counter: the leaf is added to the pending subtree sums of
-//               equal size, left operand first, and the result is either the
-//               unit's sum (stored) or pushed as a pending sum.  Pending sums
-//               live in a per-block slice of the workspace (one 128 KB slot
-//               per tree level, written and read by the same threads).
-// The epilogue of leaf i overlaps the MMAs of leaf i + 1.  With R > 1 ranks
-// the unit sums go to the workspace and k_pik_combine applies the levels
-// above the ranks, again neighbours first.  Whatever R is, every addition of
+//   warps 2-9   epilogue: read finished leaves back (one tile row and half the
+//               columns per thread) and advance the balanced tree.  With two
+//               or more leaves per unit they come in pairs: a pair fills both
+//               buffers and is added as it is read (the tree's lowest level,
+//               even leaf first), and both buffers are handed back at once.
+//               The pair sums go through a binary counter: a sum is added to
+//               the pending subtree sums of equal size, left operand first,
+//               and the result is either the unit's sum (stored) or pushed as
+//               a pending sum.  Pending sums live in a per-block slice of the
+//               workspace (one 128 KB slot per level, written and read by the
+//               same threads).
+// The MMAs of the next leaves wait only for the pair's tensor-memory reads,
+// not for the pending-sum traffic.  With R > 1 ranks the unit sums go to
+// the workspace and k_pik_combine applies the levels above the ranks, again
+// neighbours first.  Whatever R is, every addition of
 // the tree happens in the same order on the same operands.
 //
 // Operands: A [M, K] and B [N, K] bf16, both K-major (row-major with K
@@ -138,7 +142,7 @@ __global__ void __launch_bounds__(kPikThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m_tiles = (M + kPikBM - 1) / kPikBM, n_tiles = (N + kPikBN - 1) / kPikBN;
   const int spl = leaf_k / kPikKStep;  // K steps per leaf
-  const int depth = 31 - __clz(leaves);
+  const int depth = 31 - __clz(leaves >= 2 ? leaves / 2 : 1);  // pending-sum levels
 
   if (warp == 1) tmem_alloc(smem_u32(&sm.tmem_slot), 2 * kPikBN);
   if (tid == 0) {
@@ -229,83 +233,102 @@ __global__ void __launch_bounds__(kPikThreads, 1)
     if (!ok && lane == 0) *abort_flag = 1;
   } else {
     // Epilogue: tile row r (tensor-memory lane quarter warp % 4) and one half
-    // of the tile's columns per thread (two warps per lane quarter).
+    // of the tile's columns per thread (two warps per lane quarter).  Leaves
+    // are read in groups of G = min(leaves, 2): a pair of leaves occupies both
+    // buffers and is added (the tree's lowest level) as it is read back, then
+    // both buffers are released at once; the levels above go through the
+    // pending sums.
     const int q = warp & 3, r = q * 32 + lane, half = (warp - 2) >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    const int G = leaves >= 2 ? 2 : 1, groups = leaves / G;
     float4* my_stack = stack + (size_t)blockIdx.x * depth * (kPikBM * kPikBN / 4);
     int lc = 0;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const PikUnit w = pik_unit(u, m_tiles, n_tiles);
       const int m = w.tm * kPikBM + r, n0 = w.tn * kPikBN;
       float* orow = out + (size_t)w.z * M * N + (size_t)m * N + n0;
-      for (int leaf = 0; leaf < leaves; leaf++, lc++) {
-        const int b = lc & 1, use = lc >> 1;
-        bool got = mbar_wait(smem_u32(&sm.acc_full[b]), (uint32_t)(use & 1), kPikPolls);
+      for (int grp = 0; grp < groups; grp++) {
+        bool got = true;
+        for (int i = 0; i < G; i++)
+          got = got && mbar_wait(smem_u32(&sm.acc_full[(lc + i) & 1]),
+                                 (uint32_t)(((lc + i) >> 1) & 1), kPikPolls);
         got = __all_sync(0xffffffffu, got) && !*abort_flag;
         if (!got) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int combos = ctz32((uint32_t)(leaf + 1));  // pending sums this leaf closes
-        const bool last = leaf == leaves - 1;
-#pragma unroll 1
+        const int b0 = lc & 1;
+        float x[kPikChunksPerThread][32];
+#pragma unroll
         for (int cc = 0; cc < kPikChunksPerThread; cc++) {
-          const int c = half * kPikChunksPerThread + cc;  // 32-column chunk of the tile
-          float x[32];
-          tmem_ld32(lane_base + (uint32_t)(b * kPikBN + c * 32), x);
-          tmem_wait_ld(x);
-          if (cc == kPikChunksPerThread - 1) {
-            // this thread has read all its columns of the buffer
-            tc_fence_before();
-            mbar_arrive(smem_u32(&sm.acc_empty[b]));
+          const uint32_t col = (uint32_t)((half * kPikChunksPerThread + cc) * 32);
+          tmem_ld32(lane_base + (uint32_t)(b0 * kPikBN) + col, x[cc]);
+          if (G == 2) {
+            // the odd leaf in two 16-column halves (register pressure)
+#pragma unroll
+            for (int hh = 0; hh < 2; hh++) {
+              float y[16];
+              tmem_ld16(lane_base + (uint32_t)((b0 ^ 1) * kPikBN) + col + 16 * hh, y);
+              tmem_wait_ld(x[cc]);
+              tmem_wait_ld(y);
+#pragma unroll
+              for (int e = 0; e < 16; e++)
+                x[cc][16 * hh + e] = __fadd_rn(x[cc][16 * hh + e], y[e]);  // even + odd
+            }
+          } else {
+            tmem_wait_ld(x[cc]);
           }
-          // x = pending(level 0) + x, then pending(level 1) + x, ...: each
-          // pending sum is the left (earlier) subtree.  Two levels' loads are
-          // issued together.
+        }
+        // every column of the group's buffers has been read: hand them back
+        tc_fence_before();
+        for (int i = 0; i < G; i++) mbar_arrive(smem_u32(&sm.acc_empty[(lc + i) & 1]));
+        lc += G;
+        // x = pending(level 0) + x, then pending(level 1) + x, ...: each
+        // pending sum is the left (earlier) subtree.
+        const int combos = ctz32((uint32_t)(grp + 1));
+        const bool last = grp == groups - 1;
 #pragma unroll 1
-          for (int lev = 0; lev < combos; lev += 2) {
-            const bool two = lev + 1 < combos;
-            const float4* s0 = my_stack + ((size_t)(lev * 8 + c) * 8) * kPikBM + r;
-            const float4* s1 = s0 + (size_t)64 * kPikBM;
-            float4 y0[8], y1[8];
+        for (int lev = 0; lev < combos; lev++) {
 #pragma unroll
-            for (int f = 0; f < 8; f++) y0[f] = s0[(size_t)f * kPikBM];
-            if (two) {
+          for (int cc = 0; cc < kPikChunksPerThread; cc++) {
+            const int c = half * kPikChunksPerThread + cc;
+            const float4* src = my_stack + ((size_t)(lev * 8 + c) * 8) * kPikBM + r;
+            // four float4 loads in flight at a time (the pair sum already
+            // holds 128 registers)
 #pragma unroll
-              for (int f = 0; f < 8; f++) y1[f] = s1[(size_t)f * kPikBM];
-            }
+            for (int f0 = 0; f0 < 8; f0 += 4) {
+              float4 yv[4];
 #pragma unroll
-            for (int f = 0; f < 8; f++) {
-              x[4 * f + 0] = __fadd_rn(y0[f].x, x[4 * f + 0]);
-              x[4 * f + 1] = __fadd_rn(y0[f].y, x[4 * f + 1]);
-              x[4 * f + 2] = __fadd_rn(y0[f].z, x[4 * f + 2]);
-              x[4 * f + 3] = __fadd_rn(y0[f].w, x[4 * f + 3]);
-            }
-            if (two) {
+              for (int f = 0; f < 4; f++) yv[f] = src[(size_t)(f0 + f) * kPikBM];
 #pragma unroll
-              for (int f = 0; f < 8; f++) {
-                x[4 * f + 0] = __fadd_rn(y1[f].x, x[4 * f + 0]);
-                x[4 * f + 1] = __fadd_rn(y1[f].y, x[4 * f + 1]);
-                x[4 * f + 2] = __fadd_rn(y1[f].z, x[4 * f + 2]);
-                x[4 * f + 3] = __fadd_rn(y1[f].w, x[4 * f + 3]);
+              for (int f = 0; f < 4; f++) {
+                x[cc][4 * (f0 + f) + 0] = __fadd_rn(yv[f].x, x[cc][4 * (f0 + f) + 0]);
+                x[cc][4 * (f0 + f) + 1] = __fadd_rn(yv[f].y, x[cc][4 * (f0 + f) + 1]);
+                x[cc][4 * (f0 + f) + 2] = __fadd_rn(yv[f].z, x[cc][4 * (f0 + f) + 2]);
+                x[cc][4 * (f0 + f) + 3] = __fadd_rn(yv[f].w, x[cc][4 * (f0 + f) + 3]);
               }
+              asm volatile("" ::: "memory");
             }
           }
+        }
+#pragma unroll
+        for (int cc = 0; cc < kPikChunksPerThread; cc++) {
+          const int c = half * kPikChunksPerThread + cc;
           if (last) {
             if (m < M) {
 #pragma unroll
               for (int f = 0; f < 8; f++)
                 if (n0 + c * 32 + 4 * f < N)
-                  *reinterpret_cast<float4*>(orow + c * 32 + 4 * f) =
-                      make_float4(x[4 * f], x[4 * f + 1], x[4 * f + 2], x[4 * f + 3]);
+                  *reinterpret_cast<float4*>(orow + c * 32 + 4 * f) = make_float4(
+                      x[cc][4 * f], x[cc][4 * f + 1], x[cc][4 * f + 2], x[cc][4 * f + 3]);
             }
           } else {
             float4* dst = my_stack + ((size_t)(combos * 8 + c) * 8) * kPikBM + r;
 #pragma unroll
             for (int f = 0; f < 8; f++)
-              dst[(size_t)f * kPikBM] = make_float4(x[4 * f], x[4 * f + 1], x[4 * f + 2],
-                                                    x[4 * f + 3]);
+              dst[(size_t)f * kPikBM] = make_float4(x[cc][4 * f], x[cc][4 * f + 1],
+                                                    x[cc][4 * f + 2], x[cc][4 * f + 3]);
           }
         }
       }
@@ -388,8 +411,8 @@ PikPlan pik_plan(int64_t M, int64_t N, int L, int R) {
   const int64_t tiles = ((M + kPikBM - 1) / kPikBM) * ((N + kPikBN - 1) / kPikBN);
   p.units = (int)(tiles * R);
   p.blocks = p.units < kPikMaxBlocks ? p.units : kPikMaxBlocks;
-  p.depth = 0;
-  while ((1 << p.depth) < p.leaves) p.depth++;
+  p.depth = 0;  // levels of pending sums: the tree over the unit's leaf pairs
+  while ((2 << p.depth) < p.leaves) p.depth++;
   p.ws_ranks = R > 1 ? (size_t)R * (size_t)M * (size_t)N * sizeof(float) : 0;
   p.ws_stack = (size_t)p.blocks * p.depth * kPikBM * kPikBN * sizeof(float);
   return p;

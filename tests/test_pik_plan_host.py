@@ -1,9 +1,10 @@
 """Host-side checks of the K-leaf GEMM's work split (no GPU).
 
 gdn_pik_gemm runs one work unit per 128 x 256 tile and emulated rank: the
-rank's L / R leaves, added in the kernel by the balanced tree evaluated as a
-binary counter (pending subtree sums in a per-block workspace slice, one
-128 x 256 fp32 slot per tree level, at most 148 persistent blocks).  With
+rank's L / R leaves, added in the kernel by the balanced tree: leaf pairs
+first, then a binary counter over the pair sums (pending subtree sums in a
+per-block workspace slice, one 128 x 256 fp32 slot per level above the pairs,
+at most 148 persistent blocks).  With
 R > 1 the rank sums go to the workspace (one fp32 M x N slice per rank) and a
 combine kernel applies the levels above the ranks with the same counter.  The
 split is read back through gdn_pik_workspace_bytes; the counter's order of
@@ -27,7 +28,7 @@ def test_workspace_for_every_rank_count(L):
     tiles = (M // 128) * (N // 256)
     R = 1
     while R <= L:
-        depth = int(np.log2(L // R))
+        depth = int(np.log2(max(L // R // 2, 1)))  # pending sums over leaf pairs
         blocks = min(tiles * R, 148)
         want = (R * M * N * 4 if R > 1 else 0) + blocks * depth * 128 * 256 * 4
         assert gdn.pik_workspace_bytes(M, N, K, L, R) == want, (L, R)
