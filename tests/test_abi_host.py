@@ -196,7 +196,7 @@ def pik(**over):
     (dict(err=None), gdn.GDN_ERR_INVALID_ARG),
     (dict(C=MIS), gdn.GDN_ERR_INVALID_ARG),
     (dict(err=MIS + 2), gdn.GDN_ERR_INVALID_ARG),
-    (dict(ws=None), gdn.GDN_ERR_WORKSPACE),         # 8 leaves: four groups of two
+    (dict(ws=None), gdn.GDN_ERR_WORKSPACE),         # 8 leaves: pending sums above 4 pairs
     (dict(L=16, wsb=16), gdn.GDN_ERR_WORKSPACE),
 ])
 def test_pik_rejects_on_host(over, expect):
@@ -205,11 +205,12 @@ def test_pik_rejects_on_host(over, expect):
 
 def test_pik_workspace_and_empty_shapes():
     w = gdn.pik_workspace_bytes
-    assert w(256, 256, 1024, 2, 1) == 0           # one group of 2 leaves: no workspace
+    slot = 128 * 256 * 4  # one pending sum of a 128 x 256 tile
+    assert w(256, 256, 1024, 2, 1) == 0           # one pair of leaves: no pending sums
     assert w(256, 256, 1024, 1, 1) == 0
-    assert w(256, 256, 1024, 8, 1) == 4 * 256 * 256 * 4   # four groups of two leaves
-    assert w(256, 256, 1024, 16, 1) == 8 * 256 * 256 * 4
-    assert w(256, 256, 1024, 8, 8) == 8 * 256 * 256 * 4
+    assert w(256, 256, 1024, 8, 1) == 2 * 2 * slot     # 2 blocks x 2 levels above 4 pairs
+    assert w(256, 256, 1024, 16, 1) == 2 * 3 * slot
+    assert w(256, 256, 1024, 8, 8) == 8 * 256 * 256 * 4   # 8 rank sums, one leaf each
     assert w(256, 200, 1024, 8, 1) == 0 and w(256, 256, 1024, 3, 1) == 0
     assert pik(M=0, A=None, B=None, C=None, err=None) == gdn.GDN_OK
     assert pik(N=0, A=None, B=None, C=None, err=None) == gdn.GDN_OK
