@@ -139,3 +139,61 @@ def test_adjoint_chunk_map_is_the_transposed_boundary_map():
     mu_e = rng.normal(size=(d, d))
     W_loc = adjoint(np.zeros((d, d)))
     assert np.allclose(adjoint(mu_e), mu_e @ Pt + W_loc, rtol=0, atol=1e-12)
+
+
+def chunked_adjoint(q, k, beta, g, cu, do, dsf, scale, C, n, h):
+    """The chunk form of the adjoint (the CUDA backward runs the token
+    recurrence; this form is what a chunk-parallel adjoint evaluates): per
+    chunk (in parallel)
+    Z = (I + A)^{-T} R, Y = (I + A)^{-T} diag(e^{G_{L-1} - G}) K and
+    W_loc = scale DO^T diag(e^G) Q - Z^T diag(beta e^G) K; then a reverse walk
+    over the chunks, mu_a = e^{G_{L-1}} mu_e - (mu_e Y^T) diag(beta e^G) K + W_loc;
+    then W = Z + Y mu_e^T per chunk.  Returns (W, mu at every chunk end, dh0)."""
+    a0, e0 = int(cu[n]), int(cu[n + 1])
+    d = q.shape[2]
+    W, mu_end, pre = np.zeros((e0 - a0, d)), {}, {}
+    for a in range(a0, e0, C):
+        e = min(a + C, e0)
+        L = e - a
+        G = np.cumsum(g[a:e, h])
+        K, Q, DO, bt = k[a:e, h], q[a:e, h], do[a:e, h], beta[a:e, h]
+        ii = np.arange(L)
+        A = (np.where(ii[:, None] > ii[None, :], np.exp(G[:, None] - G[None, :]), 0.0)
+             * (K @ K.T) * bt[:, None])                        # A[r, t], r > t
+        M = np.where(ii[None, :] >= ii[:, None], np.exp(G[None, :] - G[:, None]), 0.0) * (K @ Q.T)
+        I_A = np.eye(L) + A
+        Z = np.linalg.solve(I_A.T, scale * M @ DO)
+        Y = np.linalg.solve(I_A.T, np.exp(G[-1] - G)[:, None] * K)
+        bg = bt * np.exp(G)
+        Wl = scale * DO.T @ (np.exp(G)[:, None] * Q) - Z.T @ (bg[:, None] * K)
+        pre[a] = (Z, Y, bg, K, np.exp(G[-1]), Wl)
+    mu = dsf[n, h].copy()
+    for a in reversed(range(a0, e0, C)):
+        e = min(a + C, e0)
+        Z, Y, bg, K, gam, Wl = pre[a]
+        mu_end[e] = mu.copy()
+        W[a - a0:e - a0] = Z + Y @ mu.T
+        mu = gam * mu - ((mu @ Y.T) * bg[None, :]) @ K + Wl
+    return W, mu_end, mu
+
+
+@pytest.mark.parametrize("C", [1, 3, 16, 64])
+def test_chunked_adjoint_equals_the_token_recurrence(C):
+    q, k, v, beta, g, cu, h0, do, dsf = _batch([1, 63, 64, 65, 130, 0, 7], 2, 6, seed=10 + C)
+    scale = 0.6
+    for n in range(len(cu) - 1):
+        a0, e0 = int(cu[n]), int(cu[n + 1])
+        for h in range(2):
+            mu, W, ends = dsf[n, h].copy(), np.zeros((e0 - a0, 6)), {}
+            for j in range(e0 - 1, a0 - 1, -1):
+                if (j - a0) % C == C - 1 or j == e0 - 1:
+                    ends[j + 1] = mu.copy()
+                lam = mu + scale * np.outer(do[j, h], q[j, h])
+                W[j - a0] = lam @ k[j, h]
+                mu = np.exp(g[j, h]) * (lam - beta[j, h] * np.outer(W[j - a0], k[j, h]))
+            W2, ends2, mu2 = chunked_adjoint(q, k, beta, g, cu, do, dsf, scale, C, n, h)
+            assert np.max(np.abs(W2 - W), initial=0.0) < 1e-12
+            assert np.max(np.abs(mu2 - mu)) < 1e-12
+            assert ends.keys() == ends2.keys()
+            for e in ends:
+                assert np.max(np.abs(ends2[e] - ends[e])) < 1e-12
