@@ -739,22 +739,17 @@ __global__ void __launch_bounds__(unit_threads<D, IN>())
 }
 
 // ----------------------------------------------------------------------------
-// Decode step.  Two kernels per step on the caller's stream, running side by
-// side: k_resync first lists the units whose chunk buffer this step's token
-// completes (pos == C - 1 before the step), lets the step kernel start
-// (programmatic dependent launch) and advances those units' boundary states
-// over their C buffered tokens, the last one taken from the step's inputs;
-// k_dec_step runs the recurrence step of every unit, one block per (row,
-// head).  They touch disjoint data: k_resync reads pos before the step kernel
-// can start and writes only the listed units' boundary states and last
-// buffer row; k_dec_step reads a listed unit's running state (not its
-// boundary state) and does not write that buffer row.
+// Decode step: one block per (row, head) unit.  The block that appends the
+// last token of a chunk then runs the chunk boundary for its unit (the
+// resync), while the other units' blocks are still stepping.
 // ----------------------------------------------------------------------------
 constexpr int kDecThreads = 128;  // four state rows per thread
 
-// The resync list (rows x heads whose unit resyncs this step) lives in the
-// decode state's work array from this word on.
-constexpr int kResyncList = 4;
+// Words of a decode state's resync work list.
+constexpr int kResyncCount = 0;  // units listed by this step
+constexpr int kResyncNext = 1;   // work counter of k_resync
+constexpr int kResyncDone = 2;   // k_resync blocks finished
+constexpr int kResyncList = 4;   // the units
 
 template <int D, class IN, class OUT>
 __global__ void __launch_bounds__(kDecThreads)
@@ -762,7 +757,8 @@ __global__ void __launch_bounds__(kDecThreads)
                const float* __restrict__ beta, const float* __restrict__ g,
                const int32_t* __restrict__ slot_idx, int H, float scale, float* s_run,
                float* s_scale, float* s_bnd, IN* buf_k, IN* buf_v, float* buf_beta,
-               float* buf_g, int32_t* pos, int32_t* error, int n_slots, OUT* __restrict__ o) {
+               float* buf_g, int32_t* pos, int32_t* error, int32_t* resync, int n_slots,
+               OUT* __restrict__ o) {
   constexpr int RT = D / 32, M4 = D / 16;
   __shared__ int sh_pos, sh_slot;
   const int b = blockIdx.x, h = blockIdx.y;
@@ -807,122 +803,53 @@ __global__ void __launch_bounds__(kDecThreads)
     slice_store<RT, M4>(S, s_run + unit * DD, D, r0, l);
     if (tid == 0) s_scale[unit] = c;
   }
-  if (p0 + 1 < kChunk) {
-    // append the token to the chunk buffer (bit copies)
-    const size_t brow = (unit * kChunk + p0) * D;
-    for (int e = tid; e < D; e += kDecThreads) {
-      buf_k[brow + e] = k[tok * D + e];
-      buf_v[brow + e] = v[tok * D + e];
-    }
-    if (tid == 0) {
-      buf_beta[unit * kChunk + p0] = bt;
-      buf_g[unit * kChunk + p0] = g[tok];
-      pos[unit] = p0 + 1;
-    }
-  } else if (tid == 0) {
-    // This token completes the chunk: k_resync (running beside this kernel)
-    // appends it and advances the boundary state, which is the running state
-    // of the next step (pos = 0).
+  // append the token to the chunk buffer (bit copies)
+  const size_t brow = (unit * kChunk + p0) * D;
+  for (int e = tid; e < D; e += kDecThreads) {
+    buf_k[brow + e] = k[tok * D + e];
+    buf_v[brow + e] = v[tok * D + e];
+  }
+  if (tid == 0) {
+    buf_beta[unit * kChunk + p0] = bt;
+    buf_g[unit * kChunk + p0] = g[tok];
+    if (p0 + 1 < kChunk) pos[unit] = p0 + 1;
+  }
+  if (p0 + 1 == kChunk && tid == 0) {
+    // The buffer is full: k_resync advances the boundary state over its C
+    // tokens, and that becomes the running state of the next step (pos = 0).
+    const int j = atomicAdd(&resync[kResyncCount], 1);
+    if (j < n_slots * H) resync[kResyncList + j] = (int32_t)unit;
+    else atomicOr(error, kErrPos);  // rows naming the same slot twice
     pos[unit] = 0;
   }
 }
 
-// The resync of one decode step, in place on s_bnd.  Every block scans the
-// step's rows and lists, in row-major (row, head) order, the units at
-// pos == C - 1; list entry r belongs to block r mod gridDim.x.  Once the scan
-// has read pos, the step kernel may start.  Each block then, for each of its
-// entries, appends the step's token as the buffer's last row and runs the
-// chunk boundary on the unit (the same device code as the forward's first
-// pass).
+// The chunk boundary of every unit that k_dec_step listed, in place on s_bnd.
+// Persistent blocks take list entries from a counter; the last block to
+// finish empties the list for the next step.
 template <int D, class IN>
 __global__ void __launch_bounds__(unit_threads<D, IN>())
-    k_resync(const IN* __restrict__ k, const IN* __restrict__ v, const float* __restrict__ beta,
-             const float* __restrict__ g, const int32_t* __restrict__ slot_idx, int B, int H,
-             float* s_bnd, IN* buf_k, IN* buf_v, float* buf_beta, float* buf_g,
-             const int32_t* __restrict__ pos, int32_t* list, int n_slots, int32_t* error) {
-  constexpr int NT = unit_threads<D, IN>(), NW = NT / 32;
-  constexpr int PER = 16;  // (row, head) entries per thread and scan pass
+    k_resync(int H, float* s_bnd, const IN* buf_k, const IN* buf_v, const float* buf_beta,
+             const float* buf_g, int32_t* resync, int n_slots, int32_t* error) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   BndUnitSmem<D, IN>& sm = *reinterpret_cast<BndUnitSmem<D, IN>*>(smem_raw);
-  __shared__ int sh_warp[NW];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int total = B * H, cap = n_slots * H;
-  const int passes = (total + NT * PER - 1) / (NT * PER);
-  int listed = 0;  // entries listed so far (the same in every thread)
-  for (int pass = 0; pass < passes; pass++) {
-    // Thread tid owns entries e0 .. e0 + PER - 1 of this pass: every load is
-    // issued before any is used.
-    const int e0 = pass * NT * PER + tid * PER;
-    int slot[PER];
-#pragma unroll
-    for (int j = 0; j < PER; j++) {
-      const int e = e0 + j;
-      slot[j] = -1;
-      if (e < total) slot[j] = slot_idx ? slot_idx[e / H] : e / H;
-    }
-    int pv[PER];
-#pragma unroll
-    for (int j = 0; j < PER; j++) {
-      const int e = e0 + j;
-      pv[j] = -1;
-      if (slot[j] >= 0 && slot[j] < n_slots) pv[j] = pos[(size_t)slot[j] * H + (e % H)];
-    }
-    unsigned flags = 0;
-#pragma unroll
-    for (int j = 0; j < PER; j++) flags |= (pv[j] == kChunk - 1 ? 1u : 0u) << j;
-    if (pass == passes - 1) {
-      // pos has been read (and used) by every thread of this block: the step
-      // kernel may start.
-      __syncthreads();
-      asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    }
-    // ranks: an exclusive scan of the per-thread counts over the block
-    const int cnt = __popc(flags);
-    int x = cnt;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(kFull, x, off);
-      if (lane >= off) x += y;
-    }
-    if (lane == 31) sh_warp[warp] = x;
+  __shared__ int sh_j;
+  const int count = min(resync[kResyncCount], n_slots * H);
+  for (;;) {
+    if (threadIdx.x == 0) sh_j = atomicAdd(&resync[kResyncNext], 1);
     __syncthreads();
-    int before = x - cnt, sum = 0;
-#pragma unroll
-    for (int w = 0; w < NW; w++) {
-      before += w < warp ? sh_warp[w] : 0;
-      sum += sh_warp[w];
-    }
-    int rank = listed + before;
-#pragma unroll
-    for (int j = 0; j < PER; j++) {
-      if ((flags >> j) & 1u) {
-        if (rank < cap && rank % (int)gridDim.x == (int)blockIdx.x)
-          list[kResyncList + rank] = e0 + j;
-        rank++;
-      }
-    }
-    listed += sum;
-    __syncthreads();  // sh_warp is rewritten by the next pass
-  }
-  if (listed > cap) listed = cap;
-  for (int r = blockIdx.x; r < listed; r += gridDim.x) {
-    const int e = list[kResyncList + r];
-    const int b = e / H, h = e - b * H;
-    const size_t unit = (size_t)(slot_idx ? slot_idx[b] : b) * H + h;
-    const size_t tok = (size_t)b * H + h;
-    const size_t brow = (unit * kChunk + kChunk - 1) * D;
-    for (int c = tid; c < D; c += NT) {
-      buf_k[brow + c] = k[tok * D + c];
-      buf_v[brow + c] = v[tok * D + c];
-    }
-    if (tid == 0) {
-      buf_beta[unit * kChunk + kChunk - 1] = beta[tok];
-      buf_g[unit * kChunk + kChunk - 1] = g[tok];
-    }
-    __threadfence();
-    __syncthreads();  // the row is in place before the unit's staging reads it
-    if (!bnd_unit<D, IN>(sm, s_bnd, buf_k, buf_v, buf_beta, buf_g, unit, s_bnd) && tid == 0)
+    const int j = sh_j;
+    __syncthreads();  // every thread has j before thread 0 takes the next one
+    if (j >= count) break;
+    const size_t unit = (size_t)resync[kResyncList + j];
+    if (!bnd_unit<D, IN>(sm, s_bnd, buf_k, buf_v, buf_beta, buf_g, unit, s_bnd) &&
+        threadIdx.x == 0)
       atomicOr(error, kErrTimeout);
+  }
+  if (threadIdx.x == 0 && atomicAdd(&resync[kResyncDone], 1) == (int)gridDim.x - 1) {
+    resync[kResyncCount] = 0;  // every block has read the count and left the loop
+    resync[kResyncNext] = 0;
+    resync[kResyncDone] = 0;
   }
 }
 
@@ -1080,33 +1007,20 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
 
 template <int D, class IN, class OUT>
 static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
-  auto rk = k_resync<D, IN>;
-  const size_t sm = sizeof(BndUnitSmem<D, IN>);
-  GDN_TRY(set_smem(rk, sm));
-  int grid = 0;
-  GDN_TRY(persistent_grid(rk, unit_threads<D, IN>(), sm, &grid));
-  rk<<<grid, unit_threads<D, IN>(), sm, st>>>(
-      static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, a.slot_idx, a.B,
-      a.H, a.s_bnd, static_cast<IN*>(a.buf_k), static_cast<IN*>(a.buf_v), a.buf_beta, a.buf_g,
-      a.pos, a.resync, a.n_slots, a.error);
+  k_dec_step<D, IN, OUT><<<dim3((unsigned)a.B, (unsigned)a.H), kDecThreads, 0, st>>>(
+      static_cast<const IN*>(a.q), static_cast<const IN*>(a.k), static_cast<const IN*>(a.v),
+      a.beta, a.g, a.slot_idx, a.H, a.scale, a.s_run, a.s_scale, a.s_bnd,
+      static_cast<IN*>(a.buf_k), static_cast<IN*>(a.buf_v), a.buf_beta, a.buf_g, a.pos, a.error,
+      a.resync, a.n_slots, static_cast<OUT*>(a.o));
   GDN_TRY(cudaGetLastError());
-  // The step kernel may start once every resync block has read pos
-  // (programmatic dependent launch); it consumes nothing k_resync writes.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)a.B, (unsigned)a.H);
-  cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  GDN_TRY(cudaLaunchKernelEx(&cfg, k_dec_step<D, IN, OUT>, static_cast<const IN*>(a.q),
-                             static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta,
-                             a.g, a.slot_idx, a.H, a.scale, a.s_run, a.s_scale, a.s_bnd,
-                             static_cast<IN*>(a.buf_k), static_cast<IN*>(a.buf_v), a.buf_beta,
-                             a.buf_g, a.pos, a.error, a.n_slots, static_cast<OUT*>(a.o)));
+  auto kern = k_resync<D, IN>;
+  const size_t sm = sizeof(BndUnitSmem<D, IN>);
+  GDN_TRY(set_smem(kern, sm));
+  int grid = 0;
+  GDN_TRY(persistent_grid(kern, unit_threads<D, IN>(), sm, &grid));
+  kern<<<grid, unit_threads<D, IN>(), sm, st>>>(
+      a.H, a.s_bnd, static_cast<const IN*>(a.buf_k), static_cast<const IN*>(a.buf_v), a.buf_beta,
+      a.buf_g, a.resync, a.n_slots, a.error);
   return cudaGetLastError();
 }
 
