@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define GDN_CPR_ABI_VERSION 6
+#define GDN_CPR_ABI_VERSION 7
 
 typedef enum {
   GDN_OK = 0,
@@ -268,6 +268,54 @@ int gdn_cpr_decode_step(const void* q, const void* k, const void* v, int in_dtyp
 int gdn_chunk_boundary(const float* s_start, const void* k, const void* v, int in_dtype,
                        const float* beta, const float* g, int B, int H, int dk, int dv, int C,
                        float* s_end, void* stream);
+
+/*
+ * gdn_recurrent_forward -- the "recurrent everywhere" forward: the per-token
+ * recurrence from h0 over every token of each sequence, with no chunk
+ * boundaries.
+ *
+ * Defines: the section "Solving the linear-attention headache" and its
+ * per-layer table, whose second column runs the recurrent form for training,
+ * prefill and decode alike (one rounding schedule, a serial sweep over every
+ * token).  Each token runs the same step as gdn_cpr_forward's fill and
+ * gdn_cpr_decode_step (the running state kept as scale x mantissa), so:
+ * the first C tokens of every sequence give bitwise gdn_cpr_forward's
+ * outputs, and a forward over a prefix that returns (s_final, s_final_scale)
+ * continued by gdn_recurrent_decode_step gives bitwise the forward over the
+ * whole sequence.
+ * Arguments as gdn_cpr_forward (C is fixed at 64 and not passed; no
+ * workspace): q, k [T, H, dk], v [T, H, dv] in_dtype; beta, g [T, H] fp32;
+ * cu_seqlens [n_seqs + 1] int32 on the device; h0 [n_seqs, H, dv, dk] fp32
+ * or NULL; o [T, H, dv] out_dtype.
+ * s_final [n_seqs, H, dv, dk] fp32 or NULL: the state after each sequence's
+ * last token; with s_final_scale ([n_seqs, H] fp32) it holds the mantissa and
+ * s_final_scale the scale, else the state itself.
+ * error_word: optional device int32 (4-byte aligned), cleared by the call;
+ * cu_seqlens that do not start at 0, decrease or do not end at total_tokens
+ * set GDN_DEVERR_CU_SEQLENS there and leave the offending sequences'
+ * outputs unwritten.  Host-side errors are returned before any device work.
+ * Supported shapes: dk = dv = 64 (bf16 or fp32 inputs) or 128 (bf16 inputs).
+ */
+int gdn_recurrent_forward(const void* q, const void* k, const void* v, int in_dtype,
+                          const float* beta, const float* g, const int32_t* cu_seqlens,
+                          int n_seqs, int64_t total_tokens, int H, int dk, int dv, float scale,
+                          const float* h0, void* o, int out_dtype, float* s_final,
+                          float* s_final_scale, int32_t* error_word, void* stream);
+
+/*
+ * gdn_recurrent_decode_step -- one batched step of the recurrent-everywhere
+ * decode: the step of gdn_cpr_decode_step without the chunk buffer and the
+ * resync.  For row b and head h: from the running state
+ * s_scale[b,h] x s[b,h], one token gives o[b,h]; (s, s_scale) are updated in
+ * place (mantissa and scale).
+ * q, k [B, H, dk], v [B, H, dv] in_dtype; beta, g [B, H] fp32;
+ * s [B, H, dv, dk] fp32; s_scale [B, H] fp32; o [B, H, dv] out_dtype.
+ * A state that starts from a full state X uses (s = X, s_scale = 1).
+ */
+int gdn_recurrent_decode_step(const void* q, const void* k, const void* v, int in_dtype,
+                              const float* beta, const float* g, int B, int H, int dk, int dv,
+                              float scale, float* s, float* s_scale, void* o, int out_dtype,
+                              void* stream);
 
 /*
  * Bytes of device workspace gdn_cpr_backward needs for this problem size.

@@ -74,6 +74,10 @@ def _load() -> ctypes.CDLL:
         "gdn_cpr_decode_step": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32,
                                       DecodeStateStruct, vp, i32, vp]),
         "gdn_chunk_boundary": (i32, [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
+        "gdn_recurrent_forward": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, f32,
+                                        vp, vp, i32, vp, vp, vp, vp]),
+        "gdn_recurrent_decode_step": (i32, [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, f32, vp,
+                                            vp, vp, i32, vp]),
         "gdn_cpr_backward_workspace_bytes": (sz, [i32, i64, i32, i32, i32, i32, i32]),
         "gdn_cpr_backward": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32,
                                    f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, vp]),
@@ -193,6 +197,50 @@ def forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=No
                                 _stream(stream))
     _check(st, "gdn_cpr_forward")
     return o, s_run_final, s_bnd_final, workspace
+
+
+def recurrent_forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=None,
+                      scale: float = 1.0, out_dtype=None, o=None, s_final=None,
+                      s_final_scale=None, want_state: bool = True, error=None, stream=None):
+    """gdn_recurrent_forward (the recurrent-everywhere forward).  Returns
+    (o, s_final, s_final_scale, error word).  s_final is the state itself
+    unless an ``s_final_scale`` tensor [N, H] fp32 is passed: then s_final
+    holds the mantissa and s_final_scale the scale."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = (cu_seqlens.numel() - 1) if n_seqs is None else int(n_seqs)
+    in_code = _dtype_code(q)
+    out_code = _out_code(in_code, out_dtype, o)
+    dev = q.device
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=_torch_dtype(out_code), device=dev)
+    if want_state and s_final is None:
+        s_final = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    if error is None:
+        error = torch.zeros(1, dtype=torch.int32, device=dev)
+    st = lib.gdn_recurrent_forward(_ptr(q), _ptr(k), _ptr(v), in_code, _ptr(beta), _ptr(g),
+                                   _ptr(cu_seqlens), N, T, H, dk, dv, float(scale), _ptr(h0),
+                                   _ptr(o), out_code, _ptr(s_final), _ptr(s_final_scale),
+                                   _ptr(error), _stream(stream))
+    _check(st, "gdn_recurrent_forward")
+    return o, s_final, s_final_scale, error
+
+
+def recurrent_decode_step(q, k, v, beta, g, s, s_scale, *, scale: float = 1.0, out_dtype=None,
+                          o=None, stream=None):
+    """gdn_recurrent_decode_step: one token per row b; (s, s_scale) updated in
+    place.  q, k, v [B, H, d]; beta, g [B, H].  Returns o [B, H, dv]."""
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    in_code = _dtype_code(q)
+    out_code = _out_code(in_code, out_dtype, o)
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=_torch_dtype(out_code), device=q.device)
+    st = lib.gdn_recurrent_decode_step(_ptr(q), _ptr(k), _ptr(v), in_code, _ptr(beta), _ptr(g),
+                                       B, H, dk, dv, float(scale), _ptr(s), _ptr(s_scale),
+                                       _ptr(o), out_code, _stream(stream))
+    _check(st, "gdn_recurrent_decode_step")
+    return o
 
 
 def backward_workspace_bytes(n_seqs: int, total_tokens: int, H: int, dk: int, dv: int,

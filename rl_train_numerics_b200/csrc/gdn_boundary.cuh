@@ -129,10 +129,11 @@ using PrepAT = float[kChunk][kChunk];
 // (core-matrix layout) written with plain loads and stores: bf16 inputs are
 // copied, fp32 inputs split into three bf16 terms.  A warp takes 8 rows x 4
 // column groups of bf16 input: 64 contiguous bytes of each row, 128
-// contiguous destination bytes per quarter warp.
+// contiguous destination bytes per quarter warp.  Rows at or past `rows`
+// are written as zeros (a chunk's padding past its length).
 template <int D, class IN>
 __device__ __forceinline__ void copy_planes(__nv_bfloat16 (*dst)[kChunk * D], const IN* src,
-                                            size_t ld, int nthreads) {
+                                            size_t ld, int nthreads, int rows = kChunk) {
   constexpr int NK = Splits<IN>::K;
   if constexpr (NK == 1) {
     constexpr int P = D / 8;  // 16-byte pieces per row
@@ -141,13 +142,14 @@ __device__ __forceinline__ void copy_planes(__nv_bfloat16 (*dst)[kChunk * D], co
       const int w = e >> 5, l = e & 31;
       const int cg = (w % (P / 4)) * 4 + (l >> 3), r = (w / (P / 4)) * 8 + (l & 7);
       *reinterpret_cast<uint4*>(&dst[0][core_off<kChunk>(r, 8 * cg)]) =
-          *reinterpret_cast<const uint4*>(src + (size_t)r * ld + 8 * cg);
+          r < rows ? *reinterpret_cast<const uint4*>(src + (size_t)r * ld + 8 * cg)
+                   : make_uint4(0u, 0u, 0u, 0u);
     }
   } else {
     constexpr int G4 = D / 4;
     for (int e = threadIdx.x; e < kChunk * G4; e += nthreads) {
       const int r = e / G4, c = (e % G4) * 4;
-      const float4 x4 = ld4(src + (size_t)r * ld + c);
+      const float4 x4 = r < rows ? ld4(src + (size_t)r * ld + c) : make_float4(0.f, 0.f, 0.f, 0.f);
       const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
       for (int q = 0; q < 4; q++) {
@@ -180,12 +182,14 @@ struct PlaneRows {
       c = (e % kPerRow) * 4;
     }
   }
-  __device__ __forceinline__ void load(const IN* src, size_t ld) {
+  // Rows at or past `rows` load as zeros.
+  __device__ __forceinline__ void load(const IN* src, size_t ld, int rows = kChunk) {
 #pragma unroll
     for (int j = 0; j < kPieces; j++) {
       int r, c;
       where((int)threadIdx.x + j * NT, r, c);
-      x[j] = *reinterpret_cast<const uint4*>(src + (size_t)r * ld + c);
+      x[j] = r < rows ? *reinterpret_cast<const uint4*>(src + (size_t)r * ld + c)
+                      : make_uint4(0u, 0u, 0u, 0u);
     }
   }
   __device__ __forceinline__ void store(__nv_bfloat16 (*dst)[kChunk * D]) const {
@@ -211,19 +215,22 @@ struct PlaneRows {
 };
 
 // The same into shared memory; bf16 inputs go with cp.async (the caller
-// commits and waits).
+// commits and waits).  Rows at or past `rows` are written as zeros.
 template <int D, class IN>
 __device__ __forceinline__ void stage_planes(__nv_bfloat16 (*dst)[kChunk * D], const IN* src,
-                                             size_t ld, int nthreads) {
+                                             size_t ld, int nthreads, int rows = kChunk) {
   if constexpr (Splits<IN>::K == 1) {
     constexpr int P = D / 8;
     for (int e = threadIdx.x; e < kChunk * P; e += nthreads) {
       const int w = e >> 5, l = e & 31;
       const int cg = (w % (P / 4)) * 4 + (l >> 3), r = (w / (P / 4)) * 8 + (l & 7);
-      cp_async16(&dst[0][core_off<kChunk>(r, 8 * cg)], src + (size_t)r * ld + 8 * cg);
+      if (r < rows)
+        cp_async16(&dst[0][core_off<kChunk>(r, 8 * cg)], src + (size_t)r * ld + 8 * cg);
+      else
+        *reinterpret_cast<uint4*>(&dst[0][core_off<kChunk>(r, 8 * cg)]) = make_uint4(0u, 0u, 0u, 0u);
     }
   } else {
-    copy_planes<D, IN>(dst, src, ld, nthreads);
+    copy_planes<D, IN>(dst, src, ld, nthreads, rows);
   }
 }
 
@@ -254,15 +261,18 @@ __device__ __forceinline__ const __nv_bfloat16* bfrag_kn_addr(const __nv_bfloat1
 }
 
 // Stage one chunk for the prep: keys (rows at stride ld), beta and g
-// (stride ldbg).  Ends with the data landed and a block barrier.
+// (stride ldbg).  Tokens at or past `rows` (the padding of a chunk shorter
+// than C) stage as zeros: beta = g = 0 and a zero key make them identity
+// steps.  Ends with the data landed and a block barrier.
 template <int D, class IN>
 __device__ __forceinline__ void prep_stage(PrepSmem<D, IN>& sm, const IN* k, size_t ld,
-                                           const float* bsrc, const float* gsrc, size_t ldbg) {
-  stage_planes<D, IN>(sm.K, k, ld, (int)blockDim.x);
+                                           const float* bsrc, const float* gsrc, size_t ldbg,
+                                           int rows = kChunk) {
+  stage_planes<D, IN>(sm.K, k, ld, (int)blockDim.x, rows);
   cp_async_commit();
   for (int i = threadIdx.x; i < kChunk; i += kBndThreads) {
-    sm.beta[i] = bsrc[i * ldbg];
-    sm.g[i] = gsrc[i * ldbg];
+    sm.beta[i] = i < rows ? bsrc[i * ldbg] : 0.f;
+    sm.g[i] = i < rows ? gsrc[i * ldbg] : 0.f;
   }
   cp_async_wait<0>();
   __syncthreads();
@@ -355,6 +365,24 @@ __device__ __forceinline__ void t_stage(PrepAT& AT, float* X, int tid) {
   __syncthreads();
 }
 
+// G = cumulative sum of a chunk's g in double, by one warp: lane l sums
+// g_2l + g_2l+1, then an inclusive Kogge-Stone scan over the 32 pair sums
+// (offsets 1, 2, 4, 8, 16); G_2l+1 = scan_l, G_2l = scan_(l-1) + g_2l
+// (scan_(-1) = 0).
+__device__ __forceinline__ void chunk_cumsum_g(const float* g, double* G) {
+  const int lane = threadIdx.x & 31;
+  const double g0 = (double)g[2 * lane], g1 = (double)g[2 * lane + 1];
+  double x = g0 + g1;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const double y = __shfl_up_sync(kFull, x, off);
+    if (lane >= off) x += y;
+  }
+  const double e = __shfl_up_sync(kFull, x, 1);
+  G[2 * lane + 1] = x;
+  G[2 * lane] = lane > 0 ? e + g0 : g0;
+}
+
 struct PrepNoHook {
   __device__ void operator()() const {}
 };
@@ -400,18 +428,7 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT, const AfterP& after_p 
   // G = cumulative sum of g in double: warp 0, lane l sums g_2l + g_2l+1,
   // then an inclusive Kogge-Stone scan over the 32 pair sums (offsets 1, 2,
   // 4, 8, 16); G_2l+1 = scan_l, G_2l = scan_(l-1) + g_2l (scan_(-1) = 0).
-  if (warp == 0) {
-    const double g0 = (double)sm.g[2 * lane], g1 = (double)sm.g[2 * lane + 1];
-    double x = g0 + g1;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const double y = __shfl_up_sync(kFull, x, off);
-      if (lane >= off) x += y;
-    }
-    const double e = __shfl_up_sync(kFull, x, 1);
-    sm.G[2 * lane + 1] = x;
-    sm.G[2 * lane] = lane > 0 ? e + g0 : g0;
-  }
+  if (warp == 0) chunk_cumsum_g(sm.g, sm.G);
   after_p();
   if (tid < kBndThreads)
     for (int e = tid; e < kChunk * kChunk / 4; e += kBndThreads)
@@ -745,8 +762,9 @@ struct TcCtx {
 };
 
 // Allocate tensor memory (warp 0) and initialise the mbarrier; all threads.
-__device__ __forceinline__ void tc_setup(TcCtx& cx, uint64_t* mbar, uint32_t* tmem_slot) {
-  if (threadIdx.x < 32) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+__device__ __forceinline__ void tc_setup(TcCtx& cx, uint64_t* mbar, uint32_t* tmem_slot,
+                                         uint32_t cols = kTmemCols) {
+  if (threadIdx.x < 32) tmem_alloc(smem_u32(tmem_slot), cols);
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(mbar), 1);
     fence_mbar_init();
@@ -773,11 +791,11 @@ __device__ __forceinline__ void tc_drain(TcCtx& cx) { (void)tc_wait(cx); }
 
 // Release tensor memory (warp 0) once every thread's tensor-memory accesses
 // are done; all threads.
-__device__ __forceinline__ void tc_teardown(const TcCtx& cx) {
+__device__ __forceinline__ void tc_teardown(const TcCtx& cx, uint32_t cols = kTmemCols) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (threadIdx.x < 32) tmem_dealloc(cx.tmem, kTmemCols);
+  if (threadIdx.x < 32) tmem_dealloc(cx.tmem, cols);
   if (threadIdx.x == 0) mbar_inval(cx.mbar);
 }
 
@@ -952,6 +970,33 @@ __device__ __forceinline__ int tc_walk_step(float (&s)[128 / NCS],
   }
   tc_fence_before();
   return __syncthreads_or(!ok) ? kStepFailed : kStepDone;
+}
+
+// Pack arrival: thread 0 issues one bulk copy per chunk into a buffer whose
+// mbarrier counts the bytes; every thread waits (bounded) on that barrier.
+// Buffer b's j-th use completes phase j, so chunk c waits for parity
+// (c >> 1) & 1 on buffer c & 1.
+template <int D, class IN>
+__device__ __forceinline__ void pack_fetch(WalkPack<D, IN>& dst, const char* src, uint64_t* bar) {
+  const uint32_t mb = smem_u32(bar);
+  mbar_expect_tx(mb, (uint32_t)sizeof(WalkPack<D, IN>));
+  bulk_load(smem_u32(&dst), src, (uint32_t)sizeof(WalkPack<D, IN>), mb);
+}
+__device__ __forceinline__ bool pack_wait(uint64_t* bars, int64_t c) {
+  return mbar_wait(smem_u32(&bars[c & 1]), (uint32_t)((c >> 1) & 1), kTcWaitPolls);
+}
+// After a failed wait: wait (bounded) for every pack copy still in flight,
+// chunks c .. issued - 1.
+__device__ __forceinline__ void pack_drain(uint64_t* bars, int64_t c, int64_t issued) {
+  for (int64_t j = c; j < issued; j++) (void)pack_wait(bars, j);
+}
+__device__ __forceinline__ void pack_bars_init(uint64_t* bars) {
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars[0]), 1);
+    mbar_init(smem_u32(&bars[1]), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
 }
 
 // A state row of D fp32 values (16-byte pieces).

@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kBndThreads, prep_at_on_keys<D, IN>() ? 4 : 3)
            const float* __restrict__ g,
            const int32_t* __restrict__ cu, int H, const int32_t* __restrict__ hdr,
            const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
-           char* __restrict__ packs) {
+           char* __restrict__ packs, int all_chunks) {
   static_assert(sizeof(PackHead<D, IN>) % 16 == 0 && sizeof(KVPlanes<D, IN>) % 16 == 0,
                 "pack copies are 16-byte pieces");
   using PS = PrepSmem<D, IN>;
@@ -138,12 +138,15 @@ __global__ void __launch_bounds__(kBndThreads, prep_at_on_keys<D, IN>() ? 4 : 3)
   const int n = chunk_seq[c];
   const int ci = c - chunk_off[n];
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
-  if ((int64_t)(ci + 1) * kChunk > L) return;  // trailing partial chunk: no boundary
+  // A trailing partial chunk has no boundary after it; with all_chunks (the
+  // chunked forward's outputs need its pack) it is prepared zero-padded.
+  const int rows = (int)min((int64_t)kChunk, L - (int64_t)ci * kChunk);
+  if (rows < kChunk && !all_chunks) return;
   const int64_t t0 = (int64_t)cu[n] + (int64_t)ci * kChunk;
   const size_t tok = (size_t)t0 * H + h;
   PlaneRows<D, IN, kBndThreads> vrows;  // the chunk's values, in flight during the prep
-  vrows.load(v + tok * D, (size_t)H * D);
-  prep_stage<D, IN>(sm, k + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H);
+  vrows.load(v + tok * D, (size_t)H * D, rows);
+  prep_stage<D, IN>(sm, k + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H, rows);
   WalkPack<D, IN>& pk =
       *reinterpret_cast<WalkPack<D, IN>*>(packs + ((size_t)c * H + h) * pack_size<D, IN>());
   if constexpr (prep_at_on_keys<D, IN>()) {
@@ -182,33 +185,6 @@ __global__ void __launch_bounds__(kBndThreads, prep_at_on_keys<D, IN>() ? 4 : 3)
 // One block per (sequence, head): D/16 warps, 16 state rows each.
 template <int D>
 constexpr int walk_threads() { return 32 * (D / 16); }
-
-// Pack arrival: thread 0 issues one bulk copy per chunk into a buffer whose
-// mbarrier counts the bytes; every thread waits (bounded) on that barrier.
-// Buffer b's j-th use completes phase j, so chunk c waits for parity
-// (c >> 1) & 1 on buffer c & 1.
-template <int D, class IN>
-__device__ __forceinline__ void pack_fetch(WalkPack<D, IN>& dst, const char* src, uint64_t* bar) {
-  const uint32_t mb = smem_u32(bar);
-  mbar_expect_tx(mb, (uint32_t)sizeof(WalkPack<D, IN>));
-  bulk_load(smem_u32(&dst), src, (uint32_t)sizeof(WalkPack<D, IN>), mb);
-}
-__device__ __forceinline__ bool pack_wait(uint64_t* bars, int64_t c) {
-  return mbar_wait(smem_u32(&bars[c & 1]), (uint32_t)((c >> 1) & 1), kTcWaitPolls);
-}
-// After a failed wait: wait (bounded) for every pack copy still in flight,
-// chunks c .. issued - 1.
-__device__ __forceinline__ void pack_drain(uint64_t* bars, int64_t c, int64_t issued) {
-  for (int64_t j = c; j < issued; j++) (void)pack_wait(bars, j);
-}
-__device__ __forceinline__ void pack_bars_init(uint64_t* bars) {
-  if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&bars[0]), 1);
-    mbar_init(smem_u32(&bars[1]), 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-}
 
 template <int D, class IN>
 struct WalkSmem {
@@ -967,7 +943,7 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     const size_t sm = sizeof(PrepKernelSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
     kern<<<gchunks, kBndThreads, sm, st>>>(k, v, a.beta, a.g, a.cu_seqlens, a.H, hdr, chunk_off,
-                                           chunk_seq, packs);
+                                           chunk_seq, packs, 0);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(2));

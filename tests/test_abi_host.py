@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert gdn.lib.gdn_cpr_abi_version() == 6
+    assert gdn.lib.gdn_cpr_abi_version() == 7
     for code in range(-6, 1):
         assert gdn.status_string(code).startswith("GDN_")
     assert "unknown" in gdn.status_string(42)
