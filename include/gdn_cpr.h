@@ -318,6 +318,36 @@ int gdn_recurrent_decode_step(const void* q, const void* k, const void* v, int i
                               void* stream);
 
 /*
+ * gdn_native_forward -- the chunked ("native mixed") forward: outputs from
+ * each chunk's entry state by the chunkwise-parallel (UT / WY) products
+ * instead of the per-token recurrence.
+ *
+ * Defines: the section "Solving the linear-attention headache" and its
+ * per-layer table, whose first column evaluates training and prefill
+ * chunkwise in parallel while decode runs the recurrent form (the layout
+ * whose prefill and decode round differently).  With G the chunk's
+ * cumulative log-decay and U = T diag(beta) V - T diag(beta e^G) K S^T
+ * (T = (I + A)^{-1} as in gdn_chunk_boundary):
+ *     o_i = scale (e^{G_i} S q_i + sum_{j <= i} e^{G_i - G_j} (q_i . k_j) u_j)
+ * The entry states S are gdn_cpr_forward's first-pass boundary states
+ * (the same kernels); the output products run on the tensor cores with
+ * two-term bf16 splits of the non-bf16 operands, so o agrees with
+ * gdn_cpr_forward within the forward's bounds but not bit for bit.
+ * Arguments as gdn_cpr_forward (same workspace size); s_final receives the
+ * state after the last token (the state itself) and s_bnd_final the last
+ * boundary state.  Supported shape: dk = dv = 128 with bf16 inputs
+ * (GDN_ERR_UNSUPPORTED otherwise).  kernel_events: NULL, or 5 cudaEvent_t
+ * recorded before the chunk table, the boundary prep, the walk, the output
+ * products and after them.
+ */
+int gdn_native_forward(const void* q, const void* k, const void* v, int in_dtype,
+                       const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
+                       int64_t total_tokens, int H, int dk, int dv, int C, float scale,
+                       const float* h0, void* o, int out_dtype, float* s_final,
+                       float* s_bnd_final, void* workspace, size_t workspace_bytes,
+                       void* const* kernel_events, void* stream);
+
+/*
  * Bytes of device workspace gdn_cpr_backward needs for this problem size.
  * Returns 0 for arguments gdn_cpr_backward would reject.
  */

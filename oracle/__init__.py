@@ -354,5 +354,61 @@ def cpr_forward(q, k, v, beta, g, cu_seqlens, C: int, h0=None, scale: float = 1.
     return o, s_run, s_bnd, bstates
 
 
+def chunked_outputs(S0, Q, K, V, beta, g, scale: float = 1.0):
+    """Outputs of one chunk of n tokens from the state S0 at its start, by
+    the chunkwise-parallel (UT / WY) products (float64).
+
+    This is how the usual ("native mixed") layout of the per-layer table in
+    "NovaSky's IsoExec Fixes the Hidden Math Bug Corrupting AI Training
+    Runs" (section "Solving the linear-attention headache") evaluates a
+    chunk in training and prefill.  From the unrolled recurrence of
+    ``chunk_boundary``, S_i = gamma_i S0 + sum_{j<=i} exp(G_i - G_j) u_j k_j^T,
+    so o_i = scale S_i q_i is
+        o_i = scale (exp(G_i) S0 q_i + sum_{j<=i} exp(G_i - G_j) (q_i . k_j) u_j)
+    with U the rows u_j of ``chunk_boundary``.  Returns (o [n, dv], S_n).
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    S0 = np.asarray(S0, dtype=np.float64)
+    cb = chunk_boundary(S0, K, V, beta, g)
+    G, U = cb["G"], cb["U"]
+    n = len(G)
+    Pm = np.zeros((n, n))
+    for i in range(n):
+        for j in range(i + 1):
+            Pm[i, j] = np.exp(G[i] - G[j]) * (Q[i] @ K[j])
+    o = scale * (np.exp(G)[:, None] * (Q @ S0.T) + Pm @ U)
+    return o, cb["S"]
+
+
+def native_forward(q, k, v, beta, g, cu_seqlens, C: int, h0=None, scale: float = 1.0):
+    """The chunked ("native mixed") forward in float64: the boundary states of
+    ``cpr_forward``'s first pass, then every chunk's outputs (trailing partial
+    chunks included) by ``chunked_outputs``.  Returns (o, S_final, S_bnd_final)."""
+    q, k, v, beta, g = (_f64(a) for a in (q, k, v, beta, g))
+    cu = [int(x) for x in np.asarray(cu_seqlens)]
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = len(cu) - 1
+    o = np.zeros((T, H, dv))
+    s_fin = np.zeros((N, H, dv, dk))
+    s_bnd = np.zeros((N, H, dv, dk))
+    for n in range(N):
+        t0, t1 = cu[n], cu[n + 1]
+        for h in range(H):
+            S = np.zeros((dv, dk)) if h0 is None else _f64(h0)[n, h]
+            s_bnd[n, h] = S
+            for a in range(t0, t1, C):
+                b = min(a + C, t1)
+                oc, Se = chunked_outputs(S, q[a:b, h], k[a:b, h], v[a:b, h], beta[a:b, h],
+                                         g[a:b, h], scale)
+                o[a:b, h] = oc
+                if b - a == C:
+                    s_bnd[n, h] = Se
+                S = Se
+            s_fin[n, h] = S
+    return o, s_fin, s_bnd
+
+
 __all__ = ["build", "forward", "forward_alpha", "max_threads", "explicit_product_state",
-           "chunk_boundary", "cpr_forward"]
+           "chunk_boundary", "cpr_forward", "chunked_outputs", "native_forward"]

@@ -78,6 +78,8 @@ def _load() -> ctypes.CDLL:
                                         vp, vp, i32, vp, vp, vp, vp]),
         "gdn_recurrent_decode_step": (i32, [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, f32, vp,
                                             vp, vp, i32, vp]),
+        "gdn_native_forward": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                     f32, vp, vp, i32, vp, vp, vp, sz, vp, vp]),
         "gdn_cpr_backward_workspace_bytes": (sz, [i32, i64, i32, i32, i32, i32, i32]),
         "gdn_cpr_backward": (i32, [vp, vp, vp, i32, vp, vp, vp, i32, i64, i32, i32, i32, i32,
                                    f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, vp]),
@@ -197,6 +199,42 @@ def forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=No
                                 _stream(stream))
     _check(st, "gdn_cpr_forward")
     return o, s_run_final, s_bnd_final, workspace
+
+
+def native_forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=None,
+                   C: int = CHUNK, scale: float = 1.0, out_dtype=None, o=None, s_final=None,
+                   s_bnd_final=None, want_states: bool = True, workspace=None, stream=None,
+                   kernel_events=None):
+    """gdn_native_forward (the chunked, "native mixed" forward; d = 128, bf16).
+    Returns (o, s_final, s_bnd_final, workspace); the workspace is the CPR
+    forward's (same size).  kernel_events: 5 recorded torch.cuda.Event objects."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = (cu_seqlens.numel() - 1) if n_seqs is None else int(n_seqs)
+    in_code = _dtype_code(q)
+    out_code = _out_code(in_code, out_dtype, o)
+    dev = q.device
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=_torch_dtype(out_code), device=dev)
+    if want_states:
+        if s_final is None:
+            s_final = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+        if s_bnd_final is None:
+            s_bnd_final = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    need = forward_workspace_bytes(N, T, H, dk, dv, C, q.dtype)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    ev = None
+    if kernel_events is not None:
+        if len(kernel_events) != 5 or any(e.cuda_event == 0 for e in kernel_events):
+            raise ValueError("kernel_events: 5 torch.cuda.Event objects, each recorded once")
+        ev = (ctypes.c_void_p * 5)(*[e.cuda_event for e in kernel_events])
+    st = lib.gdn_native_forward(_ptr(q), _ptr(k), _ptr(v), in_code, _ptr(beta), _ptr(g),
+                                _ptr(cu_seqlens), N, T, H, dk, dv, C, float(scale), _ptr(h0),
+                                _ptr(o), out_code, _ptr(s_final), _ptr(s_bnd_final),
+                                _ptr(workspace), workspace.numel(), ev, _stream(stream))
+    _check(st, "gdn_native_forward")
+    return o, s_final, s_bnd_final, workspace
 
 
 def recurrent_forward(q, k, v, beta, g, cu_seqlens, *, n_seqs: Optional[int] = None, h0=None,

@@ -136,6 +136,45 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
   return from_cuda(gdn::launch_forward(a, static_cast<cudaStream_t>(stream)));
 }
 
+int gdn_native_forward(const void* q, const void* k, const void* v, int in_dtype,
+                       const float* beta, const float* g, const int32_t* cu_seqlens, int n_seqs,
+                       int64_t total_tokens, int H, int dk, int dv, int C, float scale,
+                       const float* h0, void* o, int out_dtype, float* s_final,
+                       float* s_bnd_final, void* workspace, size_t workspace_bytes,
+                       void* const* kernel_events, void* stream) {
+  const int rc = gdn::forward_check_args(q, k, v, in_dtype, beta, g, cu_seqlens, n_seqs,
+                                         total_tokens, H, dk, dv, C, scale, h0, o, out_dtype,
+                                         s_final, nullptr, s_bnd_final);
+  if (rc != GDN_OK && rc != gdn::kFwdEmpty) return rc;
+  if (in_dtype != GDN_BF16 || dk != 128) return GDN_ERR_UNSUPPORTED;
+  if (rc == gdn::kFwdEmpty) return GDN_OK;
+  const gdn::FwdLayout lay = gdn::fwd_layout(n_seqs, total_tokens, H, dk, dv, C, true);
+  if (!workspace || workspace_bytes < lay.total) return GDN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDN_ERR_INVALID_ARG;
+  gdn::FwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.in_bf16 = 1;
+  a.beta = beta;
+  a.g = g;
+  a.cu_seqlens = cu_seqlens;
+  a.n_seqs = n_seqs;
+  a.T = total_tokens;
+  a.H = H;
+  a.D = dk;
+  a.scale = scale;
+  a.h0 = h0;
+  a.o = o;
+  a.out_bf16 = out_dtype == GDN_BF16;
+  a.s_run_final = s_final;
+  a.s_bnd_final = s_bnd_final;
+  a.ws = static_cast<char*>(workspace);
+  a.lay = lay;
+  a.events = kernel_events;
+  return from_cuda(gdn::launch_native_forward(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t gdn_cpr_backward_workspace_bytes(int n_seqs, int64_t total_tokens, int H, int dk, int dv,
                                         int C, int in_dtype) {
   if (n_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return 0;

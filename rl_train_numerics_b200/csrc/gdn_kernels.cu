@@ -20,6 +20,7 @@
 #include "gdn_boundary.cuh"
 #include "gdn_fill.cuh"
 #include "gdn_layout.h"
+#include "gdn_native.cuh"
 
 namespace gdn {
 
@@ -981,6 +982,65 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   return mark(4);
 }
 
+// The chunked ("native mixed") forward, d = 128 with bf16 inputs: the CPR
+// first pass with every chunk prepared (trailing partial chunks zero-padded),
+// then the output products of gdn_native.cuh from the chunks' entry states.
+template <class OUT>
+static cudaError_t native_impl(const FwdArgs& a, cudaStream_t st) {
+  using IN = __nv_bfloat16;
+  constexpr int D = 128;
+  const FwdLayout& L = a.lay;
+  char* ws = a.ws;
+  int32_t* hdr = reinterpret_cast<int32_t*>(ws + L.hdr);
+  int32_t* chunk_off = reinterpret_cast<int32_t*>(ws + L.chunk_off);
+  int32_t* chunk_seq = reinterpret_cast<int32_t*>(ws + L.chunk_seq);
+  float* bstate = reinterpret_cast<float*>(ws + L.bstate);
+  char* packs = ws + L.pack;
+  auto mark = [&](int i) -> cudaError_t {
+    return a.events ? cudaEventRecord(static_cast<cudaEvent_t>(a.events[i]), st) : cudaSuccess;
+  };
+  GDN_TRY(mark(0));
+  k_chunk_table<<<1, kTableThreads, 0, st>>>(a.cu_seqlens, a.n_seqs, a.T, hdr, chunk_off,
+                                             chunk_seq, L.max_chunks);
+  GDN_TRY(cudaGetLastError());
+  GDN_TRY(mark(1));
+  {
+    auto kern = k_prep<D, IN>;
+    const size_t sm = sizeof(PrepKernelSmem<D, IN>);
+    GDN_TRY(set_smem(kern, sm));
+    kern<<<dim3((unsigned)L.max_chunks, (unsigned)a.H), kBndThreads, sm, st>>>(
+        static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, a.cu_seqlens,
+        a.H, hdr, chunk_off, chunk_seq, packs, 1);
+    GDN_TRY(cudaGetLastError());
+  }
+  GDN_TRY(mark(2));
+  {
+    auto kern = k_walk_tc<D, IN>;
+    const size_t sm = sizeof(WalkTcSmem<D, IN>);
+    GDN_TRY(set_smem(kern, sm));
+    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), kWalkThreads, sm, st>>>(
+        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final, nullptr,
+        a.s_bnd_final);
+    GDN_TRY(cudaGetLastError());
+  }
+  GDN_TRY(mark(3));
+  {
+    auto kern = k_native_tc<OUT>;
+    const size_t sm = sizeof(NativeSmem);
+    GDN_TRY(set_smem(kern, sm));
+    int dev = 0, sms = 0;
+    GDN_TRY(cudaGetDevice(&dev));
+    GDN_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const int64_t items = L.max_chunks * a.H;
+    const int grid = (int)(items < sms ? items : sms);
+    kern<<<grid, kNtThreads, sm, st>>>(static_cast<const IN*>(a.q), a.g, a.cu_seqlens, a.H,
+                                       a.scale, hdr, chunk_off, chunk_seq, packs, bstate,
+                                       static_cast<OUT*>(a.o), a.s_run_final);
+    GDN_TRY(cudaGetLastError());
+  }
+  return mark(4);
+}
+
 template <int D, class IN, class OUT>
 static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
   k_dec_step<D, IN, OUT><<<dim3((unsigned)a.B, (unsigned)a.H), kDecThreads, 0, st>>>(
@@ -1031,6 +1091,11 @@ cudaError_t launch_forward(const FwdArgs& a, cudaStream_t st) {
   }
   if (!a.in_bf16) return cudaErrorNotSupported;  // fp32 inputs: d = 64 only
   return a.out_bf16 ? forward_impl<128, bf16, bf16>(a, st) : forward_impl<128, bf16, float>(a, st);
+}
+
+cudaError_t launch_native_forward(const FwdArgs& a, cudaStream_t st) {
+  if (a.D != 128 || !a.in_bf16) return cudaErrorNotSupported;
+  return a.out_bf16 ? native_impl<bf16>(a, st) : native_impl<float>(a, st);
 }
 
 cudaError_t launch_decode_step(const DecArgs& a, cudaStream_t st) {

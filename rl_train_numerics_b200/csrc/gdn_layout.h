@@ -24,7 +24,8 @@ constexpr size_t pack_bytes(int D, bool in_bf16) {
 //   chunk_off  int32[N+1]   first global chunk index of each sequence
 //   chunk_seq  int32[MC]    sequence of each global chunk
 //   bstate     f32[MC,H,dv,dk]  state at the start of every chunk
-//   pack       [MC,H] walk packs (boundary prep of full chunks)
+//   pack       [MC,H] walk packs (boundary prep of full chunks; the chunked
+//                     forward also prepares trailing partial chunks, zero-padded)
 // MC = floor(T/C) + N + 1 bounds the number of chunks for any valid
 // cu_seqlens (each sequence adds at most one partial chunk).
 struct FwdLayout {
@@ -182,6 +183,9 @@ struct BwdArgs {
 };
 
 cudaError_t launch_forward(const FwdArgs& a, cudaStream_t stream);
+// The chunked ("native mixed") forward (d = 128, bf16 inputs): the forward
+// workspace, s_run_final as the state itself (s_run_scale unused).
+cudaError_t launch_native_forward(const FwdArgs& a, cudaStream_t stream);
 
 // Host-side argument checks of gdn_cpr_forward (all but the workspace);
 // kFwdEmpty marks a valid call with nothing to launch.

@@ -291,3 +291,55 @@ def test_selftest_rejects_on_host():
     assert L.gdn_selftest_bounded_wait(0, FAKE, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_selftest_bounded_wait((1 << 22) + 1, FAKE, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_selftest_bounded_wait(10, None, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_native_forward_host_checks():
+    """gdn_native_forward: d = 128 with bf16 inputs only; the forward's argument
+    checks and workspace size otherwise (all rejected before any launch)."""
+    L = gdn.lib
+
+    def call(**over):
+        a = dict(q=FAKE, in_dtype=gdn.GDN_BF16, N=2, T=128, H=2, dk=128, dv=128, C=64,
+                 ws=FAKE, wsb=1 << 40)
+        a.update(over)
+        return L.gdn_native_forward(a["q"], FAKE, FAKE, a["in_dtype"], FAKE, FAKE, FAKE, a["N"],
+                                    a["T"], a["H"], a["dk"], a["dv"], a["C"], 1.0, None, FAKE,
+                                    gdn.GDN_BF16, None, None, a["ws"], a["wsb"], None, None)
+    assert call(dk=64, dv=64) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(dk=64, dv=64, in_dtype=gdn.GDN_F32) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(q=MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert call(C=32) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(wsb=16) == gdn.GDN_ERR_WORKSPACE
+    assert call(ws=None) == gdn.GDN_ERR_WORKSPACE
+
+
+def test_recurrent_host_checks():
+    L = gdn.lib
+
+    def fwd_call(**over):
+        a = dict(q=FAKE, in_dtype=gdn.GDN_BF16, N=2, T=128, dk=128, dv=128, sf=None, sfs=None,
+                 err=None)
+        a.update(over)
+        return L.gdn_recurrent_forward(a["q"], FAKE, FAKE, a["in_dtype"], FAKE, FAKE, FAKE,
+                                       a["N"], a["T"], 2, a["dk"], a["dv"], 1.0, None, FAKE,
+                                       gdn.GDN_BF16, a["sf"], a["sfs"], a["err"], None)
+    assert fwd_call(dk=96, dv=96) == gdn.GDN_ERR_UNSUPPORTED
+    assert fwd_call(in_dtype=gdn.GDN_F32) == gdn.GDN_ERR_UNSUPPORTED  # fp32 inputs: d = 64
+    assert fwd_call(q=MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert fwd_call(sfs=FAKE) == gdn.GDN_ERR_INVALID_ARG  # a scale without the state
+    assert fwd_call(err=MIS + 2) == gdn.GDN_ERR_INVALID_ARG  # misaligned error word
+    assert fwd_call(N=0, T=5) == gdn.GDN_ERR_INVALID_ARG
+
+    def step_call(**over):
+        a = dict(B=4, dk=128, dv=128, in_dtype=gdn.GDN_BF16, s=FAKE, o=FAKE)
+        a.update(over)
+        return L.gdn_recurrent_decode_step(FAKE, FAKE, FAKE, a["in_dtype"], FAKE, FAKE, a["B"],
+                                           2, a["dk"], a["dv"], 1.0, a["s"], FAKE, a["o"],
+                                           gdn.GDN_BF16, None)
+    assert step_call(dk=96, dv=96) == gdn.GDN_ERR_UNSUPPORTED
+    assert step_call(dk=128, dv=64) == gdn.GDN_ERR_UNSUPPORTED
+    assert step_call(in_dtype=gdn.GDN_F32) == gdn.GDN_ERR_UNSUPPORTED
+    assert step_call(s=MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert step_call(s=None) == gdn.GDN_ERR_INVALID_ARG
+    assert step_call(B=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert step_call(B=0) == gdn.GDN_OK  # nothing to do
