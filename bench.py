@@ -38,6 +38,10 @@ H, D, C = 16, 128, 64
 PREFILL_LENS = [2048] * 5
 FLUSH_BYTES = 256 << 20
 PAGES_H100 = {"prefill_ms": 1.412, "decode_ms": 0.0846, "trainer_fwd_bwd_ms": 7.386}
+# The per-layer table's three layouts on H100 (ms; trainer row is forward +
+# backward): native mixed, recurrent everywhere, CPR.
+PAGES_H100_LAYOUTS = {"prefill": (0.844, 3.639, 1.412), "trainer_fwd_bwd": (5.177, 22.863, 7.386),
+                      "decode": (0.0612, 0.0612, 0.0846)}
 
 
 # Source files whose kernels a traffic figure belongs to: a recorded figure is
@@ -395,6 +399,115 @@ def run_decode_part(gdn, W, dev, rank, world, args, peaks):
             "pages_h100_ms": PAGES_H100["decode_ms"]}
 
 
+def _mean_ms(fn, steps, warmup, flush):
+    """Mean device time of fn() over `steps` calls (L2 flushed before each),
+    and the per-kernel split when fn takes 5 recorded events."""
+    for _ in range(warmup):
+        flush.zero_()
+        fn(None)
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(steps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        for x in e:
+            x.record()
+        evs.append(e)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        fn(evs[i])
+    torch.cuda.synchronize()
+    total = sum(e[0].elapsed_time(e[4]) for e in evs) / steps
+    split = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / steps for j in range(4)]
+    return total, split
+
+
+def run_layouts_part(gdn, W, dev, rank, world, args, flush, cpr_decode_ms):
+    """The per-layer table's three layouts on this GPU: CPR (gdn_cpr_forward),
+    native mixed (gdn_native_forward: chunked outputs, recurrent decode) and
+    recurrent everywhere (gdn_recurrent_forward / gdn_recurrent_decode_step),
+    on the rollout prefill and trainer-forward batches and the 256-row decode."""
+    out = {}
+    for name, b in (("prefill", W.prefill(device=dev, seed=rank)),
+                    ("trainer_forward", W.trainer(device=dev, seed=rank))):
+        T, N = b.total_tokens, len(b.lengths)
+        o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+        s = torch.empty((N, H, D, D), dtype=torch.float32, device=dev)
+        sb = torch.empty_like(s)
+        ws = torch.zeros(gdn.forward_workspace_bytes(N, T, H, D, D), dtype=torch.uint8, device=dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        args_in = (b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens)
+
+        def cpr(evs):
+            gdn.forward(*args_in, o=o, s_run_final=s, s_bnd_final=sb, workspace=ws,
+                        kernel_events=evs)
+
+        def nat(evs):
+            gdn.native_forward(*args_in, o=o, s_final=s, s_bnd_final=sb, workspace=ws,
+                               kernel_events=evs)
+
+        def rec(evs):
+            if evs is not None:
+                evs[0].record()
+            gdn.recurrent_forward(*args_in, o=o, s_final=s, error=err)
+            if evs is not None:
+                for e in evs[1:]:
+                    e.record()
+
+        t_cpr, k_cpr = _mean_ms(cpr, args.steps, args.warmup, flush)
+        t_nat, k_nat = _mean_ms(nat, args.steps, args.warmup, flush)
+        t_rec, _ = _mean_ms(rec, args.steps, args.warmup, flush)
+        if gdn.check_error(ws) != 0 or gdn.check_error(err) != 0:
+            raise RuntimeError("device error word set in the layout comparison")
+        t_cpr, t_nat, t_rec = (max_over_ranks(x, world) for x in (t_cpr, t_nat, t_rec))
+        out[name] = {
+            "tokens": T, "cpr_ms": round(t_cpr, 5), "native_ms": round(t_nat, 5),
+            "recurrent_ms": round(t_rec, 5),
+            "native_kernels_ms": dict(zip(["chunk_table", "boundary_prep", "boundary_walk",
+                                           "chunked_outputs"], [round(x, 5) for x in k_nat])),
+            "cpr_over_native": round(t_cpr / t_nat, 3),
+            "recurrent_over_native": round(t_rec / t_nat, 3),
+            "cpr_over_recurrent": round(t_cpr / t_rec, 3)}
+    nat_p, rec_p, cpr_p = PAGES_H100_LAYOUTS["prefill"]
+    out["prefill"]["pages_h100"] = {"native_ms": nat_p, "recurrent_ms": rec_p, "cpr_ms": cpr_p,
+                                    "cpr_over_native": round(cpr_p / nat_p, 3),
+                                    "recurrent_over_native": round(rec_p / nat_p, 3)}
+    nat_t, rec_t, cpr_t = PAGES_H100_LAYOUTS["trainer_fwd_bwd"]
+    out["trainer_forward"]["pages_h100_fwd_bwd"] = {
+        "native_ms": nat_t, "recurrent_ms": rec_t, "cpr_ms": cpr_t,
+        "cpr_over_native": round(cpr_t / nat_t, 3),
+        "recurrent_over_native": round(rec_t / nat_t, 3),
+        "note": "the pages' trainer row is forward + backward; the layouts here are forwards"}
+    # decode: the recurrent step (the native and recurrent layouts' decode)
+    slots, steps = args.decode_slots, 128
+    st = torch.zeros((slots, H, D, D), dtype=torch.float32, device=dev)
+    sc = torch.ones((slots, H), dtype=torch.float32, device=dev)
+    toks = W.decode_tokens(16 + steps, slots, H, D, D, seed=300 + rank, device=dev)
+    o = torch.empty((slots, H, D), dtype=torch.bfloat16, device=dev)
+    for i in range(16):
+        gdn.recurrent_decode_step(toks[0][i], toks[1][i], toks[2][i], toks[3][i], toks[4][i],
+                                  st, sc, o=o)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        j = 16 + i
+        ev[i][0].record()
+        gdn.recurrent_decode_step(toks[0][j], toks[1][j], toks[2][j], toks[3][j], toks[4][j],
+                                  st, sc, o=o)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    t_rd = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in ev) / steps, world)
+    nat_d, _, cpr_d = PAGES_H100_LAYOUTS["decode"]
+    out["decode"] = {"recurrent_ms_per_step": round(t_rd, 5),
+                     "cpr_ms_per_step": None if cpr_decode_ms is None else round(cpr_decode_ms, 5),
+                     "cpr_over_recurrent": None if cpr_decode_ms is None
+                     else round(cpr_decode_ms / t_rd, 3),
+                     "pages_h100": {"recurrent_ms": nat_d, "cpr_ms": cpr_d,
+                                    "cpr_over_recurrent": round(cpr_d / nat_d, 3)}}
+    return out
+
+
 def bwd_gemm_flops(lengths, H, D):
     """Algorithmic FLOPs of the backward's chunk products: per chunk of length L,
     Y (lower triangle incl. diagonal) and X (strict) over d, the three L x d x d
@@ -708,6 +821,10 @@ def run_ours(args):
     pikr = None
     if args.only in ("all", "pik"):
         pikr = run_pik_part(gdn, dev, rank, world, args, flush, peaks)
+    layouts = None
+    if args.only in ("all", "layouts"):
+        layouts = run_layouts_part(gdn, W, dev, rank, world, args, flush,
+                                   None if decode is None else decode["ms_per_step"])
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -728,6 +845,7 @@ def run_ours(args):
         "decode": decode,
         "train_step": train,
         "pik_gemm": pikr,
+        "layouts": layouts,
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
         "wall_s_timed_region": round(wall, 4),
@@ -792,7 +910,8 @@ def main():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--decode-steps", type=int, default=512)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--only", choices=["all", "prefill", "decode", "train", "pik", "bwd-small"],
+    p.add_argument("--only", choices=["all", "prefill", "decode", "train", "pik", "layouts",
+                                      "bwd-small"],
                    default="all",
                    help="profiling aid: run only part of the benchmark")
     p.add_argument("--decode-slots", type=int, default=256)

@@ -222,9 +222,12 @@ __global__ void __launch_bounds__(kRecurStepThreads)
 // ----------------------------------------------------------------------------
 // Launchers
 // ----------------------------------------------------------------------------
-// Rows per quad of the recurrent forward: 1 (32 rows per block) gives the most
-// blocks for the few long sequences of a prefill batch.
-constexpr int kRecurRT = 1;
+// Rows per quad of the recurrent forward (at most D / 32).  Four rows (one
+// block per unit at d = 128) ran the 5 x 2048 prefill in 1.11 ms against
+// 1.24 ms with two and 1.38 ms with one: the per-token chain of dependent
+// steps, not the number of blocks, sets the time, and more rows per thread
+// give it more independent work.
+constexpr int kRecurRT = 4;
 
 template <int D, class IN, class OUT>
 static cudaError_t recur_forward_impl(const void* q, const void* k, const void* v,
@@ -232,7 +235,7 @@ static cudaError_t recur_forward_impl(const void* q, const void* k, const void* 
                                       int N, int64_t T, int H, float scale, const float* h0,
                                       void* o, float* s_final, float* s_final_scale,
                                       int32_t* error, cudaStream_t st) {
-  constexpr int RT = kRecurRT, RB = 32 * RT;
+  constexpr int RT = 32 * kRecurRT <= D ? kRecurRT : D / 32, RB = 32 * RT;
   static_assert(D % RB == 0, "whole row blocks");
   auto kern = k_recur<D, IN, OUT, RT>;
   const size_t smem = sizeof(RecurSmem<D, IN, RB>);
