@@ -52,6 +52,9 @@ TRAFFIC_SOURCES = {
     "backward": ("gdn_backward.cu", "gdn_boundary.cuh", "gdn_common.cuh", "gdn_fill.cuh",
                  "gdn_mma.cuh", "gdn_umma.cuh", "gdn_layout.h"),
     "pik": ("gdn_pik.cu", "gdn_mma.cuh", "gdn_umma.cuh"),
+    "native": ("gdn_native.cuh", "gdn_boundary.cuh", "gdn_common.cuh", "gdn_fill.cuh",
+               "gdn_mma.cuh", "gdn_umma.cuh"),
+    "recurrent": ("gdn_recurrent.cu", "gdn_fill.cuh", "gdn_common.cuh", "gdn_mma.cuh"),
 }
 
 
@@ -399,6 +402,18 @@ def run_decode_part(gdn, W, dev, rank, world, args, peaks):
             "pages_h100_ms": PAGES_H100["decode_ms"]}
 
 
+def native_out_bytes(lens, H_, d, c=C, pack=65808):
+    """Algorithmic bytes of the chunked layout's output kernel: per (chunk, head)
+    the entry state (fp32 d x d), the chunk's pack, its queries (bf16), g and
+    its outputs (bf16)."""
+    tot = 0
+    for L in lens:
+        for a in range(0, L, c):
+            n = min(c, L - a)
+            tot += H_ * (d * d * 4 + pack + n * d * 2 + n * 4 + n * d * 2)
+    return tot
+
+
 def _mean_ms(fn, steps, warmup, flush):
     """Mean device time of fn() over `steps` calls (L2 flushed before each),
     and the per-kernel split when fn takes 5 recorded events."""
@@ -422,7 +437,7 @@ def _mean_ms(fn, steps, warmup, flush):
     return total, split
 
 
-def run_layouts_part(gdn, W, dev, rank, world, args, flush, cpr_decode_ms):
+def run_layouts_part(gdn, W, dev, rank, world, args, flush, cpr_decode_ms, peaks):
     """The per-layer table's three layouts on this GPU: CPR (gdn_cpr_forward),
     native mixed (gdn_native_forward: chunked outputs, recurrent decode) and
     recurrent everywhere (gdn_recurrent_forward / gdn_recurrent_decode_step),
@@ -460,7 +475,22 @@ def run_layouts_part(gdn, W, dev, rank, world, args, flush, cpr_decode_ms):
         if gdn.check_error(ws) != 0 or gdn.check_error(err) != 0:
             raise RuntimeError("device error word set in the layout comparison")
         t_cpr, t_nat, t_rec = (max_over_ranks(x, world) for x in (t_cpr, t_nat, t_rec))
+        nb = native_out_bytes(b.lengths, H, D)
+        nat_gbs = nb / (max_over_ranks(k_nat[3], world) / 1e3) / 1e9
+        rec_tf = fill_flops(T, H, D) / (t_rec / 1e3) / 1e12
+        fp32_peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
         out[name] = {
+            "native_outputs_roofline": {
+                "kernel": "k_native_tc", "bound": "hbm", "achieved": round(nat_gbs, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(nat_gbs / peaks["hbm_gbs"], 4),
+                "traffic": ncu_traffic("native_outputs") if name == "prefill" else None,
+                "algorithmic_bytes": nb},
+            "recurrent_roofline": {
+                "kernel": "k_recur", "bound": "alu", "achieved": round(rec_tf, 2),
+                "peak": round(fp32_peak, 2), "unit": "TFLOP/s",
+                "frac": round(rec_tf / fp32_peak, 4),
+                "traffic": ncu_traffic("recurrent_forward") if name == "prefill" else None},
             "tokens": T, "cpr_ms": round(t_cpr, 5), "native_ms": round(t_nat, 5),
             "recurrent_ms": round(t_rec, 5),
             "native_kernels_ms": dict(zip(["chunk_table", "boundary_prep", "boundary_walk",
@@ -824,7 +854,7 @@ def run_ours(args):
     layouts = None
     if args.only in ("all", "layouts"):
         layouts = run_layouts_part(gdn, W, dev, rank, world, args, flush,
-                                   None if decode is None else decode["ms_per_step"])
+                                   None if decode is None else decode["ms_per_step"], peaks)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
