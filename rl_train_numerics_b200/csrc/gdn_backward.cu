@@ -51,6 +51,7 @@
 //   k_bwd_gemm       one block per (chunk, head): DQ and DK from the
 //                    products above, in fp32 fused multiply-adds
 // Every sum has a fixed order, so repeated runs give identical bits.
+#include "gdn_boundary.cuh"
 #include "gdn_fill.cuh"
 #include "gdn_layout.h"
 
@@ -626,6 +627,324 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ----------------------------------------------------------------------------
+// Chunk products on the tensor cores (bf16 inputs)
+// ----------------------------------------------------------------------------
+// The same DQ and DK as k_bwd_gemm, as mma.sync m16n8k16 contractions with
+// fp32 accumulation.  do, q and k are exact in bf16; every fp32 operand (w, u,
+// S_a, mu_e, A, -(B + B^T)) is split exactly into two bf16 terms and the term
+// pairs (hi, hi), (hi, lo), (lo, hi) accumulate in that order (the split
+// scheme of the forward's boundary pass).  One block of 8 warps per (chunk,
+// head); warp w owns tokens 16 (w % 4) .. + 15 and, for the C x C products,
+// columns 32 (w / 4) .. + 31, for the C x D products (D / 2) (w / 4) .. + D / 2 - 1.
+//   1. Y = DO U^T, X = W U^T -> A_ts = [s <= t] e^{G_t - G_s} Y_ts and
+//      Bn = -(B + B^T), B_ts = [s < t] beta_t e^{G_t - G_s} X_ts, both as
+//      term planes in shared memory.
+//   2. Over 16-row slabs of S_a and mu_e (cp.async, split per slab):
+//      Pq = DO S_a, Pw = W S_a, Pu = U mu_e.
+//   3. DQ = scale (diag(e^G) Pq + A K);
+//      DK = diag(-beta e^G) Pw + diag(e^{G_{L-1} - G}) Pu + scale (A^T Q)
+//           + Bn K  (A^T read through transposed ldmatrix).
+// Every sum has a fixed order, so repeated runs give identical bits.
+template <int D>
+struct GemmTcSmem {
+  __nv_bfloat16 DO[1][kChunk * D];      // [t][i]
+  __nv_bfloat16 W[2][kChunk * D];       // [t][i], two terms
+  __nv_bfloat16 U[2][kChunk * D];       // [s][i]
+  __nv_bfloat16 Q[1][kChunk * D];       // [t][j]
+  __nv_bfloat16 K[1][kChunk * D];       // [s][j]
+  __nv_bfloat16 A[2][kChunk * kChunk];  // [t][s]
+  __nv_bfloat16 Bn[2][kChunk * kChunk]; // [t][s], -(B + B^T)
+  __nv_bfloat16 Sp[2][kSlab * D];       // the current slab's terms, [i][j] (16-row core layout)
+  __nv_bfloat16 Mp[2][kSlab * D];
+  double G[kChunk];
+  float graw[kChunk];
+  float bet[kChunk];
+};
+
+// B fragments (x4.trans, two n8 tiles) of B[k][n] = M[k][n] in a 16-row plane.
+__device__ __forceinline__ const __nv_bfloat16* bfrag_kn16_addr(const __nv_bfloat16* base, int n0) {
+  const int lane = threadIdx.x & 31, mi = lane >> 3;
+  return base + core_off<kSlab>((mi & 1) * 8 + (lane & 7), n0 + (mi >> 1) * 8);
+}
+
+// Eight consecutive fp32 values as two bf16 term pieces (16 bytes each).
+__device__ __forceinline__ void split8(const float4& a, const float4& b, uint4& hi, uint4& lo) {
+  split2(a.x, a.y, hi.x, lo.x);
+  split2(a.z, a.w, hi.y, lo.y);
+  split2(b.x, b.y, hi.z, lo.z);
+  split2(b.z, b.w, hi.w, lo.w);
+}
+
+// Two-term planes of two C x D fp32 blocks (rows at stride ld; rows past len
+// zero).  Work item e is row e % C, columns 8 (e / C) .. + 7, so that a warp
+// writes 32 consecutive 16-byte pieces of the core layout; every load is
+// issued before the first split.
+template <int D>
+__device__ __forceinline__ void split_rows2x2(__nv_bfloat16 (*dst0)[kChunk * D], const float* src0,
+                                              __nv_bfloat16 (*dst1)[kChunk * D], const float* src1,
+                                              size_t ld, int len) {
+  constexpr int IT = kChunk * D / 8 / kGemmThreads;
+  static_assert(kChunk * D / 8 % kGemmThreads == 0, "whole pieces per thread");
+  float4 x[2][IT][2];
+#pragma unroll
+  for (int j = 0; j < IT; j++) {
+    const int e = threadIdx.x + j * kGemmThreads, t = e % kChunk, c = (e / kChunk) * 8;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      x[0][j][h] = t < len ? ld4(src0 + (size_t)t * ld + c + 4 * h) : z;
+      x[1][j][h] = t < len ? ld4(src1 + (size_t)t * ld + c + 4 * h) : z;
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 2; m++) {
+    __nv_bfloat16(*dst)[kChunk * D] = m == 0 ? dst0 : dst1;
+#pragma unroll
+    for (int j = 0; j < IT; j++) {
+      const int e = threadIdx.x + j * kGemmThreads, t = e % kChunk, c = (e / kChunk) * 8;
+      uint4 hi, lo;
+      split8(x[m][j][0], x[m][j][1], hi, lo);
+      *reinterpret_cast<uint4*>(&dst[0][core_off<kChunk>(t, c)]) = hi;
+      *reinterpret_cast<uint4*>(&dst[1][core_off<kChunk>(t, c)]) = lo;
+    }
+  }
+}
+
+// One bf16 term pair of a 2-term split into the 64-row planes P at (r, c).
+__device__ __forceinline__ void put_terms(__nv_bfloat16 (*P)[kChunk * kChunk], int r, int c,
+                                          float x) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+  P[0][core_off<kChunk>(r, c)] = hi;
+  P[1][core_off<kChunk>(r, c)] = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_bwd_gemm_tc(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                  const float* __restrict__ beta, const float* __restrict__ g,
+                  const __nv_bfloat16* __restrict__ d_o, const int32_t* __restrict__ cu, int H,
+                  float scale, const int32_t* __restrict__ hdr,
+                  const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
+                  const float* __restrict__ bstate, const float* __restrict__ mu_end,
+                  const float* __restrict__ wbuf, const float* __restrict__ ubuf,
+                  float* __restrict__ d_q, float* __restrict__ d_k) {
+  using bf16 = __nv_bfloat16;
+  constexpr int NS = D / kSlab;
+  constexpr int NT8 = D / 16;  // n8 tiles of a warp's C x D columns (D / 2 of them)
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  GemmTcSmem<D>& sm = *reinterpret_cast<GemmTcSmem<D>*>(smem_raw);
+  if (hdr[kHdrValid] != 1) return;
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (c >= hdr[kHdrChunks]) return;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+  const int mt = w & 3, nh = w >> 2;
+  const size_t DD = (size_t)D * D;
+  const FillItem it = fill_item(c * H + h, H, cu, chunk_off, chunk_seq);
+  const int len = it.len;
+  const size_t tb = (size_t)it.t0 * H + h;
+  const float* Sa = bstate + ((size_t)c * H + h) * DD;
+  const float* Me = mu_end + ((size_t)c * H + h) * DD;
+
+  // Slabs of S_a and mu_e pass through registers, one slab ahead: work item e
+  // is row e % 16 of the slab, columns 8 (e / 16) .. + 7 (S_a from its
+  // permuted layout).
+  constexpr int SLI = kSlab * D / 8;  // work items of a slab (per matrix)
+  const bool slab_item = tid < SLI;
+  const int sr = tid % kSlab, sc = (tid / kSlab) * 8;
+  float4 sx[2], mx[2];
+  auto slab_load = [&](int j) {
+    if (!slab_item) return;
+    const int i = j * kSlab + sr;
+#pragma unroll
+    for (int hh = 0; hh < 2; hh++) {
+      sx[hh] = ld4(Sa + (size_t)i * D + bst_col(i, sc + 4 * hh));
+      mx[hh] = ld4(Me + (size_t)i * D + sc + 4 * hh);
+    }
+  };
+  slab_load(0);
+  stage_planes<D, bf16>(sm.DO, d_o + tb * D, (size_t)H * D, kGemmThreads, len);
+  stage_planes<D, bf16>(sm.Q, q + tb * D, (size_t)H * D, kGemmThreads, len);
+  stage_planes<D, bf16>(sm.K, k + tb * D, (size_t)H * D, kGemmThreads, len);
+  cp_async_commit();
+  split_rows2x2<D>(sm.W, wbuf + tb * D, sm.U, ubuf + tb * D, (size_t)H * D, len);
+  if (tid < kChunk) {
+    sm.graw[tid] = tid < len ? g[tb + (size_t)tid * H] : 0.f;
+    sm.bet[tid] = tid < len ? beta[tb + (size_t)tid * H] : 0.f;
+  }
+  __syncthreads();
+  if (w == 0) chunk_cumsum_g(sm.graw, sm.G);
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // 1. Y and X on this warp's 16 x 32 tile, then A and Bn.
+  {
+    float y[4][4], x[4][4];
+#pragma unroll
+    for (int n = 0; n < 4; n++)
+#pragma unroll
+      for (int e = 0; e < 4; e++) y[n][e] = x[n][e] = 0.f;
+#pragma unroll 2
+    for (int ks = 0; ks < D / 16; ks++) {
+      uint32_t ad[1][4], aw[2][4];
+      ldsm_x4(ad[0], afrag_addr(sm.DO[0], 16 * mt, 16 * ks));
+#pragma unroll
+      for (int qq = 0; qq < 2; qq++) ldsm_x4(aw[qq], afrag_addr(sm.W[qq], 16 * mt, 16 * ks));
+#pragma unroll
+      for (int np = 0; np < 2; np++) {
+        uint32_t bu[2][4];
+#pragma unroll
+        for (int qq = 0; qq < 2; qq++)
+          ldsm_x4(bu[qq], bfrag_nk_addr(sm.U[qq], 32 * nh + 16 * np, 16 * ks));
+        using PY = SplitPairs<1, 2>;
+#pragma unroll
+        for (int p = 0; p < PY::kCount; p++) {
+          mma16816(y[2 * np], ad[PY::a(p)], bu[PY::b(p)][0], bu[PY::b(p)][1]);
+          mma16816(y[2 * np + 1], ad[PY::a(p)], bu[PY::b(p)][2], bu[PY::b(p)][3]);
+        }
+        using PX = SplitPairs<2, 2>;
+#pragma unroll
+        for (int p = 0; p < PX::kCount; p++) {
+          mma16816(x[2 * np], aw[PX::a(p)], bu[PX::b(p)][0], bu[PX::b(p)][1]);
+          mma16816(x[2 * np + 1], aw[PX::a(p)], bu[PX::b(p)][2], bu[PX::b(p)][3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < 4; n++)
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        const int t = 16 * mt + gq + 8 * (e >> 1), s = 32 * nh + 8 * n + 2 * tq + (e & 1);
+        float av = 0.f, bv = 0.f;
+        if (s <= t) {
+          const float dec = expf(__double2float_rn(sm.G[t] - sm.G[s]));
+          av = __fmul_rn(dec, y[n][e]);
+          if (s < t) bv = -__fmul_rn(__fmul_rn(sm.bet[t], dec), x[n][e]);
+        }
+        put_terms(sm.A, t, s, av);
+        if (s <= t) {
+          put_terms(sm.Bn, t, s, bv);
+          if (s < t) put_terms(sm.Bn, s, t, bv);
+        }
+      }
+  }
+
+  // 2. The slab products.
+  float aq[NT8][4], aw[NT8][4], au[NT8][4];
+#pragma unroll
+  for (int n = 0; n < NT8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) aq[n][e] = aw[n][e] = au[n][e] = 0.f;
+  static_assert(SLI <= kGemmThreads, "one slab item per thread at most");
+  for (int j = 0; j < NS; j++) {
+    __syncthreads();  // the previous slab's terms are no longer read
+    if (slab_item) {
+      uint4 hi, lo;
+      split8(sx[0], sx[1], hi, lo);
+      *reinterpret_cast<uint4*>(&sm.Sp[0][core_off<kSlab>(sr, sc)]) = hi;
+      *reinterpret_cast<uint4*>(&sm.Sp[1][core_off<kSlab>(sr, sc)]) = lo;
+      split8(mx[0], mx[1], hi, lo);
+      *reinterpret_cast<uint4*>(&sm.Mp[0][core_off<kSlab>(sr, sc)]) = hi;
+      *reinterpret_cast<uint4*>(&sm.Mp[1][core_off<kSlab>(sr, sc)]) = lo;
+    }
+    if (j + 1 < NS) slab_load(j + 1);  // in flight during this slab's products
+    __syncthreads();
+    uint32_t ad[1][4], awf[2][4], auf[2][4];
+    ldsm_x4(ad[0], afrag_addr(sm.DO[0], 16 * mt, 16 * j));
+#pragma unroll
+    for (int qq = 0; qq < 2; qq++) {
+      ldsm_x4(awf[qq], afrag_addr(sm.W[qq], 16 * mt, 16 * j));
+      ldsm_x4(auf[qq], afrag_addr(sm.U[qq], 16 * mt, 16 * j));
+    }
+#pragma unroll
+    for (int np = 0; np < NT8 / 2; np++) {
+      const int n0 = (D / 2) * nh + 16 * np;
+      uint32_t bs[2][4], bm[2][4];
+#pragma unroll
+      for (int qq = 0; qq < 2; qq++) {
+        ldsm_x4_t(bs[qq], bfrag_kn16_addr(sm.Sp[qq], n0));
+        ldsm_x4_t(bm[qq], bfrag_kn16_addr(sm.Mp[qq], n0));
+      }
+      using P1 = SplitPairs<1, 2>;
+#pragma unroll
+      for (int p = 0; p < P1::kCount; p++) {
+        mma16816(aq[2 * np], ad[P1::a(p)], bs[P1::b(p)][0], bs[P1::b(p)][1]);
+        mma16816(aq[2 * np + 1], ad[P1::a(p)], bs[P1::b(p)][2], bs[P1::b(p)][3]);
+      }
+      using P2 = SplitPairs<2, 2>;
+#pragma unroll
+      for (int p = 0; p < P2::kCount; p++) {
+        mma16816(aw[2 * np], awf[P2::a(p)], bs[P2::b(p)][0], bs[P2::b(p)][1]);
+        mma16816(aw[2 * np + 1], awf[P2::a(p)], bs[P2::b(p)][2], bs[P2::b(p)][3]);
+      }
+#pragma unroll
+      for (int p = 0; p < P2::kCount; p++) {
+        mma16816(au[2 * np], auf[P2::a(p)], bm[P2::b(p)][0], bm[P2::b(p)][1]);
+        mma16816(au[2 * np + 1], auf[P2::a(p)], bm[P2::b(p)][2], bm[P2::b(p)][3]);
+      }
+    }
+  }
+
+  // 3. Row factors, then the C x C products.
+  const double GL = sm.G[kChunk - 1];  // = G_{L-1}: the padding's g is 0
+#pragma unroll
+  for (int hf = 0; hf < 2; hf++) {
+    const int t = 16 * mt + gq + 8 * hf;
+    const float eg = expf(__double2float_rn(sm.G[t]));
+    const float fw = -__fmul_rn(sm.bet[t], eg), fu = expf(__double2float_rn(GL - sm.G[t]));
+#pragma unroll
+    for (int n = 0; n < NT8; n++)
+#pragma unroll
+      for (int e = 2 * hf; e < 2 * hf + 2; e++) {
+        aq[n][e] = __fmul_rn(eg, aq[n][e]);
+        aw[n][e] = __fmaf_rn(fu, au[n][e], __fmul_rn(fw, aw[n][e]));
+        au[n][e] = 0.f;
+      }
+  }
+#pragma unroll
+  for (int ks = 0; ks < kChunk / 16; ks++) {
+    uint32_t fa[2][4], fat[2][4], fb[2][4];
+#pragma unroll
+    for (int qq = 0; qq < 2; qq++) {
+      ldsm_x4(fa[qq], afrag_addr(sm.A[qq], 16 * mt, 16 * ks));
+      ldsm_x4_t(fat[qq], afrag_t_addr(sm.A[qq], 16 * mt, 16 * ks));
+      ldsm_x4(fb[qq], afrag_addr(sm.Bn[qq], 16 * mt, 16 * ks));
+    }
+#pragma unroll
+    for (int np = 0; np < NT8 / 2; np++) {
+      const int n0 = (D / 2) * nh + 16 * np;
+      uint32_t bk[1][4], bq[1][4];
+      ldsm_x4_t(bk[0], bfrag_kn_addr(sm.K[0], 16 * ks, n0));
+      ldsm_x4_t(bq[0], bfrag_kn_addr(sm.Q[0], 16 * ks, n0));
+      using P3 = SplitPairs<2, 1>;
+#pragma unroll
+      for (int p = 0; p < P3::kCount; p++) {
+        mma16816(aq[2 * np], fa[P3::a(p)], bk[0][0], bk[0][1]);
+        mma16816(aq[2 * np + 1], fa[P3::a(p)], bk[0][2], bk[0][3]);
+        mma16816(au[2 * np], fat[P3::a(p)], bq[0][0], bq[0][1]);
+        mma16816(au[2 * np + 1], fat[P3::a(p)], bq[0][2], bq[0][3]);
+        mma16816(aw[2 * np], fb[P3::a(p)], bk[0][0], bk[0][1]);
+        mma16816(aw[2 * np + 1], fb[P3::a(p)], bk[0][2], bk[0][3]);
+      }
+    }
+  }
+  // DK = (row terms + Bn K) + scale (A^T Q); DQ = scale (diag(e^G) Pq + A K).
+#pragma unroll
+  for (int n = 0; n < NT8; n++)
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+      const int t = 16 * mt + gq + 8 * hf;
+      if (t >= len) continue;
+      const int col = (D / 2) * nh + 8 * n + 2 * tq;
+      const size_t o = (tb + (size_t)t * H) * D + col;
+      *reinterpret_cast<float2*>(d_q + o) =
+          f2(__fmul_rn(scale, aq[n][2 * hf]), __fmul_rn(scale, aq[n][2 * hf + 1]));
+      *reinterpret_cast<float2*>(d_k + o) =
+          f2(__fmaf_rn(scale, au[n][2 * hf], aw[n][2 * hf]),
+             __fmaf_rn(scale, au[n][2 * hf + 1], aw[n][2 * hf + 1]));
+    }
+}
+
+// ----------------------------------------------------------------------------
 // Launcher
 // ----------------------------------------------------------------------------
 template <class KernelT>
@@ -682,12 +1001,21 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   }
   GDN_BWD_TRY(mark(3));
   {
-    auto kern = k_bwd_gemm<D, IN>;
-    const size_t sm = sizeof(GemmSmem<D, IN>);
-    GDN_BWD_TRY(bwd_set_smem(kern, sm));
-    kern<<<gchunks, kGemmThreads, sm, st>>>(q, k, f.beta, f.g, d_o, f.cu_seqlens, f.H, f.scale,
-                                            hdr, chunk_off, chunk_seq, bstate, mu_end, wbuf, ubuf,
-                                            a.d_q, a.d_k);
+    if constexpr (sizeof(IN) == 2) {  // bf16 inputs: the products on the tensor cores
+      auto kern = k_bwd_gemm_tc<D>;
+      const size_t sm = sizeof(GemmTcSmem<D>);
+      GDN_BWD_TRY(bwd_set_smem(kern, sm));
+      kern<<<gchunks, kGemmThreads, sm, st>>>(q, k, f.beta, f.g, d_o, f.cu_seqlens, f.H, f.scale,
+                                              hdr, chunk_off, chunk_seq, bstate, mu_end, wbuf,
+                                              ubuf, a.d_q, a.d_k);
+    } else {  // fp32 inputs: fp32 fused multiply-adds (their tighter bound)
+      auto kern = k_bwd_gemm<D, IN>;
+      const size_t sm = sizeof(GemmSmem<D, IN>);
+      GDN_BWD_TRY(bwd_set_smem(kern, sm));
+      kern<<<gchunks, kGemmThreads, sm, st>>>(q, k, f.beta, f.g, d_o, f.cu_seqlens, f.H, f.scale,
+                                              hdr, chunk_off, chunk_seq, bstate, mu_end, wbuf,
+                                              ubuf, a.d_q, a.d_k);
+    }
     GDN_BWD_TRY(cudaGetLastError());
   }
   return mark(4);
