@@ -197,3 +197,62 @@ def test_chunked_adjoint_equals_the_token_recurrence(C):
             assert ends.keys() == ends2.keys()
             for e in ends:
                 assert np.max(np.abs(ends2[e] - ends[e])) < 1e-12
+
+
+def kernel_adjoint(q, k, beta, g, cu, do, dsf, scale, C, n, h):
+    """The chunk form of the adjoint as the bf16-input CUDA backward evaluates
+    it (k_adj_prep, k_adj_walk, k_adj_w), with T = (I + A)^{-1} from the
+    forward prep, Tb = T diag(beta e^G), dvec = e^{G_{L-1} - G} and
+    Pm[r][t] = [t <= r] e^{G_r - G_t} q_r . k_t:
+      X   = scale (diag(e^G) Q - Pm Tb K)                      (per chunk)
+      mu <- e^{G_{L-1}} mu - ((mu K^T) diag(dvec)) Tb K + DO^T X  (serial walk)
+      W   = T^T (diag(dvec) (mu_e K^T)^T + scale Pm^T DO)        (per chunk)
+    Returns (W, mu at every chunk end, dh0)."""
+    a0, e0 = int(cu[n]), int(cu[n + 1])
+    d = q.shape[2]
+    W, mu_end, pre = np.zeros((e0 - a0, d)), {}, {}
+    for a in range(a0, e0, C):
+        e = min(a + C, e0)
+        L = e - a
+        G = np.cumsum(g[a:e, h])
+        K, Q, DO, bt = k[a:e, h], q[a:e, h], do[a:e, h], beta[a:e, h]
+        ii = np.arange(L)
+        A = (np.where(ii[:, None] > ii[None, :], np.exp(G[:, None] - G[None, :]), 0.0)
+             * (K @ K.T) * bt[:, None])
+        T = np.linalg.inv(np.eye(L) + A)
+        Tb = T * (bt * np.exp(G))[None, :]
+        dvec = np.exp(G[-1] - G)
+        Pm = np.where(ii[None, :] <= ii[:, None], np.exp(G[:, None] - G[None, :]), 0.0) * (Q @ K.T)
+        X = scale * (np.exp(G)[:, None] * Q - Pm @ Tb @ K)
+        pre[a] = (K, DO, T, Tb, dvec, Pm, X, np.exp(G[-1]))
+    mu = dsf[n, h].copy()
+    for a in reversed(range(a0, e0, C)):
+        e = min(a + C, e0)
+        K, DO, T, Tb, dvec, Pm, X, gam = pre[a]
+        mu_end[e] = mu.copy()
+        Ydv = (mu @ K.T) * dvec[None, :]                       # [row][t]
+        W[a - a0:e - a0] = T.T @ (Ydv.T + scale * Pm.T @ DO)
+        mu = gam * mu - (Ydv @ Tb) @ K + DO.T @ X
+    return W, mu_end, mu
+
+
+@pytest.mark.parametrize("C", [1, 3, 16, 64])
+def test_kernel_adjoint_form_equals_the_token_recurrence(C):
+    q, k, v, beta, g, cu, h0, do, dsf = _batch([1, 63, 64, 65, 130, 0, 7], 2, 6, seed=30 + C)
+    scale = 0.6
+    for n in range(len(cu) - 1):
+        a0, e0 = int(cu[n]), int(cu[n + 1])
+        for h in range(2):
+            mu, W, ends = dsf[n, h].copy(), np.zeros((e0 - a0, 6)), {}
+            for j in range(e0 - 1, a0 - 1, -1):
+                if (j - a0) % C == C - 1 or j == e0 - 1:
+                    ends[j + 1] = mu.copy()
+                lam = mu + scale * np.outer(do[j, h], q[j, h])
+                W[j - a0] = lam @ k[j, h]
+                mu = np.exp(g[j, h]) * (lam - beta[j, h] * np.outer(W[j - a0], k[j, h]))
+            W2, ends2, mu2 = kernel_adjoint(q, k, beta, g, cu, do, dsf, scale, C, n, h)
+            assert np.max(np.abs(W2 - W), initial=0.0) < 1e-12
+            assert np.max(np.abs(mu2 - mu)) < 1e-12
+            assert ends.keys() == ends2.keys()
+            for e in ends:
+                assert np.max(np.abs(ends2[e] - ends[e])) < 1e-12
