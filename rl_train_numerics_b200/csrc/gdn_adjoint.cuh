@@ -1,0 +1,538 @@
+// gdn_adjoint.cuh -- the adjoint of the CPR backward in chunk form (bf16
+// inputs): a chunk-parallel prep, a serial reverse walk over chunk ends, and
+// a chunk-parallel solve for the per-token vectors w.
+//
+// The token recurrence of the adjoint (gdn_backward.cu's header), per
+// (sequence, head) and chunk of length L with T = (I + A)^{-1} of the
+// forward's boundary prep, Tb = T diag(beta e^G), dvec = e^{G_{L-1} - G},
+// gamma = e^{G_{L-1}} and Pm[r][t] = [t <= r] e^{G_r - G_t} q_r . k_t,
+// unrolls to
+//   X       = scale (diag(e^G) Q - Pm Tb K)                         (L x d_k)
+//   mu_a    = gamma mu_e - ((mu_e K^T) diag(dvec)) Tb K + DO^T X     (the
+//             chunk map of the adjoint: the forward boundary map's linear
+//             part transposed, plus the chunk's own do terms)
+//   W       = T^T (diag(dvec) (mu_e K^T)^T + scale Pm^T DO)          (L x d_v)
+// with mu_e the adjoint at the chunk's end and mu_a at its start (the end of
+// the chunk before).  The identities are exact (pinned in float64 by
+// tests/test_backward_algebra.py); the kernels evaluate them on the tensor
+// cores (mma.sync m16n8k16) with every fp32 operand split exactly into three
+// bf16 terms and all term pairs down to the third term's order accumulated in
+// fp32 (fp32 accuracy; keys, queries and do are exact in bf16).  The walk is
+// the only serial part: a chain of L x d x d products per chunk instead of the
+// token scan's chain per token.
+//   k_adj_prep  per (chunk, head): the forward prep's T (trailing partial
+//               chunks zero-padded), Pm, X; writes the chunk's adjoint pack
+//   k_adj_walk  per (sequence, head, 32 state rows), last chunk first: mu at
+//               every chunk end, dh0, and Ydv = (mu_e K^T) diag(dvec)
+//   k_adj_w     per (chunk, head): W -> w and dv = beta w
+#pragma once
+
+#include <cstddef>
+
+#include "gdn_boundary.cuh"
+#include "gdn_fill.cuh"
+
+namespace gdn {
+
+constexpr int kAdjNT = 3;  // bf16 terms of an fp32 operand
+
+// The adjoint pack of one (chunk, head).  Planes are bf16 in the core layout
+// (64 rows); the walk bulk-copies [0, offsetof(T)), the solve the rest.
+template <int D>
+struct AdjPack {
+  float dvec[kChunk];
+  float beta[kChunk];  // 0 past the chunk's length
+  float gamma[4];      // [0] = e^{G_{L-1}}
+  __nv_bfloat16 K[1][kChunk * D];               // [t][j]
+  __nv_bfloat16 DO[1][kChunk * D];              // [t][i]
+  __nv_bfloat16 X[kAdjNT][kChunk * D];          // [t][j]
+  __nv_bfloat16 Tb[kAdjNT][kChunk * kChunk];    // [t][m], m <= t
+  __nv_bfloat16 T[kAdjNT][kChunk * kChunk];     // [m][t], t <= m
+  __nv_bfloat16 Pm[kAdjNT][kChunk * kChunk];    // [r][t], t <= r
+};
+template <int D>
+constexpr size_t adj_walk_bytes() {
+  return offsetof(AdjPack<D>, T);
+}
+template <int D>
+constexpr size_t adj_pack_bytes() {
+  return round_up(sizeof(AdjPack<D>), 128);
+}
+
+// Three-term split of (x0, x1) stored as bf16 pairs at element offset off of
+// three planes nelem elements apart.
+__device__ __forceinline__ void put3(__nv_bfloat16* p, size_t nelem, int off, float x0, float x1) {
+  __nv_bfloat16 a[kAdjNT], b[kAdjNT];
+  split_bf16<kAdjNT>(x0, a);
+  split_bf16<kAdjNT>(x1, b);
+#pragma unroll
+  for (int q = 0; q < kAdjNT; q++)
+    *reinterpret_cast<uint32_t*>(p + q * nelem + off) = pack_bf16(a[q], b[q]);
+}
+
+// ----------------------------------------------------------------------------
+// k_adj_prep
+// ----------------------------------------------------------------------------
+template <int D>
+struct AdjPrepSmem {
+  PrepSmem<D, __nv_bfloat16> prep;  // head reused for the Tb terms once the prep is done
+  PrepAT AT;
+  __nv_bfloat16 Q[1][kChunk * D];
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBndThreads, 2)
+    k_adj_prep(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+               const __nv_bfloat16* __restrict__ d_o, const float* __restrict__ beta,
+               const float* __restrict__ g, const int32_t* __restrict__ cu, int H, float scale,
+               const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+               const int32_t* __restrict__ chunk_seq, char* __restrict__ apacks) {
+  using bf16 = __nv_bfloat16;
+  constexpr int C = kChunk, PL = C * C, PD = C * D;
+  static_assert(sizeof(PackHead<D, bf16>) >= kAdjNT * PL * sizeof(bf16), "Tb terms fit the head");
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  AdjPrepSmem<D>& sm = *reinterpret_cast<AdjPrepSmem<D>*>(smem_raw);
+  if (hdr[kHdrValid] != 1) return;
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (c >= hdr[kHdrChunks]) return;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+  const FillItem it = fill_item(c * H + h, H, cu, chunk_off, chunk_seq);
+  const int len = it.len;
+  const size_t tok = (size_t)it.t0 * H + h;
+  AdjPack<D>& pk = *reinterpret_cast<AdjPack<D>*>(apacks + ((size_t)c * H + h) * adj_pack_bytes<D>());
+
+  PlaneRows<D, bf16, kBndThreads> dorows;  // do rows in flight during the prep
+  dorows.load(d_o + tok * D, (size_t)H * D, len);
+  stage_planes<D, bf16>(sm.Q, q + tok * D, (size_t)H * D, kBndThreads, len);
+  prep_stage<D, bf16>(sm.prep, k + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H, len);
+  bnd_prep<D, bf16>(sm.prep, sm.AT);
+
+  if (tid < C) {
+    pk.dvec[tid] = sm.prep.head.dvec[tid];
+    pk.beta[tid] = sm.prep.beta[tid];
+  }
+  if (tid < 4) pk.gamma[tid] = sm.prep.head.gamma[tid];
+  for (int e = tid; e < PD / 8; e += kBndThreads)
+    reinterpret_cast<uint4*>(pk.K[0])[e] = reinterpret_cast<const uint4*>(sm.prep.K[0])[e];
+  dorows.store(pk.DO);
+  // T (rows m, columns t) and Tb = T diag(beta e^G) (rows t, columns m).
+  bf16* tb3 = reinterpret_cast<bf16*>(&sm.prep.head);
+  for (int e = tid; e < PL / 2; e += kBndThreads) {
+    const int i = e / (C / 2), j = 2 * (e % (C / 2));
+    const float t0 = i >= j ? sm.AT[i][j] : 0.f, t1 = i >= j + 1 ? sm.AT[i][j + 1] : 0.f;
+    const float b0 = __fmul_rn(t0, sm.prep.bg[j]), b1 = __fmul_rn(t1, sm.prep.bg[j + 1]);
+    const int off = core_off<C>(i, j);
+    put3(pk.T[0], PL, off, t0, t1);
+    put3(pk.Tb[0], PL, off, b0, b1);
+    put3(tb3, PL, off, b0, b1);
+  }
+  __syncthreads();
+
+  // Pm on warp w's rows 16w .. 16w + 15 (n8 tiles up to the diagonal block).
+  float pm[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) pm[n][e] = 0.f;
+#pragma unroll 2
+  for (int ks = 0; ks < D / 16; ks++) {
+    uint32_t a[4];
+    ldsm_x4(a, afrag_addr(sm.Q[0], 16 * w, 16 * ks));
+#pragma unroll
+    for (int np = 0; np < 4; np++) {
+      if (np <= w) {
+        uint32_t b[4];
+        ldsm_x4(b, bfrag_nk_addr(sm.prep.K[0], 16 * np, 16 * ks));
+        mma16816(pm[2 * np], a, b[0], b[1]);
+        mma16816(pm[2 * np + 1], a, b[2], b[3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < 8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const int r = 16 * w + gq + 8 * (e >> 1), t = 8 * n + 2 * tq + (e & 1);
+      pm[n][e] = (t <= r && r < len)
+                     ? __fmul_rn(expf(__double2float_rn(sm.prep.G[r] - sm.prep.G[t])), pm[n][e])
+                     : 0.f;
+    }
+#pragma unroll
+  for (int n = 0; n < 8; n++)
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++)
+      put3(pk.Pm[0], PL, core_off<C>(16 * w + gq + 8 * hf, 8 * n + 2 * tq), pm[n][2 * hf],
+           pm[n][2 * hf + 1]);
+
+  // Y2 = Pm Tb on the same rows (both lower triangular).
+  float y2[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) y2[n][e] = 0.f;
+  using P33 = SplitPairs<kAdjNT, kAdjNT>;
+  using P31 = SplitPairs<kAdjNT, 1>;
+#pragma unroll
+  for (int ks = 0; ks < 4; ks++) {
+    if (ks > w) continue;
+    uint32_t a[kAdjNT][4];
+    acc_to_afrag<kAdjNT>(pm[2 * ks], pm[2 * ks + 1], a);
+#pragma unroll
+    for (int np = 0; np < 4; np++) {
+      if (np > ks) continue;
+      uint32_t b[kAdjNT][4];
+#pragma unroll
+      for (int qq = 0; qq < kAdjNT; qq++) ldsm_x4_t(b[qq], bfrag_kn_addr(tb3 + qq * PL, 16 * ks, 16 * np));
+#pragma unroll
+      for (int p = 0; p < P33::kCount; p++) {
+        mma16816(y2[2 * np], a[P33::a(p)], b[P33::b(p)][0], b[P33::b(p)][1]);
+        mma16816(y2[2 * np + 1], a[P33::a(p)], b[P33::b(p)][2], b[P33::b(p)][3]);
+      }
+    }
+  }
+  // X = scale (e^{G_r} q_r - (Y2 K)_r), rows of this warp.
+  float x[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) x[n][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 4; ks++) {
+    if (ks > w) continue;
+    uint32_t a[kAdjNT][4];
+    acc_to_afrag<kAdjNT>(y2[2 * ks], y2[2 * ks + 1], a);
+#pragma unroll
+    for (int np = 0; np < D / 16; np++) {
+      uint32_t b[4];
+      ldsm_x4_t(b, bfrag_kn_addr(sm.prep.K[0], 16 * ks, 16 * np));
+#pragma unroll
+      for (int p = 0; p < P31::kCount; p++) {
+        mma16816(x[2 * np], a[P31::a(p)], b[0], b[1]);
+        mma16816(x[2 * np + 1], a[P31::a(p)], b[2], b[3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int hf = 0; hf < 2; hf++) {
+    const int r = 16 * w + gq + 8 * hf;
+    const float eg = expf(__double2float_rn(sm.prep.G[r]));
+#pragma unroll
+    for (int n = 0; n < D / 8; n++) {
+      const int j = 8 * n + 2 * tq, off = core_off<C>(r, j);
+      const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162*>(&sm.Q[0][off]);
+      const float x0 = __fmul_rn(scale, __fsub_rn(__fmul_rn(eg, __low2float(qv)), x[n][2 * hf]));
+      const float x1 =
+          __fmul_rn(scale, __fsub_rn(__fmul_rn(eg, __high2float(qv)), x[n][2 * hf + 1]));
+      put3(pk.X[0], PD, off, x0, x1);
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// k_adj_walk
+// ----------------------------------------------------------------------------
+constexpr int kAdjWalkWarps = 2;  // 32 state rows per block
+
+template <int D>
+struct AdjWalkSmem {
+  alignas(128) unsigned char buf[2][round_up(adj_walk_bytes<D>(), 128)];
+  uint64_t bar[2];
+};
+
+// One reverse step on a warp's 16 state rows (sacc, accumulator layout):
+//   Ydv = (mu K^T) diag(dvec)  (written to ydv_rows, [row][t])
+//   mu <- gamma mu + (-Ydv) Tb K + DO^T X
+template <int D>
+__device__ __forceinline__ void adj_walk_warp(float (&sacc)[D / 8][4], const unsigned char* pb,
+                                              int r0, float* ydv_rows) {
+  using bf16 = __nv_bfloat16;
+  constexpr int C = kChunk, PL = C * C, PD = C * D;
+  const AdjPack<D>& pk = *reinterpret_cast<const AdjPack<D>*>(pb);
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  using P33 = SplitPairs<kAdjNT, kAdjNT>;
+  using P31 = SplitPairs<kAdjNT, 1>;
+  using P13 = SplitPairs<1, kAdjNT>;
+  float y[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) y[n][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ks++) {
+    uint32_t a[kAdjNT][4];
+    acc_to_afrag<kAdjNT>(sacc[2 * ks], sacc[2 * ks + 1], a);
+#pragma unroll
+    for (int np = 0; np < 4; np++) {
+      uint32_t b[4];
+      ldsm_x4(b, bfrag_nk_addr(pk.K[0], 16 * np, 16 * ks));
+#pragma unroll
+      for (int p = 0; p < P31::kCount; p++) {
+        mma16816(y[2 * np], a[P31::a(p)], b[0], b[1]);
+        mma16816(y[2 * np + 1], a[P31::a(p)], b[2], b[3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < 8; n++) {
+    const int t = 8 * n + 2 * tq;
+    const float d0 = pk.dvec[t], d1 = pk.dvec[t + 1];
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+      y[n][2 * hf] = __fmul_rn(d0, y[n][2 * hf]);
+      y[n][2 * hf + 1] = __fmul_rn(d1, y[n][2 * hf + 1]);
+      *reinterpret_cast<float2*>(ydv_rows + (size_t)(gq + 8 * hf) * C + t) =
+          f2(y[n][2 * hf], y[n][2 * hf + 1]);
+    }
+  }
+  // Z = (-Ydv) Tb
+  float z[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) z[n][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 4; ks++) {
+    float n0[4], n1[4];
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      n0[e] = -y[2 * ks][e];
+      n1[e] = -y[2 * ks + 1][e];
+    }
+    uint32_t a[kAdjNT][4];
+    acc_to_afrag<kAdjNT>(n0, n1, a);
+#pragma unroll
+    for (int np = 0; np < 4; np++) {
+      if (np > ks) continue;
+      uint32_t b[kAdjNT][4];
+#pragma unroll
+      for (int qq = 0; qq < kAdjNT; qq++)
+        ldsm_x4_t(b[qq], bfrag_kn_addr(pk.Tb[qq], 16 * ks, 16 * np));
+#pragma unroll
+      for (int p = 0; p < P33::kCount; p++) {
+        mma16816(z[2 * np], a[P33::a(p)], b[P33::b(p)][0], b[P33::b(p)][1]);
+        mma16816(z[2 * np + 1], a[P33::a(p)], b[P33::b(p)][2], b[P33::b(p)][3]);
+      }
+    }
+  }
+  // mu <- gamma mu, then + Z K, then + DO^T X
+  const float gam = pk.gamma[0];
+#pragma unroll
+  for (int n = 0; n < D / 8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) sacc[n][e] = __fmul_rn(gam, sacc[n][e]);
+#pragma unroll
+  for (int ks = 0; ks < 4; ks++) {
+    uint32_t a[kAdjNT][4];
+    acc_to_afrag<kAdjNT>(z[2 * ks], z[2 * ks + 1], a);
+#pragma unroll
+    for (int np = 0; np < D / 16; np++) {
+      uint32_t b[4];
+      ldsm_x4_t(b, bfrag_kn_addr(pk.K[0], 16 * ks, 16 * np));
+#pragma unroll
+      for (int p = 0; p < P31::kCount; p++) {
+        mma16816(sacc[2 * np], a[P31::a(p)], b[0], b[1]);
+        mma16816(sacc[2 * np + 1], a[P31::a(p)], b[2], b[3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int ks = 0; ks < 4; ks++) {
+    uint32_t a[1][4];
+    ldsm_x4_t(a[0], afrag_t_addr(pk.DO[0], r0, 16 * ks));
+#pragma unroll
+    for (int np = 0; np < D / 16; np++) {
+      uint32_t b[kAdjNT][4];
+#pragma unroll
+      for (int qq = 0; qq < kAdjNT; qq++)
+        ldsm_x4_t(b[qq], bfrag_kn_addr(pk.X[qq], 16 * ks, 16 * np));
+#pragma unroll
+      for (int p = 0; p < P13::kCount; p++) {
+        mma16816(sacc[2 * np], a[P13::a(p)], b[P13::b(p)][0], b[P13::b(p)][1]);
+        mma16816(sacc[2 * np + 1], a[P13::a(p)], b[P13::b(p)][2], b[P13::b(p)][3]);
+      }
+    }
+  }
+  (void)PL;
+  (void)PD;
+}
+
+template <int D>
+__global__ void __launch_bounds__(32 * kAdjWalkWarps, 1)
+    k_adj_walk(const int32_t* __restrict__ cu, int H, int32_t* __restrict__ hdr,
+               const int32_t* __restrict__ chunk_off, const char* __restrict__ apacks,
+               const float* __restrict__ ds_final, float* __restrict__ mu_end,
+               float* __restrict__ ydv, float* __restrict__ d_h0) {
+  constexpr int C = kChunk;
+  constexpr uint32_t WB = (uint32_t)adj_walk_bytes<D>();
+  static_assert(WB % 16 == 0, "bulk copies are 16-byte pieces");
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  AdjWalkSmem<D>& sm = *reinterpret_cast<AdjWalkSmem<D>*>(smem_raw);
+  if (hdr[kHdrValid] != 1) return;
+  const int n = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
+  const int r0 = blockIdx.z * 16 * kAdjWalkWarps + 16 * (t >> 5);
+  const size_t DD = (size_t)D * D;
+  const int64_t L = (int64_t)cu[n + 1] - cu[n];
+  const int64_t nc = (L + C - 1) / C;
+  const int64_t base = chunk_off[n];
+  auto pack = [&](int64_t cc) {
+    return apacks + ((size_t)(base + cc) * H + h) * adj_pack_bytes<D>();
+  };
+  auto fetch = [&](int b, int64_t cc) {
+    const uint32_t mb = smem_u32(&sm.bar[b]);
+    mbar_expect_tx(mb, WB);
+    bulk_load(smem_u32(sm.buf[b]), pack(cc), WB, mb);
+  };
+  pack_bars_init(sm.bar);
+  float sacc[D / 8][4];
+  if (ds_final) sacc_load<D>(sacc, ds_final + ((size_t)n * H + h) * DD, r0);
+  else sacc_zero<D>(sacc);
+  if (t == 0 && nc > 0) fetch(0, nc - 1);
+  int64_t issued = nc > 0 ? 1 : 0;
+  bool ok = true;
+  for (int64_t j = 0; j < nc; j++) {
+    const int64_t cc = nc - 1 - j;
+    if (cc >= 1) {
+      if (t == 0) fetch((int)((j + 1) & 1), cc - 1);
+      issued = j + 2;
+    }
+    const size_t unit = (size_t)(base + cc) * H + h;
+    sacc_store<D>(sacc, mu_end + unit * DD, r0);
+    if (__syncthreads_or(!pack_wait(sm.bar, j))) {
+      ok = false;
+      pack_drain(sm.bar, j, issued);
+      break;
+    }
+    adj_walk_warp<D>(sacc, sm.buf[j & 1], r0, ydv + (unit * D + r0) * C);
+    __syncthreads();  // buffer j & 1 is refilled with chunk cc - 2
+  }
+  if (!ok) {
+    if (t == 0) atomicOr(&hdr[kHdrError], kErrTimeout);
+    return;
+  }
+  if (d_h0) sacc_store<D>(sacc, d_h0 + ((size_t)n * H + h) * DD, r0);
+}
+
+// ----------------------------------------------------------------------------
+// k_adj_w
+// ----------------------------------------------------------------------------
+constexpr int kAdjWThreads = 256;
+
+template <int D>
+struct AdjWSmem {
+  float dvec[kChunk];
+  float beta[kChunk];
+  float gamma[4];
+  __nv_bfloat16 DO[1][kChunk * D];                 // [r][i]
+  __nv_bfloat16 T[kAdjNT][kChunk * kChunk];        // [m][t]
+  __nv_bfloat16 Pm[kAdjNT][kChunk * kChunk];       // [r][t]
+  __nv_bfloat16 R[kAdjNT][kChunk * D];             // right-hand side, [m][i]
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAdjWThreads, 1)
+    k_adj_w(const int32_t* __restrict__ cu, int H, float scale, const int32_t* __restrict__ hdr,
+            const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
+            const char* __restrict__ apacks, const float* __restrict__ ydv,
+            float* __restrict__ wbuf, float* __restrict__ d_v) {
+  using bf16 = __nv_bfloat16;
+  constexpr int C = kChunk, PL = C * C, PD = C * D, NT8 = D / 16;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  AdjWSmem<D>& sm = *reinterpret_cast<AdjWSmem<D>*>(smem_raw);
+  if (hdr[kHdrValid] != 1) return;
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (c >= hdr[kHdrChunks]) return;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+  const int mt = w & 3, nh = w >> 2;
+  const FillItem it = fill_item(c * H + h, H, cu, chunk_off, chunk_seq);
+  const int len = it.len;
+  const size_t tb = (size_t)it.t0 * H + h;
+  const AdjPack<D>& pk =
+      *reinterpret_cast<const AdjPack<D>*>(apacks + ((size_t)c * H + h) * adj_pack_bytes<D>());
+  // The pack's head, do plane, T and Pm terms (16-byte pieces).
+  for (int e = tid; e < (int)(2 * C + 4) / 4; e += kAdjWThreads)
+    cp_async16(reinterpret_cast<float4*>(sm.dvec) + e, reinterpret_cast<const float4*>(pk.dvec) + e);
+  for (int e = tid; e < PD / 8; e += kAdjWThreads)
+    cp_async16(reinterpret_cast<uint4*>(sm.DO[0]) + e, reinterpret_cast<const uint4*>(pk.DO[0]) + e);
+  for (int e = tid; e < 2 * kAdjNT * PL / 8; e += kAdjWThreads)
+    cp_async16(reinterpret_cast<uint4*>(sm.T[0]) + e, reinterpret_cast<const uint4*>(pk.T[0]) + e);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  using P33 = SplitPairs<kAdjNT, kAdjNT>;
+  using P31 = SplitPairs<kAdjNT, 1>;
+  // R = Ydv^T + scale Pm^T DO on warp (mt, nh)'s tile: tokens 16 mt .., rows
+  // i = (D / 2) nh .. (Pm^T[t][r] = Pm[r][t] vanishes for r < t).
+  float acc[NT8][4];
+#pragma unroll
+  for (int n = 0; n < NT8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) acc[n][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 4; ks++) {
+    if (ks < mt) continue;
+    uint32_t a[kAdjNT][4];
+#pragma unroll
+    for (int qq = 0; qq < kAdjNT; qq++) ldsm_x4_t(a[qq], afrag_t_addr(sm.Pm[qq], 16 * mt, 16 * ks));
+#pragma unroll
+    for (int np = 0; np < NT8 / 2; np++) {
+      uint32_t b[4];
+      ldsm_x4_t(b, bfrag_kn_addr(sm.DO[0], 16 * ks, (D / 2) * nh + 16 * np));
+#pragma unroll
+      for (int p = 0; p < P31::kCount; p++) {
+        mma16816(acc[2 * np], a[P31::a(p)], b[0], b[1]);
+        mma16816(acc[2 * np + 1], a[P31::a(p)], b[2], b[3]);
+      }
+    }
+  }
+  const float* yd = ydv + ((size_t)c * H + h) * D * C;
+#pragma unroll
+  for (int n = 0; n < NT8; n++)
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+      const int m = 16 * mt + gq + 8 * hf, i = (D / 2) * nh + 8 * n + 2 * tq;
+      const float r0v = __fmaf_rn(scale, acc[n][2 * hf], yd[(size_t)i * C + m]);
+      const float r1v = __fmaf_rn(scale, acc[n][2 * hf + 1], yd[(size_t)(i + 1) * C + m]);
+      put3(sm.R[0], PD, core_off<C>(m, i), r0v, r1v);
+    }
+  __syncthreads();
+  // W = T^T R (T^T[t][m] = T[m][t] vanishes for m < t).
+#pragma unroll
+  for (int n = 0; n < NT8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) acc[n][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 4; ks++) {
+    if (ks < mt) continue;
+    uint32_t a[kAdjNT][4];
+#pragma unroll
+    for (int qq = 0; qq < kAdjNT; qq++) ldsm_x4_t(a[qq], afrag_t_addr(sm.T[qq], 16 * mt, 16 * ks));
+#pragma unroll
+    for (int np = 0; np < NT8 / 2; np++) {
+      uint32_t b[kAdjNT][4];
+#pragma unroll
+      for (int qq = 0; qq < kAdjNT; qq++)
+        ldsm_x4_t(b[qq], bfrag_kn_addr(sm.R[qq], 16 * ks, (D / 2) * nh + 16 * np));
+#pragma unroll
+      for (int p = 0; p < P33::kCount; p++) {
+        mma16816(acc[2 * np], a[P33::a(p)], b[P33::b(p)][0], b[P33::b(p)][1]);
+        mma16816(acc[2 * np + 1], a[P33::a(p)], b[P33::b(p)][2], b[P33::b(p)][3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NT8; n++)
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+      const int t = 16 * mt + gq + 8 * hf;
+      if (t >= len) continue;
+      const int i = (D / 2) * nh + 8 * n + 2 * tq;
+      const size_t o = (tb + (size_t)t * H) * D + i;
+      const float bt = sm.beta[t];
+      *reinterpret_cast<float2*>(wbuf + o) = f2(acc[n][2 * hf], acc[n][2 * hf + 1]);
+      *reinterpret_cast<float2*>(d_v + o) =
+          f2(__fmul_rn(bt, acc[n][2 * hf]), __fmul_rn(bt, acc[n][2 * hf + 1]));
+    }
+}
+
+}  // namespace gdn

@@ -51,6 +51,7 @@
 //   k_bwd_gemm       one block per (chunk, head): DQ and DK from the
 //                    products above, in fp32 fused multiply-adds
 // Every sum has a fixed order, so repeated runs give identical bits.
+#include "gdn_adjoint.cuh"
 #include "gdn_boundary.cuh"
 #include "gdn_fill.cuh"
 #include "gdn_layout.h"
@@ -979,7 +980,39 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
   const IN* k = static_cast<const IN*>(f.k);
   const IN* v = static_cast<const IN*>(f.v);
   const IN* d_o = static_cast<const IN*>(a.d_o);
-  {
+  const dim3 gchunks((unsigned)L.fwd.max_chunks, (unsigned)f.H);
+  if constexpr (sizeof(IN) == 2) {
+    // bf16 inputs: the adjoint in chunk form (gdn_adjoint.cuh)
+    static_assert(adj_pack_bytes<D>() == adj_pack_bytes_host(D), "adjoint pack layout mismatch");
+    char* apack = ws + L.apack;
+    float* ydv = reinterpret_cast<float*>(ws + L.ydv);
+    int32_t* hdr_w = reinterpret_cast<int32_t*>(ws + L.fwd.hdr);
+    {
+      auto kern = k_adj_prep<D>;
+      const size_t sm = sizeof(AdjPrepSmem<D>);
+      GDN_BWD_TRY(bwd_set_smem(kern, sm));
+      kern<<<gchunks, kBndThreads, sm, st>>>(q, k, d_o, f.beta, f.g, f.cu_seqlens, f.H, f.scale,
+                                             hdr, chunk_off, chunk_seq, apack);
+      GDN_BWD_TRY(cudaGetLastError());
+    }
+    {
+      auto kern = k_adj_walk<D>;
+      const size_t sm = sizeof(AdjWalkSmem<D>);
+      GDN_BWD_TRY(bwd_set_smem(kern, sm));
+      kern<<<dim3((unsigned)f.n_seqs, (unsigned)f.H, D / (16 * kAdjWalkWarps)),
+             32 * kAdjWalkWarps, sm, st>>>(f.cu_seqlens, f.H, hdr_w, chunk_off, apack,
+                                           a.ds_final, mu_end, ydv, a.d_h0);
+      GDN_BWD_TRY(cudaGetLastError());
+    }
+    {
+      auto kern = k_adj_w<D>;
+      const size_t sm = sizeof(AdjWSmem<D>);
+      GDN_BWD_TRY(bwd_set_smem(kern, sm));
+      kern<<<gchunks, kAdjWThreads, sm, st>>>(f.cu_seqlens, f.H, f.scale, hdr, chunk_off,
+                                              chunk_seq, apack, ydv, wbuf, a.d_v);
+      GDN_BWD_TRY(cudaGetLastError());
+    }
+  } else {
     auto kern = k_bwd_scan<D, IN>;
     const size_t sm = sizeof(ScanSmem<D, IN>);
     GDN_BWD_TRY(bwd_set_smem(kern, sm));
@@ -988,7 +1021,6 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
         wbuf, a.d_v, a.d_h0);
     GDN_BWD_TRY(cudaGetLastError());
   }
-  const dim3 gchunks((unsigned)L.fwd.max_chunks, (unsigned)f.H);
   GDN_BWD_TRY(mark(2));
   {
     auto kern = k_bwd_rows<D, IN>;

@@ -148,9 +148,21 @@ struct BndArgs {
 //                            every chunk (from the tokens after it)
 //   wbuf    f32[T,H,dv]      w_t = Lambda_t k_t, one value per state row
 //   ubuf    f32[T,H,dv]      u_t = beta_t (v_t - alpha_t S_{t-1} k_t) per row
+//   with bf16 inputs (the adjoint in chunk form, gdn_adjoint.cuh), also
+//   apack   [MC,H] adjoint packs (mirrors adj_pack_bytes<D>(): head of
+//                  2C + 4 floats, keys and do as bf16 planes C x D, X as three
+//                  bf16 term planes C x D, Tb, T and Pm as three term planes
+//                  C x C each)
+//   ydv     f32[MC,H,dv,C]  (mu_e K^T) diag(dvec) per chunk (the walk's output)
+constexpr size_t adj_pack_bytes_host(int D) {
+  const size_t C = 64;
+  const size_t b = (2 * C + 4) * 4 + 2 * C * (size_t)D * 2 + 3 * C * (size_t)D * 2 + 9 * C * C * 2;
+  return (b + 127) / 128 * 128;
+}
+
 struct BwdLayout {
   FwdLayout fwd;
-  size_t mu_end, wbuf, ubuf, total;
+  size_t mu_end, wbuf, ubuf, apack, ydv, total;
 };
 
 inline BwdLayout bwd_layout(int n_seqs, int64_t T, int H, int dk, int dv, int C, bool in_bf16) {
@@ -163,6 +175,12 @@ inline BwdLayout bwd_layout(int n_seqs, int64_t T, int H, int dk, int dv, int C,
   off += align256((size_t)T * H * dv * sizeof(float));
   L.ubuf = off;
   off += align256((size_t)T * H * dv * sizeof(float));
+  L.apack = L.ydv = off;
+  if (in_bf16) {
+    off += align256((size_t)L.fwd.max_chunks * H * adj_pack_bytes_host(dk));
+    L.ydv = off;
+    off += align256((size_t)L.fwd.max_chunks * H * dv * C * sizeof(float));
+  }
   L.total = off;
   return L;
 }
