@@ -150,11 +150,12 @@ std::string descriptor(int kind, int in_dtype, int out_dtype, int dk, int dv, in
                                              : "state/Y/U 3 bf16 terms, Tb/Tv 3, K/V 3");
     s += line("backward",
               in_dtype == GDN_BF16
-                  ? "boundary states by the forward's first pass; adjoint scan per row (4 "
-                    "packed accumulators per lane, xor butterfly 1,2); chunk states by the "
-                    "step schedule; chunk products Y,X,DQ,DK by mma.sync m16n8k16 bf16 with "
-                    "w,u,S_a,mu_e,A,-(B+B^T) in 2 bf16 terms, pairs (hi,hi),(hi,lo),(lo,hi); "
-                    "dg by a telescoped sum"
+                  ? "boundary states by the forward's first pass; adjoint in chunk form "
+                    "(prep: T, Pm, X; reverse walk over chunk ends; W = T^T R) by mma.sync "
+                    "m16n8k16 bf16 with fp32 operands in 3 bf16 terms, all pairs of order < 3; "
+                    "chunk states by the step schedule; chunk products Y,X,DQ,DK by mma.sync "
+                    "with w,u,S_a,mu_e,A,-(B+B^T) in 2 bf16 terms, pairs (hi,hi),(hi,lo),"
+                    "(lo,hi); dg by a telescoped sum"
                   : "boundary states by the forward's first pass; adjoint scan per row (4 "
                     "packed accumulators per lane, xor butterfly 1,2); chunk states by the "
                     "step schedule; chunk products Y,X,A,B,DQ,DK in f32 fma, fixed order; dg "
