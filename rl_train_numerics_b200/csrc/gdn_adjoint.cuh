@@ -73,15 +73,19 @@ __device__ __forceinline__ void put3(__nv_bfloat16* p, size_t nelem, int off, fl
 // ----------------------------------------------------------------------------
 // k_adj_prep
 // ----------------------------------------------------------------------------
+// The queries go where the prep's fp32 T was, once T is split; the prep's head
+// takes the Tb terms.
 template <int D>
 struct AdjPrepSmem {
-  PrepSmem<D, __nv_bfloat16> prep;  // head reused for the Tb terms once the prep is done
-  PrepAT AT;
-  __nv_bfloat16 Q[1][kChunk * D];
+  PrepSmem<D, __nv_bfloat16> prep;
+  union {
+    PrepAT AT;
+    __nv_bfloat16 Q[1][kChunk * D];
+  };
 };
 
 template <int D>
-__global__ void __launch_bounds__(kBndThreads, 2)
+__global__ void __launch_bounds__(kBndThreads, 3)
     k_adj_prep(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                const __nv_bfloat16* __restrict__ d_o, const float* __restrict__ beta,
                const float* __restrict__ g, const int32_t* __restrict__ cu, int H, float scale,
@@ -101,9 +105,11 @@ __global__ void __launch_bounds__(kBndThreads, 2)
   const size_t tok = (size_t)it.t0 * H + h;
   AdjPack<D>& pk = *reinterpret_cast<AdjPack<D>*>(apacks + ((size_t)c * H + h) * adj_pack_bytes<D>());
 
-  PlaneRows<D, bf16, kBndThreads> dorows;  // do rows in flight during the prep
-  dorows.load(d_o + tok * D, (size_t)H * D, len);
-  stage_planes<D, bf16>(sm.Q, q + tok * D, (size_t)H * D, kBndThreads, len);
+  {
+    PlaneRows<D, bf16, kBndThreads> dorows;  // do rows: global -> the pack's plane
+    dorows.load(d_o + tok * D, (size_t)H * D, len);
+    dorows.store(pk.DO);
+  }
   prep_stage<D, bf16>(sm.prep, k + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H, len);
   bnd_prep<D, bf16>(sm.prep, sm.AT);
 
@@ -114,7 +120,6 @@ __global__ void __launch_bounds__(kBndThreads, 2)
   if (tid < 4) pk.gamma[tid] = sm.prep.head.gamma[tid];
   for (int e = tid; e < PD / 8; e += kBndThreads)
     reinterpret_cast<uint4*>(pk.K[0])[e] = reinterpret_cast<const uint4*>(sm.prep.K[0])[e];
-  dorows.store(pk.DO);
   // T (rows m, columns t) and Tb = T diag(beta e^G) (rows t, columns m).
   bf16* tb3 = reinterpret_cast<bf16*>(&sm.prep.head);
   for (int e = tid; e < PL / 2; e += kBndThreads) {
@@ -126,6 +131,10 @@ __global__ void __launch_bounds__(kBndThreads, 2)
     put3(pk.Tb[0], PL, off, b0, b1);
     put3(tb3, PL, off, b0, b1);
   }
+  __syncthreads();  // T is read: its space takes the queries
+  stage_planes<D, bf16>(sm.Q, q + tok * D, (size_t)H * D, kBndThreads, len);
+  cp_async_commit();
+  cp_async_wait<0>();
   __syncthreads();
 
   // Pm on warp w's rows 16w .. 16w + 15 (n8 tiles up to the diagonal block).
