@@ -49,7 +49,8 @@ PAGES_H100_LAYOUTS = {"prefill": (0.844, 3.639, 1.412), "trainer_fwd_bwd": (5.17
 TRAFFIC_SOURCES = {
     "forward": ("gdn_kernels.cu", "gdn_boundary.cuh", "gdn_common.cuh", "gdn_fill.cuh",
                 "gdn_mma.cuh", "gdn_umma.cuh", "gdn_layout.h"),
-    "backward": ("gdn_backward.cu", "gdn_boundary.cuh", "gdn_common.cuh", "gdn_fill.cuh",
+    "backward": ("gdn_backward.cu", "gdn_adjoint.cuh", "gdn_boundary.cuh", "gdn_common.cuh",
+                 "gdn_fill.cuh",
                  "gdn_mma.cuh", "gdn_umma.cuh", "gdn_layout.h"),
     "pik": ("gdn_pik.cu", "gdn_mma.cuh", "gdn_umma.cuh"),
     "native": ("gdn_native.cuh", "gdn_boundary.cuh", "gdn_common.cuh", "gdn_fill.cuh",
