@@ -541,15 +541,17 @@ def run_layouts_part(gdn, W, dev, rank, world, args, flush, cpr_decode_ms, peaks
 
 def bwd_gemm_flops(lengths, H, D):
     """Algorithmic FLOPs of the backward's chunk products: per chunk of length L,
-    Y (lower triangle incl. diagonal) and X (strict) over d, the three L x d x d
-    products (DO S_a, W S_a, U mu_e), A K and A^T Q (triangles incl. diagonal)
-    and (B + B^T) K (off-diagonal), two FLOPs per multiply-add."""
+    Y (lower triangle incl. diagonal) and X and K K^T (strict) over d, the three
+    L x d x d products (DO S_a, W S_a, U mu_e), A K and A^T Q (triangles incl.
+    diagonal) and (B + B^T) K (off-diagonal), the dbeta / dg dots (w . v,
+    k . (W S_a), k . (U mu_e), q . dq per token, <mu_e, S_a>), two FLOPs per
+    multiply-add."""
     mac = 0
     for Ln in lengths:
         for c0 in range(0, Ln, C):
             L = min(C, Ln - c0)
             tri, stri = L * (L + 1) // 2, L * (L - 1) // 2
-            mac += D * (3 * tri + stri + 2 * stri) + 3 * L * D * D
+            mac += D * (3 * tri + 2 * stri + 2 * stri) + 3 * L * D * D + 4 * L * D + D * D
     return 2 * mac * H
 
 
@@ -599,7 +601,7 @@ def run_train_part(gdn, W, dev, rank, world, args, flush, peaks):
     fwd, bwd = el(0, 4), el(5, 9)
     kern = {"fwd_chunk_table": el(0, 1), "fwd_boundary_prep": el(1, 2),
             "fwd_boundary_walk": el(2, 3), "fwd_intra_chunk_fill": el(3, 4),
-            "bwd_adjoint_scan": el(6, 7), "bwd_chunk_rows": el(7, 8),
+            "bwd_adjoint_scan": el(6, 7), "bwd_chunk_u": el(7, 8),
             "bwd_chunk_products": el(8, 9)}
     ms = max_over_ranks(fwd + bwd, world)
     fwd_max = max_over_ranks(fwd, world)

@@ -366,8 +366,10 @@ size_t gdn_cpr_backward_workspace_bytes(int n_seqs, int64_t total_tokens, int H,
  * o_t = scale S_t q_t, alpha_t = exp(g_t).
  * Schedule: the forward's first pass runs again (boundary states); an
  * adjoint recurrence runs over each sequence, last token first (row-parallel,
- * like the state); each chunk's states are recomputed from its boundary state
- * with the forward's per-token step; each chunk's dq and dk come from
+ * like the state); each chunk's update vectors u are recomputed from its
+ * boundary state (bf16 inputs: in product form, U = T diag(beta)(V -
+ * diag(e^G) K S_a^T); fp32 inputs: with the forward's per-token step); each
+ * chunk's dq and dk, and with bf16 inputs its dbeta and dg, come from
  * products of C x C and C x d matrices.  Every reduction has a fixed order,
  * so repeated calls return identical bits.
  *

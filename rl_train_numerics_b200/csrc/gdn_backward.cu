@@ -39,17 +39,32 @@
 // (the A^T Q term collects both scale q_t (do_t . u_t) and the do part of
 // mu_t^T u_t; B^T collects the w part of mu_t^T u_t).
 //
+// The scalar gradients in product form (bf16 inputs): with
+// A'_ts = e^{G_t - G_s} k_t . k_s and X = W U^T as above,
+//   dbeta_t = w_t . v_t - e^{G_t} k_t . (W S_a)_t - sum_{s<t} A'_ts X_ts
+// (w_t . (v_t - alpha_t S_{t-1} k_t) with S_{t-1} unrolled from S_a), and the
+// telescoped dg starts from Z at the chunk's end,
+//   Z_end = <mu_e, S_{L-1}> = e^{G_{L-1}} <mu_e, S_a> + sum_t e^{G_{L-1} - G_t} k_t . (U mu_e)_t,
+// with do_t . o_t = q_t . dq_t (both are scale do_t^T S_t q_t).
+//
 // Kernels, in launch order:
 //   forward pass 1   chunk table and boundary states S_a, exactly as the
 //                    forward computes them
-//   k_bwd_scan       one block per (sequence, head, 32 rows): the adjoint
-//                    recurrence over the whole sequence, last token first;
-//                    writes w, dv, the adjoint at every chunk end and dh0
-//   k_bwd_rows       one block per (chunk, head): recomputes the chunk's
-//                    states from S_a with the forward fill's per-token step
-//                    (the states the outputs came from); writes u, dbeta, dg
-//   k_bwd_gemm       one block per (chunk, head): DQ and DK from the
-//                    products above, in fp32 fused multiply-adds
+//   adjoint          bf16 inputs: k_adj_prep, k_adj_walk, k_adj_w
+//                    (gdn_adjoint.cuh), the adjoint in chunk form; fp32
+//                    inputs: k_bwd_scan, one block per (sequence, head, 32
+//                    rows), the adjoint recurrence over the whole sequence,
+//                    last token first.  Both write w, dv, the adjoint at
+//                    every chunk end and dh0
+//   k_bwd_u          bf16 inputs, one block per (chunk, head): u in product
+//                    form from S_a and the prep's T
+//   k_bwd_rows       fp32 inputs, one block per (chunk, head): recomputes the
+//                    chunk's states from S_a with the forward fill's per-token
+//                    step (the states the outputs came from); writes u,
+//                    dbeta, dg
+//   k_bwd_gemm_tc    bf16 inputs, one block per (chunk, head): DQ, DK, dbeta
+//                    and dg from the products above on mma.sync
+//   k_bwd_gemm       fp32 inputs: DQ and DK in fp32 fused multiply-adds
 // Every sum has a fixed order, so repeated runs give identical bits.
 #include "gdn_adjoint.cuh"
 #include "gdn_boundary.cuh"
@@ -631,10 +646,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // Chunk products on the tensor cores (bf16 inputs)
 // ----------------------------------------------------------------------------
 // The same DQ and DK as k_bwd_gemm, as mma.sync m16n8k16 contractions with
-// fp32 accumulation.  do, q and k are exact in bf16; every fp32 operand (w, u,
-// S_a, mu_e, A, -(B + B^T)) is split exactly into two bf16 terms and the term
-// pairs (hi, hi), (hi, lo), (lo, hi) accumulate in that order (the split
-// scheme of the forward's boundary pass).  One block of 8 warps per (chunk,
+// fp32 accumulation, plus dbeta and dg.  do, q and k are exact in bf16; every
+// fp32 operand is split exactly into bf16 terms and the term pairs of order
+// below the finer split accumulate in ascending order.  One block of 8 warps per (chunk,
 // head); warp w owns tokens 16 (w % 4) .. + 15 and, for the C x C products,
 // columns 32 (w / 4) .. + 31, for the C x D products (D / 2) (w / 4) .. + D / 2 - 1.
 //   1. Y = DO U^T, X = W U^T -> A_ts = [s <= t] e^{G_t - G_s} Y_ts and
@@ -645,22 +659,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //   3. DQ = scale (diag(e^G) Pq + A K);
 //      DK = diag(-beta e^G) Pw + diag(e^{G_{L-1} - G}) Pu + scale (A^T Q)
 //           + Bn K  (A^T read through transposed ldmatrix).
+//   4. dbeta and dg from per-token sums gathered on the way: w . v (while W
+//      is split), sum_{s<t} A'_ts X_ts (step 1, with K K^T), k . Pw and
+//      k . Pu (before the row factors), q . dq, and <mu_e, S_a> (the slabs).
+// u and A carry three bf16 terms (their products feed dq, whose q . dq sums
+// build dg), the other fp32 operands two.
 // Every sum has a fixed order, so repeated runs give identical bits.
 template <int D>
 struct GemmTcSmem {
   __nv_bfloat16 DO[1][kChunk * D];      // [t][i]
   __nv_bfloat16 W[2][kChunk * D];       // [t][i], two terms
-  __nv_bfloat16 U[2][kChunk * D];       // [s][i]
+  __nv_bfloat16 U[3][kChunk * D];       // [s][i], three terms
   __nv_bfloat16 Q[1][kChunk * D];       // [t][j]
   __nv_bfloat16 K[1][kChunk * D];       // [s][j]
-  __nv_bfloat16 A[2][kChunk * kChunk];  // [t][s]
+  __nv_bfloat16 A[3][kChunk * kChunk];  // [t][s], three terms
   __nv_bfloat16 Bn[2][kChunk * kChunk]; // [t][s], -(B + B^T)
   __nv_bfloat16 Sp[2][kSlab * D];       // the current slab's terms, [i][j] (16-row core layout)
   __nv_bfloat16 Mp[2][kSlab * D];
   double G[kChunk];
   float graw[kChunk];
   float bet[kChunk];
+  // The per-token sums of dbeta and dg: w . v by column quarter; then by
+  // column half (warp nh) [0] sum_{s<t} A'_ts X_ts, [1] k_t . (W S_a)_t,
+  // [2] k_t . (U mu_e)_t, [3] q_t . dq_t; and <mu_e, S_a> by warp.
+  float wv[kGemmThreads];
+  float rs[4][2][kChunk];
+  float zp[kGemmThreads / 32];
 };
+
+// Sum over the four lanes of a quad (a fixed butterfly: every lane gets the
+// same bits).
+__device__ __forceinline__ float quad_total(float x) {
+  x = __fadd_rn(x, __shfl_xor_sync(kFull, x, 1));
+  return __fadd_rn(x, __shfl_xor_sync(kFull, x, 2));
+}
 
 // B fragments (x4.trans, two n8 tiles) of B[k][n] = M[k][n] in a 16-row plane.
 __device__ __forceinline__ const __nv_bfloat16* bfrag_kn16_addr(const __nv_bfloat16* base, int n0) {
@@ -676,17 +708,38 @@ __device__ __forceinline__ void split8(const float4& a, const float4& b, uint4& 
   split2(b.z, b.w, hi.w, lo.w);
 }
 
-// Two-term planes of two C x D fp32 blocks (rows at stride ld; rows past len
-// zero).  Work item e is row e % C, columns 8 (e / C) .. + 7, so that a warp
+// Eight consecutive fp32 values as three bf16 term pieces.
+__device__ __forceinline__ void split8x3(const float4& a, const float4& b, uint4 (&o)[3]) {
+  const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t w[3][4];
+#pragma unroll
+  for (int q = 0; q < 4; q++) {
+    __nv_bfloat16 t0[3], t1[3];
+    split_bf16<3>(x[2 * q], t0);
+    split_bf16<3>(x[2 * q + 1], t1);
+#pragma unroll
+    for (int m = 0; m < 3; m++) w[m][q] = pack_bf16(t0[m], t1[m]);
+  }
+#pragma unroll
+  for (int m = 0; m < 3; m++) o[m] = make_uint4(w[m][0], w[m][1], w[m][2], w[m][3]);
+}
+
+// Term planes of two C x D fp32 blocks (rows at stride ld; rows past len
+// zero): two terms of the first, three of the second.  Work item e is row e % C, columns 8 (e / C) .. + 7, so that a warp
 // writes 32 consecutive 16-byte pieces of the core layout; every load is
-// issued before the first split.
+// issued before the first split.  With the first block W and bf16 rows V at
+// the same stride, the thread's part of w_t . v_t (its items in order) goes to
+// wv[(threadIdx.x / C) * C + t].
 template <int D>
-__device__ __forceinline__ void split_rows2x2(__nv_bfloat16 (*dst0)[kChunk * D], const float* src0,
+__device__ __forceinline__ void split_rows2x3(__nv_bfloat16 (*dst0)[kChunk * D], const float* src0,
                                               __nv_bfloat16 (*dst1)[kChunk * D], const float* src1,
-                                              size_t ld, int len) {
+                                              const __nv_bfloat16* vsrc, float* wv, size_t ld,
+                                              int len) {
   constexpr int IT = kChunk * D / 8 / kGemmThreads;
   static_assert(kChunk * D / 8 % kGemmThreads == 0, "whole pieces per thread");
+  static_assert(kGemmThreads % kChunk == 0, "a thread's items share one row");
   float4 x[2][IT][2];
+  uint4 vv[IT];
 #pragma unroll
   for (int j = 0; j < IT; j++) {
     const int e = threadIdx.x + j * kGemmThreads, t = e % kChunk, c = (e / kChunk) * 8;
@@ -696,27 +749,47 @@ __device__ __forceinline__ void split_rows2x2(__nv_bfloat16 (*dst0)[kChunk * D],
       x[0][j][h] = t < len ? ld4(src0 + (size_t)t * ld + c + 4 * h) : z;
       x[1][j][h] = t < len ? ld4(src1 + (size_t)t * ld + c + 4 * h) : z;
     }
+    vv[j] = t < len ? *reinterpret_cast<const uint4*>(vsrc + (size_t)t * ld + c)
+                    : make_uint4(0u, 0u, 0u, 0u);
   }
-#pragma unroll
-  for (int m = 0; m < 2; m++) {
-    __nv_bfloat16(*dst)[kChunk * D] = m == 0 ? dst0 : dst1;
+  {
+    float acc = 0.f;
 #pragma unroll
     for (int j = 0; j < IT; j++) {
-      const int e = threadIdx.x + j * kGemmThreads, t = e % kChunk, c = (e / kChunk) * 8;
-      uint4 hi, lo;
-      split8(x[m][j][0], x[m][j][1], hi, lo);
-      *reinterpret_cast<uint4*>(&dst[0][core_off<kChunk>(t, c)]) = hi;
-      *reinterpret_cast<uint4*>(&dst[1][core_off<kChunk>(t, c)]) = lo;
+      const uint32_t pv[4] = {vv[j].x, vv[j].y, vv[j].z, vv[j].w};
+      const float xw[8] = {x[0][j][0].x, x[0][j][0].y, x[0][j][0].z, x[0][j][0].w,
+                           x[0][j][1].x, x[0][j][1].y, x[0][j][1].z, x[0][j][1].w};
+#pragma unroll
+      for (int q = 0; q < 4; q++) {
+        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&pv[q]);
+        acc = __fmaf_rn(xw[2 * q], __low2float(b2), acc);
+        acc = __fmaf_rn(xw[2 * q + 1], __high2float(b2), acc);
+      }
     }
+    wv[threadIdx.x] = acc;  // = (threadIdx.x / C) * C + t
+  }
+#pragma unroll
+  for (int j = 0; j < IT; j++) {
+    const int e = threadIdx.x + j * kGemmThreads, t = e % kChunk, c = (e / kChunk) * 8;
+    const int off = core_off<kChunk>(t, c);
+    uint4 hi, lo, u3[3];
+    split8(x[0][j][0], x[0][j][1], hi, lo);
+    *reinterpret_cast<uint4*>(&dst0[0][off]) = hi;
+    *reinterpret_cast<uint4*>(&dst0[1][off]) = lo;
+    split8x3(x[1][j][0], x[1][j][1], u3);
+#pragma unroll
+    for (int m = 0; m < 3; m++) *reinterpret_cast<uint4*>(&dst1[m][off]) = u3[m];
   }
 }
 
-// One bf16 term pair of a 2-term split into the 64-row planes P at (r, c).
+// The NT-term bf16 split of x into the 64-row planes P at (r, c).
+template <int NT>
 __device__ __forceinline__ void put_terms(__nv_bfloat16 (*P)[kChunk * kChunk], int r, int c,
                                           float x) {
-  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-  P[0][core_off<kChunk>(r, c)] = hi;
-  P[1][core_off<kChunk>(r, c)] = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
+  __nv_bfloat16 t[NT];
+  split_bf16<NT>(x, t);
+#pragma unroll
+  for (int m = 0; m < NT; m++) P[m][core_off<kChunk>(r, c)] = t[m];
 }
 
 template <int D>
@@ -728,7 +801,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                   const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
                   const float* __restrict__ bstate, const float* __restrict__ mu_end,
                   const float* __restrict__ wbuf, const float* __restrict__ ubuf,
-                  float* __restrict__ d_q, float* __restrict__ d_k) {
+                  const __nv_bfloat16* __restrict__ v, float* __restrict__ d_q,
+                  float* __restrict__ d_k, float* __restrict__ d_beta, float* __restrict__ d_g) {
   using bf16 = __nv_bfloat16;
   constexpr int NS = D / kSlab;
   constexpr int NT8 = D / 16;  // n8 tiles of a warp's C x D columns (D / 2 of them)
@@ -767,7 +841,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   stage_planes<D, bf16>(sm.Q, q + tb * D, (size_t)H * D, kGemmThreads, len);
   stage_planes<D, bf16>(sm.K, k + tb * D, (size_t)H * D, kGemmThreads, len);
   cp_async_commit();
-  split_rows2x2<D>(sm.W, wbuf + tb * D, sm.U, ubuf + tb * D, (size_t)H * D, len);
+  split_rows2x3<D>(sm.W, wbuf + tb * D, sm.U, ubuf + tb * D, v + tb * D, sm.wv, (size_t)H * D,
+                   len);
   if (tid < kChunk) {
     sm.graw[tid] = tid < len ? g[tb + (size_t)tid * H] : 0.f;
     sm.bet[tid] = tid < len ? beta[tb + (size_t)tid * H] : 0.f;
@@ -777,26 +852,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cp_async_wait<0>();
   __syncthreads();
 
-  // 1. Y and X on this warp's 16 x 32 tile, then A and Bn.
+  // 1. Y, X and K K^T on this warp's 16 x 32 tile, then A, Bn and the
+  //    dbeta term sum_{s<t} A'_ts X_ts (A'_ts = e^{G_t - G_s} k_t . k_s).
   {
-    float y[4][4], x[4][4];
+    float y[4][4], x[4][4], kk[4][4];
 #pragma unroll
     for (int n = 0; n < 4; n++)
 #pragma unroll
-      for (int e = 0; e < 4; e++) y[n][e] = x[n][e] = 0.f;
+      for (int e = 0; e < 4; e++) y[n][e] = x[n][e] = kk[n][e] = 0.f;
 #pragma unroll 2
     for (int ks = 0; ks < D / 16; ks++) {
-      uint32_t ad[1][4], aw[2][4];
+      uint32_t ad[1][4], aw[2][4], ak[4];
       ldsm_x4(ad[0], afrag_addr(sm.DO[0], 16 * mt, 16 * ks));
+      ldsm_x4(ak, afrag_addr(sm.K[0], 16 * mt, 16 * ks));
 #pragma unroll
       for (int qq = 0; qq < 2; qq++) ldsm_x4(aw[qq], afrag_addr(sm.W[qq], 16 * mt, 16 * ks));
 #pragma unroll
       for (int np = 0; np < 2; np++) {
-        uint32_t bu[2][4];
+        uint32_t bu[3][4], bk[4];
 #pragma unroll
-        for (int qq = 0; qq < 2; qq++)
+        for (int qq = 0; qq < 3; qq++)
           ldsm_x4(bu[qq], bfrag_nk_addr(sm.U[qq], 32 * nh + 16 * np, 16 * ks));
-        using PY = SplitPairs<1, 2>;
+        ldsm_x4(bk, bfrag_nk_addr(sm.K[0], 32 * nh + 16 * np, 16 * ks));
+        mma16816(kk[2 * np], ak, bk[0], bk[1]);
+        mma16816(kk[2 * np + 1], ak, bk[2], bk[3]);
+        using PY = SplitPairs<1, 3>;
 #pragma unroll
         for (int p = 0; p < PY::kCount; p++) {
           mma16816(y[2 * np], ad[PY::a(p)], bu[PY::b(p)][0], bu[PY::b(p)][1]);
@@ -810,6 +890,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     }
+    float ax[2] = {0.f, 0.f};
 #pragma unroll
     for (int n = 0; n < 4; n++)
 #pragma unroll
@@ -819,14 +900,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (s <= t) {
           const float dec = expf(__double2float_rn(sm.G[t] - sm.G[s]));
           av = __fmul_rn(dec, y[n][e]);
-          if (s < t) bv = -__fmul_rn(__fmul_rn(sm.bet[t], dec), x[n][e]);
+          if (s < t) {
+            bv = -__fmul_rn(__fmul_rn(sm.bet[t], dec), x[n][e]);
+            ax[e >> 1] = __fmaf_rn(__fmul_rn(dec, kk[n][e]), x[n][e], ax[e >> 1]);
+          }
         }
-        put_terms(sm.A, t, s, av);
+        put_terms<3>(sm.A, t, s, av);
         if (s <= t) {
-          put_terms(sm.Bn, t, s, bv);
-          if (s < t) put_terms(sm.Bn, s, t, bv);
+          put_terms<2>(sm.Bn, t, s, bv);
+          if (s < t) put_terms<2>(sm.Bn, s, t, bv);
         }
       }
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+      const float tot = quad_total(ax[hf]);
+      if (tq == 0) sm.rs[0][nh][16 * mt + gq + 8 * hf] = tot;
+    }
   }
 
   // 2. The slab products.
@@ -836,9 +925,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
     for (int e = 0; e < 4; e++) aq[n][e] = aw[n][e] = au[n][e] = 0.f;
   static_assert(SLI <= kGemmThreads, "one slab item per thread at most");
+  float zms = 0.f;  // this thread's part of <mu_e, S_a>
   for (int j = 0; j < NS; j++) {
     __syncthreads();  // the previous slab's terms are no longer read
     if (slab_item) {
+#pragma unroll
+      for (int hh = 0; hh < 2; hh++) {
+        zms = __fmaf_rn(sx[hh].x, mx[hh].x, zms);
+        zms = __fmaf_rn(sx[hh].y, mx[hh].y, zms);
+        zms = __fmaf_rn(sx[hh].z, mx[hh].z, zms);
+        zms = __fmaf_rn(sx[hh].w, mx[hh].w, zms);
+      }
       uint4 hi, lo;
       split8(sx[0], sx[1], hi, lo);
       *reinterpret_cast<uint4*>(&sm.Sp[0][core_off<kSlab>(sr, sc)]) = hi;
@@ -885,63 +982,306 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
 
-  // 3. Row factors, then the C x C products.
+  zms = warp_sum(zms);
+  if (lane == 0) sm.zp[w] = zms;
+
+  // 3. Row factors (and the key dots k_t . (W S_a)_t, k_t . (U mu_e)_t), then
+  //    the C x C products.
   const double GL = sm.G[kChunk - 1];  // = G_{L-1}: the padding's g is 0
 #pragma unroll
   for (int hf = 0; hf < 2; hf++) {
     const int t = 16 * mt + gq + 8 * hf;
     const float eg = expf(__double2float_rn(sm.G[t]));
     const float fw = -__fmul_rn(sm.bet[t], eg), fu = expf(__double2float_rn(GL - sm.G[t]));
+    float kw = 0.f, ku = 0.f;
 #pragma unroll
-    for (int n = 0; n < NT8; n++)
+    for (int n = 0; n < NT8; n++) {
+      const int col = (D / 2) * nh + 8 * n + 2 * tq;
+      const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162*>(&sm.K[0][core_off<kChunk>(t, col)]);
+      const float kc[2] = {__low2float(k2), __high2float(k2)};
 #pragma unroll
       for (int e = 2 * hf; e < 2 * hf + 2; e++) {
+        kw = __fmaf_rn(kc[e & 1], aw[n][e], kw);
+        ku = __fmaf_rn(kc[e & 1], au[n][e], ku);
         aq[n][e] = __fmul_rn(eg, aq[n][e]);
         aw[n][e] = __fmaf_rn(fu, au[n][e], __fmul_rn(fw, aw[n][e]));
         au[n][e] = 0.f;
       }
+    }
+    kw = quad_total(kw);
+    ku = quad_total(ku);
+    if (tq == 0) {
+      sm.rs[1][nh][t] = kw;
+      sm.rs[2][nh][t] = ku;
+    }
   }
 #pragma unroll
   for (int ks = 0; ks < kChunk / 16; ks++) {
-    uint32_t fa[2][4], fat[2][4], fb[2][4];
+    uint32_t fa[3][4], fat[3][4], fb[2][4];
 #pragma unroll
-    for (int qq = 0; qq < 2; qq++) {
+    for (int qq = 0; qq < 3; qq++) {
       ldsm_x4(fa[qq], afrag_addr(sm.A[qq], 16 * mt, 16 * ks));
       ldsm_x4_t(fat[qq], afrag_t_addr(sm.A[qq], 16 * mt, 16 * ks));
-      ldsm_x4(fb[qq], afrag_addr(sm.Bn[qq], 16 * mt, 16 * ks));
     }
+#pragma unroll
+    for (int qq = 0; qq < 2; qq++) ldsm_x4(fb[qq], afrag_addr(sm.Bn[qq], 16 * mt, 16 * ks));
 #pragma unroll
     for (int np = 0; np < NT8 / 2; np++) {
       const int n0 = (D / 2) * nh + 16 * np;
       uint32_t bk[1][4], bq[1][4];
       ldsm_x4_t(bk[0], bfrag_kn_addr(sm.K[0], 16 * ks, n0));
       ldsm_x4_t(bq[0], bfrag_kn_addr(sm.Q[0], 16 * ks, n0));
-      using P3 = SplitPairs<2, 1>;
+      using P3 = SplitPairs<3, 1>;
 #pragma unroll
       for (int p = 0; p < P3::kCount; p++) {
         mma16816(aq[2 * np], fa[P3::a(p)], bk[0][0], bk[0][1]);
         mma16816(aq[2 * np + 1], fa[P3::a(p)], bk[0][2], bk[0][3]);
         mma16816(au[2 * np], fat[P3::a(p)], bq[0][0], bq[0][1]);
         mma16816(au[2 * np + 1], fat[P3::a(p)], bq[0][2], bq[0][3]);
-        mma16816(aw[2 * np], fb[P3::a(p)], bk[0][0], bk[0][1]);
-        mma16816(aw[2 * np + 1], fb[P3::a(p)], bk[0][2], bk[0][3]);
+      }
+      using P2B = SplitPairs<2, 1>;
+#pragma unroll
+      for (int p = 0; p < P2B::kCount; p++) {
+        mma16816(aw[2 * np], fb[P2B::a(p)], bk[0][0], bk[0][1]);
+        mma16816(aw[2 * np + 1], fb[P2B::a(p)], bk[0][2], bk[0][3]);
       }
     }
   }
   // DK = (row terms + Bn K) + scale (A^T Q); DQ = scale (diag(e^G) Pq + A K).
+  float qdq[2] = {0.f, 0.f};
+#pragma unroll
+  for (int n = 0; n < NT8; n++)
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+      const int t = 16 * mt + gq + 8 * hf;
+      const int col = (D / 2) * nh + 8 * n + 2 * tq;
+      const float dq0 = __fmul_rn(scale, aq[n][2 * hf]), dq1 = __fmul_rn(scale, aq[n][2 * hf + 1]);
+      const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162*>(&sm.Q[0][core_off<kChunk>(t, col)]);
+      qdq[hf] = __fmaf_rn(__high2float(q2), dq1, __fmaf_rn(__low2float(q2), dq0, qdq[hf]));
+      if (t >= len) continue;
+      const size_t o = (tb + (size_t)t * H) * D + col;
+      *reinterpret_cast<float2*>(d_q + o) = f2(dq0, dq1);
+      *reinterpret_cast<float2*>(d_k + o) =
+          f2(__fmaf_rn(scale, au[n][2 * hf], aw[n][2 * hf]),
+             __fmaf_rn(scale, au[n][2 * hf + 1], aw[n][2 * hf + 1]));
+    }
+#pragma unroll
+  for (int hf = 0; hf < 2; hf++) {
+    const float tot = quad_total(qdq[hf]);
+    if (tq == 0) sm.rs[3][nh][16 * mt + gq + 8 * hf] = tot;
+  }
+  __syncthreads();
+
+  // 4. dbeta and dg, by warp 0 (lane l: tokens 2l, 2l + 1).  With R_t =
+  //    v_t - alpha_t S_{t-1} k_t the residual the forward step forms,
+  //      dbeta_t = w_t . R_t = w_t . v_t - e^{G_t} k_t . (W S_a)_t - sum_{s<t} A'_ts X_ts,
+  //    and dg_t = Z_{t-1} telescoped from the chunk's end, Z_end = <mu_e, S_e>
+  //    = e^{G_{L-1}} <mu_e, S_a> + sum_t e^{G_{L-1} - G_t} k_t . (U mu_e)_t, with
+  //    do_t . o_t = q_t . dq_t (both are scale do_t^T S_t q_t).
+  if (w == 0) {
+    float ms = 0.f;
+#pragma unroll
+    for (int q8 = 0; q8 < kGemmThreads / 32; q8++) ms = __fadd_rn(ms, sm.zp[q8]);
+    float term[2], kum[2];
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+      const int t = 2 * lane + e;
+      float wvt = 0.f;
+#pragma unroll
+      for (int p = 0; p < kGemmThreads / kChunk; p++) wvt = __fadd_rn(wvt, sm.wv[p * kChunk + t]);
+      const float sa = __fadd_rn(sm.rs[0][0][t], sm.rs[0][1][t]);
+      const float kws = __fadd_rn(sm.rs[1][0][t], sm.rs[1][1][t]);
+      const float kus = __fadd_rn(sm.rs[2][0][t], sm.rs[2][1][t]);
+      const float qd = __fadd_rn(sm.rs[3][0][t], sm.rs[3][1][t]);
+      const float eg = expf(__double2float_rn(sm.G[t]));
+      const float fu = expf(__double2float_rn(GL - sm.G[t]));
+      if (t < len) d_beta[tb + (size_t)t * H] = __fsub_rn(__fmaf_rn(-eg, kws, wvt), sa);
+      term[e] = t < len ? __fmaf_rn(-sm.bet[t], wvt, qd) : 0.f;
+      kum[e] = __fmul_rn(fu, kus);
+    }
+    const float zend = __fmaf_rn(expf(__double2float_rn(GL)), ms, warp_sum(__fadd_rn(kum[0], kum[1])));
+    // Suffix sums over the pairs: x_l = sum_{m >= l} (term_2m + term_2m+1).
+    float x = __fadd_rn(term[0], term[1]);
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_down_sync(kFull, x, off);
+      if (lane + off < 32) x = __fadd_rn(x, y);
+    }
+    const float xn = __shfl_down_sync(kFull, x, 1);
+    const float after = lane < 31 ? xn : 0.f;  // sum over tokens >= 2l + 2
+    if (2 * lane < len) d_g[tb + (size_t)(2 * lane) * H] = __fadd_rn(zend, x);
+    if (2 * lane + 1 < len)
+      d_g[tb + (size_t)(2 * lane + 1) * H] = __fadd_rn(zend, __fadd_rn(term[1], after));
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Chunk u in product form (bf16 inputs)
+// ----------------------------------------------------------------------------
+// u_t = beta_t (v_t - alpha_t S_{t-1} k_t) over a chunk that starts from S_a
+// is, with T = (I + A)^{-1} of the forward's boundary prep (the adjoint pack
+// keeps its three terms),
+//   U = T diag(beta) (V - diag(e^G) K S_a^T)
+// (the U of the forward's boundary map).  One block of 256 threads per
+// (chunk, head), warp w on tokens 16 (w & 3) .. + 15 and state rows
+// (D / 2)(w >> 2) ..: Ya = K S_a^T with S_a split into two bf16 terms (keys
+// exact), Z = diag(beta)(V - diag(e^G) Ya) split into three, U = T Z with all
+// term pairs down to the third order.
+constexpr int kUThreads = 256;
+
+template <int D>
+struct BwdUSmem {
+  union {
+    __nv_bfloat16 S[2][D * D];            // S_a terms, [i][j] in 64-row tiles
+    __nv_bfloat16 Z[kAdjNT][kChunk * D];  // [m][i]
+  } a;
+  union {
+    __nv_bfloat16 K[1][kChunk * D];            // [t][j]
+    __nv_bfloat16 T[kAdjNT][kChunk * kChunk];  // [t][m], m <= t
+  } b;
+  __nv_bfloat16 V[1][kChunk * D];  // [t][i]
+  double G[kChunk];
+  float graw[kChunk];
+  float bet[kChunk];
+};
+
+template <int D>
+__global__ void __launch_bounds__(kUThreads, 2)
+    k_bwd_u(const __nv_bfloat16* __restrict__ v, const float* __restrict__ beta,
+            const float* __restrict__ g, const int32_t* __restrict__ cu, int H,
+            const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+            const int32_t* __restrict__ chunk_seq, const float* __restrict__ bstate,
+            const char* __restrict__ apacks, float* __restrict__ ubuf) {
+  using bf16 = __nv_bfloat16;
+  constexpr int C = kChunk, PL = C * C, PD = C * D, NT8 = D / 16, ST = 64 * D;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  BwdUSmem<D>& sm = *reinterpret_cast<BwdUSmem<D>*>(smem_raw);
+  if (hdr[kHdrValid] != 1) return;
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (c >= hdr[kHdrChunks]) return;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+  const int mt = w & 3, nh = w >> 2;
+  const FillItem it = fill_item(c * H + h, H, cu, chunk_off, chunk_seq);
+  const int len = it.len;
+  const size_t tb = (size_t)it.t0 * H + h;
+  const AdjPack<D>& pk =
+      *reinterpret_cast<const AdjPack<D>*>(apacks + ((size_t)c * H + h) * adj_pack_bytes<D>());
+  const float* Sa = bstate + ((size_t)c * H + h) * (size_t)D * D;
+
+  for (int e = tid; e < PD / 8; e += kUThreads)
+    cp_async16(reinterpret_cast<uint4*>(sm.b.K[0]) + e, reinterpret_cast<const uint4*>(pk.K[0]) + e);
+  stage_planes<D, bf16>(sm.V, v + tb * D, (size_t)H * D, kUThreads, len);
+  cp_async_commit();
+  if (tid < C) {
+    sm.graw[tid] = tid < len ? g[tb + (size_t)tid * H] : 0.f;
+    sm.bet[tid] = tid < len ? beta[tb + (size_t)tid * H] : 0.f;
+  }
+  // S_a (permuted boundary layout) as two bf16 terms: item e is row e % D,
+  // columns 8 (e / D) .. + 7, so that a warp stores 32 consecutive pieces.
+  constexpr int SI = D * D / 8 / kUThreads, SB = SI > 4 ? 4 : SI;
+  static_assert(D * D / 8 % kUThreads == 0 && SI % SB == 0, "whole items per thread");
+#pragma unroll
+  for (int j0 = 0; j0 < SI; j0 += SB) {
+    float4 x[SB][2];
+#pragma unroll
+    for (int j = 0; j < SB; j++) {
+      const int e = tid + (j0 + j) * kUThreads, i = e % D, cc = (e / D) * 8;
+      x[j][0] = ld4(Sa + (size_t)i * D + bst_col(i, cc));
+      x[j][1] = ld4(Sa + (size_t)i * D + bst_col(i, cc + 4));
+    }
+#pragma unroll
+    for (int j = 0; j < SB; j++) {
+      const int e = tid + (j0 + j) * kUThreads, i = e % D, cc = (e / D) * 8;
+      uint4 hi, lo;
+      split8(x[j][0], x[j][1], hi, lo);
+      const int off = (i / 64) * ST + core_off<64>(i % 64, cc);
+      *reinterpret_cast<uint4*>(&sm.a.S[0][off]) = hi;
+      *reinterpret_cast<uint4*>(&sm.a.S[1][off]) = lo;
+    }
+  }
+  __syncthreads();
+  if (w == 0) chunk_cumsum_g(sm.graw, sm.G);
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // Ya = K S_a^T on this warp's tile.
+  float acc[NT8][4];
+#pragma unroll
+  for (int n = 0; n < NT8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) acc[n][e] = 0.f;
+#pragma unroll 2
+  for (int ks = 0; ks < D / 16; ks++) {
+    uint32_t a[4];
+    ldsm_x4(a, afrag_addr(sm.b.K[0], 16 * mt, 16 * ks));
+#pragma unroll
+    for (int np = 0; np < NT8 / 2; np++) {
+      const int n0 = (D / 2) * nh + 16 * np;
+      uint32_t b[2][4];
+#pragma unroll
+      for (int qq = 0; qq < 2; qq++)
+        ldsm_x4(b[qq], bfrag_nk_addr(sm.a.S[qq] + (n0 / 64) * ST, n0 % 64, 16 * ks));
+      using P12 = SplitPairs<1, 2>;
+#pragma unroll
+      for (int p = 0; p < P12::kCount; p++) {
+        mma16816(acc[2 * np], a, b[P12::b(p)][0], b[P12::b(p)][1]);
+        mma16816(acc[2 * np + 1], a, b[P12::b(p)][2], b[P12::b(p)][3]);
+      }
+    }
+  }
+  __syncthreads();  // K and the S_a terms are read: their space takes T and Z
+  for (int e = tid; e < kAdjNT * PL / 8; e += kUThreads)
+    cp_async16(reinterpret_cast<uint4*>(sm.b.T[0]) + e, reinterpret_cast<const uint4*>(pk.T[0]) + e);
+  cp_async_commit();
+#pragma unroll
+  for (int hf = 0; hf < 2; hf++) {
+    const int t = 16 * mt + gq + 8 * hf;
+    const float eg = expf(__double2float_rn(sm.G[t])), bt = sm.bet[t];
+#pragma unroll
+    for (int n = 0; n < NT8; n++) {
+      const int i = (D / 2) * nh + 8 * n + 2 * tq, off = core_off<C>(t, i);
+      const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&sm.V[0][off]);
+      const float z0 = __fmul_rn(bt, __fmaf_rn(-eg, acc[n][2 * hf], __low2float(v2)));
+      const float z1 = __fmul_rn(bt, __fmaf_rn(-eg, acc[n][2 * hf + 1], __high2float(v2)));
+      put3(sm.a.Z[0], PD, off, z0, z1);
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // U = T Z (T[t][m] vanishes for m > t).
+#pragma unroll
+  for (int n = 0; n < NT8; n++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) acc[n][e] = 0.f;
+  using P33 = SplitPairs<kAdjNT, kAdjNT>;
+#pragma unroll
+  for (int ks = 0; ks < 4; ks++) {
+    if (ks > mt) continue;
+    uint32_t a[kAdjNT][4];
+#pragma unroll
+    for (int qq = 0; qq < kAdjNT; qq++) ldsm_x4(a[qq], afrag_addr(sm.b.T[qq], 16 * mt, 16 * ks));
+#pragma unroll
+    for (int np = 0; np < NT8 / 2; np++) {
+      uint32_t b[kAdjNT][4];
+#pragma unroll
+      for (int qq = 0; qq < kAdjNT; qq++)
+        ldsm_x4_t(b[qq], bfrag_kn_addr(sm.a.Z[qq], 16 * ks, (D / 2) * nh + 16 * np));
+#pragma unroll
+      for (int p = 0; p < P33::kCount; p++) {
+        mma16816(acc[2 * np], a[P33::a(p)], b[P33::b(p)][0], b[P33::b(p)][1]);
+        mma16816(acc[2 * np + 1], a[P33::a(p)], b[P33::b(p)][2], b[P33::b(p)][3]);
+      }
+    }
+  }
 #pragma unroll
   for (int n = 0; n < NT8; n++)
 #pragma unroll
     for (int hf = 0; hf < 2; hf++) {
       const int t = 16 * mt + gq + 8 * hf;
       if (t >= len) continue;
-      const int col = (D / 2) * nh + 8 * n + 2 * tq;
-      const size_t o = (tb + (size_t)t * H) * D + col;
-      *reinterpret_cast<float2*>(d_q + o) =
-          f2(__fmul_rn(scale, aq[n][2 * hf]), __fmul_rn(scale, aq[n][2 * hf + 1]));
-      *reinterpret_cast<float2*>(d_k + o) =
-          f2(__fmaf_rn(scale, au[n][2 * hf], aw[n][2 * hf]),
-             __fmaf_rn(scale, au[n][2 * hf + 1], aw[n][2 * hf + 1]));
+      const size_t o = (tb + (size_t)t * H) * D + (D / 2) * nh + 8 * n + 2 * tq;
+      *reinterpret_cast<float2*>(ubuf + o) = f2(acc[n][2 * hf], acc[n][2 * hf + 1]);
     }
 }
 
@@ -1022,7 +1362,14 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
     GDN_BWD_TRY(cudaGetLastError());
   }
   GDN_BWD_TRY(mark(2));
-  {
+  if constexpr (sizeof(IN) == 2) {  // bf16 inputs: u in product form, dbeta and dg with dq, dk
+    auto kern = k_bwd_u<D>;
+    const size_t sm = sizeof(BwdUSmem<D>);
+    GDN_BWD_TRY(bwd_set_smem(kern, sm));
+    kern<<<gchunks, kUThreads, sm, st>>>(v, f.beta, f.g, f.cu_seqlens, f.H, hdr, chunk_off,
+                                         chunk_seq, bstate, ws + L.apack, ubuf);
+    GDN_BWD_TRY(cudaGetLastError());
+  } else {
     auto kern = k_bwd_rows<D, IN>;
     const size_t sm = sizeof(RowsSmem<D, IN>);
     GDN_BWD_TRY(bwd_set_smem(kern, sm));
@@ -1039,7 +1386,7 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
       GDN_BWD_TRY(bwd_set_smem(kern, sm));
       kern<<<gchunks, kGemmThreads, sm, st>>>(q, k, f.beta, f.g, d_o, f.cu_seqlens, f.H, f.scale,
                                               hdr, chunk_off, chunk_seq, bstate, mu_end, wbuf,
-                                              ubuf, a.d_q, a.d_k);
+                                              ubuf, v, a.d_q, a.d_k, a.d_beta, a.d_g);
     } else {  // fp32 inputs: fp32 fused multiply-adds (their tighter bound)
       auto kern = k_bwd_gemm<D, IN>;
       const size_t sm = sizeof(GemmSmem<D, IN>);

@@ -153,9 +153,11 @@ std::string descriptor(int kind, int in_dtype, int out_dtype, int dk, int dv, in
                   ? "boundary states by the forward's first pass; adjoint in chunk form "
                     "(prep: T, Pm, X; reverse walk over chunk ends; W = T^T R) by mma.sync "
                     "m16n8k16 bf16 with fp32 operands in 3 bf16 terms, all pairs of order < 3; "
-                    "chunk states by the step schedule; chunk products Y,X,DQ,DK by mma.sync "
-                    "with w,u,S_a,mu_e,A,-(B+B^T) in 2 bf16 terms, pairs (hi,hi),(hi,lo),"
-                    "(lo,hi); dg by a telescoped sum"
+                    "chunk u = T diag(beta)(V - diag(e^G) K S_a^T) by mma.sync (S_a 2 terms, "
+                    "T and Z 3); chunk products Y,X,DQ,DK by mma.sync with w,S_a,mu_e,"
+                    "-(B+B^T) in 2 bf16 terms and u,A in 3, all pairs of order < the finer "
+                    "split; dbeta = w.v - e^G k.(W S_a) - sum A'X, dg by a telescoped sum "
+                    "with do.o = q.dq"
                   : "boundary states by the forward's first pass; adjoint scan per row (4 "
                     "packed accumulators per lane, xor butterfly 1,2); chunk states by the "
                     "step schedule; chunk products Y,X,A,B,DQ,DK in f32 fma, fixed order; dg "

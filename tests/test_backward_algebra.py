@@ -256,3 +256,73 @@ def test_kernel_adjoint_form_equals_the_token_recurrence(C):
             assert ends.keys() == ends2.keys()
             for e in ends:
                 assert np.max(np.abs(ends2[e] - ends[e])) < 1e-12
+
+
+
+def kernel_rows(q, k, v, beta, g, S_a, W, mu_e, do, scale):
+    """The per-chunk u, dbeta and dg of the bf16-input CUDA backward (k_bwd_u,
+    then the epilogue of k_bwd_gemm_tc), for one chunk of length L from its
+    entry state S_a, its w rows W, the adjoint mu_e at its end and its do rows:
+      U       = T diag(beta) (V - diag(e^G) K S_a^T),  T = (I + A)^{-1},
+                A_ts = [s < t] beta_t e^{G_t - G_s} k_t . k_s
+      DQ      = scale (diag(e^G) DO S_a + Ad K),  Ad_ts = [s <= t] e^{G_t - G_s} do_t . u_s
+      dbeta_t = w_t . v_t - e^{G_t} k_t . (W S_a)_t - sum_{s<t} A'_ts X_ts,
+                A'_ts = e^{G_t - G_s} k_t . k_s,  X = W U^T
+      Z_end   = e^{G_{L-1}} <mu_e, S_a> + sum_t e^{G_{L-1} - G_t} k_t . (U mu_e)_t
+      dg_t    = Z_end + sum_{s >= t} (q_s . dq_s - beta_s v_s . w_s).
+    Returns (U, DQ, dbeta, Z_end, dg)."""
+    L, d = k.shape
+    G = np.cumsum(g)
+    ii = np.arange(L)
+    low = ii[:, None] > ii[None, :]
+    dec = np.exp(G[:, None] - G[None, :])
+    KK = k @ k.T
+    A = np.where(low, dec, 0.0) * KK * beta[:, None]
+    T = np.linalg.inv(np.eye(L) + A)
+    U = T @ (beta[:, None] * (v - np.exp(G)[:, None] * (k @ S_a.T)))
+    Ad = np.where(ii[:, None] >= ii[None, :], dec, 0.0) * (do @ U.T)
+    DQ = scale * (np.exp(G)[:, None] * (do @ S_a) + Ad @ k)
+    X = W @ U.T
+    dbeta = (np.sum(W * v, axis=1) - np.exp(G) * np.sum(k * (W @ S_a), axis=1)
+             - np.sum(np.where(low, dec, 0.0) * KK * X, axis=1))
+    dvec = np.exp(G[-1] - G)
+    Z_end = np.exp(G[-1]) * np.sum(mu_e * S_a) + np.sum(dvec * np.sum(k * (U @ mu_e), axis=1))
+    term = np.sum(q * DQ, axis=1) - beta * np.sum(v * W, axis=1)
+    dg = Z_end + np.cumsum(term[::-1])[::-1]
+    return U, DQ, dbeta, Z_end, dg
+
+
+def test_kernel_rows_form_equals_the_token_recurrence():
+    """u, dq, dbeta = w . (v - alpha S_{t-1} k) and dg = <mu_{t-1}, S_{t-1}> of the
+    kernels' product form against the token recurrence and its adjoint."""
+    rng = np.random.default_rng(41)
+    for L in (1, 7, 64):
+        d, scale = 6, 0.7
+        k = rng.normal(size=(L, d)); k /= np.linalg.norm(k, axis=1, keepdims=True)
+        q, v, do = rng.normal(size=(L, d)), rng.normal(size=(L, d)), rng.normal(size=(L, d))
+        beta = 1.0 / (1.0 + np.exp(-rng.normal(size=L)))
+        g = -np.log1p(np.exp(2.0 * rng.normal(size=L)))
+        S_a, mu_e = rng.normal(size=(d, d)), rng.normal(size=(d, d))
+        # The adjoint inside the chunk, last token first (mu_t, Lambda_t, w_t).
+        states = [S_a]
+        for t in range(L):
+            a = np.exp(g[t])
+            u = beta[t] * (v[t] - a * (states[-1] @ k[t]))
+            states.append(a * states[-1] + np.outer(u, k[t]))
+        mu = mu_e.copy()
+        W = np.zeros((L, d))
+        dg_ref = np.zeros(L)
+        for t in range(L - 1, -1, -1):
+            Lam = mu + scale * np.outer(do[t], q[t])
+            W[t] = Lam @ k[t]
+            mu = np.exp(g[t]) * (Lam - beta[t] * np.outer(W[t], k[t]))
+            dg_ref[t] = np.sum(mu * states[t])  # <mu_{t-1}, S_{t-1}>
+        U, DQ, dbeta, Z_end, dg = kernel_rows(q, k, v, beta, g, S_a, W, mu_e, do, scale)
+        for t in range(L):
+            S_prev, S_t = states[t], states[t + 1]
+            r = v[t] - np.exp(g[t]) * (S_prev @ k[t])
+            assert np.max(np.abs(U[t] - beta[t] * r)) < 1e-12
+            assert np.max(np.abs(DQ[t] - scale * (S_t.T @ do[t]))) < 1e-12
+            assert abs(dbeta[t] - W[t] @ r) < 1e-12
+        assert abs(Z_end - np.sum(mu_e * states[-1])) < 1e-12 * max(1.0, abs(Z_end))
+        assert np.max(np.abs(dg - dg_ref)) < 1e-11 * max(1.0, np.max(np.abs(dg_ref)))
