@@ -368,7 +368,8 @@ __device__ __forceinline__ void adj_walk_warp(float (&sacc)[D / 8][4], const uns
 template <int D>
 __global__ void __launch_bounds__(32 * kAdjWalkWarps, 1)
     k_adj_walk(const int32_t* __restrict__ cu, int H, int32_t* __restrict__ hdr,
-               const int32_t* __restrict__ chunk_off, const char* __restrict__ apacks,
+               const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ seq_order,
+               const char* __restrict__ apacks,
                const float* __restrict__ ds_final, float* __restrict__ mu_end,
                float* __restrict__ ydv, float* __restrict__ d_h0) {
   constexpr int C = kChunk;
@@ -377,8 +378,13 @@ __global__ void __launch_bounds__(32 * kAdjWalkWarps, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   AdjWalkSmem<D>& sm = *reinterpret_cast<AdjWalkSmem<D>*>(smem_raw);
   if (hdr[kHdrValid] != 1) return;
-  const int n = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
-  const int r0 = blockIdx.z * 16 * kAdjWalkWarps + 16 * (t >> 5);
+  // Blocks go out sequence by sequence, most chunks first (the chunk table's
+  // order), so that the longest serial chains start in the first wave.
+  constexpr int RB = D / (16 * kAdjWalkWarps);  // row blocks per (sequence, head)
+  const int per_seq = H * RB;
+  const int n = seq_order[blockIdx.x / per_seq];
+  const int h = (blockIdx.x % per_seq) / RB, t = threadIdx.x;
+  const int r0 = (blockIdx.x % RB) * 16 * kAdjWalkWarps + 16 * (t >> 5);
   const size_t DD = (size_t)D * D;
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
   const int64_t nc = (L + C - 1) / C;

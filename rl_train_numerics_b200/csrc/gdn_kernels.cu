@@ -4,7 +4,8 @@
 // Training Runs", section "Solving the linear-attention headache": a first
 // pass computes the recurrent state at chunk boundaries, then the outputs
 // within each chunk are filled in):
-//   k_chunk_table   one block: validates cu_seqlens, numbers the chunks
+//   k_chunk_table   one block: validates cu_seqlens, numbers the chunks,
+//                   orders the sequences by chunk count
 //   k_prep          one block per (chunk, head): boundary prep of full chunks
 //   k_walk          one block per (sequence, head): serial walk (mma.sync,
 //                   d = 64)
@@ -31,8 +32,10 @@ constexpr int kTableThreads = 1024;
 
 __global__ void __launch_bounds__(kTableThreads)
     k_chunk_table(const int32_t* __restrict__ cu, int N, int64_t T, int32_t* hdr,
-                  int32_t* chunk_off, int32_t* chunk_seq, int64_t max_chunks) {
+                  int32_t* chunk_off, int32_t* seq_order, int32_t* chunk_seq,
+                  int64_t max_chunks) {
   __shared__ long long part[64 + kTableThreads];
+  __shared__ int bucket[kTableThreads];
   __shared__ int bad;
   const int tid = threadIdx.x;
   if (tid == 0) bad = (cu[0] != 0 || (int64_t)cu[N] != T) ? 1 : 0;
@@ -93,6 +96,44 @@ __global__ void __launch_bounds__(kTableThreads)
     for (long long i = 0; i < nc; i++) chunk_seq[off + i] = (int32_t)n;
     off += nc;
   }
+  // The sequences by chunk count, most first (counts from kTableThreads - 1
+  // up share one place): the order in which serial per-sequence passes
+  // launch their blocks, so that the longest chains start in the first wave.
+  // Equal counts land in any order; no result depends on it.
+  bucket[tid] = 0;
+  __syncthreads();
+  auto key = [&](int64_t n) {
+    const int64_t nc = ((int64_t)cu[n + 1] - (int64_t)cu[n] + kChunk - 1) / kChunk;
+    return (int)min(nc, (int64_t)kTableThreads - 1);
+  };
+  for (int64_t n = n0; n < n1; n++) atomicAdd(&bucket[key(n)], 1);
+  __syncthreads();
+  {
+    // Exclusive scan in descending key order: thread tid takes key
+    // kTableThreads - 1 - tid.
+    const int mine = bucket[kTableThreads - 1 - tid];
+    int xs = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, xs, o);
+      if (lane >= o) xs += y;
+    }
+    if (lane == 31) part[warp] = xs;
+    __syncthreads();
+    if (warp == 0) {
+      long long ws = part[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(kFull, ws, o);
+        if (lane >= o) ws += y;
+      }
+      part[32 + lane] = ws;
+    }
+    __syncthreads();
+    bucket[kTableThreads - 1 - tid] = xs - mine + (warp > 0 ? (int)part[32 + warp - 1] : 0);
+  }
+  __syncthreads();
+  for (int64_t n = n0; n < n1; n++) seq_order[atomicAdd(&bucket[key(n)], 1)] = (int32_t)n;
   if (tid == 0) hdr[kHdrValid] = 1;
 }
 
@@ -197,14 +238,18 @@ template <int D, class IN>
 __global__ void __launch_bounds__(walk_threads<D>(), 1)
     k_walk(const int32_t* __restrict__ cu, int H, const float* __restrict__ h0,
            int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
-           const char* __restrict__ packs, float* __restrict__ bstate,
+           const int32_t* __restrict__ seq_order, const char* __restrict__ packs,
+           float* __restrict__ bstate,
            float* __restrict__ s_run_final, float* __restrict__ s_run_scale,
            float* __restrict__ s_bnd_final) {
   constexpr size_t PB = pack_size<D, IN>();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   WalkSmem<D, IN>& sm = *reinterpret_cast<WalkSmem<D, IN>*>(smem_raw);
-  const int n = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
+  // One block per (sequence, head), sequences in the chunk table's order
+  // (most chunks first).
+  const int t = threadIdx.x;
   if (hdr[kHdrValid] != 1) return;
+  const int n = seq_order[blockIdx.x / H], h = blockIdx.x % H;
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
   const int64_t nf = L / kChunk, nc = (L + kChunk - 1) / kChunk;
   const int64_t base = chunk_off[n];
@@ -316,7 +361,8 @@ template <int D, class IN>
 __global__ void __launch_bounds__(kWalkThreads, 1)
     k_walk_tc(const int32_t* __restrict__ cu, int H, const float* __restrict__ h0,
               int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
-              const char* __restrict__ packs, float* __restrict__ bstate,
+              const int32_t* __restrict__ seq_order, const char* __restrict__ packs,
+              float* __restrict__ bstate,
               float* __restrict__ s_run_final, float* __restrict__ s_run_scale,
               float* __restrict__ s_bnd_final) {
   static_assert(use_tc<D, IN>(), "tcgen05 walk: d = 128, bf16 inputs");
@@ -324,8 +370,11 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
   constexpr size_t PB = pack_size<D, IN>();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   WalkTcSmem<D, IN>& sm = *reinterpret_cast<WalkTcSmem<D, IN>*>(smem_raw);
-  const int n = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
+  // One block per (sequence, head), sequences in the chunk table's order
+  // (most chunks first).
+  const int t = threadIdx.x;
   if (hdr[kHdrValid] != 1) return;
+  const int n = seq_order[blockIdx.x / H], h = blockIdx.x % H;
   const int w = t >> 5, row = 32 * (w & 3) + (t & 31), col0 = SC * (w >> 2);
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
   const int64_t nf = L / kChunk, nc = (L + kChunk - 1) / kChunk;
@@ -934,8 +983,9 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     return a.events ? cudaEventRecord(static_cast<cudaEvent_t>(a.events[i]), st) : cudaSuccess;
   };
   GDN_TRY(mark(0));
+  int32_t* seq_order = reinterpret_cast<int32_t*>(ws + L.seq_order);
   k_chunk_table<<<1, kTableThreads, 0, st>>>(a.cu_seqlens, a.n_seqs, a.T, hdr, chunk_off,
-                                             chunk_seq, L.max_chunks);
+                                             seq_order, chunk_seq, L.max_chunks);
   GDN_TRY(cudaGetLastError());
   const dim3 gchunks((unsigned)L.max_chunks, (unsigned)a.H);
   GDN_TRY(mark(1));
@@ -952,16 +1002,16 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     auto kern = k_walk_tc<D, IN>;
     const size_t sm = sizeof(WalkTcSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
-    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), kWalkThreads, sm, st>>>(
-        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final, a.s_run_scale,
+    kern<<<(unsigned)((size_t)a.n_seqs * a.H), kWalkThreads, sm, st>>>(
+        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, seq_order, packs, bstate, a.s_run_final, a.s_run_scale,
         a.s_bnd_final);
     GDN_TRY(cudaGetLastError());
   } else {
     auto kern = k_walk<D, IN>;
     const size_t sm = sizeof(WalkSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
-    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), walk_threads<D>(), sm, st>>>(
-        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final, a.s_run_scale,
+    kern<<<(unsigned)((size_t)a.n_seqs * a.H), walk_threads<D>(), sm, st>>>(
+        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, seq_order, packs, bstate, a.s_run_final, a.s_run_scale,
         a.s_bnd_final);
     GDN_TRY(cudaGetLastError());
   }
@@ -1000,8 +1050,9 @@ static cudaError_t native_impl(const FwdArgs& a, cudaStream_t st) {
     return a.events ? cudaEventRecord(static_cast<cudaEvent_t>(a.events[i]), st) : cudaSuccess;
   };
   GDN_TRY(mark(0));
+  int32_t* seq_order = reinterpret_cast<int32_t*>(ws + L.seq_order);
   k_chunk_table<<<1, kTableThreads, 0, st>>>(a.cu_seqlens, a.n_seqs, a.T, hdr, chunk_off,
-                                             chunk_seq, L.max_chunks);
+                                             seq_order, chunk_seq, L.max_chunks);
   GDN_TRY(cudaGetLastError());
   GDN_TRY(mark(1));
   {
@@ -1018,8 +1069,8 @@ static cudaError_t native_impl(const FwdArgs& a, cudaStream_t st) {
     auto kern = k_walk_tc<D, IN>;
     const size_t sm = sizeof(WalkTcSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
-    kern<<<dim3((unsigned)a.n_seqs, (unsigned)a.H), kWalkThreads, sm, st>>>(
-        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, packs, bstate, a.s_run_final, nullptr,
+    kern<<<(unsigned)((size_t)a.n_seqs * a.H), kWalkThreads, sm, st>>>(
+        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, seq_order, packs, bstate, a.s_run_final, nullptr,
         a.s_bnd_final);
     GDN_TRY(cudaGetLastError());
   }

@@ -31,7 +31,7 @@ constexpr size_t pack_bytes(int D, bool in_bf16) {
 struct FwdLayout {
   int64_t max_chunks;
   size_t pack_bytes;
-  size_t hdr, chunk_off, chunk_seq, bstate, pack, total;
+  size_t hdr, chunk_off, seq_order, chunk_seq, bstate, pack, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -46,6 +46,8 @@ inline FwdLayout fwd_layout(int n_seqs, int64_t T, int H, int dk, int dv, int C,
   off += align256(64 * sizeof(int32_t));
   L.chunk_off = off;
   off += align256((size_t)(n_seqs + 1) * sizeof(int32_t));
+  L.seq_order = off;
+  off += align256((size_t)n_seqs * sizeof(int32_t));
   L.chunk_seq = off;
   off += align256(mc * sizeof(int32_t));
   L.bstate = off;
