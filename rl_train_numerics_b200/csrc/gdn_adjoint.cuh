@@ -22,7 +22,7 @@
 // token scan's chain per token.
 //   k_adj_prep  per (chunk, head): the forward prep's T (trailing partial
 //               chunks zero-padded), Pm, X; writes the chunk's adjoint pack
-//   k_adj_walk  per (sequence, head, 32 state rows), last chunk first: mu at
+//   k_adj_walk  per (sequence, head, 64 state rows), last chunk first: mu at
 //               every chunk end, dh0, and Ydv = (mu_e K^T) diag(dvec)
 //   k_adj_w     per (chunk, head): W -> w and dv = beta w
 #pragma once
@@ -37,7 +37,8 @@ namespace gdn {
 constexpr int kAdjNT = 3;  // bf16 terms of an fp32 operand
 
 // The adjoint pack of one (chunk, head).  Planes are bf16 in the core layout
-// (64 rows); the walk bulk-copies [0, offsetof(T)), the solve the rest.
+// (64 rows); the walk bulk-copies the head, the keys, its rows' do columns, X and
+// Tb, the solve the rest.
 template <int D>
 struct AdjPack {
   float dvec[kChunk];
@@ -50,10 +51,6 @@ struct AdjPack {
   __nv_bfloat16 T[kAdjNT][kChunk * kChunk];     // [m][t], t <= m
   __nv_bfloat16 Pm[kAdjNT][kChunk * kChunk];    // [r][t], t <= r
 };
-template <int D>
-constexpr size_t adj_walk_bytes() {
-  return offsetof(AdjPack<D>, T);
-}
 template <int D>
 constexpr size_t adj_pack_bytes() {
   return round_up(sizeof(AdjPack<D>), 128);
@@ -240,23 +237,97 @@ __global__ void __launch_bounds__(kBndThreads, 3)
 // ----------------------------------------------------------------------------
 // k_adj_walk
 // ----------------------------------------------------------------------------
-constexpr int kAdjWalkWarps = 2;  // 32 state rows per block
+// A block takes 32 state rows of one (sequence, head): two pairs of warps,
+// 16 rows per pair; the pair's two warps hold columns 0 .. D/2 - 1 and
+// D/2 .. D - 1 of those rows.  (64-row blocks, eight warps to an SM, made
+// each chunk step slower: 0.84 against 0.64 ms on the trainer batch.)
+constexpr int kAdjWalkRows = 32;
+constexpr int kAdjWalkPairs = kAdjWalkRows / 16;
+constexpr int kAdjWalkThreads = 64 * kAdjWalkPairs;
+
+// One chunk's walk operands in shared memory: the pack's head and keys, the
+// do columns of the block's rows (their core-layout column groups), X and Tb.
+template <int D>
+struct AdjWalkBuf {
+  float dvec[kChunk];
+  float beta[kChunk];
+  float gamma[4];
+  __nv_bfloat16 K[1][kChunk * D];                 // [t][j]
+  __nv_bfloat16 DOr[1][kChunk * kAdjWalkRows];    // [t][i - first row of the block]
+  __nv_bfloat16 X[kAdjNT][kChunk * D];            // [t][j]
+  __nv_bfloat16 Tb[kAdjNT][kChunk * kChunk];      // [t][m], m <= t
+};
+template <int D>
+constexpr uint32_t adj_walk_head_bytes() {
+  return (uint32_t)offsetof(AdjPack<D>, DO);
+}
+template <int D>
+constexpr uint32_t adj_walk_xtb_bytes() {
+  return (uint32_t)(offsetof(AdjPack<D>, T) - offsetof(AdjPack<D>, X));
+}
+template <int D>
+constexpr uint32_t adj_walk_copy_bytes() {
+  return adj_walk_head_bytes<D>() + (uint32_t)(kChunk * kAdjWalkRows * 2) +
+         adj_walk_xtb_bytes<D>();
+}
 
 template <int D>
 struct AdjWalkSmem {
-  alignas(128) unsigned char buf[2][round_up(adj_walk_bytes<D>(), 128)];
+  alignas(128) AdjWalkBuf<D> buf[2];
+  float4 xch[kAdjWalkPairs][2][8][32];  // each warp's half of mu K^T, [n8 tile][lane]
   uint64_t bar[2];
 };
 
-// One reverse step on a warp's 16 state rows (sacc, accumulator layout):
-//   Ydv = (mu K^T) diag(dvec)  (written to ydv_rows, [row][t])
-//   mu <- gamma mu + (-Ydv) Tb K + DO^T X
+// The accumulator-layout rows r0 .. r0 + 15, columns c0 .. c0 + 8 NT - 1 of a
+// D x D row-major matrix (load; store with lanes t and t^1 swapping halves so
+// that every lane writes one 16-byte run).
+template <int D, int NT>
+__device__ __forceinline__ void sacc_load_cols(float (&sacc)[NT][4], const float* S, int r0, int c0) {
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int n = 0; n < NT; n++)
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+      const float2 x = *reinterpret_cast<const float2*>(S + (size_t)(r0 + gq + 8 * hf) * D + c0 +
+                                                        8 * n + 2 * tq);
+      sacc[n][2 * hf] = x.x;
+      sacc[n][2 * hf + 1] = x.y;
+    }
+}
+template <int D, int NT>
+__device__ __forceinline__ void sacc_store_cols(const float (&sacc)[NT][4], float* S, int r0, int c0) {
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3, odd = tq & 1;
+#pragma unroll
+  for (int n = 0; n < NT; n++) {
+    const float s0 = odd ? sacc[n][0] : sacc[n][2];
+    const float s1 = odd ? sacc[n][1] : sacc[n][3];
+    const float r0v = __shfl_xor_sync(kFull, s0, 1);
+    const float r1v = __shfl_xor_sync(kFull, s1, 1);
+    float4 out;
+    if (!odd) out = make_float4(sacc[n][0], sacc[n][1], r0v, r1v);
+    else out = make_float4(r0v, r1v, sacc[n][2], sacc[n][3]);
+    const int row = r0 + gq + 8 * odd, col = c0 + 8 * n + 2 * (tq & 2);
+    *reinterpret_cast<float4*>(S + (size_t)row * D + col) = out;
+  }
+}
+
+__device__ __forceinline__ void pair_sync(int id) {
+  asm volatile("bar.sync %0, 64;\n" ::"r"(id) : "memory");
+}
+
+// One reverse step on a warp's 16 state rows and D / 2 columns (sacc,
+// accumulator layout; ch = 0 or 1 the column half):
+//   Ydv = (mu K^T) diag(dvec)  (the pair's halves of the contraction added
+//         through shared memory; each warp writes half of its tokens to
+//         ydv_rows, [row][t])
+//   mu <- gamma mu + (-Ydv) Tb K + DO^T X       (this warp's columns)
+// rl is the pair's first row within the block (its do columns in DOr).
 template <int D>
-__device__ __forceinline__ void adj_walk_warp(float (&sacc)[D / 8][4], const unsigned char* pb,
-                                              int r0, float* ydv_rows) {
-  using bf16 = __nv_bfloat16;
-  constexpr int C = kChunk, PL = C * C, PD = C * D;
-  const AdjPack<D>& pk = *reinterpret_cast<const AdjPack<D>*>(pb);
+__device__ __forceinline__ void adj_walk_warp(float (&sacc)[D / 16][4], const AdjWalkBuf<D>& pk,
+                                              int rl, int ch, float4 (*xs)[32],
+                                              const float4 (*xo)[32], int bar_id,
+                                              float* ydv_rows) {
+  constexpr int C = kChunk, KH = D / 32;  // k16 steps (and n16 pairs) of a column half
   const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
   using P33 = SplitPairs<kAdjNT, kAdjNT>;
   using P31 = SplitPairs<kAdjNT, 1>;
@@ -267,19 +338,30 @@ __device__ __forceinline__ void adj_walk_warp(float (&sacc)[D / 8][4], const uns
 #pragma unroll
     for (int e = 0; e < 4; e++) y[n][e] = 0.f;
 #pragma unroll
-  for (int ks = 0; ks < D / 16; ks++) {
+  for (int kl = 0; kl < KH; kl++) {
     uint32_t a[kAdjNT][4];
-    acc_to_afrag<kAdjNT>(sacc[2 * ks], sacc[2 * ks + 1], a);
+    acc_to_afrag<kAdjNT>(sacc[2 * kl], sacc[2 * kl + 1], a);
 #pragma unroll
     for (int np = 0; np < 4; np++) {
       uint32_t b[4];
-      ldsm_x4(b, bfrag_nk_addr(pk.K[0], 16 * np, 16 * ks));
+      ldsm_x4(b, bfrag_nk_addr(pk.K[0], 16 * np, 16 * (KH * ch + kl)));
 #pragma unroll
       for (int p = 0; p < P31::kCount; p++) {
         mma16816(y[2 * np], a[P31::a(p)], b[0], b[1]);
         mma16816(y[2 * np + 1], a[P31::a(p)], b[2], b[3]);
       }
     }
+  }
+#pragma unroll
+  for (int n = 0; n < 8; n++) xs[n][lane] = make_float4(y[n][0], y[n][1], y[n][2], y[n][3]);
+  pair_sync(bar_id);
+#pragma unroll
+  for (int n = 0; n < 8; n++) {
+    const float4 o = xo[n][lane];
+    y[n][0] = __fadd_rn(y[n][0], o.x);
+    y[n][1] = __fadd_rn(y[n][1], o.y);
+    y[n][2] = __fadd_rn(y[n][2], o.z);
+    y[n][3] = __fadd_rn(y[n][3], o.w);
   }
 #pragma unroll
   for (int n = 0; n < 8; n++) {
@@ -289,11 +371,13 @@ __device__ __forceinline__ void adj_walk_warp(float (&sacc)[D / 8][4], const uns
     for (int hf = 0; hf < 2; hf++) {
       y[n][2 * hf] = __fmul_rn(d0, y[n][2 * hf]);
       y[n][2 * hf + 1] = __fmul_rn(d1, y[n][2 * hf + 1]);
-      *reinterpret_cast<float2*>(ydv_rows + (size_t)(gq + 8 * hf) * C + t) =
-          f2(y[n][2 * hf], y[n][2 * hf + 1]);
+      if ((n >> 2) == ch)
+        *reinterpret_cast<float2*>(ydv_rows + (size_t)(gq + 8 * hf) * C + t) =
+            f2(y[n][2 * hf], y[n][2 * hf + 1]);
     }
   }
-  // Z = (-Ydv) Tb
+  // Z = (-Ydv) Tb, the full 16 x C on both warps of the pair (splitting it
+  // between them costs a second exchange and was slower)
   float z[8][4];
 #pragma unroll
   for (int n = 0; n < 8; n++)
@@ -323,10 +407,10 @@ __device__ __forceinline__ void adj_walk_warp(float (&sacc)[D / 8][4], const uns
       }
     }
   }
-  // mu <- gamma mu, then + Z K, then + DO^T X
+  // mu <- gamma mu, then + Z K, then + DO^T X (this warp's columns)
   const float gam = pk.gamma[0];
 #pragma unroll
-  for (int n = 0; n < D / 8; n++)
+  for (int n = 0; n < D / 16; n++)
 #pragma unroll
     for (int e = 0; e < 4; e++) sacc[n][e] = __fmul_rn(gam, sacc[n][e]);
 #pragma unroll
@@ -334,9 +418,9 @@ __device__ __forceinline__ void adj_walk_warp(float (&sacc)[D / 8][4], const uns
     uint32_t a[kAdjNT][4];
     acc_to_afrag<kAdjNT>(z[2 * ks], z[2 * ks + 1], a);
 #pragma unroll
-    for (int np = 0; np < D / 16; np++) {
+    for (int np = 0; np < KH; np++) {
       uint32_t b[4];
-      ldsm_x4_t(b, bfrag_kn_addr(pk.K[0], 16 * ks, 16 * np));
+      ldsm_x4_t(b, bfrag_kn_addr(pk.K[0], 16 * ks, 16 * (KH * ch + np)));
 #pragma unroll
       for (int p = 0; p < P31::kCount; p++) {
         mma16816(sacc[2 * np], a[P31::a(p)], b[0], b[1]);
@@ -347,13 +431,13 @@ __device__ __forceinline__ void adj_walk_warp(float (&sacc)[D / 8][4], const uns
 #pragma unroll
   for (int ks = 0; ks < 4; ks++) {
     uint32_t a[1][4];
-    ldsm_x4_t(a[0], afrag_t_addr(pk.DO[0], r0, 16 * ks));
+    ldsm_x4_t(a[0], afrag_t_addr(pk.DOr[0], rl, 16 * ks));
 #pragma unroll
-    for (int np = 0; np < D / 16; np++) {
+    for (int np = 0; np < KH; np++) {
       uint32_t b[kAdjNT][4];
 #pragma unroll
       for (int qq = 0; qq < kAdjNT; qq++)
-        ldsm_x4_t(b[qq], bfrag_kn_addr(pk.X[qq], 16 * ks, 16 * np));
+        ldsm_x4_t(b[qq], bfrag_kn_addr(pk.X[qq], 16 * ks, 16 * (KH * ch + np)));
 #pragma unroll
       for (int p = 0; p < P13::kCount; p++) {
         mma16816(sacc[2 * np], a[P13::a(p)], b[P13::b(p)][0], b[P13::b(p)][1]);
@@ -361,30 +445,35 @@ __device__ __forceinline__ void adj_walk_warp(float (&sacc)[D / 8][4], const uns
       }
     }
   }
-  (void)PL;
-  (void)PD;
 }
 
 template <int D>
-__global__ void __launch_bounds__(32 * kAdjWalkWarps, 1)
+__global__ void __launch_bounds__(kAdjWalkThreads, 1)
     k_adj_walk(const int32_t* __restrict__ cu, int H, int32_t* __restrict__ hdr,
                const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ seq_order,
                const char* __restrict__ apacks,
                const float* __restrict__ ds_final, float* __restrict__ mu_end,
                float* __restrict__ ydv, float* __restrict__ d_h0) {
-  constexpr int C = kChunk;
-  constexpr uint32_t WB = (uint32_t)adj_walk_bytes<D>();
-  static_assert(WB % 16 == 0, "bulk copies are 16-byte pieces");
+  constexpr int C = kChunk, RB = D / kAdjWalkRows, NT = D / 16;
+  static_assert(D % kAdjWalkRows == 0, "whole row blocks");
+  constexpr uint32_t HB = adj_walk_head_bytes<D>(), XB = adj_walk_xtb_bytes<D>();
+  constexpr uint32_t DB = (uint32_t)(C * kAdjWalkRows * 2);
+  static_assert(HB % 16 == 0 && XB % 16 == 0 && DB % 16 == 0 &&
+                    offsetof(AdjWalkBuf<D>, K) == offsetof(AdjPack<D>, K) &&
+                    offsetof(AdjWalkBuf<D>, X) % 16 == 0 &&
+                    offsetof(AdjWalkBuf<D>, Tb) - offsetof(AdjWalkBuf<D>, X) ==
+                        offsetof(AdjPack<D>, Tb) - offsetof(AdjPack<D>, X),
+                "bulk copies of 16-byte pieces into matching layouts");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   AdjWalkSmem<D>& sm = *reinterpret_cast<AdjWalkSmem<D>*>(smem_raw);
   if (hdr[kHdrValid] != 1) return;
   // Blocks go out sequence by sequence, most chunks first (the chunk table's
   // order), so that the longest serial chains start in the first wave.
-  constexpr int RB = D / (16 * kAdjWalkWarps);  // row blocks per (sequence, head)
   const int per_seq = H * RB;
   const int n = seq_order[blockIdx.x / per_seq];
-  const int h = (blockIdx.x % per_seq) / RB, t = threadIdx.x;
-  const int r0 = (blockIdx.x % RB) * 16 * kAdjWalkWarps + 16 * (t >> 5);
+  const int h = (blockIdx.x % per_seq) / RB, rb = blockIdx.x % RB, t = threadIdx.x;
+  const int w = t >> 5, pair = w >> 1, ch = w & 1;
+  const int rl = 16 * pair, r0 = kAdjWalkRows * rb + rl, c0 = (D / 2) * ch;
   const size_t DD = (size_t)D * D;
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
   const int64_t nc = (L + C - 1) / C;
@@ -392,15 +481,26 @@ __global__ void __launch_bounds__(32 * kAdjWalkWarps, 1)
   auto pack = [&](int64_t cc) {
     return apacks + ((size_t)(base + cc) * H + h) * adj_pack_bytes<D>();
   };
+  // The block's do columns are core-layout column groups 8 rb .. 8 rb + 7 of
+  // the pack's do plane: one contiguous run.
   auto fetch = [&](int b, int64_t cc) {
     const uint32_t mb = smem_u32(&sm.bar[b]);
-    mbar_expect_tx(mb, WB);
-    bulk_load(smem_u32(sm.buf[b]), pack(cc), WB, mb);
+    const char* src = pack(cc);
+    mbar_expect_tx(mb, HB + DB + XB);
+    bulk_load(smem_u32(&sm.buf[b]), src, HB, mb);
+    bulk_load(smem_u32(sm.buf[b].DOr[0]), src + offsetof(AdjPack<D>, DO) + (size_t)rb * DB, DB, mb);
+    bulk_load(smem_u32(sm.buf[b].X[0]), src + offsetof(AdjPack<D>, X), XB, mb);
   };
   pack_bars_init(sm.bar);
-  float sacc[D / 8][4];
-  if (ds_final) sacc_load<D>(sacc, ds_final + ((size_t)n * H + h) * DD, r0);
-  else sacc_zero<D>(sacc);
+  float sacc[NT][4];
+  if (ds_final) {
+    sacc_load_cols<D, NT>(sacc, ds_final + ((size_t)n * H + h) * DD, r0, c0);
+  } else {
+#pragma unroll
+    for (int i = 0; i < NT; i++)
+#pragma unroll
+      for (int e = 0; e < 4; e++) sacc[i][e] = 0.f;
+  }
   if (t == 0 && nc > 0) fetch(0, nc - 1);
   int64_t issued = nc > 0 ? 1 : 0;
   bool ok = true;
@@ -411,20 +511,21 @@ __global__ void __launch_bounds__(32 * kAdjWalkWarps, 1)
       issued = j + 2;
     }
     const size_t unit = (size_t)(base + cc) * H + h;
-    sacc_store<D>(sacc, mu_end + unit * DD, r0);
+    sacc_store_cols<D, NT>(sacc, mu_end + unit * DD, r0, c0);
     if (__syncthreads_or(!pack_wait(sm.bar, j))) {
       ok = false;
       pack_drain(sm.bar, j, issued);
       break;
     }
-    adj_walk_warp<D>(sacc, sm.buf[j & 1], r0, ydv + (unit * D + r0) * C);
-    __syncthreads();  // buffer j & 1 is refilled with chunk cc - 2
+    adj_walk_warp<D>(sacc, sm.buf[j & 1], rl, ch, sm.xch[pair][ch], sm.xch[pair][ch ^ 1],
+                     1 + pair, ydv + (unit * D + r0) * C);
+    __syncthreads();  // buffer j & 1 is refilled with chunk cc - 2; xch is free
   }
   if (!ok) {
     if (t == 0) atomicOr(&hdr[kHdrError], kErrTimeout);
     return;
   }
-  if (d_h0) sacc_store<D>(sacc, d_h0 + ((size_t)n * H + h) * DD, r0);
+  if (d_h0) sacc_store_cols<D, NT>(sacc, d_h0 + ((size_t)n * H + h) * DD, r0, c0);
 }
 
 // ----------------------------------------------------------------------------

@@ -1340,8 +1340,8 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
       const size_t sm = sizeof(AdjWalkSmem<D>);
       GDN_BWD_TRY(bwd_set_smem(kern, sm));
       const int32_t* seq_order = reinterpret_cast<const int32_t*>(ws + L.fwd.seq_order);
-      kern<<<(unsigned)((size_t)f.n_seqs * f.H * (D / (16 * kAdjWalkWarps))),
-             32 * kAdjWalkWarps, sm, st>>>(f.cu_seqlens, f.H, hdr_w, chunk_off, seq_order, apack,
+      kern<<<(unsigned)((size_t)f.n_seqs * f.H * (D / kAdjWalkRows)), kAdjWalkThreads, sm,
+             st>>>(f.cu_seqlens, f.H, hdr_w, chunk_off, seq_order, apack,
                                            a.ds_final, mu_end, ydv, a.d_h0);
       GDN_BWD_TRY(cudaGetLastError());
     }
