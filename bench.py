@@ -601,7 +601,7 @@ def run_train_part(gdn, W, dev, rank, world, args, flush, peaks):
     fwd, bwd = el(0, 4), el(5, 9)
     kern = {"fwd_chunk_table": el(0, 1), "fwd_boundary_prep": el(1, 2),
             "fwd_boundary_walk": el(2, 3), "fwd_intra_chunk_fill": el(3, 4),
-            "bwd_adjoint_scan": el(6, 7), "bwd_chunk_u": el(7, 8),
+            "bwd_adjoint_prep_walk": el(6, 7), "bwd_w_solve_and_u": el(7, 8),
             "bwd_chunk_products": el(8, 9)}
     ms = max_over_ranks(fwd + bwd, world)
     fwd_max = max_over_ranks(fwd, world)

@@ -24,7 +24,8 @@
 //               chunks zero-padded), Pm, X; writes the chunk's adjoint pack
 //   k_adj_walk  per (sequence, head, 64 state rows), last chunk first: mu at
 //               every chunk end, dh0, and Ydv = (mu_e K^T) diag(dvec)
-//   k_adj_w     per (chunk, head): W -> w and dv = beta w
+//   adj_w_item  per (chunk, head): W -> w and dv = beta w (launched with the
+//               chunk u of the backward, gdn_backward.cu's k_bwd_wu)
 #pragma once
 
 #include <cstddef>
@@ -529,7 +530,7 @@ __global__ void __launch_bounds__(kAdjWalkThreads, 1)
 }
 
 // ----------------------------------------------------------------------------
-// k_adj_w
+// The W solve (one (chunk, head) per block)
 // ----------------------------------------------------------------------------
 constexpr int kAdjWThreads = 256;
 
@@ -544,19 +545,17 @@ struct AdjWSmem {
   __nv_bfloat16 R[kAdjNT][kChunk * D];             // right-hand side, [m][i]
 };
 
+// The W solve of one (chunk, head) item; one block of kAdjWThreads threads.
 template <int D>
-__global__ void __launch_bounds__(kAdjWThreads, 1)
-    k_adj_w(const int32_t* __restrict__ cu, int H, float scale, const int32_t* __restrict__ hdr,
-            const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
-            const char* __restrict__ apacks, const float* __restrict__ ydv,
-            float* __restrict__ wbuf, float* __restrict__ d_v) {
+__device__ __forceinline__ void adj_w_item(AdjWSmem<D>& sm, int c, int h,
+                                           const int32_t* __restrict__ cu, int H, float scale,
+                                           const int32_t* __restrict__ chunk_off,
+                                           const int32_t* __restrict__ chunk_seq,
+                                           const char* __restrict__ apacks,
+                                           const float* __restrict__ ydv, float* __restrict__ wbuf,
+                                           float* __restrict__ d_v) {
   using bf16 = __nv_bfloat16;
   constexpr int C = kChunk, PL = C * C, PD = C * D, NT8 = D / 16;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  AdjWSmem<D>& sm = *reinterpret_cast<AdjWSmem<D>*>(smem_raw);
-  if (hdr[kHdrValid] != 1) return;
-  const int c = blockIdx.x, h = blockIdx.y;
-  if (c >= hdr[kHdrChunks]) return;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
   const int mt = w & 3, nh = w >> 2;
   const FillItem it = fill_item(c * H + h, H, cu, chunk_off, chunk_seq);

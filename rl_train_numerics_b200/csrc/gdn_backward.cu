@@ -50,14 +50,16 @@
 // Kernels, in launch order:
 //   forward pass 1   chunk table and boundary states S_a, exactly as the
 //                    forward computes them
-//   adjoint          bf16 inputs: k_adj_prep, k_adj_walk, k_adj_w
-//                    (gdn_adjoint.cuh), the adjoint in chunk form; fp32
+//   adjoint          bf16 inputs: k_adj_prep, k_adj_walk (gdn_adjoint.cuh),
+//                    the adjoint in chunk form, then its W solve in k_bwd_wu
+//                    below; fp32
 //                    inputs: k_bwd_scan, one block per (sequence, head, 32
 //                    rows), the adjoint recurrence over the whole sequence,
 //                    last token first.  Both write w, dv, the adjoint at
 //                    every chunk end and dh0
-//   k_bwd_u          bf16 inputs, one block per (chunk, head): u in product
-//                    form from S_a and the prep's T
+//   k_bwd_wu         bf16 inputs: blocks alternating between the adjoint's W
+//                    solve and u in product form from S_a and the prep's T,
+//                    one (chunk, head) each
 //   k_bwd_rows       fp32 inputs, one block per (chunk, head): recomputes the
 //                    chunk's states from S_a with the forward fill's per-token
 //                    step (the states the outputs came from); writes u,
@@ -1146,19 +1148,18 @@ struct BwdUSmem {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kUThreads, 2)
-    k_bwd_u(const __nv_bfloat16* __restrict__ v, const float* __restrict__ beta,
-            const float* __restrict__ g, const int32_t* __restrict__ cu, int H,
-            const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
-            const int32_t* __restrict__ chunk_seq, const float* __restrict__ bstate,
-            const char* __restrict__ apacks, float* __restrict__ ubuf) {
+__device__ __forceinline__ void bwd_u_item(BwdUSmem<D>& sm, int c, int h,
+                                           const __nv_bfloat16* __restrict__ v,
+                                           const float* __restrict__ beta,
+                                           const float* __restrict__ g,
+                                           const int32_t* __restrict__ cu, int H,
+                                           const int32_t* __restrict__ chunk_off,
+                                           const int32_t* __restrict__ chunk_seq,
+                                           const float* __restrict__ bstate,
+                                           const char* __restrict__ apacks,
+                                           float* __restrict__ ubuf) {
   using bf16 = __nv_bfloat16;
   constexpr int C = kChunk, PL = C * C, PD = C * D, NT8 = D / 16, ST = 64 * D;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  BwdUSmem<D>& sm = *reinterpret_cast<BwdUSmem<D>*>(smem_raw);
-  if (hdr[kHdrValid] != 1) return;
-  const int c = blockIdx.x, h = blockIdx.y;
-  if (c >= hdr[kHdrChunks]) return;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
   const int mt = w & 3, nh = w >> 2;
   const FillItem it = fill_item(c * H + h, H, cu, chunk_off, chunk_seq);
@@ -1286,6 +1287,39 @@ __global__ void __launch_bounds__(kUThreads, 2)
 }
 
 // ----------------------------------------------------------------------------
+// W solve and chunk u in one launch (bf16 inputs)
+// ----------------------------------------------------------------------------
+// Two independent per-chunk passes, both latency-bound: blocks alternate
+// between them (even x: the W solve, odd x: u), so that an SM holds one of
+// each and their waits overlap.
+static_assert(kAdjWThreads == kUThreads, "one block shape for both passes");
+
+template <int D>
+union BwdWUSmem {
+  AdjWSmem<D> w;
+  BwdUSmem<D> u;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kUThreads, 2)
+    k_bwd_wu(const __nv_bfloat16* __restrict__ v, const float* __restrict__ beta,
+             const float* __restrict__ g, const int32_t* __restrict__ cu, int H, float scale,
+             const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+             const int32_t* __restrict__ chunk_seq, const float* __restrict__ bstate,
+             const char* __restrict__ apacks, const float* __restrict__ ydv,
+             float* __restrict__ wbuf, float* __restrict__ d_v, float* __restrict__ ubuf) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  BwdWUSmem<D>& sm = *reinterpret_cast<BwdWUSmem<D>*>(smem_raw);
+  if (hdr[kHdrValid] != 1) return;
+  const int c = blockIdx.x >> 1, h = blockIdx.y;
+  if (c >= hdr[kHdrChunks]) return;
+  if ((blockIdx.x & 1) == 0)
+    adj_w_item<D>(sm.w, c, h, cu, H, scale, chunk_off, chunk_seq, apacks, ydv, wbuf, d_v);
+  else
+    bwd_u_item<D>(sm.u, c, h, v, beta, g, cu, H, chunk_off, chunk_seq, bstate, apacks, ubuf);
+}
+
+// ----------------------------------------------------------------------------
 // Launcher
 // ----------------------------------------------------------------------------
 template <class KernelT>
@@ -1345,12 +1379,14 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
                                            a.ds_final, mu_end, ydv, a.d_h0);
       GDN_BWD_TRY(cudaGetLastError());
     }
-    {
-      auto kern = k_adj_w<D>;
-      const size_t sm = sizeof(AdjWSmem<D>);
+    GDN_BWD_TRY(mark(2));
+    {  // the W solve and u (dbeta and dg come with dq and dk)
+      auto kern = k_bwd_wu<D>;
+      const size_t sm = sizeof(BwdWUSmem<D>);
       GDN_BWD_TRY(bwd_set_smem(kern, sm));
-      kern<<<gchunks, kAdjWThreads, sm, st>>>(f.cu_seqlens, f.H, f.scale, hdr, chunk_off,
-                                              chunk_seq, apack, ydv, wbuf, a.d_v);
+      kern<<<dim3(2 * (unsigned)L.fwd.max_chunks, (unsigned)f.H), kUThreads, sm, st>>>(
+          v, f.beta, f.g, f.cu_seqlens, f.H, f.scale, hdr, chunk_off, chunk_seq, bstate, apack,
+          ydv, wbuf, a.d_v, ubuf);
       GDN_BWD_TRY(cudaGetLastError());
     }
   } else {
@@ -1361,22 +1397,13 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
         q, k, f.beta, f.g, d_o, a.ds_final, f.cu_seqlens, f.H, f.scale, hdr, chunk_off, mu_end,
         wbuf, a.d_v, a.d_h0);
     GDN_BWD_TRY(cudaGetLastError());
-  }
-  GDN_BWD_TRY(mark(2));
-  if constexpr (sizeof(IN) == 2) {  // bf16 inputs: u in product form, dbeta and dg with dq, dk
-    auto kern = k_bwd_u<D>;
-    const size_t sm = sizeof(BwdUSmem<D>);
-    GDN_BWD_TRY(bwd_set_smem(kern, sm));
-    kern<<<gchunks, kUThreads, sm, st>>>(v, f.beta, f.g, f.cu_seqlens, f.H, hdr, chunk_off,
-                                         chunk_seq, bstate, ws + L.apack, ubuf);
-    GDN_BWD_TRY(cudaGetLastError());
-  } else {
-    auto kern = k_bwd_rows<D, IN>;
-    const size_t sm = sizeof(RowsSmem<D, IN>);
-    GDN_BWD_TRY(bwd_set_smem(kern, sm));
-    kern<<<gchunks, kFillThreads, sm, st>>>(q, k, v, f.beta, f.g, d_o, f.cu_seqlens, f.H, f.scale,
-                                            hdr, chunk_off, chunk_seq, bstate, mu_end, wbuf, ubuf,
-                                            a.d_beta, a.d_g);
+    GDN_BWD_TRY(mark(2));
+    auto kern2 = k_bwd_rows<D, IN>;
+    const size_t sm2 = sizeof(RowsSmem<D, IN>);
+    GDN_BWD_TRY(bwd_set_smem(kern2, sm2));
+    kern2<<<gchunks, kFillThreads, sm2, st>>>(q, k, v, f.beta, f.g, d_o, f.cu_seqlens, f.H,
+                                              f.scale, hdr, chunk_off, chunk_seq, bstate, mu_end,
+                                              wbuf, ubuf, a.d_beta, a.d_g);
     GDN_BWD_TRY(cudaGetLastError());
   }
   GDN_BWD_TRY(mark(3));
