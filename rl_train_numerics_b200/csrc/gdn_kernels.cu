@@ -711,9 +711,7 @@ __device__ __forceinline__ bool bnd_unit(BndUnitSmem<D, IN>& sm, const float* s_
                     gb + unit * kChunk, 1);
   if constexpr (use_tc<D, IN>()) {
     constexpr int SC = D / kWalkSlices;
-    bnd_prep<D, IN>(sm.prep, sm.AT);
-    TcCtx cx;
-    tc_setup(cx, &sm.mbar, &sm.tmem);
+    // The state's loads are issued before the prep, which does not need them.
     const int w = threadIdx.x >> 5, row = 32 * (w & 3) + (threadIdx.x & 31);
     const size_t off = unit * DD + (size_t)row * D + SC * (w >> 2);
     float s[SC];
@@ -725,6 +723,9 @@ __device__ __forceinline__ bool bnd_unit(BndUnitSmem<D, IN>& sm, const float* s_
       s[c + 2] = x.z;
       s[c + 3] = x.w;
     }
+    bnd_prep<D, IN>(sm.prep, sm.AT);
+    TcCtx cx;
+    tc_setup(cx, &sm.mbar, &sm.tmem);
     const int st =
         tc_walk_step<kWalkSlices>(s, sm.prep.head, sm.prep.K[0], sm.V[0], cx, TcNoHooks{});
     if (st != kStepDone) {
