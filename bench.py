@@ -635,7 +635,9 @@ def run_train_part(gdn, W, dev, rank, world, args, flush, peaks):
                              "traffic": ncu_traffic("bwd_chunk_products"),
                              "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x sm_max_mhz "
                                             "(nominal)"},
-            "gpu_launches_per_step": 4 + 3,
+            # forward: chunk table, prep, walk, fill; backward on the forward's
+            # first pass: adjoint prep, reverse walk, W solve + u, chunk products
+            "gpu_launches_per_step": 4 + 4,
             "l2": "flushed (256 MiB write) before every timed step",
             "pages_h100_ms": PAGES_H100["trainer_fwd_bwd_ms"]}
 
@@ -689,7 +691,7 @@ def run_pik_part(gdn, dev, rank, world, args, flush, peaks):
                          "peak_source": f"measured cuBLAS bf16 burst ({peaks['source']})"},
             "cublas_bf16_ms": round(ms_cublas, 4),
             "cublas_bf16_tflops": round(2.0 * M * N * K / (ms_cublas / 1e3) / 1e12, 1),
-            "gpu_launches_per_call": 2,
+            "gpu_launches_per_call": 1,  # k_pik_gemm (one rank: no combine)
             "l2": "flushed (256 MiB write) before every timed call"}
 
 
