@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(kTableThreads)
   __shared__ long long part[64 + kTableThreads];
   __shared__ int bucket[kTableThreads];
   __shared__ int bad;
+  pdl_trigger();
   const int tid = threadIdx.x;
   if (tid == 0) bad = (cu[0] != 0 || (int64_t)cu[N] != T) ? 1 : 0;
   __syncthreads();
@@ -176,6 +177,8 @@ __global__ void __launch_bounds__(kBndThreads, prep_at_on_keys<D, IN>() ? 4 : 3)
   PrepKernelSmem<D, IN>& ks = *reinterpret_cast<PrepKernelSmem<D, IN>*>(smem_raw);
   PrepSmem<D, IN>& sm = ks.prep;
   const int c = blockIdx.x, h = blockIdx.y;
+  pdl_wait();
+  pdl_trigger();
   if (hdr[kHdrValid] != 1 || c >= hdr[kHdrChunks]) return;
   const int n = chunk_seq[c];
   const int ci = c - chunk_off[n];
@@ -248,6 +251,8 @@ __global__ void __launch_bounds__(walk_threads<D>(), 1)
   // One block per (sequence, head), sequences in the chunk table's order
   // (most chunks first).
   const int t = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (hdr[kHdrValid] != 1) return;
   const int n = seq_order[blockIdx.x / H], h = blockIdx.x % H;
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
@@ -373,6 +378,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
   // One block per (sequence, head), sequences in the chunk table's order
   // (most chunks first).
   const int t = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (hdr[kHdrValid] != 1) return;
   const int n = seq_order[blockIdx.x / H], h = blockIdx.x % H;
   const int w = t >> 5, row = 32 * (w & 3) + (t & 31), col0 = SC * (w >> 2);
@@ -465,6 +472,7 @@ __global__ void __launch_bounds__(kFillThreads, 3)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   FillSmem<D, IN>& sm = *reinterpret_cast<FillSmem<D, IN>*>(smem_raw);
   __shared__ int sh_item;
+  pdl_wait();
   if (hdr[kHdrValid] != 1) return;
   const int n_items = hdr[kHdrChunks] * H;
   const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * RT;
@@ -538,6 +546,7 @@ __global__ void __launch_bounds__(kFillThreads, 3)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Fill128Smem& sm = *reinterpret_cast<Fill128Smem*>(smem_raw);
   __shared__ int sh_item;
+  pdl_wait();
   if (hdr[kHdrValid] != 1) return;
   const int n_items = hdr[kHdrChunks] * H;
   const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * 4, sg = quad_sigma(l);
@@ -788,6 +797,7 @@ __global__ void __launch_bounds__(kDecThreads)
                OUT* __restrict__ o) {
   constexpr int RT = D / 32, M4 = D / 16;
   __shared__ int sh_pos, sh_slot;
+  pdl_trigger();  // the resync may be scheduled; it waits for this grid
   const int b = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * RT;
   if (tid == 0) {
@@ -861,6 +871,7 @@ __global__ void __launch_bounds__(unit_threads<D, IN>())
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   BndUnitSmem<D, IN>& sm = *reinterpret_cast<BndUnitSmem<D, IN>*>(smem_raw);
   __shared__ int sh_j;
+  pdl_wait();  // the step kernel's list and buffers
   const int count = min(resync[kResyncCount], n_slots * H);
   for (;;) {
     if (threadIdx.x == 0) sh_j = atomicAdd(&resync[kResyncNext], 1);
@@ -939,6 +950,25 @@ static cudaError_t set_smem(KernelT kern, size_t bytes) {
     if (e_ != cudaSuccess) return e_; \
   } while (0)
 
+// Launches kern as the programmatic dependent of the previous kernel on st:
+// its blocks may be scheduled while that kernel's last blocks run, and they
+// wait (pdl_wait, first thing) until it has completed.
+template <class... KArgs, class... Args>
+static cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // Persistent grid size of a kernel: resident blocks per SM x SMs.
 template <class KernelT>
 static cudaError_t persistent_grid(KernelT kern, int threads, size_t smem, int* grid) {
@@ -991,30 +1021,33 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   const dim3 gchunks((unsigned)L.max_chunks, (unsigned)a.H);
   GDN_TRY(mark(1));
   {
+    // prep, walk and fill are programmatic dependents of the kernel before
+    // them (each waits for it in pdl_wait before touching memory)
     auto kern = k_prep<D, IN>;
     const size_t sm = sizeof(PrepKernelSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
-    kern<<<gchunks, kBndThreads, sm, st>>>(k, v, a.beta, a.g, a.cu_seqlens, a.H, hdr, chunk_off,
-                                           chunk_seq, packs, 0);
-    GDN_TRY(cudaGetLastError());
+    GDN_TRY(launch_dependent(kern, gchunks, dim3(kBndThreads), sm, st, k, v, a.beta, a.g,
+                             a.cu_seqlens, a.H, (const int32_t*)hdr, (const int32_t*)chunk_off,
+                             (const int32_t*)chunk_seq, packs, 0));
   }
   GDN_TRY(mark(2));
+  const dim3 gunits((unsigned)((size_t)a.n_seqs * a.H));
   if constexpr (use_tc<D, IN>()) {
     auto kern = k_walk_tc<D, IN>;
     const size_t sm = sizeof(WalkTcSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
-    kern<<<(unsigned)((size_t)a.n_seqs * a.H), kWalkThreads, sm, st>>>(
-        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, seq_order, packs, bstate, a.s_run_final, a.s_run_scale,
-        a.s_bnd_final);
-    GDN_TRY(cudaGetLastError());
+    GDN_TRY(launch_dependent(kern, gunits, dim3(kWalkThreads), sm, st, a.cu_seqlens, a.H, a.h0,
+                             hdr, (const int32_t*)chunk_off, (const int32_t*)seq_order,
+                             (const char*)packs, bstate, a.s_run_final, a.s_run_scale,
+                             a.s_bnd_final));
   } else {
     auto kern = k_walk<D, IN>;
     const size_t sm = sizeof(WalkSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
-    kern<<<(unsigned)((size_t)a.n_seqs * a.H), walk_threads<D>(), sm, st>>>(
-        a.cu_seqlens, a.H, a.h0, hdr, chunk_off, seq_order, packs, bstate, a.s_run_final, a.s_run_scale,
-        a.s_bnd_final);
-    GDN_TRY(cudaGetLastError());
+    GDN_TRY(launch_dependent(kern, gunits, dim3(walk_threads<D>()), sm, st, a.cu_seqlens, a.H,
+                             a.h0, hdr, (const int32_t*)chunk_off, (const int32_t*)seq_order,
+                             (const char*)packs, bstate, a.s_run_final, a.s_run_scale,
+                             a.s_bnd_final));
   }
   GDN_TRY(mark(3));
   if (!a.pass1_only) {
@@ -1025,10 +1058,11 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     GDN_TRY(persistent_grid(kern, kFillThreads, sm, &grid));
     const int64_t items = L.max_chunks * a.H;
     if ((int64_t)grid > items) grid = (int)items;
-    kern<<<grid, kFillThreads, sm, st>>>(q, k, v, a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
-                                         chunk_off, chunk_seq, bstate, static_cast<OUT*>(a.o),
-                                         a.s_run_final, a.s_run_scale);
-    GDN_TRY(cudaGetLastError());
+    GDN_TRY(launch_dependent(kern, dim3((unsigned)grid), dim3(kFillThreads), sm, st, q, k, v,
+                             a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
+                             (const int32_t*)chunk_off, (const int32_t*)chunk_seq,
+                             (const float*)bstate, static_cast<OUT*>(a.o), a.s_run_final,
+                             a.s_run_scale));
   }
   return mark(4);
 }
@@ -1106,10 +1140,10 @@ static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
   GDN_TRY(set_smem(kern, sm));
   int grid = 0;
   GDN_TRY(persistent_grid(kern, unit_threads<D, IN>(), sm, &grid));
-  kern<<<grid, unit_threads<D, IN>(), sm, st>>>(
-      a.H, a.s_bnd, static_cast<const IN*>(a.buf_k), static_cast<const IN*>(a.buf_v), a.buf_beta,
-      a.buf_g, a.resync, a.n_slots, a.error);
-  return cudaGetLastError();
+  return launch_dependent(kern, dim3((unsigned)grid), dim3(unit_threads<D, IN>()), sm, st, a.H,
+                          a.s_bnd, static_cast<const IN*>(a.buf_k),
+                          static_cast<const IN*>(a.buf_v), (const float*)a.buf_beta,
+                          (const float*)a.buf_g, a.resync, a.n_slots, a.error);
 }
 
 template <int D, class IN>

@@ -53,6 +53,17 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
 }
+// Programmatic dependent launch.  pdl_wait: a kernel launched as the
+// dependent of the previous kernel on its stream waits here until that grid
+// has completed and its writes are visible (a no-op for an ordinary launch);
+// every dependent kernel calls it before it touches global memory.
+// pdl_trigger: lets the dependent grid be scheduled once every block of this
+// grid has passed here (it still waits for this grid's completion).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // Asynchronous prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes));
