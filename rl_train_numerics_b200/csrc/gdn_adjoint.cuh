@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kBndThreads, 3)
   static_assert(sizeof(PackHead<D, bf16>) >= kAdjNT * PL * sizeof(bf16), "Tb terms fit the head");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   AdjPrepSmem<D>& sm = *reinterpret_cast<AdjPrepSmem<D>*>(smem_raw);
+  pdl_trigger();  // the reverse walk may be scheduled; it waits for this grid
   if (hdr[kHdrValid] != 1) return;
   const int c = blockIdx.x, h = blockIdx.y;
   if (c >= hdr[kHdrChunks]) return;
@@ -467,6 +468,8 @@ __global__ void __launch_bounds__(kAdjWalkThreads, 1)
                 "bulk copies of 16-byte pieces into matching layouts");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   AdjWalkSmem<D>& sm = *reinterpret_cast<AdjWalkSmem<D>*>(smem_raw);
+  pdl_wait();  // the adjoint prep's packs
+  pdl_trigger();
   if (hdr[kHdrValid] != 1) return;
   // Blocks go out sequence by sequence, most chunks first (the chunk table's
   // order), so that the longest serial chains start in the first wave.

@@ -810,6 +810,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr int NT8 = D / 16;  // n8 tiles of a warp's C x D columns (D / 2 of them)
   extern __shared__ __align__(16) unsigned char smem_raw[];
   GemmTcSmem<D>& sm = *reinterpret_cast<GemmTcSmem<D>*>(smem_raw);
+  pdl_wait();  // w and u
   if (hdr[kHdrValid] != 1) return;
   const int c = blockIdx.x, h = blockIdx.y;
   if (c >= hdr[kHdrChunks]) return;
@@ -1310,6 +1311,8 @@ __global__ void __launch_bounds__(kUThreads, 2)
              float* __restrict__ wbuf, float* __restrict__ d_v, float* __restrict__ ubuf) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   BwdWUSmem<D>& sm = *reinterpret_cast<BwdWUSmem<D>*>(smem_raw);
+  pdl_wait();  // the reverse walk's Ydv and adjoints
+  pdl_trigger();
   if (hdr[kHdrValid] != 1) return;
   const int c = blockIdx.x >> 1, h = blockIdx.y;
   if (c >= hdr[kHdrChunks]) return;
@@ -1374,20 +1377,22 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
       const size_t sm = sizeof(AdjWalkSmem<D>);
       GDN_BWD_TRY(bwd_set_smem(kern, sm));
       const int32_t* seq_order = reinterpret_cast<const int32_t*>(ws + L.fwd.seq_order);
-      kern<<<(unsigned)((size_t)f.n_seqs * f.H * (D / kAdjWalkRows)), kAdjWalkThreads, sm,
-             st>>>(f.cu_seqlens, f.H, hdr_w, chunk_off, seq_order, apack,
-                                           a.ds_final, mu_end, ydv, a.d_h0);
-      GDN_BWD_TRY(cudaGetLastError());
+      // walk, W solve + u and the products are programmatic dependents of
+      // the kernel before them (each waits for it first thing)
+      GDN_BWD_TRY(launch_dependent(
+          kern, dim3((unsigned)((size_t)f.n_seqs * f.H * (D / kAdjWalkRows))),
+          dim3(kAdjWalkThreads), sm, st, f.cu_seqlens, f.H, hdr_w, chunk_off, seq_order,
+          (const char*)apack, a.ds_final, mu_end, ydv, a.d_h0));
     }
     GDN_BWD_TRY(mark(2));
     {  // the W solve and u (dbeta and dg come with dq and dk)
       auto kern = k_bwd_wu<D>;
       const size_t sm = sizeof(BwdWUSmem<D>);
       GDN_BWD_TRY(bwd_set_smem(kern, sm));
-      kern<<<dim3(2 * (unsigned)L.fwd.max_chunks, (unsigned)f.H), kUThreads, sm, st>>>(
-          v, f.beta, f.g, f.cu_seqlens, f.H, f.scale, hdr, chunk_off, chunk_seq, bstate, apack,
-          ydv, wbuf, a.d_v, ubuf);
-      GDN_BWD_TRY(cudaGetLastError());
+      GDN_BWD_TRY(launch_dependent(kern, dim3(2 * (unsigned)L.fwd.max_chunks, (unsigned)f.H),
+                                   dim3(kUThreads), sm, st, v, f.beta, f.g, f.cu_seqlens, f.H,
+                                   f.scale, hdr, chunk_off, chunk_seq, bstate,
+                                   (const char*)apack, (const float*)ydv, wbuf, a.d_v, ubuf));
     }
   } else {
     auto kern = k_bwd_scan<D, IN>;
@@ -1412,9 +1417,10 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
       auto kern = k_bwd_gemm_tc<D>;
       const size_t sm = sizeof(GemmTcSmem<D>);
       GDN_BWD_TRY(bwd_set_smem(kern, sm));
-      kern<<<gchunks, kGemmThreads, sm, st>>>(q, k, f.beta, f.g, d_o, f.cu_seqlens, f.H, f.scale,
-                                              hdr, chunk_off, chunk_seq, bstate, mu_end, wbuf,
-                                              ubuf, v, a.d_q, a.d_k, a.d_beta, a.d_g);
+      GDN_BWD_TRY(launch_dependent(kern, gchunks, dim3(kGemmThreads), sm, st, q, k, f.beta, f.g,
+                                   d_o, f.cu_seqlens, f.H, f.scale, hdr, chunk_off, chunk_seq,
+                                   bstate, (const float*)mu_end, (const float*)wbuf,
+                                   (const float*)ubuf, v, a.d_q, a.d_k, a.d_beta, a.d_g));
     } else {  // fp32 inputs: fp32 fused multiply-adds (their tighter bound)
       auto kern = k_bwd_gemm<D, IN>;
       const size_t sm = sizeof(GemmSmem<D, IN>);

@@ -950,25 +950,6 @@ static cudaError_t set_smem(KernelT kern, size_t bytes) {
     if (e_ != cudaSuccess) return e_; \
   } while (0)
 
-// Launches kern as the programmatic dependent of the previous kernel on st:
-// its blocks may be scheduled while that kernel's last blocks run, and they
-// wait (pdl_wait, first thing) until it has completed.
-template <class... KArgs, class... Args>
-static cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                                    cudaStream_t st, Args... args) {
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, args...);
-}
-
 // Persistent grid size of a kernel: resident blocks per SM x SMs.
 template <class KernelT>
 static cudaError_t persistent_grid(KernelT kern, int threads, size_t smem, int* grid) {
