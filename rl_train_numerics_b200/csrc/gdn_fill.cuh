@@ -13,6 +13,7 @@ constexpr int kHdrError = 0;     // device error word (GDN_DEVERR_* bits)
 constexpr int kHdrChunks = 1;    // number of chunks of this call
 constexpr int kHdrValid = 2;     // 1 when this call's chunk table is valid
 constexpr int kHdrFillNext = 3;  // work counter of k_fill
+constexpr int kHdrFill0Next = 4; // work counter of the fill's first chunks (k_fill128)
 
 constexpr int kFillThreads = 128;
 
@@ -145,6 +146,21 @@ __device__ __forceinline__ void slice4_load_bst(Slice<4, M4>& S, const float* ro
     for (int m = 0; m < M4; m++) {
       const int r = r0 + (i ^ sg);
       const float4 x = ld4(rows + (size_t)r * ld + bst_col(r, group_col(l, m)));
+      S.s[i][m][0] = f2(x.x, x.y);
+      S.s[i][m][1] = f2(x.z, x.w);
+    }
+}
+
+// The same from a row-major D x D state (h0), or zeros when rows is null.
+template <int M4>
+__device__ __forceinline__ void slice4_load_plain(Slice<4, M4>& S, const float* rows, int ld,
+                                                  int r0, int sg, int l) {
+#pragma unroll
+  for (int i = 0; i < 4; i++)
+#pragma unroll
+    for (int m = 0; m < M4; m++) {
+      const float4 x = rows ? ld4(rows + (size_t)(r0 + (i ^ sg)) * ld + group_col(l, m))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
       S.s[i][m][0] = f2(x.x, x.y);
       S.s[i][m][1] = f2(x.z, x.w);
     }

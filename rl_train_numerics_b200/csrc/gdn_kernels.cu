@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(kTableThreads)
     if (run > max_chunks) bad = 1;
     hdr[kHdrChunks] = bad ? 0 : (int32_t)run;
     hdr[kHdrFillNext] = 0;
+    hdr[kHdrFill0Next] = 0;
     if (!bad) chunk_off[N] = (int32_t)run;
   }
   __syncthreads();
@@ -467,7 +468,10 @@ __global__ void __launch_bounds__(kFillThreads, 3)
            const int32_t* __restrict__ cu, int H, float scale, int32_t* __restrict__ hdr,
            const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
            const float* __restrict__ bstate, OUT* __restrict__ o,
-           float* __restrict__ s_run_final, float* __restrict__ s_run_scale) {
+           float* __restrict__ s_run_final, float* __restrict__ s_run_scale, int n_seqs,
+           const float* __restrict__ h0) {
+  (void)n_seqs;
+  (void)h0;
   constexpr int RT = D / 32, M4 = D / 16;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   FillSmem<D, IN>& sm = *reinterpret_cast<FillSmem<D, IN>*>(smem_raw);
@@ -541,24 +545,62 @@ __global__ void __launch_bounds__(kFillThreads, 3)
               int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
               const int32_t* __restrict__ chunk_seq, const float* __restrict__ bstate,
               OUT* __restrict__ o, float* __restrict__ s_run_final,
-              float* __restrict__ s_run_scale) {
+              float* __restrict__ s_run_scale, int n_seqs, const float* __restrict__ h0) {
   constexpr int D = 128, M4 = D / 16;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Fill128Smem& sm = *reinterpret_cast<Fill128Smem*>(smem_raw);
   __shared__ int sh_item;
-  pdl_wait();
-  if (hdr[kHdrValid] != 1) return;
+  // Two phases.  Phase 0, before waiting for the boundary walk: the first
+  // chunk of every sequence, whose entry state is h0 (or zero), not a walk
+  // result, so that these items run on the SMs the walk leaves idle (the
+  // walk only writes boundary states, the bound final states and the pack
+  // reads, none of which a first chunk touches).  Phase 1, after the wait:
+  // every other chunk.  The chunk table (read in both) completed before the
+  // walk started.
+  if (hdr[kHdrValid] != 1) {
+    pdl_wait();
+    return;
+  }
   const int n_items = hdr[kHdrChunks] * H;
   const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * 4, sg = quad_sigma(l);
   const int my_row = r0 + sg;
   const size_t DD = (size_t)D * D;
 
   for (int c = tid; c < D; c += kFillThreads) sm.k[kChunk][c] = 0.f;
-  if (tid == 0) sh_item = atomicAdd(&hdr[kHdrFillNext], 1);
-  __syncthreads();
-  int item = sh_item;
-  while (item < n_items) {
-    const FillItem cur = fill_item(item, H, cu, chunk_off, chunk_seq);
+  int phase = 0, limit = n_seqs * H;
+  int32_t* counter = &hdr[kHdrFill0Next];
+  auto claim = [&]() {
+    __syncthreads();
+    if (tid == 0) sh_item = atomicAdd(counter, 1);
+    __syncthreads();
+    return sh_item;
+  };
+  int item = claim();
+  for (;;) {
+    if (item >= limit) {
+      if (phase == 1) break;
+      phase = 1;
+      pdl_wait();  // the boundary walk's states
+      counter = &hdr[kHdrFillNext];
+      limit = n_items;
+      item = claim();
+      continue;
+    }
+    FillItem cur;
+    if (phase == 0) {
+      const int n = item / H, hh = item - n * H;
+      if (chunk_off[n] == chunk_off[n + 1]) {  // empty sequence
+        item = claim();
+        continue;
+      }
+      cur = fill_item(chunk_off[n] * H + hh, H, cu, chunk_off, chunk_seq);
+    } else {
+      cur = fill_item(item, H, cu, chunk_off, chunk_seq);
+      if (cur.ci == 0) {  // done in phase 0
+        item = claim();
+        continue;
+      }
+    }
     const size_t tb = (size_t)cur.t0 * H + cur.h;
     // Keys (widened), queries and values of the item (rows past its length
     // are zero): 2 x 8 float4 groups of each per thread, loads issued in
@@ -624,11 +666,15 @@ __global__ void __launch_bounds__(kFillThreads, 3)
       }
     }
     Slice<4, M4> S;
-    slice4_load_bst<M4>(S, bstate + ((size_t)cur.c * H + cur.h) * DD, D, r0, sg, l);
-    if (tid == 0) sh_item = atomicAdd(&hdr[kHdrFillNext], 1);
+    if (phase == 0)
+      slice4_load_plain<M4>(S, h0 ? h0 + ((size_t)cur.n * H + cur.h) * DD : nullptr, D, r0, sg,
+                            l);
+    else
+      slice4_load_bst<M4>(S, bstate + ((size_t)cur.c * H + cur.h) * DD, D, r0, sg, l);
+    if (tid == 0) sh_item = atomicAdd(counter, 1);
     __syncthreads();
     const int next = sh_item;
-    if (next < n_items)
+    if (phase == 1 && next < n_items)
       fill_prefetch<D, __nv_bfloat16>(fill_item(next, H, cu, chunk_off, chunk_seq), bstate, q,
                                       k, v, H);
 
@@ -1043,7 +1089,7 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
                              a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
                              (const int32_t*)chunk_off, (const int32_t*)chunk_seq,
                              (const float*)bstate, static_cast<OUT*>(a.o), a.s_run_final,
-                             a.s_run_scale));
+                             a.s_run_scale, a.n_seqs, a.h0));
   }
   return mark(4);
 }
