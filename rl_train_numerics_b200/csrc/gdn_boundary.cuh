@@ -85,7 +85,7 @@ struct PackHead {
   __nv_bfloat16 TbT[NW][kChunk * kChunk];
   __nv_bfloat16 TvT[NW][kChunk * kChunk];
   float dvec[kChunk];
-  float gamma[4];  // [0] = exp(G_C)
+  float gamma[32];  // [0] = exp(G_C), the rest zero (the head is whole 128-byte lines)
 };
 
 // Keys and values of one chunk as bf16 term planes, core-matrix layout with
@@ -454,10 +454,7 @@ __device__ void bnd_prep(PrepSmem<D, IN>& sm, PrepAT& AT, const AfterP& after_p 
     sm.bg[i] = __fmul_rn(sm.beta[i], expf(__double2float_rn(sm.G[i])));
     sm.head.dvec[i] = expf(__double2float_rn(sm.G[kChunk - 1] - sm.G[i]));
   }
-  if (tid == 0) {
-    sm.head.gamma[0] = expf(__double2float_rn(sm.G[kChunk - 1]));
-    sm.head.gamma[1] = sm.head.gamma[2] = sm.head.gamma[3] = 0.f;
-  }
+  if (tid < 32) sm.head.gamma[tid] = tid == 0 ? expf(__double2float_rn(sm.G[kChunk - 1])) : 0.f;
   __syncthreads();
 
   // T = (I + A)^{-1} (unit lower triangular) by blocked forward substitution

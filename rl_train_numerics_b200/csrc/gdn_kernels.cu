@@ -18,10 +18,14 @@
 //   k_resync        persistent blocks: the chunk boundary of listed units
 //   k_bnd           one block per (row, head): gdn_chunk_boundary
 //   k_handoff       prefill -> decode state
+#include <cuda.h>
+#include <string.h>
+
 #include "gdn_boundary.cuh"
 #include "gdn_fill.cuh"
 #include "gdn_layout.h"
 #include "gdn_native.cuh"
+#include "gdn_tmap.h"
 
 namespace gdn {
 
@@ -190,8 +194,12 @@ __global__ void __launch_bounds__(kBndThreads, prep_at_on_keys<D, IN>() ? 4 : 3)
   if (rows < kChunk && !all_chunks) return;
   const int64_t t0 = (int64_t)cu[n] + (int64_t)ci * kChunk;
   const size_t tok = (size_t)t0 * H + h;
+  // The tcgen05 walk copies the value planes from the inputs itself (a
+  // tensor-map copy), so for it the pack carries the head and the keys; the
+  // chunked layout's output kernel (all_chunks) reads the values from the pack.
+  const bool vp = !use_tc<D, IN>() || all_chunks;
   PlaneRows<D, IN, kBndThreads> vrows;  // the chunk's values, in flight during the prep
-  vrows.load(v + tok * D, (size_t)H * D, rows);
+  if (vp) vrows.load(v + tok * D, (size_t)H * D, rows);
   prep_stage<D, IN>(sm, k + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H, rows);
   WalkPack<D, IN>& pk =
       *reinterpret_cast<WalkPack<D, IN>*>(packs + ((size_t)c * H + h) * pack_size<D, IN>());
@@ -221,7 +229,7 @@ __global__ void __launch_bounds__(kBndThreads, prep_at_on_keys<D, IN>() ? 4 : 3)
     bulk_store(&pk.head, smem_u32(&sm.head), kOut);
     bulk_commit();
   }
-  vrows.store(pk.kv.V);
+  if (vp) vrows.store(pk.kv.V);
   if (threadIdx.x == 0) bulk_wait_read();  // shared memory must outlive the copy's reads
 }
 
@@ -301,13 +309,64 @@ __global__ void __launch_bounds__(walk_threads<D>(), 1)
 
 // The walk on tcgen05 (d = 128, bf16): one block of 512 threads per
 // (sequence, head); warp w holds columns 32 (w / 4) .. + 31 of the rows of its
-// tensor-memory lane quadrant.  Chunk c + 1's pack is copied in (one bulk
-// copy) and chunk c + 2's prefetched into L2 while chunk c's products run.
+// tensor-memory lane quadrant.  Chunk c + 1's inputs are copied in (its pack
+// head and key planes by one bulk copy, its value planes by one tensor-map
+// copy from the input) and chunk c + 2's pack prefetched into L2 while chunk
+// c's products run.
 // Each boundary state goes to the workspace through a shared-memory staging
 // copy (permuted rows, conflict-free) and one bulk asynchronous store, issued
 // with the chunk's first products.
 constexpr int kWalkSlices = 4;
 constexpr int kWalkThreads = kTcRows * kWalkSlices;
+
+// Value planes of one chunk and head straight from a [T][H][D] bf16 input
+// (D = 128): a 4-D map over (8 channels, T tokens, D / 8 channel groups,
+// H heads) whose box of 8 x 64 x 16 x 1 elements lands in shared memory as
+// [group][token][8], the planes' core-matrix layout.  False if the encoder
+// is missing or refuses the map.
+static bool make_plane_map(CUtensorMap* map, const void* base, int64_t T, int H) {
+  constexpr int D = 128;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {8, (cuuint64_t)T, D / 8, (cuuint64_t)H};
+  const cuuint64_t strides[3] = {(cuuint64_t)H * D * 2, 16, D * 2};  // bytes, dims 1..3
+  const cuuint32_t box[4] = {8, (cuuint32_t)kChunk, D / 8, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Bytes of a walk pack ahead of its value planes (the head and the keys).
+template <int D, class IN>
+constexpr uint32_t pack_bytes_before_v() {
+  using WP = WalkPack<D, IN>;
+  return (uint32_t)offsetof(WP, kv.V);
+}
+
+// The tcgen05 walk's value map; zeroed (never read) when no sequence holds a
+// full chunk.  A refused map is an error: there is no other route.
+static cudaError_t value_map(CUtensorMap* mv, const void* v, int64_t T, int H) {
+  memset(mv, 0, sizeof(*mv));
+  if (T < kChunk) return cudaSuccess;
+  return make_plane_map(mv, v, T, H) ? cudaSuccess : cudaErrorNotSupported;
+}
+
+// The tcgen05 walk's inputs of one full chunk into dst: the pack head and key
+// planes by one bulk copy, the value planes by one tensor-map copy (tok0: the
+// chunk's first token), all counted on the mbarrier at bar.  One thread.
+template <int D, class IN>
+__device__ __forceinline__ void pack_fetch_tc(WalkPack<D, IN>& dst, const char* pack,
+                                              const CUtensorMap* mv, int tok0, int h,
+                                              uint64_t* bar) {
+  using WP = WalkPack<D, IN>;
+  static_assert(sizeof(WP) % 128 == 0 && pack_bytes_before_v<D, IN>() % 128 == 0,
+                "tensor-map destinations are 128-byte aligned");
+  const uint32_t mb = smem_u32(bar);
+  mbar_expect_tx(mb, (uint32_t)sizeof(WalkPack<D, IN>));
+  bulk_load(smem_u32(&dst.head), pack, pack_bytes_before_v<D, IN>(), mb);
+  tma_load_4d(smem_u32(dst.kv.V[0]), mv, 0, tok0, 0, h, mb);
+}
 
 template <int D, class IN>
 struct WalkTcSmem {
@@ -343,14 +402,17 @@ struct WalkHooks {
   const char* ahead; // pack of chunk c + 2, or null
   float* dst;        // boundary state of chunk c in the workspace
   int row, col0;
+  const CUtensorMap* mv;  // value planes
+  int tok_next, h;        // chunk c + 1's first token; the head
   __device__ bool inputs_ready() const {
     if (threadIdx.x == 0) bulk_wait_read();
     return pack_wait(sm->ld_bar, c);
   }
   __device__ void after_first() const {
     if ((threadIdx.x & 31) != 0) return;
-    if (next) pack_fetch<D, IN>(sm->buf[(c + 1) & 1], next, &sm->ld_bar[(c + 1) & 1]);
-    if (ahead) prefetch_l2(ahead, (uint32_t)sizeof(WalkPack<D, IN>));
+    if (next) pack_fetch_tc<D, IN>(sm->buf[(c + 1) & 1], next, mv, tok_next, h,
+                                   &sm->ld_bar[(c + 1) & 1]);
+    if (ahead) prefetch_l2(ahead, pack_bytes_before_v<D, IN>());
   }
   __device__ void during_first(const float* s) const {
     stage_slice<D, D / kWalkSlices>(sm->stage, s, row, col0);
@@ -370,7 +432,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
               const int32_t* __restrict__ seq_order, const char* __restrict__ packs,
               float* __restrict__ bstate,
               float* __restrict__ s_run_final, float* __restrict__ s_run_scale,
-              float* __restrict__ s_bnd_final) {
+              float* __restrict__ s_bnd_final, const __grid_constant__ CUtensorMap map_v) {
   static_assert(use_tc<D, IN>(), "tcgen05 walk: d = 128, bf16 inputs");
   constexpr int SC = D / kWalkSlices;
   constexpr size_t PB = pack_size<D, IN>();
@@ -392,8 +454,10 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
   pack_bars_init(sm.ld_bar);
   TcCtx cx;
   tc_setup(cx, &sm.mbar, &sm.tmem);
-  if (t == 0 && nf > 0) pack_fetch<D, IN>(sm.buf[0], pack(0), &sm.ld_bar[0]);
-  if (t == 0 && nf > 1) prefetch_l2(pack(1), (uint32_t)sizeof(WalkPack<D, IN>));
+  const int tok0 = cu[n];
+  if (t == 0 && nf > 0)
+    pack_fetch_tc<D, IN>(sm.buf[0], pack(0), &map_v, tok0, h, &sm.ld_bar[0]);
+  if (t == 0 && nf > 1) prefetch_l2(pack(1), pack_bytes_before_v<D, IN>());
   float s[SC];
   if (h0) {
     const float* src = h0 + ((size_t)n * H + h) * DD + (size_t)row * D + col0;
@@ -415,7 +479,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     const size_t unit = (size_t)(base + c) * H + h;
     const WalkHooks<D, IN> hooks{&sm, c, c + 1 < nf ? pack(c + 1) : nullptr,
                                  c + 2 < nf ? pack(c + 2) : nullptr, bstate + unit * DD, row,
-                                 col0};
+                                 col0, &map_v, tok0 + (int)(c + 1) * kChunk, h};
     const WalkPack<D, IN>& b = sm.buf[c & 1];
     status = tc_walk_step<kWalkSlices>(s, b.head, b.kv.K[0], b.kv.V[0], cx, hooks);
     if (status != kStepDone) break;
@@ -1063,10 +1127,12 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     auto kern = k_walk_tc<D, IN>;
     const size_t sm = sizeof(WalkTcSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
+    CUtensorMap mv;
+    GDN_TRY(value_map(&mv, v, a.T, a.H));
     GDN_TRY(launch_dependent(kern, gunits, dim3(kWalkThreads), sm, st, a.cu_seqlens, a.H, a.h0,
                              hdr, (const int32_t*)chunk_off, (const int32_t*)seq_order,
                              (const char*)packs, bstate, a.s_run_final, a.s_run_scale,
-                             a.s_bnd_final));
+                             a.s_bnd_final, mv));
   } else {
     auto kern = k_walk<D, IN>;
     const size_t sm = sizeof(WalkSmem<D, IN>);
@@ -1131,9 +1197,11 @@ static cudaError_t native_impl(const FwdArgs& a, cudaStream_t st) {
     auto kern = k_walk_tc<D, IN>;
     const size_t sm = sizeof(WalkTcSmem<D, IN>);
     GDN_TRY(set_smem(kern, sm));
+    CUtensorMap mv;
+    GDN_TRY(value_map(&mv, a.v, a.T, a.H));
     kern<<<(unsigned)((size_t)a.n_seqs * a.H), kWalkThreads, sm, st>>>(
         a.cu_seqlens, a.H, a.h0, hdr, chunk_off, seq_order, packs, bstate, a.s_run_final, nullptr,
-        a.s_bnd_final);
+        a.s_bnd_final, mv);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(3));

@@ -55,6 +55,7 @@
 
 #include "../../include/gdn_pik.h"
 #include "gdn_mma.cuh"
+#include "gdn_tmap.h"
 #include "gdn_umma.cuh"
 
 namespace gdn {
@@ -429,26 +430,6 @@ int validate(int64_t M, int64_t N, int64_t K, int L, int R) {
   if (((M + kPikBM - 1) / kPikBM) * ((N + kPikBN - 1) / kPikBN) * R >= 0x7fffffff)
     return GDN_ERR_UNSUPPORTED;
   return GDN_OK;
-}
-
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
-// against the driver library).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
 }
 
 // Map over a [rows, K] bf16 row-major matrix with a box of 64 K columns

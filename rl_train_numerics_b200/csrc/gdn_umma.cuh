@@ -215,6 +215,19 @@ __device__ __forceinline__ void bulk_load(uint32_t sdst, const void* gsrc, uint3
       "l"(gsrc), "r"(bytes), "r"(mbar)
       : "memory");
 }
+// Tiled tensor copy of one 4-D box from global to shared memory through the
+// tensor map at `map` (a kernel parameter), its completion counted in
+// transaction bytes on the mbarrier at `mbar`.  The innermost coordinate x
+// times the element size is a multiple of 16 bytes and the destination is
+// 128-byte aligned.  Issued by one thread, after mbar_expect_tx.
+__device__ __forceinline__ void tma_load_4d(uint32_t sdst, const void* map, int x, int y, int z,
+                                            int w, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(sdst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(mbar)
+      : "memory");
+}
 // Arrive on the mbarrier (count 1) and expect `bytes` transaction bytes.
 __device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes)
