@@ -311,8 +311,8 @@ __global__ void __launch_bounds__(walk_threads<D>(), 1)
 // (sequence, head); warp w holds columns 32 (w / 4) .. + 31 of the rows of its
 // tensor-memory lane quadrant.  Chunk c + 1's inputs are copied in (its pack
 // head and key planes by one bulk copy, its value planes by one tensor-map
-// copy from the input) and chunk c + 2's pack prefetched into L2 while chunk
-// c's products run.
+// copy from the input) from the start of chunk c's step, and chunk c + 2's
+// pack prefetched into L2 while chunk c's products run.
 // Each boundary state goes to the workspace through a shared-memory staging
 // copy (permuted rows, conflict-free) and one bulk asynchronous store, issued
 // with the chunk's first products.
@@ -389,11 +389,12 @@ __device__ __forceinline__ void stage_slice(float* stage, const float* s, int ro
 }
 
 // The walk's work around the step of chunk c (warp-0 parts by lane 0):
-// before the first barrier, wait until the previous chunk's state store has
-// read the staging buffer (thread 0) and for this chunk's pack; issue chunk
-// c + 1's pack copy and chunk c + 2's L2 prefetch with the first products;
-// stage the boundary state while they run and store it with the second
-// round.
+// before the first barrier, issue chunk c + 1's copies into the buffer chunk
+// c - 1 left (every thread is past its last read of it: the previous step
+// ended with a block barrier), wait until the previous chunk's state store
+// has read the staging buffer (thread 0) and for this chunk's inputs; issue
+// chunk c + 2's L2 prefetch with the first products; stage the boundary
+// state while they run and store it with the second round.
 template <int D, class IN>
 struct WalkHooks {
   WalkTcSmem<D, IN>* sm;
@@ -405,13 +406,15 @@ struct WalkHooks {
   const CUtensorMap* mv;  // value planes
   int tok_next, h;        // chunk c + 1's first token; the head
   __device__ bool inputs_ready() const {
-    if (threadIdx.x == 0) bulk_wait_read();
+    if (threadIdx.x == 0) {
+      if (next) pack_fetch_tc<D, IN>(sm->buf[(c + 1) & 1], next, mv, tok_next, h,
+                                     &sm->ld_bar[(c + 1) & 1]);
+      bulk_wait_read();
+    }
     return pack_wait(sm->ld_bar, c);
   }
   __device__ void after_first() const {
     if ((threadIdx.x & 31) != 0) return;
-    if (next) pack_fetch_tc<D, IN>(sm->buf[(c + 1) & 1], next, mv, tok_next, h,
-                                   &sm->ld_bar[(c + 1) & 1]);
     if (ahead) prefetch_l2(ahead, pack_bytes_before_v<D, IN>());
   }
   __device__ void during_first(const float* s) const {
@@ -485,9 +488,9 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     if (status != kStepDone) break;
   }
   if (status != kStepDone) {
-    // Pack copies possibly in flight: chunks c .. issued - 1 (the step issues
-    // chunk c + 1's copy once it is past its first barrier).
-    const int64_t issued = status == kStepNoInputs ? c + 1 : (c + 2 < nf ? c + 2 : nf);
+    // Input copies possibly in flight: chunks c .. issued - 1 (the step issues
+    // chunk c + 1's copies before its first barrier).
+    const int64_t issued = c + 2 < nf ? c + 2 : nf;
     pack_drain(sm.ld_bar, c, issued);
     if (status == kStepFailed) tc_drain(cx);
     if (t == 0) atomicOr(&hdr[kHdrError], kErrTimeout);
