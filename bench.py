@@ -413,7 +413,7 @@ def run_decode_part(gdn, W, dev, rank, world, args, peaks):
             "pages_h100_ms": PAGES_H100["decode_ms"]}
 
 
-def native_out_bytes(lens, H_, d, c=C, pack=65808):
+def native_out_bytes(lens, H_, d, c=C, pack=65920):
     """Algorithmic bytes of the chunked layout's output kernel: per (chunk, head)
     the entry state (fp32 d x d), the chunk's pack, its queries (bf16), g and
     its outputs (bf16)."""
