@@ -196,12 +196,15 @@ __device__ __forceinline__ void slice4_store_scaled(const Slice<4, M4>& S, float
 // scalars, computed once per item:
 //   t0 = (a = exp(g), beta, c before the token, c after it),
 //   t1 = (c' = a c, 1 / c' (0 when renormalising), renormalise flag, 0).
+// q and v are filled by tensor-map copies (v first holds the raw keys, which
+// are widened into k), counted on bar[0] (keys, queries) and bar[1] (values).
 struct Fill128Smem {
   float k[kChunk + 1][128];  // row kChunk stays zero: the "next key" of the last token
   __nv_bfloat16 q[kChunk][128];
   __nv_bfloat16 v[kChunk][128];
   float4 t0[kChunk];
   float4 t1[kChunk];
+  uint64_t bar[2];
 };
 
 }  // namespace gdn

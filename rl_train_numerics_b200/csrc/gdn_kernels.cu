@@ -344,6 +344,35 @@ constexpr uint32_t pack_bytes_before_v() {
   return (uint32_t)offsetof(WP, kv.V);
 }
 
+// One chunk's rows of one head from a [T][H][128] bf16 input: a 3-D map over
+// (128 channels, H heads, T tokens) whose box of 128 x 1 x 64 elements lands
+// as [token][channel] (tokens past T read as zeros).
+static bool make_row_map(CUtensorMap* map, const void* base, int64_t T, int H) {
+  constexpr int D = 128;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {D, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {D * 2, (cuuint64_t)H * D * 2};  // bytes, dims 1..2
+  const cuuint32_t box[3] = {D, 1, (cuuint32_t)kChunk};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The fill's query, key and value maps; zeroed (never read) without tokens.
+// A refused map is an error: there is no other route.
+static cudaError_t row_maps(CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv, const void* q,
+                            const void* k, const void* v, int64_t T, int H) {
+  memset(mq, 0, sizeof(*mq));
+  memset(mk, 0, sizeof(*mk));
+  memset(mv, 0, sizeof(*mv));
+  if (T < 1) return cudaSuccess;
+  const bool ok = make_row_map(mq, q, T, H) && make_row_map(mk, k, T, H) &&
+                  make_row_map(mv, v, T, H);
+  return ok ? cudaSuccess : cudaErrorNotSupported;
+}
+
 // The tcgen05 walk's value map; zeroed (never read) when no sequence holds a
 // full chunk.  A refused map is an error: there is no other route.
 static cudaError_t value_map(CUtensorMap* mv, const void* v, int64_t T, int H) {
@@ -595,14 +624,21 @@ __global__ void __launch_bounds__(kFillThreads, 3)
   }
 }
 
+// The two bf16 halves of a packed pair (the element at the lower address in
+// the low half), exactly as fp32.
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+constexpr int kFillWaitPolls = 1 << 22;
+
 // ----------------------------------------------------------------------------
 // Pass 2 at d = 128 with bf16 inputs: the same step, in the same order, with
 // the quad reductions of gdn_fill.cuh (reduce-scatter of the row sums, the
 // row's scalar work on its owning lane, all-gather of the update weight),
-// keys widened to fp32 in shared memory once per item, and the per-token
-// scale sequence (c, c' = a c, 1 / c', renormalise) computed once per item (a
-// left-to-right chain, then the reciprocals in parallel).  Bits are those of
-// k_fill.
+// keys and queries copied in by tensor map (while the item's state slice
+// loads) and the keys widened to fp32 in shared memory once per item, the
+// values copied in behind them, and the per-token scale sequence (c,
+// c' = a c, 1 / c', renormalise) computed once per item (a left-to-right
+// chain, then the reciprocals in parallel).  Bits are those of k_fill.
 // ----------------------------------------------------------------------------
 template <class OUT>
 __global__ void __launch_bounds__(kFillThreads, 3)
@@ -612,7 +648,9 @@ __global__ void __launch_bounds__(kFillThreads, 3)
               int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
               const int32_t* __restrict__ chunk_seq, const float* __restrict__ bstate,
               OUT* __restrict__ o, float* __restrict__ s_run_final,
-              float* __restrict__ s_run_scale, int n_seqs, const float* __restrict__ h0) {
+              float* __restrict__ s_run_scale, int n_seqs, const float* __restrict__ h0,
+              const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+              const __grid_constant__ CUtensorMap map_v) {
   constexpr int D = 128, M4 = D / 16;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Fill128Smem& sm = *reinterpret_cast<Fill128Smem*>(smem_raw);
@@ -634,6 +672,12 @@ __global__ void __launch_bounds__(kFillThreads, 3)
   const size_t DD = (size_t)D * D;
 
   for (int c = tid; c < D; c += kFillThreads) sm.k[kChunk][c] = 0.f;
+  if (tid == 0) {
+    mbar_init(smem_u32(&sm.bar[0]), 1);
+    mbar_init(smem_u32(&sm.bar[1]), 1);
+    fence_mbar_init();
+  }
+  uint32_t par = 0;  // phase of both barriers the next item waits for
   int phase = 0, limit = n_seqs * H;
   int32_t* counter = &hdr[kHdrFill0Next];
   auto claim = [&]() {
@@ -669,32 +713,14 @@ __global__ void __launch_bounds__(kFillThreads, 3)
       }
     }
     const size_t tb = (size_t)cur.t0 * H + cur.h;
-    // Keys (widened), queries and values of the item (rows past its length
-    // are zero): 2 x 8 float4 groups of each per thread, loads issued in
-    // batches.
-#pragma unroll
-    for (int half = 0; half < 2; half++) {
-      float4 xk[8];
-      uint2 xq[8], xv[8];
-#pragma unroll
-      for (int j = 0; j < 8; j++) {
-        const int e = tid + (half * 8 + j) * kFillThreads, r = e >> 5, c = (e & 31) * 4;
-        xk[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        xq[j] = xv[j] = make_uint2(0u, 0u);
-        if (r < cur.len) {
-          const size_t off = (tb + (size_t)r * H) * D + c;
-          xk[j] = ld4(k + off);
-          xq[j] = *reinterpret_cast<const uint2*>(q + off);
-          xv[j] = *reinterpret_cast<const uint2*>(v + off);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; j++) {
-        const int e = tid + (half * 8 + j) * kFillThreads, r = e >> 5, c = (e & 31) * 4;
-        *reinterpret_cast<float4*>(&sm.k[r][c]) = xk[j];
-        *reinterpret_cast<uint2*>(&sm.q[r][c]) = xq[j];
-        *reinterpret_cast<uint2*>(&sm.v[r][c]) = xv[j];
-      }
+    const uint32_t bar_kq = smem_u32(&sm.bar[0]), bar_v = smem_u32(&sm.bar[1]);
+    // The item's keys (raw, into the value buffer) and queries by tensor-map
+    // copies (rows past the item's length hold the next tokens or zeros and
+    // are not read), while its scalars and the state slice load.
+    if (tid == 0) {
+      mbar_expect_tx(bar_kq, 2u * kChunk * D * 2);
+      tma_load_3d(smem_u32(&sm.v[0][0]), &map_k, 0, cur.h, (int)cur.t0, bar_kq);
+      tma_load_3d(smem_u32(&sm.q[0][0]), &map_q, 0, cur.h, (int)cur.t0, bar_kq);
     }
     // Per-token scalars: a = exp(g) and beta, two tokens per thread of warps
     // 0-1 in parallel.
@@ -706,51 +732,81 @@ __global__ void __launch_bounds__(kFillThreads, 3)
       }
       sm.t0[tid] = make_float4(a, b, 0.f, 0.f);
     }
-    {
-      __syncthreads();
-      // The scale sequence: a left-to-right chain that every lane of warp 0
-      // follows (a_t read ahead from shared memory), keeping the values of
-      // its own two tokens; then each lane writes its tokens' entries.
-      if (tid < 32) {
-        float c = 1.f, my_c[2] = {1.f, 1.f}, my_cn[2] = {0.f, 0.f};
-        for (int t = 0; t < cur.len; t++) {
-          const float cn = __fmul_rn(sm.t0[t].x, c);
-          if (t == tid) { my_c[0] = c; my_cn[0] = cn; }
-          if (t == tid + 32) { my_c[1] = c; my_cn[1] = cn; }
-          c = scale_ok(cn) ? cn : 1.f;
-        }
-#pragma unroll
-        for (int j = 0; j < 2; j++) {
-          const int t = tid + 32 * j;
-          if (t < cur.len) {
-            const bool keep = scale_ok(my_cn[j]);
-            sm.t0[t].z = my_c[j];
-            sm.t0[t].w = keep ? my_cn[j] : 1.f;
-            sm.t1[t] = make_float4(my_cn[j], keep ? __frcp_rn(my_cn[j]) : 0.f,
-                                   keep ? 0.f : 1.f, 0.f);
-          }
-        }
-      }
-    }
     Slice<4, M4> S;
     if (phase == 0)
       slice4_load_plain<M4>(S, h0 ? h0 + ((size_t)cur.n * H + cur.h) * DD : nullptr, D, r0, sg,
                             l);
     else
       slice4_load_bst<M4>(S, bstate + ((size_t)cur.c * H + cur.h) * DD, D, r0, sg, l);
-    if (tid == 0) sh_item = atomicAdd(counter, 1);
-    __syncthreads();
-    const int next = sh_item;
-    if (phase == 1 && next < n_items)
-      fill_prefetch<D, __nv_bfloat16>(fill_item(next, H, cu, chunk_off, chunk_seq), bstate, q,
-                                      k, v, H);
-
+    // Keys widened to fp32; rows past the length are zero (row len is the
+    // last token's next key).
+    bool ok = mbar_wait(bar_kq, par, kFillWaitPolls);
+    if (ok) {
+#pragma unroll
+      for (int j = 0; j < kChunk * D / 8 / kFillThreads; j++) {
+        const int e = tid + j * kFillThreads, r = e >> 4, cc = (e & 15) * 8;
+        const uint4 x = *reinterpret_cast<const uint4*>(&sm.v[r][cc]);
+        float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+        if (r < cur.len) {
+          lo = make_float4(bf_lo(x.x), bf_hi(x.x), bf_lo(x.y), bf_hi(x.y));
+          hi = make_float4(bf_lo(x.z), bf_hi(x.z), bf_lo(x.w), bf_hi(x.w));
+        }
+        *reinterpret_cast<float4*>(&sm.k[r][cc]) = lo;
+        *reinterpret_cast<float4*>(&sm.k[r][cc + 4]) = hi;
+      }
+    }
+    if (__syncthreads_or(!ok)) {  // keys and queries never arrived: wait once more and stop
+      if (tid == 0) atomicOr(&hdr[kHdrError], kErrTimeout);
+      (void)mbar_wait(bar_kq, par, kFillWaitPolls);
+      return;
+    }
+    // The raw keys are read: the values go to their buffer.
+    if (tid == 0) {
+      mbar_expect_tx(bar_v, (uint32_t)kChunk * D * 2);
+      tma_load_3d(smem_u32(&sm.v[0][0]), &map_v, 0, cur.h, (int)cur.t0, bar_v);
+    }
+    // The scale sequence: a left-to-right chain that every lane of warp 0
+    // follows (a_t read ahead from shared memory), keeping the values of its
+    // own two tokens; then each lane writes its tokens' entries.
+    if (tid < 32) {
+      float c = 1.f, my_c[2] = {1.f, 1.f}, my_cn[2] = {0.f, 0.f};
+      for (int t = 0; t < cur.len; t++) {
+        const float cn = __fmul_rn(sm.t0[t].x, c);
+        if (t == tid) { my_c[0] = c; my_cn[0] = cn; }
+        if (t == tid + 32) { my_c[1] = c; my_cn[1] = cn; }
+        c = scale_ok(cn) ? cn : 1.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 2; j++) {
+        const int t = tid + 32 * j;
+        if (t < cur.len) {
+          const bool keep = scale_ok(my_cn[j]);
+          sm.t0[t].z = my_c[j];
+          sm.t0[t].w = keep ? my_cn[j] : 1.f;
+          sm.t1[t] = make_float4(my_cn[j], keep ? __frcp_rn(my_cn[j]) : 0.f,
+                                 keep ? 0.f : 1.f, 0.f);
+        }
+      }
+    }
     float p_own;
     {
       float x[4];
       slice_dot<4, M4>(S, [&](int m) { return sld4(&sm.k[0][group_col(l, m)]); }, x);
       p_own = quad_rs(x);
     }
+    ok = mbar_wait(bar_v, par, kFillWaitPolls);
+    par ^= 1u;
+    if (tid == 0) sh_item = atomicAdd(counter, 1);
+    if (__syncthreads_or(!ok)) {  // the values never arrived: wait once more and stop
+      if (tid == 0) atomicOr(&hdr[kHdrError], kErrTimeout);
+      (void)mbar_wait(bar_v, par ^ 1u, kFillWaitPolls);
+      return;
+    }
+    const int next = sh_item;
+    if (phase == 1 && next < n_items)
+      fill_prefetch<D, __nv_bfloat16>(fill_item(next, H, cu, chunk_off, chunk_seq), bstate, q,
+                                      k, v, H);
+
     float c = 1.f;  // scale of the running state: 1 at the chunk boundary
     OUT* ob = o + tb * D + my_row;
     for (int t = 0; t < cur.len; t++) {
@@ -1154,11 +1210,21 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     GDN_TRY(persistent_grid(kern, kFillThreads, sm, &grid));
     const int64_t items = L.max_chunks * a.H;
     if ((int64_t)grid > items) grid = (int)items;
-    GDN_TRY(launch_dependent(kern, dim3((unsigned)grid), dim3(kFillThreads), sm, st, q, k, v,
-                             a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
-                             (const int32_t*)chunk_off, (const int32_t*)chunk_seq,
-                             (const float*)bstate, static_cast<OUT*>(a.o), a.s_run_final,
-                             a.s_run_scale, a.n_seqs, a.h0));
+    if constexpr (D == 128 && sizeof(IN) == 2) {
+      CUtensorMap mq, mk, mv;
+      GDN_TRY(row_maps(&mq, &mk, &mv, q, k, v, a.T, a.H));
+      GDN_TRY(launch_dependent(kern, dim3((unsigned)grid), dim3(kFillThreads), sm, st, q, k, v,
+                               a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
+                               (const int32_t*)chunk_off, (const int32_t*)chunk_seq,
+                               (const float*)bstate, static_cast<OUT*>(a.o), a.s_run_final,
+                               a.s_run_scale, a.n_seqs, a.h0, mq, mk, mv));
+    } else {
+      GDN_TRY(launch_dependent(kern, dim3((unsigned)grid), dim3(kFillThreads), sm, st, q, k, v,
+                               a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
+                               (const int32_t*)chunk_off, (const int32_t*)chunk_seq,
+                               (const float*)bstate, static_cast<OUT*>(a.o), a.s_run_final,
+                               a.s_run_scale, a.n_seqs, a.h0));
+    }
   }
   return mark(4);
 }

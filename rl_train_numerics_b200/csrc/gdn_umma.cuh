@@ -215,6 +215,15 @@ __device__ __forceinline__ void bulk_load(uint32_t sdst, const void* gsrc, uint3
       "l"(gsrc), "r"(bytes), "r"(mbar)
       : "memory");
 }
+// The same for a 3-D box.
+__device__ __forceinline__ void tma_load_3d(uint32_t sdst, const void* map, int x, int y, int z,
+                                            uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(sdst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(mbar)
+      : "memory");
+}
 // Tiled tensor copy of one 4-D box from global to shared memory through the
 // tensor map at `map` (a kernel parameter), its completion counted in
 // transaction bytes on the mbarrier at `mbar`.  The innermost coordinate x
