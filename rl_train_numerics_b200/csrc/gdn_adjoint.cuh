@@ -28,6 +28,8 @@
 //               chunk u of the backward, gdn_backward.cu's k_bwd_wu)
 #pragma once
 
+#include <cuda.h>
+
 #include <cstddef>
 
 #include "gdn_boundary.cuh"
@@ -38,15 +40,15 @@ namespace gdn {
 constexpr int kAdjNT = 3;  // bf16 terms of an fp32 operand
 
 // The adjoint pack of one (chunk, head).  Planes are bf16 in the core layout
-// (64 rows); the walk bulk-copies the head, the keys, its rows' do columns, X and
-// Tb, the solve the rest.
+// (64 rows); the walk bulk-copies the head, the keys, X and Tb, the solve the
+// rest.  The do rows are not in it: both read them from the input (the walk
+// by a tensor-map copy of its rows' columns, the solve by cp.async).
 template <int D>
 struct AdjPack {
   float dvec[kChunk];
   float beta[kChunk];  // 0 past the chunk's length
   float gamma[4];      // [0] = e^{G_{L-1}}
   __nv_bfloat16 K[1][kChunk * D];               // [t][j]
-  __nv_bfloat16 DO[1][kChunk * D];              // [t][i]
   __nv_bfloat16 X[kAdjNT][kChunk * D];          // [t][j]
   __nv_bfloat16 Tb[kAdjNT][kChunk * kChunk];    // [t][m], m <= t
   __nv_bfloat16 T[kAdjNT][kChunk * kChunk];     // [m][t], t <= m
@@ -85,7 +87,7 @@ struct AdjPrepSmem {
 template <int D>
 __global__ void __launch_bounds__(kBndThreads, 3)
     k_adj_prep(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-               const __nv_bfloat16* __restrict__ d_o, const float* __restrict__ beta,
+               const float* __restrict__ beta,
                const float* __restrict__ g, const int32_t* __restrict__ cu, int H, float scale,
                const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
                const int32_t* __restrict__ chunk_seq, char* __restrict__ apacks) {
@@ -104,11 +106,6 @@ __global__ void __launch_bounds__(kBndThreads, 3)
   const size_t tok = (size_t)it.t0 * H + h;
   AdjPack<D>& pk = *reinterpret_cast<AdjPack<D>*>(apacks + ((size_t)c * H + h) * adj_pack_bytes<D>());
 
-  {
-    PlaneRows<D, bf16, kBndThreads> dorows;  // do rows: global -> the pack's plane
-    dorows.load(d_o + tok * D, (size_t)H * D, len);
-    dorows.store(pk.DO);
-  }
   prep_stage<D, bf16>(sm.prep, k + tok * D, (size_t)H * D, beta + tok, g + tok, (size_t)H, len);
   bnd_prep<D, bf16>(sm.prep, sm.AT);
 
@@ -248,20 +245,21 @@ constexpr int kAdjWalkPairs = kAdjWalkRows / 16;
 constexpr int kAdjWalkThreads = 64 * kAdjWalkPairs;
 
 // One chunk's walk operands in shared memory: the pack's head and keys, the
-// do columns of the block's rows (their core-layout column groups), X and Tb.
+// do columns of the block's rows (their core-layout column groups, a
+// tensor-map destination), X and Tb.
 template <int D>
 struct AdjWalkBuf {
   float dvec[kChunk];
   float beta[kChunk];
   float gamma[4];
-  __nv_bfloat16 K[1][kChunk * D];                 // [t][j]
-  __nv_bfloat16 DOr[1][kChunk * kAdjWalkRows];    // [t][i - first row of the block]
+  __nv_bfloat16 K[1][kChunk * D];                           // [t][j]
+  alignas(128) __nv_bfloat16 DOr[1][kChunk * kAdjWalkRows];  // [t][i - first row of the block]
   __nv_bfloat16 X[kAdjNT][kChunk * D];            // [t][j]
   __nv_bfloat16 Tb[kAdjNT][kChunk * kChunk];      // [t][m], m <= t
 };
 template <int D>
 constexpr uint32_t adj_walk_head_bytes() {
-  return (uint32_t)offsetof(AdjPack<D>, DO);
+  return (uint32_t)offsetof(AdjPack<D>, X);
 }
 template <int D>
 constexpr uint32_t adj_walk_xtb_bytes() {
@@ -455,12 +453,14 @@ __global__ void __launch_bounds__(kAdjWalkThreads, 1)
                const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ seq_order,
                const char* __restrict__ apacks,
                const float* __restrict__ ds_final, float* __restrict__ mu_end,
-               float* __restrict__ ydv, float* __restrict__ d_h0) {
+               float* __restrict__ ydv, float* __restrict__ d_h0,
+               const __grid_constant__ CUtensorMap map_do) {
   constexpr int C = kChunk, RB = D / kAdjWalkRows, NT = D / 16;
   static_assert(D % kAdjWalkRows == 0, "whole row blocks");
   constexpr uint32_t HB = adj_walk_head_bytes<D>(), XB = adj_walk_xtb_bytes<D>();
   constexpr uint32_t DB = (uint32_t)(C * kAdjWalkRows * 2);
   static_assert(HB % 16 == 0 && XB % 16 == 0 && DB % 16 == 0 &&
+                    offsetof(AdjWalkBuf<D>, DOr) % 128 == 0 && sizeof(AdjWalkBuf<D>) % 128 == 0 &&
                     offsetof(AdjWalkBuf<D>, K) == offsetof(AdjPack<D>, K) &&
                     offsetof(AdjWalkBuf<D>, X) % 16 == 0 &&
                     offsetof(AdjWalkBuf<D>, Tb) - offsetof(AdjWalkBuf<D>, X) ==
@@ -485,14 +485,17 @@ __global__ void __launch_bounds__(kAdjWalkThreads, 1)
   auto pack = [&](int64_t cc) {
     return apacks + ((size_t)(base + cc) * H + h) * adj_pack_bytes<D>();
   };
-  // The block's do columns are core-layout column groups 8 rb .. 8 rb + 7 of
-  // the pack's do plane: one contiguous run.
+  // The block's do columns, core-layout column groups R rb .. R rb + R - 1
+  // (R = kAdjWalkRows / 8) of the chunk's do plane, come from the input by
+  // one tensor-map copy.
+  const int tok0 = cu[n];
   auto fetch = [&](int b, int64_t cc) {
     const uint32_t mb = smem_u32(&sm.bar[b]);
     const char* src = pack(cc);
     mbar_expect_tx(mb, HB + DB + XB);
     bulk_load(smem_u32(&sm.buf[b]), src, HB, mb);
-    bulk_load(smem_u32(sm.buf[b].DOr[0]), src + offsetof(AdjPack<D>, DO) + (size_t)rb * DB, DB, mb);
+    tma_load_4d(smem_u32(sm.buf[b].DOr[0]), &map_do, 0, tok0 + (int)cc * C,
+                (kAdjWalkRows / 8) * rb, h, mb);
     bulk_load(smem_u32(sm.buf[b].X[0]), src + offsetof(AdjPack<D>, X), XB, mb);
   };
   pack_bars_init(sm.bar);
@@ -521,6 +524,17 @@ __global__ void __launch_bounds__(kAdjWalkThreads, 1)
       pack_drain(sm.bar, j, issued);
       break;
     }
+    if (j == 0 && L % C != 0) {
+      // The trailing partial chunk: its do rows past the sequence's end are
+      // the next sequence's tokens (or zeros past T); they must be zero.
+      const int len = (int)(L % C);
+      __nv_bfloat16* dor = sm.buf[0].DOr[0];
+      for (int e = t; e < (kAdjWalkRows / 8) * (C - len); e += kAdjWalkThreads) {
+        const int grp = e / (C - len), r = len + e % (C - len);
+        *reinterpret_cast<uint4*>(dor + (grp * C + r) * 8) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncthreads();
+    }
     adj_walk_warp<D>(sacc, sm.buf[j & 1], rl, ch, sm.xch[pair][ch], sm.xch[pair][ch ^ 1],
                      1 + pair, ydv + (unit * D + r0) * C);
     __syncthreads();  // buffer j & 1 is refilled with chunk cc - 2; xch is free
@@ -542,11 +556,17 @@ struct AdjWSmem {
   float dvec[kChunk];
   float beta[kChunk];
   float gamma[4];
-  __nv_bfloat16 DO[1][kChunk * D];                 // [r][i]
+  alignas(128) __nv_bfloat16 DO[1][kChunk * D];    // [r][i], a tensor-map destination
   __nv_bfloat16 T[kAdjNT][kChunk * kChunk];        // [m][t]
   __nv_bfloat16 Pm[kAdjNT][kChunk * kChunk];       // [r][t]
   __nv_bfloat16 R[kAdjNT][kChunk * D];             // right-hand side, [m][i]
+  uint64_t bar;                                    // the do copy's completion
 };
+// cp.async pieces and ldmatrix rows are 16-byte aligned in every plane.
+static_assert(offsetof(AdjWSmem<128>, T) % 16 == 0 && offsetof(AdjWSmem<128>, Pm) % 16 == 0 &&
+                  offsetof(AdjWSmem<128>, R) % 16 == 0 && offsetof(AdjWSmem<64>, T) % 16 == 0 &&
+                  offsetof(AdjWSmem<64>, R) % 16 == 0,
+              "16-byte aligned planes");
 
 // The W solve of one (chunk, head) item; one block of kAdjWThreads threads.
 template <int D>
@@ -555,6 +575,7 @@ __device__ __forceinline__ void adj_w_item(AdjWSmem<D>& sm, int c, int h,
                                            const int32_t* __restrict__ chunk_off,
                                            const int32_t* __restrict__ chunk_seq,
                                            const char* __restrict__ apacks,
+                                           const CUtensorMap* map_do, int32_t* __restrict__ error,
                                            const float* __restrict__ ydv, float* __restrict__ wbuf,
                                            float* __restrict__ d_v) {
   using bf16 = __nv_bfloat16;
@@ -566,16 +587,37 @@ __device__ __forceinline__ void adj_w_item(AdjWSmem<D>& sm, int c, int h,
   const size_t tb = (size_t)it.t0 * H + h;
   const AdjPack<D>& pk =
       *reinterpret_cast<const AdjPack<D>*>(apacks + ((size_t)c * H + h) * adj_pack_bytes<D>());
-  // The pack's head, do plane, T and Pm terms (16-byte pieces).
+  // The chunk's do rows from the input by one tensor-map copy (rows past its
+  // length zeroed once it lands); the pack's head, T and Pm terms by
+  // cp.async (16-byte pieces).
+  const uint32_t bar = smem_u32(&sm.bar);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    mbar_expect_tx(bar, (uint32_t)PD * 2);
+    tma_load_4d(smem_u32(sm.DO[0]), map_do, 0, (int)it.t0, 0, h, bar);
+  }
   for (int e = tid; e < (int)(2 * C + 4) / 4; e += kAdjWThreads)
     cp_async16(reinterpret_cast<float4*>(sm.dvec) + e, reinterpret_cast<const float4*>(pk.dvec) + e);
-  for (int e = tid; e < PD / 8; e += kAdjWThreads)
-    cp_async16(reinterpret_cast<uint4*>(sm.DO[0]) + e, reinterpret_cast<const uint4*>(pk.DO[0]) + e);
   for (int e = tid; e < 2 * kAdjNT * PL / 8; e += kAdjWThreads)
     cp_async16(reinterpret_cast<uint4*>(sm.T[0]) + e, reinterpret_cast<const uint4*>(pk.T[0]) + e);
   cp_async_commit();
   cp_async_wait<0>();
-  __syncthreads();
+  const bool ok = mbar_wait(bar, 0, kTcWaitPolls);
+  if (ok && len < C) {
+    for (int e = tid; e < (D / 8) * (C - len); e += kAdjWThreads) {
+      const int grp = e / (C - len), r = len + e % (C - len);
+      *reinterpret_cast<uint4*>(&sm.DO[0][(grp * C + r) * 8]) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  if (__syncthreads_or(!ok)) {  // the do rows never arrived: wait once more and stop
+    if (tid == 0) atomicOr(error, kErrTimeout);
+    (void)mbar_wait(bar, 0, kTcWaitPolls);
+    return;
+  }
 
   using P33 = SplitPairs<kAdjNT, kAdjNT>;
   using P31 = SplitPairs<kAdjNT, 1>;

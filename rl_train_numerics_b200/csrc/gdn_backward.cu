@@ -68,10 +68,13 @@
 //                    and dg from the products above on mma.sync
 //   k_bwd_gemm       fp32 inputs: DQ and DK in fp32 fused multiply-adds
 // Every sum has a fixed order, so repeated runs give identical bits.
+#include <string.h>
+
 #include "gdn_adjoint.cuh"
 #include "gdn_boundary.cuh"
 #include "gdn_fill.cuh"
 #include "gdn_layout.h"
+#include "gdn_tmap.h"
 
 namespace gdn {
 
@@ -1305,10 +1308,11 @@ template <int D>
 __global__ void __launch_bounds__(kUThreads, 2)
     k_bwd_wu(const __nv_bfloat16* __restrict__ v, const float* __restrict__ beta,
              const float* __restrict__ g, const int32_t* __restrict__ cu, int H, float scale,
-             const int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
+             int32_t* __restrict__ hdr, const int32_t* __restrict__ chunk_off,
              const int32_t* __restrict__ chunk_seq, const float* __restrict__ bstate,
              const char* __restrict__ apacks, const float* __restrict__ ydv,
-             float* __restrict__ wbuf, float* __restrict__ d_v, float* __restrict__ ubuf) {
+             float* __restrict__ wbuf, float* __restrict__ d_v, float* __restrict__ ubuf,
+             const __grid_constant__ CUtensorMap map_do) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   BwdWUSmem<D>& sm = *reinterpret_cast<BwdWUSmem<D>*>(smem_raw);
   pdl_wait();  // the reverse walk's Ydv and adjoints
@@ -1317,7 +1321,8 @@ __global__ void __launch_bounds__(kUThreads, 2)
   const int c = blockIdx.x >> 1, h = blockIdx.y;
   if (c >= hdr[kHdrChunks]) return;
   if ((blockIdx.x & 1) == 0)
-    adj_w_item<D>(sm.w, c, h, cu, H, scale, chunk_off, chunk_seq, apacks, ydv, wbuf, d_v);
+    adj_w_item<D>(sm.w, c, h, cu, H, scale, chunk_off, chunk_seq, apacks, &map_do, &hdr[kHdrError],
+                  ydv, wbuf, d_v);
   else
     bwd_u_item<D>(sm.u, c, h, v, beta, g, cu, H, chunk_off, chunk_seq, bstate, apacks, ubuf);
 }
@@ -1364,12 +1369,13 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
     char* apack = ws + L.apack;
     float* ydv = reinterpret_cast<float*>(ws + L.ydv);
     int32_t* hdr_w = reinterpret_cast<int32_t*>(ws + L.fwd.hdr);
+    CUtensorMap map_do_all;
     {
       auto kern = k_adj_prep<D>;
       const size_t sm = sizeof(AdjPrepSmem<D>);
       GDN_BWD_TRY(bwd_set_smem(kern, sm));
-      kern<<<gchunks, kBndThreads, sm, st>>>(q, k, d_o, f.beta, f.g, f.cu_seqlens, f.H, f.scale,
-                                             hdr, chunk_off, chunk_seq, apack);
+      kern<<<gchunks, kBndThreads, sm, st>>>(q, k, f.beta, f.g, f.cu_seqlens, f.H, f.scale, hdr,
+                                             chunk_off, chunk_seq, apack);
       GDN_BWD_TRY(cudaGetLastError());
     }
     {
@@ -1377,12 +1383,22 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
       const size_t sm = sizeof(AdjWalkSmem<D>);
       GDN_BWD_TRY(bwd_set_smem(kern, sm));
       const int32_t* seq_order = reinterpret_cast<const int32_t*>(ws + L.fwd.seq_order);
+      // The walk's do columns by tensor map (a box of 64 tokens x its rows'
+      // column groups); zeroed (never read) without tokens.
+      CUtensorMap map_do;
+      memset(&map_do, 0, sizeof(map_do));
+      if (f.T > 0 && !encode_plane_map(&map_do, d_o, f.T, f.H, D, kChunk, kAdjWalkRows / 8))
+        return cudaErrorNotSupported;  // a refused map: there is no other route
+      // The W solve's: all D / 8 column groups of 64 tokens.
+      memset(&map_do_all, 0, sizeof(map_do_all));
+      if (f.T > 0 && !encode_plane_map(&map_do_all, d_o, f.T, f.H, D, kChunk, D / 8))
+        return cudaErrorNotSupported;
       // walk, W solve + u and the products are programmatic dependents of
       // the kernel before them (each waits for it first thing)
       GDN_BWD_TRY(launch_dependent(
           kern, dim3((unsigned)((size_t)f.n_seqs * f.H * (D / kAdjWalkRows))),
           dim3(kAdjWalkThreads), sm, st, f.cu_seqlens, f.H, hdr_w, chunk_off, seq_order,
-          (const char*)apack, a.ds_final, mu_end, ydv, a.d_h0));
+          (const char*)apack, a.ds_final, mu_end, ydv, a.d_h0, map_do));
     }
     GDN_BWD_TRY(mark(2));
     {  // the W solve and u (dbeta and dg come with dq and dk)
@@ -1391,8 +1407,9 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
       GDN_BWD_TRY(bwd_set_smem(kern, sm));
       GDN_BWD_TRY(launch_dependent(kern, dim3(2 * (unsigned)L.fwd.max_chunks, (unsigned)f.H),
                                    dim3(kUThreads), sm, st, v, f.beta, f.g, f.cu_seqlens, f.H,
-                                   f.scale, hdr, chunk_off, chunk_seq, bstate,
-                                   (const char*)apack, (const float*)ydv, wbuf, a.d_v, ubuf));
+                                   f.scale, hdr_w, chunk_off, chunk_seq, bstate,
+                                   (const char*)apack, (const float*)ydv, wbuf, a.d_v, ubuf,
+                                   map_do_all));
     }
   } else {
     auto kern = k_bwd_scan<D, IN>;

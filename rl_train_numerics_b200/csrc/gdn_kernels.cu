@@ -319,45 +319,11 @@ __global__ void __launch_bounds__(walk_threads<D>(), 1)
 constexpr int kWalkSlices = 4;
 constexpr int kWalkThreads = kTcRows * kWalkSlices;
 
-// Value planes of one chunk and head straight from a [T][H][D] bf16 input
-// (D = 128): a 4-D map over (8 channels, T tokens, D / 8 channel groups,
-// H heads) whose box of 8 x 64 x 16 x 1 elements lands in shared memory as
-// [group][token][8], the planes' core-matrix layout.  False if the encoder
-// is missing or refuses the map.
-static bool make_plane_map(CUtensorMap* map, const void* base, int64_t T, int H) {
-  constexpr int D = 128;
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[4] = {8, (cuuint64_t)T, D / 8, (cuuint64_t)H};
-  const cuuint64_t strides[3] = {(cuuint64_t)H * D * 2, 16, D * 2};  // bytes, dims 1..3
-  const cuuint32_t box[4] = {8, (cuuint32_t)kChunk, D / 8, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Bytes of a walk pack ahead of its value planes (the head and the keys).
 template <int D, class IN>
 constexpr uint32_t pack_bytes_before_v() {
   using WP = WalkPack<D, IN>;
   return (uint32_t)offsetof(WP, kv.V);
-}
-
-// One chunk's rows of one head from a [T][H][128] bf16 input: a 3-D map over
-// (128 channels, H heads, T tokens) whose box of 128 x 1 x 64 elements lands
-// as [token][channel] (tokens past T read as zeros).
-static bool make_row_map(CUtensorMap* map, const void* base, int64_t T, int H) {
-  constexpr int D = 128;
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {D, (cuuint64_t)H, (cuuint64_t)T};
-  const cuuint64_t strides[2] = {D * 2, (cuuint64_t)H * D * 2};  // bytes, dims 1..2
-  const cuuint32_t box[3] = {D, 1, (cuuint32_t)kChunk};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // The fill's query, key and value maps; zeroed (never read) without tokens.
@@ -368,8 +334,9 @@ static cudaError_t row_maps(CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv, c
   memset(mk, 0, sizeof(*mk));
   memset(mv, 0, sizeof(*mv));
   if (T < 1) return cudaSuccess;
-  const bool ok = make_row_map(mq, q, T, H) && make_row_map(mk, k, T, H) &&
-                  make_row_map(mv, v, T, H);
+  const bool ok = encode_row_map(mq, q, T, H, 128, kChunk) &&
+                  encode_row_map(mk, k, T, H, 128, kChunk) &&
+                  encode_row_map(mv, v, T, H, 128, kChunk);
   return ok ? cudaSuccess : cudaErrorNotSupported;
 }
 
@@ -378,7 +345,7 @@ static cudaError_t row_maps(CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv, c
 static cudaError_t value_map(CUtensorMap* mv, const void* v, int64_t T, int H) {
   memset(mv, 0, sizeof(*mv));
   if (T < kChunk) return cudaSuccess;
-  return make_plane_map(mv, v, T, H) ? cudaSuccess : cudaErrorNotSupported;
+  return encode_plane_map(mv, v, T, H, 128, kChunk, 16) ? cudaSuccess : cudaErrorNotSupported;
 }
 
 // The tcgen05 walk's inputs of one full chunk into dst: the pack head and key

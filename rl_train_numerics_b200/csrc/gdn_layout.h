@@ -152,13 +152,13 @@ struct BndArgs {
 //   ubuf    f32[T,H,dv]      u_t = beta_t (v_t - alpha_t S_{t-1} k_t) per row
 //   with bf16 inputs (the adjoint in chunk form, gdn_adjoint.cuh), also
 //   apack   [MC,H] adjoint packs (mirrors adj_pack_bytes<D>(): head of
-//                  2C + 4 floats, keys and do as bf16 planes C x D, X as three
+//                  2C + 4 floats, keys as a bf16 plane C x D, X as three
 //                  bf16 term planes C x D, Tb, T and Pm as three term planes
 //                  C x C each)
 //   ydv     f32[MC,H,dv,C]  (mu_e K^T) diag(dvec) per chunk (the walk's output)
 constexpr size_t adj_pack_bytes_host(int D) {
   const size_t C = 64;
-  const size_t b = (2 * C + 4) * 4 + 2 * C * (size_t)D * 2 + 3 * C * (size_t)D * 2 + 9 * C * C * 2;
+  const size_t b = (2 * C + 4) * 4 + C * (size_t)D * 2 + 3 * C * (size_t)D * 2 + 9 * C * C * 2;
   return (b + 127) / 128 * 128;
 }
 
