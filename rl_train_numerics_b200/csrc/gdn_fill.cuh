@@ -14,6 +14,8 @@ constexpr int kHdrChunks = 1;    // number of chunks of this call
 constexpr int kHdrValid = 2;     // 1 when this call's chunk table is valid
 constexpr int kHdrFillNext = 3;  // work counter of k_fill
 constexpr int kHdrFill0Next = 4; // work counter of the fill's first chunks (k_fill128)
+constexpr int kHdrFill1Chunks = 5; // entries of the fill order (k_fill128)
+constexpr int kHdrFillUniform = 6; // 1 when every sequence has the same chunk count
 
 constexpr int kFillThreads = 128;
 

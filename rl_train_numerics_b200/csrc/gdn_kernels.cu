@@ -35,9 +35,9 @@ namespace gdn {
 constexpr int kTableThreads = 1024;
 
 __global__ void __launch_bounds__(kTableThreads)
-    k_chunk_table(const int32_t* __restrict__ cu, int N, int64_t T, int32_t* hdr,
+    k_chunk_table(const int32_t* __restrict__ cu, int N, int64_t T, int H, int32_t* hdr,
                   int32_t* chunk_off, int32_t* seq_order, int32_t* chunk_seq,
-                  int64_t max_chunks) {
+                  int32_t* walk_done, int32_t* fill_order, int64_t max_chunks) {
   __shared__ long long part[64 + kTableThreads];
   __shared__ int bucket[kTableThreads];
   __shared__ int bad;
@@ -140,6 +140,56 @@ __global__ void __launch_bounds__(kTableThreads)
   }
   __syncthreads();
   for (int64_t n = n0; n < n1; n++) seq_order[atomicAdd(&bucket[key(n)], 1)] = (int32_t)n;
+  // One word per (sequence, head), zero until the walk has stored that
+  // unit's boundary states.
+  for (int64_t i = tid; i < (int64_t)N * H; i += kTableThreads) walk_done[i] = 0;
+  __syncthreads();  // seq_order complete
+  // The fill order: every chunk after a sequence's first, the sequences in
+  // seq_order reversed (fewest chunks first: their walks end first), chunks
+  // ascending within a sequence.  Exclusive scan of the per-thread entry
+  // counts as above.
+  {
+    long long mine = 0;
+    for (int64_t r = n0; r < n1; r++) {
+      const int sq = seq_order[N - 1 - r];
+      const long long nc = chunk_off[sq + 1] - chunk_off[sq];
+      mine += nc > 1 ? nc - 1 : 0;
+    }
+    long long xs = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(kFull, xs, o);
+      if (lane >= o) xs += y;
+    }
+    if (lane == 31) part[warp] = xs;
+    __syncthreads();
+    if (warp == 0) {
+      long long ws = part[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(kFull, ws, o);
+        if (lane >= o) ws += y;
+      }
+      part[32 + lane] = ws;
+    }
+    __syncthreads();
+    long long at = xs - mine + (warp > 0 ? part[32 + warp - 1] : 0);
+    for (int64_t r = n0; r < n1; r++) {
+      const int sq = seq_order[N - 1 - r];
+      for (int32_t c = chunk_off[sq] + 1; c < chunk_off[sq + 1]; c++) fill_order[at++] = c;
+    }
+    if (tid == 0) {
+      hdr[kHdrFill1Chunks] = (int32_t)part[32 + 31];
+      // Equal chunk counts: every walk ends at about the same time, so the
+      // fill waits for the walk grid once instead of checking its units.
+      int uniform = 1;
+      if (N > 0) {
+        const int a = seq_order[0], b = seq_order[N - 1];
+        uniform = chunk_off[a + 1] - chunk_off[a] == chunk_off[b + 1] - chunk_off[b];
+      }
+      hdr[kHdrFillUniform] = uniform;
+    }
+  }
   if (tid == 0) hdr[kHdrValid] = 1;
 }
 
@@ -431,7 +481,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
               const int32_t* __restrict__ seq_order, const char* __restrict__ packs,
               float* __restrict__ bstate,
               float* __restrict__ s_run_final, float* __restrict__ s_run_scale,
-              float* __restrict__ s_bnd_final, const __grid_constant__ CUtensorMap map_v) {
+              float* __restrict__ s_bnd_final, int32_t* __restrict__ walk_done,
+              const __grid_constant__ CUtensorMap map_v) {
   static_assert(use_tc<D, IN>(), "tcgen05 walk: d = 128, bf16 inputs");
   constexpr int SC = D / kWalkSlices;
   constexpr size_t PB = pack_size<D, IN>();
@@ -513,6 +564,17 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       s_run_scale[(size_t)n * H + h] = 1.f;
   }
   if (t == 0) bulk_wait();  // every bulk store complete before the block exits
+  if (status == kStepDone) {
+    // Publish the unit: the block's stores (a barrier), then thread 0,
+    // after its bulk stores completed, releases the unit's word, which the
+    // fill acquires before it reads these states.
+    __syncthreads();
+    if (t == 0) {
+      fence_proxy_async_global();
+      __threadfence();
+      st_release_gpu(&walk_done[(size_t)n * H + h], 1);
+    }
+  }
   tc_teardown(cx);
 }
 
@@ -616,24 +678,27 @@ __global__ void __launch_bounds__(kFillThreads, 3)
               const int32_t* __restrict__ chunk_seq, const float* __restrict__ bstate,
               OUT* __restrict__ o, float* __restrict__ s_run_final,
               float* __restrict__ s_run_scale, int n_seqs, const float* __restrict__ h0,
+              const int32_t* __restrict__ fill_order, const int32_t* walk_done,
               const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v) {
   constexpr int D = 128, M4 = D / 16;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Fill128Smem& sm = *reinterpret_cast<Fill128Smem*>(smem_raw);
-  __shared__ int sh_item;
-  // Two phases.  Phase 0, before waiting for the boundary walk: the first
-  // chunk of every sequence, whose entry state is h0 (or zero), not a walk
-  // result, so that these items run on the SMs the walk leaves idle (the
-  // walk only writes boundary states, the bound final states and the pack
-  // reads, none of which a first chunk touches).  Phase 1, after the wait:
-  // every other chunk.  The chunk table (read in both) completed before the
-  // walk started.
+  __shared__ int sh_item, sh_ready;
+  // Two phases.  Phase 0: the first chunk of every sequence, whose entry
+  // state is h0 (or zero), not a walk result, so that these items run on the
+  // SMs the walk leaves idle (the walk only writes boundary states, the bound
+  // final states and the pack reads, none of which a first chunk touches).
+  // Phase 1: every other chunk, in the fill order (sequences with the fewest
+  // chunks first: their walks end first).  An item starts once its unit's
+  // walk word is set (acquired by thread 0, then a block barrier); the first
+  // item whose word is not set yet makes the block wait for the whole walk
+  // grid (griddepcontrol.wait), after which every word is.  The chunk table
+  // (read in both phases) completed before the walk started.
   if (hdr[kHdrValid] != 1) {
     pdl_wait();
     return;
   }
-  const int n_items = hdr[kHdrChunks] * H;
   const int tid = threadIdx.x, l = tid & 3, r0 = (tid >> 2) * 4, sg = quad_sigma(l);
   const int my_row = r0 + sg;
   const size_t DD = (size_t)D * D;
@@ -644,7 +709,8 @@ __global__ void __launch_bounds__(kFillThreads, 3)
     mbar_init(smem_u32(&sm.bar[1]), 1);
     fence_mbar_init();
   }
-  uint32_t par = 0;  // phase of both barriers the next item waits for
+  uint32_t par = 0;     // phase of both barriers the next item waits for
+  bool walked = false;  // this block has waited for the whole walk grid
   int phase = 0, limit = n_seqs * H;
   int32_t* counter = &hdr[kHdrFill0Next];
   auto claim = [&]() {
@@ -658,9 +724,12 @@ __global__ void __launch_bounds__(kFillThreads, 3)
     if (item >= limit) {
       if (phase == 1) break;
       phase = 1;
-      pdl_wait();  // the boundary walk's states
       counter = &hdr[kHdrFillNext];
-      limit = n_items;
+      limit = hdr[kHdrFill1Chunks] * H;
+      if (hdr[kHdrFillUniform]) {
+        pdl_wait();  // the whole walk grid
+        walked = true;
+      }
       item = claim();
       continue;
     }
@@ -673,11 +742,7 @@ __global__ void __launch_bounds__(kFillThreads, 3)
       }
       cur = fill_item(chunk_off[n] * H + hh, H, cu, chunk_off, chunk_seq);
     } else {
-      cur = fill_item(item, H, cu, chunk_off, chunk_seq);
-      if (cur.ci == 0) {  // done in phase 0
-        item = claim();
-        continue;
-      }
+      cur = fill_item(fill_order[item / H] * H + item % H, H, cu, chunk_off, chunk_seq);
     }
     const size_t tb = (size_t)cur.t0 * H + cur.h;
     const uint32_t bar_kq = smem_u32(&sm.bar[0]), bar_v = smem_u32(&sm.bar[1]);
@@ -698,6 +763,16 @@ __global__ void __launch_bounds__(kFillThreads, 3)
         b = beta[tb + (size_t)tid * H];
       }
       sm.t0[tid] = make_float4(a, b, 0.f, 0.f);
+    }
+    // A phase-1 item's entry state is its unit's walk result: acquired here,
+    // behind the input copies and scalar loads, which do not depend on it.
+    if (phase == 1 && !walked) {
+      if (tid == 0) sh_ready = ld_acquire_gpu(&walk_done[(size_t)cur.n * H + cur.h]);
+      __syncthreads();
+      if (!sh_ready) {
+        pdl_wait();  // the whole walk grid
+        walked = true;
+      }
     }
     Slice<4, M4> S;
     if (phase == 0)
@@ -770,9 +845,10 @@ __global__ void __launch_bounds__(kFillThreads, 3)
       return;
     }
     const int next = sh_item;
-    if (phase == 1 && next < n_items)
-      fill_prefetch<D, __nv_bfloat16>(fill_item(next, H, cu, chunk_off, chunk_seq), bstate, q,
-                                      k, v, H);
+    if (phase == 1 && next < limit)
+      fill_prefetch<D, __nv_bfloat16>(
+          fill_item(fill_order[next / H] * H + next % H, H, cu, chunk_off, chunk_seq), bstate, q,
+          k, v, H);
 
     float c = 1.f;  // scale of the running state: 1 at the chunk boundary
     OUT* ob = o + tb * D + my_row;
@@ -810,6 +886,7 @@ __global__ void __launch_bounds__(kFillThreads, 3)
     item = next;
     __syncthreads();  // shared memory is reloaded for the next item
   }
+  pdl_wait();  // the fill grid does not complete before the walk grid
 }
 
 // ----------------------------------------------------------------------------
@@ -1132,8 +1209,11 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   };
   GDN_TRY(mark(0));
   int32_t* seq_order = reinterpret_cast<int32_t*>(ws + L.seq_order);
-  k_chunk_table<<<1, kTableThreads, 0, st>>>(a.cu_seqlens, a.n_seqs, a.T, hdr, chunk_off,
-                                             seq_order, chunk_seq, L.max_chunks);
+  int32_t* walk_done = reinterpret_cast<int32_t*>(ws + L.walk_done);
+  int32_t* fill_order = reinterpret_cast<int32_t*>(ws + L.fill_order);
+  k_chunk_table<<<1, kTableThreads, 0, st>>>(a.cu_seqlens, a.n_seqs, a.T, a.H, hdr, chunk_off,
+                                             seq_order, chunk_seq, walk_done, fill_order,
+                                             L.max_chunks);
   GDN_TRY(cudaGetLastError());
   const dim3 gchunks((unsigned)L.max_chunks, (unsigned)a.H);
   GDN_TRY(mark(1));
@@ -1158,7 +1238,7 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     GDN_TRY(launch_dependent(kern, gunits, dim3(kWalkThreads), sm, st, a.cu_seqlens, a.H, a.h0,
                              hdr, (const int32_t*)chunk_off, (const int32_t*)seq_order,
                              (const char*)packs, bstate, a.s_run_final, a.s_run_scale,
-                             a.s_bnd_final, mv));
+                             a.s_bnd_final, walk_done, mv));
   } else {
     auto kern = k_walk<D, IN>;
     const size_t sm = sizeof(WalkSmem<D, IN>);
@@ -1184,7 +1264,8 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
                                a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
                                (const int32_t*)chunk_off, (const int32_t*)chunk_seq,
                                (const float*)bstate, static_cast<OUT*>(a.o), a.s_run_final,
-                               a.s_run_scale, a.n_seqs, a.h0, mq, mk, mv));
+                               a.s_run_scale, a.n_seqs, a.h0, (const int32_t*)fill_order,
+                               (const int32_t*)walk_done, mq, mk, mv));
     } else {
       GDN_TRY(launch_dependent(kern, dim3((unsigned)grid), dim3(kFillThreads), sm, st, q, k, v,
                                a.beta, a.g, a.cu_seqlens, a.H, a.scale, hdr,
@@ -1215,8 +1296,11 @@ static cudaError_t native_impl(const FwdArgs& a, cudaStream_t st) {
   };
   GDN_TRY(mark(0));
   int32_t* seq_order = reinterpret_cast<int32_t*>(ws + L.seq_order);
-  k_chunk_table<<<1, kTableThreads, 0, st>>>(a.cu_seqlens, a.n_seqs, a.T, hdr, chunk_off,
-                                             seq_order, chunk_seq, L.max_chunks);
+  int32_t* walk_done = reinterpret_cast<int32_t*>(ws + L.walk_done);
+  int32_t* fill_order = reinterpret_cast<int32_t*>(ws + L.fill_order);
+  k_chunk_table<<<1, kTableThreads, 0, st>>>(a.cu_seqlens, a.n_seqs, a.T, a.H, hdr, chunk_off,
+                                             seq_order, chunk_seq, walk_done, fill_order,
+                                             L.max_chunks);
   GDN_TRY(cudaGetLastError());
   GDN_TRY(mark(1));
   {
@@ -1237,7 +1321,7 @@ static cudaError_t native_impl(const FwdArgs& a, cudaStream_t st) {
     GDN_TRY(value_map(&mv, a.v, a.T, a.H));
     kern<<<(unsigned)((size_t)a.n_seqs * a.H), kWalkThreads, sm, st>>>(
         a.cu_seqlens, a.H, a.h0, hdr, chunk_off, seq_order, packs, bstate, a.s_run_final, nullptr,
-        a.s_bnd_final, mv);
+        a.s_bnd_final, walk_done, mv);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(3));

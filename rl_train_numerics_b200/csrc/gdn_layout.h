@@ -23,6 +23,9 @@ constexpr size_t pack_bytes(int D, bool in_bf16) {
 //                         [2] 1 when this call's chunk table is valid
 //   chunk_off  int32[N+1]   first global chunk index of each sequence
 //   chunk_seq  int32[MC]    sequence of each global chunk
+//   walk_done  int32[N,H]   nonzero once the walk has stored a unit's boundary states
+//   fill_order int32[MC]    the chunks after each sequence's first, fewest-chunk
+//                           sequences first (the fill's order for them)
 //   bstate     f32[MC,H,dv,dk]  state at the start of every chunk
 //   pack       [MC,H] walk packs (boundary prep of full chunks; the chunked
 //                     forward also prepares trailing partial chunks, zero-padded)
@@ -31,7 +34,7 @@ constexpr size_t pack_bytes(int D, bool in_bf16) {
 struct FwdLayout {
   int64_t max_chunks;
   size_t pack_bytes;
-  size_t hdr, chunk_off, seq_order, chunk_seq, bstate, pack, total;
+  size_t hdr, chunk_off, seq_order, chunk_seq, walk_done, fill_order, bstate, pack, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -49,6 +52,10 @@ inline FwdLayout fwd_layout(int n_seqs, int64_t T, int H, int dk, int dv, int C,
   L.seq_order = off;
   off += align256((size_t)n_seqs * sizeof(int32_t));
   L.chunk_seq = off;
+  off += align256(mc * sizeof(int32_t));
+  L.walk_done = off;
+  off += align256((size_t)n_seqs * H * sizeof(int32_t));
+  L.fill_order = off;
   off += align256(mc * sizeof(int32_t));
   L.bstate = off;
   off += align256(mc * H * dv * dk * sizeof(float));
