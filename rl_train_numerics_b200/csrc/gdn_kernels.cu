@@ -37,7 +37,7 @@ constexpr int kTableThreads = 1024;
 __global__ void __launch_bounds__(kTableThreads)
     k_chunk_table(const int32_t* __restrict__ cu, int N, int64_t T, int H, int32_t* hdr,
                   int32_t* chunk_off, int32_t* seq_order, int32_t* chunk_seq,
-                  int32_t* walk_done, int32_t* fill_order, int64_t max_chunks) {
+                  int32_t* fill_off, int64_t max_chunks) {
   __shared__ long long part[64 + kTableThreads];
   __shared__ int bucket[kTableThreads];
   __shared__ int bad;
@@ -140,14 +140,12 @@ __global__ void __launch_bounds__(kTableThreads)
   }
   __syncthreads();
   for (int64_t n = n0; n < n1; n++) seq_order[atomicAdd(&bucket[key(n)], 1)] = (int32_t)n;
-  // One word per (sequence, head), zero until the walk has stored that
-  // unit's boundary states.
-  for (int64_t i = tid; i < (int64_t)N * H; i += kTableThreads) walk_done[i] = 0;
   __syncthreads();  // seq_order complete
   // The fill order: every chunk after a sequence's first, the sequences in
   // seq_order reversed (fewest chunks first: their walks end first), chunks
-  // ascending within a sequence.  Exclusive scan of the per-thread entry
-  // counts as above.
+  // ascending within a sequence.  Here each sequence's first entry
+  // (exclusive scan of the per-thread entry counts as above); the prep's
+  // blocks write the entries.
   {
     long long mine = 0;
     for (int64_t r = n0; r < n1; r++) {
@@ -176,7 +174,9 @@ __global__ void __launch_bounds__(kTableThreads)
     long long at = xs - mine + (warp > 0 ? part[32 + warp - 1] : 0);
     for (int64_t r = n0; r < n1; r++) {
       const int sq = seq_order[N - 1 - r];
-      for (int32_t c = chunk_off[sq] + 1; c < chunk_off[sq + 1]; c++) fill_order[at++] = c;
+      const long long nc = chunk_off[sq + 1] - chunk_off[sq];
+      fill_off[sq] = (int32_t)at;
+      at += nc > 1 ? nc - 1 : 0;
     }
     if (tid == 0) {
       hdr[kHdrFill1Chunks] = (int32_t)part[32 + 31];
@@ -220,7 +220,8 @@ __global__ void __launch_bounds__(kBndThreads, prep_at_on_keys<D, IN>() ? 4 : 3)
            const float* __restrict__ g,
            const int32_t* __restrict__ cu, int H, const int32_t* __restrict__ hdr,
            const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ chunk_seq,
-           char* __restrict__ packs, int all_chunks) {
+           char* __restrict__ packs, int all_chunks, int n_seqs, int32_t* __restrict__ walk_done,
+           const int32_t* __restrict__ fill_off, int32_t* __restrict__ fill_order) {
   static_assert(sizeof(PackHead<D, IN>) % 16 == 0 && sizeof(KVPlanes<D, IN>) % 16 == 0,
                 "pack copies are 16-byte pieces");
   using PS = PrepSmem<D, IN>;
@@ -234,9 +235,14 @@ __global__ void __launch_bounds__(kBndThreads, prep_at_on_keys<D, IN>() ? 4 : 3)
   const int c = blockIdx.x, h = blockIdx.y;
   pdl_wait();
   pdl_trigger();
-  if (hdr[kHdrValid] != 1 || c >= hdr[kHdrChunks]) return;
+  if (hdr[kHdrValid] != 1) return;
+  // The walk's word of unit (c, h) starts at zero; the fill order's entry of
+  // chunk c (not a sequence's first) is written here.
+  if (c < n_seqs && threadIdx.x == 0) walk_done[(size_t)c * H + h] = 0;
+  if (c >= hdr[kHdrChunks]) return;
   const int n = chunk_seq[c];
   const int ci = c - chunk_off[n];
+  if (h == 0 && ci >= 1 && threadIdx.x == 0) fill_order[fill_off[n] + ci - 1] = c;
   const int64_t L = (int64_t)cu[n + 1] - cu[n];
   // A trailing partial chunk has no boundary after it; with all_chunks (the
   // chunked forward's outputs need its pack) it is prepared zero-padded.
@@ -1210,10 +1216,10 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
   GDN_TRY(mark(0));
   int32_t* seq_order = reinterpret_cast<int32_t*>(ws + L.seq_order);
   int32_t* walk_done = reinterpret_cast<int32_t*>(ws + L.walk_done);
+  int32_t* fill_off = reinterpret_cast<int32_t*>(ws + L.fill_off);
   int32_t* fill_order = reinterpret_cast<int32_t*>(ws + L.fill_order);
   k_chunk_table<<<1, kTableThreads, 0, st>>>(a.cu_seqlens, a.n_seqs, a.T, a.H, hdr, chunk_off,
-                                             seq_order, chunk_seq, walk_done, fill_order,
-                                             L.max_chunks);
+                                             seq_order, chunk_seq, fill_off, L.max_chunks);
   GDN_TRY(cudaGetLastError());
   const dim3 gchunks((unsigned)L.max_chunks, (unsigned)a.H);
   GDN_TRY(mark(1));
@@ -1225,7 +1231,8 @@ static cudaError_t forward_impl(const FwdArgs& a, cudaStream_t st) {
     GDN_TRY(set_smem(kern, sm));
     GDN_TRY(launch_dependent(kern, gchunks, dim3(kBndThreads), sm, st, k, v, a.beta, a.g,
                              a.cu_seqlens, a.H, (const int32_t*)hdr, (const int32_t*)chunk_off,
-                             (const int32_t*)chunk_seq, packs, 0));
+                             (const int32_t*)chunk_seq, packs, 0, a.n_seqs, walk_done,
+                             (const int32_t*)fill_off, fill_order));
   }
   GDN_TRY(mark(2));
   const dim3 gunits((unsigned)((size_t)a.n_seqs * a.H));
@@ -1297,10 +1304,10 @@ static cudaError_t native_impl(const FwdArgs& a, cudaStream_t st) {
   GDN_TRY(mark(0));
   int32_t* seq_order = reinterpret_cast<int32_t*>(ws + L.seq_order);
   int32_t* walk_done = reinterpret_cast<int32_t*>(ws + L.walk_done);
+  int32_t* fill_off = reinterpret_cast<int32_t*>(ws + L.fill_off);
   int32_t* fill_order = reinterpret_cast<int32_t*>(ws + L.fill_order);
   k_chunk_table<<<1, kTableThreads, 0, st>>>(a.cu_seqlens, a.n_seqs, a.T, a.H, hdr, chunk_off,
-                                             seq_order, chunk_seq, walk_done, fill_order,
-                                             L.max_chunks);
+                                             seq_order, chunk_seq, fill_off, L.max_chunks);
   GDN_TRY(cudaGetLastError());
   GDN_TRY(mark(1));
   {
@@ -1309,7 +1316,7 @@ static cudaError_t native_impl(const FwdArgs& a, cudaStream_t st) {
     GDN_TRY(set_smem(kern, sm));
     kern<<<dim3((unsigned)L.max_chunks, (unsigned)a.H), kBndThreads, sm, st>>>(
         static_cast<const IN*>(a.k), static_cast<const IN*>(a.v), a.beta, a.g, a.cu_seqlens,
-        a.H, hdr, chunk_off, chunk_seq, packs, 1);
+        a.H, hdr, chunk_off, chunk_seq, packs, 1, a.n_seqs, walk_done, fill_off, fill_order);
     GDN_TRY(cudaGetLastError());
   }
   GDN_TRY(mark(2));

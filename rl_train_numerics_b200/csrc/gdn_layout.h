@@ -24,6 +24,7 @@ constexpr size_t pack_bytes(int D, bool in_bf16) {
 //   chunk_off  int32[N+1]   first global chunk index of each sequence
 //   chunk_seq  int32[MC]    sequence of each global chunk
 //   walk_done  int32[N,H]   nonzero once the walk has stored a unit's boundary states
+//   fill_off   int32[N]     each sequence's first entry in fill_order
 //   fill_order int32[MC]    the chunks after each sequence's first, fewest-chunk
 //                           sequences first (the fill's order for them)
 //   bstate     f32[MC,H,dv,dk]  state at the start of every chunk
@@ -34,7 +35,8 @@ constexpr size_t pack_bytes(int D, bool in_bf16) {
 struct FwdLayout {
   int64_t max_chunks;
   size_t pack_bytes;
-  size_t hdr, chunk_off, seq_order, chunk_seq, walk_done, fill_order, bstate, pack, total;
+  size_t hdr, chunk_off, seq_order, chunk_seq, walk_done, fill_off, fill_order, bstate, pack,
+      total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -55,6 +57,8 @@ inline FwdLayout fwd_layout(int n_seqs, int64_t T, int H, int dk, int dv, int C,
   off += align256(mc * sizeof(int32_t));
   L.walk_done = off;
   off += align256((size_t)n_seqs * H * sizeof(int32_t));
+  L.fill_off = off;
+  off += align256((size_t)n_seqs * sizeof(int32_t));
   L.fill_order = off;
   off += align256(mc * sizeof(int32_t));
   L.bstate = off;
