@@ -1,9 +1,9 @@
 // gdn_kernels.cu -- CUDA kernels of the CPR Gated DeltaNet layer (sm_100a).
 //
 // Forward ("NovaSky's IsoExec Fixes the Hidden Math Bug Corrupting AI
-// Training Runs", section "Solving the linear-attention headache": a first
-// pass computes the recurrent state at chunk boundaries, then the outputs
-// within each chunk are filled in):
+// Training Runs", section "Solving the linear-attention headache"): two
+// passes, the states at the chunk edges first, then every chunk's tokens
+// from its entry state:
 //   k_chunk_table   one block: validates cu_seqlens, numbers the chunks,
 //                   orders the sequences by chunk count
 //   k_prep          one block per (chunk, head): boundary prep of full chunks

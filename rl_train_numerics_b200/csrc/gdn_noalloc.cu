@@ -29,8 +29,6 @@
 // array: callers must order them.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "../../include/gdn_cpr.h"
 #include "gdn_layout.h"
 
@@ -38,23 +36,14 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device (looked up once).
+// Device address of g_noalloc_scratch in the current context, looked up on
+// every call (a host-side lookup; a cached address would outlive a reset or
+// re-created primary context).
 int scratch_on_current_device(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr) return GDN_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr) return GDN_ERR_CUDA;
+  *out = p;
   return GDN_OK;
 }
 
