@@ -363,16 +363,17 @@ __global__ void __launch_bounds__(walk_threads<D>(), 1)
   }
 }
 
-// The walk on tcgen05 (d = 128, bf16): one block of 512 threads per
-// (sequence, head); warp w holds columns 32 (w / 4) .. + 31 of the rows of its
-// tensor-memory lane quadrant.  Chunk c + 1's inputs are copied in (its pack
+// The walk on tcgen05 (d = 128, bf16): one block of 256 threads per
+// (sequence, head); warp w holds columns 64 (w / 4) .. + 63 of the rows of its
+// tensor-memory lane quadrant (two column slices: 2.5 % faster per chunk step
+// than four, and one slice spills registers; the bits do not depend on it).  Chunk c + 1's inputs are copied in (its pack
 // head and key planes by one bulk copy, its value planes by one tensor-map
 // copy from the input) from the start of chunk c's step, and chunk c + 2's
 // pack prefetched into L2 while chunk c's products run.
 // Each boundary state goes to the workspace through a shared-memory staging
 // copy (permuted rows, conflict-free) and one bulk asynchronous store, issued
 // with the chunk's first products.
-constexpr int kWalkSlices = 4;
+constexpr int kWalkSlices = 2;
 constexpr int kWalkThreads = kTcRows * kWalkSlices;
 
 // Bytes of a walk pack ahead of its value planes (the head and the keys).
@@ -919,7 +920,7 @@ template <int D, class IN>
 using BndUnitSmem = typename std::conditional<use_tc<D, IN>(), BndTcSmem<D, IN>, BndSmem<D, IN>>::type;
 
 // Threads of a block that runs whole chunk boundaries: the tcgen05 walk uses
-// four column slices (512 threads), the mma.sync walk 128 threads.
+// kWalkSlices column slices (256 threads), the mma.sync walk 128 threads.
 template <int D, class IN>
 constexpr int unit_threads() {
   return use_tc<D, IN>() ? kTcRows * kWalkSlices : kBndThreads;
