@@ -191,3 +191,28 @@ def test_hard_reset_tokens(gdn):
     b = W.Batch(b.q, b.k, b.v, b.beta, g.contiguous(), b.cu_seqlens, b.lengths)
     o, srun, sbnd = run(gdn, b.to("cuda"), out_dtype=torch.float32)
     check_units(gdn, b, o, srun, sbnd, [(n, h) for n in range(3) for h in range(2)])
+
+
+def test_more_sequences_than_table_threads(gdn):
+    """1500 sequences (more than the chunk table's 1024 threads, so each of its
+    threads takes several sequences when it orders them and lays out the fill
+    order), lengths 0..299 with every seventh empty, unequal chunk counts (the
+    fill starts each unit once its walk has ended): each sequence's bits are
+    those of a shuffled batch, and sampled units match the oracle."""
+    rng = np.random.default_rng(41)
+    lens = [int(x) for x in rng.integers(0, 300, size=1500)]
+    for i in range(0, len(lens), 7):
+        lens[i] = 0
+    H, d = 2, 128
+    bcpu = W.make_batch(lens, H, d, d, dtype=torch.bfloat16, seed=42)
+    b = bcpu.to("cuda")
+    o, srun, sbnd = run(gdn, b, out_dtype=torch.float32)
+    perm = rng.permutation(len(lens)).tolist()
+    bs = b.select(perm)
+    o2, srun2, sbnd2 = run(gdn, bs, out_dtype=torch.float32)
+    cu, cu2 = b.cu_seqlens.tolist(), bs.cu_seqlens.tolist()
+    for i, n in enumerate(perm):
+        assert torch.equal(o2[cu2[i]:cu2[i + 1]], o[cu[n]:cu[n + 1]]), ("shuffled", n)
+        assert torch.equal(srun2[i], srun[n]) and torch.equal(sbnd2[i], sbnd[n]), n
+    picks = [int(x) for x in rng.choice(len(lens), size=6, replace=False)]
+    check_units(gdn, bcpu, o.cpu(), srun.cpu(), sbnd.cpu(), [(n, n % H) for n in picks])
