@@ -96,10 +96,21 @@ __global__ void __launch_bounds__(kBndThreads, 3)
   static_assert(sizeof(PackHead<D, bf16>) >= kAdjNT * PL * sizeof(bf16), "Tb terms fit the head");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   AdjPrepSmem<D>& sm = *reinterpret_cast<AdjPrepSmem<D>*>(smem_raw);
+  // Launched as a programmatic dependent of the kernel before it (the
+  // forward's fill or walk), whose outputs it does not read: it starts in
+  // that grid's tail and waits for it only before it ends, so that this grid,
+  // and everything after it, completes after it.  The chunk table it reads
+  // completed before that kernel started.
   pdl_trigger();  // the reverse walk may be scheduled; it waits for this grid
-  if (hdr[kHdrValid] != 1) return;
+  if (hdr[kHdrValid] != 1) {
+    pdl_wait();
+    return;
+  }
   const int c = blockIdx.x, h = blockIdx.y;
-  if (c >= hdr[kHdrChunks]) return;
+  if (c >= hdr[kHdrChunks]) {
+    pdl_wait();
+    return;
+  }
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
   const FillItem it = fill_item(c * H + h, H, cu, chunk_off, chunk_seq);
   const int len = it.len;
@@ -231,6 +242,7 @@ __global__ void __launch_bounds__(kBndThreads, 3)
       put3(pk.X[0], PD, off, x0, x1);
     }
   }
+  pdl_wait();  // the kernel before it (see above)
 }
 
 // ----------------------------------------------------------------------------

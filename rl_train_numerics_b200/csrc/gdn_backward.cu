@@ -1374,9 +1374,10 @@ static cudaError_t backward_impl(const BwdArgs& a, cudaStream_t st) {
       auto kern = k_adj_prep<D>;
       const size_t sm = sizeof(AdjPrepSmem<D>);
       GDN_BWD_TRY(bwd_set_smem(kern, sm));
-      kern<<<gchunks, kBndThreads, sm, st>>>(q, k, f.beta, f.g, f.cu_seqlens, f.H, f.scale, hdr,
-                                             chunk_off, chunk_seq, apack);
-      GDN_BWD_TRY(cudaGetLastError());
+      // a programmatic dependent of the forward's last kernel (see k_adj_prep)
+      GDN_BWD_TRY(launch_dependent(kern, gchunks, dim3(kBndThreads), sm, st, q, k, f.beta, f.g,
+                                   f.cu_seqlens, f.H, f.scale, hdr, chunk_off, chunk_seq,
+                                   apack));
     }
     {
       auto kern = k_adj_walk<D>;

@@ -702,6 +702,9 @@ __global__ void __launch_bounds__(kFillThreads, 3)
   // item whose word is not set yet makes the block wait for the whole walk
   // grid (griddepcontrol.wait), after which every word is.  The chunk table
   // (read in both phases) completed before the walk started.
+  // A programmatic dependent (the backward's adjoint prep, which reads none of
+  // this kernel's outputs) may start on the SMs this grid's tail leaves.
+  pdl_trigger();
   if (hdr[kHdrValid] != 1) {
     pdl_wait();
     return;
