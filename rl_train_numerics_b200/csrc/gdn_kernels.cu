@@ -32,7 +32,8 @@ namespace gdn {
 // ----------------------------------------------------------------------------
 // Chunk table
 // ----------------------------------------------------------------------------
-constexpr int kTableThreads = 1024;
+constexpr int kTableThreads = 256;
+constexpr int kTableWarps = kTableThreads / 32;  // at most 32
 
 __global__ void __launch_bounds__(kTableThreads)
     k_chunk_table(const int32_t* __restrict__ cu, int N, int64_t T, int H, int32_t* hdr,
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(kTableThreads)
   if (lane == 31) part[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    long long wsum = part[lane];
+    long long wsum = lane < kTableWarps ? part[lane] : 0;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const long long y = __shfl_up_sync(kFull, wsum, off);
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(kTableThreads)
     part[32 + lane] = wsum;  // inclusive over warps 0 .. lane
   }
   __syncthreads();
-  const long long run = part[32 + 31];
+  const long long run = part[32 + kTableWarps - 1];
   part[64 + tid] = x - local + (warp > 0 ? part[32 + warp - 1] : 0);  // exclusive, this thread
   if (tid == 0) {
     if (run > max_chunks) bad = 1;
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kTableThreads)
     if (lane == 31) part[warp] = xs;
     __syncthreads();
     if (warp == 0) {
-      long long ws = part[lane];
+      long long ws = lane < kTableWarps ? part[lane] : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const long long y = __shfl_up_sync(kFull, ws, o);
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(kTableThreads)
     if (lane == 31) part[warp] = xs;
     __syncthreads();
     if (warp == 0) {
-      long long ws = part[lane];
+      long long ws = lane < kTableWarps ? part[lane] : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const long long y = __shfl_up_sync(kFull, ws, o);
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(kTableThreads)
       at += nc > 1 ? nc - 1 : 0;
     }
     if (tid == 0) {
-      hdr[kHdrFill1Chunks] = (int32_t)part[32 + 31];
+      hdr[kHdrFill1Chunks] = (int32_t)part[32 + kTableWarps - 1];
       // Equal chunk counts: every walk ends at about the same time, so the
       // fill waits for the walk grid once instead of checking its units.
       int uniform = 1;
