@@ -166,9 +166,9 @@ int gdn_cpr_forward_ex(const void* q, const void* k, const void* v, int in_dtype
  *   readable with gdn_check_error(error_word, ...).  An empty batch sets it to
  *   zero.  Argument errors are returned before any device work, as for
  *   gdn_cpr_forward.
- * - The array's device address is cached per device for the process; after
- *   cudaDeviceReset (or any other teardown of the device's primary context)
- *   the cache is stale, so this entry point must not be called again.
+ * - The array's device address is looked up in the current context on every
+ *   call, so the entry point stays valid after cudaDeviceReset or a re-created
+ *   primary context.
  */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 int gdn_cpr_forward_noalloc(const void* q, const void* k, const void* v, int in_dtype,
