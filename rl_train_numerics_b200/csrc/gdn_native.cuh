@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kNtThreads, 1)
     const WalkPack<D, bf16>& pk = sm.buf[j & 1];
     const uint32_t kb = smem_u32(pk.kv.K[0]), vb = smem_u32(pk.kv.V[0]);
     const uint32_t tbb = smem_u32(pk.head.TbT[0]), tvb = smem_u32(pk.head.TvT[0]);
-    // Round 1
+    // First product round
     if (w == 0) {
       tc_fence_after();
 #pragma unroll
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(kNtThreads, 1)
       status = kStepFailed;
       break;
     }
-    // Round 2: Z -= Y Tb^T
+    // Second product round: Z -= Y Tb^T
     if (w == 0) {
       tc_fence_after();
       using PY = SplitPairs<2, 2>;
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kNtThreads, 1)
       status = kStepFailed;
       break;
     }
-    // Round 3: Ob = Z Pm^T (Pm lower triangular: k16 step ks reaches the
+    // Third product round: Ob = Z Pm^T (Pm lower triangular: k16 step ks reaches the
     // columns i >= 16 ks); P = Ud K for a trailing partial chunk
     if (w == 0) {
       tc_fence_after();
