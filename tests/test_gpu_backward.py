@@ -138,7 +138,9 @@ def test_repeat_runs_are_identical(gdn):
 
 def test_reusing_the_forwards_first_pass_changes_no_bit(gdn):
     """forward() on the backward's workspace, then backward(reuse_forward=True):
-    the same bits as a backward that runs the first pass itself."""
+    the same bits as a backward that runs the first pass itself, and the
+    forward's outputs (written while the backward's adjoint prep may already
+    run) the same bits as a forward alone."""
     b = W.make_batch([300, 64, 5, 190], 3, 128, 128, seed=32).to("cuda")
     d_o, dsf = cotangents(b, 3, 128, 33, torch.bfloat16)
     d_o, dsf = d_o.cuda(), dsf.cuda()
@@ -146,12 +148,15 @@ def test_reusing_the_forwards_first_pass_changes_no_bit(gdn):
     ref, _ = gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o, ds_final=dsf, h0=h0)
     ws = torch.zeros(gdn.backward_workspace_bytes(4, b.total_tokens, 3, 128, 128),
                      dtype=torch.uint8, device="cuda")
-    gdn.forward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, h0=h0, workspace=ws)
+    o, srun, _, _ = gdn.forward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, h0=h0, workspace=ws)
     got, _ = gdn.backward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, d_o, ds_final=dsf, h0=h0,
                           workspace=ws, reuse_forward=True)
     assert gdn.check_error(ws) == 0
     for k in NAMES:
         assert torch.equal(ref[k], got[k]), k
+    o_alone, srun_alone, _, ws2 = gdn.forward(b.q, b.k, b.v, b.beta, b.g, b.cu_seqlens, h0=h0)
+    assert gdn.check_error(ws2) == 0
+    assert torch.equal(o, o_alone) and torch.equal(srun, srun_alone)
 
 
 def test_bad_cu_seqlens_sets_the_error_word(gdn):
